@@ -1,0 +1,93 @@
+"""Seeded synthetic inputs shared by the tests, the smoke check and the benchmark.
+
+This module only draws random numbers and casts them; it holds none of the codec's
+arithmetic. The recipes stand in for the trained checkpoints and K/V caches that the
+pages measure (ZipNN's BF16/FP32 models, FP8 weights and K/V caches), which are not
+available here:
+
+* ``bf16_small``: 1,048,576 values N(0, 0.02^2) from CPU seed 0, rounded to BF16.
+* ``checkpoint_7b``: the 225 tensors of a 7B-shaped BF16 checkpoint (32 layers of
+  q, k, v, o 4096x4096 and gate, up, down 4096x11008, then a 32000x4096 embedding);
+  tensor t has sigma_t = exp(U(ln 0.005, ln 0.05)) (225 draws, CPU seed 0) and values
+  N(0, 1) * sigma_t from a generator seeded t + 1 on the tensor's device.
+* ``fp32_tensor``: N(0, 0.02^2) FP32; the "clean" variant is the same values rounded
+  through BF16 (low 16 fraction bits zero).
+* ``fp8_tensor``: rows of N(0, 1) * scale_r, scale_r = exp(U(ln 0.25, ln 4)) per
+  4096-wide row, clamped to +-448 and cast to float8_e4m3fn (round to nearest).
+* ``kv_cache``: [layers, 2, batch, heads, seq, dim] BF16 with per-channel std
+  exp(ln 0.5 + N(0, 1)) for every (layer, k/v, head, dim), shared over batch and seq.
+"""
+import math
+
+import torch
+
+CHUNK_BYTES = 262144
+
+
+def bf16_small(n=1048576, seed=0, sigma=0.02):
+    g = torch.Generator("cpu").manual_seed(seed)
+    return (torch.randn(n, generator=g) * sigma).to(torch.bfloat16)
+
+
+def checkpoint_7b_shapes(layers=32, hidden=4096, mlp=11008, vocab=32000):
+    shapes = []
+    for layer in range(layers):
+        for name in ("q", "k", "v", "o"):
+            shapes.append((f"layers.{layer}.attn.{name}", (hidden, hidden)))
+        for name in ("gate", "up", "down"):
+            shapes.append((f"layers.{layer}.mlp.{name}", (hidden, mlp)))
+    shapes.append(("embedding", (vocab, hidden)))
+    return shapes
+
+
+def checkpoint_7b_sigmas(count=225, seed=0):
+    g = torch.Generator("cpu").manual_seed(seed)
+    u = torch.rand(count, generator=g, dtype=torch.float64)
+    lo, hi = math.log(0.005), math.log(0.05)
+    return torch.exp(lo + (hi - lo) * u).tolist()
+
+
+def checkpoint_7b_tensor(t, shape, sigma, device="cuda"):
+    g = torch.Generator(device).manual_seed(t + 1)
+    x = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    return (x * sigma).to(torch.bfloat16)
+
+
+def checkpoint_7b(device="cuda", layers=32, hidden=4096, mlp=11008, vocab=32000):
+    shapes = checkpoint_7b_shapes(layers, hidden, mlp, vocab)
+    sig = checkpoint_7b_sigmas(len(shapes))
+    return [(name, checkpoint_7b_tensor(t, shape, sig[t], device)) for t, (name, shape) in enumerate(shapes)]
+
+
+def fp32_tensor(n=268435456, seed=0, sigma=0.02, clean=False, device="cpu", block=1 << 26):
+    g = torch.Generator(device).manual_seed(seed)
+    out = torch.empty(n, dtype=torch.float32, device=device)
+    for lo in range(0, n, block):
+        hi = min(n, lo + block)
+        out[lo:hi] = torch.randn(hi - lo, generator=g, device=device) * sigma
+    if clean:
+        out = out.to(torch.bfloat16).to(torch.float32)
+    return out
+
+
+def fp8_tensor(rows=262144, cols=4096, seed=0, device="cpu", block_rows=16384):
+    g = torch.Generator(device).manual_seed(seed)
+    lo, hi = math.log(0.25), math.log(4.0)
+    scale = torch.exp(lo + (hi - lo) * torch.rand(rows, 1, generator=g, device=device))
+    out = torch.empty(rows, cols, dtype=torch.float8_e4m3fn, device=device)
+    for r in range(0, rows, block_rows):
+        r2 = min(rows, r + block_rows)
+        x = torch.randn(r2 - r, cols, generator=g, device=device) * scale[r:r2]
+        out[r:r2] = x.clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
+    return out.reshape(-1)
+
+
+def kv_cache(shape=(32, 2, 16, 8, 4096, 128), seed=0, device="cpu"):
+    layers, kv, batch, heads, seq, dim = shape
+    g = torch.Generator(device).manual_seed(seed)
+    std = torch.exp(math.log(0.5) + torch.randn(layers, kv, 1, heads, 1, dim, generator=g, device=device))
+    out = torch.empty(shape, dtype=torch.bfloat16, device=device)
+    for layer in range(layers):
+        x = torch.randn((kv, batch, heads, seq, dim), generator=g, device=device)
+        out[layer] = (x * std[layer]).to(torch.bfloat16)
+    return out.reshape(-1)

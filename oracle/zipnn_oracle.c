@@ -1,0 +1,842 @@
+/*
+ * zipnn_oracle.c -- plain, slow, obviously-correct CPU oracle for the ZipNN-style
+ * float-tensor codec.
+ *
+ * TEST INFRASTRUCTURE. Only tests, the smoke check and the benchmark's CPU baseline
+ * load this file's library. The product (the CUDA library) shares nothing with it:
+ * no header, no helper, no table. Everything here is written out step by step, in
+ * the order the method states it, with no blocking or fusion.
+ *
+ * Method, by page title and section:
+ *  - Field split: "ZipNN: Lossless Compression for AI Models", abstract; THEORY-599
+ *    note, "Per-field compressibility (Table II)": the exponent field compresses,
+ *    the sign and fraction bytes do not.
+ *  - Order-0 histogram and Huffman code per chunk: THEORY-599 note, "Order-0 only
+ *    (section III-A b)": Huffman after exponent extraction, no context model.
+ *  - FP8 exponent and mantissa coded independently: "Lossless Compression of Neural
+ *    Network Components: Weights, Checkpoints, and K/V Caches in Low-Precision
+ *    Formats", abstract.
+ *  - Grouped chunks with shared Huffman codes from a reusable setup: "NeuralZip:
+ *    Reusable Setup for Fast Lossless Compression", abstract.
+ *
+ * Readings where the pages are silent (each one is listed in the design notes):
+ *  - Huffman ties: the two nodes with the smallest (weight, order) keys merge first;
+ *    a leaf's order is its symbol value, the i-th merged node's order is 256 + i.
+ *  - Length limit 12: halve every non-zero frequency (never below 1) and rebuild,
+ *    until the longest code is at most 12 bits.
+ *  - Canonical code values: the deflate rule (RFC 1951, section 3.2.2).
+ *  - Container layout, sub-block index, ZERO/RAW/HUFF choice: the format written in
+ *    the design notes; pinned by a hand-derived golden container, not by the pages.
+ *  - Grouping: Lloyd's k-means with SplitMix64 seeding (parity unpinned by the pages:
+ *    pinned only by invariants and small separable cases).
+ */
+#include "zipnn_oracle.h"
+
+#include <pthread.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define LMAX 12
+#define MAX_GROUPS 64
+#define HEADER_BYTES 64
+#define ENTRY_BYTES 16
+#define MODE_RAW 0
+#define MODE_ZERO 1
+#define MODE_HUFF 2
+#define NO_CODE 0xFFFFFFFFu
+
+/* ------------------------------------------------------------------ field map */
+
+int orc_n_streams(int dtype) { return dtype == ORC_BF16 ? 2 : dtype == ORC_FP32 ? 4 : 3; }
+int orc_n_entropy(int dtype) { return dtype == ORC_FP8 ? 2 : 1; }
+static int value_bytes(int dtype) { return dtype == ORC_BF16 ? 2 : dtype == ORC_FP32 ? 4 : 1; }
+static int is_entropy(int dtype, int s) { return s == 0 || (dtype == ORC_FP8 && s == 1); }
+/* bits per symbol when a stream is stored RAW */
+static int raw_width(int dtype, int s) {
+  if (dtype == ORC_FP8) return s == 0 ? 4 : s == 1 ? 3 : 1;
+  return 8;
+}
+int orc_alphabet(int dtype, int s) { return 1 << raw_width(dtype, s); }
+/* bytes of one packed code record (4-bit lengths), rounded up to 16 */
+static uint64_t round16(uint64_t x) { return (x + 15) & ~(uint64_t)15; }
+static uint64_t record_bytes(int dtype, int s) { return round16((uint64_t)orc_alphabet(dtype, s) / 2); }
+
+/* The split. BF16 w: exponent = bits 14..7; sign+fraction byte = sign in bit 7,
+ * fraction bits 6..0. FP32 u: exponent = bits 30..23; p1 = sign + fraction bits
+ * 22..16; p2 = fraction bits 15..8; p3 = bits 7..0. FP8 E4M3 b: exponent bits 6..3,
+ * mantissa bits 2..0, sign bit 7. Streams are numbered in that order. */
+uint8_t orc_field(int dtype, const uint8_t* src, uint64_t i, int s) {
+  if (dtype == ORC_BF16) {
+    uint32_t w = (uint32_t)src[2 * i] | ((uint32_t)src[2 * i + 1] << 8);
+    if (s == 0) return (uint8_t)((w >> 7) & 0xFF);
+    return (uint8_t)(((w >> 8) & 0x80) | (w & 0x7F));
+  }
+  if (dtype == ORC_FP32) {
+    uint32_t u = (uint32_t)src[4 * i] | ((uint32_t)src[4 * i + 1] << 8) |
+                 ((uint32_t)src[4 * i + 2] << 16) | ((uint32_t)src[4 * i + 3] << 24);
+    if (s == 0) return (uint8_t)((u >> 23) & 0xFF);
+    if (s == 1) return (uint8_t)(((u >> 24) & 0x80) | ((u >> 16) & 0x7F));
+    if (s == 2) return (uint8_t)((u >> 8) & 0xFF);
+    return (uint8_t)(u & 0xFF);
+  }
+  {
+    uint32_t b = src[i];
+    if (s == 0) return (uint8_t)((b >> 3) & 0xF);
+    if (s == 1) return (uint8_t)(b & 7);
+    return (uint8_t)(b >> 7);
+  }
+}
+
+/* The merge: the inverse of the split, writing value i. */
+static void put_value(int dtype, uint8_t* dst, uint64_t i, const uint8_t* f) {
+  if (dtype == ORC_BF16) {
+    uint32_t w = ((uint32_t)(f[1] & 0x80) << 8) | ((uint32_t)f[0] << 7) | (f[1] & 0x7F);
+    dst[2 * i] = (uint8_t)(w & 0xFF);
+    dst[2 * i + 1] = (uint8_t)(w >> 8);
+  } else if (dtype == ORC_FP32) {
+    uint32_t u = ((uint32_t)(f[1] & 0x80) << 24) | ((uint32_t)f[0] << 23) |
+                 ((uint32_t)(f[1] & 0x7F) << 16) | ((uint32_t)f[2] << 8) | f[3];
+    dst[4 * i] = (uint8_t)(u & 0xFF);
+    dst[4 * i + 1] = (uint8_t)((u >> 8) & 0xFF);
+    dst[4 * i + 2] = (uint8_t)((u >> 16) & 0xFF);
+    dst[4 * i + 3] = (uint8_t)(u >> 24);
+  } else {
+    dst[i] = (uint8_t)((f[2] << 7) | (f[0] << 3) | f[1]);
+  }
+}
+
+void orc_histogram(int dtype, const uint8_t* src, uint64_t lo, uint64_t hi, int s, uint64_t* hist) {
+  int a = orc_alphabet(dtype, s);
+  for (int k = 0; k < a; k++) hist[k] = 0;
+  for (uint64_t i = lo; i < hi; i++) hist[orc_field(dtype, src, i, s)]++;
+}
+
+/* ------------------------------------------------------------------ Huffman */
+
+/* Huffman code lengths. Every present symbol is a node with key (weight, order).
+ * Repeatedly take out the two nodes with the smallest keys and put back one node
+ * whose weight is their sum; the i-th such node gets order 256 + i. A symbol's
+ * length is the depth of its leaf. A lone symbol gets length 1. */
+int orc_huffman_lengths(const uint64_t* freq, int alphabet, uint8_t* len) {
+  uint64_t w[512];
+  uint32_t order[512];
+  int parent[512], alive[512], leaf_of[256];
+  int nodes = 0, leaves = 0;
+  if (alphabet < 1 || alphabet > 256) return ORC_EINVAL;
+  for (int s = 0; s < alphabet; s++) {
+    len[s] = 0;
+    leaf_of[s] = -1;
+    if (freq[s] > 0) {
+      w[nodes] = freq[s];
+      order[nodes] = (uint32_t)s;
+      parent[nodes] = -1;
+      alive[nodes] = 1;
+      leaf_of[s] = nodes;
+      nodes++;
+      leaves++;
+    }
+  }
+  if (leaves == 0) return ORC_OK;
+  if (leaves == 1) {
+    for (int s = 0; s < alphabet; s++)
+      if (leaf_of[s] >= 0) len[s] = 1;
+    return ORC_OK;
+  }
+  for (int merged = 0; merged < leaves - 1; merged++) {
+    int pick[2];
+    for (int t = 0; t < 2; t++) {
+      int best = -1;
+      for (int j = 0; j < nodes; j++) {
+        if (!alive[j]) continue;
+        if (best < 0 || w[j] < w[best] || (w[j] == w[best] && order[j] < order[best])) best = j;
+      }
+      alive[best] = 0;
+      pick[t] = best;
+    }
+    w[nodes] = w[pick[0]] + w[pick[1]];
+    order[nodes] = 256u + (uint32_t)merged;
+    parent[nodes] = -1;
+    alive[nodes] = 1;
+    parent[pick[0]] = nodes;
+    parent[pick[1]] = nodes;
+    nodes++;
+  }
+  for (int s = 0; s < alphabet; s++) {
+    if (leaf_of[s] < 0) continue;
+    int depth = 0;
+    for (int j = leaf_of[s]; parent[j] >= 0; j = parent[j]) depth++;
+    len[s] = (uint8_t)depth;
+  }
+  return ORC_OK;
+}
+
+/* Lengths limited to lmax: with k = 0, 1, 2, ... build the code for the frequencies
+ * max(1, f >> k) (zero stays zero) and keep the first one whose longest code fits. */
+int orc_limited_lengths(const uint64_t* freq, int alphabet, int lmax, uint8_t* len) {
+  uint64_t g[256];
+  if (alphabet < 1 || alphabet > 256 || lmax < 1) return ORC_EINVAL;
+  for (int k = 0; k < 64; k++) {
+    int longest = 0;
+    for (int s = 0; s < alphabet; s++) {
+      if (freq[s] == 0) g[s] = 0;
+      else g[s] = (freq[s] >> k) > 0 ? (freq[s] >> k) : 1;
+    }
+    orc_huffman_lengths(g, alphabet, len);
+    for (int s = 0; s < alphabet; s++)
+      if (len[s] > longest) longest = len[s];
+    if (longest <= lmax) return ORC_OK;
+  }
+  return ORC_EINVAL; /* unreachable for alphabets up to 2^lmax symbols */
+}
+
+/* Canonical code values, RFC 1951 section 3.2.2: count the codes of each length,
+ * compute the first code of each length, then number the symbols in increasing
+ * order within each length. */
+void orc_canonical_codes(const uint8_t* len, int alphabet, uint32_t* code) {
+  uint32_t count[16] = {0}, next[16] = {0};
+  for (int s = 0; s < alphabet; s++)
+    if (len[s]) count[len[s]]++;
+  uint32_t c = 0;
+  count[0] = 0;
+  for (int bits = 1; bits < 16; bits++) {
+    c = (c + count[bits - 1]) << 1;
+    next[bits] = c;
+  }
+  for (int s = 0; s < alphabet; s++) code[s] = len[s] ? next[len[s]]++ : 0;
+}
+
+/* ------------------------------------------------------------------ bit I/O */
+
+/* Bit t of a bit string is bit (7 - t mod 8) of byte t / 8: most significant first. */
+static void put_bits(uint8_t* buf, uint64_t* t, uint32_t value, int nbits) {
+  for (int b = nbits - 1; b >= 0; b--) {
+    if ((value >> b) & 1u) buf[*t >> 3] |= (uint8_t)(0x80u >> (*t & 7));
+    (*t)++;
+  }
+}
+
+static int get_bit(const uint8_t* buf, uint64_t cap_bits, uint64_t* t) {
+  if (*t >= cap_bits) return -1;
+  int bit = (buf[*t >> 3] >> (7 - (*t & 7))) & 1;
+  (*t)++;
+  return bit;
+}
+
+static void put_u32(uint8_t* p, uint32_t v) {
+  for (int i = 0; i < 4; i++) p[i] = (uint8_t)(v >> (8 * i));
+}
+static void put_u64(uint8_t* p, uint64_t v) {
+  for (int i = 0; i < 8; i++) p[i] = (uint8_t)(v >> (8 * i));
+}
+static uint32_t get_u32(const uint8_t* p) {
+  uint32_t v = 0;
+  for (int i = 0; i < 4; i++) v |= (uint32_t)p[i] << (8 * i);
+  return v;
+}
+static uint64_t get_u64(const uint8_t* p) {
+  uint64_t v = 0;
+  for (int i = 0; i < 8; i++) v |= (uint64_t)p[i] << (8 * i);
+  return v;
+}
+
+/* ------------------------------------------------------------------ layout rules */
+
+static uint64_t ceil_div(uint64_t a, uint64_t b) { return (a + b - 1) / b; }
+
+static uint64_t chunk_values(int dtype, uint32_t chunk_bytes) { return chunk_bytes / (uint32_t)value_bytes(dtype); }
+
+static uint64_t table_end(int dtype, uint64_t n_chunks) {
+  return HEADER_BYTES + (uint64_t)ENTRY_BYTES * n_chunks * (uint64_t)orc_n_streams(dtype);
+}
+
+/* bytes of all shared code records for n_groups groups */
+static uint64_t shared_bytes(int dtype, uint32_t n_groups) {
+  uint64_t b = 0;
+  for (int s = 0; s < orc_n_entropy(dtype); s++) b += (uint64_t)n_groups * record_bytes(dtype, s);
+  return b;
+}
+
+/* byte position of shared record r = e * n_groups + g inside the code section */
+static uint64_t shared_record_pos(int dtype, uint32_t n_groups, uint32_t r) {
+  uint32_t e = r / n_groups, g = r % n_groups;
+  uint64_t pos = 0;
+  for (uint32_t k = 0; k < e; k++) pos += (uint64_t)n_groups * record_bytes(dtype, (int)k);
+  return pos + (uint64_t)g * record_bytes(dtype, (int)e);
+}
+
+static uint64_t raw_payload_bytes(uint64_t m, int width) { return round16(ceil_div(m * (uint64_t)width, 8)); }
+
+uint64_t orc_max_compressed_bytes(int dtype, uint64_t n, uint32_t chunk_bytes, uint32_t n_groups) {
+  uint64_t m0 = chunk_values(dtype, chunk_bytes);
+  if (m0 == 0 || n == 0) return 0;
+  uint64_t chunks = ceil_div(n, m0);
+  uint64_t total = table_end(dtype, chunks) + shared_bytes(dtype, n_groups);
+  for (uint64_t c = 0; c < chunks; c++) {
+    uint64_t m = (c + 1) * m0 <= n ? m0 : n - c * m0;
+    for (int s = 0; s < orc_n_streams(dtype); s++) total += raw_payload_bytes(m, raw_width(dtype, s));
+  }
+  return total;
+}
+
+/* ------------------------------------------------------------------ compress */
+
+typedef struct {
+  uint8_t mode;
+  uint32_t code; /* shared record index, or NO_CODE */
+  uint64_t size;
+  uint8_t* bytes; /* size bytes, owned */
+} entry_t;
+
+typedef struct {
+  int dtype;
+  const uint8_t* src;
+  uint64_t n, m0, chunks;
+  uint32_t S;
+  const uint8_t* plan_lens;
+  uint32_t n_groups;
+  entry_t* entries;
+  int thread, threads;
+  int status;
+} job_t;
+
+/* Encode stream s of one chunk (values [lo, lo + m)) into one entry. */
+static int encode_entry(const job_t* jb, uint64_t lo, uint64_t m, int s, entry_t* en) {
+  int dt = jb->dtype, a = orc_alphabet(dt, s), w = raw_width(dt, s);
+  uint8_t* sym = (uint8_t*)malloc(m);
+  uint8_t len[256];
+  uint32_t code[256];
+  uint64_t hist[256];
+  if (!sym) return ORC_EINVAL;
+  int all_zero = 1;
+  for (uint64_t i = 0; i < m; i++) {
+    sym[i] = orc_field(dt, jb->src, lo + i, s);
+    if (sym[i]) all_zero = 0;
+  }
+  en->code = NO_CODE;
+  en->bytes = NULL;
+  en->size = 0;
+  if (all_zero) {
+    en->mode = MODE_ZERO;
+    free(sym);
+    return ORC_OK;
+  }
+  uint64_t p_raw = raw_payload_bytes(m, w);
+  en->mode = MODE_RAW;
+  if (is_entropy(dt, s)) {
+    int e = s; /* entropy streams are streams 0 (and 1 for FP8) */
+    for (int k = 0; k < a; k++) hist[k] = 0;
+    for (uint64_t i = 0; i < m; i++) hist[sym[i]]++;
+    int use_group = -1;
+    uint64_t best_bits = 0;
+    if (jb->plan_lens) {
+      /* a group is eligible if its code has a length for every present symbol;
+       * the one with the fewest coded bits wins, ties to the smaller group */
+      for (uint32_t g = 0; g < jb->n_groups; g++) {
+        const uint8_t* lg = jb->plan_lens + ((uint64_t)e * jb->n_groups + g) * 256;
+        int ok = 1;
+        uint64_t bits = 0;
+        for (int k = 0; k < a; k++) {
+          if (hist[k] == 0) continue;
+          if (lg[k] == 0) ok = 0;
+          bits += hist[k] * lg[k];
+        }
+        if (ok && (use_group < 0 || bits < best_bits)) {
+          use_group = (int)g;
+          best_bits = bits;
+        }
+      }
+    }
+    if (use_group >= 0) memcpy(len, jb->plan_lens + ((uint64_t)e * jb->n_groups + (uint32_t)use_group) * 256, 256);
+    else orc_limited_lengths(hist, a, LMAX, len);
+    uint64_t bits = 0;
+    for (int k = 0; k < a; k++) bits += hist[k] * len[k];
+    uint64_t nsub = ceil_div(m, jb->S);
+    uint64_t rec = use_group >= 0 ? 0 : record_bytes(dt, s);
+    uint64_t p_huff = rec + round16(4 * nsub) + round16(ceil_div(bits, 8));
+    if (p_huff < p_raw) {
+      en->mode = MODE_HUFF;
+      en->code = use_group >= 0 ? (uint32_t)e * jb->n_groups + (uint32_t)use_group : NO_CODE;
+      en->size = p_huff;
+      en->bytes = (uint8_t*)calloc(p_huff, 1);
+      if (!en->bytes) {
+        free(sym);
+        return ORC_EINVAL;
+      }
+      uint8_t* p = en->bytes;
+      if (rec) {
+        for (int k = 0; k < a / 2; k++) p[k] = (uint8_t)(len[2 * k] | (len[2 * k + 1] << 4));
+        p += rec;
+      }
+      orc_canonical_codes(len, a, code);
+      uint8_t* bs = p + round16(4 * nsub);
+      uint64_t t = 0;
+      for (uint64_t i = 0; i < m; i++) {
+        if (i % jb->S == 0) put_u32(p + 4 * (i / jb->S), (uint32_t)t);
+        put_bits(bs, &t, code[sym[i]], len[sym[i]]);
+      }
+      free(sym);
+      return ORC_OK;
+    }
+  }
+  en->mode = MODE_RAW;
+  en->size = p_raw;
+  en->bytes = (uint8_t*)calloc(p_raw, 1);
+  if (!en->bytes) {
+    free(sym);
+    return ORC_EINVAL;
+  }
+  uint64_t t = 0;
+  for (uint64_t i = 0; i < m; i++) put_bits(en->bytes, &t, sym[i], w);
+  free(sym);
+  return ORC_OK;
+}
+
+static void* compress_worker(void* arg) {
+  job_t* jb = (job_t*)arg;
+  int ns = orc_n_streams(jb->dtype);
+  for (uint64_t c = (uint64_t)jb->thread; c < jb->chunks; c += (uint64_t)jb->threads) {
+    uint64_t lo = c * jb->m0;
+    uint64_t m = lo + jb->m0 <= jb->n ? jb->m0 : jb->n - lo;
+    for (int s = 0; s < ns; s++) {
+      int st = encode_entry(jb, lo, m, s, &jb->entries[c * (uint64_t)ns + (uint64_t)s]);
+      if (st != ORC_OK) jb->status = st;
+    }
+  }
+  return NULL;
+}
+
+static int run_jobs(job_t* base, int threads, void* (*fn)(void*)) {
+  if (threads < 1) threads = 1;
+  if (threads > 256) threads = 256;
+  job_t* jobs = (job_t*)malloc(sizeof(job_t) * (size_t)threads);
+  pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)threads);
+  if (!jobs || !th) {
+    free(jobs);
+    free(th);
+    return ORC_EINVAL;
+  }
+  for (int t = 0; t < threads; t++) {
+    jobs[t] = *base;
+    jobs[t].thread = t;
+    jobs[t].threads = threads;
+    jobs[t].status = ORC_OK;
+  }
+  for (int t = 1; t < threads; t++) pthread_create(&th[t], NULL, fn, &jobs[t]);
+  fn(&jobs[0]);
+  for (int t = 1; t < threads; t++) pthread_join(th[t], NULL);
+  int st = ORC_OK;
+  for (int t = 0; t < threads; t++)
+    if (jobs[t].status != ORC_OK) st = jobs[t].status;
+  free(jobs);
+  free(th);
+  return st;
+}
+
+int orc_compress(int dtype, const void* src, uint64_t n, uint32_t chunk_bytes, uint32_t S,
+                 const uint8_t* plan_lens, uint32_t n_groups, void* out, uint64_t cap,
+                 uint64_t* out_bytes, int threads) {
+  if (dtype < 0 || dtype > 2 || !src || !out || n == 0 || S == 0) return ORC_EINVAL;
+  if (chunk_bytes == 0 || chunk_bytes % (uint32_t)value_bytes(dtype) != 0) return ORC_EINVAL;
+  if (plan_lens && (n_groups == 0 || n_groups > MAX_GROUPS)) return ORC_EINVAL;
+  if (!plan_lens) n_groups = 0;
+  int ns = orc_n_streams(dtype);
+  uint64_t m0 = chunk_values(dtype, chunk_bytes);
+  uint64_t chunks = ceil_div(n, m0);
+  if (cap < orc_max_compressed_bytes(dtype, n, chunk_bytes, n_groups)) return ORC_ESMALL;
+  entry_t* entries = (entry_t*)calloc(chunks * (uint64_t)ns, sizeof(entry_t));
+  if (!entries) return ORC_EINVAL;
+  job_t jb;
+  memset(&jb, 0, sizeof(jb));
+  jb.dtype = dtype;
+  jb.src = (const uint8_t*)src;
+  jb.n = n;
+  jb.m0 = m0;
+  jb.chunks = chunks;
+  jb.S = S;
+  jb.plan_lens = plan_lens;
+  jb.n_groups = n_groups;
+  jb.entries = entries;
+  int st = run_jobs(&jb, threads, compress_worker);
+  if (st == ORC_OK) {
+    uint8_t* o = (uint8_t*)out;
+    uint64_t off_codes = table_end(dtype, chunks);
+    uint64_t off_payload = off_codes + shared_bytes(dtype, n_groups);
+    memset(o, 0, off_payload);
+    /* header */
+    o[0] = 'Z';
+    o[1] = 'N';
+    o[2] = 'N';
+    o[3] = '1';
+    o[4] = 1;
+    o[5] = 0;
+    o[6] = (uint8_t)dtype;
+    o[7] = (uint8_t)ns;
+    put_u64(o + 8, n);
+    put_u32(o + 16, chunk_bytes);
+    put_u32(o + 20, S);
+    put_u32(o + 24, (uint32_t)chunks);
+    put_u32(o + 28, n_groups * (uint32_t)orc_n_entropy(dtype));
+    put_u64(o + 32, off_codes);
+    put_u64(o + 40, off_payload);
+    o[56] = LMAX;
+    o[57] = (uint8_t)n_groups;
+    /* shared code records */
+    for (int e = 0; e < orc_n_entropy(dtype) && n_groups; e++) {
+      int a = orc_alphabet(dtype, e);
+      for (uint32_t g = 0; g < n_groups; g++) {
+        const uint8_t* lg = plan_lens + ((uint64_t)e * n_groups + g) * 256;
+        uint8_t* rp = o + off_codes + shared_record_pos(dtype, n_groups, (uint32_t)e * n_groups + g);
+        for (int k = 0; k < a / 2; k++) rp[k] = (uint8_t)(lg[2 * k] | (lg[2 * k + 1] << 4));
+      }
+    }
+    /* chunk table and payloads, in entry order: offsets are the running sum */
+    uint64_t pos = off_payload;
+    for (uint64_t k = 0; k < chunks * (uint64_t)ns; k++) {
+      uint8_t* te = o + HEADER_BYTES + ENTRY_BYTES * k;
+      te[0] = entries[k].mode;
+      put_u32(te + 4, entries[k].code);
+      put_u64(te + 8, pos);
+      if (entries[k].size) memcpy(o + pos, entries[k].bytes, entries[k].size);
+      pos += entries[k].size;
+    }
+    put_u64(o + 48, pos);
+    *out_bytes = pos;
+  }
+  for (uint64_t k = 0; k < chunks * (uint64_t)ns; k++) free(entries[k].bytes);
+  free(entries);
+  return st;
+}
+
+/* ------------------------------------------------------------------ decompress */
+
+typedef struct {
+  int dtype;
+  const uint8_t* in;
+  uint64_t in_bytes, n, m0, chunks, total, off_codes;
+  uint32_t S, n_groups;
+  uint8_t* out;
+  int thread, threads;
+  int status;
+} djob_t;
+
+/* Read the 4-bit lengths of a code record and check it: every length at most 12, at
+ * least one symbol, and the Kraft sum of 2^-len at most 1. */
+static int read_record(const uint8_t* rp, int a, uint8_t* len) {
+  uint64_t kraft = 0;
+  int present = 0;
+  for (int k = 0; k < a / 2; k++) {
+    len[2 * k] = rp[k] & 0xF;
+    len[2 * k + 1] = rp[k] >> 4;
+  }
+  for (int k = 0; k < a; k++) {
+    if (len[k] > LMAX) return ORC_ECORRUPT;
+    if (len[k]) {
+      present++;
+      kraft += (uint64_t)1 << (LMAX - len[k]);
+    }
+  }
+  if (!present || kraft > ((uint64_t)1 << LMAX)) return ORC_ECORRUPT;
+  return ORC_OK;
+}
+
+/* Canonical decoding of one symbol, one bit at a time: at each length l the codes
+ * of that length are the values [first, first + count[l]). */
+static int decode_symbol(const uint8_t* bs, uint64_t cap_bits, uint64_t* t, const uint32_t* count,
+                         const uint8_t* sorted) {
+  int64_t code = 0, first = 0, index = 0;
+  for (int l = 1; l <= LMAX; l++) {
+    int b = get_bit(bs, cap_bits, t);
+    if (b < 0) return -1;
+    code |= b;
+    if (code >= first && code - first < (int64_t)count[l]) return sorted[index + (code - first)];
+    index += count[l];
+    first = (first + (int64_t)count[l]) << 1;
+    code <<= 1;
+  }
+  return -1;
+}
+
+static int decode_entry(const djob_t* jb, uint64_t c, int s, uint64_t m, uint8_t* sym) {
+  int dt = jb->dtype, a = orc_alphabet(dt, s), w = raw_width(dt, s), ns = orc_n_streams(dt);
+  uint64_t k = c * (uint64_t)ns + (uint64_t)s;
+  const uint8_t* te = jb->in + HEADER_BYTES + ENTRY_BYTES * k;
+  uint8_t mode = te[0];
+  uint32_t code_ix = get_u32(te + 4);
+  uint64_t off = get_u64(te + 8);
+  uint64_t end = k + 1 < jb->chunks * (uint64_t)ns ? get_u64(te + ENTRY_BYTES + 8) : jb->total;
+  if (te[1] || te[2] || te[3]) return ORC_ECORRUPT;
+  if (off % 16 || end % 16 || off > end || end > jb->total) return ORC_ECORRUPT;
+  if (mode == MODE_ZERO) {
+    if (code_ix != NO_CODE) return ORC_ECORRUPT;
+    memset(sym, 0, m);
+    return ORC_OK;
+  }
+  if (mode == MODE_RAW) {
+    if (code_ix != NO_CODE) return ORC_ECORRUPT;
+    uint64_t cap_bits = (end - off) * 8, t = 0;
+    if (cap_bits < m * (uint64_t)w) return ORC_ECORRUPT;
+    for (uint64_t i = 0; i < m; i++) {
+      uint32_t v = 0;
+      for (int b = 0; b < w; b++) v = (v << 1) | (uint32_t)get_bit(jb->in + off, cap_bits, &t);
+      sym[i] = (uint8_t)v;
+    }
+    return ORC_OK;
+  }
+  if (mode != MODE_HUFF || !is_entropy(dt, s)) return ORC_ECORRUPT;
+  uint8_t len[256];
+  const uint8_t* p = jb->in + off;
+  uint64_t avail = end - off;
+  if (code_ix == NO_CODE) {
+    uint64_t rec = record_bytes(dt, s);
+    if (avail < rec) return ORC_ECORRUPT;
+    if (read_record(p, a, len) != ORC_OK) return ORC_ECORRUPT;
+    p += rec;
+    avail -= rec;
+  } else {
+    if (jb->n_groups == 0 || code_ix / jb->n_groups != (uint32_t)s) return ORC_ECORRUPT;
+    if (read_record(jb->in + jb->off_codes + shared_record_pos(dt, jb->n_groups, code_ix), a, len) != ORC_OK)
+      return ORC_ECORRUPT;
+  }
+  uint64_t nsub = ceil_div(m, jb->S);
+  if (avail < round16(4 * nsub)) return ORC_ECORRUPT;
+  const uint8_t* bs = p + round16(4 * nsub);
+  uint64_t cap_bits = (avail - round16(4 * nsub)) * 8;
+  /* canonical order: symbols sorted by (length, symbol) */
+  uint32_t count[LMAX + 1] = {0};
+  uint8_t sorted[256];
+  int ns_sorted = 0;
+  for (int l = 1; l <= LMAX; l++)
+    for (int k2 = 0; k2 < a; k2++)
+      if (len[k2] == l) {
+        sorted[ns_sorted++] = (uint8_t)k2;
+        count[l]++;
+      }
+  if (get_u32(p) != 0) return ORC_ECORRUPT;
+  for (uint64_t j = 0; j < nsub; j++) {
+    uint64_t t = get_u32(p + 4 * j);
+    if (t > cap_bits) return ORC_ECORRUPT;
+    uint64_t lo = j * jb->S, hi = lo + jb->S < m ? lo + jb->S : m;
+    for (uint64_t i = lo; i < hi; i++) {
+      int v = decode_symbol(bs, cap_bits, &t, count, sorted);
+      if (v < 0) return ORC_ECORRUPT;
+      sym[i] = (uint8_t)v;
+    }
+    if (j + 1 < nsub && t != get_u32(p + 4 * (j + 1))) return ORC_ECORRUPT;
+  }
+  return ORC_OK;
+}
+
+static void* decompress_worker(void* arg) {
+  djob_t* jb = (djob_t*)arg;
+  int ns = orc_n_streams(jb->dtype);
+  uint8_t* sym[4] = {NULL, NULL, NULL, NULL};
+  for (int s = 0; s < ns; s++) {
+    sym[s] = (uint8_t*)malloc(jb->m0);
+    if (!sym[s]) jb->status = ORC_EINVAL;
+  }
+  for (uint64_t c = (uint64_t)jb->thread; c < jb->chunks && jb->status == ORC_OK; c += (uint64_t)jb->threads) {
+    uint64_t lo = c * jb->m0;
+    uint64_t m = lo + jb->m0 <= jb->n ? jb->m0 : jb->n - lo;
+    for (int s = 0; s < ns && jb->status == ORC_OK; s++) {
+      int st = decode_entry(jb, c, s, m, sym[s]);
+      if (st != ORC_OK) jb->status = st;
+    }
+    if (jb->status != ORC_OK) break;
+    for (uint64_t i = 0; i < m; i++) {
+      uint8_t f[4] = {0, 0, 0, 0};
+      for (int s = 0; s < ns; s++) f[s] = sym[s][i];
+      put_value(jb->dtype, jb->out, lo + i, f);
+    }
+  }
+  for (int s = 0; s < ns; s++) free(sym[s]);
+  return NULL;
+}
+
+int orc_decompress(int dtype, const void* in, uint64_t in_bytes, uint64_t n, uint32_t chunk_bytes,
+                   void* out, int threads) {
+  const uint8_t* h = (const uint8_t*)in;
+  if (dtype < 0 || dtype > 2 || !in || !out || n == 0) return ORC_EINVAL;
+  if (chunk_bytes == 0 || chunk_bytes % (uint32_t)value_bytes(dtype) != 0) return ORC_EINVAL;
+  if (in_bytes < HEADER_BYTES) return ORC_ECORRUPT;
+  if (h[0] != 'Z' || h[1] != 'N' || h[2] != 'N' || h[3] != '1' || h[4] != 1 || h[5] != 0) return ORC_ECORRUPT;
+  int ns = orc_n_streams(dtype);
+  uint64_t m0 = chunk_values(dtype, chunk_bytes);
+  uint64_t chunks = ceil_div(n, m0);
+  if (h[6] != dtype || h[7] != ns || get_u64(h + 8) != n || get_u32(h + 16) != chunk_bytes) return ORC_ECORRUPT;
+  uint32_t S = get_u32(h + 20), n_groups = h[57];
+  if (S == 0 || get_u32(h + 24) != chunks || h[56] != LMAX || n_groups > MAX_GROUPS) return ORC_ECORRUPT;
+  if (get_u32(h + 28) != n_groups * (uint32_t)orc_n_entropy(dtype)) return ORC_ECORRUPT;
+  if (h[58] || h[59] || get_u32(h + 60)) return ORC_ECORRUPT;
+  uint64_t off_codes = get_u64(h + 32), off_payload = get_u64(h + 40), total = get_u64(h + 48);
+  if (off_codes != table_end(dtype, chunks) || off_payload != off_codes + shared_bytes(dtype, n_groups))
+    return ORC_ECORRUPT;
+  if (total > in_bytes || total < off_payload) return ORC_ECORRUPT;
+  if (get_u64(h + HEADER_BYTES + 8) != off_payload) return ORC_ECORRUPT;
+  djob_t jb;
+  memset(&jb, 0, sizeof(jb));
+  jb.dtype = dtype;
+  jb.in = h;
+  jb.in_bytes = in_bytes;
+  jb.n = n;
+  jb.m0 = m0;
+  jb.chunks = chunks;
+  jb.total = total;
+  jb.off_codes = off_codes;
+  jb.S = S;
+  jb.n_groups = n_groups;
+  jb.out = (uint8_t*)out;
+  if (threads < 1) threads = 1;
+  if (threads > 256) threads = 256;
+  djob_t* jobs = (djob_t*)malloc(sizeof(djob_t) * (size_t)threads);
+  pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)threads);
+  if (!jobs || !th) {
+    free(jobs);
+    free(th);
+    return ORC_EINVAL;
+  }
+  for (int t = 0; t < threads; t++) {
+    jobs[t] = jb;
+    jobs[t].thread = t;
+    jobs[t].threads = threads;
+    jobs[t].status = ORC_OK;
+  }
+  for (int t = 1; t < threads; t++) pthread_create(&th[t], NULL, decompress_worker, &jobs[t]);
+  decompress_worker(&jobs[0]);
+  for (int t = 1; t < threads; t++) pthread_join(th[t], NULL);
+  int st = ORC_OK;
+  for (int t = 0; t < threads; t++)
+    if (jobs[t].status != ORC_OK) st = jobs[t].status;
+  free(jobs);
+  free(th);
+  return st;
+}
+
+/* ------------------------------------------------------------------ plan (grouping) */
+
+uint64_t orc_splitmix64(uint64_t* state) {
+  uint64_t z = (*state += 0x9E3779B97F4A7C15ull);
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+/* squared Euclidean distance, summed over i in ascending order */
+static double sq_distance(const double* a, const double* b, int dims) {
+  double s = 0.0;
+  for (int i = 0; i < dims; i++) {
+    double t = a[i] - b[i];
+    s = s + t * t;
+  }
+  return s;
+}
+
+/* Grouping by exponent-distribution similarity:
+ *  1. x_c[i] = h_c[i] / m_c for the exponent stream of every chunk c.
+ *  2. If there are no more chunks than groups, chunk c is group c.
+ *  3. Otherwise pick the starting centres with a partial Fisher-Yates shuffle driven
+ *     by SplitMix64(seed): for j < G, r = j + next() mod (C - j), swap, centre j =
+ *     x of the chunk now at position j.
+ *  4. Lloyd passes (at most 100): assign every chunk to its nearest centre (ties to
+ *     the smaller group); stop when no assignment changed; else set every non-empty
+ *     group's centre to the mean of its members (summed in ascending chunk order).
+ *  5. Each group's code for each entropy stream is the length-limited Huffman code of
+ *     the summed histograms of its members (an empty group gets no code). */
+int orc_plan_build(int dtype, const void* src, uint64_t n, uint32_t chunk_bytes, uint32_t n_groups,
+                   uint64_t seed, uint8_t* lens_out, uint32_t* assign_out, int* iters_out,
+                   double* inertia_out) {
+  if (dtype < 0 || dtype > 2 || !src || n == 0 || n_groups == 0 || n_groups > MAX_GROUPS) return ORC_EINVAL;
+  if (chunk_bytes == 0 || chunk_bytes % (uint32_t)value_bytes(dtype) != 0) return ORC_EINVAL;
+  const uint8_t* in = (const uint8_t*)src;
+  int E = orc_n_entropy(dtype), A = orc_alphabet(dtype, 0);
+  uint64_t m0 = chunk_values(dtype, chunk_bytes), C = ceil_div(n, m0), G = n_groups;
+  uint64_t* hist = (uint64_t*)calloc(C * (uint64_t)E * 256, sizeof(uint64_t));
+  double* x = (double*)calloc(C * (uint64_t)A, sizeof(double));
+  double* mu = (double*)calloc(G * (uint64_t)A, sizeof(double));
+  uint32_t* assign = (uint32_t*)malloc(C * sizeof(uint32_t));
+  uint64_t* perm = (uint64_t*)malloc(C * sizeof(uint64_t));
+  if (!hist || !x || !mu || !assign || !perm) {
+    free(hist);
+    free(x);
+    free(mu);
+    free(assign);
+    free(perm);
+    return ORC_EINVAL;
+  }
+  for (uint64_t c = 0; c < C; c++) {
+    uint64_t lo = c * m0, hi = lo + m0 <= n ? lo + m0 : n;
+    for (int e = 0; e < E; e++) orc_histogram(dtype, in, lo, hi, e, hist + (c * (uint64_t)E + (uint64_t)e) * 256);
+    for (int i = 0; i < A; i++) x[c * (uint64_t)A + (uint64_t)i] = (double)hist[c * (uint64_t)E * 256 + (uint64_t)i] / (double)(hi - lo);
+  }
+  int iters = 0;
+  if (C <= G) {
+    for (uint64_t c = 0; c < C; c++) assign[c] = (uint32_t)c;
+  } else {
+    uint64_t state = seed;
+    for (uint64_t c = 0; c < C; c++) perm[c] = c;
+    for (uint64_t j = 0; j < G; j++) {
+      uint64_t r = j + orc_splitmix64(&state) % (C - j);
+      uint64_t tmp = perm[j];
+      perm[j] = perm[r];
+      perm[r] = tmp;
+      memcpy(mu + j * (uint64_t)A, x + perm[j] * (uint64_t)A, sizeof(double) * (size_t)A);
+    }
+    for (uint64_t c = 0; c < C; c++) assign[c] = 0xFFFFFFFFu;
+    for (int it = 0; it < 100; it++) {
+      int changed = 0;
+      double inertia = 0.0;
+      for (uint64_t c = 0; c < C; c++) {
+        uint32_t best = 0;
+        double bd = sq_distance(x + c * (uint64_t)A, mu, A);
+        for (uint64_t j = 1; j < G; j++) {
+          double d = sq_distance(x + c * (uint64_t)A, mu + j * (uint64_t)A, A);
+          if (d < bd) {
+            bd = d;
+            best = (uint32_t)j;
+          }
+        }
+        if (assign[c] != best) changed = 1;
+        assign[c] = best;
+        inertia = inertia + bd;
+      }
+      if (inertia_out) inertia_out[it] = inertia;
+      iters = it + 1;
+      if (!changed) break;
+      for (uint64_t j = 0; j < G; j++) {
+        uint64_t members = 0;
+        for (uint64_t c = 0; c < C; c++)
+          if (assign[c] == j) members++;
+        if (!members) continue;
+        for (int i = 0; i < A; i++) {
+          double s = 0.0;
+          for (uint64_t c = 0; c < C; c++)
+            if (assign[c] == j) s = s + x[c * (uint64_t)A + (uint64_t)i];
+          mu[j * (uint64_t)A + (uint64_t)i] = s / (double)members;
+        }
+      }
+    }
+  }
+  for (int e = 0; e < E; e++) {
+    int a = orc_alphabet(dtype, e);
+    for (uint64_t g = 0; g < G; g++) {
+      uint64_t sum[256];
+      int any = 0;
+      for (int k = 0; k < 256; k++) sum[k] = 0;
+      for (uint64_t c = 0; c < C; c++)
+        if (assign[c] == g)
+          for (int k = 0; k < a; k++) sum[k] += hist[(c * (uint64_t)E + (uint64_t)e) * 256 + (uint64_t)k];
+      uint8_t* lo = lens_out + ((uint64_t)e * G + g) * 256;
+      memset(lo, 0, 256);
+      for (int k = 0; k < a; k++)
+        if (sum[k]) any = 1;
+      if (any) orc_limited_lengths(sum, a, LMAX, lo);
+    }
+  }
+  if (assign_out) memcpy(assign_out, assign, C * sizeof(uint32_t));
+  if (iters_out) *iters_out = iters;
+  free(hist);
+  free(x);
+  free(mu);
+  free(assign);
+  free(perm);
+  return ORC_OK;
+}
