@@ -1,0 +1,169 @@
+/*
+ * zipnn.h -- C ABI of libzipnn_b200: ZipNN-style lossless compression of BF16, FP32
+ * and FP8 (E4M3) tensors on an NVIDIA B200 (sm_100a).
+ *
+ * What the calls compute, by page title and section:
+ *  - "ZipNN: Lossless Compression for AI Models" (abstract) and the THEORY-599 note
+ *    on it, "Per-field compressibility (Table II)": every value is split into its
+ *    exponent field and its sign/fraction bytes; the exponent field is entropy-coded,
+ *    the sign/fraction bytes are stored as they are ("raw"), or omitted when a chunk of
+ *    them is all zero (the "clean" models of the same table).
+ *  - THEORY-599, "Order-0 only (section III-A b)": one order-0 symbol histogram and one
+ *    Huffman code per chunk; no context model.
+ *  - "Lossless Compression of Neural Network Components: Weights, Checkpoints, and K/V
+ *    Caches in Low-Precision Formats" (abstract): FP8 exponent and mantissa are
+ *    entropy-coded independently.
+ *  - "NeuralZip: Reusable Setup for Fast Lossless Compression" (abstract): chunks are
+ *    grouped by the similarity of their exponent distributions, each group shares one
+ *    Huffman code, and this setup (a "plan") is built once and reused.
+ *
+ * Container format (all integers little-endian; every section and payload starts on a
+ * 16-byte boundary; every pad byte and pad bit is zero):
+ *   header, 64 bytes: 'Z','N','N','1' | u16 version=1 | u8 dtype | u8 n_streams |
+ *     u64 n | u32 chunk_bytes | u32 S | u32 n_chunks | u32 n_shared | u64 off_codes |
+ *     u64 off_payload | u64 total_bytes | u8 L_MAX=12 | u8 n_groups | 6 zero bytes
+ *   chunk table at 64: one 16-byte entry per (chunk c, stream s), index k = c*n_streams+s:
+ *     u8 mode (0 RAW, 1 ZERO, 2 HUFF) | 3 zero bytes | u32 code | u64 payload offset.
+ *     code is the shared record index for a HUFF entry coded with a plan's code, and
+ *     0xFFFFFFFF otherwise.
+ *   shared code records at off_codes (n_shared = n_groups * entropy streams), record
+ *     r = e*n_groups + g: code lengths, 4 bits each (byte i = len[2i] | len[2i+1] << 4),
+ *     padded to 16 bytes (128 bytes for a 256-symbol alphabet, 16 for FP8's).
+ *   payloads at off_payload in increasing k, each at the running offset:
+ *     RAW : the chunk's symbols at a fixed width, most significant bit first, padded.
+ *     ZERO: nothing (every symbol of that chunk and stream is 0).
+ *     HUFF: [local code record if code == 0xFFFFFFFF] [u32 idx[ceil(m/S)], padded]
+ *           [bitstream, padded]; idx[j] is the bit offset of symbol j*S.
+ *   Streams: BF16 [exponent, sign+fraction byte]; FP32 [exponent, sign + fraction
+ *   bits 22..16, fraction bits 15..8, fraction bits 7..0]; FP8 E4M3 [exponent (4 bits),
+ *   mantissa (3 bits), sign (1 bit)]. Entropy-coded streams: the exponent, and for FP8
+ *   also the mantissa. Codes are canonical (RFC 1951 rule), at most 12 bits long.
+ *   A stream is ZERO when all its symbols in the chunk are 0; an entropy stream is HUFF
+ *   when that payload is strictly smaller than RAW, else RAW.
+ *
+ * Conventions for every call:
+ *  - Device pointers (src, out, in, ws) are owned by the caller, must be 16-byte
+ *    aligned, and are only read or written on `stream`, in stream order.
+ *  - Compress and decompress are asynchronous; they allocate nothing. Argument errors
+ *    are returned before anything is launched. Errors found on the device (a corrupt
+ *    container, a container that does not match the arguments) are written to the
+ *    workspace and returned by zipnn_get_status.
+ *  - `ws` is scratch owned by the caller, at least zipnn_workspace_bytes(...) bytes.
+ *    One workspace must not be used by two calls that may run at the same time.
+ */
+#ifndef ZIPNN_H
+#define ZIPNN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* zipnn_stream_t;
+
+typedef enum { ZIPNN_BF16 = 0, ZIPNN_FP32 = 1, ZIPNN_FP8_E4M3 = 2 } zipnn_dtype;
+
+typedef enum {
+  ZIPNN_OK = 0,
+  ZIPNN_ERR_INVALID_ARG = 1,  /* bad pointer, size, alignment or dtype */
+  ZIPNN_ERR_OUT_TOO_SMALL = 2, /* out_cap or ws_bytes below the required size */
+  ZIPNN_ERR_CORRUPT = 3,       /* container damaged or not matching the arguments */
+  ZIPNN_ERR_PLAN_MISMATCH = 4, /* plan made for another dtype */
+  ZIPNN_ERR_CUDA = 5,          /* a CUDA runtime call failed */
+  ZIPNN_ERR_UNSUPPORTED = 6,   /* no sm_100 device, or a size beyond the limits below */
+  ZIPNN_ERR_TIMEOUT = 7        /* a bounded device-side wait gave up (never expected) */
+} zipnn_status;
+
+typedef struct zipnn_plan zipnn_plan_t; /* opaque; owns device code tables */
+
+#define ZIPNN_DEFAULT_CHUNK_BYTES 262144u /* 256 KiB of uncompressed values per chunk */
+#define ZIPNN_DEFAULT_SUBBLOCK 1024u      /* symbols per sub-block index entry */
+#define ZIPNN_MAX_GROUPS 64u
+#define ZIPNN_LMAX 12u
+
+/* Upper bound of the container size for n values: header, chunk table, room for
+ * ZIPNN_MAX_GROUPS shared records, and every payload stored RAW (a HUFF payload is
+ * only chosen when it is smaller). Returns 0 for invalid arguments.
+ * chunk_bytes: a multiple of 16 in [16, 2^30]. */
+size_t zipnn_max_compressed_bytes(zipnn_dtype dtype, uint64_t n, uint32_t chunk_bytes);
+
+/* Bytes of device scratch that compress, decompress and plan creation need for n
+ * values; the same size serves every call on tensors of at most n values. */
+size_t zipnn_workspace_bytes(zipnn_dtype dtype, uint64_t n, uint32_t chunk_bytes);
+
+/* Compress n values at `src` (device) into the container at `out` (device, out_cap
+ * bytes, out_cap >= zipnn_max_compressed_bytes). Each chunk_bytes of input is one
+ * chunk with its own order-0 histogram and Huffman code (THEORY-599, "Order-0 only");
+ * with a plan, a chunk takes the cheapest shared group code that covers its symbols
+ * (NeuralZip, abstract), or a local code when none does. The container size is
+ * written at out+48 (read it with zipnn_compressed_size). Sub-blocks of
+ * ZIPNN_DEFAULT_SUBBLOCK symbols. */
+zipnn_status zipnn_compress(zipnn_dtype dtype, const void* src, uint64_t n, uint32_t chunk_bytes,
+                            const zipnn_plan_t* plan, void* out, size_t out_cap, void* ws,
+                            size_t ws_bytes, zipnn_stream_t stream);
+
+/* As zipnn_compress with an explicit sub-block length S (a multiple of 16 in
+ * [16, 65536]; 0 selects ZIPNN_DEFAULT_SUBBLOCK). A shorter S gives the decoder more
+ * parallel work at 32 bits of index per S symbols. */
+zipnn_status zipnn_compress_ex(zipnn_dtype dtype, const void* src, uint64_t n, uint32_t chunk_bytes,
+                               uint32_t subblock, const zipnn_plan_t* plan, void* out, size_t out_cap,
+                               void* ws, size_t ws_bytes, zipnn_stream_t stream);
+
+/* Decompress the container `in` (device, in_bytes readable bytes) into n values at
+ * `out` (device). The container must have been made for the same dtype, n and
+ * chunk_bytes; anything else, and any damage found, sets ZIPNN_ERR_CORRUPT in the
+ * workspace (output contents are then unspecified). Every read stays inside in_bytes. */
+zipnn_status zipnn_decompress(zipnn_dtype dtype, const void* in, size_t in_bytes, uint64_t n,
+                              uint32_t chunk_bytes, void* out, void* ws, size_t ws_bytes,
+                              zipnn_stream_t stream);
+
+/* Wait for `stream`, then read the container size from the header at `out`. */
+zipnn_status zipnn_compressed_size(const void* out, zipnn_stream_t stream, uint64_t* bytes);
+
+/* Wait for `stream`, then return the device-side status of the last call on `ws`. */
+zipnn_status zipnn_get_status(const void* ws, zipnn_stream_t stream);
+
+/* Order-0 histograms (step "split + histogram" alone): hist_out (device, u32) receives
+ * n_chunks x n_entropy x 256 counts for the entropy streams of every chunk. */
+zipnn_status zipnn_histogram(zipnn_dtype dtype, const void* src, uint64_t n, uint32_t chunk_bytes,
+                             uint32_t* hist_out, zipnn_stream_t stream);
+
+/* Code lengths (step "code build" alone): for `count` histograms of 256 u64 counts
+ * (device), writes 256 length bytes each (device): minimum-variance Huffman lengths
+ * with ties by (weight, order), limited to ZIPNN_LMAX by halving the counts. Symbols
+ * at or above `alphabet` must have count 0. */
+zipnn_status zipnn_code_lengths(const uint64_t* hist, uint32_t count, uint32_t alphabet, uint8_t* lens_out,
+                                zipnn_stream_t stream);
+
+/* Build a plan on the tensor at `src`: k-means (Lloyd, SplitMix64(seed) seeding, at
+ * most 100 passes) over the chunks' normalised exponent histograms into `groups`
+ * groups (1..ZIPNN_MAX_GROUPS), then one length-limited Huffman code per group and
+ * entropy stream from the group's summed histograms. Setup call: it allocates the
+ * plan's device tables and synchronises `stream`. ws as for compress. */
+zipnn_status zipnn_plan_create(zipnn_dtype dtype, const void* src, uint64_t n, uint32_t chunk_bytes,
+                               uint32_t groups, uint64_t seed, void* ws, size_t ws_bytes,
+                               zipnn_stream_t stream, zipnn_plan_t** plan);
+
+/* Serialise a plan into host memory: "ZNP1", u8 dtype, u8 groups, 2 zero bytes, then
+ * the code records as in the container. *bytes receives the size; host_buf may be NULL
+ * to query it. */
+zipnn_status zipnn_plan_export(const zipnn_plan_t* plan, void* host_buf, size_t cap, size_t* bytes);
+
+/* Rebuild a plan from exported bytes (host memory); allocates its device tables. */
+zipnn_status zipnn_plan_import(const void* host_buf, size_t bytes, zipnn_plan_t** plan);
+
+/* Per-chunk group chosen by the plan's k-means (host memory, n_chunks entries of the
+ * tensor the plan was built on); *count receives the number of entries. */
+zipnn_status zipnn_plan_assignment(const zipnn_plan_t* plan, uint32_t* host_buf, size_t cap, size_t* count);
+
+void zipnn_plan_destroy(zipnn_plan_t* plan);
+
+const char* zipnn_status_string(zipnn_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,424 @@
+// api.cu -- the C ABI of include/zipnn.h: argument checks, workspace carving, launches.
+// No call here computes any part of the codec on the host: histograms, codes, layout,
+// encoding, decoding and the plan's grouping all run in the kernels.
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "zipnn.h"
+#include "common.cuh"
+#include "launch.h"
+
+using namespace zipnn;
+
+struct zipnn_plan {
+  int dt;
+  uint32_t groups;
+  uint8_t* d_lens;   // [n_entropy][groups][256]
+  uint32_t* d_enc;   // [n_entropy][groups][256]
+  std::vector<uint8_t> h_lens;
+  std::vector<uint32_t> assign;
+};
+
+namespace {
+
+constexpr uint64_t kAlign = 256;
+constexpr uint32_t kMaxChunkBytes = 1u << 28;
+
+inline uint64_t align_up(uint64_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+inline bool valid_dtype(int dt) { return dt == kBF16 || dt == kFP32 || dt == kFP8; }
+
+bool make_geo(int dt, uint64_t n, uint32_t chunk_bytes, uint32_t S, uint32_t G, Geo& g) {
+  if (!valid_dtype(dt) || n == 0) return false;
+  if (chunk_bytes < 16 || chunk_bytes % 16 || chunk_bytes > kMaxChunkBytes) return false;
+  if (S < 16 || S % 16 || S > 65536) return false;
+  g.dt = dt;
+  g.n = n;
+  g.chunk_bytes = chunk_bytes;
+  g.m0 = chunk_bytes / (uint32_t)value_bytes(dt);
+  const uint64_t chunks = ceil_div(n, g.m0);
+  const uint64_t tpc = ceil_div(g.m0, kTileValues);
+  if (chunks * (uint64_t)n_streams(dt) > 0x7FFFFFFFull || chunks * tpc > 0x7FFFFFFFull) return false;
+  g.n_chunks = (uint32_t)chunks;
+  g.S = S;
+  g.n_groups = G;
+  g.tiles_per_chunk = (uint32_t)tpc;
+  g.n_tiles = (uint32_t)(chunks * tpc);
+  g.n_entries = (uint32_t)(chunks * n_streams(dt));
+  g.off_codes = kHeaderBytes + (uint64_t)kEntryBytes * g.n_entries;
+  g.off_payload = g.off_codes + shared_bytes(dt, G);
+  return true;
+}
+
+struct WsPlan {
+  uint64_t status, hist, nonzero, scan_desc, tile_desc, slot, zero_end;
+  uint64_t esize, emode, ecode, eoff, enc;
+  uint64_t km_mu, km_perm, km_assign, km_changed, km_gsum, total;
+};
+
+WsPlan ws_plan(const Geo& g) {
+  const uint64_t C = g.n_chunks, NE = (uint64_t)n_entropy(g.dt), K = g.n_entries;
+  WsPlan p;
+  uint64_t o = 0;
+  p.status = o;     o = align_up(o + 256);
+  p.hist = o;       o = align_up(o + C * NE * 256 * 4);
+  p.nonzero = o;    o = align_up(o + K * 4);
+  p.scan_desc = o;  o = align_up(o + (uint64_t)layout_tiles(g.n_entries) * 8);
+  p.tile_desc = o;  o = align_up(o + NE * g.n_tiles * 8);
+  p.slot = o;       o = align_up(o + NE * g.n_tiles * 8);
+  p.zero_end = o;
+  p.esize = o;      o = align_up(o + K * 8);
+  p.emode = o;      o = align_up(o + K * 4);
+  p.ecode = o;      o = align_up(o + K * 4);
+  p.eoff = o;       o = align_up(o + K * 8);
+  p.enc = o;        o = align_up(o + C * NE * 256 * 4);
+  p.km_mu = o;      o = align_up(o + (uint64_t)kMaxGroups * 256 * 8);
+  p.km_perm = o;    o = align_up(o + C * 4);
+  p.km_assign = o;  o = align_up(o + C * 4);
+  p.km_changed = o; o = align_up(o + 4);
+  p.km_gsum = o;    o = align_up(o + NE * kMaxGroups * 256 * 8);
+  p.total = o;
+  return p;
+}
+
+Ws carve(const WsPlan& p, void* base) {
+  uint8_t* b = static_cast<uint8_t*>(base);
+  Ws w;
+  w.status = reinterpret_cast<uint32_t*>(b + p.status);
+  w.hist = reinterpret_cast<uint32_t*>(b + p.hist);
+  w.nonzero = reinterpret_cast<uint32_t*>(b + p.nonzero);
+  w.scan_desc = reinterpret_cast<uint64_t*>(b + p.scan_desc);
+  w.tile_desc = reinterpret_cast<uint64_t*>(b + p.tile_desc);
+  w.slot = reinterpret_cast<uint64_t*>(b + p.slot);
+  w.esize = reinterpret_cast<uint64_t*>(b + p.esize);
+  w.emode = reinterpret_cast<uint32_t*>(b + p.emode);
+  w.ecode = reinterpret_cast<uint32_t*>(b + p.ecode);
+  w.eoff = reinterpret_cast<uint64_t*>(b + p.eoff);
+  w.enc = reinterpret_cast<uint32_t*>(b + p.enc);
+  return w;
+}
+
+uint64_t max_bytes(const Geo& g) {
+  uint64_t total = g.off_codes + shared_bytes(g.dt, kMaxGroups);
+  const uint64_t full = g.n / g.m0, tail = g.n % g.m0;
+  for (int s = 0; s < n_streams(g.dt); s++) {
+    const int w = raw_width(g.dt, s);
+    total += full * raw_payload(g.m0, w);
+    if (tail) total += raw_payload(tail, w);
+  }
+  return total;
+}
+
+zipnn_status cuda_status(cudaError_t e) { return e == cudaSuccess ? ZIPNN_OK : ZIPNN_ERR_CUDA; }
+
+PlanDev plan_dev(const zipnn_plan* p) {
+  PlanDev d;
+  d.lens = p ? p->d_lens : nullptr;
+  d.enc = p ? p->d_enc : nullptr;
+  d.groups = p ? p->groups : 0;
+  return d;
+}
+
+bool device_ok() {
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
+  return major == 10;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t zipnn_max_compressed_bytes(zipnn_dtype dtype, uint64_t n, uint32_t chunk_bytes) {
+  Geo g;
+  if (!make_geo(dtype, n, chunk_bytes, ZIPNN_DEFAULT_SUBBLOCK, 0, g)) return 0;
+  return (size_t)max_bytes(g);
+}
+
+size_t zipnn_workspace_bytes(zipnn_dtype dtype, uint64_t n, uint32_t chunk_bytes) {
+  Geo g;
+  if (!make_geo(dtype, n, chunk_bytes, ZIPNN_DEFAULT_SUBBLOCK, 0, g)) return 0;
+  return (size_t)ws_plan(g).total;
+}
+
+zipnn_status zipnn_compress_ex(zipnn_dtype dtype, const void* src, uint64_t n, uint32_t chunk_bytes, uint32_t subblock,
+                               const zipnn_plan_t* plan, void* out, size_t out_cap, void* ws, size_t ws_bytes,
+                               zipnn_stream_t stream) {
+  if (subblock == 0) subblock = ZIPNN_DEFAULT_SUBBLOCK;
+  if (!src || !out || !ws || !aligned16(src) || !aligned16(out) || !aligned16(ws)) return ZIPNN_ERR_INVALID_ARG;
+  if (plan && plan->dt != (int)dtype) return ZIPNN_ERR_PLAN_MISMATCH;
+  Geo g;
+  if (!make_geo(dtype, n, chunk_bytes, subblock, plan ? plan->groups : 0, g)) return ZIPNN_ERR_INVALID_ARG;
+  if (out_cap < max_bytes(g)) return ZIPNN_ERR_OUT_TOO_SMALL;
+  const WsPlan wp = ws_plan(g);
+  if (ws_bytes < wp.total) return ZIPNN_ERR_OUT_TOO_SMALL;
+  if (!device_ok()) return ZIPNN_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const Ws w = carve(wp, ws);
+  const PlanDev pd = plan_dev(plan);
+  cudaError_t e = cudaMemsetAsync(ws, 0, wp.zero_end, st);
+  if (e == cudaSuccess) e = launch_split_hist(src, g, w.hist, w.nonzero, st);
+  if (e == cudaSuccess) e = launch_build_tables(g, w, pd, st);
+  if (e == cudaSuccess) e = launch_layout(g, w, pd, static_cast<uint8_t*>(out), st);
+  if (e == cudaSuccess) e = launch_encode(src, g, w, static_cast<uint8_t*>(out), st);
+  return cuda_status(e);
+}
+
+zipnn_status zipnn_compress(zipnn_dtype dtype, const void* src, uint64_t n, uint32_t chunk_bytes,
+                            const zipnn_plan_t* plan, void* out, size_t out_cap, void* ws, size_t ws_bytes,
+                            zipnn_stream_t stream) {
+  return zipnn_compress_ex(dtype, src, n, chunk_bytes, 0, plan, out, out_cap, ws, ws_bytes, stream);
+}
+
+zipnn_status zipnn_decompress(zipnn_dtype dtype, const void* in, size_t in_bytes, uint64_t n, uint32_t chunk_bytes,
+                              void* out, void* ws, size_t ws_bytes, zipnn_stream_t stream) {
+  if (!in || !out || !ws || !aligned16(in) || !aligned16(out) || !aligned16(ws)) return ZIPNN_ERR_INVALID_ARG;
+  Geo g;
+  if (!make_geo(dtype, n, chunk_bytes, ZIPNN_DEFAULT_SUBBLOCK, 0, g)) return ZIPNN_ERR_INVALID_ARG;
+  if (ws_bytes < 256) return ZIPNN_ERR_OUT_TOO_SMALL;
+  if (!device_ok()) return ZIPNN_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(ws, 0, 4, st);
+  if (e == cudaSuccess)
+    e = launch_decode(static_cast<const uint8_t*>(in), in_bytes, g, static_cast<uint8_t*>(out),
+                      static_cast<uint32_t*>(ws), st);
+  return cuda_status(e);
+}
+
+zipnn_status zipnn_compressed_size(const void* out, zipnn_stream_t stream, uint64_t* bytes) {
+  if (!out || !bytes) return ZIPNN_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint64_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, static_cast<const uint8_t*>(out) + 48, 8, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return ZIPNN_ERR_CUDA;
+  *bytes = v;
+  return ZIPNN_OK;
+}
+
+zipnn_status zipnn_get_status(const void* ws, zipnn_stream_t stream) {
+  if (!ws) return ZIPNN_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, ws, 4, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return ZIPNN_ERR_CUDA;
+  return (zipnn_status)v;
+}
+
+zipnn_status zipnn_histogram(zipnn_dtype dtype, const void* src, uint64_t n, uint32_t chunk_bytes, uint32_t* hist_out,
+                             zipnn_stream_t stream) {
+  if (!src || !hist_out || !aligned16(src)) return ZIPNN_ERR_INVALID_ARG;
+  Geo g;
+  if (!make_geo(dtype, n, chunk_bytes, ZIPNN_DEFAULT_SUBBLOCK, 0, g)) return ZIPNN_ERR_INVALID_ARG;
+  if (!device_ok()) return ZIPNN_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(hist_out, 0, (size_t)g.n_chunks * n_entropy(dtype) * 256 * 4, st);
+  if (e == cudaSuccess) e = launch_split_hist(src, g, hist_out, nullptr, st);
+  return cuda_status(e);
+}
+
+zipnn_status zipnn_code_lengths(const uint64_t* hist, uint32_t count, uint32_t alphabet, uint8_t* lens_out,
+                                zipnn_stream_t stream) {
+  if (!hist || !lens_out || alphabet < 1 || alphabet > 256) return ZIPNN_ERR_INVALID_ARG;
+  if (!device_ok()) return ZIPNN_ERR_UNSUPPORTED;
+  return cuda_status(launch_code_lengths(hist, count, alphabet, lens_out, nullptr, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+static zipnn_status plan_alloc(int dt, uint32_t groups, zipnn_plan** out) {
+  zipnn_plan* p = new (std::nothrow) zipnn_plan();
+  if (!p) return ZIPNN_ERR_INVALID_ARG;
+  p->dt = dt;
+  p->groups = groups;
+  const size_t recs = (size_t)n_entropy(dt) * groups;
+  if (cudaMalloc(&p->d_lens, recs * 256) != cudaSuccess) {
+    delete p;
+    return ZIPNN_ERR_CUDA;
+  }
+  if (cudaMalloc(&p->d_enc, recs * 256 * 4) != cudaSuccess) {
+    cudaFree(p->d_lens);
+    delete p;
+    return ZIPNN_ERR_CUDA;
+  }
+  p->h_lens.assign(recs * 256, 0);
+  *out = p;
+  return ZIPNN_OK;
+}
+
+zipnn_status zipnn_plan_create(zipnn_dtype dtype, const void* src, uint64_t n, uint32_t chunk_bytes, uint32_t groups,
+                               uint64_t seed, void* ws, size_t ws_bytes, zipnn_stream_t stream, zipnn_plan_t** plan) {
+  if (!src || !ws || !plan || !aligned16(src) || !aligned16(ws)) return ZIPNN_ERR_INVALID_ARG;
+  if (groups < 1 || groups > kMaxGroups) return ZIPNN_ERR_INVALID_ARG;
+  Geo g;
+  if (!make_geo(dtype, n, chunk_bytes, ZIPNN_DEFAULT_SUBBLOCK, 0, g)) return ZIPNN_ERR_INVALID_ARG;
+  const WsPlan wp = ws_plan(g);
+  if (ws_bytes < wp.total) return ZIPNN_ERR_OUT_TOO_SMALL;
+  if (!device_ok()) return ZIPNN_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  const Ws w = carve(wp, ws);
+  const int NE = n_entropy(dtype);
+  KmeansDev k;
+  k.hist = w.hist;
+  k.C = g.n_chunks;
+  k.A = (uint32_t)alphabet(dtype, 0);
+  k.NE = (uint32_t)NE;
+  k.G = groups;
+  k.m0 = g.m0;
+  k.n = n;
+  k.mu = reinterpret_cast<double*>(b + wp.km_mu);
+  k.perm = reinterpret_cast<uint32_t*>(b + wp.km_perm);
+  k.assign = reinterpret_cast<uint32_t*>(b + wp.km_assign);
+  k.changed = reinterpret_cast<uint32_t*>(b + wp.km_changed);
+  k.gsum = reinterpret_cast<uint64_t*>(b + wp.km_gsum);
+  zipnn_plan* p = nullptr;
+  zipnn_status zs = plan_alloc(dtype, groups, &p);
+  if (zs != ZIPNN_OK) return zs;
+  cudaError_t e = cudaMemsetAsync(ws, 0, wp.zero_end, st);
+  if (e == cudaSuccess) e = launch_split_hist(src, g, w.hist, nullptr, st);
+  if (e == cudaSuccess) {
+    if (g.n_chunks <= groups) {
+      e = launch_identity_assign(k.assign, k.C, st);
+    } else {
+      e = launch_kmeans_init(k, seed, st);
+      for (int it = 0; it < 100 && e == cudaSuccess; it++) {
+        uint32_t changed = 0;
+        e = cudaMemsetAsync(k.changed, 0, 4, st);
+        if (e == cudaSuccess) e = launch_kmeans_assign(k, st);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(&changed, k.changed, 4, cudaMemcpyDeviceToHost, st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess || !changed) break;
+        e = launch_kmeans_update(k, st);
+      }
+    }
+  }
+  if (e == cudaSuccess) e = cudaMemsetAsync(k.gsum, 0, (size_t)NE * groups * 256 * 8, st);
+  if (e == cudaSuccess) e = launch_group_sums(k, st);
+  for (int ei = 0; ei < NE && e == cudaSuccess; ei++)
+    e = launch_code_lengths(k.gsum + (size_t)ei * groups * 256, groups, (uint32_t)alphabet(dtype, ei),
+                            p->d_lens + (size_t)ei * groups * 256, p->d_enc + (size_t)ei * groups * 256, st);
+  if (e == cudaSuccess) {
+    p->assign.resize(g.n_chunks);
+    e = cudaMemcpyAsync(p->h_lens.data(), p->d_lens, p->h_lens.size(), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(p->assign.data(), k.assign, (size_t)g.n_chunks * 4, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  }
+  if (e != cudaSuccess) {
+    zipnn_plan_destroy(p);
+    return ZIPNN_ERR_CUDA;
+  }
+  *plan = p;
+  return ZIPNN_OK;
+}
+
+zipnn_status zipnn_plan_export(const zipnn_plan_t* plan, void* host_buf, size_t cap, size_t* bytes) {
+  if (!plan || !bytes) return ZIPNN_ERR_INVALID_ARG;
+  const int dt = plan->dt, NE = n_entropy(dt);
+  const size_t need = 8 + shared_bytes(dt, plan->groups);
+  *bytes = need;
+  if (!host_buf) return ZIPNN_OK;
+  if (cap < need) return ZIPNN_ERR_OUT_TOO_SMALL;
+  uint8_t* o = static_cast<uint8_t*>(host_buf);
+  std::memset(o, 0, need);
+  o[0] = 'Z';
+  o[1] = 'N';
+  o[2] = 'P';
+  o[3] = '1';
+  o[4] = (uint8_t)dt;
+  o[5] = (uint8_t)plan->groups;
+  for (int e = 0; e < NE; e++) {
+    const int A = alphabet(dt, e);
+    for (uint32_t gi = 0; gi < plan->groups; gi++) {
+      const uint8_t* l = plan->h_lens.data() + ((size_t)e * plan->groups + gi) * 256;
+      uint8_t* r = o + 8 + shared_record_pos(dt, plan->groups, (uint32_t)e * plan->groups + gi);
+      for (int i = 0; i < A / 2; i++) r[i] = (uint8_t)(l[2 * i] | (l[2 * i + 1] << 4));
+    }
+  }
+  return ZIPNN_OK;
+}
+
+zipnn_status zipnn_plan_import(const void* host_buf, size_t bytes, zipnn_plan_t** plan) {
+  if (!host_buf || !plan || bytes < 8) return ZIPNN_ERR_INVALID_ARG;
+  const uint8_t* in = static_cast<const uint8_t*>(host_buf);
+  if (in[0] != 'Z' || in[1] != 'N' || in[2] != 'P' || in[3] != '1' || in[6] || in[7]) return ZIPNN_ERR_CORRUPT;
+  const int dt = in[4];
+  const uint32_t groups = in[5];
+  if (!valid_dtype(dt) || groups < 1 || groups > kMaxGroups) return ZIPNN_ERR_CORRUPT;
+  if (bytes < 8 + shared_bytes(dt, groups)) return ZIPNN_ERR_CORRUPT;
+  if (!device_ok()) return ZIPNN_ERR_UNSUPPORTED;
+  zipnn_plan* p = nullptr;
+  zipnn_status zs = plan_alloc(dt, groups, &p);
+  if (zs != ZIPNN_OK) return zs;
+  const int NE = n_entropy(dt);
+  for (int e = 0; e < NE; e++) {
+    const int A = alphabet(dt, e);
+    const uint32_t rb = record_bytes(dt, e);
+    for (uint32_t gi = 0; gi < groups; gi++) {
+      const uint8_t* r = in + 8 + shared_record_pos(dt, groups, (uint32_t)e * groups + gi);
+      uint8_t* l = p->h_lens.data() + ((size_t)e * groups + gi) * 256;
+      uint64_t kraft = 0;
+      for (int i = 0; i < A; i++) {
+        l[i] = (i & 1) ? (r[i >> 1] >> 4) : (r[i >> 1] & 15);
+        if (l[i] > kLmax) {
+          zipnn_plan_destroy(p);
+          return ZIPNN_ERR_CORRUPT;
+        }
+        if (l[i]) kraft += 1ull << (kLmax - l[i]);
+      }
+      for (uint32_t i = (uint32_t)A / 2; i < rb; i++)
+        if (r[i]) {
+          zipnn_plan_destroy(p);
+          return ZIPNN_ERR_CORRUPT;
+        }
+      if (kraft > (1ull << kLmax)) {
+        zipnn_plan_destroy(p);
+        return ZIPNN_ERR_CORRUPT;
+      }
+    }
+  }
+  cudaError_t e = cudaMemcpy(p->d_lens, p->h_lens.data(), p->h_lens.size(), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = launch_canonical(p->d_lens, (uint32_t)NE * groups, p->d_enc, 0);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    zipnn_plan_destroy(p);
+    return ZIPNN_ERR_CUDA;
+  }
+  *plan = p;
+  return ZIPNN_OK;
+}
+
+zipnn_status zipnn_plan_assignment(const zipnn_plan_t* plan, uint32_t* host_buf, size_t cap, size_t* count) {
+  if (!plan || !count) return ZIPNN_ERR_INVALID_ARG;
+  *count = plan->assign.size();
+  if (!host_buf) return ZIPNN_OK;
+  if (cap < plan->assign.size()) return ZIPNN_ERR_OUT_TOO_SMALL;
+  std::memcpy(host_buf, plan->assign.data(), plan->assign.size() * 4);
+  return ZIPNN_OK;
+}
+
+void zipnn_plan_destroy(zipnn_plan_t* plan) {
+  if (!plan) return;
+  if (plan->d_lens) cudaFree(plan->d_lens);
+  if (plan->d_enc) cudaFree(plan->d_enc);
+  delete plan;
+}
+
+const char* zipnn_status_string(zipnn_status status) {
+  switch (status) {
+    case ZIPNN_OK: return "ok";
+    case ZIPNN_ERR_INVALID_ARG: return "invalid argument";
+    case ZIPNN_ERR_OUT_TOO_SMALL: return "output or workspace too small";
+    case ZIPNN_ERR_CORRUPT: return "corrupt container or arguments that do not match it";
+    case ZIPNN_ERR_PLAN_MISMATCH: return "plan made for another dtype";
+    case ZIPNN_ERR_CUDA: return "CUDA runtime error";
+    case ZIPNN_ERR_UNSUPPORTED: return "unsupported device or size";
+    case ZIPNN_ERR_TIMEOUT: return "device-side wait gave up";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,177 @@
+// common.cuh -- device-side definitions shared by the kernels of libzipnn_b200.
+//
+// The container layout these constants describe is the one documented in
+// include/zipnn.h. This file is the CUDA library's own statement of it; the CPU
+// oracle under oracle/ states it independently.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda/atomic>
+
+namespace zipnn {
+
+constexpr int kLmax = 12;
+constexpr uint32_t kNoCode = 0xFFFFFFFFu;
+constexpr uint32_t kModeRaw = 0, kModeZero = 1, kModeHuff = 2;
+constexpr int kBF16 = 0, kFP32 = 1, kFP8 = 2;
+constexpr int kHeaderBytes = 64, kEntryBytes = 16;
+constexpr uint32_t kMaxGroups = 64;
+
+// Device status codes (the public zipnn_status values).
+constexpr uint32_t kStCorrupt = 3, kStTimeout = 7;
+
+// Values one thread owns in the compress kernels, and values per encode tile.
+constexpr int kGroupValues = 16;
+constexpr int kEncodeThreads = 256;
+constexpr int kTileValues = kEncodeThreads * kGroupValues;  // 4096
+
+__host__ __device__ constexpr int n_streams(int dt) { return dt == kBF16 ? 2 : dt == kFP32 ? 4 : 3; }
+__host__ __device__ constexpr int n_entropy(int dt) { return dt == kFP8 ? 2 : 1; }
+__host__ __device__ constexpr int value_bytes(int dt) { return dt == kBF16 ? 2 : dt == kFP32 ? 4 : 1; }
+// bits per symbol of a stream stored RAW
+__host__ __device__ constexpr int raw_width(int dt, int s) {
+  return dt == kFP8 ? (s == 0 ? 4 : s == 1 ? 3 : 1) : 8;
+}
+__host__ __device__ constexpr int alphabet(int dt, int s) { return 1 << raw_width(dt, s); }
+__host__ __device__ constexpr bool is_entropy(int dt, int s) { return s == 0 || (dt == kFP8 && s == 1); }
+__host__ __device__ constexpr uint64_t min64(uint64_t a, uint64_t b) { return a < b ? a : b; }
+__host__ __device__ constexpr uint32_t min32(uint32_t a, uint32_t b) { return a < b ? a : b; }
+__host__ __device__ constexpr uint64_t round16(uint64_t x) { return (x + 15) & ~uint64_t(15); }
+__host__ __device__ constexpr uint64_t ceil_div(uint64_t a, uint64_t b) { return (a + b - 1) / b; }
+__host__ __device__ constexpr uint32_t record_bytes(int dt, int s) { return (uint32_t)round16(alphabet(dt, s) / 2); }
+__host__ __device__ constexpr uint64_t raw_payload(uint64_t m, int w) { return round16(ceil_div(m * (uint64_t)w, 8)); }
+
+// Bytes of all shared code records for g groups, and the position of record r.
+__host__ __device__ inline uint64_t shared_bytes(int dt, uint32_t g) {
+  uint64_t b = 0;
+  for (int e = 0; e < n_entropy(dt); e++) b += (uint64_t)g * record_bytes(dt, e);
+  return b;
+}
+__host__ __device__ inline uint64_t shared_record_pos(int dt, uint32_t g, uint32_t r) {
+  uint32_t e = r / g, k = r % g;
+  uint64_t pos = 0;
+  for (uint32_t i = 0; i < e; i++) pos += (uint64_t)g * record_bytes(dt, (int)i);
+  return pos + (uint64_t)k * record_bytes(dt, (int)e);
+}
+
+// Geometry of one call.
+struct Geo {
+  int dt;
+  uint64_t n;
+  uint32_t chunk_bytes, m0, n_chunks, S;
+  uint32_t n_groups;          // 0 without a plan
+  uint32_t tiles_per_chunk;   // encode tiles per chunk
+  uint32_t n_tiles;           // n_chunks * tiles_per_chunk
+  uint32_t n_entries;         // n_chunks * n_streams
+  uint64_t off_codes, off_payload;
+};
+
+// Workspace carve-up (device pointers). The first group is cleared by every
+// compress call; the rest is fully overwritten before it is read.
+struct Ws {
+  uint32_t* status;     // [0] status, [1] encode ticket, [2] layout ticket
+  uint32_t* hist;       // [n_chunks][n_entropy][256]
+  uint32_t* nonzero;    // [n_entries]: OR of the stream's symbols
+  uint64_t* scan_desc;  // [layout tiles] look-back descriptors
+  uint64_t* tile_desc;  // [n_tiles][n_entropy] look-back descriptors
+  uint64_t* slot;       // [n_tiles][n_entropy] shared boundary words
+  uint64_t* esize;      // [n_entries] payload bytes
+  uint32_t* emode;      // [n_entries]
+  uint32_t* ecode;      // [n_entries]
+  uint64_t* eoff;       // [n_entries] payload offsets
+  uint32_t* enc;        // [n_chunks][n_entropy][256]: len << 16 | code
+};
+
+// Device-side tables of a plan.
+struct PlanDev {
+  const uint8_t* lens;  // [n_entropy][groups][256]
+  const uint32_t* enc;  // [n_entropy][groups][256]: len << 16 | code
+  uint32_t groups;
+};
+
+__device__ __forceinline__ void set_status(uint32_t* st, uint32_t code) { atomicCAS(st, 0u, code); }
+
+__device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
+
+// ---------------------------------------------------------------- look-back
+// Descriptor: bits 63..62 flag (0 empty, 1 aggregate, 2 inclusive prefix), 61..0 value.
+constexpr uint64_t kFlagAgg = 1ull << 62, kFlagPrefix = 2ull << 62, kValueMask = (1ull << 62) - 1;
+// Spin limit for every wait on another block; after it the wait records a timeout and
+// continues, so no kernel can hang on a descriptor that is never written.
+constexpr uint32_t kSpinLimit = 1u << 22;
+
+__device__ __forceinline__ void publish(uint64_t* d, uint64_t v) {
+  cuda::atomic_ref<uint64_t, cuda::thread_scope_device> a(*d);
+  a.store(v, cuda::memory_order_release);
+}
+__device__ __forceinline__ uint64_t observe(uint64_t* d) {
+  cuda::atomic_ref<uint64_t, cuda::thread_scope_device> a(*d);
+  return a.load(cuda::memory_order_acquire);
+}
+
+// Single-pass decoupled look-back (one thread): publish this tile's aggregate, walk
+// back over the predecessors of the same segment (tiles first..tile-1), summing
+// aggregates until an inclusive prefix is found, publish the inclusive prefix and
+// return the exclusive one. Tiles are handed out in launch order (a ticket), so every
+// predecessor has started and the walk ends; the spin limit only guards against bugs.
+__device__ inline uint64_t lookback(uint64_t* desc, uint32_t tile, uint32_t first, uint64_t aggregate,
+                                    uint32_t* status) {
+  if (tile == first) {
+    publish(desc + tile, kFlagPrefix | aggregate);
+    return 0;
+  }
+  publish(desc + tile, kFlagAgg | aggregate);
+  uint64_t excl = 0;
+  uint32_t j = tile - 1;
+  while (true) {
+    uint64_t d = observe(desc + j);
+    uint32_t spins = 0;
+    while ((d >> 62) == 0) {
+      if (++spins > kSpinLimit) {
+        set_status(status, kStTimeout);
+        d = kFlagPrefix;  // give up: treat as prefix 0
+        break;
+      }
+      __nanosleep(spins < 64 ? 32 : 256);
+      d = observe(desc + j);
+    }
+    excl += d & kValueMask;
+    if ((d >> 62) == 2 || j == first) break;
+    j--;
+  }
+  publish(desc + tile, kFlagPrefix | (excl + aggregate));
+  return excl;
+}
+
+// Block-wide exclusive scan of one 32-bit value per thread (blockDim = NT).
+template <int NT>
+__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* s_warp, uint32_t& total) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_warp[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t w = lane < NW ? s_warp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      uint32_t y = __shfl_up_sync(0xFFFFFFFFu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < NW) s_warp[lane] = w;  // inclusive warp totals
+  }
+  __syncthreads();
+  total = s_warp[NW - 1];
+  uint32_t before = warp ? s_warp[warp - 1] : 0;
+  uint32_t r = before + x - v;
+  __syncthreads();
+  return r;
+}
+
+}  // namespace zipnn

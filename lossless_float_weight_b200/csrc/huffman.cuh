@@ -1,0 +1,188 @@
+// huffman.cuh -- per-chunk canonical Huffman code construction on the GPU.
+//
+// THEORY-599 note on ZipNN, "Order-0 only (section III-A b)": the exponent stream is
+// coded with a Huffman code built from its order-0 histogram. The pages leave the
+// construction's details open; this library fixes them so that the code is a
+// function of the histogram alone:
+//  * ties: the two nodes with the smallest (weight, order) keys merge first, a leaf's
+//    order being its symbol and the i-th merged node's order 256 + i (minimum-variance
+//    Huffman). Leaves sorted by (weight, symbol) and merged nodes in creation order
+//    form two queues whose heads give that minimum, a leaf winning a weight tie;
+//  * length limit 12: the code of the weights max(1, f >> k) for the smallest k >= 0
+//    whose longest code is at most 12 bits. The eight warps of a block try eight
+//    values of k at once;
+//  * canonical code values by the deflate rule (RFC 1951, section 3.2.2).
+#pragma once
+#include "common.cuh"
+
+namespace zipnn {
+
+constexpr int kHuffWarps = 8;
+
+struct HuffScratch {
+  uint64_t sorted[256];  // leaves (weight << 8 | symbol), ascending
+  uint64_t iw[256];      // unsorted leaf keys, then merged-node weights
+  uint16_t lpar[256];    // parent (merged-node index) of sorted leaf i
+  uint16_t ipar[256];    // parent of merged node i
+  uint8_t idep[256];     // depth of merged node i
+  uint8_t lens[256];     // result, by symbol
+};
+
+struct HuffBlockSmem {
+  uint64_t f[256];
+  HuffScratch w[kHuffWarps];
+  int maxlen[kHuffWarps];
+  uint64_t cost[kMaxGroups];
+  uint32_t elig[kMaxGroups];
+  uint64_t red[kHuffWarps];
+  int pick;
+  uint32_t bits_lo, bits_hi;
+};
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// One warp: lengths of the Huffman code for the weights max(1, f >> k) of the present
+// symbols of f[0..A). Returns the longest length (0 if no symbol is present).
+__device__ inline int warp_huffman(const uint64_t* f, int A, int k, HuffScratch& sc) {
+  const int lane = threadIdx.x & 31;
+  int n = 0;
+#pragma unroll
+  for (int i = 0; i < 8; i++) {
+    const int s = i * 32 + lane;
+    const uint64_t fs = s < A ? f[s] : 0;
+    const bool p = fs > 0;
+    const uint32_t b = __ballot_sync(0xFFFFFFFFu, p);
+    if (p) {
+      uint64_t g = k < 64 ? (fs >> k) : 0;
+      if (g == 0) g = 1;
+      sc.iw[n + __popc(b & lanemask_lt())] = (g << 8) | (uint64_t)s;
+    }
+    n += __popc(b);
+  }
+  for (int s = lane; s < 256; s += 32) sc.lens[s] = 0;
+  __syncwarp();
+  if (n == 0) return 0;
+  if (n == 1) {
+    if (lane == 0) sc.lens[sc.iw[0] & 0xFF] = 1;
+    __syncwarp();
+    return 1;
+  }
+  // rank sort of the distinct keys (weight, symbol)
+  for (int p = lane; p < n; p += 32) {
+    const uint64_t kp = sc.iw[p];
+    int r = 0;
+    for (int q = 0; q < n; q++) r += sc.iw[q] < kp;
+    sc.sorted[r] = kp;
+  }
+  __syncwarp();
+  if (lane == 0) {
+    // two-queue merge: node t (t = 0..n-2) joins the two smallest heads
+    int li = 0, ii = 0;
+    for (int t = 0; t < n - 1; t++) {
+      uint64_t sum = 0;
+#pragma unroll
+      for (int pick = 0; pick < 2; pick++) {
+        const bool leaf = li < n && (ii >= t || (sc.sorted[li] >> 8) <= sc.iw[ii]);
+        if (leaf) {
+          sum += sc.sorted[li] >> 8;
+          sc.lpar[li] = (uint16_t)t;
+          li++;
+        } else {
+          sum += sc.iw[ii];
+          sc.ipar[ii] = (uint16_t)t;
+          ii++;
+        }
+      }
+      sc.iw[t] = sum;
+    }
+    sc.idep[n - 2] = 0;
+    for (int t = n - 3; t >= 0; t--) sc.idep[t] = (uint8_t)(sc.idep[sc.ipar[t]] + 1);
+  }
+  __syncwarp();
+  int mx = 0;
+  for (int p = lane; p < n; p += 32) {
+    const int d = sc.idep[sc.lpar[p]] + 1;
+    sc.lens[sc.sorted[p] & 0xFF] = (uint8_t)(d > 255 ? 255 : d);
+    mx = d > mx ? d : mx;
+  }
+  __syncwarp();
+  return __reduce_max_sync(0xFFFFFFFFu, (uint32_t)mx);
+}
+
+// Whole block (kHuffWarps warps): length-limited lengths of sm.f[0..A). Returns the
+// index of the warp whose sm.w[].lens holds the result. Call with all threads.
+__device__ inline int block_limited_lengths(HuffBlockSmem& sm, int A) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int round = 0; round < 8; round++) {
+    const int k = round * kHuffWarps + warp;
+    const int mx = warp_huffman(sm.f, A, k, sm.w[warp]);
+    if (lane == 0) sm.maxlen[warp] = mx;
+    __syncthreads();
+    int found = -1;
+    for (int w = 0; w < kHuffWarps; w++)
+      if (sm.maxlen[w] <= kLmax) {
+        found = w;
+        break;
+      }
+    __syncthreads();
+    if (found >= 0) return found;
+  }
+  return 0;  // unreachable: at k = 63 every weight is 1 and lengths are <= 8
+}
+
+// One warp: canonical code values (RFC 1951, 3.2.2) for lens[0..256); writes
+// enc[s] = len << 16 | code (0 for absent symbols).
+__device__ inline void warp_canonical(const uint8_t* lens, uint32_t* enc) {
+  const int lane = threadIdx.x & 31;
+  uint32_t L[8];
+#pragma unroll
+  for (int i = 0; i < 8; i++) L[i] = lens[lane * 8 + i];
+  uint32_t excl[kLmax + 1], total[kLmax + 1];
+#pragma unroll
+  for (int l = 1; l <= kLmax; l++) {
+    uint32_t c = 0;
+#pragma unroll
+    for (int i = 0; i < 8; i++) c += L[i] == (uint32_t)l;
+    uint32_t x = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+      if (lane >= o) x += y;
+    }
+    excl[l] = x - c;
+    total[l] = __shfl_sync(0xFFFFFFFFu, x, 31);
+  }
+  uint32_t next[kLmax + 1];
+  uint32_t code = 0;
+  next[0] = 0;
+  total[0] = 0;
+#pragma unroll
+  for (int l = 1; l <= kLmax; l++) {
+    code = (code + total[l - 1]) << 1;
+    next[l] = code;
+  }
+#pragma unroll
+  for (int i = 0; i < 8; i++) {
+    uint32_t v = 0;
+    if (L[i]) {
+      uint32_t r = 0;
+#pragma unroll
+      for (int j = 0; j < i; j++) r += L[j] == L[i];
+      uint32_t base = 0, ex = 0;
+#pragma unroll
+      for (int l = 1; l <= kLmax; l++)
+        if ((uint32_t)l == L[i]) {
+          base = next[l];
+          ex = excl[l];
+        }
+      v = (L[i] << 16) | (base + ex + r);
+    }
+    enc[lane * 8 + i] = v;
+  }
+}
+
+}  // namespace zipnn

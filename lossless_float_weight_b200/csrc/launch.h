@@ -1,0 +1,36 @@
+// launch.h -- host-side launchers of the kernels (internal to libzipnn_b200).
+#pragma once
+#include <cuda_runtime.h>
+#include "common.cuh"
+
+namespace zipnn {
+
+cudaError_t launch_split_hist(const void* src, const Geo& g, uint32_t* hist, uint32_t* nonzero, cudaStream_t st);
+cudaError_t launch_build_tables(const Geo& g, const Ws& ws, const PlanDev& plan, cudaStream_t st);
+cudaError_t launch_code_lengths(const uint64_t* hist, uint32_t count, uint32_t alphabet_size, uint8_t* lens,
+                                uint32_t* enc, cudaStream_t st);
+cudaError_t launch_layout(const Geo& g, const Ws& ws, const PlanDev& plan, uint8_t* out, cudaStream_t st);
+uint32_t layout_tiles(uint32_t n_entries);
+cudaError_t launch_encode(const void* src, const Geo& g, const Ws& ws, uint8_t* out, cudaStream_t st);
+cudaError_t launch_decode(const uint8_t* in, uint64_t in_bytes, const Geo& g, uint8_t* out, uint32_t* status,
+                          cudaStream_t st);
+
+// plan (grouping) steps
+struct KmeansDev {
+  const uint32_t* hist;  // [C][n_entropy][256] (entropy stream 0 is the feature)
+  uint32_t C, A, NE, G;
+  uint64_t m0, n;
+  double* mu;            // [G][A]
+  uint32_t* assign;      // [C]
+  uint32_t* perm;        // [C]
+  uint32_t* changed;     // [1]
+  uint64_t* gsum;        // [NE][G][256]
+};
+cudaError_t launch_kmeans_init(const KmeansDev& k, uint64_t seed, cudaStream_t st);
+cudaError_t launch_kmeans_assign(const KmeansDev& k, cudaStream_t st);
+cudaError_t launch_kmeans_update(const KmeansDev& k, cudaStream_t st);
+cudaError_t launch_group_sums(const KmeansDev& k, cudaStream_t st);
+cudaError_t launch_canonical(const uint8_t* lens, uint32_t count, uint32_t* enc, cudaStream_t st);
+cudaError_t launch_identity_assign(uint32_t* assign, uint32_t C, cudaStream_t st);
+
+}  // namespace zipnn

@@ -1,0 +1,363 @@
+// prelude.cu -- the compress steps before encoding:
+//   k_split_hist   : byte-plane split + order-0 histogram per chunk (warp-aggregated
+//                    shared-memory atomics) + all-zero detection per chunk stream;
+//   k_build_tables : per (chunk, entropy stream) code choice: shared group code or a
+//                    local length-limited Huffman code, then HUFF / RAW / ZERO;
+//   k_layout       : exclusive scan of payload sizes (single-pass decoupled look-back)
+//                    into payload offsets; writes header, chunk table, shared records.
+#include "common.cuh"
+#include "fields.cuh"
+#include "huffman.cuh"
+#include "launch.h"
+
+namespace zipnn {
+
+constexpr int kHistThreads = 256;
+constexpr uint32_t kHistSlice = 16384;  // values of one chunk per histogram block
+
+// THEORY-599 note, "Order-0 only (section III-A b)": the model of a chunk is the count
+// of each symbol. Each warp keeps its own 256-bin table in shared memory; lanes holding
+// the same symbol are found with __match_any_sync and one of them adds their number.
+template <int DT>
+__global__ void __launch_bounds__(kHistThreads) k_split_hist(const uint8_t* __restrict__ src, Geo g, uint32_t slices,
+                                                             uint32_t* __restrict__ hist, uint32_t* __restrict__ nonzero) {
+  constexpr int NS = n_streams(DT), NE = n_entropy(DT), VB = value_bytes(DT), NW = kHistThreads / 32;
+  __shared__ uint32_t sh[NW][NE][256];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < NW * NE * 256; i += kHistThreads) (&sh[0][0][0])[i] = 0;
+  __syncthreads();
+  const uint32_t c = blockIdx.x / slices, sl = blockIdx.x % slices;
+  const uint64_t clo = (uint64_t)c * g.m0;
+  const uint32_t m = (uint32_t)min64(g.m0, g.n - clo);
+  const uint32_t lo = sl * kHistSlice, hi = min(lo + kHistSlice, m);
+  uint32_t nz[NS];
+#pragma unroll
+  for (int s = 0; s < NS; s++) nz[s] = 0;
+  for (uint32_t base = lo + warp * 32 * kGroupValues; base < hi; base += NW * 32 * kGroupValues) {
+    const uint32_t v0 = base + lane * kGroupValues;
+    const int cnt = v0 < hi ? (int)min32(kGroupValues, hi - v0) : 0;
+    uint32_t sym[NS][16];
+    load_split16<DT>(src + (clo + v0) * VB, cnt, sym);
+#pragma unroll
+    for (int i = 0; i < 16; i++) {
+      const bool valid = i < cnt;
+#pragma unroll
+      for (int e = 0; e < NE; e++) {
+        const uint32_t key = valid ? sym[e][i] : 0x100u;
+        const uint32_t peers = __match_any_sync(0xFFFFFFFFu, key);
+        if (valid && lane == __ffs(peers) - 1) atomicAdd(&sh[warp][e][key], (uint32_t)__popc(peers));
+      }
+#pragma unroll
+      for (int s = 0; s < NS; s++) nz[s] |= sym[s][i];
+    }
+  }
+#pragma unroll
+  for (int s = 0; s < NS; s++) {
+    const uint32_t v = __reduce_or_sync(0xFFFFFFFFu, nz[s]);
+    if (nonzero && lane == 0 && v) atomicOr(&nonzero[(uint64_t)c * NS + s], v);
+  }
+  __syncthreads();
+#pragma unroll
+  for (int e = 0; e < NE; e++) {
+    uint32_t sum = 0;
+#pragma unroll
+    for (int w = 0; w < NW; w++) sum += sh[w][e][tid];
+    if (sum) atomicAdd(&hist[((uint64_t)c * NE + e) * 256 + tid], sum);
+  }
+}
+
+// Per (chunk, entropy stream), one block of kHuffWarps warps.
+// With a plan ("NeuralZip: Reusable Setup for Fast Lossless Compression", abstract):
+// a group is eligible when its code has a length for every symbol the chunk uses; the
+// eligible group with the fewest coded bits wins (ties to the smaller group). Without
+// an eligible group, or without a plan, the chunk gets its own limited Huffman code.
+// The entry is HUFF when that payload is strictly smaller than RAW, ZERO when every
+// symbol is 0.
+template <int DT>
+__global__ void __launch_bounds__(kHuffWarps * 32) k_build_tables(Geo g, Ws ws, PlanDev plan) {
+  constexpr int NS = n_streams(DT), NE = n_entropy(DT);
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  HuffBlockSmem& sm = *reinterpret_cast<HuffBlockSmem*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t c = blockIdx.x / NE, e = blockIdx.x % NE;
+  const uint32_t k = c * NS + e;
+  const uint64_t clo = (uint64_t)c * g.m0;
+  const uint64_t m = min64(g.m0, g.n - clo);
+  const int A = alphabet(DT, e), w = raw_width(DT, e);
+  if (ws.nonzero[k] == 0) {
+    if (tid == 0) {
+      ws.emode[k] = kModeZero;
+      ws.ecode[k] = kNoCode;
+      ws.esize[k] = 0;
+    }
+    return;
+  }
+  const uint32_t* h = ws.hist + ((uint64_t)c * NE + e) * 256;
+  sm.f[tid] = tid < A ? h[tid] : 0;
+  __syncthreads();
+  int group = -1;
+  uint64_t bits = 0;
+  if (plan.groups) {
+    for (uint32_t gi = warp; gi < plan.groups; gi += kHuffWarps) {
+      const uint8_t* lg = plan.lens + ((uint64_t)e * plan.groups + gi) * 256;
+      uint64_t cost = 0;
+      bool ok = true;
+      for (int s = lane; s < A; s += 32) {
+        const uint64_t f = sm.f[s];
+        if (f) {
+          ok = ok && lg[s] != 0;
+          cost += f * lg[s];
+        }
+      }
+      for (int o = 16; o; o >>= 1) cost += __shfl_xor_sync(0xFFFFFFFFu, cost, o);
+      const bool all = __all_sync(0xFFFFFFFFu, ok);
+      if (lane == 0) {
+        sm.cost[gi] = cost;
+        sm.elig[gi] = all;
+      }
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int best = -1;
+      for (uint32_t gi = 0; gi < plan.groups; gi++)
+        if (sm.elig[gi] && (best < 0 || sm.cost[gi] < sm.cost[best])) best = (int)gi;
+      sm.pick = best;
+    }
+    __syncthreads();
+    group = sm.pick;
+    if (group >= 0) bits = sm.cost[group];
+  }
+  const uint8_t* lens = nullptr;
+  if (group < 0) {
+    const int wbest = block_limited_lengths(sm, A);
+    lens = sm.w[wbest].lens;
+    uint64_t part = tid < A ? sm.f[tid] * lens[tid] : 0;
+    for (int o = 16; o; o >>= 1) part += __shfl_xor_sync(0xFFFFFFFFu, part, o);
+    if (lane == 0) sm.red[warp] = part;
+    __syncthreads();
+    bits = 0;
+    for (int i = 0; i < kHuffWarps; i++) bits += sm.red[i];
+  }
+  const uint64_t nsub = ceil_div(m, g.S);
+  const uint64_t p_huff = (group < 0 ? record_bytes(DT, e) : 0) + round16(4 * nsub) + round16(ceil_div(bits, 8));
+  const uint64_t p_raw = raw_payload(m, w);
+  uint32_t* enc = ws.enc + ((uint64_t)c * NE + e) * 256;
+  if (p_huff < p_raw) {
+    if (group >= 0) {
+      enc[tid] = plan.enc[((uint64_t)e * plan.groups + group) * 256 + tid];
+    } else if (warp == 0) {
+      warp_canonical(lens, enc);
+    }
+    if (tid == 0) {
+      ws.emode[k] = kModeHuff;
+      ws.ecode[k] = group >= 0 ? e * plan.groups + (uint32_t)group : kNoCode;
+      ws.esize[k] = p_huff;
+    }
+  } else if (tid == 0) {
+    ws.emode[k] = kModeRaw;
+    ws.ecode[k] = kNoCode;
+    ws.esize[k] = p_raw;
+  }
+}
+
+// Stand-alone code lengths for `count` histograms (u64 x 256 each); also used by the
+// plan for its group codes. Optionally writes canonical code values.
+__global__ void __launch_bounds__(kHuffWarps * 32) k_code_lengths(const uint64_t* __restrict__ hist, uint32_t alphabet_size,
+                                                                 uint8_t* __restrict__ lens_out, uint32_t* __restrict__ enc_out) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  HuffBlockSmem& sm = *reinterpret_cast<HuffBlockSmem*>(smem_raw);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const uint64_t* h = hist + (uint64_t)blockIdx.x * 256;
+  sm.f[tid] = tid < (int)alphabet_size ? h[tid] : 0;
+  __syncthreads();
+  const int wbest = block_limited_lengths(sm, (int)alphabet_size);
+  const uint8_t* lens = sm.w[wbest].lens;
+  lens_out[(uint64_t)blockIdx.x * 256 + tid] = lens[tid];
+  if (enc_out && warp == 0) warp_canonical(lens, enc_out + (uint64_t)blockIdx.x * 256);
+}
+
+constexpr int kLayoutThreads = 256, kLayoutPer = 4, kLayoutTile = kLayoutThreads * kLayoutPer;
+
+// Block-wide exclusive scan of 64-bit values (blockDim = kLayoutThreads).
+__device__ inline uint64_t block_scan_u64(uint64_t v, uint64_t* s_warp, uint64_t& total) {
+  constexpr int NW = kLayoutThreads / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint64_t x = v;
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint64_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_warp[warp] = x;
+  __syncthreads();
+  uint64_t before = 0;
+  for (int i = 0; i < warp; i++) before += s_warp[i];
+  total = 0;
+  for (int i = 0; i < NW; i++) total += s_warp[i];
+  __syncthreads();
+  return before + x - v;
+}
+
+// Layout: payload k (entry order) starts at off_payload + sum of sizes of entries < k.
+// Entropy entries take their mode and size from k_build_tables; raw-plane entries are
+// ZERO when all their symbols are 0, else RAW.
+template <int DT>
+__global__ void __launch_bounds__(kLayoutThreads) k_layout(Geo g, Ws ws, PlanDev plan, uint8_t* __restrict__ out) {
+  constexpr int NS = n_streams(DT), NE = n_entropy(DT);
+  __shared__ uint64_t s_warp[kLayoutThreads / 32];
+  __shared__ uint32_t s_tile;
+  __shared__ uint64_t s_prefix;
+  const int tid = threadIdx.x;
+  if (tid == 0) s_tile = atomicAdd(&ws.status[2], 1u);
+  __syncthreads();
+  const uint32_t tile = s_tile;
+  const uint32_t k0 = tile * kLayoutTile + tid * kLayoutPer;
+  uint64_t size[kLayoutPer];
+  uint32_t mode[kLayoutPer], code[kLayoutPer];
+  uint64_t mine = 0;
+#pragma unroll
+  for (int i = 0; i < kLayoutPer; i++) {
+    const uint32_t k = k0 + i;
+    size[i] = 0;
+    mode[i] = kModeZero;
+    code[i] = kNoCode;
+    if (k < g.n_entries) {
+      const uint32_t s = k % NS;
+      if (is_entropy(DT, (int)s)) {
+        mode[i] = ws.emode[k];
+        code[i] = ws.ecode[k];
+        size[i] = ws.esize[k];
+      } else {
+        const uint32_t c = k / NS;
+        const uint64_t m = min64(g.m0, g.n - (uint64_t)c * g.m0);
+        if (ws.nonzero[k]) {
+          mode[i] = kModeRaw;
+          size[i] = raw_payload(m, raw_width(DT, (int)s));
+        }
+        ws.emode[k] = mode[i];
+        ws.ecode[k] = kNoCode;
+        ws.esize[k] = size[i];
+      }
+      mine += size[i];
+    }
+  }
+  uint64_t total;
+  uint64_t before = block_scan_u64(mine, s_warp, total);
+  if (tid == 0) s_prefix = lookback(ws.scan_desc, tile, 0, total, ws.status);
+  __syncthreads();
+  uint64_t pos = g.off_payload + s_prefix + before;
+#pragma unroll
+  for (int i = 0; i < kLayoutPer; i++) {
+    const uint32_t k = k0 + i;
+    if (k < g.n_entries) {
+      ws.eoff[k] = pos;
+      uint4 ent;
+      ent.x = mode[i];
+      ent.y = code[i];
+      ent.z = (uint32_t)pos;
+      ent.w = (uint32_t)(pos >> 32);
+      *reinterpret_cast<uint4*>(out + kHeaderBytes + (uint64_t)kEntryBytes * k) = ent;
+      pos += size[i];
+    }
+  }
+  const uint32_t n_layout_tiles = (uint32_t)ceil_div(g.n_entries, kLayoutTile);
+  if (tile == n_layout_tiles - 1 && tid == 0) {
+    uint32_t hdr[16];
+    hdr[0] = 0x314E4E5Au;  // "ZNN1"
+    hdr[1] = 1u | ((uint32_t)DT << 16) | ((uint32_t)NS << 24);
+    hdr[2] = (uint32_t)g.n;
+    hdr[3] = (uint32_t)(g.n >> 32);
+    hdr[4] = g.chunk_bytes;
+    hdr[5] = g.S;
+    hdr[6] = g.n_chunks;
+    hdr[7] = g.n_groups * NE;
+    hdr[8] = (uint32_t)g.off_codes;
+    hdr[9] = (uint32_t)(g.off_codes >> 32);
+    hdr[10] = (uint32_t)g.off_payload;
+    hdr[11] = (uint32_t)(g.off_payload >> 32);
+    const uint64_t tb = g.off_payload + s_prefix + total;
+    hdr[12] = (uint32_t)tb;
+    hdr[13] = (uint32_t)(tb >> 32);
+    hdr[14] = (uint32_t)kLmax | (g.n_groups << 8);
+    hdr[15] = 0;
+    for (int i = 0; i < 4; i++)
+      reinterpret_cast<uint4*>(out)[i] = make_uint4(hdr[4 * i], hdr[4 * i + 1], hdr[4 * i + 2], hdr[4 * i + 3]);
+  }
+  // shared code records (4-bit lengths), written by the first tile
+  if (tile == 0 && plan.groups) {
+    for (int e = 0; e < NE; e++) {
+      const int A = alphabet(DT, e);
+      const uint32_t rb = record_bytes(DT, e);
+      for (uint32_t gi = 0; gi < plan.groups; gi++) {
+        const uint8_t* lg = plan.lens + ((uint64_t)e * plan.groups + gi) * 256;
+        uint8_t* rp = out + g.off_codes + shared_record_pos(DT, plan.groups, (uint32_t)e * plan.groups + gi);
+        for (uint32_t b = tid; b < rb; b += kLayoutThreads)
+          rp[b] = (int)(2 * b) < A ? (uint8_t)(lg[2 * b] | (lg[2 * b + 1] << 4)) : 0;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- launchers
+
+template <int DT>
+static cudaError_t split_hist_t(const void* src, const Geo& g, uint32_t* hist, uint32_t* nonzero, cudaStream_t st) {
+  const uint32_t slices = (uint32_t)ceil_div(g.m0, kHistSlice);
+  const uint64_t blocks = (uint64_t)g.n_chunks * slices;
+  if (blocks > 0x7FFFFFFFull) return cudaErrorInvalidConfiguration;
+  k_split_hist<DT><<<(uint32_t)blocks, kHistThreads, 0, st>>>(static_cast<const uint8_t*>(src), g, slices, hist, nonzero);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_split_hist(const void* src, const Geo& g, uint32_t* hist, uint32_t* nonzero, cudaStream_t st) {
+  switch (g.dt) {
+    case kBF16: return split_hist_t<kBF16>(src, g, hist, nonzero, st);
+    case kFP32: return split_hist_t<kFP32>(src, g, hist, nonzero, st);
+    default: return split_hist_t<kFP8>(src, g, hist, nonzero, st);
+  }
+}
+
+template <int DT>
+static cudaError_t tables_t(const Geo& g, const Ws& ws, const PlanDev& plan, cudaStream_t st) {
+  const size_t smem = sizeof(HuffBlockSmem);
+  cudaError_t e = cudaFuncSetAttribute(k_build_tables<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k_build_tables<DT><<<g.n_chunks * n_entropy(DT), kHuffWarps * 32, smem, st>>>(g, ws, plan);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_build_tables(const Geo& g, const Ws& ws, const PlanDev& plan, cudaStream_t st) {
+  switch (g.dt) {
+    case kBF16: return tables_t<kBF16>(g, ws, plan, st);
+    case kFP32: return tables_t<kFP32>(g, ws, plan, st);
+    default: return tables_t<kFP8>(g, ws, plan, st);
+  }
+}
+
+cudaError_t launch_code_lengths(const uint64_t* hist, uint32_t count, uint32_t alphabet_size, uint8_t* lens,
+                                uint32_t* enc, cudaStream_t st) {
+  const size_t smem = sizeof(HuffBlockSmem);
+  cudaError_t e = cudaFuncSetAttribute(k_code_lengths, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  if (count == 0) return cudaSuccess;
+  k_code_lengths<<<count, kHuffWarps * 32, smem, st>>>(hist, alphabet_size, lens, enc);
+  return cudaGetLastError();
+}
+
+template <int DT>
+static cudaError_t layout_t(const Geo& g, const Ws& ws, const PlanDev& plan, uint8_t* out, cudaStream_t st) {
+  const uint32_t tiles = (uint32_t)ceil_div(g.n_entries, kLayoutTile);
+  k_layout<DT><<<tiles, kLayoutThreads, 0, st>>>(g, ws, plan, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_layout(const Geo& g, const Ws& ws, const PlanDev& plan, uint8_t* out, cudaStream_t st) {
+  switch (g.dt) {
+    case kBF16: return layout_t<kBF16>(g, ws, plan, out, st);
+    case kFP32: return layout_t<kFP32>(g, ws, plan, out, st);
+    default: return layout_t<kFP8>(g, ws, plan, out, st);
+  }
+}
+
+uint32_t layout_tiles(uint32_t n_entries) { return (uint32_t)ceil_div(n_entries, kLayoutTile); }
+
+}  // namespace zipnn

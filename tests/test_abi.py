@@ -1,0 +1,57 @@
+"""The C-ABI library loads and exports every entry point include/zipnn.h declares, and
+its host-only calls (sizes, argument checks) behave; no kernel is launched (CPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "zipnn.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(zipnn_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from lossless_float_weight_b200 import build
+    build.build()
+    return ctypes.CDLL(build.LIB)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 15
+    for name in names:
+        assert hasattr(lib, name), name
+
+
+def test_binding_covers_the_abi(lib):
+    from lossless_float_weight_b200 import zipnn
+    assert sorted(zipnn.C_ABI_NAMES) == _declared()
+
+
+def test_sizes_match_the_oracle(lib, orc):
+    from lossless_float_weight_b200 import zipnn as Z
+    for dt, name in ((Z.BF16, "bf16"), (Z.FP32, "fp32"), (Z.FP8_E4M3, "fp8_e4m3")):
+        for n in (1, 17, 131072, 6607077376 // 225, 10 ** 7 + 3):
+            for cb in (4096, 262144):
+                assert Z.zipnn_max_compressed_bytes(dt, n, cb) == orc.max_compressed_bytes(name, n, cb, 64)
+                assert Z.zipnn_workspace_bytes(dt, n, cb) > 0
+    assert Z.zipnn_max_compressed_bytes(Z.BF16, 0, 262144) == 0
+    assert Z.zipnn_max_compressed_bytes(Z.BF16, 10, 100) == 0      # not a multiple of 16
+    assert Z.zipnn_max_compressed_bytes(7, 10, 262144) == 0        # bad dtype
+
+
+def test_argument_errors_without_a_device(lib):
+    from lossless_float_weight_b200 import zipnn as Z
+    # null pointers and bad sizes are rejected before anything touches the device
+    assert Z.zipnn_compress(Z.BF16, None, 10, 262144, None, None, 0, None, 0, None) == Z.ERR_INVALID_ARG
+    assert Z.zipnn_decompress(Z.BF16, None, 0, 10, 262144, None, None, 0, None) == Z.ERR_INVALID_ARG
+    assert Z.zipnn_code_lengths(None, 1, 256, None, None) == Z.ERR_INVALID_ARG
+    assert Z.zipnn_plan_import(None, 0, None) == Z.ERR_INVALID_ARG
+    assert Z.zipnn_status_string(Z.ERR_CORRUPT).startswith(b"corrupt")

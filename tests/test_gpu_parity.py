@@ -1,0 +1,264 @@
+"""Parity of the CUDA path with the CPU oracle (B200 only).
+
+Every compressed container must equal the oracle's byte for byte, and every
+decompressed tensor must equal the input byte for byte (integer work: bit-exact is the
+only bar). Inputs come from lossless_float_weight_b200.workloads, seeded; the oracle
+sees the same bytes copied to the host.
+"""
+import numpy as np
+import pytest
+import torch
+
+import container_util as CU
+import golden_util as GU
+
+pytestmark = pytest.mark.gpu
+
+S_DEFAULT = 1024
+CB = 262144
+
+
+@pytest.fixture(scope="module")
+def z():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from lossless_float_weight_b200 import zipnn
+    return zipnn
+
+
+def _host_bytes(t):
+    return t.detach().contiguous().cpu().reshape(-1).view(torch.uint8).numpy()
+
+
+def _check_roundtrip(z, orc, x, name, chunk_bytes=CB, subblock=S_DEFAULT, plan=None, plan_lens=None):
+    dtype = {torch.bfloat16: "bf16", torch.float32: "fp32", torch.float8_e4m3fn: "fp8_e4m3"}[x.dtype]
+    xd = x.reshape(-1).cuda()
+    cont = z.compress(xd, chunk_bytes=chunk_bytes, plan=plan, subblock=subblock)
+    got = cont.cpu().numpy()
+    ref = orc.compress(dtype, _host_bytes(x), x.numel(), chunk_bytes=chunk_bytes, S=subblock, plan_lens=plan_lens,
+                       threads=8)
+    assert got.size == ref.size, f"{name}: size {got.size} != oracle {ref.size}"
+    bad = np.nonzero(got != ref)[0]
+    assert bad.size == 0, f"{name}: {bad.size} bytes differ, first at {bad[:5]}"
+    y = z.decompress(cont, x.dtype, x.numel(), chunk_bytes=chunk_bytes)
+    assert torch.equal(y.view(torch.uint8).cpu(), x.reshape(-1).contiguous().view(torch.uint8).cpu()), name
+    # and the GPU decodes the oracle's container
+    y2 = z.decompress(torch.from_numpy(ref).cuda(), x.dtype, x.numel(), chunk_bytes=chunk_bytes)
+    assert torch.equal(y2.view(torch.uint8).cpu(), x.reshape(-1).contiguous().view(torch.uint8).cpu()), name
+    return got
+
+
+def test_bf16_small_config(z, orc):
+    from lossless_float_weight_b200 import workloads as W
+    x = W.bf16_small()
+    c = _check_roundtrip(z, orc, x, "bf16 1M")
+    assert 0.64 <= c.size / (2 * x.numel()) <= 0.68
+
+
+def test_golden_containers(z, orc):
+    x = GU.three_chunk_input().cuda()
+    fx = GU.load("bf16_three_chunks.json")
+    got = z.compress(x, chunk_bytes=512, subblock=64).cpu().numpy()
+    assert np.array_equal(got, GU.expected_bytes(fx))
+    y = z.decompress(torch.from_numpy(GU.expected_bytes(fx).copy()).cuda(), torch.bfloat16, 517, chunk_bytes=512)
+    assert torch.equal(y.cpu(), x.cpu())
+
+
+@pytest.mark.parametrize("n", [1, 7, 8, 15, 16, 17, 1023, 4095, 4096, 4097, 131071, 131072, 131073, 400000])
+def test_bf16_ragged_sizes(z, orc, n):
+    x = (torch.randn(n, generator=torch.Generator().manual_seed(n)) * 0.02).to(torch.bfloat16)
+    _check_roundtrip(z, orc, x, f"bf16 n={n}")
+
+
+@pytest.mark.parametrize("chunk_bytes,subblock", [(16, 16), (4096, 64), (65536, 256), (262144, 1024),
+                                                  (1 << 20, 2048), (262144, 65536)])
+def test_bf16_chunk_and_subblock_shapes(z, orc, chunk_bytes, subblock):
+    x = (torch.randn(300001, generator=torch.Generator().manual_seed(1)) * 0.05).to(torch.bfloat16)
+    _check_roundtrip(z, orc, x, f"cb={chunk_bytes} S={subblock}", chunk_bytes=chunk_bytes, subblock=subblock)
+
+
+def test_every_bf16_and_fp8_pattern(z, orc):
+    rng = np.random.default_rng(0)
+    pats = torch.from_numpy(rng.permutation(np.arange(65536, dtype=np.int64)).astype(np.int16))
+    _check_roundtrip(z, orc, pats.view(torch.bfloat16), "bf16 patterns", chunk_bytes=4096, subblock=64)
+    _check_roundtrip(z, orc, torch.arange(65536, dtype=torch.int32).to(torch.int16).view(torch.bfloat16),
+                     "bf16 ordered patterns", chunk_bytes=4096)
+    f8 = torch.from_numpy(np.tile(np.arange(256, dtype=np.uint8), 500)).view(torch.float8_e4m3fn)
+    _check_roundtrip(z, orc, f8, "fp8 patterns", chunk_bytes=4096, subblock=128)
+
+
+def test_constant_and_zero_tensors(z, orc):
+    for x in (torch.zeros(300000, dtype=torch.bfloat16), torch.ones(300000, dtype=torch.bfloat16),
+              torch.full((70000,), -2.5, dtype=torch.float32), torch.zeros(70000, dtype=torch.float32),
+              torch.zeros(90000, dtype=torch.uint8).view(torch.float8_e4m3fn)):
+        _check_roundtrip(z, orc, x, f"constant {x.dtype}")
+
+
+def test_fp32_and_clean(z, orc):
+    from lossless_float_weight_b200 import workloads as W
+    x = W.fp32_tensor(n=(1 << 21) + 333)
+    c = _check_roundtrip(z, orc, x, "fp32")
+    assert 0.82 <= c.size / (4 * x.numel()) <= 0.85
+    xc = x.to(torch.bfloat16).to(torch.float32)
+    c = _check_roundtrip(z, orc, xc, "fp32 clean")
+    assert c.size / (4 * x.numel()) < 0.35
+
+
+def test_fp32_special_values(z, orc):
+    rng = np.random.default_rng(2)
+    bits = rng.integers(0, 2 ** 32, size=100000, dtype=np.uint64).astype(np.uint32)
+    specials = np.array([0.0, -0.0, np.inf, -np.inf, np.nan, 1e-45, -1e-45, 3.4028235e38], dtype=np.float32)
+    x = np.concatenate([specials.view(np.uint32), bits]).view(np.int32)
+    _check_roundtrip(z, orc, torch.from_numpy(x).view(torch.float32), "fp32 bits", chunk_bytes=4096)
+
+
+def test_fp8(z, orc):
+    from lossless_float_weight_b200 import workloads as W
+    q = W.fp8_tensor(rows=600, cols=4096)
+    q = torch.cat([q, q[:777]])
+    c = _check_roundtrip(z, orc, q, "fp8")
+    assert c.size / q.numel() < 0.9
+
+
+def test_histogram_entry_point(z, orc):
+    from lossless_float_weight_b200 import workloads as W
+    for x, dt, cb in ((W.bf16_small(n=500001), "bf16", CB), (W.fp8_tensor(rows=70, cols=4096), "fp8_e4m3", 65536),
+                      (W.fp32_tensor(n=100003), "fp32", 65536)):
+        h = z.histogram(x.cuda(), chunk_bytes=cb).cpu().numpy()
+        vb = {"bf16": 2, "fp32": 4, "fp8_e4m3": 1}[dt]
+        m0 = cb // vb
+        hb = _host_bytes(x)
+        n = x.numel()
+        for c in range(h.shape[0]):
+            for e in range(h.shape[1]):
+                ref = orc.histogram(dt, hb, c * m0, min(n, (c + 1) * m0), e)
+                assert np.array_equal(h[c, e].astype(np.uint64), ref), (dt, c, e)
+
+
+def test_code_lengths_entry_point(z, orc):
+    rng = np.random.default_rng(3)
+    hists = []
+    for t in range(200):
+        a = int(rng.integers(2, 257))
+        kind = t % 5
+        f = np.zeros(256, dtype=np.int64)
+        if kind == 0:
+            f[:a] = rng.integers(0, 50, size=a)
+        elif kind == 1:
+            f[:a] = (1e9 * rng.random(a) ** 12).astype(np.int64)
+        elif kind == 2:  # Fibonacci weights: the deepest possible trees
+            a = min(a, 60)
+            fib = [1, 1]
+            while len(fib) < a:
+                fib.append(fib[-1] + fib[-2])
+            f[:a] = np.array(fib[:a], dtype=np.int64)[rng.permutation(a)]
+        elif kind == 3:  # many ties
+            f[:a] = rng.integers(1, 4, size=a)
+        else:
+            f[:a] = rng.integers(0, 2 ** 40, size=a)
+        hists.append(f)
+    H = torch.from_numpy(np.stack(hists)).cuda()
+    got = z.code_lengths(H).cpu().numpy()
+    for i, f in enumerate(hists):
+        assert np.array_equal(got[i], orc.limited_lengths(f.astype(np.uint64))), i
+
+
+def test_plan_parity(z, orc):
+    from lossless_float_weight_b200 import workloads as W
+    kv = W.kv_cache(shape=(2, 2, 4, 4, 4096, 128))  # 128 chunks
+    plan = z.Plan.create(kv.cuda(), groups=8, seed=0)
+    lens, assign, iters, _ = orc.plan_build("bf16", _host_bytes(kv), kv.numel(), CB, groups=8, seed=0)
+    assert plan.assignment() == assign.tolist()
+    exported = plan.export()
+    # export = "ZNP1", dtype, groups, 2 zero bytes, 4-bit length records
+    assert exported[:4] == b"ZNP1" and exported[4] == 0 and exported[5] == 8
+    rec = np.frombuffer(exported[8:], dtype=np.uint8).reshape(8, 128)
+    got_lens = np.zeros((8, 256), dtype=np.uint8)
+    got_lens[:, 0::2] = rec & 15
+    got_lens[:, 1::2] = rec >> 4
+    assert np.array_equal(got_lens, lens[0])
+    _check_roundtrip(z, orc, kv, "kv with plan", plan=plan, plan_lens=lens)
+    # the plan applies to another tensor (reuse), and survives export/import
+    other = W.kv_cache(shape=(1, 2, 4, 4, 4096, 128), seed=5)
+    p2 = z.Plan.from_bytes(exported)
+    _check_roundtrip(z, orc, other, "kv reuse", plan=p2, plan_lens=lens)
+
+
+def test_plan_fp8_and_small(z, orc):
+    from lossless_float_weight_b200 import workloads as W
+    q = W.fp8_tensor(rows=512, cols=4096)
+    plan = z.Plan.create(q.cuda(), groups=4, seed=3, chunk_bytes=65536)
+    lens, assign, _, _ = orc.plan_build("fp8_e4m3", _host_bytes(q), q.numel(), 65536, groups=4, seed=3)
+    assert plan.assignment() == assign.tolist()
+    _check_roundtrip(z, orc, q, "fp8 plan", chunk_bytes=65536, plan=plan, plan_lens=lens)
+    x = W.bf16_small(n=300000)  # 3 chunks <= 8 groups: identity grouping
+    plan = z.Plan.create(x.cuda(), groups=8)
+    lens, assign, _, _ = orc.plan_build("bf16", _host_bytes(x), x.numel(), CB, groups=8, seed=0)
+    assert plan.assignment() == [0, 1, 2]
+    _check_roundtrip(z, orc, x, "bf16 identity plan", plan=plan, plan_lens=lens)
+
+
+def test_plan_dtype_mismatch(z):
+    from lossless_float_weight_b200 import workloads as W
+    x = W.bf16_small(n=300000).cuda()
+    plan = z.Plan.create(x, groups=2)
+    f = torch.zeros(1000, dtype=torch.float32, device="cuda")
+    with pytest.raises(z.ZipnnError) as ei:
+        z.compress(f, plan=plan)
+    assert ei.value.status == z.ERR_PLAN_MISMATCH
+
+
+def test_corrupt_containers_report_status(z, orc):
+    import struct
+    from lossless_float_weight_b200 import workloads as W
+    x = W.bf16_small(n=300000)
+    c = z.compress(x.cuda()).cpu().numpy()
+    off0 = struct.unpack_from("<Q", c, 64 + 8)[0]
+    cases = []
+    d = c.copy(); d[0] ^= 1; cases.append(d)
+    cases.append(c[: c.size - 16].copy())
+    d = c.copy(); struct.pack_into("<Q", d, 48, c.size + 16); cases.append(d)
+    d = c.copy(); struct.pack_into("<Q", d, 64 + 16 + 8, 10 ** 9); cases.append(d)
+    d = c.copy(); d[64] = 7; cases.append(d)
+    d = c.copy(); d[off0 + 63] = 0xFF; cases.append(d)
+    d = c.copy(); d[off0: off0 + 128] = 0x11; cases.append(d)
+    d = c.copy(); struct.pack_into("<I", d, off0 + 128, 5); cases.append(d)
+    d = c.copy(); struct.pack_into("<I", d, off0 + 128 + 4, 0x7FFFFFFF); cases.append(d)
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    out = torch.empty(300000, dtype=torch.bfloat16, device="cuda")
+    for i, d in enumerate(cases):
+        dd = torch.from_numpy(d).cuda()
+        z.decompress_into(dd, dd.numel(), out, ws)
+        assert z.status(ws) == z.ERR_CORRUPT, i
+        assert orc.decompress_status("bf16", d, 300000) == orc.ECORRUPT, i
+    # wrong n / dtype for a valid container
+    cd = torch.from_numpy(c).cuda()
+    z.decompress_into(cd, cd.numel(), out[:299999], ws)
+    assert z.status(ws) == z.ERR_CORRUPT
+    # random bit flips: either detected or decoded, never a fault
+    rng = np.random.default_rng(4)
+    for _ in range(30):
+        d = c.copy()
+        d[int(rng.integers(64, c.size))] ^= 1 << int(rng.integers(0, 8))
+        dd = torch.from_numpy(d).cuda()
+        z.decompress_into(dd, dd.numel(), out, ws)
+        assert z.status(ws) in (z.OK, z.ERR_CORRUPT)
+    torch.cuda.synchronize()
+
+
+def test_argument_errors(z):
+    x = torch.zeros(1000, dtype=torch.bfloat16, device="cuda")
+    ws = z.workspace(z.BF16, 1000)
+    out = torch.empty(100000, dtype=torch.uint8, device="cuda")
+    with pytest.raises(z.ZipnnError) as ei:
+        z.compress_into(x, out[:10], ws)
+    assert ei.value.status == z.ERR_OUT_TOO_SMALL
+    with pytest.raises(z.ZipnnError) as ei:
+        z.compress_into(x, out, ws, chunk_bytes=100)
+    assert ei.value.status == z.ERR_INVALID_ARG
+    with pytest.raises(z.ZipnnError) as ei:
+        z.compress_into(x[1:], out, ws)  # 2-byte aligned pointer
+    assert ei.value.status == z.ERR_INVALID_ARG
+    with pytest.raises(z.ZipnnError) as ei:
+        z.compress_into(x, out, ws, subblock=24)
+    assert ei.value.status == z.ERR_INVALID_ARG
