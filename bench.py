@@ -1,0 +1,418 @@
+"""Benchmark: ZipNN-style compress + decompress of a 7B-shaped BF16 checkpoint on B200.
+
+One step = zipnn_compress of each of the 225 tensors of the checkpoint (6,607,077,376
+BF16 values, 13.21 GB), back to back on one stream, then zipnn_decompress of each.
+The metric is GB/s of uncompressed bytes; `value` is the round-trip rate (uncompressed
+bytes / (compress time + decompress time)) summed over all ranks, and the JSON line
+also carries each direction and its fraction of the measured HBM copy bandwidth.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun (N > 1) every rank compresses its own checkpoint (weak scaling, no
+collective on the data path); time is the max over ranks.
+"""
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch
+
+METRIC = "decompress/compress GB/s (uncompressed) at 1 B200; % of HBM roofline"
+WORKLOAD = ("BF16 7B-shaped checkpoint: 32 x [q,k,v,o 4096x4096; gate,up,down 4096x11008] + embedding "
+            "32000x4096, 225 tensors, 6,607,077,376 values (13.21 GB), sigma_t log-uniform [0.005, 0.05], "
+            "256 KiB chunks, one zipnn call per tensor on one stream")
+CHUNK = 262144
+SUBBLOCK = 512  # the library default (include/zipnn.h)
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ------------------------------------------------------------------ distributed helpers
+
+def dist_env():
+    """(rank, world, local_rank) from the torchrun environment; (0, 1, 0) without it."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_dist(world, backend):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(value, world, device):
+    """Max of a float over all ranks (identity for one rank)."""
+    if world == 1:
+        return float(value)
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def rank_seed(rank):
+    """Each rank compresses its own checkpoint: the generator seeds shift by rank."""
+    return 1000003 * rank
+
+
+# ------------------------------------------------------------------ measurement helpers
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples every 200 ms while running."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                mhz.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        mhz.sort()
+        return {"sm_mhz": mhz[len(mhz) // 2] if mhz else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+# ------------------------------------------------------------------ our arm
+
+def make_workload(device, rank, tensors=None, only=None):
+    from lossless_float_weight_b200 import workloads as W
+    shapes = W.checkpoint_7b_shapes()
+    sig = W.checkpoint_7b_sigmas(len(shapes))
+    pick = [only] if only is not None else list(range(len(shapes)))[:tensors]
+    return [W.checkpoint_7b_tensor(t + rank_seed(rank), shapes[t][1], sig[t], device).reshape(-1) for t in pick]
+
+
+def cpu_baseline(xs, budget_s=15.0):
+    """The oracle as it stands, on this host's cores, over a bounded sample of the
+    workload's tensors (chunk-parallel threads); same round-trip metric."""
+    import oracle
+    threads = os.cpu_count() or 1
+    done_bytes, t_c, t_d, used = 0, 0.0, 0.0, 0
+    for x in xs:
+        h = x.cpu().view(torch.uint8).numpy()
+        t0 = time.perf_counter()
+        c = oracle.compress("bf16", h, x.numel(), CHUNK, SUBBLOCK, threads=threads)
+        t1 = time.perf_counter()
+        y = oracle.decompress("bf16", c, x.numel(), CHUNK, threads=threads)
+        t2 = time.perf_counter()
+        assert (y == h).all()
+        t_c += t1 - t0
+        t_d += t2 - t1
+        done_bytes += h.size
+        used += 1
+        if t_c + t_d > budget_s:
+            break
+    return {
+        "value": done_bytes / (t_c + t_d) / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+        "compress_GBps": done_bytes / t_c / 1e9, "decompress_GBps": done_bytes / t_d / 1e9,
+        "sample": f"first {used} of 225 tensors ({done_bytes / 1e9:.3f} GB), compress+decompress, "
+                  f"{threads} threads (chunk-parallel)",
+    }
+
+
+def run_ours(args):
+    from lossless_float_weight_b200 import zipnn as Z
+    rank, world, local = dist_env()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    init_dist(world, "nccl")
+    stream = torch.cuda.current_stream(dev)
+
+    xs = make_workload(dev, rank, args.tensors, args.only)
+    nbytes = sum(x.numel() * 2 for x in xs)
+    outs = [torch.empty(Z.zipnn_max_compressed_bytes(Z.BF16, x.numel(), CHUNK), dtype=torch.uint8, device=dev)
+            for x in xs]
+    ws = Z.workspace(Z.BF16, max(x.numel() for x in xs), CHUNK, dev)
+    decs = [torch.empty_like(x) for x in xs]
+    torch.cuda.synchronize()
+
+    def compress_all():
+        for x, o in zip(xs, outs):
+            Z.compress_into(x, o, ws, CHUNK, stream=stream)
+
+    def decompress_all():
+        for o, d in zip(outs, decs):
+            Z.decompress_into(o, o.numel(), d, ws, CHUNK, stream=stream)
+
+    for _ in range(args.warmup):
+        compress_all()
+        decompress_all()
+    torch.cuda.synchronize()
+    csizes = [Z.compressed_size(o) for o in outs]
+    ok = all(torch.equal(d.view(torch.int16), x.view(torch.int16)) for d, x in zip(decs, xs))
+    if not ok:
+        raise RuntimeError("round trip mismatch")
+    cbytes = sum(csizes)
+
+    # timed region: K steps, events on the launching stream, kernel events on
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    Z.zipnn_timing_enable(1)
+    Z.kernel_times()
+    barrier(world, dev)
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for k in range(args.steps):
+        ev[k][0].record(stream)
+        compress_all()
+        ev[k][1].record(stream)
+        decompress_all()
+        ev[k][2].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    clk = clocks.stop()
+    ktimes = Z.kernel_times()
+    Z.zipnn_timing_enable(0)
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
+    comp_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps, world, dev)
+    dec_ms = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps, world, dev)
+    ms_step = total_ms / args.steps
+    ok = all(torch.equal(d.view(torch.int16), x.view(torch.int16)) for d, x in zip(decs, xs))
+
+    peak, peak_src = measured_peaks()
+    algo_bytes = nbytes + cbytes  # read + written, per direction
+    gpu_launches = sum(v[1] for v in ktimes.values())
+    # dominant kernel: the one with the largest share of device time
+    dom = max(ktimes.items(), key=lambda kv: kv[1][0])
+    dom_name, (dom_ms, dom_n) = dom
+    if dom_name == "decode_merge":
+        dom_bytes = (cbytes + nbytes) * args.steps
+    elif dom_name == "encode":
+        dom_bytes = (nbytes + cbytes) * args.steps
+    elif dom_name == "split_hist":
+        dom_bytes = nbytes * args.steps
+    else:
+        dom_bytes = 0
+    achieved = dom_bytes / (dom_ms / 1e3) / 1e9 if dom_ms > 0 else 0.0
+
+    # end to end through the public API, host buffers (pinned), copies inside the timed region
+    e2e = run_e2e(Z, xs, csizes, dev, stream, args, world) if not args.no_extras else None
+
+    if rank == 0:
+        cpu = cpu_baseline(xs) if world == 1 and not args.no_extras else None
+        line = {
+            "metric": METRIC,
+            "value": round(world * nbytes / (ms_step / 1e3) / 1e9, 2),
+            "unit": "GB/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(ms_step, 4),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "u32",
+            "data": "synthetic (seeded N(0, sigma_t^2) BF16 tensors of a 7B checkpoint's shapes; no trained weights)",
+            "config": {
+                "workload": WORKLOAD,
+                "step": "compress all 225 tensors, then decompress all 225 (value = uncompressed bytes per "
+                        "step / step time, x ranks)",
+                "global_batch": world * nbytes,
+                "parallelism": f"weak scaling, {world} independent checkpoint(s), no collective on the data path",
+                "l2": "inputs larger than L2 (13.2 GB per rank; no flush needed)",
+                "subblock": SUBBLOCK,
+                "chunk_bytes": CHUNK,
+            },
+            "compress": {"GBps": round(world * nbytes / (comp_ms / 1e3) / 1e9, 2), "ms": round(comp_ms, 4),
+                         "hbm_frac": round(algo_bytes / (comp_ms / 1e3) / 1e9 / peak, 4)},
+            "decompress": {"GBps": round(world * nbytes / (dec_ms / 1e3) / 1e9, 2), "ms": round(dec_ms, 4),
+                           "hbm_frac": round(algo_bytes / (dec_ms / 1e3) / 1e9 / peak, 4)},
+            "compression_ratio": round(cbytes / nbytes, 5),
+            "roofline": {
+                "kernel": dom_name,
+                "bound": "hbm",
+                "achieved": round(achieved, 1),
+                "peak": peak,
+                "peak_source": peak_src,
+                "unit": "GB/s",
+                "frac": round(achieved / peak, 4),
+                "traffic": None,
+                "avg_launch_ms": round(dom_ms / max(1, dom_n), 5),
+                "algorithmic_bytes_per_step": dom_bytes // max(1, args.steps),
+            },
+            "kernel_ms_per_step": {k: round(v[0] / args.steps, 4) for k, v in ktimes.items() if v[1]},
+            "gpu_launches": int(gpu_launches),
+            "e2e": e2e,
+            "clocks": clk,
+            "roundtrip_ok": bool(ok),
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(Z, xs, csizes, dev, stream, args, world):
+    """Same metric through the public host-buffer API: pinned host tensors in, pinned
+    host tensors out; every step copies each tensor in, compresses, copies the container
+    out and back, decompresses and copies the result out."""
+    nbytes = sum(x.numel() * 2 for x in xs)
+    h_in = [x.cpu().pin_memory() for x in xs]
+    h_cont = [torch.empty(c, dtype=torch.uint8).pin_memory() for c in csizes]
+    h_out = [torch.empty_like(h) .pin_memory() for h in h_in]
+    d_in = [torch.empty_like(x) for x in xs]
+    d_cont = [torch.empty(Z.zipnn_max_compressed_bytes(Z.BF16, x.numel(), CHUNK), dtype=torch.uint8, device=dev)
+              for x in xs]
+    d_out = [torch.empty_like(x) for x in xs]
+    ws = Z.workspace(Z.BF16, max(x.numel() for x in xs), CHUNK, dev)
+
+    def step():
+        for i in range(len(xs)):
+            Z.compress_host(h_in[i], h_cont[i], d_in[i], d_cont[i], ws, CHUNK, stream=stream)
+        for i in range(len(xs)):
+            Z.decompress_host(h_cont[i], csizes[i], h_out[i], d_cont[i], d_out[i], ws, CHUNK, stream=stream)
+
+    steps = max(1, min(args.steps, 3))
+    step()
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        step()
+    e.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(s.elapsed_time(e) / steps, world, dev)
+    ok = all(torch.equal(a.view(torch.int16), b.view(torch.int16)) for a, b in zip(h_out, h_in))
+    cb = sum(csizes)
+    return {"value": round(world * nbytes / (ms / 1e3) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": nbytes + cb, "d2h_bytes_per_step": cb + nbytes, "ms_per_step": round(ms, 3),
+            "steps": steps, "roundtrip_ok": bool(ok)}
+
+
+# ------------------------------------------------------------------ reference arm (the oracle)
+
+def run_reference(args):
+    rank, world, local = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    from lossless_float_weight_b200 import workloads as W
+    shapes = W.checkpoint_7b_shapes()
+    sig = W.checkpoint_7b_sigmas(len(shapes))
+    threads = os.cpu_count() or 1
+    # bounded sample: the first tensor of the checkpoint (4096 x 4096), generated on the CPU
+    x = W.checkpoint_7b_tensor(0, shapes[0][1], sig[0], "cpu").reshape(-1)
+    h = x.view(torch.uint8).numpy()
+    nb = h.size
+
+    def step():
+        c = oracle.compress("bf16", h, x.numel(), CHUNK, SUBBLOCK, threads=threads)
+        y = oracle.decompress("bf16", c, x.numel(), CHUNK, threads=threads)
+        return c, y
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        c, y = step()
+    dt = (time.perf_counter() - t0) / args.steps
+    assert (y == h).all()
+    v = nb / dt / 1e9
+    sample = f"tensor 0 of 225 (4096x4096, {nb / 1e6:.1f} MB), compress+decompress per step, {threads} threads"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "u32", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample": sample},
+        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--tensors", type=int, default=None,
+                    help="only the first T tensors of the checkpoint (small cases for profilers)")
+    ap.add_argument("--only", type=int, default=None, help="only tensor IDX of the checkpoint (profiler cases)")
+    ap.add_argument("--no-extras", action="store_true", help="skip the e2e and CPU-baseline legs")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+    rank, world, _ = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        if dist.is_initialized():
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -80,7 +80,7 @@ typedef enum {
 typedef struct zipnn_plan zipnn_plan_t; /* opaque; owns device code tables */
 
 #define ZIPNN_DEFAULT_CHUNK_BYTES 262144u /* 256 KiB of uncompressed values per chunk */
-#define ZIPNN_DEFAULT_SUBBLOCK 1024u      /* symbols per sub-block index entry */
+#define ZIPNN_DEFAULT_SUBBLOCK 512u       /* symbols per sub-block index entry */
 #define ZIPNN_MAX_GROUPS 64u
 #define ZIPNN_LMAX 12u
 
@@ -160,6 +160,16 @@ zipnn_status zipnn_plan_import(const void* host_buf, size_t bytes, zipnn_plan_t*
 zipnn_status zipnn_plan_assignment(const zipnn_plan_t* plan, uint32_t* host_buf, size_t cap, size_t* count);
 
 void zipnn_plan_destroy(zipnn_plan_t* plan);
+
+/* Kernel timing, a measurement aid (off by default; not a step of the codec). While
+ * enabled, every kernel the library launches is bracketed by two CUDA events on its
+ * stream. zipnn_timing_collect waits for the recorded events and writes, for kernel
+ * ids 0..count-1, the summed duration in ms and the number of launches since the last
+ * collect (either pointer may be NULL), then resets the totals. */
+zipnn_status zipnn_timing_enable(int enable);
+zipnn_status zipnn_timing_collect(double* ms, uint64_t* launches, uint32_t count);
+uint32_t zipnn_kernel_count(void);
+const char* zipnn_kernel_name(uint32_t id);
 
 const char* zipnn_status_string(zipnn_status status);
 

@@ -121,11 +121,15 @@ PlanDev plan_dev(const zipnn_plan* p) {
   return d;
 }
 
+// The kernels are built for sm_100a only; the answer is cached per device.
 bool device_ok() {
+  static int cache[128] = {0};  // 0 unknown, 1 usable, 2 not
   int dev = 0, major = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
-  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
-  return major == 10;
+  if (dev >= 0 && dev < 128 && cache[dev]) return cache[dev] == 1;
+  const bool ok = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) == cudaSuccess && major == 10;
+  if (dev >= 0 && dev < 128) cache[dev] = ok ? 1 : 2;
+  return ok;
 }
 
 }  // namespace
@@ -160,10 +164,22 @@ zipnn_status zipnn_compress_ex(zipnn_dtype dtype, const void* src, uint64_t n, u
   const Ws w = carve(wp, ws);
   const PlanDev pd = plan_dev(plan);
   cudaError_t e = cudaMemsetAsync(ws, 0, wp.zero_end, st);
-  if (e == cudaSuccess) e = launch_split_hist(src, g, w.hist, w.nonzero, st);
-  if (e == cudaSuccess) e = launch_build_tables(g, w, pd, st);
-  if (e == cudaSuccess) e = launch_layout(g, w, pd, static_cast<uint8_t*>(out), st);
-  if (e == cudaSuccess) e = launch_encode(src, g, w, static_cast<uint8_t*>(out), st);
+  if (e == cudaSuccess) {
+    TimedLaunch t(kIdHist, st);
+    e = launch_split_hist(src, g, w.hist, w.nonzero, st);
+  }
+  if (e == cudaSuccess) {
+    TimedLaunch t(kIdTables, st);
+    e = launch_build_tables(g, w, pd, st);
+  }
+  if (e == cudaSuccess) {
+    TimedLaunch t(kIdLayout, st);
+    e = launch_layout(g, w, pd, static_cast<uint8_t*>(out), st);
+  }
+  if (e == cudaSuccess) {
+    TimedLaunch t(kIdEncode, st);
+    e = launch_encode(src, g, w, static_cast<uint8_t*>(out), st);
+  }
   return cuda_status(e);
 }
 
@@ -182,9 +198,11 @@ zipnn_status zipnn_decompress(zipnn_dtype dtype, const void* in, size_t in_bytes
   if (!device_ok()) return ZIPNN_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(ws, 0, 4, st);
-  if (e == cudaSuccess)
+  if (e == cudaSuccess) {
+    TimedLaunch t(kIdDecode, st);
     e = launch_decode(static_cast<const uint8_t*>(in), in_bytes, g, static_cast<uint8_t*>(out),
                       static_cast<uint32_t*>(ws), st);
+  }
   return cuda_status(e);
 }
 

@@ -21,10 +21,11 @@ constexpr uint32_t kMaxGroups = 64;
 // Device status codes (the public zipnn_status values).
 constexpr uint32_t kStCorrupt = 3, kStTimeout = 7;
 
-// Values one thread owns in the compress kernels, and values per encode tile.
+// Values per 128-bit group of one thread, groups per encode thread, values per tile.
 constexpr int kGroupValues = 16;
+constexpr int kEncGroups = 4;
 constexpr int kEncodeThreads = 256;
-constexpr int kTileValues = kEncodeThreads * kGroupValues;  // 4096
+constexpr int kTileValues = kEncodeThreads * kGroupValues * kEncGroups;  // 16384
 
 __host__ __device__ constexpr int n_streams(int dt) { return dt == kBF16 ? 2 : dt == kFP32 ? 4 : 3; }
 __host__ __device__ constexpr int n_entropy(int dt) { return dt == kFP8 ? 2 : 1; }
@@ -110,37 +111,48 @@ __device__ __forceinline__ uint64_t observe(uint64_t* d) {
   return a.load(cuda::memory_order_acquire);
 }
 
-// Single-pass decoupled look-back (one thread): publish this tile's aggregate, walk
-// back over the predecessors of the same segment (tiles first..tile-1), summing
-// aggregates until an inclusive prefix is found, publish the inclusive prefix and
-// return the exclusive one. Tiles are handed out in launch order (a ticket), so every
-// predecessor has started and the walk ends; the spin limit only guards against bugs.
-__device__ inline uint64_t lookback(uint64_t* desc, uint32_t tile, uint32_t first, uint64_t aggregate,
-                                    uint32_t* status) {
+// Single-pass decoupled look-back, run by one whole warp: publish this tile's
+// aggregate, then inspect the 32 nearest predecessors of the same segment (tiles
+// first..tile-1) at once; the nearest one holding an inclusive prefix ends the walk,
+// otherwise all 32 aggregates are summed and the window moves back. Publishes the
+// inclusive prefix and returns the exclusive one (to every lane). Tiles are handed out
+// in launch order (a ticket), so every predecessor has started and the walk ends; the
+// spin limit only guards against bugs.
+__device__ inline uint64_t warp_lookback(uint64_t* desc, uint32_t tile, uint32_t first, uint64_t aggregate,
+                                         uint32_t* status) {
+  const int lane = threadIdx.x & 31;
   if (tile == first) {
-    publish(desc + tile, kFlagPrefix | aggregate);
+    if (lane == 0) publish(desc + tile, kFlagPrefix | aggregate);
     return 0;
   }
-  publish(desc + tile, kFlagAgg | aggregate);
+  if (lane == 0) publish(desc + tile, kFlagAgg | aggregate);
   uint64_t excl = 0;
-  uint32_t j = tile - 1;
+  int64_t base = (int64_t)tile - 1;
+  uint32_t spins = 0;
   while (true) {
-    uint64_t d = observe(desc + j);
-    uint32_t spins = 0;
-    while ((d >> 62) == 0) {
+    const int64_t j = base - lane;
+    const uint64_t d = j >= (int64_t)first ? observe(desc + j) : kFlagPrefix;  // before the segment: prefix 0
+    const uint32_t flag = (uint32_t)(d >> 62);
+    const uint32_t not_ready = __ballot_sync(0xFFFFFFFFu, flag == 0);
+    const uint32_t is_prefix = __ballot_sync(0xFFFFFFFFu, flag == 2);
+    const int pl = is_prefix ? __ffs(is_prefix) - 1 : 32;  // nearest prefix
+    const uint32_t need = pl == 32 ? 0xFFFFFFFFu : (uint32_t)((2ull << pl) - 1);
+    if (not_ready & need) {
       if (++spins > kSpinLimit) {
-        set_status(status, kStTimeout);
-        d = kFlagPrefix;  // give up: treat as prefix 0
+        if (lane == 0) set_status(status, kStTimeout);
         break;
       }
       __nanosleep(spins < 64 ? 32 : 256);
-      d = observe(desc + j);
+      continue;
     }
-    excl += d & kValueMask;
-    if ((d >> 62) == 2 || j == first) break;
-    j--;
+    uint64_t v = lane <= pl ? (d & kValueMask) : 0;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    excl += v;
+    if (pl < 32) break;
+    base -= 32;
   }
-  publish(desc + tile, kFlagPrefix | (excl + aggregate));
+  if (lane == 0) publish(desc + tile, kFlagPrefix | (excl + aggregate));
   return excl;
 }
 

@@ -16,22 +16,28 @@
 
 namespace zipnn {
 
-constexpr int kDecodeThreads = 128;
+constexpr int kDecodeThreads = 256;
 constexpr uint32_t kLutInvalid = 0x8000u;
 
 // Big-endian-within-word bit reader over 32-bit words [0, end); words past `end`
-// read as zero. buf holds nb valid bits, most significant first.
+// read as zero. buf holds nb valid bits, most significant first; the next two words
+// are already loaded (q0, q1), so a refill never waits on memory that was requested
+// less than two refills ago.
 struct BitReader {
   const uint32_t* w;
-  uint32_t pos, end;
+  uint32_t pos, end;  // pos: next word to request
   uint64_t buf;
   int nb;
+  uint32_t q0, q1;
   __device__ __forceinline__ uint32_t load(uint32_t i) const { return i < end ? bswap32(__ldg(w + i)) : 0u; }
   __device__ __forceinline__ void init(const uint32_t* words, uint32_t nwords, uint64_t bit) {
     w = words;
     end = nwords;
-    pos = (uint32_t)(bit >> 5);
-    buf = (uint64_t)load(pos++) << 32;
+    const uint32_t p0 = (uint32_t)(bit >> 5);
+    buf = (uint64_t)load(p0) << 32;
+    q0 = load(p0 + 1);
+    q1 = load(p0 + 2);
+    pos = p0 + 3;
     nb = 32;
     const int skip = (int)(bit & 31);
     buf <<= skip;
@@ -40,8 +46,10 @@ struct BitReader {
   }
   __device__ __forceinline__ void refill() {
     if (nb <= 32) {
-      buf |= (uint64_t)load(pos++) << (32 - nb);
+      buf |= (uint64_t)q0 << (32 - nb);
       nb += 32;
+      q0 = q1;
+      q1 = load(pos++);
     }
   }
   __device__ __forceinline__ uint32_t fixed(int width) {
@@ -58,7 +66,8 @@ struct BitReader {
     acc |= e;
     return (e >> 4) & 0xFFu;
   }
-  __device__ __forceinline__ uint64_t position() const { return (uint64_t)pos * 32 - (uint64_t)nb; }
+  // absolute index of the next unread bit
+  __device__ __forceinline__ uint64_t position() const { return (uint64_t)(pos - 2) * 32 - (uint64_t)nb; }
 };
 
 enum Kind : int { kKZero = 0, kKBytes = 1, kKBits = 2, kKHuff = 3 };
@@ -120,6 +129,253 @@ __device__ __forceinline__ void next_symbols(StreamState& st, uint32_t (&o)[GV],
   }
 }
 
+
+// BF16 with a HUFF exponent stream and a RAW (or ZERO) sign/fraction stream: the case
+// of every chunk of a trained or Gaussian checkpoint. 16 values per step; the
+// sign/fraction bytes of the next step are requested one step ahead.
+template <bool SM_ZERO>
+__device__ __forceinline__ int decode_bf16_fast(const uint8_t* __restrict__ in, const uint16_t* lut, const uint8_t* smp,
+                                                const uint32_t* bs, uint32_t bs_words, uint64_t start, uint64_t expect,
+                                                bool exact, uint32_t count, uint8_t* __restrict__ dst) {
+  BitReader br;
+  br.init(bs, bs_words, start);
+  uint32_t acc = 0;
+  const uint32_t full = count / 16;
+  uint4 cur = make_uint4(0, 0, 0, 0), nxt = cur, nx2 = cur, nx3 = cur;
+  if (!SM_ZERO) {
+    const uint4* sp = reinterpret_cast<const uint4*>(smp);
+    if (full > 0) cur = __ldg(sp);
+    if (full > 1) nxt = __ldg(sp + 1);
+    if (full > 2) nx2 = __ldg(sp + 2);
+    if (full > 3) nx3 = __ldg(sp + 3);
+  }
+  for (uint32_t gi = 0; gi < full; gi++) {
+    uint32_t ex[16];
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+      br.refill();
+      ex[i] = br.huff(lut, acc);
+      ex[i + 1] = br.huff(lut, acc);
+    }
+    const uint32_t x[4] = {cur.x, cur.y, cur.z, cur.w};
+    if (!SM_ZERO) {
+      cur = nxt;
+      nxt = nx2;
+      nx2 = nx3;
+      if (gi + 4 < full) nx3 = __ldg(reinterpret_cast<const uint4*>(smp) + gi + 4);
+    }
+    uint32_t o[8];
+#pragma unroll
+    for (int q = 0; q < 8; q++) {
+      const uint32_t t = SM_ZERO ? 0u : __byte_perm(x[q >> 1], 0, (q & 1) ? 0x4342 : 0x4140);
+      o[q] = (t & 0x007F007Fu) | ((t & 0x00800080u) << 8) | (ex[2 * q] << 7) | (ex[2 * q + 1] << 23);
+    }
+    uint4* d = reinterpret_cast<uint4*>(dst + (uint64_t)gi * 32);
+    d[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    d[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+  for (uint32_t v = full * 16; v < count; v++) {
+    br.refill();
+    const uint32_t e = br.huff(lut, acc);
+    const uint32_t b = SM_ZERO ? 0u : smp[v];
+    reinterpret_cast<uint16_t*>(dst)[v] = (uint16_t)merge_value<kBF16>(e, b, 0, 0);
+  }
+  const uint64_t pos = br.position();
+  return (acc & kLutInvalid) || (exact ? pos != expect : pos > expect);
+}
+
+// ---------------------------------------------------------------- staged BF16 path
+// For a BF16 chunk whose exponent stream is HUFF and whose bitstream fits a 48 KB
+// window, the whole bitstream is brought into shared memory by one TMA bulk copy
+// (cp.async.bulk, completion on an mbarrier) while the block builds its lookup table.
+// Then, in rounds, every thread decodes the next 32 exponents of its sub-block into a
+// padded shared buffer (rows of 36 bytes: conflict-free), and the block merges them
+// with the sign/fraction bytes: those are loaded as whole 32-byte sectors one round
+// ahead of use, and the merged words leave as whole 64-byte row segments.
+constexpr uint32_t kWindowBytes = 48 * 1024;
+constexpr int kRound = 32;
+constexpr int kExStride = kRound + 4;
+constexpr uint32_t kWaitLimit = 1u << 26;
+
+struct StagedSmem {
+  uint32_t bits[kWindowBytes / 4];
+  uint8_t ex[kDecodeThreads * kExStride];
+  uint64_t bar;
+};
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
+}
+// 1-D bulk copy global -> shared (no multicast); src, dst 16-byte aligned, bytes % 16 == 0
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_addr(dst)),
+               "l"(src), "r"(bytes), "r"(smem_addr(bar))
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(phase)
+      : "memory");
+  return ok != 0;
+}
+
+// Bit reader over words in shared memory; the next word is always already loaded.
+struct SmemBitReader {
+  const uint32_t* w;
+  uint32_t pos, end;
+  uint64_t buf;
+  int nb;
+  uint32_t q;
+  __device__ __forceinline__ uint32_t ld(uint32_t i) const { return i < end ? bswap32(w[i]) : 0u; }
+  __device__ __forceinline__ void init(const uint32_t* words, uint32_t nwords, uint64_t bit) {
+    w = words;
+    end = nwords;
+    const uint32_t p0 = (uint32_t)(bit >> 5);
+    buf = (uint64_t)ld(p0) << 32;
+    q = ld(p0 + 1);
+    pos = p0 + 2;
+    nb = 32;
+    const int skip = (int)(bit & 31);
+    buf <<= skip;
+    nb -= skip;
+    refill();
+  }
+  __device__ __forceinline__ void refill() {
+    if (nb <= 32) {
+      buf |= (uint64_t)q << (32 - nb);
+      nb += 32;
+      q = ld(pos++);
+    }
+  }
+  __device__ __forceinline__ uint32_t huff(const uint16_t* lut, uint32_t& acc) {
+    const uint32_t e = lut[buf >> 52];
+    const uint32_t l = e & 15u;
+    buf <<= l;
+    nb -= (int)l;
+    acc |= e;
+    return (e >> 4) & 0xFFu;
+  }
+  __device__ __forceinline__ uint64_t position() const { return (uint64_t)(pos - 1) * 32 - (uint64_t)nb; }
+};
+
+// One chunk, all threads of the block. smp: the chunk's sign/fraction payload (RAW) or
+// nullptr (ZERO); outc: the chunk's first output value. Returns nonzero if the stream
+// is inconsistent.
+__device__ int decode_bf16_staged(StagedSmem& st, const uint16_t* lut, const uint32_t* __restrict__ idx,
+                                  uint32_t bs_words, const uint8_t* __restrict__ smp, uint32_t m, uint32_t S,
+                                  uint32_t nsub, uint8_t* __restrict__ outc) {
+  const int tid = threadIdx.x;
+  int bad = 0;
+  const uint64_t cap_bits = (uint64_t)bs_words * 32;
+  const uint32_t rounds = (S + kRound - 1) / kRound;
+  for (uint32_t batch = 0; batch < nsub; batch += kDecodeThreads) {
+    const uint32_t j = batch + tid;
+    const uint32_t count = j < nsub ? min32(S, m - j * S) : 0;
+    SmemBitReader br;
+    uint32_t acc = 0;
+    uint64_t expect = 0;
+    bool exact = false;
+    if (count) {
+      const uint64_t start = __ldg(idx + j);
+      exact = j + 1 < nsub;
+      expect = exact ? __ldg(idx + j + 1) : cap_bits;
+      if ((j == 0 && start != 0) || start > cap_bits || expect < start || expect > cap_bits) bad = 1;
+      br.init(st.bits, bs_words, bad ? 0 : start);
+    }
+    for (uint32_t r = 0; r < rounds; r++) {
+      // sign/fraction bytes of this round's merge units, requested before the decode
+      uint2 smv[4];
+      uint32_t uval[4], ucnt[4];
+#pragma unroll
+      for (int p = 0; p < 4; p++) {
+        const uint32_t u = tid + p * kDecodeThreads;
+        const uint32_t row = batch + (u >> 2), part = u & 3;
+        const uint32_t rc = row < nsub ? min32(S, m - row * S) : 0;
+        const uint32_t off = r * kRound + part * 8;
+        const uint32_t n = off < rc ? min32(8, rc - off) : 0;
+        uval[p] = row * S + off;
+        ucnt[p] = n;
+        smv[p] = make_uint2(0, 0);
+        if (smp && n == 8) smv[p] = __ldg(reinterpret_cast<const uint2*>(smp + uval[p]));
+        else if (smp && n) {
+          uint32_t lo = 0, hi = 0;
+          for (uint32_t i = 0; i < n; i++) {
+            const uint32_t b = smp[uval[p] + i];
+            if (i < 4) lo |= b << (8 * i);
+            else hi |= b << (8 * (i - 4));
+          }
+          smv[p] = make_uint2(lo, hi);
+        }
+      }
+      // decode up to 32 exponents of my sub-block
+      const uint32_t base = r * kRound;
+      if (base < count) {
+        uint32_t* row = reinterpret_cast<uint32_t*>(st.ex + tid * kExStride);
+        if (base + kRound <= count) {
+#pragma unroll
+          for (int k = 0; k < kRound / 4; k++) {
+            br.refill();
+            const uint32_t e0 = br.huff(lut, acc);
+            const uint32_t e1 = br.huff(lut, acc);
+            br.refill();
+            const uint32_t e2 = br.huff(lut, acc);
+            const uint32_t e3 = br.huff(lut, acc);
+            row[k] = e0 | (e1 << 8) | (e2 << 16) | (e3 << 24);
+          }
+        } else {
+          const uint32_t n = count - base;
+          for (uint32_t k = 0; k < n; k++) {
+            br.refill();
+            st.ex[tid * kExStride + k] = (uint8_t)br.huff(lut, acc);
+          }
+        }
+      }
+      __syncthreads();
+      // merge and store
+#pragma unroll
+      for (int p = 0; p < 4; p++) {
+        const uint32_t u = tid + p * kDecodeThreads;
+        if (!ucnt[p]) continue;
+        const uint8_t* exr = st.ex + (u >> 2) * kExStride + (u & 3) * 8;
+        const uint32_t ea = *reinterpret_cast<const uint32_t*>(exr);
+        const uint32_t eb = *reinterpret_cast<const uint32_t*>(exr + 4);
+        const uint32_t xs[2] = {smv[p].x, smv[p].y};
+        const uint32_t es[2] = {ea, eb};
+        uint32_t o[4];
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+          const uint32_t t = __byte_perm(xs[q >> 1], 0, (q & 1) ? 0x4342 : 0x4140);
+          const uint32_t ee = __byte_perm(es[q >> 1], 0, (q & 1) ? 0x4342 : 0x4140);
+          o[q] = (t & 0x007F007Fu) | ((t & 0x00800080u) << 8) | (ee << 7);
+        }
+        uint8_t* d = outc + (uint64_t)uval[p] * 2;
+        if (ucnt[p] == 8) {
+          *reinterpret_cast<uint4*>(d) = make_uint4(o[0], o[1], o[2], o[3]);
+        } else {
+          for (uint32_t i = 0; i < ucnt[p]; i++)
+            reinterpret_cast<uint16_t*>(d)[i] = (uint16_t)(o[i >> 1] >> (16 * (i & 1)));
+        }
+      }
+      __syncthreads();
+    }
+    if (count) {
+      const uint64_t pos = br.position();
+      if ((acc & kLutInvalid) || (exact ? pos != expect : pos > expect)) bad = 1;
+    }
+  }
+  return bad;
+}
+
 template <int DT>
 struct DecodeSmem {
   uint16_t lut[n_entropy(DT)][4096];
@@ -133,15 +389,16 @@ struct DecodeSmem {
   uint64_t off[n_streams(DT)], end[n_streams(DT)];
   uint64_t off_codes;
   uint32_t S, G;
-  int bad;
+  int bad, staged;
 };
 
 template <int DT>
-__global__ void __launch_bounds__(kDecodeThreads) k_decode(const uint8_t* __restrict__ in, uint64_t in_bytes, Geo g,
+__global__ void __launch_bounds__(kDecodeThreads, DT == kBF16 ? 3 : 1) k_decode(const uint8_t* __restrict__ in, uint64_t in_bytes, Geo g,
                                                            uint8_t* __restrict__ out, uint32_t* status) {
   constexpr int NS = n_streams(DT), NE = n_entropy(DT), VB = value_bytes(DT);
   constexpr int GV = DT == kBF16 ? 8 : DT == kFP32 ? 4 : 16;  // values per 16-byte store
   __shared__ DecodeSmem<DT> sm;
+  extern __shared__ __align__(128) uint8_t dyn_smem[];  // StagedSmem for BF16 launches
   const int tid = threadIdx.x;
   const uint32_t c = blockIdx.x;
   const uint64_t clo = (uint64_t)c * g.m0;
@@ -212,6 +469,26 @@ __global__ void __launch_bounds__(kDecodeThreads) k_decode(const uint8_t* __rest
     sm.S = S;
     sm.G = G;
     sm.bad = bad;
+    sm.staged = 0;
+    if constexpr (DT == kBF16) {
+      // staged path: HUFF exponents, RAW or ZERO sign/fraction bytes, bitstream in the window
+      if (!bad && sm.mode[0] == kModeHuff && sm.mode[1] != kModeHuff) {
+        const uint64_t nsub = ceil_div(m, S);
+        const uint32_t rec = sm.code[0] == kNoCode ? record_bytes(DT, 0) : 0;
+        const uint64_t bs_off = sm.off[0] + rec + round16(4 * nsub);
+        const uint64_t bs_bytes = sm.end[0] > bs_off ? sm.end[0] - bs_off : 0;
+        if (bs_off <= sm.end[0] && bs_bytes <= kWindowBytes && nsub <= 0xFFFFFFFFull) {
+          StagedSmem& stg = *reinterpret_cast<StagedSmem*>(dyn_smem);
+          mbar_init(&stg.bar, 1);
+          mbar_expect_tx(&stg.bar, (uint32_t)bs_bytes);
+          for (uint64_t o = 0; o < bs_bytes; o += 16384) {
+            const uint32_t nb = (uint32_t)min64(16384, bs_bytes - o);
+            bulk_g2s(reinterpret_cast<uint8_t*>(stg.bits) + o, in + bs_off + o, nb, &stg.bar);
+          }
+          sm.staged = 1;
+        }
+      }
+    }
   }
   __syncthreads();
   if (sm.bad) {
@@ -261,19 +538,25 @@ __global__ void __launch_bounds__(kDecodeThreads) k_decode(const uint8_t* __rest
       if (lane == 0) sm.bad = 1;
     } else {
       warp_canonical(sm.lens[e], sm.enc[e]);
-      if (lane == 0) {
-        uint32_t count[kLmax + 1] = {0};
-        for (int s = 0; s < 256; s++) count[sm.lens[e][s]]++;
-        uint32_t code = 0, offs = 0;
-        count[0] = 0;
-        sm.limit[e][0] = 0;
-        for (int l = 1; l <= kLmax; l++) {
-          code = (code + count[l - 1]) << 1;
+      // number of codes of each length, by ballots over the 256 symbols
+      uint32_t L[8];
+#pragma unroll
+      for (int i = 0; i < 8; i++) L[i] = sm.lens[e][i * 32 + lane];
+      uint32_t code = 0, offs = 0, prev = 0;
+      if (lane == 0) sm.limit[e][0] = 0;
+#pragma unroll
+      for (int l = 1; l <= kLmax; l++) {
+        uint32_t cnt = 0;
+#pragma unroll
+        for (int i = 0; i < 8; i++) cnt += __popc(__ballot_sync(0xFFFFFFFFu, L[i] == (uint32_t)l));
+        code = (code + prev) << 1;
+        if (lane == 0) {
           sm.first[e][l] = code;
           sm.offset[e][l] = offs;
-          offs += count[l];
-          sm.limit[e][l] = (code + count[l]) << (kLmax - l);
+          sm.limit[e][l] = (code + cnt) << (kLmax - l);
         }
+        offs += cnt;
+        prev = cnt;
       }
     }
   }
@@ -309,11 +592,55 @@ __global__ void __launch_bounds__(kDecodeThreads) k_decode(const uint8_t* __rest
   }
   __syncthreads();
 
-  // decode: one sub-block per thread per pass
   const uint64_t nsub = ceil_div(m, S);
+  if constexpr (DT == kBF16) {
+    if (sm.staged) {
+      StagedSmem& stg = *reinterpret_cast<StagedSmem*>(dyn_smem);
+      uint32_t spins = 0;
+      while (!mbar_try_wait(&stg.bar, 0)) {
+        if (++spins > kWaitLimit) {  // the copy never landed: report, keep waiting for it (bounded again)
+          if (tid == 0) set_status(status, kStTimeout);
+          for (uint32_t k = 0; k < kWaitLimit && !mbar_try_wait(&stg.bar, 0); k++) __nanosleep(1024);
+          return;
+        }
+        __nanosleep(32);
+      }
+      const uint32_t rec = sm.code[0] == kNoCode ? record_bytes(DT, 0) : 0;
+      const uint32_t* idx = reinterpret_cast<const uint32_t*>(in + sm.off[0] + rec);
+      const uint64_t bs_off = sm.off[0] + rec + round16(4 * nsub);
+      const uint32_t bs_words = (uint32_t)((sm.end[0] - bs_off) / 4);
+      const uint8_t* smp = sm.mode[1] == kModeRaw ? in + sm.off[1] : nullptr;
+      const int bad = decode_bf16_staged(stg, sm.lut[0], idx, bs_words, smp, m, S, (uint32_t)nsub, out + clo * VB);
+      if (bad) set_status(status, kStCorrupt);
+      return;
+    }
+  }
+  // decode: one sub-block per thread per pass
   for (uint64_t j = tid; j < nsub; j += kDecodeThreads) {
     const uint32_t sb_lo = (uint32_t)(j * S);
     const uint32_t count = min32(S, m - sb_lo);
+    if constexpr (DT == kBF16) {
+      if (sm.mode[0] == kModeHuff && sm.mode[1] != kModeHuff) {
+        const uint32_t rec = sm.code[0] == kNoCode ? record_bytes(DT, 0) : 0;
+        const uint32_t* idx = reinterpret_cast<const uint32_t*>(in + sm.off[0] + rec);
+        const uint64_t bs_off = sm.off[0] + rec + round16(4 * nsub);
+        const uint64_t cap_bits = (sm.end[0] - bs_off) * 8;
+        const uint64_t start = __ldg(idx + j);
+        const bool exact = j + 1 < nsub;
+        const uint64_t expect = exact ? __ldg(idx + j + 1) : cap_bits;
+        int bad = (j == 0 && start != 0) || start > cap_bits || expect < start || expect > cap_bits;
+        const uint32_t* bs = reinterpret_cast<const uint32_t*>(in + bs_off);
+        uint8_t* dst = out + (clo + sb_lo) * VB;
+        if (sm.mode[1] == kModeZero)
+          bad |= decode_bf16_fast<true>(in, sm.lut[0], nullptr, bs, (uint32_t)(cap_bits / 32), bad ? 0 : start, expect,
+                                        exact, count, dst);
+        else
+          bad |= decode_bf16_fast<false>(in, sm.lut[0], in + sm.off[1] + sb_lo, bs, (uint32_t)(cap_bits / 32),
+                                         bad ? 0 : start, expect, exact, count, dst);
+        if (bad) set_status(status, kStCorrupt);
+        continue;
+      }
+    }
     StreamState st[NS];
     uint64_t expect_end[NS];
     bool check_exact[NS];
@@ -411,7 +738,20 @@ __global__ void __launch_bounds__(kDecodeThreads) k_decode(const uint8_t* __rest
 template <int DT>
 static cudaError_t decode_t(const uint8_t* in, uint64_t in_bytes, const Geo& g, uint8_t* out, uint32_t* status,
                             cudaStream_t st) {
-  k_decode<DT><<<g.n_chunks, kDecodeThreads, 0, st>>>(in, in_bytes, g, out, status);
+  const size_t dyn = DT == kBF16 ? sizeof(StagedSmem) : 0;
+  if (dyn) {
+    static int done[128] = {0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 128 || !done[dev]) {
+      e = cudaFuncSetAttribute(k_decode<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+      if (e == cudaSuccess) e = cudaFuncSetAttribute(k_decode<DT>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+      if (e != cudaSuccess) return e;
+      if (dev >= 0 && dev < 128) done[dev] = 1;
+    }
+  }
+  k_decode<DT><<<g.n_chunks, kDecodeThreads, dyn, st>>>(in, in_bytes, g, out, status);
   return cudaGetLastError();
 }
 

@@ -85,6 +85,56 @@ __device__ __forceinline__ void load_split16(const uint8_t* __restrict__ p, int 
   }
 }
 
+// The raw 32-bit words of NV consecutive values held by one thread.
+template <int DT, int NV>
+struct RawValues {
+  static constexpr int kWords = NV * value_bytes(DT) / 4;
+  uint32_t w[kWords];
+};
+
+// Load NV consecutive values (16-byte aligned); values at or beyond cnt read as 0 and
+// are never fetched.
+template <int DT, int NV>
+__device__ __forceinline__ void load_values(const uint8_t* __restrict__ p, int cnt, RawValues<DT, NV>& r) {
+  constexpr int W = RawValues<DT, NV>::kWords;
+  if (cnt >= NV) {
+#pragma unroll
+    for (int j = 0; j < W / 4; j++) {
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(p) + j);
+      r.w[4 * j] = a.x;
+      r.w[4 * j + 1] = a.y;
+      r.w[4 * j + 2] = a.z;
+      r.w[4 * j + 3] = a.w;
+    }
+  } else {
+    constexpr int VB = value_bytes(DT);
+#pragma unroll
+    for (int j = 0; j < W; j++) {
+      uint32_t x = 0;
+#pragma unroll
+      for (int b = 0; b < 4; b++)
+        if ((4 * j + b) / VB < cnt) x |= (uint32_t)p[4 * j + b] << (8 * b);
+      r.w[j] = x;
+    }
+  }
+}
+
+// Symbol of stream s for value i (the split above).
+template <int DT, int NV>
+__device__ __forceinline__ uint32_t symbol(const RawValues<DT, NV>& r, int s, int i) {
+  if constexpr (DT == kBF16) {
+    const uint32_t v = (r.w[i >> 1] >> (16 * (i & 1))) & 0xFFFFu;
+    return s == 0 ? (v >> 7) & 0xFFu : ((v >> 8) & 0x80u) | (v & 0x7Fu);
+  } else if constexpr (DT == kFP32) {
+    const uint32_t u = r.w[i];
+    return s == 0 ? (u >> 23) & 0xFFu
+                  : s == 1 ? ((u >> 24) & 0x80u) | ((u >> 16) & 0x7Fu) : s == 2 ? (u >> 8) & 0xFFu : u & 0xFFu;
+  } else {
+    const uint32_t b = (r.w[i >> 2] >> (8 * (i & 3))) & 0xFFu;
+    return s == 0 ? (b >> 3) & 0xFu : s == 1 ? b & 7u : b >> 7;
+  }
+}
+
 // Merge: the inverse of the split for one value.
 template <int DT>
 __device__ __forceinline__ uint32_t merge_value(uint32_t s0, uint32_t s1, uint32_t s2, uint32_t s3) {

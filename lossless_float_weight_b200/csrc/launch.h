@@ -5,6 +5,23 @@
 
 namespace zipnn {
 
+// Kernel ids of the optional event timing (timing.cu).
+enum KernelId { kIdHist = 0, kIdTables, kIdLayout, kIdEncode, kIdDecode, kIdCodeLengths, kIdPlan, kNumKernelIds };
+
+// Brackets one launch with CUDA events on `st` while timing is enabled.
+class TimedLaunch {
+ public:
+  TimedLaunch(int id, cudaStream_t st);
+  ~TimedLaunch();
+  TimedLaunch(const TimedLaunch&) = delete;
+  TimedLaunch& operator=(const TimedLaunch&) = delete;
+
+ private:
+  int id_;
+  cudaStream_t st_;
+  cudaEvent_t start_ = nullptr, stop_ = nullptr;
+};
+
 cudaError_t launch_split_hist(const void* src, const Geo& g, uint32_t* hist, uint32_t* nonzero, cudaStream_t st);
 cudaError_t launch_build_tables(const Geo& g, const Ws& ws, const PlanDev& plan, cudaStream_t st);
 cudaError_t launch_code_lengths(const uint64_t* hist, uint32_t count, uint32_t alphabet_size, uint8_t* lens,

@@ -13,18 +13,20 @@
 namespace zipnn {
 
 constexpr int kHistThreads = 256;
-constexpr uint32_t kHistSlice = 16384;  // values of one chunk per histogram block
+constexpr uint32_t kHistSlice = 32768;  // values of one chunk per histogram block
 
 // THEORY-599 note, "Order-0 only (section III-A b)": the model of a chunk is the count
-// of each symbol. Each warp keeps its own 256-bin table in shared memory; lanes holding
-// the same symbol are found with __match_any_sync and one of them adds their number.
+// of each symbol. The block keeps one counter per (symbol, lane) in shared memory, so
+// the 32 lanes of a warp always add into 32 different banks (lane l owns column l);
+// warps share the table through shared atomics. The columns are summed at the end.
 template <int DT>
 __global__ void __launch_bounds__(kHistThreads) k_split_hist(const uint8_t* __restrict__ src, Geo g, uint32_t slices,
                                                              uint32_t* __restrict__ hist, uint32_t* __restrict__ nonzero) {
   constexpr int NS = n_streams(DT), NE = n_entropy(DT), VB = value_bytes(DT), NW = kHistThreads / 32;
-  __shared__ uint32_t sh[NW][NE][256];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int i = tid; i < NW * NE * 256; i += kHistThreads) (&sh[0][0][0])[i] = 0;
+  constexpr int A0 = alphabet(DT, 0), A1 = NE > 1 ? alphabet(DT, 1) : 0;
+  __shared__ uint32_t sh[(A0 + A1) * 32];
+  const int tid = threadIdx.x, lane = tid & 31;
+  for (int i = tid; i < (A0 + A1) * 32; i += kHistThreads) sh[i] = 0;
   __syncthreads();
   const uint32_t c = blockIdx.x / slices, sl = blockIdx.x % slices;
   const uint64_t clo = (uint64_t)c * g.m0;
@@ -33,23 +35,24 @@ __global__ void __launch_bounds__(kHistThreads) k_split_hist(const uint8_t* __re
   uint32_t nz[NS];
 #pragma unroll
   for (int s = 0; s < NS; s++) nz[s] = 0;
-  for (uint32_t base = lo + warp * 32 * kGroupValues; base < hi; base += NW * 32 * kGroupValues) {
-    const uint32_t v0 = base + lane * kGroupValues;
-    const int cnt = v0 < hi ? (int)min32(kGroupValues, hi - v0) : 0;
-    uint32_t sym[NS][16];
-    load_split16<DT>(src + (clo + v0) * VB, cnt, sym);
+  uint32_t* col0 = sh + lane;
+  uint32_t* col1 = sh + A0 * 32 + lane;
+  constexpr int NV = 64;  // consecutive values per thread per pass, loaded up front
+  for (uint32_t v0 = lo + tid * NV; v0 < hi; v0 += kHistThreads * NV) {
+    const int cnt = (int)min32(NV, hi - v0);
+    RawValues<DT, NV> raw;
+    load_values<DT, NV>(src + (clo + v0) * VB, cnt, raw);
 #pragma unroll
-    for (int i = 0; i < 16; i++) {
-      const bool valid = i < cnt;
-#pragma unroll
-      for (int e = 0; e < NE; e++) {
-        const uint32_t key = valid ? sym[e][i] : 0x100u;
-        const uint32_t peers = __match_any_sync(0xFFFFFFFFu, key);
-        if (valid && lane == __ffs(peers) - 1) atomicAdd(&sh[warp][e][key], (uint32_t)__popc(peers));
+    for (int i = 0; i < NV; i++) {
+      if (i < cnt) {
+        atomicAdd(col0 + symbol<DT, NV>(raw, 0, i) * 32, 1u);
+        if (NE > 1) atomicAdd(col1 + symbol<DT, NV>(raw, 1, i) * 32, 1u);
       }
-#pragma unroll
-      for (int s = 0; s < NS; s++) nz[s] |= sym[s][i];
     }
+#pragma unroll
+    for (int i = 0; i < NV; i++)
+#pragma unroll
+      for (int s = 0; s < NS; s++) nz[s] |= symbol<DT, NV>(raw, s, i);
   }
 #pragma unroll
   for (int s = 0; s < NS; s++) {
@@ -57,12 +60,13 @@ __global__ void __launch_bounds__(kHistThreads) k_split_hist(const uint8_t* __re
     if (nonzero && lane == 0 && v) atomicOr(&nonzero[(uint64_t)c * NS + s], v);
   }
   __syncthreads();
-#pragma unroll
-  for (int e = 0; e < NE; e++) {
+  // column sums: thread b reads its row starting at lane b, so a warp hits 32 banks
+  for (int b = tid; b < A0 + A1; b += kHistThreads) {
     uint32_t sum = 0;
-#pragma unroll
-    for (int w = 0; w < NW; w++) sum += sh[w][e][tid];
-    if (sum) atomicAdd(&hist[((uint64_t)c * NE + e) * 256 + tid], sum);
+#pragma unroll 8
+    for (int l = 0; l < 32; l++) sum += sh[b * 32 + ((l + b) & 31)];
+    const int e = b < A0 ? 0 : 1, sym = b < A0 ? b : b - A0;
+    if (sum) atomicAdd(&hist[((uint64_t)c * NE + e) * 256 + sym], sum);
   }
 }
 
@@ -242,7 +246,10 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout(Geo g, Ws ws, PlanDev
   }
   uint64_t total;
   uint64_t before = block_scan_u64(mine, s_warp, total);
-  if (tid == 0) s_prefix = lookback(ws.scan_desc, tile, 0, total, ws.status);
+  if (tid < 32) {
+    const uint64_t p = warp_lookback(ws.scan_desc, tile, 0, total, ws.status);
+    if (tid == 0) s_prefix = p;
+  }
   __syncthreads();
   uint64_t pos = g.off_payload + s_prefix + before;
 #pragma unroll
@@ -316,10 +323,23 @@ cudaError_t launch_split_hist(const void* src, const Geo& g, uint32_t* hist, uin
   }
 }
 
+// Opt a kernel into more than 48 KB of dynamic shared memory, once per device.
+template <typename K>
+static cudaError_t allow_smem(K kernel, size_t bytes, int slot) {
+  static int done[8][128] = {{0}};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 128 && done[slot][dev]) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < 128) done[slot][dev] = 1;
+  return e;
+}
+
 template <int DT>
 static cudaError_t tables_t(const Geo& g, const Ws& ws, const PlanDev& plan, cudaStream_t st) {
   const size_t smem = sizeof(HuffBlockSmem);
-  cudaError_t e = cudaFuncSetAttribute(k_build_tables<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = allow_smem(k_build_tables<DT>, smem, DT);
   if (e != cudaSuccess) return e;
   k_build_tables<DT><<<g.n_chunks * n_entropy(DT), kHuffWarps * 32, smem, st>>>(g, ws, plan);
   return cudaGetLastError();
@@ -336,7 +356,7 @@ cudaError_t launch_build_tables(const Geo& g, const Ws& ws, const PlanDev& plan,
 cudaError_t launch_code_lengths(const uint64_t* hist, uint32_t count, uint32_t alphabet_size, uint8_t* lens,
                                 uint32_t* enc, cudaStream_t st) {
   const size_t smem = sizeof(HuffBlockSmem);
-  cudaError_t e = cudaFuncSetAttribute(k_code_lengths, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = allow_smem(k_code_lengths, smem, 3);
   if (e != cudaSuccess) return e;
   if (count == 0) return cudaSuccess;
   k_code_lengths<<<count, kHuffWarps * 32, smem, st>>>(hist, alphabet_size, lens, enc);

@@ -22,7 +22,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 BF16, FP32, FP8_E4M3 = 0, 1, 2
 OK, ERR_INVALID_ARG, ERR_OUT_TOO_SMALL, ERR_CORRUPT, ERR_PLAN_MISMATCH, ERR_CUDA, ERR_UNSUPPORTED, ERR_TIMEOUT = range(8)
 DEFAULT_CHUNK_BYTES = 262144
-DEFAULT_SUBBLOCK = 1024
+DEFAULT_SUBBLOCK = 512
 MAX_GROUPS = 64
 
 _u64, _u32, _vp, _sz, _i = ctypes.c_uint64, ctypes.c_uint32, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
@@ -51,12 +51,17 @@ zipnn_plan_import = _sig("zipnn_plan_import", _i, _vp, _sz, ctypes.POINTER(_vp))
 zipnn_plan_assignment = _sig("zipnn_plan_assignment", _i, _vp, _vp, _sz, ctypes.POINTER(_sz))
 zipnn_plan_destroy = _sig("zipnn_plan_destroy", None, _vp)
 zipnn_status_string = _sig("zipnn_status_string", ctypes.c_char_p, _i)
+zipnn_timing_enable = _sig("zipnn_timing_enable", _i, _i)
+zipnn_timing_collect = _sig("zipnn_timing_collect", _i, _vp, _vp, _u32)
+zipnn_kernel_count = _sig("zipnn_kernel_count", _u32)
+zipnn_kernel_name = _sig("zipnn_kernel_name", ctypes.c_char_p, _u32)
 
 C_ABI_NAMES = [
     "zipnn_max_compressed_bytes", "zipnn_workspace_bytes", "zipnn_compress", "zipnn_compress_ex",
     "zipnn_decompress", "zipnn_compressed_size", "zipnn_get_status", "zipnn_histogram", "zipnn_code_lengths",
     "zipnn_plan_create", "zipnn_plan_export", "zipnn_plan_import", "zipnn_plan_assignment", "zipnn_plan_destroy",
-    "zipnn_status_string",
+    "zipnn_status_string", "zipnn_timing_enable", "zipnn_timing_collect", "zipnn_kernel_count",
+    "zipnn_kernel_name",
 ]
 
 
@@ -218,6 +223,16 @@ def decompress_host(container_host, nbytes, out_host, dev_in, dev_out, ws, chunk
     dev_in[:nbytes].copy_(container_host[:nbytes], non_blocking=True)
     decompress_into(dev_in, nbytes, dev_out, ws, chunk_bytes, stream)
     out_host.reshape(-1).copy_(dev_out, non_blocking=True)
+
+
+def kernel_times():
+    """Collect the event timing of every kernel launched since the last call:
+    {name: (total ms, launches)}. Waits for the recorded events."""
+    k = zipnn_kernel_count()
+    ms = (ctypes.c_double * k)()
+    n = (ctypes.c_uint64 * k)()
+    check(zipnn_timing_collect(ms, n, k), "zipnn_timing_collect")
+    return {zipnn_kernel_name(i).decode(): (ms[i], n[i]) for i in range(k)}
 
 
 def histogram(x, chunk_bytes=DEFAULT_CHUNK_BYTES, stream=None):

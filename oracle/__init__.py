@@ -101,7 +101,7 @@ def max_compressed_bytes(dtype, n, chunk_bytes, n_groups=0):
     return int(lib().orc_max_compressed_bytes(DTYPES[dtype], n, chunk_bytes, n_groups))
 
 
-def compress(dtype, data, n=None, chunk_bytes=262144, S=1024, plan_lens=None, threads=1):
+def compress(dtype, data, n=None, chunk_bytes=262144, S=512, plan_lens=None, threads=1):
     """Return the container (numpy uint8) for the n values held in data."""
     b = _bytes_view(data)
     if n is None:

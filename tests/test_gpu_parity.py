@@ -14,7 +14,7 @@ import golden_util as GU
 
 pytestmark = pytest.mark.gpu
 
-S_DEFAULT = 1024
+S_DEFAULT = 512
 CB = 262144
 
 
