@@ -190,17 +190,30 @@ def run_ours(args):
     nbytes = sum(x.numel() * 2 for x in xs)
     outs = [torch.empty(Z.zipnn_max_compressed_bytes(Z.BF16, x.numel(), CHUNK), dtype=torch.uint8, device=dev)
             for x in xs]
-    ws = Z.workspace(Z.BF16, max(x.numel() for x in xs), CHUNK, dev)
+    # tensors go round-robin to NSTREAMS streams, each with its own workspace, so that
+    # one tensor's tail overlaps the next tensor's work
+    streams = [torch.cuda.Stream(dev) for _ in range(args.streams)]
+    wss = [Z.workspace(Z.BF16, max(x.numel() for x in xs), CHUNK, dev) for _ in streams]
     decs = [torch.empty_like(x) for x in xs]
     torch.cuda.synchronize()
 
+    def fan_out(fn):
+        ev = torch.cuda.Event()
+        ev.record(stream)
+        for s in streams:
+            s.wait_event(ev)
+        for i in range(len(xs)):
+            fn(i, streams[i % len(streams)], wss[i % len(streams)])
+        for s in streams:
+            e2 = torch.cuda.Event()
+            e2.record(s)
+            stream.wait_event(e2)
+
     def compress_all():
-        for x, o in zip(xs, outs):
-            Z.compress_into(x, o, ws, CHUNK, stream=stream)
+        fan_out(lambda i, s, w: Z.compress_into(xs[i], outs[i], w, CHUNK, stream=s))
 
     def decompress_all():
-        for o, d in zip(outs, decs):
-            Z.decompress_into(o, o.numel(), d, ws, CHUNK, stream=stream)
+        fan_out(lambda i, s, w: Z.decompress_into(outs[i], outs[i].numel(), decs[i], w, CHUNK, stream=s))
 
     for _ in range(args.warmup):
         compress_all()
@@ -259,7 +272,7 @@ def run_ours(args):
     achieved = dom_bytes / (dom_ms / 1e3) / 1e9 if dom_ms > 0 else 0.0
 
     # end to end through the public API, host buffers (pinned), copies inside the timed region
-    e2e = run_e2e(Z, xs, csizes, dev, stream, args, world) if not args.no_extras else None
+    e2e = run_e2e(Z, xs, csizes, dev, stream, streams, args, world) if not args.no_extras else None
 
     if rank == 0:
         cpu = cpu_baseline(xs) if world == 1 and not args.no_extras else None
@@ -284,6 +297,7 @@ def run_ours(args):
                 "parallelism": f"weak scaling, {world} independent checkpoint(s), no collective on the data path",
                 "l2": "inputs larger than L2 (13.2 GB per rank; no flush needed)",
                 "subblock": SUBBLOCK,
+                "streams": args.streams,
                 "chunk_bytes": CHUNK,
             },
             "compress": {"GBps": round(world * nbytes / (comp_ms / 1e3) / 1e9, 2), "ms": round(comp_ms, 4),
@@ -314,37 +328,60 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
 
 
-def run_e2e(Z, xs, csizes, dev, stream, args, world):
-    """Same metric through the public host-buffer API: pinned host tensors in, pinned
-    host tensors out; every step copies each tensor in, compresses, copies the container
-    out and back, decompresses and copies the result out."""
+def run_e2e(Z, xs, csizes, dev, stream, streams, args, world):
+    """Same metric through the public API with host buffers: pinned host tensors in,
+    pinned host tensors out. Every step copies each tensor to the device, compresses
+    it, reads its size and copies the container back, then copies each container to
+    the device, decompresses it and copies the values back."""
     nbytes = sum(x.numel() * 2 for x in xs)
     h_in = [x.cpu().pin_memory() for x in xs]
     h_cont = [torch.empty(c, dtype=torch.uint8).pin_memory() for c in csizes]
-    h_out = [torch.empty_like(h) .pin_memory() for h in h_in]
+    h_out = [torch.empty_like(h).pin_memory() for h in h_in]
     d_in = [torch.empty_like(x) for x in xs]
     d_cont = [torch.empty(Z.zipnn_max_compressed_bytes(Z.BF16, x.numel(), CHUNK), dtype=torch.uint8, device=dev)
               for x in xs]
     d_out = [torch.empty_like(x) for x in xs]
-    ws = Z.workspace(Z.BF16, max(x.numel() for x in xs), CHUNK, dev)
+    wss = [Z.workspace(Z.BF16, max(x.numel() for x in xs), CHUNK, dev) for _ in streams]
+    ns = len(streams)
 
     def step():
+        ev = torch.cuda.Event()
+        ev.record(stream)
+        for s in streams:
+            s.wait_event(ev)
         for i in range(len(xs)):
-            Z.compress_host(h_in[i], h_cont[i], d_in[i], d_cont[i], ws, CHUNK, stream=stream)
+            s = streams[i % ns]
+            with torch.cuda.stream(s):
+                d_in[i].copy_(h_in[i], non_blocking=True)
+            Z.compress_into(d_in[i], d_cont[i], wss[i % ns], CHUNK, stream=s)
         for i in range(len(xs)):
-            Z.decompress_host(h_cont[i], csizes[i], h_out[i], d_cont[i], d_out[i], ws, CHUNK, stream=stream)
+            s = streams[i % ns]
+            size = Z.compressed_size(d_cont[i], stream=s)
+            with torch.cuda.stream(s):
+                h_cont[i][:size].copy_(d_cont[i][:size], non_blocking=True)
+        for i in range(len(xs)):
+            s = streams[i % ns]
+            with torch.cuda.stream(s):
+                d_cont[i][: csizes[i]].copy_(h_cont[i], non_blocking=True)
+            Z.decompress_into(d_cont[i], csizes[i], d_out[i], wss[i % ns], CHUNK, stream=s)
+            with torch.cuda.stream(s):
+                h_out[i].copy_(d_out[i], non_blocking=True)
+        for s in streams:
+            e2 = torch.cuda.Event()
+            e2.record(s)
+            stream.wait_event(e2)
 
     steps = max(1, min(args.steps, 3))
     step()
     torch.cuda.synchronize()
     barrier(world, dev)
-    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record(stream)
+    s0, e0 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
     for _ in range(steps):
         step()
-    e.record(stream)
+    e0.record(stream)
     torch.cuda.synchronize()
-    ms = max_over_ranks(s.elapsed_time(e) / steps, world, dev)
+    ms = max_over_ranks(s0.elapsed_time(e0) / steps, world, dev)
     ok = all(torch.equal(a.view(torch.int16), b.view(torch.int16)) for a, b in zip(h_out, h_in))
     cb = sum(csizes)
     return {"value": round(world * nbytes / (ms / 1e3) / 1e9, 2), "unit": "GB/s",
@@ -402,6 +439,7 @@ def main():
                     help="only the first T tensors of the checkpoint (small cases for profilers)")
     ap.add_argument("--only", type=int, default=None, help="only tensor IDX of the checkpoint (profiler cases)")
     ap.add_argument("--no-extras", action="store_true", help="skip the e2e and CPU-baseline legs")
+    ap.add_argument("--streams", type=int, default=4, help="CUDA streams the tensors are spread over")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

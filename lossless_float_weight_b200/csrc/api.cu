@@ -62,7 +62,7 @@ WsPlan ws_plan(const Geo& g) {
   const uint64_t C = g.n_chunks, NE = (uint64_t)n_entropy(g.dt), K = g.n_entries;
   WsPlan p;
   uint64_t o = 0;
-  p.status = o;     o = align_up(o + 256);
+  p.status = o;     o = align_up(o + 16 + C * 4);  // status, tickets, per-chunk counters
   p.hist = o;       o = align_up(o + C * NE * 256 * 4);
   p.nonzero = o;    o = align_up(o + K * 4);
   p.scan_desc = o;  o = align_up(o + (uint64_t)layout_tiles(g.n_entries) * 8);
@@ -166,11 +166,7 @@ zipnn_status zipnn_compress_ex(zipnn_dtype dtype, const void* src, uint64_t n, u
   cudaError_t e = cudaMemsetAsync(ws, 0, wp.zero_end, st);
   if (e == cudaSuccess) {
     TimedLaunch t(kIdHist, st);
-    e = launch_split_hist(src, g, w.hist, w.nonzero, st);
-  }
-  if (e == cudaSuccess) {
-    TimedLaunch t(kIdTables, st);
-    e = launch_build_tables(g, w, pd, st);
+    e = launch_split_hist(src, g, w.hist, w.nonzero, &w, pd, st);
   }
   if (e == cudaSuccess) {
     TimedLaunch t(kIdLayout, st);
@@ -235,7 +231,7 @@ zipnn_status zipnn_histogram(zipnn_dtype dtype, const void* src, uint64_t n, uin
   if (!device_ok()) return ZIPNN_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(hist_out, 0, (size_t)g.n_chunks * n_entropy(dtype) * 256 * 4, st);
-  if (e == cudaSuccess) e = launch_split_hist(src, g, hist_out, nullptr, st);
+  if (e == cudaSuccess) e = launch_split_hist(src, g, hist_out, nullptr, nullptr, PlanDev{}, st);
   return cuda_status(e);
 }
 
@@ -296,7 +292,7 @@ zipnn_status zipnn_plan_create(zipnn_dtype dtype, const void* src, uint64_t n, u
   zipnn_status zs = plan_alloc(dtype, groups, &p);
   if (zs != ZIPNN_OK) return zs;
   cudaError_t e = cudaMemsetAsync(ws, 0, wp.zero_end, st);
-  if (e == cudaSuccess) e = launch_split_hist(src, g, w.hist, nullptr, st);
+  if (e == cudaSuccess) e = launch_split_hist(src, g, w.hist, nullptr, nullptr, PlanDev{}, st);
   if (e == cudaSuccess) {
     if (g.n_chunks <= groups) {
       e = launch_identity_assign(k.assign, k.C, st);

@@ -71,7 +71,8 @@ struct Geo {
 // Workspace carve-up (device pointers). The first group is cleared by every
 // compress call; the rest is fully overwritten before it is read.
 struct Ws {
-  uint32_t* status;     // [0] status, [1] encode ticket, [2] layout ticket
+  uint32_t* status;     // [0] status, [1] encode ticket, [2] layout ticket, [4 + c] chunk c's
+                        // finished histogram blocks
   uint32_t* hist;       // [n_chunks][n_entropy][256]
   uint32_t* nonzero;    // [n_entries]: OR of the stream's symbols
   uint64_t* scan_desc;  // [layout tiles] look-back descriptors

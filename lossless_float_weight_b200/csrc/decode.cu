@@ -292,18 +292,27 @@ __device__ int decode_bf16_staged(StagedSmem& st, const uint16_t* lut, const uin
       if ((j == 0 && start != 0) || start > cap_bits || expect < start || expect > cap_bits) bad = 1;
       br.init(st.bits, bs_words, bad ? 0 : start);
     }
+    // my merge units: unit u = tid + 256p is row u/4 of the batch, values 8(u%4).. of
+    // each round; ubase is its first value in round 0, urem the values its row has
+    // from there on
+    uint32_t ubase[4], urem[4];
+#pragma unroll
+    for (int p = 0; p < 4; p++) {
+      const uint32_t u = tid + p * kDecodeThreads;
+      const uint32_t row = batch + (u >> 2), part = u & 3;
+      const uint32_t rc = row < nsub ? min32(S, m - row * S) : 0;
+      ubase[p] = row * S + part * 8;
+      urem[p] = rc > part * 8 ? rc - part * 8 : 0;
+    }
     for (uint32_t r = 0; r < rounds; r++) {
       // sign/fraction bytes of this round's merge units, requested before the decode
       uint2 smv[4];
       uint32_t uval[4], ucnt[4];
 #pragma unroll
       for (int p = 0; p < 4; p++) {
-        const uint32_t u = tid + p * kDecodeThreads;
-        const uint32_t row = batch + (u >> 2), part = u & 3;
-        const uint32_t rc = row < nsub ? min32(S, m - row * S) : 0;
-        const uint32_t off = r * kRound + part * 8;
-        const uint32_t n = off < rc ? min32(8, rc - off) : 0;
-        uval[p] = row * S + off;
+        const uint32_t off = r * kRound;
+        const uint32_t n = off < urem[p] ? min32(8, urem[p] - off) : 0;
+        uval[p] = ubase[p] + off;
         ucnt[p] = n;
         smv[p] = make_uint2(0, 0);
         if (smp && n == 8) smv[p] = __ldg(reinterpret_cast<const uint2*>(smp + uval[p]));

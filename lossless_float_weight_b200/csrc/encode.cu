@@ -87,6 +87,25 @@ __global__ void __launch_bounds__(kEncodeThreads) k_encode(const uint8_t* __rest
     if (mode == kModeZero) continue;
     const int w = raw_width(DT, s);
     if (mode == kModeRaw && w == 8) {
+      if constexpr (DT == kBF16) {
+        if (cnt == kEncValues) {
+          // two values at a time: the exponent is bits 14..7 of each half, the
+          // sign/fraction byte bits 15 and 6..0
+#pragma unroll
+          for (int q = 0; q < kEncValues / 16; q++) {
+            uint32_t x[4];
+#pragma unroll
+            for (int k = 0; k < 4; k++) {
+              const uint32_t a = raw.w[8 * q + 2 * k], b = raw.w[8 * q + 2 * k + 1];
+              const uint32_t ta = s == 0 ? (a >> 7) & 0x00FF00FFu : (a & 0x007F007Fu) | ((a >> 8) & 0x00800080u);
+              const uint32_t tb = s == 0 ? (b >> 7) & 0x00FF00FFu : (b & 0x007F007Fu) | ((b >> 8) & 0x00800080u);
+              x[k] = __byte_perm(ta, tb, 0x6420);
+            }
+            *reinterpret_cast<uint4*>(out + sm.off[s] + v0 + 16 * q) = make_uint4(x[0], x[1], x[2], x[3]);
+          }
+          continue;
+        }
+      }
 #pragma unroll
       for (int q = 0; q < kEncValues / 16; q++) {
         if (16 * q < cnt) {
@@ -113,26 +132,45 @@ __global__ void __launch_bounds__(kEncodeThreads) k_encode(const uint8_t* __rest
     uint32_t mybits = 0, nw = 0, nfill = 0;
     uint32_t qoff[kEncValues / 16];
     uint64_t acc = 0;
+    if (huff && cnt == kEncValues) {
+      // the common case, without per-value guards; a full word is written (predicated)
+      // whenever 32 bits are pending
 #pragma unroll
-    for (int i = 0; i < kEncValues; i++) {
-      if ((i & 15) == 0) qoff[i >> 4] = mybits;
-      if (i < cnt) {
-        const uint32_t sy = symbol<DT, kEncValues>(raw, s, i);
-        uint32_t l, cv;
-        if (huff) {
-          const uint32_t e = enc[sy];
-          l = e >> 16;
-          cv = e & 0xFFFFu;
-        } else {
-          l = (uint32_t)w;
-          cv = sy;
-        }
+      for (int i = 0; i < kEncValues; i++) {
+        if ((i & 15) == 0) qoff[i >> 4] = mybits;
+        const uint32_t e = enc[symbol<DT, kEncValues>(raw, s, i)];
+        const uint32_t l = e >> 16;
         mybits += l;
-        acc = (acc << l) | cv;
+        acc = (acc << l) | (e & 0xFFFFu);
         nfill += l;
-        if (nfill >= 32) {
-          nfill -= 32;
-          pw[nw++] = (uint32_t)(acc >> nfill);
+        const bool full = nfill >= 32;
+        nfill -= full ? 32u : 0u;
+        const uint32_t word = (uint32_t)(acc >> nfill);
+        if (full) pw[nw] = word;
+        nw += full ? 1u : 0u;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < kEncValues; i++) {
+        if ((i & 15) == 0) qoff[i >> 4] = mybits;
+        if (i < cnt) {
+          const uint32_t sy = symbol<DT, kEncValues>(raw, s, i);
+          uint32_t l, cv;
+          if (huff) {
+            const uint32_t e = enc[sy];
+            l = e >> 16;
+            cv = e & 0xFFFFu;
+          } else {
+            l = (uint32_t)w;
+            cv = sy;
+          }
+          mybits += l;
+          acc = (acc << l) | cv;
+          nfill += l;
+          if (nfill >= 32) {
+            nfill -= 32;
+            pw[nw++] = (uint32_t)(acc >> nfill);
+          }
         }
       }
     }

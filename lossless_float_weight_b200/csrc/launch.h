@@ -22,8 +22,9 @@ class TimedLaunch {
   cudaEvent_t start_ = nullptr, stop_ = nullptr;
 };
 
-cudaError_t launch_split_hist(const void* src, const Geo& g, uint32_t* hist, uint32_t* nonzero, cudaStream_t st);
-cudaError_t launch_build_tables(const Geo& g, const Ws& ws, const PlanDev& plan, cudaStream_t st);
+// Histograms; with ws, the last block of each chunk also builds the chunk's codes.
+cudaError_t launch_split_hist(const void* src, const Geo& g, uint32_t* hist, uint32_t* nonzero, const Ws* ws,
+                              const PlanDev& plan, cudaStream_t st);
 cudaError_t launch_code_lengths(const uint64_t* hist, uint32_t count, uint32_t alphabet_size, uint8_t* lens,
                                 uint32_t* enc, cudaStream_t st);
 cudaError_t launch_layout(const Geo& g, const Ws& ws, const PlanDev& plan, uint8_t* out, cudaStream_t st);

@@ -1,8 +1,9 @@
 // prelude.cu -- the compress steps before encoding:
 //   k_split_hist   : byte-plane split + order-0 histogram per chunk (warp-aggregated
 //                    shared-memory atomics) + all-zero detection per chunk stream;
-//   k_build_tables : per (chunk, entropy stream) code choice: shared group code or a
-//                    local length-limited Huffman code, then HUFF / RAW / ZERO;
+//                    the last block of each chunk then builds the chunk's codes: per
+//                    entropy stream a shared group code or a local length-limited
+//                    Huffman code, then HUFF / RAW / ZERO;
 //   k_layout       : exclusive scan of payload sizes (single-pass decoupled look-back)
 //                    into payload offsets; writes header, chunk table, shared records.
 #include "common.cuh"
@@ -15,61 +16,6 @@ namespace zipnn {
 constexpr int kHistThreads = 256;
 constexpr uint32_t kHistSlice = 32768;  // values of one chunk per histogram block
 
-// THEORY-599 note, "Order-0 only (section III-A b)": the model of a chunk is the count
-// of each symbol. The block keeps one counter per (symbol, lane) in shared memory, so
-// the 32 lanes of a warp always add into 32 different banks (lane l owns column l);
-// warps share the table through shared atomics. The columns are summed at the end.
-template <int DT>
-__global__ void __launch_bounds__(kHistThreads) k_split_hist(const uint8_t* __restrict__ src, Geo g, uint32_t slices,
-                                                             uint32_t* __restrict__ hist, uint32_t* __restrict__ nonzero) {
-  constexpr int NS = n_streams(DT), NE = n_entropy(DT), VB = value_bytes(DT), NW = kHistThreads / 32;
-  constexpr int A0 = alphabet(DT, 0), A1 = NE > 1 ? alphabet(DT, 1) : 0;
-  __shared__ uint32_t sh[(A0 + A1) * 32];
-  const int tid = threadIdx.x, lane = tid & 31;
-  for (int i = tid; i < (A0 + A1) * 32; i += kHistThreads) sh[i] = 0;
-  __syncthreads();
-  const uint32_t c = blockIdx.x / slices, sl = blockIdx.x % slices;
-  const uint64_t clo = (uint64_t)c * g.m0;
-  const uint32_t m = (uint32_t)min64(g.m0, g.n - clo);
-  const uint32_t lo = sl * kHistSlice, hi = min(lo + kHistSlice, m);
-  uint32_t nz[NS];
-#pragma unroll
-  for (int s = 0; s < NS; s++) nz[s] = 0;
-  uint32_t* col0 = sh + lane;
-  uint32_t* col1 = sh + A0 * 32 + lane;
-  constexpr int NV = 64;  // consecutive values per thread per pass, loaded up front
-  for (uint32_t v0 = lo + tid * NV; v0 < hi; v0 += kHistThreads * NV) {
-    const int cnt = (int)min32(NV, hi - v0);
-    RawValues<DT, NV> raw;
-    load_values<DT, NV>(src + (clo + v0) * VB, cnt, raw);
-#pragma unroll
-    for (int i = 0; i < NV; i++) {
-      if (i < cnt) {
-        atomicAdd(col0 + symbol<DT, NV>(raw, 0, i) * 32, 1u);
-        if (NE > 1) atomicAdd(col1 + symbol<DT, NV>(raw, 1, i) * 32, 1u);
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < NV; i++)
-#pragma unroll
-      for (int s = 0; s < NS; s++) nz[s] |= symbol<DT, NV>(raw, s, i);
-  }
-#pragma unroll
-  for (int s = 0; s < NS; s++) {
-    const uint32_t v = __reduce_or_sync(0xFFFFFFFFu, nz[s]);
-    if (nonzero && lane == 0 && v) atomicOr(&nonzero[(uint64_t)c * NS + s], v);
-  }
-  __syncthreads();
-  // column sums: thread b reads its row starting at lane b, so a warp hits 32 banks
-  for (int b = tid; b < A0 + A1; b += kHistThreads) {
-    uint32_t sum = 0;
-#pragma unroll 8
-    for (int l = 0; l < 32; l++) sum += sh[b * 32 + ((l + b) & 31)];
-    const int e = b < A0 ? 0 : 1, sym = b < A0 ? b : b - A0;
-    if (sum) atomicAdd(&hist[((uint64_t)c * NE + e) * 256 + sym], sum);
-  }
-}
-
 // Per (chunk, entropy stream), one block of kHuffWarps warps.
 // With a plan ("NeuralZip: Reusable Setup for Fast Lossless Compression", abstract):
 // a group is eligible when its code has a length for every symbol the chunk uses; the
@@ -78,17 +24,15 @@ __global__ void __launch_bounds__(kHistThreads) k_split_hist(const uint8_t* __re
 // The entry is HUFF when that payload is strictly smaller than RAW, ZERO when every
 // symbol is 0.
 template <int DT>
-__global__ void __launch_bounds__(kHuffWarps * 32) k_build_tables(Geo g, Ws ws, PlanDev plan) {
+__device__ void build_chunk_table(const Geo& g, const Ws& ws, const PlanDev& plan, uint32_t c, uint32_t e,
+                                  HuffBlockSmem& sm) {
   constexpr int NS = n_streams(DT), NE = n_entropy(DT);
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  HuffBlockSmem& sm = *reinterpret_cast<HuffBlockSmem*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint32_t c = blockIdx.x / NE, e = blockIdx.x % NE;
   const uint32_t k = c * NS + e;
   const uint64_t clo = (uint64_t)c * g.m0;
   const uint64_t m = min64(g.m0, g.n - clo);
   const int A = alphabet(DT, e), w = raw_width(DT, e);
-  if (ws.nonzero[k] == 0) {
+  if (__ldcg(ws.nonzero + k) == 0) {
     if (tid == 0) {
       ws.emode[k] = kModeZero;
       ws.ecode[k] = kNoCode;
@@ -97,7 +41,7 @@ __global__ void __launch_bounds__(kHuffWarps * 32) k_build_tables(Geo g, Ws ws, 
     return;
   }
   const uint32_t* h = ws.hist + ((uint64_t)c * NE + e) * 256;
-  sm.f[tid] = tid < A ? h[tid] : 0;
+  sm.f[tid] = tid < A ? __ldcg(h + tid) : 0;
   __syncthreads();
   int group = -1;
   uint64_t bits = 0;
@@ -164,6 +108,79 @@ __global__ void __launch_bounds__(kHuffWarps * 32) k_build_tables(Geo g, Ws ws, 
   }
 }
 
+// THEORY-599 note, "Order-0 only (section III-A b)": the model of a chunk is the count
+// of each symbol. The block keeps one counter per (symbol, lane) in shared memory, so
+// the 32 lanes of a warp always add into 32 different banks (lane l owns column l);
+// warps share the table through shared atomics. The columns are summed at the end.
+template <int DT>
+__global__ void __launch_bounds__(kHistThreads) k_split_hist(const uint8_t* __restrict__ src, Geo g, uint32_t slices,
+                                                             uint32_t* __restrict__ hist, uint32_t* __restrict__ nonzero,
+                                                             Ws ws, PlanDev plan, int build) {
+  constexpr int NS = n_streams(DT), NE = n_entropy(DT), VB = value_bytes(DT);
+  constexpr int A0 = alphabet(DT, 0), A1 = NE > 1 ? alphabet(DT, 1) : 0;
+  extern __shared__ __align__(16) uint8_t smem_raw[];  // histogram columns, then the code builder
+  uint32_t* sh = reinterpret_cast<uint32_t*>(smem_raw);
+  __shared__ int s_last;
+  const int tid = threadIdx.x, lane = tid & 31;
+  for (int i = tid; i < (A0 + A1) * 32; i += kHistThreads) sh[i] = 0;
+  __syncthreads();
+  const uint32_t c = blockIdx.x / slices, sl = blockIdx.x % slices;
+  const uint64_t clo = (uint64_t)c * g.m0;
+  const uint32_t m = (uint32_t)min64(g.m0, g.n - clo);
+  const uint32_t lo = sl * kHistSlice, hi = min(lo + kHistSlice, m);
+  uint32_t nz[NS];
+#pragma unroll
+  for (int s = 0; s < NS; s++) nz[s] = 0;
+  uint32_t* col0 = sh + lane;
+  uint32_t* col1 = sh + A0 * 32 + lane;
+  constexpr int NV = 64;  // consecutive values per thread per pass, loaded up front
+  for (uint32_t v0 = lo + tid * NV; v0 < hi; v0 += kHistThreads * NV) {
+    const int cnt = (int)min32(NV, hi - v0);
+    RawValues<DT, NV> raw;
+    load_values<DT, NV>(src + (clo + v0) * VB, cnt, raw);
+#pragma unroll
+    for (int i = 0; i < NV; i++) {
+      if (i < cnt) {
+        atomicAdd(col0 + symbol<DT, NV>(raw, 0, i) * 32, 1u);
+        if (NE > 1) atomicAdd(col1 + symbol<DT, NV>(raw, 1, i) * 32, 1u);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < NV; i++)
+#pragma unroll
+      for (int s = 0; s < NS; s++) nz[s] |= symbol<DT, NV>(raw, s, i);
+  }
+#pragma unroll
+  for (int s = 0; s < NS; s++) {
+    const uint32_t v = __reduce_or_sync(0xFFFFFFFFu, nz[s]);
+    if (nonzero && lane == 0 && v) atomicOr(&nonzero[(uint64_t)c * NS + s], v);
+  }
+  __syncthreads();
+  // column sums: thread b reads its row starting at lane b, so a warp hits 32 banks
+  for (int b = tid; b < A0 + A1; b += kHistThreads) {
+    uint32_t sum = 0;
+#pragma unroll 8
+    for (int l = 0; l < 32; l++) sum += sh[b * 32 + ((l + b) & 31)];
+    const int e = b < A0 ? 0 : 1, sym = b < A0 ? b : b - A0;
+    if (sum) atomicAdd(&hist[((uint64_t)c * NE + e) * 256 + sym], sum);
+  }
+  if (!build) return;
+  // the last block to finish a chunk builds that chunk's codes (its histogram is then
+  // complete), so the serial part of the code build overlaps other blocks' loads
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(ws.status + 4 + c, 1u) == slices - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  HuffBlockSmem& hs = *reinterpret_cast<HuffBlockSmem*>(smem_raw);
+#pragma unroll
+  for (int e = 0; e < NE; e++) {
+    build_chunk_table<DT>(g, ws, plan, c, (uint32_t)e, hs);
+    __syncthreads();
+  }
+}
+
 // Stand-alone code lengths for `count` histograms (u64 x 256 each); also used by the
 // plan for its group codes. Optionally writes canonical code values.
 __global__ void __launch_bounds__(kHuffWarps * 32) k_code_lengths(const uint64_t* __restrict__ hist, uint32_t alphabet_size,
@@ -202,7 +219,7 @@ __device__ inline uint64_t block_scan_u64(uint64_t v, uint64_t* s_warp, uint64_t
 }
 
 // Layout: payload k (entry order) starts at off_payload + sum of sizes of entries < k.
-// Entropy entries take their mode and size from k_build_tables; raw-plane entries are
+// Entropy entries take their mode and size from the code build; raw-plane entries are
 // ZERO when all their symbols are 0, else RAW.
 template <int DT>
 __global__ void __launch_bounds__(kLayoutThreads) k_layout(Geo g, Ws ws, PlanDev plan, uint8_t* __restrict__ out) {
@@ -307,19 +324,27 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout(Geo g, Ws ws, PlanDev
 // ---------------------------------------------------------------- launchers
 
 template <int DT>
-static cudaError_t split_hist_t(const void* src, const Geo& g, uint32_t* hist, uint32_t* nonzero, cudaStream_t st) {
+static cudaError_t split_hist_t(const void* src, const Geo& g, uint32_t* hist, uint32_t* nonzero, const Ws* ws,
+                                const PlanDev& plan, cudaStream_t st) {
   const uint32_t slices = (uint32_t)ceil_div(g.m0, kHistSlice);
   const uint64_t blocks = (uint64_t)g.n_chunks * slices;
   if (blocks > 0x7FFFFFFFull) return cudaErrorInvalidConfiguration;
-  k_split_hist<DT><<<(uint32_t)blocks, kHistThreads, 0, st>>>(static_cast<const uint8_t*>(src), g, slices, hist, nonzero);
+  constexpr int NE = n_entropy(DT);
+  constexpr size_t cols = (size_t)(alphabet(DT, 0) + (NE > 1 ? alphabet(DT, 1) : 0)) * 32 * 4;
+  const size_t smem = ws ? (sizeof(HuffBlockSmem) > cols ? sizeof(HuffBlockSmem) : cols) : cols;
+  Ws w{};
+  if (ws) w = *ws;
+  k_split_hist<DT><<<(uint32_t)blocks, kHistThreads, smem, st>>>(static_cast<const uint8_t*>(src), g, slices, hist,
+                                                                 nonzero, w, plan, ws ? 1 : 0);
   return cudaGetLastError();
 }
 
-cudaError_t launch_split_hist(const void* src, const Geo& g, uint32_t* hist, uint32_t* nonzero, cudaStream_t st) {
+cudaError_t launch_split_hist(const void* src, const Geo& g, uint32_t* hist, uint32_t* nonzero, const Ws* ws,
+                              const PlanDev& plan, cudaStream_t st) {
   switch (g.dt) {
-    case kBF16: return split_hist_t<kBF16>(src, g, hist, nonzero, st);
-    case kFP32: return split_hist_t<kFP32>(src, g, hist, nonzero, st);
-    default: return split_hist_t<kFP8>(src, g, hist, nonzero, st);
+    case kBF16: return split_hist_t<kBF16>(src, g, hist, nonzero, ws, plan, st);
+    case kFP32: return split_hist_t<kFP32>(src, g, hist, nonzero, ws, plan, st);
+    default: return split_hist_t<kFP8>(src, g, hist, nonzero, ws, plan, st);
   }
 }
 
@@ -334,23 +359,6 @@ static cudaError_t allow_smem(K kernel, size_t bytes, int slot) {
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e == cudaSuccess && dev >= 0 && dev < 128) done[slot][dev] = 1;
   return e;
-}
-
-template <int DT>
-static cudaError_t tables_t(const Geo& g, const Ws& ws, const PlanDev& plan, cudaStream_t st) {
-  const size_t smem = sizeof(HuffBlockSmem);
-  cudaError_t e = allow_smem(k_build_tables<DT>, smem, DT);
-  if (e != cudaSuccess) return e;
-  k_build_tables<DT><<<g.n_chunks * n_entropy(DT), kHuffWarps * 32, smem, st>>>(g, ws, plan);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_build_tables(const Geo& g, const Ws& ws, const PlanDev& plan, cudaStream_t st) {
-  switch (g.dt) {
-    case kBF16: return tables_t<kBF16>(g, ws, plan, st);
-    case kFP32: return tables_t<kFP32>(g, ws, plan, st);
-    default: return tables_t<kFP8>(g, ws, plan, st);
-  }
 }
 
 cudaError_t launch_code_lengths(const uint64_t* hist, uint32_t count, uint32_t alphabet_size, uint8_t* lens,
