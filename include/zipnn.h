@@ -161,6 +161,23 @@ zipnn_status zipnn_plan_assignment(const zipnn_plan_t* plan, uint32_t* host_buf,
 
 void zipnn_plan_destroy(zipnn_plan_t* plan);
 
+/* Compress without allocating (the pages have no counterpart of this call). For callers
+ * that cannot allocate device memory: code that runs while a CUDA stream capture is
+ * active (cudaMalloc is not allowed then), code whose memory is owned by a framework
+ * allocator it cannot reach from C, and latency-critical paths that cannot afford the
+ * device synchronisation an allocation implies. It behaves as zipnn_compress without a
+ * plan, but its workspace is a file-scope device array of ZIPNN_NOALLOC_SCRATCH_BYTES
+ * (8 MiB) that every GPU loading the library holds until the process exits; tensors
+ * whose zipnn_workspace_bytes exceed it are rejected with ZIPNN_ERR_UNSUPPORTED before
+ * anything is launched. The caller still passes input and output. The first call on a
+ * device looks up the array's device address with that device current, so make the
+ * first call before any stream capture. All calls on a device share the array and it
+ * keeps the previous call's contents (each call clears what must start at zero): calls
+ * that may overlap on the GPU race, so issue them on one stream or order them. */
+#define ZIPNN_NOALLOC_SCRATCH_BYTES (8u << 20)
+zipnn_status zipnn_compress_noalloc(zipnn_dtype dtype, const void* src, uint64_t n, uint32_t chunk_bytes, void* out,
+                                    size_t out_cap, zipnn_stream_t stream);
+
 /* Kernel timing, a measurement aid (off by default; not a step of the codec). While
  * enabled, every kernel the library launches is bracketed by two CUDA events on its
  * stream. zipnn_timing_collect waits for the recorded events and writes, for kernel

@@ -55,13 +55,15 @@ zipnn_timing_enable = _sig("zipnn_timing_enable", _i, _i)
 zipnn_timing_collect = _sig("zipnn_timing_collect", _i, _vp, _vp, _u32)
 zipnn_kernel_count = _sig("zipnn_kernel_count", _u32)
 zipnn_kernel_name = _sig("zipnn_kernel_name", ctypes.c_char_p, _u32)
+zipnn_compress_noalloc = _sig("zipnn_compress_noalloc", _i, _i, _vp, _u64, _u32, _vp, _sz, _vp)
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 C_ABI_NAMES = [
     "zipnn_max_compressed_bytes", "zipnn_workspace_bytes", "zipnn_compress", "zipnn_compress_ex",
     "zipnn_decompress", "zipnn_compressed_size", "zipnn_get_status", "zipnn_histogram", "zipnn_code_lengths",
     "zipnn_plan_create", "zipnn_plan_export", "zipnn_plan_import", "zipnn_plan_assignment", "zipnn_plan_destroy",
     "zipnn_status_string", "zipnn_timing_enable", "zipnn_timing_collect", "zipnn_kernel_count",
-    "zipnn_kernel_name",
+    "zipnn_kernel_name", "zipnn_compress_noalloc",
 ]
 
 
