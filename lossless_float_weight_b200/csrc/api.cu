@@ -174,7 +174,8 @@ zipnn_status zipnn_compress_ex(zipnn_dtype dtype, const void* src, uint64_t n, u
   }
   if (e == cudaSuccess) {
     TimedLaunch t(kIdEncode, st);
-    e = launch_encode(src, g, w, static_cast<uint8_t*>(out), st);
+    e = cluster_encode_applies(g) ? launch_encode_bf16_cluster(src, g, w, static_cast<uint8_t*>(out), st)
+                                  : launch_encode(src, g, w, static_cast<uint8_t*>(out), st);
   }
   return cuda_status(e);
 }

@@ -185,4 +185,80 @@ __device__ inline void warp_canonical(const uint8_t* lens, uint32_t* enc) {
   }
 }
 
+// Code choice for one (chunk, entropy stream) whose histogram is in sm.f[0..A) and
+// which has at least one non-zero symbol; all threads of the block (kHuffWarps warps).
+// With a plan ("NeuralZip: Reusable Setup for Fast Lossless Compression", abstract): a
+// group is eligible when its code has a length for every symbol the chunk uses; the
+// eligible group with the fewest coded bits wins (ties to the smaller group). Without
+// an eligible group, or without a plan, the chunk gets its own limited Huffman code.
+// The payload is HUFF when strictly smaller than RAW. Thread 0 writes *mode, *code and
+// *size; enc_out receives len << 16 | code for every symbol when the result is HUFF.
+__device__ inline void decide_code(HuffBlockSmem& sm, int A, int w, uint32_t rec, uint64_t m, uint32_t S,
+                                   const PlanDev& plan, uint32_t e, uint32_t* enc_out, uint32_t* mode,
+                                   uint32_t* code, uint64_t* size) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int group = -1;
+  uint64_t bits = 0;
+  if (plan.groups) {
+    for (uint32_t gi = warp; gi < plan.groups; gi += kHuffWarps) {
+      const uint8_t* lg = plan.lens + ((uint64_t)e * plan.groups + gi) * 256;
+      uint64_t cost = 0;
+      bool ok = true;
+      for (int s = lane; s < A; s += 32) {
+        const uint64_t f = sm.f[s];
+        if (f) {
+          ok = ok && lg[s] != 0;
+          cost += f * lg[s];
+        }
+      }
+      for (int o = 16; o; o >>= 1) cost += __shfl_xor_sync(0xFFFFFFFFu, cost, o);
+      const bool all = __all_sync(0xFFFFFFFFu, ok);
+      if (lane == 0) {
+        sm.cost[gi] = cost;
+        sm.elig[gi] = all;
+      }
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int best = -1;
+      for (uint32_t gi = 0; gi < plan.groups; gi++)
+        if (sm.elig[gi] && (best < 0 || sm.cost[gi] < sm.cost[best])) best = (int)gi;
+      sm.pick = best;
+    }
+    __syncthreads();
+    group = sm.pick;
+    if (group >= 0) bits = sm.cost[group];
+  }
+  const uint8_t* lens = nullptr;
+  if (group < 0) {
+    const int wbest = block_limited_lengths(sm, A);
+    lens = sm.w[wbest].lens;
+    uint64_t part = tid < A ? sm.f[tid] * lens[tid] : 0;
+    for (int o = 16; o; o >>= 1) part += __shfl_xor_sync(0xFFFFFFFFu, part, o);
+    if (lane == 0) sm.red[warp] = part;
+    __syncthreads();
+    bits = 0;
+    for (int i = 0; i < kHuffWarps; i++) bits += sm.red[i];
+  }
+  const uint64_t nsub = ceil_div(m, S);
+  const uint64_t p_huff = (group < 0 ? rec : 0) + round16(4 * nsub) + round16(ceil_div(bits, 8));
+  const uint64_t p_raw = raw_payload(m, w);
+  if (p_huff < p_raw) {
+    if (group >= 0) {
+      enc_out[tid] = plan.enc[((uint64_t)e * plan.groups + group) * 256 + tid];
+    } else if (warp == 0) {
+      warp_canonical(lens, enc_out);
+    }
+    if (tid == 0) {
+      *mode = kModeHuff;
+      *code = group >= 0 ? e * plan.groups + (uint32_t)group : kNoCode;
+      *size = p_huff;
+    }
+  } else if (tid == 0) {
+    *mode = kModeRaw;
+    *code = kNoCode;
+    *size = p_raw;
+  }
+}
+
 }  // namespace zipnn

@@ -16,18 +16,13 @@ namespace zipnn {
 constexpr int kHistThreads = 256;
 constexpr uint32_t kHistSlice = 32768;  // values of one chunk per histogram block
 
-// Per (chunk, entropy stream), one block of kHuffWarps warps.
-// With a plan ("NeuralZip: Reusable Setup for Fast Lossless Compression", abstract):
-// a group is eligible when its code has a length for every symbol the chunk uses; the
-// eligible group with the fewest coded bits wins (ties to the smaller group). Without
-// an eligible group, or without a plan, the chunk gets its own limited Huffman code.
-// The entry is HUFF when that payload is strictly smaller than RAW, ZERO when every
-// symbol is 0.
+// Per (chunk, entropy stream), one block of kHuffWarps warps: ZERO when every symbol is
+// 0, else the code choice of decide_code.
 template <int DT>
 __device__ void build_chunk_table(const Geo& g, const Ws& ws, const PlanDev& plan, uint32_t c, uint32_t e,
                                   HuffBlockSmem& sm) {
   constexpr int NS = n_streams(DT), NE = n_entropy(DT);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   const uint32_t k = c * NS + e;
   const uint64_t clo = (uint64_t)c * g.m0;
   const uint64_t m = min64(g.m0, g.n - clo);
@@ -43,69 +38,8 @@ __device__ void build_chunk_table(const Geo& g, const Ws& ws, const PlanDev& pla
   const uint32_t* h = ws.hist + ((uint64_t)c * NE + e) * 256;
   sm.f[tid] = tid < A ? __ldcg(h + tid) : 0;
   __syncthreads();
-  int group = -1;
-  uint64_t bits = 0;
-  if (plan.groups) {
-    for (uint32_t gi = warp; gi < plan.groups; gi += kHuffWarps) {
-      const uint8_t* lg = plan.lens + ((uint64_t)e * plan.groups + gi) * 256;
-      uint64_t cost = 0;
-      bool ok = true;
-      for (int s = lane; s < A; s += 32) {
-        const uint64_t f = sm.f[s];
-        if (f) {
-          ok = ok && lg[s] != 0;
-          cost += f * lg[s];
-        }
-      }
-      for (int o = 16; o; o >>= 1) cost += __shfl_xor_sync(0xFFFFFFFFu, cost, o);
-      const bool all = __all_sync(0xFFFFFFFFu, ok);
-      if (lane == 0) {
-        sm.cost[gi] = cost;
-        sm.elig[gi] = all;
-      }
-    }
-    __syncthreads();
-    if (tid == 0) {
-      int best = -1;
-      for (uint32_t gi = 0; gi < plan.groups; gi++)
-        if (sm.elig[gi] && (best < 0 || sm.cost[gi] < sm.cost[best])) best = (int)gi;
-      sm.pick = best;
-    }
-    __syncthreads();
-    group = sm.pick;
-    if (group >= 0) bits = sm.cost[group];
-  }
-  const uint8_t* lens = nullptr;
-  if (group < 0) {
-    const int wbest = block_limited_lengths(sm, A);
-    lens = sm.w[wbest].lens;
-    uint64_t part = tid < A ? sm.f[tid] * lens[tid] : 0;
-    for (int o = 16; o; o >>= 1) part += __shfl_xor_sync(0xFFFFFFFFu, part, o);
-    if (lane == 0) sm.red[warp] = part;
-    __syncthreads();
-    bits = 0;
-    for (int i = 0; i < kHuffWarps; i++) bits += sm.red[i];
-  }
-  const uint64_t nsub = ceil_div(m, g.S);
-  const uint64_t p_huff = (group < 0 ? record_bytes(DT, e) : 0) + round16(4 * nsub) + round16(ceil_div(bits, 8));
-  const uint64_t p_raw = raw_payload(m, w);
-  uint32_t* enc = ws.enc + ((uint64_t)c * NE + e) * 256;
-  if (p_huff < p_raw) {
-    if (group >= 0) {
-      enc[tid] = plan.enc[((uint64_t)e * plan.groups + group) * 256 + tid];
-    } else if (warp == 0) {
-      warp_canonical(lens, enc);
-    }
-    if (tid == 0) {
-      ws.emode[k] = kModeHuff;
-      ws.ecode[k] = group >= 0 ? e * plan.groups + (uint32_t)group : kNoCode;
-      ws.esize[k] = p_huff;
-    }
-  } else if (tid == 0) {
-    ws.emode[k] = kModeRaw;
-    ws.ecode[k] = kNoCode;
-    ws.esize[k] = p_raw;
-  }
+  decide_code(sm, A, w, record_bytes(DT, e), m, g.S, plan, e, ws.enc + ((uint64_t)c * NE + e) * 256, ws.emode + k,
+              ws.ecode + k, ws.esize + k);
 }
 
 // THEORY-599 note, "Order-0 only (section III-A b)": the model of a chunk is the count
