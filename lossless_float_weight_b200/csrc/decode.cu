@@ -4,8 +4,14 @@
 // its chunk's table entries; every read is bounded by the container size, so a damaged
 // container yields ZIPNN_ERR_CORRUPT and never an out-of-bounds access.
 // For each HUFF stream the block rebuilds the canonical code from its 4-bit lengths
-// and fills a 4096-entry lookup table in shared memory (12-bit window -> symbol,
-// length). Each thread then decodes whole sub-blocks of S symbols, starting at the bit
+// and fills a 4096-entry lookup table in shared memory. An entry of the table, indexed
+// by the next 12 bits of the stream, holds the first code's symbol and length and,
+// when the second code also ends inside those 12 bits, that symbol and the two codes'
+// total length too, so the BF16 paths take two exponents per lookup (the window holds
+// two whole codes for almost every pair of a weight tensor's exponents). Layout:
+//   bits 0..3 first length | 4..7 total length of two codes, 0 if the window holds one
+//   bit 15 no code starts with these bits | 16..23 first symbol | 24..31 second symbol
+// Each thread then decodes whole sub-blocks of S symbols, starting at the bit
 // offset idx[j], merges the streams back into BF16/FP32/FP8 words and writes them to
 // HBM with 16-byte stores: no intermediate plane is materialised. A sub-block must end
 // exactly where the next one starts.
@@ -18,6 +24,8 @@ namespace zipnn {
 
 constexpr int kDecodeThreads = 256;
 constexpr uint32_t kLutInvalid = 0x8000u;
+
+__device__ __forceinline__ uint32_t lut_symbol(uint32_t e) { return (e >> 16) & 0xFFu; }
 
 // Big-endian-within-word bit reader over 32-bit words [0, end); words past `end`
 // read as zero. buf holds nb valid bits, most significant first; the next two words
@@ -58,17 +66,42 @@ struct BitReader {
     nb -= width;
     return v;
   }
-  __device__ __forceinline__ uint32_t huff(const uint16_t* lut, uint32_t& acc) {
+  __device__ __forceinline__ uint32_t huff(const uint32_t* lut, uint32_t& acc) {
     const uint32_t e = lut[buf >> 52];
     const uint32_t l = e & 15u;
     buf <<= l;
     nb -= (int)l;
     acc |= e;
-    return (e >> 4) & 0xFFu;
+    return lut_symbol(e);
   }
   // absolute index of the next unread bit
   __device__ __forceinline__ uint64_t position() const { return (uint64_t)(pos - 2) * 32 - (uint64_t)nb; }
 };
+
+// Two symbols from either bit reader, returned in bits 16..31 (the first in 16..23).
+// Needs at least 12 valid bits on entry and leaves at least 0; when the window holds
+// only one whole code the reader refills once between the two lookups.
+template <class Reader>
+__device__ __forceinline__ uint32_t huff_pair(Reader& br, const uint32_t* lut, uint32_t& acc) {
+  const uint32_t e = lut[br.buf >> 52];
+  acc |= e;
+  const uint32_t lp = (e >> 4) & 15u;
+  if (lp) {
+    br.buf <<= lp;
+    br.nb -= (int)lp;
+    return e;
+  }
+  const uint32_t l0 = e & 15u;
+  br.buf <<= l0;
+  br.nb -= (int)l0;
+  br.refill();
+  const uint32_t e2 = lut[br.buf >> 52];
+  acc |= e2;
+  const uint32_t l1 = e2 & 15u;
+  br.buf <<= l1;
+  br.nb -= (int)l1;
+  return (e & 0x00FF0000u) | ((e2 & 0x00FF0000u) << 8);
+}
 
 enum Kind : int { kKZero = 0, kKBytes = 1, kKBits = 2, kKHuff = 3 };
 
@@ -76,7 +109,7 @@ struct StreamState {
   int kind, width;
   const uint8_t* bytes;  // kKBytes: this sub-block's first byte
   BitReader br;
-  const uint16_t* lut;
+  const uint32_t* lut;
   uint32_t acc;
 };
 
@@ -134,9 +167,9 @@ __device__ __forceinline__ void next_symbols(StreamState& st, uint32_t (&o)[GV],
 // of every chunk of a trained or Gaussian checkpoint. 16 values per step; the
 // sign/fraction bytes of the next step are requested one step ahead.
 template <bool SM_ZERO>
-__device__ __forceinline__ int decode_bf16_fast(const uint8_t* __restrict__ in, const uint16_t* lut, const uint8_t* smp,
-                                                const uint32_t* bs, uint32_t bs_words, uint64_t start, uint64_t expect,
-                                                bool exact, uint32_t count, uint8_t* __restrict__ dst) {
+__device__ __forceinline__ int decode_bf16_fast(const uint32_t* lut, const uint8_t* smp, const uint32_t* bs,
+                                                uint32_t bs_words, uint64_t start, uint64_t expect, bool exact,
+                                                uint32_t count, uint8_t* __restrict__ dst) {
   BitReader br;
   br.init(bs, bs_words, start);
   uint32_t acc = 0;
@@ -150,12 +183,12 @@ __device__ __forceinline__ int decode_bf16_fast(const uint8_t* __restrict__ in, 
     if (full > 3) nx3 = __ldg(sp + 3);
   }
   for (uint32_t gi = 0; gi < full; gi++) {
-    uint32_t ex[16];
+    uint32_t pr[8];  // exponent pairs in bits 16..31
 #pragma unroll
-    for (int i = 0; i < 16; i += 2) {
+    for (int i = 0; i < 8; i += 2) {
       br.refill();
-      ex[i] = br.huff(lut, acc);
-      ex[i + 1] = br.huff(lut, acc);
+      pr[i] = huff_pair(br, lut, acc);
+      pr[i + 1] = huff_pair(br, lut, acc);
     }
     const uint32_t x[4] = {cur.x, cur.y, cur.z, cur.w};
     if (!SM_ZERO) {
@@ -168,7 +201,7 @@ __device__ __forceinline__ int decode_bf16_fast(const uint8_t* __restrict__ in, 
 #pragma unroll
     for (int q = 0; q < 8; q++) {
       const uint32_t t = SM_ZERO ? 0u : __byte_perm(x[q >> 1], 0, (q & 1) ? 0x4342 : 0x4140);
-      o[q] = (t & 0x007F007Fu) | ((t & 0x00800080u) << 8) | (ex[2 * q] << 7) | (ex[2 * q + 1] << 23);
+      o[q] = (t & 0x007F007Fu) | ((t & 0x00800080u) << 8) | (__byte_perm(pr[q], 0, 0x4342) << 7);
     }
     uint4* d = reinterpret_cast<uint4*>(dst + (uint64_t)gi * 32);
     d[0] = make_uint4(o[0], o[1], o[2], o[3]);
@@ -188,18 +221,20 @@ __device__ __forceinline__ int decode_bf16_fast(const uint8_t* __restrict__ in, 
 // For a BF16 chunk whose exponent stream is HUFF and whose bitstream fits a 48 KB
 // window, the whole bitstream is brought into shared memory by one TMA bulk copy
 // (cp.async.bulk, completion on an mbarrier) while the block builds its lookup table.
-// Then, in rounds, every thread decodes the next 32 exponents of its sub-block into a
-// padded shared buffer (rows of 36 bytes: conflict-free), and the block merges them
-// with the sign/fraction bytes: those are loaded as whole 32-byte sectors one round
-// ahead of use, and the merged words leave as whole 64-byte row segments.
+// Then, in rounds, every thread decodes the next 32 exponents of its sub-block into
+// its row of a shared buffer, and the block merges the rows with the sign/fraction
+// bytes: those are loaded as whole 32-byte sectors one round ahead of use, and the
+// merged words leave as whole 64-byte row segments. Word k of row r sits at
+// 8r + (k ^ (r / 4 mod 8)): the row-per-thread stores and the unit-per-thread loads
+// of the merge both touch 32 distinct banks, with no padding.
 constexpr uint32_t kWindowBytes = 48 * 1024;
-constexpr int kRound = 32;
-constexpr int kExStride = kRound + 4;
+constexpr int kRound = 32;  // exponents of a sub-block decoded per round
+constexpr int kRowWords = kRound / 4;
 constexpr uint32_t kWaitLimit = 1u << 26;
 
 struct StagedSmem {
   uint32_t bits[kWindowBytes / 4];
-  uint8_t ex[kDecodeThreads * kExStride];
+  uint32_t ex[kDecodeThreads * kRowWords];
   uint64_t bar;
 };
 
@@ -257,27 +292,32 @@ struct SmemBitReader {
       q = ld(pos++);
     }
   }
-  __device__ __forceinline__ uint32_t huff(const uint16_t* lut, uint32_t& acc) {
+  __device__ __forceinline__ uint32_t huff(const uint32_t* lut, uint32_t& acc) {
     const uint32_t e = lut[buf >> 52];
     const uint32_t l = e & 15u;
     buf <<= l;
     nb -= (int)l;
     acc |= e;
-    return (e >> 4) & 0xFFu;
+    return lut_symbol(e);
   }
   __device__ __forceinline__ uint64_t position() const { return (uint64_t)(pos - 1) * 32 - (uint64_t)nb; }
 };
 
-// One chunk, all threads of the block. smp: the chunk's sign/fraction payload (RAW) or
-// nullptr (ZERO); outc: the chunk's first output value. Returns nonzero if the stream
-// is inconsistent.
-__device__ int decode_bf16_staged(StagedSmem& st, const uint16_t* lut, const uint32_t* __restrict__ idx,
+__device__ __forceinline__ uint32_t ex_word(uint32_t row, uint32_t k) {
+  return row * kRowWords + (k ^ ((row >> 2) & (kRowWords - 1)));
+}
+
+// One chunk, all threads of the block; one sub-block per thread and batch. smp: the
+// chunk's sign/fraction payload (RAW) or nullptr (ZERO); outc: the chunk's first
+// output value. Returns nonzero if the stream is inconsistent.
+__device__ int decode_bf16_staged(StagedSmem& st, const uint32_t* lut, const uint32_t* __restrict__ idx,
                                   uint32_t bs_words, const uint8_t* __restrict__ smp, uint32_t m, uint32_t S,
                                   uint32_t nsub, uint8_t* __restrict__ outc) {
   const int tid = threadIdx.x;
   int bad = 0;
   const uint64_t cap_bits = (uint64_t)bs_words * 32;
   const uint32_t rounds = (S + kRound - 1) / kRound;
+  uint8_t* exb = reinterpret_cast<uint8_t*>(st.ex);
   for (uint32_t batch = 0; batch < nsub; batch += kDecodeThreads) {
     const uint32_t j = batch + tid;
     const uint32_t count = j < nsub ? min32(S, m - j * S) : 0;
@@ -292,8 +332,8 @@ __device__ int decode_bf16_staged(StagedSmem& st, const uint16_t* lut, const uin
       if ((j == 0 && start != 0) || start > cap_bits || expect < start || expect > cap_bits) bad = 1;
       br.init(st.bits, bs_words, bad ? 0 : start);
     }
-    // my merge units: unit u = tid + 256p is row u/4 of the batch, values 8(u%4).. of
-    // each round; ubase is its first value in round 0, urem the values its row has
+    // my merge units: unit u = tid + 256p is part u % 4 (values 8(u % 4)..) of row u / 4
+    // of the batch; ubase is its first value in round 0, urem the values its row has
     // from there on
     uint32_t ubase[4], urem[4];
 #pragma unroll
@@ -326,26 +366,22 @@ __device__ int decode_bf16_staged(StagedSmem& st, const uint16_t* lut, const uin
           smv[p] = make_uint2(lo, hi);
         }
       }
-      // decode up to 32 exponents of my sub-block
+      // decode up to 32 exponents of my sub-block, two per lookup
       const uint32_t base = r * kRound;
       if (base < count) {
-        uint32_t* row = reinterpret_cast<uint32_t*>(st.ex + tid * kExStride);
         if (base + kRound <= count) {
 #pragma unroll
-          for (int k = 0; k < kRound / 4; k++) {
+          for (int k = 0; k < kRowWords; k++) {
             br.refill();
-            const uint32_t e0 = br.huff(lut, acc);
-            const uint32_t e1 = br.huff(lut, acc);
-            br.refill();
-            const uint32_t e2 = br.huff(lut, acc);
-            const uint32_t e3 = br.huff(lut, acc);
-            row[k] = e0 | (e1 << 8) | (e2 << 16) | (e3 << 24);
+            const uint32_t a = huff_pair(br, lut, acc);
+            const uint32_t b = huff_pair(br, lut, acc);
+            st.ex[ex_word(tid, k)] = __byte_perm(a, b, 0x7632);
           }
         } else {
           const uint32_t n = count - base;
           for (uint32_t k = 0; k < n; k++) {
             br.refill();
-            st.ex[tid * kExStride + k] = (uint8_t)br.huff(lut, acc);
+            exb[ex_word(tid, k >> 2) * 4 + (k & 3)] = (uint8_t)br.huff(lut, acc);
           }
         }
       }
@@ -355,11 +391,9 @@ __device__ int decode_bf16_staged(StagedSmem& st, const uint16_t* lut, const uin
       for (int p = 0; p < 4; p++) {
         const uint32_t u = tid + p * kDecodeThreads;
         if (!ucnt[p]) continue;
-        const uint8_t* exr = st.ex + (u >> 2) * kExStride + (u & 3) * 8;
-        const uint32_t ea = *reinterpret_cast<const uint32_t*>(exr);
-        const uint32_t eb = *reinterpret_cast<const uint32_t*>(exr + 4);
+        const uint32_t row = u >> 2, part = u & 3;
+        const uint32_t es[2] = {st.ex[ex_word(row, 2 * part)], st.ex[ex_word(row, 2 * part + 1)]};
         const uint32_t xs[2] = {smv[p].x, smv[p].y};
-        const uint32_t es[2] = {ea, eb};
         uint32_t o[4];
 #pragma unroll
         for (int q = 0; q < 4; q++) {
@@ -371,8 +405,9 @@ __device__ int decode_bf16_staged(StagedSmem& st, const uint16_t* lut, const uin
         if (ucnt[p] == 8) {
           *reinterpret_cast<uint4*>(d) = make_uint4(o[0], o[1], o[2], o[3]);
         } else {
-          for (uint32_t i = 0; i < ucnt[p]; i++)
-            reinterpret_cast<uint16_t*>(d)[i] = (uint16_t)(o[i >> 1] >> (16 * (i & 1)));
+#pragma unroll
+          for (uint32_t i = 0; i < 8; i++)
+            if (i < ucnt[p]) reinterpret_cast<uint16_t*>(d)[i] = (uint16_t)(o[i >> 1] >> (16 * (i & 1)));
         }
       }
       __syncthreads();
@@ -387,7 +422,7 @@ __device__ int decode_bf16_staged(StagedSmem& st, const uint16_t* lut, const uin
 
 template <int DT>
 struct DecodeSmem {
-  uint16_t lut[n_entropy(DT)][4096];
+  uint32_t lut[n_entropy(DT)][4096];
   uint8_t lens[n_entropy(DT)][256];
   uint32_t enc[n_entropy(DT)][256];
   uint8_t sorted[n_entropy(DT)][256];
@@ -400,6 +435,9 @@ struct DecodeSmem {
   uint32_t S, G;
   int bad, staged;
 };
+
+// three BF16 decode blocks share an SM: 228 KB of shared memory, 1 KB reserved per block
+static_assert(sizeof(StagedSmem) + sizeof(DecodeSmem<kBF16>) + 1024 <= 233472 / 3, "BF16 decode: 3 blocks per SM");
 
 template <int DT>
 __global__ void __launch_bounds__(kDecodeThreads, DT == kBF16 ? 3 : 1) k_decode(const uint8_t* __restrict__ in, uint64_t in_bytes, Geo g,
@@ -594,12 +632,30 @@ __global__ void __launch_bounds__(kDecodeThreads, DT == kBF16 ? 3 : 1) k_decode(
 #pragma unroll
         for (int j = 1; j < kLmax; j++) l += x >= sm.limit[e][j];
         const uint32_t sym = sm.sorted[e][sm.offset[e][l] + (x >> (kLmax - l)) - sm.first[e][l]];
-        entry = (sym << 4) | l;
+        entry = (sym << 16) | l;
       }
-      sm.lut[e][x] = (uint16_t)entry;
+      sm.lut[e][x] = entry;
     }
   }
   __syncthreads();
+  if constexpr (DT == kBF16) {
+    // second code of each window: the entry of the window shifted by the first length
+    // decides it when that code ends inside the 12 known bits (a prefix code's entry
+    // does not depend on the bits after the code). Updating in place is safe: the
+    // fields read here (first length, first symbol, invalid flag) never change.
+    if (sm.mode[0] == kModeHuff) {
+      for (uint32_t x = tid; x < 4096; x += kDecodeThreads) {
+        const uint32_t e0 = sm.lut[0][x];
+        if (e0 & kLutInvalid) continue;
+        const uint32_t l0 = e0 & 15u;
+        const uint32_t e1 = sm.lut[0][(x << l0) & 4095u];
+        const uint32_t l1 = e1 & 15u;
+        if (!(e1 & kLutInvalid) && l0 + l1 <= (uint32_t)kLmax)
+          sm.lut[0][x] = e0 | ((l0 + l1) << 4) | ((e1 & 0x00FF0000u) << 8);
+      }
+      __syncthreads();
+    }
+  }
 
   const uint64_t nsub = ceil_div(m, S);
   if constexpr (DT == kBF16) {
@@ -641,11 +697,11 @@ __global__ void __launch_bounds__(kDecodeThreads, DT == kBF16 ? 3 : 1) k_decode(
         const uint32_t* bs = reinterpret_cast<const uint32_t*>(in + bs_off);
         uint8_t* dst = out + (clo + sb_lo) * VB;
         if (sm.mode[1] == kModeZero)
-          bad |= decode_bf16_fast<true>(in, sm.lut[0], nullptr, bs, (uint32_t)(cap_bits / 32), bad ? 0 : start, expect,
-                                        exact, count, dst);
+          bad |= decode_bf16_fast<true>(sm.lut[0], nullptr, bs, (uint32_t)(cap_bits / 32), bad ? 0 : start,
+                                                   expect, exact, count, dst);
         else
-          bad |= decode_bf16_fast<false>(in, sm.lut[0], in + sm.off[1] + sb_lo, bs, (uint32_t)(cap_bits / 32),
-                                         bad ? 0 : start, expect, exact, count, dst);
+          bad |= decode_bf16_fast<false>(sm.lut[0], in + sm.off[1] + sb_lo, bs, (uint32_t)(cap_bits / 32),
+                                                    bad ? 0 : start, expect, exact, count, dst);
         if (bad) set_status(status, kStCorrupt);
         continue;
       }
@@ -724,7 +780,9 @@ __global__ void __launch_bounds__(kDecodeThreads, DT == kBF16 ? 3 : 1) k_decode(
       uint32_t sy[NS][GV];
 #pragma unroll
       for (int s = 0; s < NS; s++) next_symbols<GV, false>(st[s], sy[s], (int)rem, full * GV);
-      for (uint32_t i = 0; i < rem; i++) {
+#pragma unroll
+      for (uint32_t i = 0; i < (uint32_t)GV; i++) {
+        if (i >= rem) break;
         const uint32_t v = merge_value<DT>(sy[0][i], sy[1][i], NS > 2 ? sy[NS > 2 ? 2 : 0][i] : 0,
                                            NS > 3 ? sy[NS > 3 ? 3 : 0][i] : 0);
         uint8_t* p = dst + (uint64_t)(full * GV + i) * VB;

@@ -135,15 +135,23 @@ __device__ inline int block_limited_lengths(HuffBlockSmem& sm, int A) {
 }
 
 // One warp: canonical code values (RFC 1951, 3.2.2) for lens[0..256); writes
-// enc[s] = len << 16 | code (0 for absent symbols).
+// enc[s] = len << 16 | code (0 for absent symbols). Lane k holds symbols 8k..8k+7.
+// Lengths are visited in increasing order; the first code of a length follows from
+// the previous length's first code and count, and within a length the codes go to
+// the symbols in increasing order (a scan over lanes gives each lane its offset).
+// Every per-length quantity lives in registers: no local-memory arrays.
 __device__ inline void warp_canonical(const uint8_t* lens, uint32_t* enc) {
   const int lane = threadIdx.x & 31;
-  uint32_t L[8];
+  uint32_t L[8], v[8];
 #pragma unroll
-  for (int i = 0; i < 8; i++) L[i] = lens[lane * 8 + i];
-  uint32_t excl[kLmax + 1], total[kLmax + 1];
+  for (int i = 0; i < 8; i++) {
+    L[i] = lens[lane * 8 + i];
+    v[i] = 0;
+  }
+  uint32_t first = 0, prev_count = 0;
 #pragma unroll
   for (int l = 1; l <= kLmax; l++) {
+    first = (first + prev_count) << 1;
     uint32_t c = 0;
 #pragma unroll
     for (int i = 0; i < 8; i++) c += L[i] == (uint32_t)l;
@@ -153,36 +161,14 @@ __device__ inline void warp_canonical(const uint8_t* lens, uint32_t* enc) {
       const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
       if (lane >= o) x += y;
     }
-    excl[l] = x - c;
-    total[l] = __shfl_sync(0xFFFFFFFFu, x, 31);
-  }
-  uint32_t next[kLmax + 1];
-  uint32_t code = 0;
-  next[0] = 0;
-  total[0] = 0;
+    uint32_t next = first + x - c;
 #pragma unroll
-  for (int l = 1; l <= kLmax; l++) {
-    code = (code + total[l - 1]) << 1;
-    next[l] = code;
+    for (int i = 0; i < 8; i++)
+      if (L[i] == (uint32_t)l) v[i] = ((uint32_t)l << 16) | next++;
+    prev_count = __shfl_sync(0xFFFFFFFFu, x, 31);
   }
 #pragma unroll
-  for (int i = 0; i < 8; i++) {
-    uint32_t v = 0;
-    if (L[i]) {
-      uint32_t r = 0;
-#pragma unroll
-      for (int j = 0; j < i; j++) r += L[j] == L[i];
-      uint32_t base = 0, ex = 0;
-#pragma unroll
-      for (int l = 1; l <= kLmax; l++)
-        if ((uint32_t)l == L[i]) {
-          base = next[l];
-          ex = excl[l];
-        }
-      v = (L[i] << 16) | (base + ex + r);
-    }
-    enc[lane * 8 + i] = v;
-  }
+  for (int i = 0; i < 8; i++) enc[lane * 8 + i] = v[i];
 }
 
 // Code choice for one (chunk, entropy stream) whose histogram is in sm.f[0..A) and

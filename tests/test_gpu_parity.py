@@ -71,7 +71,11 @@ def test_bf16_ragged_sizes(z, orc, n):
 
 
 @pytest.mark.parametrize("chunk_bytes,subblock", [(16, 16), (4096, 64), (65536, 256), (262144, 1024),
-                                                  (1 << 20, 2048), (262144, 65536)])
+                                                  (1 << 20, 2048), (262144, 65536),
+                                                  # more sub-blocks than decode threads: two per thread,
+                                                  # one or several batches, a partly filled batch
+                                                  (262144, 256), (262144, 128), (131072, 16), (262144, 48),
+                                                  (262144, 272)])
 def test_bf16_chunk_and_subblock_shapes(z, orc, chunk_bytes, subblock):
     x = (torch.randn(300001, generator=torch.Generator().manual_seed(1)) * 0.05).to(torch.bfloat16)
     _check_roundtrip(z, orc, x, f"cb={chunk_bytes} S={subblock}", chunk_bytes=chunk_bytes, subblock=subblock)
