@@ -125,20 +125,44 @@ __global__ void __launch_bounds__(kEncodeThreads) k_encode_bf16_cluster(const ui
     uint32_t nw = 0, nfill = 0, mybits = 0;
     uint32_t qoff[kFValues / 16];
     uint64_t acc = 0;
+    if (cnt == kFValues) {
+      // two values (one input word) per step: the exponent of the low value is bits
+      // 14..7, so its table entry is at byte offset (w >> 5) & 0x3FC, the high one's at
+      // (w >> 21) & 0x3FC. The two codes (at most 24 bits) join before they enter the
+      // accumulator, which then holds fewer than 56 pending bits: one flush test a pair.
+      const uint8_t* encb = reinterpret_cast<const uint8_t*>(sm.enc);
 #pragma unroll
-    for (int i = 0; i < kFValues; i++) {
-      if ((i & 15) == 0) qoff[i >> 4] = mybits;
-      if (i < cnt) {
-        const uint32_t e = sm.enc[symbol<kBF16, kFValues>(raw, 0, i)];
-        const uint32_t l = e >> 16;
-        mybits += l;
-        acc = (acc << l) | (e & 0xFFFFu);
+      for (int j = 0; j < kFValues / 2; j++) {
+        if ((j & 7) == 0) qoff[j >> 3] = nw * 32 + nfill;
+        const uint32_t w = raw.w[j];
+        const uint32_t e0 = *reinterpret_cast<const uint32_t*>(encb + ((w >> 5) & 0x3FCu));
+        const uint32_t e1 = *reinterpret_cast<const uint32_t*>(encb + ((w >> 21) & 0x3FCu));
+        const uint32_t l1 = e1 >> 16;
+        const uint32_t l = (e0 >> 16) + l1;
+        acc = (acc << l) | (((e0 & 0xFFFFu) << l1) | (e1 & 0xFFFFu));
         nfill += l;
-        const bool full = nfill >= 32;
-        nfill -= full ? 32u : 0u;
-        const uint32_t word = (uint32_t)(acc >> nfill);
-        if (full) pw[nw] = word;
-        nw += full ? 1u : 0u;
+        if (nfill >= 32) {
+          nfill -= 32;
+          pw[nw++] = (uint32_t)(acc >> nfill);
+        }
+      }
+      mybits = nw * 32 + nfill;
+    } else {
+#pragma unroll
+      for (int i = 0; i < kFValues; i++) {
+        if ((i & 15) == 0) qoff[i >> 4] = mybits;
+        if (i < cnt) {
+          const uint32_t e = sm.enc[symbol<kBF16, kFValues>(raw, 0, i)];
+          const uint32_t l = e >> 16;
+          mybits += l;
+          acc = (acc << l) | (e & 0xFFFFu);
+          nfill += l;
+          const bool full = nfill >= 32;
+          nfill -= full ? 32u : 0u;
+          const uint32_t word = (uint32_t)(acc >> nfill);
+          if (full) pw[nw] = word;
+          nw += full ? 1u : 0u;
+        }
       }
     }
     if (nfill) pw[nw++] = (uint32_t)(acc << (32 - nfill));

@@ -72,6 +72,23 @@ __global__ void __launch_bounds__(kHistThreads) k_split_hist(const uint8_t* __re
     const int cnt = (int)min32(NV, hi - v0);
     RawValues<DT, NV> raw;
     load_values<DT, NV>(src + (clo + v0) * VB, cnt, raw);
+    if constexpr (DT == kBF16) {
+      if (cnt == NV) {
+        // a whole word at a time: the exponent e of the low value is bits 14..7, so its
+        // counter (column offset e * 32 words) is at byte offset w & 0x7F80; the high
+        // value's at (w >> 16) & 0x7F80. Zero detection needs only the masked words.
+        uint8_t* colb = reinterpret_cast<uint8_t*>(col0);
+#pragma unroll
+        for (int j = 0; j < NV / 2; j++) {
+          const uint32_t w = raw.w[j];
+          atomicAdd(reinterpret_cast<uint32_t*>(colb + (w & 0x7F80u)), 1u);
+          atomicAdd(reinterpret_cast<uint32_t*>(colb + ((w >> 16) & 0x7F80u)), 1u);
+          nz[0] |= w & 0x7F807F80u;
+          nz[NS - 1] |= w & 0x807F807Fu;
+        }
+        continue;
+      }
+    }
 #pragma unroll
     for (int i = 0; i < NV; i++) {
       if (i < cnt) {
