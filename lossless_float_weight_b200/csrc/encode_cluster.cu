@@ -1,11 +1,14 @@
 // encode_cluster.cu -- BF16 encode with thread-block clusters.
 //
 // The same work as k_encode (encode.cu) for BF16 chunks of at most 8 tiles of 16384
-// values: one cluster per chunk, one block per tile, chunks handed out by ticket.
+// values: one cluster per chunk (cluster i encodes chunk i), one block per tile.
 // Each block packs its exponent codes into shared memory, and its bit offset inside
 // the chunk is the sum of the lower blocks' bit counts, read over distributed shared
 // memory (DSMEM) after a cluster barrier: no global look-back between the tiles of a
-// chunk. Words shared by two tiles are merged as in k_encode.
+// chunk, and no dependence between clusters. Words shared by two tiles are merged as
+// in k_encode. A block arrives on the closing cluster barrier as soon as its DSMEM
+// reads are done and waits on it only before it exits (its shared memory must outlive
+// the other blocks' reads).
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -29,7 +32,6 @@ struct FusedSmem {
   uint32_t enc[256];   // the chunk's code: len << 16 | code
   uint32_t warp[kEncodeThreads / 32];
   uint32_t tile_bits;  // this tile's exponent bits (read by later blocks over DSMEM)
-  uint32_t chunk;
 };
 
 // Merge a word shared by two tiles: the second arrival stores the union.
@@ -49,12 +51,8 @@ __global__ void __launch_bounds__(kEncodeThreads) k_encode_bf16_cluster(const ui
   const uint32_t T = cluster.num_blocks(), rank = cluster.block_rank();
   extern __shared__ __align__(16) uint8_t smem_raw[];
   FusedSmem& sm = *reinterpret_cast<FusedSmem*>(smem_raw);
-  const int tid = threadIdx.x;
-
-  if (rank == 0 && tid == 0) sm.chunk = atomicAdd(ws.status + 1, 1u);  // chunks in launch order
-  cluster.sync();
-  FusedSmem* s0 = cluster.map_shared_rank(&sm, 0);
-  const uint32_t c = s0->chunk;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const uint32_t c = blockIdx.x / T;
   const uint64_t clo = (uint64_t)c * g.m0;
   const uint32_t m = (uint32_t)min64(g.m0, g.n - clo);
   const uint32_t tlo = rank * (uint32_t)kTileValues;
@@ -172,8 +170,10 @@ __global__ void __launch_bounds__(kEncodeThreads) k_encode_bf16_cluster(const ui
     const uint32_t nw_max = (31 + tile_bits + 31) / 32;
     for (uint32_t i = tid; i < nw_max; i += kEncodeThreads) sm.pack.stage[i] = 0;
     cluster.sync();
-    uint64_t P = 0;  // this tile's bit offset in the chunk: the lower tiles' bits
-    for (uint32_t r = 0; r < rank; r++) P += cluster.map_shared_rank(&sm, r)->tile_bits;
+    // this tile's bit offset in the chunk: the lower tiles' bits, lane r reading rank r
+    const uint32_t lower = (uint32_t)lane < rank ? cluster.map_shared_rank(&sm, (unsigned)lane)->tile_bits : 0u;
+    const uint64_t P = __reduce_add_sync(0xFFFFFFFFu, lower);
+    cluster.barrier_arrive();
     if (cnt > 0) {
       uint32_t rr = v0 % g.S;
 #pragma unroll
@@ -214,9 +214,11 @@ __global__ void __launch_bounds__(kEncodeThreads) k_encode_bf16_cluster(const ui
         for (uint64_t i = nsub + tid; i < idx_bytes / 4; i += kEncodeThreads) idx[i] = 0;
       }
     }
+  } else {
+    cluster.barrier_arrive();
   }
   // no block leaves while another may still read its shared memory
-  cluster.sync();
+  cluster.barrier_wait();
 }
 
 // Launch: one cluster of tiles_per_chunk blocks per chunk.

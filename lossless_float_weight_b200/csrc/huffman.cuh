@@ -45,6 +45,63 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
+// The same code as warp_huffman below for 2 <= n <= 32 present symbols whose keys
+// (weight << 8 | symbol) are in sc.iw[0..n), with every per-node quantity in registers:
+// lane p holds the p-th smallest leaf and the p-th merged node. The two-queue merge
+// runs on all lanes in step (its indices and sums are warp-uniform) and fetches queue
+// heads by shuffle; depths follow by pointer jumping towards the root.
+__device__ inline int warp_huffman_regs(HuffScratch& sc, int n) {
+  const int lane = threadIdx.x & 31;
+  const uint64_t key = lane < n ? sc.iw[lane] : ~0ull;
+  // rank of my key among the n distinct keys, then leaves in ascending key order
+  int r = 0;
+#pragma unroll
+  for (int q = 0; q < 32; q++) r += __shfl_sync(0xFFFFFFFFu, key, q) < key;
+  if (lane < n) sc.sorted[r] = key;
+  __syncwarp();
+  const uint64_t leaf_key = lane < n ? sc.sorted[lane] : ~0ull;
+  const uint64_t leaf_w = leaf_key >> 8;
+  uint64_t node_w = 0;
+  uint32_t leaf_par = 0, node_par = 0;
+  uint32_t li = 0, ii = 0;
+  uint64_t lh = __shfl_sync(0xFFFFFFFFu, leaf_w, 0), ih = 0;
+  for (int t = 0; t < n - 1; t++) {
+    uint64_t sum = 0;
+#pragma unroll
+    for (int pick = 0; pick < 2; pick++) {
+      // a leaf wins a weight tie; no merged node is available while ii == t
+      if ((int)li < n && ((int)ii >= t || lh <= ih)) {
+        if (lane == (int)li) leaf_par = (uint32_t)t;
+        sum += lh;
+        li++;
+        lh = __shfl_sync(0xFFFFFFFFu, leaf_w, li & 31);
+      } else {
+        if (lane == (int)ii) node_par = (uint32_t)t;
+        sum += ih;
+        ii++;
+        ih = __shfl_sync(0xFFFFFFFFu, node_w, ii & 31);
+      }
+    }
+    if (lane == t) node_w = sum;
+    if ((int)ii == t) ih = sum;  // the head is the node just made
+  }
+  // depth of merged node t below the root (node n - 2), by pointer jumping
+  const int root = n - 2;
+  uint32_t d = lane < root ? 1u : 0u;
+  uint32_t up = lane < root ? node_par : (uint32_t)lane;
+#pragma unroll
+  for (int k = 0; k < 5; k++) {
+    const uint32_t du = __shfl_sync(0xFFFFFFFFu, d, up & 31);
+    const uint32_t uu = __shfl_sync(0xFFFFFFFFu, up, up & 31);
+    d += du;
+    up = uu;
+  }
+  const uint32_t len = __shfl_sync(0xFFFFFFFFu, d, leaf_par & 31) + 1;
+  if (lane < n) sc.lens[leaf_key & 0xFF] = (uint8_t)len;
+  __syncwarp();
+  return (int)__reduce_max_sync(0xFFFFFFFFu, lane < n ? len : 0u);
+}
+
 // One warp: lengths of the Huffman code for the weights max(1, f >> k) of the present
 // symbols of f[0..A). Returns the longest length (0 if no symbol is present).
 __device__ inline int warp_huffman(const uint64_t* f, int A, int k, HuffScratch& sc) {
@@ -71,6 +128,7 @@ __device__ inline int warp_huffman(const uint64_t* f, int A, int k, HuffScratch&
     __syncwarp();
     return 1;
   }
+  if (n <= 32) return warp_huffman_regs(sc, n);
   // rank sort of the distinct keys (weight, symbol)
   for (int p = lane; p < n; p += 32) {
     const uint64_t kp = sc.iw[p];

@@ -142,8 +142,9 @@ def test_histogram_entry_point(z, orc):
 def test_code_lengths_entry_point(z, orc):
     rng = np.random.default_rng(3)
     hists = []
-    for t in range(200):
-        a = int(rng.integers(2, 257))
+    for t in range(400):
+        # the first half: alphabets of at most 32 symbols (the builder's register path)
+        a = int(rng.integers(2, 33)) if t < 200 else int(rng.integers(2, 257))
         kind = t % 5
         f = np.zeros(256, dtype=np.int64)
         if kind == 0:
