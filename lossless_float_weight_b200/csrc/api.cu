@@ -39,7 +39,7 @@ bool make_geo(int dt, uint64_t n, uint32_t chunk_bytes, uint32_t S, uint32_t G, 
   g.chunk_bytes = chunk_bytes;
   g.m0 = chunk_bytes / (uint32_t)value_bytes(dt);
   const uint64_t chunks = ceil_div(n, g.m0);
-  const uint64_t tpc = ceil_div(g.m0, kTileValues);
+  const uint64_t tpc = ceil_div(g.m0, tile_values(dt));
   if (chunks * (uint64_t)n_streams(dt) > 0x7FFFFFFFull || chunks * tpc > 0x7FFFFFFFull) return false;
   g.n_chunks = (uint32_t)chunks;
   g.S = S;
@@ -54,8 +54,9 @@ bool make_geo(int dt, uint64_t n, uint32_t chunk_bytes, uint32_t S, uint32_t G, 
 
 struct WsPlan {
   uint64_t status, hist, nonzero, scan_desc, tile_desc, slot, zero_end;
-  uint64_t esize, emode, ecode, eoff, enc;
+  uint64_t esize, emode, ecode, eoff, enc, tile_hist, tile_off;
   uint64_t km_mu, km_perm, km_assign, km_changed, km_gsum, total;
+  bool tile_counts;  // per-tile exponent histograms (BF16)
 };
 
 WsPlan ws_plan(const Geo& g) {
@@ -74,6 +75,9 @@ WsPlan ws_plan(const Geo& g) {
   p.ecode = o;      o = align_up(o + K * 4);
   p.eoff = o;       o = align_up(o + K * 8);
   p.enc = o;        o = align_up(o + C * NE * 256 * 4);
+  p.tile_counts = g.dt == kBF16;
+  p.tile_hist = o;  o = align_up(o + (p.tile_counts ? (uint64_t)g.n_tiles * 256 * 2 : 0));
+  p.tile_off = o;   o = align_up(o + (p.tile_counts ? (uint64_t)g.n_tiles * 4 : 0));
   p.km_mu = o;      o = align_up(o + (uint64_t)kMaxGroups * 256 * 8);
   p.km_perm = o;    o = align_up(o + C * 4);
   p.km_assign = o;  o = align_up(o + C * 4);
@@ -97,6 +101,8 @@ Ws carve(const WsPlan& p, void* base) {
   w.ecode = reinterpret_cast<uint32_t*>(b + p.ecode);
   w.eoff = reinterpret_cast<uint64_t*>(b + p.eoff);
   w.enc = reinterpret_cast<uint32_t*>(b + p.enc);
+  w.tile_hist = p.tile_counts ? reinterpret_cast<uint16_t*>(b + p.tile_hist) : nullptr;
+  w.tile_off = p.tile_counts ? reinterpret_cast<uint32_t*>(b + p.tile_off) : nullptr;
   return w;
 }
 
@@ -174,8 +180,8 @@ zipnn_status zipnn_compress_ex(zipnn_dtype dtype, const void* src, uint64_t n, u
   }
   if (e == cudaSuccess) {
     TimedLaunch t(kIdEncode, st);
-    e = cluster_encode_applies(g) ? launch_encode_bf16_cluster(src, g, w, static_cast<uint8_t*>(out), st)
-                                  : launch_encode(src, g, w, static_cast<uint8_t*>(out), st);
+    e = g.dt == kBF16 ? launch_encode_bf16(src, g, w, static_cast<uint8_t*>(out), st)
+                      : launch_encode(src, g, w, static_cast<uint8_t*>(out), st);
   }
   return cuda_status(e);
 }

@@ -26,6 +26,12 @@ constexpr int kGroupValues = 16;
 constexpr int kEncGroups = 4;
 constexpr int kEncodeThreads = 256;
 constexpr int kTileValues = kEncodeThreads * kGroupValues * kEncGroups;  // 16384
+// BF16 encode: 512 threads of 64 values; the tile is also one histogram block's slice
+constexpr int kBf16EncodeThreads = 512;
+constexpr int kBf16TileValues = kBf16EncodeThreads * kGroupValues * kEncGroups;  // 32768
+__host__ __device__ constexpr uint32_t tile_values(int dt) {
+  return dt == kBF16 ? (uint32_t)kBf16TileValues : (uint32_t)kTileValues;
+}
 
 __host__ __device__ constexpr int n_streams(int dt) { return dt == kBF16 ? 2 : dt == kFP32 ? 4 : 3; }
 __host__ __device__ constexpr int n_entropy(int dt) { return dt == kFP8 ? 2 : 1; }
@@ -62,7 +68,7 @@ struct Geo {
   uint64_t n;
   uint32_t chunk_bytes, m0, n_chunks, S;
   uint32_t n_groups;          // 0 without a plan
-  uint32_t tiles_per_chunk;   // encode tiles per chunk
+  uint32_t tiles_per_chunk;   // encode tiles (tile_values(dt) values) per chunk
   uint32_t n_tiles;           // n_chunks * tiles_per_chunk
   uint32_t n_entries;         // n_chunks * n_streams
   uint64_t off_codes, off_payload;
@@ -83,6 +89,8 @@ struct Ws {
   uint32_t* ecode;      // [n_entries]
   uint64_t* eoff;       // [n_entries] payload offsets
   uint32_t* enc;        // [n_chunks][n_entropy][256]: len << 16 | code
+  uint16_t* tile_hist;  // [n_tiles][256] (BF16 compress): exponent counts of each encode tile
+  uint32_t* tile_off;   // [n_tiles] (BF16 compress): bit offset of each tile in its chunk's bitstream
 };
 
 // Device-side tables of a plan.

@@ -273,11 +273,12 @@ static cudaError_t encode_t(const void* src, const Geo& g, const Ws& ws, uint8_t
   return cudaGetLastError();
 }
 
+// FP32 and FP8 (BF16 has k_encode_bf16).
 cudaError_t launch_encode(const void* src, const Geo& g, const Ws& ws, uint8_t* out, cudaStream_t st) {
   switch (g.dt) {
-    case kBF16: return encode_t<kBF16>(src, g, ws, out, st);
     case kFP32: return encode_t<kFP32>(src, g, ws, out, st);
-    default: return encode_t<kFP8>(src, g, ws, out, st);
+    case kFP8: return encode_t<kFP8>(src, g, ws, out, st);
+    default: return cudaErrorInvalidValue;
   }
 }
 

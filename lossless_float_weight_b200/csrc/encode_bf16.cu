@@ -1,0 +1,253 @@
+// encode_bf16.cu -- k_encode_bf16: the encode of BF16 tensors.
+//
+// The same output as k_encode (encode.cu), with no wait between blocks. A tile is
+// 32768 consecutive values of one chunk (one histogram block's slice); its exponent
+// bits start, inside the chunk's bitstream, at the sum over the chunk's lower tiles of
+// count(tile, e) * len(e). The histogram pass counts per tile and the code build turns
+// the counts into tile offsets, so every tile knows its offset before it packs a bit.
+// Blocks are persistent: each takes tiles blockIdx.x, blockIdx.x + gridDim.x, ... and
+// encodes a tile in two passes of 16384 values (256 threads of 64); the second pass
+// starts where the first one's bits end. In each pass it
+//  * loads its 64 values per thread (128-bit loads) and writes the sign/fraction plane
+//    (and an exponent plane that did not compress) with 16-byte stores;
+//  * packs its exponent codes, two per step, most significant bit first, into private
+//    shared words from bit 0; a block scan gives each thread its bit offset in the tile;
+//  * moves the private words into a staging copy of the tile's bitstream at its final
+//    alignment (shared atomicOr on each thread's two edge words), then stores it with
+//    coalesced 32-bit stores, clearing the staging words as it reads them. The word
+//    shared by the two passes is carried in shared memory into the second pass's first
+//    word. A word that straddles two tiles is merged in a workspace slot: each side adds
+//    (1 << 32 | its bits) and the side that arrives second stores the complete word.
+// The sub-block index idx[j] (bit offset of symbol j*S) is written by the thread that
+// owns symbol j*S; the first tile writes a local code record, the last the padding.
+#include "common.cuh"
+#include "fields.cuh"
+#include "launch.h"
+
+namespace zipnn {
+
+constexpr int kBThreads = 256;
+constexpr int kBValues = kGroupValues * kEncGroups;             // 64 values per thread
+constexpr int kBPassValues = kBThreads * kBValues;              // 16384
+constexpr int kBPasses = kBf16TileValues / kBPassValues;        // 2
+constexpr int kBStageWords = kBPassValues * kLmax / 32 + 2;     // one pass's bitstream
+constexpr int kBPrivStride = kBValues * kLmax / 32 + 1;         // odd: conflict-free
+static_assert(kBPasses * kBPassValues == kBf16TileValues, "a tile is a whole number of passes");
+
+struct Bf16EncodeSmem {
+  uint32_t priv[kBThreads * kBPrivStride];  // each thread's codes, packed from bit 0
+  uint32_t stage[kBStageWords];                  // the tile's bitstream at its final alignment
+  uint32_t enc[256];                             // the chunk's code: len << 16 | code
+  uint32_t warp[kBThreads / 32];
+  uint32_t carry;  // the bits of the word shared with the next pass
+};
+
+__device__ __forceinline__ void bf16_slot_merge(uint64_t* slot, uint32_t part, uint32_t* dst) {
+  const uint64_t old = atomicAdd(reinterpret_cast<unsigned long long*>(slot), (1ull << 32) | (uint64_t)part);
+  if ((old >> 32) == 1) *dst = bswap32((uint32_t)old | part);
+}
+
+// Exponent (s == 0) or sign/fraction byte (s == 1) of two BF16 values, in bytes 0 and 2.
+__device__ __forceinline__ uint32_t bf16_pair_plane(uint32_t w, int s) {
+  return s == 0 ? (w >> 7) & 0x00FF00FFu : (w & 0x007F007Fu) | ((w >> 8) & 0x00800080u);
+}
+
+__global__ void __launch_bounds__(kBThreads, 4) k_encode_bf16(const uint8_t* __restrict__ src, Geo g, Ws ws,
+                                                                   uint8_t* __restrict__ out) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  Bf16EncodeSmem& sm = *reinterpret_cast<Bf16EncodeSmem*>(smem_raw);
+  const int tid = threadIdx.x;
+  const uint32_t T = g.tiles_per_chunk;
+  for (int i = tid; i < kBStageWords; i += kBThreads) sm.stage[i] = 0;
+
+  for (uint32_t tile = blockIdx.x; tile < g.n_tiles; tile += gridDim.x) {
+    const uint32_t c = tile / T, ti = tile - c * T;
+    const uint64_t clo = (uint64_t)c * g.m0;
+    const uint32_t m = (uint32_t)min64(g.m0, g.n - clo);
+    const uint32_t tlo = ti * (uint32_t)kBf16TileValues;
+    if (tlo >= m) continue;  // past the end of a ragged last chunk (uniform)
+    // the chunk's decisions and code
+    const uint32_t mode0 = ws.emode[2ull * c], mode1 = ws.emode[2ull * c + 1];
+    const uint32_t code0 = ws.ecode[2ull * c];
+    const uint64_t off0 = ws.eoff[2ull * c], off1 = ws.eoff[2ull * c + 1];
+    uint64_t P = 0;  // the pass's bit offset in the chunk
+    if (mode0 == kModeHuff) {
+      sm.enc[tid] = ws.enc[(uint64_t)c * 256 + tid];
+      P = ws.tile_off[tile];
+    }
+    __syncthreads();  // the code is visible; the previous tile's stores and clears are done
+    const uint64_t nsub = ceil_div(m, g.S);
+    const uint32_t rec = code0 == kNoCode ? record_bytes(kBF16, 0) : 0;
+    const uint64_t idx_bytes = round16(4 * nsub);
+    uint8_t* payload = out + off0;
+    uint32_t* idx = reinterpret_cast<uint32_t*>(payload + rec);
+    uint32_t* bs = reinterpret_cast<uint32_t*>(payload + rec + idx_bytes);
+
+    for (int pass = 0; pass < kBPasses; pass++) {
+      const uint32_t plo = tlo + pass * (uint32_t)kBPassValues;
+      if (plo >= m) break;  // uniform
+      const bool last = plo + (uint32_t)kBPassValues >= m;              // the chunk's last pass
+      const bool tile_end = last || pass == kBPasses - 1;               // the tile's last pass
+      const uint32_t v0 = plo + tid * kBValues;
+      const int cnt = v0 < m ? (int)min32(kBValues, m - v0) : 0;
+      RawValues<kBF16, kBValues> raw;
+      if (cnt > 0) load_values<kBF16, kBValues>(src + (clo + v0) * 2, cnt, raw);
+
+#pragma unroll
+      for (int s = 0; s < 2; s++) {
+        if ((s == 0 ? mode0 : mode1) != kModeRaw || cnt == 0) continue;
+        // RAW byte plane (the sign/fraction bytes; an exponent stream that did not compress)
+        uint8_t* dst = out + (s == 0 ? off0 : off1) + v0;
+        if (cnt == kBValues) {
+#pragma unroll
+          for (int q = 0; q < kBValues / 16; q++) {
+            uint32_t x[4];
+#pragma unroll
+            for (int k = 0; k < 4; k++)
+              x[k] = __byte_perm(bf16_pair_plane(raw.w[8 * q + 2 * k], s),
+                                 bf16_pair_plane(raw.w[8 * q + 2 * k + 1], s), 0x6420);
+            *reinterpret_cast<uint4*>(dst + 16 * q) = make_uint4(x[0], x[1], x[2], x[3]);
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < kBValues / 16; q++) {
+            if (16 * q < cnt) {
+              uint32_t x[4];
+#pragma unroll
+              for (int j = 0; j < 4; j++) {
+                x[j] = 0;
+#pragma unroll
+                for (int b = 0; b < 4; b++) {
+                  const int i = 16 * q + 4 * j + b;
+                  if (i < cnt) x[j] |= symbol<kBF16, kBValues>(raw, s, i) << (8 * b);
+                }
+              }
+              *reinterpret_cast<uint4*>(dst + 16 * q) = make_uint4(x[0], x[1], x[2], x[3]);
+            }
+          }
+        }
+      }
+      if (mode0 != kModeHuff) continue;  // uniform
+
+      // the local code record heads the payload (4-bit lengths)
+      if (rec && ti == 0 && pass == 0 && tid < 128)
+        payload[tid] = (uint8_t)((sm.enc[2 * tid] >> 16) | ((sm.enc[2 * tid + 1] >> 16) << 4));
+      // pack my codes from bit 0 of my private words
+      uint32_t* pw = sm.priv + tid * kBPrivStride;
+      uint32_t nw = 0, nfill = 0, mybits = 0;
+      uint32_t qoff[kBValues / 16];
+      uint64_t acc = 0;
+      if (cnt == kBValues) {
+        // two values (one input word) per step: the exponent of the low value is bits
+        // 14..7, so its table entry is at byte offset (w >> 5) & 0x3FC, the high one's at
+        // (w >> 21) & 0x3FC. The two codes (at most 24 bits) join before they enter the
+        // accumulator, which then holds fewer than 56 pending bits: one flush test a pair.
+        const uint8_t* encb = reinterpret_cast<const uint8_t*>(sm.enc);
+#pragma unroll
+        for (int j = 0; j < kBValues / 2; j++) {
+          if ((j & 7) == 0) qoff[j >> 3] = nw * 32 + nfill;
+          const uint32_t w = raw.w[j];
+          const uint32_t e0 = *reinterpret_cast<const uint32_t*>(encb + ((w >> 5) & 0x3FCu));
+          const uint32_t e1 = *reinterpret_cast<const uint32_t*>(encb + ((w >> 21) & 0x3FCu));
+          const uint32_t l1 = e1 >> 16;
+          const uint32_t l = (e0 >> 16) + l1;
+          acc = (acc << l) | (((e0 & 0xFFFFu) << l1) | (e1 & 0xFFFFu));
+          nfill += l;
+          if (nfill >= 32) {
+            nfill -= 32;
+            pw[nw++] = (uint32_t)(acc >> nfill);
+          }
+        }
+        mybits = nw * 32 + nfill;
+      } else {
+#pragma unroll
+        for (int i = 0; i < kBValues; i++) {
+          if ((i & 15) == 0) qoff[i >> 4] = mybits;
+          if (i < cnt) {
+            const uint32_t e = sm.enc[symbol<kBF16, kBValues>(raw, 0, i)];
+            const uint32_t l = e >> 16;
+            mybits += l;
+            acc = (acc << l) | (e & 0xFFFFu);
+            nfill += l;
+            const bool full = nfill >= 32;
+            nfill -= full ? 32u : 0u;
+            const uint32_t word = (uint32_t)(acc >> nfill);
+            if (full) pw[nw] = word;
+            nw += full ? 1u : 0u;
+          }
+        }
+      }
+      if (nfill) pw[nw++] = (uint32_t)(acc << (32 - nfill));
+      uint32_t pass_bits;
+      const uint32_t myoff = block_exclusive_scan<kBThreads>(mybits, sm.warp, pass_bits);
+      if (cnt > 0) {
+        uint32_t rr = v0 % g.S;
+#pragma unroll
+        for (int q = 0; q < kBValues / 16; q++) {
+          if (rr == 0 && 16 * q < cnt) idx[(v0 + 16 * q) / g.S] = (uint32_t)(P + myoff + qoff[q]);
+          rr += 16;
+          if (rr >= g.S) rr -= g.S;
+        }
+      }
+      if (mybits) {
+        const uint32_t q0 = (uint32_t)(P & 31) + myoff;
+        const uint32_t sh = q0 & 31, d0 = q0 >> 5, dlast = (q0 + mybits - 1) >> 5;
+        uint32_t prev = 0;
+        for (uint32_t k = 0; k <= dlast - d0; k++) {
+          const uint32_t cur = k < nw ? pw[k] : 0u;
+          const uint32_t o = (sh ? prev << (32 - sh) : 0u) | (cur >> sh);
+          if (k == 0 || k == dlast - d0) atomicOr(sm.stage + d0 + k, o);
+          else sm.stage[d0 + k] = o;
+          prev = cur;
+        }
+      }
+      __syncthreads();
+      const uint64_t end = P + pass_bits;
+      const uint32_t nwt = (uint32_t)(((P & 31) + pass_bits + 31) >> 5);
+      const uint64_t W0 = P >> 5;
+      for (uint32_t i = tid; i < nwt; i += kBThreads) {
+        uint32_t word = sm.stage[i];
+        sm.stage[i] = 0;
+        if (i == 0 && pass > 0 && (P & 31) != 0) word |= sm.carry;  // the first pass's last bits
+        uint32_t* dst = bs + W0 + i;
+        // (a first pass that is not the tile's last has 16384 values, so i == 0 and the
+        // carried word are never the same word)
+        if (i == nwt - 1 && (end & 31) != 0 && !tile_end) sm.carry = word;  // completed by the next pass
+        else if (i == 0 && pass == 0 && (P & 31) != 0) bf16_slot_merge(ws.slot + tile, word, dst);
+        else if (i == nwt - 1 && (end & 31) != 0 && !last) bf16_slot_merge(ws.slot + tile + 1, word, dst);
+        else *dst = bswap32(word);
+      }
+      P = end;
+      if (last) {
+        const uint64_t padded_words = round16(ceil_div(end, 8)) / 4;
+        for (uint64_t i = W0 + nwt + tid; i < padded_words; i += kBThreads) bs[i] = 0;
+        for (uint64_t i = nsub + tid; i < idx_bytes / 4; i += kBThreads) idx[i] = 0;
+      }
+    }
+  }
+}
+
+// Launch: a persistent grid of as many blocks as fit on the device at once.
+cudaError_t launch_encode_bf16(const void* src, const Geo& g, const Ws& ws, uint8_t* out, cudaStream_t st) {
+  const size_t smem = sizeof(Bf16EncodeSmem);
+  static int resident[128] = {0};  // blocks per device, once the attributes are set
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  int per_device = dev >= 0 && dev < 128 ? resident[dev] : 0;
+  if (!per_device) {
+    e = cudaFuncSetAttribute(k_encode_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_encode_bf16, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    int per_sm = 0, sms = 0;
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_encode_bf16, kBThreads, smem);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    per_device = (per_sm > 0 ? per_sm : 1) * (sms > 0 ? sms : 1);
+    if (dev >= 0 && dev < 128) resident[dev] = per_device;
+  }
+  const uint32_t blocks = (uint32_t)min64((uint64_t)per_device, g.n_tiles);
+  k_encode_bf16<<<blocks, kBThreads, smem, st>>>(static_cast<const uint8_t*>(src), g, ws, out);
+  return cudaGetLastError();
+}
+
+}  // namespace zipnn

@@ -35,6 +35,7 @@ struct HuffBlockSmem {
   uint64_t cost[kMaxGroups];
   uint32_t elig[kMaxGroups];
   uint64_t red[kHuffWarps];
+  uint32_t red32[kHuffWarps];
   int pick;
   uint32_t bits_lo, bits_hi;
 };

@@ -15,6 +15,45 @@ namespace zipnn {
 
 constexpr int kHistThreads = 256;
 constexpr uint32_t kHistSlice = 32768;  // values of one chunk per histogram block
+static_assert(kHistSlice == kBf16TileValues, "a BF16 histogram slice is one encode tile");
+
+// BF16 with a HUFF exponent stream: the bit offset of each encode tile in the chunk's
+// bitstream, the running sum over the lower tiles of count(tile, e) * len(e), from the
+// per-tile counts of the histogram pass. Warp w totals tiles w, w + 8, ...; a block
+// scan turns the totals into offsets. The code builder's scratch is free by now.
+__device__ void tile_offsets(const Geo& g, const Ws& ws, uint32_t c, const uint32_t* enc, HuffBlockSmem& sm) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t T = g.tiles_per_chunk;
+  const uint64_t m = min64(g.m0, g.n - (uint64_t)c * g.m0);
+  uint8_t* lens = reinterpret_cast<uint8_t*>(sm.w[0].lens);
+  uint32_t* tbits = reinterpret_cast<uint32_t*>(&sm.w[1]);  // T words: T <= 8192 fits 7 scratches
+  static_assert(sizeof(HuffScratch) * (kHuffWarps - 1) >= 8192 * 4, "tile totals fit the builder scratch");
+  lens[tid] = (uint8_t)(__ldcg(enc + tid) >> 16);
+  __syncthreads();
+  uint32_t L[8];
+#pragma unroll
+  for (int i = 0; i < 8; i++) L[i] = lens[lane * 8 + i];
+  for (uint32_t t = warp; t < T; t += kHuffWarps) {
+    uint32_t part = 0;
+    if ((uint64_t)t * kBf16TileValues < m) {
+      const uint4 q = __ldcg(reinterpret_cast<const uint4*>(ws.tile_hist + ((uint64_t)c * T + t) * 256) + lane);
+      const uint32_t x[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int i = 0; i < 8; i++) part += ((x[i >> 1] >> (16 * (i & 1))) & 0xFFFFu) * L[i];
+    }
+    part = __reduce_add_sync(0xFFFFFFFFu, part);
+    if (lane == 0) tbits[t] = part;
+  }
+  __syncthreads();
+  uint32_t carry = 0;
+  for (uint32_t base = 0; base < T; base += kHuffWarps * 32) {
+    const uint32_t t = base + tid;
+    uint32_t total;
+    const uint32_t before = block_exclusive_scan<kHuffWarps * 32>(t < T ? tbits[t] : 0u, sm.red32, total);
+    if (t < T) ws.tile_off[(uint64_t)c * T + t] = carry + before;
+    carry += total;
+  }
+}
 
 // Per (chunk, entropy stream), one block of kHuffWarps warps: ZERO when every symbol is
 // 0, else the code choice of decide_code.
@@ -38,8 +77,14 @@ __device__ void build_chunk_table(const Geo& g, const Ws& ws, const PlanDev& pla
   const uint32_t* h = ws.hist + ((uint64_t)c * NE + e) * 256;
   sm.f[tid] = tid < A ? __ldcg(h + tid) : 0;
   __syncthreads();
-  decide_code(sm, A, w, record_bytes(DT, e), m, g.S, plan, e, ws.enc + ((uint64_t)c * NE + e) * 256, ws.emode + k,
-              ws.ecode + k, ws.esize + k);
+  uint32_t* enc = ws.enc + ((uint64_t)c * NE + e) * 256;
+  decide_code(sm, A, w, record_bytes(DT, e), m, g.S, plan, e, enc, ws.emode + k, ws.ecode + k, ws.esize + k);
+  if constexpr (DT == kBF16) {
+    if (ws.tile_off) {
+      __syncthreads();
+      if (ws.emode[k] == kModeHuff) tile_offsets(g, ws, c, enc, sm);
+    }
+  }
 }
 
 // THEORY-599 note, "Order-0 only (section III-A b)": the model of a chunk is the count
@@ -68,38 +113,44 @@ __global__ void __launch_bounds__(kHistThreads) k_split_hist(const uint8_t* __re
   uint32_t* col0 = sh + lane;
   uint32_t* col1 = sh + A0 * 32 + lane;
   constexpr int NV = 64;  // consecutive values per thread per pass, loaded up front
-  for (uint32_t v0 = lo + tid * NV; v0 < hi; v0 += kHistThreads * NV) {
-    const int cnt = (int)min32(NV, hi - v0);
-    RawValues<DT, NV> raw;
-    load_values<DT, NV>(src + (clo + v0) * VB, cnt, raw);
-    if constexpr (DT == kBF16) {
-      if (cnt == NV) {
-        // a whole word at a time: the exponent e of the low value is bits 14..7, so its
-        // counter (column offset e * 32 words) is at byte offset w & 0x7F80; the high
-        // value's at (w >> 16) & 0x7F80. Zero detection needs only the masked words.
-        uint8_t* colb = reinterpret_cast<uint8_t*>(col0);
+  for (uint32_t t0 = lo; t0 < hi; t0 += kHistThreads * NV) {
+    const uint32_t v0 = t0 + tid * NV;
+    const int cnt = v0 < hi ? (int)min32(NV, hi - v0) : 0;
+    if (cnt > 0) {
+      RawValues<DT, NV> raw;
+      load_values<DT, NV>(src + (clo + v0) * VB, cnt, raw);
+      bool done = false;
+      if constexpr (DT == kBF16) {
+        if (cnt == NV) {
+          // a whole word at a time: the exponent e of the low value is bits 14..7, so its
+          // counter (column offset e * 32 words) is at byte offset w & 0x7F80; the high
+          // value's at (w >> 16) & 0x7F80. Zero detection needs only the masked words.
+          uint8_t* colb = reinterpret_cast<uint8_t*>(col0);
 #pragma unroll
-        for (int j = 0; j < NV / 2; j++) {
-          const uint32_t w = raw.w[j];
-          atomicAdd(reinterpret_cast<uint32_t*>(colb + (w & 0x7F80u)), 1u);
-          atomicAdd(reinterpret_cast<uint32_t*>(colb + ((w >> 16) & 0x7F80u)), 1u);
-          nz[0] |= w & 0x7F807F80u;
-          nz[NS - 1] |= w & 0x807F807Fu;
+          for (int j = 0; j < NV / 2; j++) {
+            const uint32_t w = raw.w[j];
+            atomicAdd(reinterpret_cast<uint32_t*>(colb + (w & 0x7F80u)), 1u);
+            atomicAdd(reinterpret_cast<uint32_t*>(colb + ((w >> 16) & 0x7F80u)), 1u);
+            nz[0] |= w & 0x7F807F80u;
+            nz[NS - 1] |= w & 0x807F807Fu;
+          }
+          done = true;
         }
-        continue;
+      }
+      if (!done) {
+#pragma unroll
+        for (int i = 0; i < NV; i++) {
+          if (i < cnt) {
+            atomicAdd(col0 + symbol<DT, NV>(raw, 0, i) * 32, 1u);
+            if (NE > 1) atomicAdd(col1 + symbol<DT, NV>(raw, 1, i) * 32, 1u);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < NV; i++)
+#pragma unroll
+          for (int s = 0; s < NS; s++) nz[s] |= symbol<DT, NV>(raw, s, i);
       }
     }
-#pragma unroll
-    for (int i = 0; i < NV; i++) {
-      if (i < cnt) {
-        atomicAdd(col0 + symbol<DT, NV>(raw, 0, i) * 32, 1u);
-        if (NE > 1) atomicAdd(col1 + symbol<DT, NV>(raw, 1, i) * 32, 1u);
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < NV; i++)
-#pragma unroll
-      for (int s = 0; s < NS; s++) nz[s] |= symbol<DT, NV>(raw, s, i);
   }
 #pragma unroll
   for (int s = 0; s < NS; s++) {
@@ -114,6 +165,8 @@ __global__ void __launch_bounds__(kHistThreads) k_split_hist(const uint8_t* __re
     for (int l = 0; l < 32; l++) sum += sh[b * 32 + ((l + b) & 31)];
     const int e = b < A0 ? 0 : 1, sym = b < A0 ? b : b - A0;
     if (sum) atomicAdd(&hist[((uint64_t)c * NE + e) * 256 + sym], sum);
+    // BF16 compress: the slice is one encode tile; its counts give the tile offsets
+    if (DT == kBF16 && ws.tile_hist) ws.tile_hist[((uint64_t)c * g.tiles_per_chunk + sl) * 256 + b] = (uint16_t)sum;
   }
   if (!build) return;
   // the last block to finish a chunk builds that chunk's codes (its histogram is then
