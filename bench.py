@@ -79,6 +79,35 @@ def rank_seed(rank):
 
 # ------------------------------------------------------------------ measurement helpers
 
+# ncu summaries under profiles/ that give a kernel's DRAM bytes per value; each names the
+# kernel sources it was taken from, by hash, so a summary of an older kernel is not used
+PROFILE_OF = {"decode_merge": "decode_merge_embedding_bf16.txt", "encode": "encode_bf16_embedding_bf16.txt",
+              "split_hist_tables": "split_hist_tables_embedding_bf16.txt"}
+
+
+def profile_traffic(kernel, values_per_launch):
+    """DRAM bytes of one launch of `kernel`, from its committed ncu summary scaled by the values
+    the launch processes; None without a summary or when the sources changed since."""
+    import hashlib
+    import re
+    name = PROFILE_OF.get(kernel)
+    path = os.path.join(ROOT, "profiles", name) if name else None
+    if not path or not os.path.exists(path):
+        return None
+    text = open(path).read()
+    bpv = re.search(r"DRAM bytes per value\s+([0-9.]+)", text)
+    src = re.search(r"kernel sources sha256 \(([^)]*)\): ([0-9a-f]{64})", text)
+    if not bpv or not src:
+        return None
+    h = hashlib.sha256()
+    for f in sorted(src.group(1).split()):
+        with open(os.path.join(ROOT, "lossless_float_weight_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest() != src.group(2):
+        return None
+    return round(float(bpv.group(1)) * values_per_launch)
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -90,7 +119,7 @@ def measured_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle samples every 200 ms while running."""
+    """nvidia-smi clock / throttle samples every 50 ms while running."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -103,7 +132,7 @@ class ClockSampler:
     def start(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -322,7 +351,9 @@ def run_ours(args):
                 "peak_source": peak_src,
                 "unit": "GB/s",
                 "frac": round(achieved / peak, 4),
-                "traffic": None,
+                "traffic": profile_traffic(dom_name, nbytes / 2 / len(xs)),
+                "traffic_note": "DRAM bytes per launch: the kernel's ncu bytes per value on the embedding tensor "
+                                "(profiles/) times the average values per launch; null if the kernel changed since",
                 "avg_launch_ms": round(dom_ms / max(1, dom_n), 5),
                 "launches": int(dom_n),
                 "measured": "CUDA events around every launch of the kernel, single-stream kernel-timing pass of "
