@@ -29,7 +29,7 @@ import torch
 METRIC = "decompress/compress GB/s (uncompressed) at 1 B200; % of HBM roofline"
 WORKLOAD = ("BF16 7B-shaped checkpoint: 32 x [q,k,v,o 4096x4096; gate,up,down 4096x11008] + embedding "
             "32000x4096, 225 tensors, 6,607,077,376 values (13.21 GB), sigma_t log-uniform [0.005, 0.05], "
-            "256 KiB chunks, one zipnn call per tensor, tensors spread round-robin over 4 streams")
+            "256 KiB chunks; compress: one zipnn call per tensor, tensors spread round-robin over 4 streams")
 CHUNK = 262144
 SUBBLOCK = 512  # the library default (include/zipnn.h)
 FALLBACK_HBM_GBS = 6650.0
@@ -242,8 +242,13 @@ def run_ours(args):
     def compress_all():
         fan_out(lambda i, s, w: Z.compress_into(xs[i], outs[i], w, CHUNK, stream=s))
 
+    bws = Z.batch_workspace(len(xs), dev)
+
     def decompress_all():
-        fan_out(lambda i, s, w: Z.decompress_into(outs[i], outs[i].numel(), decs[i], w, CHUNK, stream=s))
+        if args.per_tensor_decode:
+            fan_out(lambda i, s, w: Z.decompress_into(outs[i], outs[i].numel(), decs[i], w, CHUNK, stream=s))
+        else:  # one launch over all the tensors' chunks
+            Z.decompress_batch_into(outs, [o.numel() for o in outs], decs, bws, CHUNK, stream=stream)
 
     for _ in range(args.warmup):
         compress_all()
@@ -291,8 +296,11 @@ def run_ours(args):
     for k in range(args.steps):
         for i in range(len(xs)):
             Z.compress_into(xs[i], outs[i], wss[0], CHUNK, stream=stream)
-        for i in range(len(xs)):
-            Z.decompress_into(outs[i], outs[i].numel(), decs[i], wss[0], CHUNK, stream=stream)
+        if args.per_tensor_decode:
+            for i in range(len(xs)):
+                Z.decompress_into(outs[i], outs[i].numel(), decs[i], wss[0], CHUNK, stream=stream)
+        else:
+            Z.decompress_batch_into(outs, [o.numel() for o in outs], decs, bws, CHUNK, stream=stream)
     torch.cuda.synchronize()
     ktimes = Z.kernel_times()
     Z.zipnn_timing_enable(0)
@@ -329,7 +337,9 @@ def run_ours(args):
             "data": "synthetic (seeded N(0, sigma_t^2) BF16 tensors of a 7B checkpoint's shapes; no trained weights)",
             "config": {
                 "workload": WORKLOAD,
-                "step": "compress all 225 tensors, then decompress all 225 (value = uncompressed bytes per "
+                "step": "compress all 225 tensors (one zipnn_compress each), then decompress all 225 ("
+                        + ("one zipnn_decompress each" if args.per_tensor_decode else "one zipnn_decompress_batch")
+                        + ") (value = uncompressed bytes per "
                         "step / step time, x ranks)",
                 "global_batch": world * nbytes,
                 "parallelism": f"weak scaling, {world} independent checkpoint(s), no collective on the data path",
@@ -375,7 +385,7 @@ def run_e2e(Z, xs, csizes, dev, stream, streams, args, world):
     """Same metric through the public API with host buffers: pinned host tensors in,
     pinned host tensors out. Every step copies each tensor to the device, compresses
     it, reads its size and copies the container back, then copies each container to
-    the device, decompresses it and copies the values back."""
+    the device, decompresses them (one batched call) and copies the values back."""
     nbytes = sum(x.numel() * 2 for x in xs)
     h_in = [x.cpu().pin_memory() for x in xs]
     h_cont = [torch.empty(c, dtype=torch.uint8).pin_memory() for c in csizes]
@@ -385,6 +395,7 @@ def run_e2e(Z, xs, csizes, dev, stream, streams, args, world):
               for x in xs]
     d_out = [torch.empty_like(x) for x in xs]
     wss = [Z.workspace(Z.BF16, max(x.numel() for x in xs), CHUNK, dev) for _ in streams]
+    bws = Z.batch_workspace(len(xs), dev)
     ns = len(streams)
 
     def step():
@@ -406,13 +417,19 @@ def run_e2e(Z, xs, csizes, dev, stream, streams, args, world):
             s = streams[i % ns]
             with torch.cuda.stream(s):
                 d_cont[i][: csizes[i]].copy_(h_cont[i], non_blocking=True)
-            Z.decompress_into(d_cont[i], csizes[i], d_out[i], wss[i % ns], CHUNK, stream=s)
-            with torch.cuda.stream(s):
-                h_out[i].copy_(d_out[i], non_blocking=True)
+            if args.per_tensor_decode:
+                Z.decompress_into(d_cont[i], csizes[i], d_out[i], wss[i % ns], CHUNK, stream=s)
+                with torch.cuda.stream(s):
+                    h_out[i].copy_(d_out[i], non_blocking=True)
         for s in streams:
             e2 = torch.cuda.Event()
             e2.record(s)
             stream.wait_event(e2)
+        if not args.per_tensor_decode:
+            Z.decompress_batch_into(d_cont, csizes, d_out, bws, CHUNK, stream=stream)
+            with torch.cuda.stream(stream):
+                for i in range(len(xs)):
+                    h_out[i].copy_(d_out[i], non_blocking=True)
 
     steps = max(1, min(args.steps, 3))
     step()
@@ -483,6 +500,8 @@ def main():
     ap.add_argument("--only", type=int, default=None, help="only tensor IDX of the checkpoint (profiler cases)")
     ap.add_argument("--no-extras", action="store_true", help="skip the e2e and CPU-baseline legs")
     ap.add_argument("--streams", type=int, default=4, help="CUDA streams the tensors are spread over")
+    ap.add_argument("--per-tensor-decode", action="store_true",
+                    help="decompress with one zipnn_decompress per tensor (default: one zipnn_decompress_batch)")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

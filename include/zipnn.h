@@ -120,6 +120,32 @@ zipnn_status zipnn_decompress(zipnn_dtype dtype, const void* in, size_t in_bytes
                               uint32_t chunk_bytes, void* out, void* ws, size_t ws_bytes,
                               zipnn_stream_t stream);
 
+/* One tensor of a batched decompress: its container `in` (device, 16-byte aligned, in_bytes
+ * readable), its value count n and its output `out` (device, 16-byte aligned, n values). */
+typedef struct zipnn_decompress_item {
+  const void* in;
+  uint64_t in_bytes;
+  uint64_t n;
+  void* out;
+} zipnn_decompress_item;
+
+/* Workspace bytes for zipnn_decompress_batch of `count` tensors. */
+size_t zipnn_decompress_batch_workspace_bytes(uint32_t count);
+
+/* Decompress `count` containers of one dtype and chunk_bytes in a single launch: one block
+ * per chunk over all the tensors' chunks, so that many small tensors fill the device
+ * together ("ZipNN: Lossless Compression for AI Models", abstract: a model is many
+ * tensors). Each output equals what zipnn_decompress gives for that item alone. `items`
+ * is a host array, read before the call returns; its table is copied (stream-ordered)
+ * into `ws`, which must hold zipnn_decompress_batch_workspace_bytes(count) and must not be
+ * reused until the call completes. Argument errors (null or misaligned pointers, a count
+ * of 0, n or chunk_bytes outside the limits of zipnn_compress, more than 2^31 - 1 chunks in
+ * all) return synchronously before any launch. Damage found in any container sets
+ * ZIPNN_ERR_CORRUPT in the workspace status (outputs are then unspecified). */
+zipnn_status zipnn_decompress_batch(zipnn_dtype dtype, uint32_t chunk_bytes, uint32_t count,
+                                    const zipnn_decompress_item* items, void* ws, size_t ws_bytes,
+                                    zipnn_stream_t stream);
+
 /* Wait for `stream`, then read the container size from the header at `out`. */
 zipnn_status zipnn_compressed_size(const void* out, zipnn_stream_t stream, uint64_t* bytes);
 

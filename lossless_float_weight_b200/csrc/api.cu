@@ -209,6 +209,45 @@ zipnn_status zipnn_decompress(zipnn_dtype dtype, const void* in, size_t in_bytes
   return cuda_status(e);
 }
 
+// Batched decompress workspace: the status word, then the device copy of the item table.
+static constexpr size_t kBatchTableOffset = 256;
+
+size_t zipnn_decompress_batch_workspace_bytes(uint32_t count) {
+  return kBatchTableOffset + (size_t)align_up((uint64_t)count * sizeof(DecodeItem));
+}
+
+zipnn_status zipnn_decompress_batch(zipnn_dtype dtype, uint32_t chunk_bytes, uint32_t count,
+                                    const zipnn_decompress_item* items, void* ws, size_t ws_bytes,
+                                    zipnn_stream_t stream) {
+  if (!items || !ws || count == 0 || !aligned16(ws)) return ZIPNN_ERR_INVALID_ARG;
+  std::vector<DecodeItem> table(count);
+  Geo g0;
+  uint64_t chunks = 0;
+  for (uint32_t i = 0; i < count; i++) {
+    const zipnn_decompress_item& it = items[i];
+    Geo g;
+    if (!it.in || !it.out || !aligned16(it.in) || !aligned16(it.out)) return ZIPNN_ERR_INVALID_ARG;
+    if (!make_geo(dtype, it.n, chunk_bytes, ZIPNN_DEFAULT_SUBBLOCK, 0, g)) return ZIPNN_ERR_INVALID_ARG;
+    if (i == 0) g0 = g;
+    table[i] = DecodeItem{static_cast<const uint8_t*>(it.in), it.in_bytes, it.n, static_cast<uint8_t*>(it.out), chunks};
+    chunks += g.n_chunks;
+    if (chunks > 0x7FFFFFFFull) return ZIPNN_ERR_INVALID_ARG;
+  }
+  if (ws_bytes < zipnn_decompress_batch_workspace_bytes(count)) return ZIPNN_ERR_OUT_TOO_SMALL;
+  if (!device_ok()) return ZIPNN_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  DecodeItem* dev_table = reinterpret_cast<DecodeItem*>(static_cast<uint8_t*>(ws) + kBatchTableOffset);
+  cudaError_t e = cudaMemsetAsync(ws, 0, 4, st);
+  // from pageable memory: the table is staged before the call returns
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(dev_table, table.data(), (size_t)count * sizeof(DecodeItem), cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) {
+    TimedLaunch t(kIdDecode, st);
+    e = launch_decode_batch(dev_table, count, g0, (uint32_t)chunks, static_cast<uint32_t*>(ws), st);
+  }
+  return cuda_status(e);
+}
+
 zipnn_status zipnn_compressed_size(const void* out, zipnn_stream_t stream, uint64_t* bytes) {
   if (!out || !bytes) return ZIPNN_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

@@ -439,15 +439,16 @@ struct DecodeSmem {
 // three BF16 decode blocks share an SM: 228 KB of shared memory, 1 KB reserved per block
 static_assert(sizeof(StagedSmem) + sizeof(DecodeSmem<kBF16>) + 1024 <= 233472 / 3, "BF16 decode: 3 blocks per SM");
 
+// Chunk c of the container `in` (in_bytes readable) of a tensor with geometry g, into
+// `out` (the tensor's first value). All threads of the block.
 template <int DT>
-__global__ void __launch_bounds__(kDecodeThreads, DT == kBF16 ? 3 : 1) k_decode(const uint8_t* __restrict__ in, uint64_t in_bytes, Geo g,
-                                                           uint8_t* __restrict__ out, uint32_t* status) {
+__device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uint64_t in_bytes, const Geo& g,
+                                             uint32_t c, uint8_t* __restrict__ out, uint32_t* status) {
   constexpr int NS = n_streams(DT), NE = n_entropy(DT), VB = value_bytes(DT);
   constexpr int GV = DT == kBF16 ? 8 : DT == kFP32 ? 4 : 16;  // values per 16-byte store
   __shared__ DecodeSmem<DT> sm;
   extern __shared__ __align__(128) uint8_t dyn_smem[];  // StagedSmem for BF16 launches
   const int tid = threadIdx.x;
-  const uint32_t c = blockIdx.x;
   const uint64_t clo = (uint64_t)c * g.m0;
   const uint32_t m = (uint32_t)min64(g.m0, g.n - clo);
 
@@ -803,22 +804,77 @@ __global__ void __launch_bounds__(kDecodeThreads, DT == kBF16 ? 3 : 1) k_decode(
 }
 
 template <int DT>
+__global__ void __launch_bounds__(kDecodeThreads, DT == kBF16 ? 3 : 1)
+    k_decode(const uint8_t* __restrict__ in, uint64_t in_bytes, Geo g, uint8_t* __restrict__ out, uint32_t* status) {
+  decode_chunk<DT>(in, in_bytes, g, blockIdx.x, out, status);
+}
+
+// The item whose chunks include global chunk b: the last i with items[i].chunk0 <= b
+// (items[0].chunk0 == 0, increasing). One warp, a 32-way search: each round probes 32
+// evenly spaced items and keeps the span after the last probe at or below b.
+__device__ __forceinline__ uint32_t find_item(const DecodeItem* __restrict__ items, uint32_t count, uint64_t b) {
+  const uint32_t lane = threadIdx.x & 31;
+  uint32_t lo = 0, hi = count;  // the answer is in [lo, hi)
+  while (hi - lo > 1) {
+    const uint32_t step = (hi - lo + 31) / 32;
+    const uint32_t p = lo + lane * step;
+    const bool le = p < hi && items[p].chunk0 <= b;
+    const uint32_t mask = __ballot_sync(0xFFFFFFFFu, le);  // bit 0 is set: items[lo].chunk0 <= b
+    lo += (uint32_t)(31 - __clz(mask)) * step;
+    hi = min32(lo + step, hi);
+  }
+  return lo;
+}
+
+// Many tensors in one launch: block b decodes global chunk b.
+template <int DT>
+__global__ void __launch_bounds__(kDecodeThreads, DT == kBF16 ? 3 : 1)
+    k_decode_batch(const DecodeItem* __restrict__ items, uint32_t count, Geo g, uint32_t* status) {
+  __shared__ uint32_t s_item;
+  if (threadIdx.x < 32) {
+    const uint32_t it = find_item(items, count, blockIdx.x);
+    if (threadIdx.x == 0) s_item = it;
+  }
+  __syncthreads();
+  const DecodeItem d = items[s_item];
+  g.n = d.n;
+  g.n_chunks = (uint32_t)ceil_div(d.n, g.m0);
+  decode_chunk<DT>(d.in, d.in_bytes, g, (uint32_t)(blockIdx.x - d.chunk0), d.out, status);
+}
+
+// Dynamic shared memory (the BF16 staging window) once per device and kernel.
+template <class K>
+static cudaError_t decode_attributes(K kernel, size_t dyn, int* done) {
+  if (!dyn) return cudaSuccess;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 128 && done[dev]) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  if (e == cudaSuccess && dev >= 0 && dev < 128) done[dev] = 1;
+  return e;
+}
+
+template <int DT>
 static cudaError_t decode_t(const uint8_t* in, uint64_t in_bytes, const Geo& g, uint8_t* out, uint32_t* status,
                             cudaStream_t st) {
   const size_t dyn = DT == kBF16 ? sizeof(StagedSmem) : 0;
-  if (dyn) {
-    static int done[128] = {0};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 128 || !done[dev]) {
-      e = cudaFuncSetAttribute(k_decode<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
-      if (e == cudaSuccess) e = cudaFuncSetAttribute(k_decode<DT>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-      if (e != cudaSuccess) return e;
-      if (dev >= 0 && dev < 128) done[dev] = 1;
-    }
-  }
+  static int done[128] = {0};
+  cudaError_t e = decode_attributes(k_decode<DT>, dyn, done);
+  if (e != cudaSuccess) return e;
   k_decode<DT><<<g.n_chunks, kDecodeThreads, dyn, st>>>(in, in_bytes, g, out, status);
+  return cudaGetLastError();
+}
+
+template <int DT>
+static cudaError_t decode_batch_t(const DecodeItem* items, uint32_t count, const Geo& g, uint32_t total_chunks,
+                                  uint32_t* status, cudaStream_t st) {
+  const size_t dyn = DT == kBF16 ? sizeof(StagedSmem) : 0;
+  static int done[128] = {0};
+  cudaError_t e = decode_attributes(k_decode_batch<DT>, dyn, done);
+  if (e != cudaSuccess) return e;
+  k_decode_batch<DT><<<total_chunks, kDecodeThreads, dyn, st>>>(items, count, g, status);
   return cudaGetLastError();
 }
 
@@ -828,6 +884,15 @@ cudaError_t launch_decode(const uint8_t* in, uint64_t in_bytes, const Geo& g, ui
     case kBF16: return decode_t<kBF16>(in, in_bytes, g, out, status, st);
     case kFP32: return decode_t<kFP32>(in, in_bytes, g, out, status, st);
     default: return decode_t<kFP8>(in, in_bytes, g, out, status, st);
+  }
+}
+
+cudaError_t launch_decode_batch(const DecodeItem* items, uint32_t count, const Geo& g, uint32_t total_chunks,
+                                uint32_t* status, cudaStream_t st) {
+  switch (g.dt) {
+    case kBF16: return decode_batch_t<kBF16>(items, count, g, total_chunks, status, st);
+    case kFP32: return decode_batch_t<kFP32>(items, count, g, total_chunks, status, st);
+    default: return decode_batch_t<kFP8>(items, count, g, total_chunks, status, st);
   }
 }
 

@@ -34,6 +34,18 @@ cudaError_t launch_encode(const void* src, const Geo& g, const Ws& ws, uint8_t* 
 cudaError_t launch_encode_bf16(const void* src, const Geo& g, const Ws& ws, uint8_t* out, cudaStream_t st);
 cudaError_t launch_decode(const uint8_t* in, uint64_t in_bytes, const Geo& g, uint8_t* out, uint32_t* status,
                           cudaStream_t st);
+// One tensor of a batched decode (device table); chunk0 = its first chunk in the batch.
+struct DecodeItem {
+  const uint8_t* in;
+  uint64_t in_bytes;
+  uint64_t n;
+  uint8_t* out;
+  uint64_t chunk0;
+};
+// All chunks of `count` tensors of one dtype and chunk size in one launch; g carries the
+// dtype, chunk_bytes and m0 (n and n_chunks come from each item).
+cudaError_t launch_decode_batch(const DecodeItem* items, uint32_t count, const Geo& g, uint32_t total_chunks,
+                                uint32_t* status, cudaStream_t st);
 
 // plan (grouping) steps
 struct KmeansDev {

@@ -58,12 +58,23 @@ zipnn_kernel_name = _sig("zipnn_kernel_name", ctypes.c_char_p, _u32)
 zipnn_compress_noalloc = _sig("zipnn_compress_noalloc", _i, _i, _vp, _u64, _u32, _vp, _sz, _vp)
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
+
+class DecompressItem(ctypes.Structure):
+    """zipnn_decompress_item: one tensor of a batched decompress."""
+    _fields_ = [("in_", _vp), ("in_bytes", _u64), ("n", _u64), ("out", _vp)]
+
+
+zipnn_decompress_batch_workspace_bytes = _sig("zipnn_decompress_batch_workspace_bytes", _sz, _u32)
+zipnn_decompress_batch = _sig("zipnn_decompress_batch", _i, _i, _u32, _u32, ctypes.POINTER(DecompressItem), _vp,
+                              _sz, _vp)
+
 C_ABI_NAMES = [
     "zipnn_max_compressed_bytes", "zipnn_workspace_bytes", "zipnn_compress", "zipnn_compress_ex",
     "zipnn_decompress", "zipnn_compressed_size", "zipnn_get_status", "zipnn_histogram", "zipnn_code_lengths",
     "zipnn_plan_create", "zipnn_plan_export", "zipnn_plan_import", "zipnn_plan_assignment", "zipnn_plan_destroy",
     "zipnn_status_string", "zipnn_timing_enable", "zipnn_timing_collect", "zipnn_kernel_count",
-    "zipnn_kernel_name", "zipnn_compress_noalloc",
+    "zipnn_kernel_name", "zipnn_compress_noalloc", "zipnn_decompress_batch_workspace_bytes",
+    "zipnn_decompress_batch",
 ]
 
 
@@ -170,6 +181,25 @@ def decompress_into(container, nbytes, out, ws, chunk_bytes=DEFAULT_CHUNK_BYTES,
     dt = dtype_code(out.dtype)
     check(zipnn_decompress(dt, container.data_ptr(), nbytes, out.numel(), chunk_bytes, out.data_ptr(),
                            ws.data_ptr(), ws.numel(), _stream(stream)), "zipnn_decompress")
+
+
+def batch_workspace(count, device="cuda"):
+    """A workspace for zipnn_decompress_batch of `count` tensors."""
+    return torch.empty(zipnn_decompress_batch_workspace_bytes(count), dtype=torch.uint8, device=device)
+
+
+def decompress_batch_into(containers, nbytes, outs, ws, chunk_bytes=DEFAULT_CHUNK_BYTES, stream=None):
+    """Asynchronous: decompress the device containers (nbytes[i] readable each) into the
+    device tensors outs[i], all of one dtype, in one launch."""
+    if not outs or len(containers) != len(outs) or len(nbytes) != len(outs):
+        raise ZipnnError(ERR_INVALID_ARG, "zipnn_decompress_batch")
+    dt = dtype_code(outs[0].dtype)
+    if any(dtype_code(o.dtype) != dt for o in outs):
+        raise ZipnnError(ERR_INVALID_ARG, "zipnn_decompress_batch: one dtype per batch")
+    items = (DecompressItem * len(outs))(*[DecompressItem(c.data_ptr(), b, o.numel(), o.data_ptr())
+                                            for c, b, o in zip(containers, nbytes, outs)])
+    check(zipnn_decompress_batch(dt, chunk_bytes, len(outs), items, ws.data_ptr(), ws.numel(), _stream(stream)),
+          "zipnn_decompress_batch")
 
 
 def compressed_size(out, stream=None):

@@ -55,3 +55,23 @@ def test_argument_errors_without_a_device(lib):
     assert Z.zipnn_code_lengths(None, 1, 256, None, None) == Z.ERR_INVALID_ARG
     assert Z.zipnn_plan_import(None, 0, None) == Z.ERR_INVALID_ARG
     assert Z.zipnn_status_string(Z.ERR_CORRUPT).startswith(b"corrupt")
+
+
+def test_batch_argument_errors_without_a_device(lib):
+    from lossless_float_weight_b200 import zipnn as Z
+    fake = 1 << 20  # a 16-byte aligned address, never dereferenced: every case fails before a launch
+    ws_bytes = Z.zipnn_decompress_batch_workspace_bytes(2)
+    assert ws_bytes >= 256 + 2 * 40
+    good = (Z.DecompressItem * 2)(Z.DecompressItem(fake, 4096, 1000, fake), Z.DecompressItem(fake, 4096, 5, fake))
+    # no items, no workspace, an empty batch
+    assert Z.zipnn_decompress_batch(Z.BF16, 262144, 2, None, fake, ws_bytes, None) == Z.ERR_INVALID_ARG
+    assert Z.zipnn_decompress_batch(Z.BF16, 262144, 2, good, None, ws_bytes, None) == Z.ERR_INVALID_ARG
+    assert Z.zipnn_decompress_batch(Z.BF16, 262144, 0, good, fake, ws_bytes, None) == Z.ERR_INVALID_ARG
+    # a misaligned or null pointer, n = 0, a bad chunk size
+    for bad in (Z.DecompressItem(fake + 8, 4096, 10, fake), Z.DecompressItem(fake, 4096, 10, None),
+                Z.DecompressItem(fake, 4096, 0, fake)):
+        items = (Z.DecompressItem * 2)(good[0], bad)
+        assert Z.zipnn_decompress_batch(Z.BF16, 262144, 2, items, fake, ws_bytes, None) == Z.ERR_INVALID_ARG
+    assert Z.zipnn_decompress_batch(Z.BF16, 1000, 2, good, fake, ws_bytes, None) == Z.ERR_INVALID_ARG
+    # a workspace one byte short
+    assert Z.zipnn_decompress_batch(Z.BF16, 262144, 2, good, fake, ws_bytes - 1, None) == Z.ERR_OUT_TOO_SMALL
