@@ -489,6 +489,106 @@ def run_reference(args):
     }), flush=True)
 
 
+def run_plan_transfer(args):
+    """Shared-code setup reuse ("NeuralZip: Reusable Setup for Fast Lossless Compression",
+    abstract: a setup transferred to other weights and reused as they evolve). A plan is
+    built once on layers 0-15 of the checkpoint (one tensor, their concatenation), then
+    layers 16-31 are compressed with it, as they are and with 5% relative noise added
+    (weights after further training). Reports the size against per-chunk codes, the
+    fraction of chunks that fall back to a local code, the setup time and the compress
+    throughput with and without the plan (4 streams, as the main benchmark)."""
+    from lossless_float_weight_b200 import workloads as W
+    from lossless_float_weight_b200 import zipnn as Z
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    shapes = W.checkpoint_7b_shapes()
+    sig = W.checkpoint_7b_sigmas(len(shapes))
+    per_layer = 7
+    a_ids, b_ids = range(0, 16 * per_layer), range(16 * per_layer, 32 * per_layer)
+    a = torch.cat([W.checkpoint_7b_tensor(t, shapes[t][1], sig[t], dev).reshape(-1) for t in a_ids])
+    xs = [W.checkpoint_7b_tensor(t, shapes[t][1], sig[t], dev).reshape(-1) for t in b_ids]
+    g = torch.Generator(device=dev).manual_seed(99)
+    noisy = [(x.float() + 0.05 * float(sig[t]) * torch.randn(x.numel(), generator=g, device=dev)).to(torch.bfloat16)
+             for x, t in zip(xs, b_ids)]
+    nbytes = sum(x.numel() * 2 for x in xs)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    plan = Z.Plan.create(a, groups=args.groups, seed=0, ws=Z.workspace(Z.BF16, a.numel(), CHUNK, dev))
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    setup_ms = ev0.elapsed_time(ev1)
+    del a
+    streams = [torch.cuda.Stream(dev) for _ in range(args.streams)]
+    wss = [Z.workspace(Z.BF16, max(x.numel() for x in xs), CHUNK, dev) for _ in streams]
+    outs = [torch.empty(Z.zipnn_max_compressed_bytes(Z.BF16, x.numel(), CHUNK), dtype=torch.uint8, device=dev)
+            for x in xs]
+
+    def compress(tensors, with_plan):
+        ev = torch.cuda.Event()
+        ev.record(stream)
+        for s in streams:
+            s.wait_event(ev)
+        for i, x in enumerate(tensors):
+            Z.compress_into(x, outs[i], wss[i % len(streams)], CHUNK, plan=plan if with_plan else None,
+                            stream=streams[i % len(streams)])
+        for s in streams:
+            e = torch.cuda.Event()
+            e.record(s)
+            stream.wait_event(e)
+
+    def measure(tensors, with_plan):
+        for _ in range(args.warmup):
+            compress(tensors, with_plan)
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            compress(tensors, with_plan)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        ms = t0.elapsed_time(t1) / args.steps
+        size, huff, local = 0, 0, 0
+        for i, x in enumerate(tensors):
+            size += Z.compressed_size(outs[i])
+            c = -(-x.numel() // (CHUNK // 2))
+            table = outs[i][64: 64 + 16 * 2 * c].cpu().numpy().reshape(c, 2, 16)[:, 0]  # exponent entries
+            mode = table[:, 0]
+            code = table[:, 4:8].copy().view("<u4")[:, 0]
+            huff += int((mode == 2).sum())
+            local += int(((mode == 2) & (code == 0xFFFFFFFF)).sum())
+        # the round trip still holds with the plan
+        y = torch.empty_like(tensors[0])
+        Z.decompress_into(outs[0], outs[0].numel(), y, wss[0], CHUNK, stream=stream)
+        torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.int16), tensors[0].view(torch.int16))
+        return {"ratio": round(size / nbytes, 5), "compress_GBps": round(nbytes / (ms / 1e3) / 1e9, 1),
+                "ms": round(ms, 3), "fallback_rate": round(local / max(1, huff), 4)}
+
+    own = measure(xs, False)
+    reuse = measure(xs, True)
+    drift = measure(noisy, True)
+    drift_own = measure(noisy, False)
+    line = {
+        "mode": "plan_transfer",
+        "workload": "plan on layers 0-15 of the BF16 7B-shaped checkpoint (6.47 GB, 112 tensors concatenated); "
+                    "applied to layers 16-31 (112 tensors, %.2f GB) as generated and with N(0, (0.05 sigma_t)^2) "
+                    "added; 256 KiB chunks" % (nbytes / 1e9),
+        "groups": args.groups,
+        "setup_ms": round(setup_ms, 2),
+        "own_codes": own,
+        "plan": reuse,
+        "plan_ratio_loss_pct": round(100 * (reuse["ratio"] / own["ratio"] - 1), 3),
+        "perturbed_own_codes": drift_own,
+        "perturbed_plan": drift,
+        "perturbed_ratio_loss_pct": round(100 * (drift["ratio"] / drift_own["ratio"] - 1), 3),
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "streams": args.streams,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -500,9 +600,15 @@ def main():
     ap.add_argument("--only", type=int, default=None, help="only tensor IDX of the checkpoint (profiler cases)")
     ap.add_argument("--no-extras", action="store_true", help="skip the e2e and CPU-baseline legs")
     ap.add_argument("--streams", type=int, default=4, help="CUDA streams the tensors are spread over")
+    ap.add_argument("--plan-transfer", action="store_true",
+                    help="instead of the benchmark: build a shared-code plan on layers 0-15 and reuse it on 16-31")
+    ap.add_argument("--groups", type=int, default=8, help="plan groups for --plan-transfer")
     ap.add_argument("--per-tensor-decode", action="store_true",
                     help="decompress with one zipnn_decompress per tensor (default: one zipnn_decompress_batch)")
     args = ap.parse_args()
+    if args.plan_transfer:
+        run_plan_transfer(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -189,6 +189,19 @@ def test_plan_parity(z, orc):
     _check_roundtrip(z, orc, other, "kv reuse", plan=p2, plan_lens=lens)
 
 
+def test_plan_transfer_between_layers(z, orc):
+    # a plan built on one checkpoint tensor codes another layer's tensor exactly as the oracle does
+    from lossless_float_weight_b200 import workloads as W
+    shapes = W.checkpoint_7b_shapes()
+    sig = W.checkpoint_7b_sigmas(len(shapes))
+    a = W.checkpoint_7b_tensor(0, shapes[0][1], sig[0], "cpu").reshape(-1)    # layer 0 q, 128 chunks
+    b = W.checkpoint_7b_tensor(12, shapes[12][1], sig[12], "cpu").reshape(-1)  # layer 1 up projection
+    plan = z.Plan.create(a.cuda(), groups=8, seed=0)
+    lens, assign, _, _ = orc.plan_build("bf16", _host_bytes(a), a.numel(), CB, groups=8, seed=0)
+    assert plan.assignment() == assign.tolist()
+    _check_roundtrip(z, orc, b, "plan from another layer", plan=plan, plan_lens=lens)
+
+
 def test_plan_fp8_and_small(z, orc):
     from lossless_float_weight_b200 import workloads as W
     q = W.fp8_tensor(rows=512, cols=4096)
