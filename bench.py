@@ -589,6 +589,76 @@ def run_plan_transfer(args):
     print(json.dumps(line), flush=True)
 
 
+def run_single(args):
+    """One tensor of another workload (the parity configs, and FP4 at the FP8 config's
+    shape): compress and decompress timed separately, K steps each, CUDA events on one
+    stream; inputs resident in HBM and larger than L2. K/V cache: compress with an
+    8-group plan built once before the timed region (its setup time reported apart)."""
+    from lossless_float_weight_b200 import workloads as W
+    from lossless_float_weight_b200 import zipnn as Z
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    w = args.workload
+    if w in ("fp32", "fp32_clean"):
+        x = W.fp32_tensor(n=268435456, device=dev, clean=(w == "fp32_clean"))
+        desc = "FP32 268,435,456 values N(0, 0.02^2)" + (", rounded through BF16" if w == "fp32_clean" else "")
+    elif w == "fp8":
+        x = W.fp8_tensor(rows=262144, cols=4096, device=dev)
+        desc = "FP8 E4M3 262,144 x 4096, N(0, 1) x per-row scale log-uniform [0.25, 4]"
+    elif w == "fp4":
+        x = W.fp4_tensor(rows=262144, cols=4096, device=dev)
+        desc = "FP4 E2M1 262,144 x 4096 (1,073,741,824 values), N(0, 1) x per-row scale log-uniform [0.25, 4]"
+    else:
+        x = W.kv_cache(device=dev)
+        desc = "BF16 K/V cache [32, 2, 16, 8, 4096, 128], per-channel std log-normal, 8-group plan"
+    x = x.reshape(-1)
+    n = Z.nvalues(x)
+    nbytes = x.numel() * x.element_size()
+    dt = Z.dtype_code(x.dtype)
+    ws = Z.workspace(dt, n, CHUNK, dev)
+    out = torch.empty(Z.zipnn_max_compressed_bytes(dt, n, CHUNK), dtype=torch.uint8, device=dev)
+    y = torch.empty_like(x)
+    plan, setup_ms = None, None
+    if w == "kv_cache":
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        plan = Z.Plan.create(x, groups=8, seed=0, ws=ws)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        setup_ms = e0.elapsed_time(e1)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / args.steps
+
+    c_ms = timed(lambda: Z.compress_into(x, out, ws, CHUNK, plan=plan, stream=stream))
+    cbytes = Z.compressed_size(out)
+    d_ms = timed(lambda: Z.decompress_into(out, cbytes, y, ws, CHUNK, stream=stream))
+    ok = torch.equal(y.view(torch.uint8), x.view(torch.uint8)) and Z.status(ws) == Z.OK
+    peak, peak_src = measured_peaks()
+    algo = nbytes + cbytes
+    line = {
+        "metric": METRIC, "workload": w, "config": desc, "unit": "GB/s",
+        "compress": {"GBps": round(nbytes / (c_ms / 1e3) / 1e9, 2), "ms": round(c_ms, 4),
+                     "hbm_frac": round(algo / (c_ms / 1e3) / 1e9 / peak, 4)},
+        "decompress": {"GBps": round(nbytes / (d_ms / 1e3) / 1e9, 2), "ms": round(d_ms, 4),
+                       "hbm_frac": round(algo / (d_ms / 1e3) / 1e9 / peak, 4)},
+        "compression_ratio": round(cbytes / nbytes, 5), "bytes": nbytes, "values": n,
+        "peak": peak, "peak_source": peak_src, "steps": args.steps, "warmup": args.warmup,
+        "plan_setup_ms": None if setup_ms is None else round(setup_ms, 2), "roundtrip_ok": bool(ok),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -600,6 +670,9 @@ def main():
     ap.add_argument("--only", type=int, default=None, help="only tensor IDX of the checkpoint (profiler cases)")
     ap.add_argument("--no-extras", action="store_true", help="skip the e2e and CPU-baseline legs")
     ap.add_argument("--streams", type=int, default=4, help="CUDA streams the tensors are spread over")
+    ap.add_argument("--workload", default="checkpoint_7b",
+                    choices=["checkpoint_7b", "fp32", "fp32_clean", "fp8", "fp4", "kv_cache"],
+                    help="another workload than the benchmark's: one tensor, compress and decompress timed apart")
     ap.add_argument("--plan-transfer", action="store_true",
                     help="instead of the benchmark: build a shared-code plan on layers 0-15 and reuse it on 16-31")
     ap.add_argument("--groups", type=int, default=8, help="plan groups for --plan-transfer")
@@ -608,6 +681,9 @@ def main():
     args = ap.parse_args()
     if args.plan_transfer:
         run_plan_transfer(args)
+        return
+    if args.workload != "checkpoint_7b":
+        run_single(args)
         return
     if args.impl == "reference":
         run_reference(args)

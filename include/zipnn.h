@@ -1,6 +1,6 @@
 /*
- * zipnn.h -- C ABI of libzipnn_b200: ZipNN-style lossless compression of BF16, FP32
- * and FP8 (E4M3) tensors on an NVIDIA B200 (sm_100a).
+ * zipnn.h -- C ABI of libzipnn_b200: ZipNN-style lossless compression of BF16, FP32,
+ * FP8 (E4M3) and FP4 (E2M1) tensors on an NVIDIA B200 (sm_100a).
  *
  * What the calls compute, by page title and section:
  *  - "ZipNN: Lossless Compression for AI Models" (abstract) and the THEORY-599 note
@@ -11,8 +11,8 @@
  *  - THEORY-599, "Order-0 only (section III-A b)": one order-0 symbol histogram and one
  *    Huffman code per chunk; no context model.
  *  - "Lossless Compression of Neural Network Components: Weights, Checkpoints, and K/V
- *    Caches in Low-Precision Formats" (abstract): FP8 exponent and mantissa are
- *    entropy-coded independently.
+ *    Caches in Low-Precision Formats" (abstract): FP8 and FP4 exponent and mantissa
+ *    are entropy-coded independently.
  *  - "NeuralZip: Reusable Setup for Fast Lossless Compression" (abstract): chunks are
  *    grouped by the similarity of their exponent distributions, each group shares one
  *    Huffman code, and this setup (a "plan") is built once and reused.
@@ -36,8 +36,11 @@
  *           [bitstream, padded]; idx[j] is the bit offset of symbol j*S.
  *   Streams: BF16 [exponent, sign+fraction byte]; FP32 [exponent, sign + fraction
  *   bits 22..16, fraction bits 15..8, fraction bits 7..0]; FP8 E4M3 [exponent (4 bits),
- *   mantissa (3 bits), sign (1 bit)]. Entropy-coded streams: the exponent, and for FP8
- *   also the mantissa. Codes are canonical (RFC 1951 rule), at most 12 bits long.
+ *   mantissa (3 bits), sign (1 bit)]; FP4 E2M1 [exponent (2 bits), mantissa (1 bit),
+ *   sign (1 bit)]. Entropy-coded streams: the exponent, and for FP8 and FP4 also the
+ *   mantissa. FP4 values come two to a byte, value 2i in the low nibble of byte i
+ *   (sign bit 3, exponent bits 2..1, mantissa bit 0); n counts values and is even.
+ *   Codes are canonical (RFC 1951 rule), at most 12 bits long.
  *   A stream is ZERO when all its symbols in the chunk are 0; an entropy stream is HUFF
  *   when that payload is strictly smaller than RAW, else RAW.
  *
@@ -64,7 +67,7 @@ extern "C" {
 /* Same type as cudaStream_t; NULL is the legacy default stream. */
 typedef struct CUstream_st* zipnn_stream_t;
 
-typedef enum { ZIPNN_BF16 = 0, ZIPNN_FP32 = 1, ZIPNN_FP8_E4M3 = 2 } zipnn_dtype;
+typedef enum { ZIPNN_BF16 = 0, ZIPNN_FP32 = 1, ZIPNN_FP8_E4M3 = 2, ZIPNN_FP4_E2M1 = 3 } zipnn_dtype;
 
 typedef enum {
   ZIPNN_OK = 0,
@@ -87,7 +90,7 @@ typedef struct zipnn_plan zipnn_plan_t; /* opaque; owns device code tables */
 /* Upper bound of the container size for n values: header, chunk table, room for
  * ZIPNN_MAX_GROUPS shared records, and every payload stored RAW (a HUFF payload is
  * only chosen when it is smaller). Returns 0 for invalid arguments.
- * chunk_bytes: a multiple of 16 in [16, 2^30]. */
+ * chunk_bytes: a multiple of 16 in [16, 2^28]. */
 size_t zipnn_max_compressed_bytes(zipnn_dtype dtype, uint64_t n, uint32_t chunk_bytes);
 
 /* Bytes of device scratch that compress, decompress and plan creation need for n

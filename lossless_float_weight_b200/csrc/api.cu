@@ -28,16 +28,17 @@ constexpr uint32_t kMaxChunkBytes = 1u << 28;
 
 inline uint64_t align_up(uint64_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
-inline bool valid_dtype(int dt) { return dt == kBF16 || dt == kFP32 || dt == kFP8; }
+inline bool valid_dtype(int dt) { return dt == kBF16 || dt == kFP32 || dt == kFP8 || dt == kFP4; }
 
 bool make_geo(int dt, uint64_t n, uint32_t chunk_bytes, uint32_t S, uint32_t G, Geo& g) {
   if (!valid_dtype(dt) || n == 0) return false;
+  if (dt == kFP4 && n % 2) return false;  // FP4 values come in byte pairs
   if (chunk_bytes < 16 || chunk_bytes % 16 || chunk_bytes > kMaxChunkBytes) return false;
   if (S < 16 || S % 16 || S > 65536) return false;
   g.dt = dt;
   g.n = n;
   g.chunk_bytes = chunk_bytes;
-  g.m0 = chunk_bytes / (uint32_t)value_bytes(dt);
+  g.m0 = (uint32_t)(8ull * chunk_bytes / (uint32_t)value_bits(dt));
   const uint64_t chunks = ceil_div(n, g.m0);
   const uint64_t tpc = ceil_div(g.m0, tile_values(dt));
   if (chunks * (uint64_t)n_streams(dt) > 0x7FFFFFFFull || chunks * tpc > 0x7FFFFFFFull) return false;

@@ -14,7 +14,7 @@ namespace zipnn {
 constexpr int kLmax = 12;
 constexpr uint32_t kNoCode = 0xFFFFFFFFu;
 constexpr uint32_t kModeRaw = 0, kModeZero = 1, kModeHuff = 2;
-constexpr int kBF16 = 0, kFP32 = 1, kFP8 = 2;
+constexpr int kBF16 = 0, kFP32 = 1, kFP8 = 2, kFP4 = 3;
 constexpr int kHeaderBytes = 64, kEntryBytes = 16;
 constexpr uint32_t kMaxGroups = 64;
 
@@ -34,14 +34,20 @@ __host__ __device__ constexpr uint32_t tile_values(int dt) {
 }
 
 __host__ __device__ constexpr int n_streams(int dt) { return dt == kBF16 ? 2 : dt == kFP32 ? 4 : 3; }
-__host__ __device__ constexpr int n_entropy(int dt) { return dt == kFP8 ? 2 : 1; }
+// FP8 and FP4 entropy-code exponent and mantissa independently
+__host__ __device__ constexpr int n_entropy(int dt) { return dt == kFP8 || dt == kFP4 ? 2 : 1; }
+// bits of one value (FP4: two values share a byte, the first in the low nibble)
+__host__ __device__ constexpr int value_bits(int dt) { return dt == kBF16 ? 16 : dt == kFP32 ? 32 : dt == kFP8 ? 8 : 4; }
+// bytes of one value where whole bytes hold whole values (BF16, FP32, FP8)
 __host__ __device__ constexpr int value_bytes(int dt) { return dt == kBF16 ? 2 : dt == kFP32 ? 4 : 1; }
+// byte offset of value v (for FP4, v is even)
+__host__ __device__ constexpr uint64_t value_offset(int dt, uint64_t v) { return v * value_bits(dt) / 8; }
 // bits per symbol of a stream stored RAW
 __host__ __device__ constexpr int raw_width(int dt, int s) {
-  return dt == kFP8 ? (s == 0 ? 4 : s == 1 ? 3 : 1) : 8;
+  return dt == kFP8 ? (s == 0 ? 4 : s == 1 ? 3 : 1) : dt == kFP4 ? (s == 0 ? 2 : 1) : 8;
 }
 __host__ __device__ constexpr int alphabet(int dt, int s) { return 1 << raw_width(dt, s); }
-__host__ __device__ constexpr bool is_entropy(int dt, int s) { return s == 0 || (dt == kFP8 && s == 1); }
+__host__ __device__ constexpr bool is_entropy(int dt, int s) { return s == 0 || ((dt == kFP8 || dt == kFP4) && s == 1); }
 __host__ __device__ constexpr uint64_t min64(uint64_t a, uint64_t b) { return a < b ? a : b; }
 __host__ __device__ constexpr uint32_t min32(uint32_t a, uint32_t b) { return a < b ? a : b; }
 __host__ __device__ constexpr uint64_t round16(uint64_t x) { return (x + 15) & ~uint64_t(15); }

@@ -445,7 +445,7 @@ template <int DT>
 __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uint64_t in_bytes, const Geo& g,
                                              uint32_t c, uint8_t* __restrict__ out, uint32_t* status) {
   constexpr int NS = n_streams(DT), NE = n_entropy(DT), VB = value_bytes(DT);
-  constexpr int GV = DT == kBF16 ? 8 : DT == kFP32 ? 4 : 16;  // values per 16-byte store
+  constexpr int GV = DT == kBF16 ? 8 : DT == kFP32 ? 4 : 16;  // values per store (16 bytes; FP4 8)
   __shared__ DecodeSmem<DT> sm;
   extern __shared__ __align__(128) uint8_t dyn_smem[];  // StagedSmem for BF16 launches
   const int tid = threadIdx.x;
@@ -753,43 +753,65 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
         st[s].br.init(reinterpret_cast<const uint32_t*>(in + bs_off), (uint32_t)(cap_bits / 32), bad ? 0 : start);
       }
     }
-    uint8_t* dst = out + (clo + sb_lo) * VB;
+    uint8_t* dst = out + value_offset(DT, clo + sb_lo);
     const uint32_t full = count / GV;
     for (uint32_t gi = 0; gi < full; gi++) {
       uint32_t sy[NS][GV];
 #pragma unroll
       for (int s = 0; s < NS; s++) next_symbols<GV, true>(st[s], sy[s], GV, gi * GV);
-      uint32_t wv[4];
+      if constexpr (DT == kFP4) {  // two values a byte, the first in the low nibble
+        uint32_t wv[2];
 #pragma unroll
-      for (int q = 0; q < 4; q++) {
-        if constexpr (DT == kBF16) {
-          wv[q] = merge_value<DT>(sy[0][2 * q], sy[1][2 * q], 0, 0) |
-                  (merge_value<DT>(sy[0][2 * q + 1], sy[1][2 * q + 1], 0, 0) << 16);
-        } else if constexpr (DT == kFP32) {
-          wv[q] = merge_value<DT>(sy[0][q], sy[1][q], sy[2][q], sy[3][q]);
-        } else {
+        for (int q = 0; q < 2; q++) {
           uint32_t x = 0;
 #pragma unroll
-          for (int b = 0; b < 4; b++) x |= merge_value<DT>(sy[0][4 * q + b], sy[1][4 * q + b], sy[2][4 * q + b], 0) << (8 * b);
+          for (int b = 0; b < 8; b++) x |= merge_value<DT>(sy[0][8 * q + b], sy[1][8 * q + b], sy[2][8 * q + b], 0) << (4 * b);
           wv[q] = x;
         }
+        *reinterpret_cast<uint2*>(dst + (uint64_t)gi * 8) = make_uint2(wv[0], wv[1]);
+      } else {
+        uint32_t wv[4];
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+          if constexpr (DT == kBF16) {
+            wv[q] = merge_value<DT>(sy[0][2 * q], sy[1][2 * q], 0, 0) |
+                    (merge_value<DT>(sy[0][2 * q + 1], sy[1][2 * q + 1], 0, 0) << 16);
+          } else if constexpr (DT == kFP32) {
+            wv[q] = merge_value<DT>(sy[0][q], sy[1][q], sy[2][q], sy[3][q]);
+          } else {
+            uint32_t x = 0;
+#pragma unroll
+            for (int b = 0; b < 4; b++) x |= merge_value<DT>(sy[0][4 * q + b], sy[1][4 * q + b], sy[2][4 * q + b], 0) << (8 * b);
+            wv[q] = x;
+          }
+        }
+        *reinterpret_cast<uint4*>(dst + (uint64_t)gi * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
       }
-      *reinterpret_cast<uint4*>(dst + (uint64_t)gi * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
     }
     const uint32_t rem = count - full * GV;
     if (rem) {
       uint32_t sy[NS][GV];
 #pragma unroll
       for (int s = 0; s < NS; s++) next_symbols<GV, false>(st[s], sy[s], (int)rem, full * GV);
+      if constexpr (DT == kFP4) {  // rem is even: values come in byte pairs
 #pragma unroll
-      for (uint32_t i = 0; i < (uint32_t)GV; i++) {
-        if (i >= rem) break;
-        const uint32_t v = merge_value<DT>(sy[0][i], sy[1][i], NS > 2 ? sy[NS > 2 ? 2 : 0][i] : 0,
-                                           NS > 3 ? sy[NS > 3 ? 3 : 0][i] : 0);
-        uint8_t* p = dst + (uint64_t)(full * GV + i) * VB;
-        if constexpr (VB == 2) *reinterpret_cast<uint16_t*>(p) = (uint16_t)v;
-        else if constexpr (VB == 4) *reinterpret_cast<uint32_t*>(p) = v;
-        else *p = (uint8_t)v;
+        for (uint32_t i = 0; i < (uint32_t)GV; i += 2) {
+          if (i >= rem) break;
+          const uint32_t lo = merge_value<DT>(sy[0][i], sy[1][i], sy[2][i], 0);
+          const uint32_t hi = merge_value<DT>(sy[0][i + 1], sy[1][i + 1], sy[2][i + 1], 0);
+          dst[(full * GV + i) / 2] = (uint8_t)(lo | (hi << 4));
+        }
+      } else {
+#pragma unroll
+        for (uint32_t i = 0; i < (uint32_t)GV; i++) {
+          if (i >= rem) break;
+          const uint32_t v = merge_value<DT>(sy[0][i], sy[1][i], NS > 2 ? sy[NS > 2 ? 2 : 0][i] : 0,
+                                             NS > 3 ? sy[NS > 3 ? 3 : 0][i] : 0);
+          uint8_t* p = dst + (uint64_t)(full * GV + i) * VB;
+          if constexpr (VB == 2) *reinterpret_cast<uint16_t*>(p) = (uint16_t)v;
+          else if constexpr (VB == 4) *reinterpret_cast<uint32_t*>(p) = v;
+          else *p = (uint8_t)v;
+        }
       }
     }
 #pragma unroll
@@ -883,7 +905,8 @@ cudaError_t launch_decode(const uint8_t* in, uint64_t in_bytes, const Geo& g, ui
   switch (g.dt) {
     case kBF16: return decode_t<kBF16>(in, in_bytes, g, out, status, st);
     case kFP32: return decode_t<kFP32>(in, in_bytes, g, out, status, st);
-    default: return decode_t<kFP8>(in, in_bytes, g, out, status, st);
+    case kFP8: return decode_t<kFP8>(in, in_bytes, g, out, status, st);
+    default: return decode_t<kFP4>(in, in_bytes, g, out, status, st);
   }
 }
 
@@ -892,7 +915,8 @@ cudaError_t launch_decode_batch(const DecodeItem* items, uint32_t count, const G
   switch (g.dt) {
     case kBF16: return decode_batch_t<kBF16>(items, count, g, total_chunks, status, st);
     case kFP32: return decode_batch_t<kFP32>(items, count, g, total_chunks, status, st);
-    default: return decode_batch_t<kFP8>(items, count, g, total_chunks, status, st);
+    case kFP8: return decode_batch_t<kFP8>(items, count, g, total_chunks, status, st);
+    default: return decode_batch_t<kFP4>(items, count, g, total_chunks, status, st);
   }
 }
 

@@ -50,8 +50,8 @@ struct EncodeSmem {
 template <int DT>
 __global__ void __launch_bounds__(kEncodeThreads) k_encode(const uint8_t* __restrict__ src, Geo g, Ws ws,
                                                            uint8_t* __restrict__ out) {
-  constexpr int NS = n_streams(DT), NE = n_entropy(DT), VB = value_bytes(DT);
-  constexpr int NB = DT == kFP8 ? 3 : 1;  // streams that may be bit-packed
+  constexpr int NS = n_streams(DT), NE = n_entropy(DT);
+  constexpr int NB = DT == kFP8 || DT == kFP4 ? 3 : 1;  // streams that may be bit-packed
   extern __shared__ __align__(16) uint8_t smem_raw[];
   EncodeSmem<DT>& sm = *reinterpret_cast<EncodeSmem<DT>*>(smem_raw);
   const int tid = threadIdx.x;
@@ -68,7 +68,7 @@ __global__ void __launch_bounds__(kEncodeThreads) k_encode(const uint8_t* __rest
   const uint32_t v0 = tlo + tid * kEncValues;  // chunk-relative index of my first value
   const int cnt = v0 < m ? (int)min32(kEncValues, m - v0) : 0;
   RawValues<DT, kEncValues> raw;
-  if (cnt > 0) load_values<DT, kEncValues>(src + (clo + v0) * VB, cnt, raw);
+  if (cnt > 0) load_values<DT, kEncValues>(src + value_offset(DT, clo + v0), cnt, raw);
 
   if (tid < NS) {
     const uint64_t k = (uint64_t)c * NS + tid;
@@ -273,11 +273,12 @@ static cudaError_t encode_t(const void* src, const Geo& g, const Ws& ws, uint8_t
   return cudaGetLastError();
 }
 
-// FP32 and FP8 (BF16 has k_encode_bf16).
+// FP32, FP8 and FP4 (BF16 has k_encode_bf16).
 cudaError_t launch_encode(const void* src, const Geo& g, const Ws& ws, uint8_t* out, cudaStream_t st) {
   switch (g.dt) {
     case kFP32: return encode_t<kFP32>(src, g, ws, out, st);
     case kFP8: return encode_t<kFP8>(src, g, ws, out, st);
+    case kFP4: return encode_t<kFP4>(src, g, ws, out, st);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -95,7 +95,7 @@ template <int DT>
 __global__ void __launch_bounds__(kHistThreads) k_split_hist(const uint8_t* __restrict__ src, Geo g, uint32_t slices,
                                                              uint32_t* __restrict__ hist, uint32_t* __restrict__ nonzero,
                                                              Ws ws, PlanDev plan, int build) {
-  constexpr int NS = n_streams(DT), NE = n_entropy(DT), VB = value_bytes(DT);
+  constexpr int NS = n_streams(DT), NE = n_entropy(DT);
   constexpr int A0 = alphabet(DT, 0), A1 = NE > 1 ? alphabet(DT, 1) : 0;
   extern __shared__ __align__(16) uint8_t smem_raw[];  // histogram columns, then the code builder
   uint32_t* sh = reinterpret_cast<uint32_t*>(smem_raw);
@@ -118,7 +118,7 @@ __global__ void __launch_bounds__(kHistThreads) k_split_hist(const uint8_t* __re
     const int cnt = v0 < hi ? (int)min32(NV, hi - v0) : 0;
     if (cnt > 0) {
       RawValues<DT, NV> raw;
-      load_values<DT, NV>(src + (clo + v0) * VB, cnt, raw);
+      load_values<DT, NV>(src + value_offset(DT, clo + v0), cnt, raw);
       bool done = false;
       if constexpr (DT == kBF16) {
         if (cnt == NV) {
@@ -348,7 +348,8 @@ cudaError_t launch_split_hist(const void* src, const Geo& g, uint32_t* hist, uin
   switch (g.dt) {
     case kBF16: return split_hist_t<kBF16>(src, g, hist, nonzero, ws, plan, st);
     case kFP32: return split_hist_t<kFP32>(src, g, hist, nonzero, ws, plan, st);
-    default: return split_hist_t<kFP8>(src, g, hist, nonzero, ws, plan, st);
+    case kFP8: return split_hist_t<kFP8>(src, g, hist, nonzero, ws, plan, st);
+    default: return split_hist_t<kFP4>(src, g, hist, nonzero, ws, plan, st);
   }
 }
 
@@ -386,7 +387,8 @@ cudaError_t launch_layout(const Geo& g, const Ws& ws, const PlanDev& plan, uint8
   switch (g.dt) {
     case kBF16: return layout_t<kBF16>(g, ws, plan, out, st);
     case kFP32: return layout_t<kFP32>(g, ws, plan, out, st);
-    default: return layout_t<kFP8>(g, ws, plan, out, st);
+    case kFP8: return layout_t<kFP8>(g, ws, plan, out, st);
+    default: return layout_t<kFP4>(g, ws, plan, out, st);
   }
 }
 

@@ -82,6 +82,29 @@ def fp8_tensor(rows=262144, cols=4096, seed=0, device="cpu", block_rows=16384):
     return out.reshape(-1)
 
 
+# E2M1 magnitudes in code order (codes 0..7) and the midpoints between them
+FP4_GRID = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
+FP4_MIDPOINTS = (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0)
+
+
+def fp4_tensor(rows=262144, cols=4096, seed=0, device="cpu", block_rows=16384):
+    """The FP8 recipe in FP4 (E2M1): N(0, 1) times a per-row scale log-uniform in
+    [0.25, 4], rounded to the nearest E2M1 value (ties to the smaller magnitude),
+    saturating at 6. Returns rows * cols values as torch.float4_e2m1fn_x2 (value 2i in
+    the low nibble of element i)."""
+    g = torch.Generator(device).manual_seed(seed)
+    lo, hi = math.log(0.25), math.log(4.0)
+    scale = torch.exp(lo + (hi - lo) * torch.rand(rows, 1, generator=g, device=device))
+    mids = torch.tensor(FP4_MIDPOINTS, device=device)
+    out = torch.empty(rows, cols // 2, dtype=torch.uint8, device=device)
+    for r in range(0, rows, block_rows):
+        r2 = min(rows, r + block_rows)
+        x = torch.randn(r2 - r, cols, generator=g, device=device) * scale[r:r2]
+        code = torch.bucketize(x.abs(), mids) | ((x < 0).to(torch.int64) << 3)
+        out[r:r2] = (code[:, 0::2] | (code[:, 1::2] << 4)).to(torch.uint8)
+    return out.reshape(-1).view(torch.float4_e2m1fn_x2)
+
+
 def kv_cache(shape=(32, 2, 16, 8, 4096, 128), seed=0, device="cpu"):
     layers, kv, batch, heads, seq, dim = shape
     g = torch.Generator(device).manual_seed(seed)

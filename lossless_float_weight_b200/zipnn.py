@@ -19,7 +19,7 @@ if not os.path.exists(LIB_PATH):
 
 _lib = ctypes.CDLL(LIB_PATH)
 
-BF16, FP32, FP8_E4M3 = 0, 1, 2
+BF16, FP32, FP8_E4M3, FP4_E2M1 = 0, 1, 2, 3
 OK, ERR_INVALID_ARG, ERR_OUT_TOO_SMALL, ERR_CORRUPT, ERR_PLAN_MISMATCH, ERR_CUDA, ERR_UNSUPPORTED, ERR_TIMEOUT = range(8)
 DEFAULT_CHUNK_BYTES = 262144
 DEFAULT_SUBBLOCK = 512
@@ -92,15 +92,24 @@ def check(status, what=""):
 
 # ------------------------------------------------------------------ tensor helpers
 
-_TORCH_DTYPES = {torch.bfloat16: BF16, torch.float32: FP32, torch.float8_e4m3fn: FP8_E4M3}
-_VALUE_BYTES = {BF16: 2, FP32: 4, FP8_E4M3: 1}
+# torch.float4_e2m1fn_x2 holds two FP4 values per element (one byte, the first value in
+# the low nibble); the codec counts values, so n is twice numel() for it
+_TORCH_DTYPES = {torch.bfloat16: BF16, torch.float32: FP32, torch.float8_e4m3fn: FP8_E4M3,
+                 torch.float4_e2m1fn_x2: FP4_E2M1}
+_VALUES_PER_ELEMENT = {BF16: 1, FP32: 1, FP8_E4M3: 1, FP4_E2M1: 2}
+_VALUES_PER_BYTE = {BF16: 0.5, FP32: 0.25, FP8_E4M3: 1, FP4_E2M1: 2}
+
+
+def nvalues(x):
+    """Values held by the tensor x (FP4: two per element)."""
+    return x.numel() * _VALUES_PER_ELEMENT[dtype_code(x.dtype)]
 
 
 def dtype_code(x):
     if isinstance(x, int):
         return x
     if isinstance(x, str):
-        return {"bf16": BF16, "fp32": FP32, "fp8_e4m3": FP8_E4M3}[x]
+        return {"bf16": BF16, "fp32": FP32, "fp8_e4m3": FP8_E4M3, "fp4_e2m1": FP4_E2M1}[x]
     return _TORCH_DTYPES[x]
 
 
@@ -129,9 +138,9 @@ class Plan:
         dt = dtype_code(x.dtype)
         xf = x.reshape(-1)
         if ws is None:
-            ws = workspace(dt, xf.numel(), chunk_bytes, xf.device)
+            ws = workspace(dt, nvalues(xf), chunk_bytes, xf.device)
         h = _vp()
-        check(zipnn_plan_create(dt, xf.data_ptr(), xf.numel(), chunk_bytes, groups, seed, ws.data_ptr(),
+        check(zipnn_plan_create(dt, xf.data_ptr(), nvalues(xf), chunk_bytes, groups, seed, ws.data_ptr(),
                                 ws.numel(), _stream(stream), ctypes.byref(h)), "zipnn_plan_create")
         return cls(h.value, dt)
 
@@ -171,7 +180,7 @@ class Plan:
 def compress_into(x, out, ws, chunk_bytes=DEFAULT_CHUNK_BYTES, plan=None, subblock=0, stream=None):
     """Asynchronous: compress the device tensor x into the device byte tensor out."""
     dt = dtype_code(x.dtype)
-    check(zipnn_compress_ex(dt, x.data_ptr(), x.numel(), chunk_bytes, subblock, plan.handle if plan else None,
+    check(zipnn_compress_ex(dt, x.data_ptr(), nvalues(x), chunk_bytes, subblock, plan.handle if plan else None,
                             out.data_ptr(), out.numel(), ws.data_ptr(), ws.numel(), _stream(stream)),
           "zipnn_compress")
 
@@ -179,7 +188,7 @@ def compress_into(x, out, ws, chunk_bytes=DEFAULT_CHUNK_BYTES, plan=None, subblo
 def decompress_into(container, nbytes, out, ws, chunk_bytes=DEFAULT_CHUNK_BYTES, stream=None):
     """Asynchronous: decompress nbytes of the device container into the device tensor out."""
     dt = dtype_code(out.dtype)
-    check(zipnn_decompress(dt, container.data_ptr(), nbytes, out.numel(), chunk_bytes, out.data_ptr(),
+    check(zipnn_decompress(dt, container.data_ptr(), nbytes, nvalues(out), chunk_bytes, out.data_ptr(),
                            ws.data_ptr(), ws.numel(), _stream(stream)), "zipnn_decompress")
 
 
@@ -196,7 +205,7 @@ def decompress_batch_into(containers, nbytes, outs, ws, chunk_bytes=DEFAULT_CHUN
     dt = dtype_code(outs[0].dtype)
     if any(dtype_code(o.dtype) != dt for o in outs):
         raise ZipnnError(ERR_INVALID_ARG, "zipnn_decompress_batch: one dtype per batch")
-    items = (DecompressItem * len(outs))(*[DecompressItem(c.data_ptr(), b, o.numel(), o.data_ptr())
+    items = (DecompressItem * len(outs))(*[DecompressItem(c.data_ptr(), b, nvalues(o), o.data_ptr())
                                             for c, b, o in zip(containers, nbytes, outs)])
     check(zipnn_decompress_batch(dt, chunk_bytes, len(outs), items, ws.data_ptr(), ws.numel(), _stream(stream)),
           "zipnn_decompress_batch")
@@ -216,11 +225,11 @@ def compress(x, chunk_bytes=DEFAULT_CHUNK_BYTES, plan=None, subblock=0, stream=N
     """Compress a CUDA tensor; returns the container as a CUDA uint8 tensor (synchronises)."""
     xf = x.reshape(-1)
     dt = dtype_code(xf.dtype)
-    cap = zipnn_max_compressed_bytes(dt, xf.numel(), chunk_bytes)
+    cap = zipnn_max_compressed_bytes(dt, nvalues(xf), chunk_bytes)
     if cap == 0:
         raise ZipnnError(ERR_INVALID_ARG, "zipnn_max_compressed_bytes")
     out = torch.empty(cap, dtype=torch.uint8, device=xf.device)
-    ws = workspace(dt, xf.numel(), chunk_bytes, xf.device)
+    ws = workspace(dt, nvalues(xf), chunk_bytes, xf.device)
     compress_into(xf, out, ws, chunk_bytes, plan, subblock, stream)
     size = compressed_size(out, stream)
     check(status(ws, stream), "compress status")
@@ -228,7 +237,8 @@ def compress(x, chunk_bytes=DEFAULT_CHUNK_BYTES, plan=None, subblock=0, stream=N
 
 
 def decompress(container, dtype, shape, chunk_bytes=DEFAULT_CHUNK_BYTES, stream=None):
-    """Decompress a CUDA container into a new CUDA tensor of the given dtype and shape."""
+    """Decompress a CUDA container into a new CUDA tensor of the given dtype and shape
+    (in elements of dtype: for torch.float4_e2m1fn_x2, pairs of values)."""
     n = 1
     for d in (shape if isinstance(shape, (tuple, list, torch.Size)) else (shape,)):
         n *= d
@@ -271,11 +281,11 @@ def histogram(x, chunk_bytes=DEFAULT_CHUNK_BYTES, stream=None):
     """Per-chunk order-0 histograms of the entropy streams: (n_chunks, n_entropy, 256) int32."""
     xf = x.reshape(-1)
     dt = dtype_code(xf.dtype)
-    m0 = chunk_bytes // _VALUE_BYTES[dt]
-    C = -(-xf.numel() // m0)
-    ne = 2 if dt == FP8_E4M3 else 1
+    m0 = int(chunk_bytes * _VALUES_PER_BYTE[dt])
+    C = -(-nvalues(xf) // m0)
+    ne = 2 if dt in (FP8_E4M3, FP4_E2M1) else 1
     out = torch.zeros((C, ne, 256), dtype=torch.int32, device=xf.device)
-    check(zipnn_histogram(dt, xf.data_ptr(), xf.numel(), chunk_bytes, out.data_ptr(), _stream(stream)),
+    check(zipnn_histogram(dt, xf.data_ptr(), nvalues(xf), chunk_bytes, out.data_ptr(), _stream(stream)),
           "zipnn_histogram")
     return out
 

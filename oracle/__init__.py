@@ -10,8 +10,18 @@ import numpy as np
 
 from . import build as _build
 
-DTYPES = {"bf16": 0, "fp32": 1, "fp8_e4m3": 2}
-VALUE_BYTES = {"bf16": 2, "fp32": 4, "fp8_e4m3": 1}
+DTYPES = {"bf16": 0, "fp32": 1, "fp8_e4m3": 2, "fp4_e2m1": 3}
+VALUES_PER_BYTE = {"bf16": 0.5, "fp32": 0.25, "fp8_e4m3": 1, "fp4_e2m1": 2}  # FP4: two per byte
+
+
+def values_in(dtype, nbytes):
+    """Values held in nbytes bytes."""
+    return int(nbytes * VALUES_PER_BYTE[dtype])
+
+
+def bytes_of(dtype, n):
+    """Bytes that hold n values (FP4: n is even)."""
+    return int(n / VALUES_PER_BYTE[dtype])
 OK, EINVAL, ESMALL, ECORRUPT, EPLAN = 0, 1, 2, 3, 4
 LMAX = 12
 
@@ -105,8 +115,8 @@ def compress(dtype, data, n=None, chunk_bytes=262144, S=512, plan_lens=None, thr
     """Return the container (numpy uint8) for the n values held in data."""
     b = _bytes_view(data)
     if n is None:
-        n = b.size // VALUE_BYTES[dtype]
-    assert b.size >= n * VALUE_BYTES[dtype]
+        n = values_in(dtype, b.size)
+    assert b.size >= bytes_of(dtype, n)
     G = 0
     plan_ptr = None
     if plan_lens is not None:
@@ -126,7 +136,7 @@ def compress(dtype, data, n=None, chunk_bytes=262144, S=512, plan_lens=None, thr
 def decompress(dtype, container, n, chunk_bytes=262144, threads=1):
     """Return the n decoded values as raw bytes (numpy uint8)."""
     c = np.ascontiguousarray(container, dtype=np.uint8)
-    out = np.zeros(n * VALUE_BYTES[dtype], dtype=np.uint8)
+    out = np.zeros(bytes_of(dtype, n), dtype=np.uint8)
     st = lib().orc_decompress(DTYPES[dtype], c.ctypes.data, c.size, n, chunk_bytes, out.ctypes.data, threads)
     if st != OK:
         raise OracleError(st)
@@ -135,7 +145,7 @@ def decompress(dtype, container, n, chunk_bytes=262144, threads=1):
 
 def decompress_status(dtype, container, n, chunk_bytes=262144):
     c = np.ascontiguousarray(container, dtype=np.uint8)
-    out = np.zeros(n * VALUE_BYTES[dtype], dtype=np.uint8)
+    out = np.zeros(bytes_of(dtype, n), dtype=np.uint8)
     return lib().orc_decompress(DTYPES[dtype], c.ctypes.data, c.size, n, chunk_bytes, out.ctypes.data, 1)
 
 
@@ -147,8 +157,8 @@ def plan_build(dtype, data, n=None, chunk_bytes=262144, groups=8, seed=0):
     """Return (lens[n_entropy, groups, 256], assign[n_chunks], iterations, inertia list)."""
     b = _bytes_view(data)
     if n is None:
-        n = b.size // VALUE_BYTES[dtype]
-    m0 = chunk_bytes // VALUE_BYTES[dtype]
+        n = values_in(dtype, b.size)
+    m0 = values_in(dtype, chunk_bytes)
     C = -(-n // m0)
     lens = np.zeros((n_entropy(dtype), groups, 256), dtype=np.uint8)
     assign = np.zeros(C, dtype=np.uint32)

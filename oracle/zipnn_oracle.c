@@ -48,12 +48,15 @@
 /* ------------------------------------------------------------------ field map */
 
 int orc_n_streams(int dtype) { return dtype == ORC_BF16 ? 2 : dtype == ORC_FP32 ? 4 : 3; }
-int orc_n_entropy(int dtype) { return dtype == ORC_FP8 ? 2 : 1; }
+/* FP8 and FP4: exponent and mantissa are entropy-coded independently */
+int orc_n_entropy(int dtype) { return dtype == ORC_FP8 || dtype == ORC_FP4 ? 2 : 1; }
+/* bytes of one value (FP4: two values share a byte; see chunk_values) */
 static int value_bytes(int dtype) { return dtype == ORC_BF16 ? 2 : dtype == ORC_FP32 ? 4 : 1; }
-static int is_entropy(int dtype, int s) { return s == 0 || (dtype == ORC_FP8 && s == 1); }
+static int is_entropy(int dtype, int s) { return s == 0 || ((dtype == ORC_FP8 || dtype == ORC_FP4) && s == 1); }
 /* bits per symbol when a stream is stored RAW */
 static int raw_width(int dtype, int s) {
   if (dtype == ORC_FP8) return s == 0 ? 4 : s == 1 ? 3 : 1;
+  if (dtype == ORC_FP4) return s == 0 ? 2 : 1;
   return 8;
 }
 int orc_alphabet(int dtype, int s) { return 1 << raw_width(dtype, s); }
@@ -64,7 +67,9 @@ static uint64_t record_bytes(int dtype, int s) { return round16((uint64_t)orc_al
 /* The split. BF16 w: exponent = bits 14..7; sign+fraction byte = sign in bit 7,
  * fraction bits 6..0. FP32 u: exponent = bits 30..23; p1 = sign + fraction bits
  * 22..16; p2 = fraction bits 15..8; p3 = bits 7..0. FP8 E4M3 b: exponent bits 6..3,
- * mantissa bits 2..0, sign bit 7. Streams are numbered in that order. */
+ * mantissa bits 2..0, sign bit 7. FP4 E2M1: value i is the low nibble of byte i/2
+ * when i is even, the high nibble when odd; exponent = nibble bits 2..1, mantissa =
+ * bit 0, sign = bit 3. Streams are numbered in that order. */
 uint8_t orc_field(int dtype, const uint8_t* src, uint64_t i, int s) {
   if (dtype == ORC_BF16) {
     uint32_t w = (uint32_t)src[2 * i] | ((uint32_t)src[2 * i + 1] << 8);
@@ -78,6 +83,12 @@ uint8_t orc_field(int dtype, const uint8_t* src, uint64_t i, int s) {
     if (s == 1) return (uint8_t)(((u >> 24) & 0x80) | ((u >> 16) & 0x7F));
     if (s == 2) return (uint8_t)((u >> 8) & 0xFF);
     return (uint8_t)(u & 0xFF);
+  }
+  if (dtype == ORC_FP4) {
+    uint32_t v = (src[i / 2] >> (4 * (i % 2))) & 0xF;
+    if (s == 0) return (uint8_t)((v >> 1) & 3);
+    if (s == 1) return (uint8_t)(v & 1);
+    return (uint8_t)(v >> 3);
   }
   {
     uint32_t b = src[i];
@@ -100,6 +111,10 @@ static void put_value(int dtype, uint8_t* dst, uint64_t i, const uint8_t* f) {
     dst[4 * i + 1] = (uint8_t)((u >> 8) & 0xFF);
     dst[4 * i + 2] = (uint8_t)((u >> 16) & 0xFF);
     dst[4 * i + 3] = (uint8_t)(u >> 24);
+  } else if (dtype == ORC_FP4) {
+    uint32_t v = ((uint32_t)f[2] << 3) | ((uint32_t)f[0] << 1) | f[1];
+    uint32_t sh = 4 * (uint32_t)(i % 2);
+    dst[i / 2] = (uint8_t)((dst[i / 2] & ~(0xFu << sh)) | (v << sh));
   } else {
     dst[i] = (uint8_t)((f[2] << 7) | (f[0] << 3) | f[1]);
   }
@@ -243,7 +258,11 @@ static uint64_t get_u64(const uint8_t* p) {
 
 static uint64_t ceil_div(uint64_t a, uint64_t b) { return (a + b - 1) / b; }
 
-static uint64_t chunk_values(int dtype, uint32_t chunk_bytes) { return chunk_bytes / (uint32_t)value_bytes(dtype); }
+static uint64_t chunk_values(int dtype, uint32_t chunk_bytes) {
+  return dtype == ORC_FP4 ? 2 * (uint64_t)chunk_bytes : chunk_bytes / (uint32_t)value_bytes(dtype);
+}
+/* FP4 values come in byte pairs */
+static int bad_count(int dtype, uint64_t n) { return n == 0 || (dtype == ORC_FP4 && n % 2 != 0); }
 
 static uint64_t table_end(int dtype, uint64_t n_chunks) {
   return HEADER_BYTES + (uint64_t)ENTRY_BYTES * n_chunks * (uint64_t)orc_n_streams(dtype);
@@ -435,7 +454,7 @@ static int run_jobs(job_t* base, int threads, void* (*fn)(void*)) {
 int orc_compress(int dtype, const void* src, uint64_t n, uint32_t chunk_bytes, uint32_t S,
                  const uint8_t* plan_lens, uint32_t n_groups, void* out, uint64_t cap,
                  uint64_t* out_bytes, int threads) {
-  if (dtype < 0 || dtype > 2 || !src || !out || n == 0 || S == 0) return ORC_EINVAL;
+  if (dtype < 0 || dtype > 3 || !src || !out || bad_count(dtype, n) || S == 0) return ORC_EINVAL;
   if (chunk_bytes == 0 || chunk_bytes % (uint32_t)value_bytes(dtype) != 0) return ORC_EINVAL;
   if (plan_lens && (n_groups == 0 || n_groups > MAX_GROUPS)) return ORC_EINVAL;
   if (!plan_lens) n_groups = 0;
@@ -655,7 +674,7 @@ static void* decompress_worker(void* arg) {
 int orc_decompress(int dtype, const void* in, uint64_t in_bytes, uint64_t n, uint32_t chunk_bytes,
                    void* out, int threads) {
   const uint8_t* h = (const uint8_t*)in;
-  if (dtype < 0 || dtype > 2 || !in || !out || n == 0) return ORC_EINVAL;
+  if (dtype < 0 || dtype > 3 || !in || !out || bad_count(dtype, n)) return ORC_EINVAL;
   if (chunk_bytes == 0 || chunk_bytes % (uint32_t)value_bytes(dtype) != 0) return ORC_EINVAL;
   if (in_bytes < HEADER_BYTES) return ORC_ECORRUPT;
   if (h[0] != 'Z' || h[1] != 'N' || h[2] != 'N' || h[3] != '1' || h[4] != 1 || h[5] != 0) return ORC_ECORRUPT;
@@ -744,7 +763,7 @@ static double sq_distance(const double* a, const double* b, int dims) {
 int orc_plan_build(int dtype, const void* src, uint64_t n, uint32_t chunk_bytes, uint32_t n_groups,
                    uint64_t seed, uint8_t* lens_out, uint32_t* assign_out, int* iters_out,
                    double* inertia_out) {
-  if (dtype < 0 || dtype > 2 || !src || n == 0 || n_groups == 0 || n_groups > MAX_GROUPS) return ORC_EINVAL;
+  if (dtype < 0 || dtype > 3 || !src || bad_count(dtype, n) || n_groups == 0 || n_groups > MAX_GROUPS) return ORC_EINVAL;
   if (chunk_bytes == 0 || chunk_bytes % (uint32_t)value_bytes(dtype) != 0) return ORC_EINVAL;
   const uint8_t* in = (const uint8_t*)src;
   int E = orc_n_entropy(dtype), A = orc_alphabet(dtype, 0);

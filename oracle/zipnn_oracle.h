@@ -12,7 +12,8 @@
  *  - THEORY-599, "Order-0 only (section III-A b)": one order-0 model (a symbol
  *    histogram) per chunk, Huffman-coded after the exponent is extracted.
  *  - "Lossless Compression of Neural Network Components ... in Low-Precision
- *    Formats" (abstract): FP8 exponent and mantissa entropy-coded independently.
+ *    Formats" (abstract): FP8 and FP4 exponent and mantissa entropy-coded
+ *    independently.
  *  - "NeuralZip: Reusable Setup for Fast Lossless Compression" (abstract): chunks
  *    grouped by exponent-distribution similarity share one Huffman code, chosen
  *    once by a reusable setup (the plan).
@@ -34,6 +35,7 @@ extern "C" {
 #define ORC_BF16 0
 #define ORC_FP32 1
 #define ORC_FP8 2
+#define ORC_FP4 3
 
 /* return codes */
 #define ORC_OK 0

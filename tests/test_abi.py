@@ -45,6 +45,10 @@ def test_sizes_match_the_oracle(lib, orc):
     assert Z.zipnn_max_compressed_bytes(Z.BF16, 0, 262144) == 0
     assert Z.zipnn_max_compressed_bytes(Z.BF16, 10, 100) == 0      # not a multiple of 16
     assert Z.zipnn_max_compressed_bytes(7, 10, 262144) == 0        # bad dtype
+    for n in (2, 18, 524288, 524290, 2 * 10 ** 7 + 6):               # FP4: values in pairs
+        for cb in (4096, 262144):
+            assert Z.zipnn_max_compressed_bytes(Z.FP4_E2M1, n, cb) == orc.max_compressed_bytes("fp4_e2m1", n, cb, 64)
+    assert Z.zipnn_max_compressed_bytes(Z.FP4_E2M1, 7, 262144) == 0  # an odd FP4 count
 
 
 def test_argument_errors_without_a_device(lib):

@@ -31,11 +31,12 @@ def _host_bytes(t):
 
 
 def _check_roundtrip(z, orc, x, name, chunk_bytes=CB, subblock=S_DEFAULT, plan=None, plan_lens=None):
-    dtype = {torch.bfloat16: "bf16", torch.float32: "fp32", torch.float8_e4m3fn: "fp8_e4m3"}[x.dtype]
+    dtype = {torch.bfloat16: "bf16", torch.float32: "fp32", torch.float8_e4m3fn: "fp8_e4m3",
+             torch.float4_e2m1fn_x2: "fp4_e2m1"}[x.dtype]
     xd = x.reshape(-1).cuda()
     cont = z.compress(xd, chunk_bytes=chunk_bytes, plan=plan, subblock=subblock)
     got = cont.cpu().numpy()
-    ref = orc.compress(dtype, _host_bytes(x), x.numel(), chunk_bytes=chunk_bytes, S=subblock, plan_lens=plan_lens,
+    ref = orc.compress(dtype, _host_bytes(x), z.nvalues(x), chunk_bytes=chunk_bytes, S=subblock, plan_lens=plan_lens,
                        threads=8)
     assert got.size == ref.size, f"{name}: size {got.size} != oracle {ref.size}"
     bad = np.nonzero(got != ref)[0]
@@ -122,6 +123,51 @@ def test_fp8(z, orc):
     q = torch.cat([q, q[:777]])
     c = _check_roundtrip(z, orc, q, "fp8")
     assert c.size / q.numel() < 0.9
+
+
+def _fp4(raw):
+    return torch.from_numpy(np.ascontiguousarray(raw, dtype=np.uint8)).view(torch.float4_e2m1fn_x2)
+
+
+def test_fp4(z, orc):
+    from lossless_float_weight_b200 import workloads as W
+    q = W.fp4_tensor(rows=512, cols=4096)  # 2,097,152 values, 4 chunks
+    got = _check_roundtrip(z, orc, q, "fp4")
+    assert got.size < 0.95 * q.numel()  # the exponent plane compresses
+    _check_roundtrip(z, orc, q, "fp4 S=64", chunk_bytes=65536, subblock=64)
+
+
+def test_every_fp4_byte_pattern_and_ragged_sizes(z, orc):
+    pats = np.arange(256, dtype=np.uint8)
+    rng = np.random.default_rng(11)
+    _check_roundtrip(z, orc, _fp4(np.tile(pats, 64)), "fp4 patterns", chunk_bytes=4096, subblock=64)
+    _check_roundtrip(z, orc, _fp4(rng.permutation(np.tile(pats, 700))), "fp4 shuffled", chunk_bytes=65536)
+    for nbytes in (1, 9, 8192, 8193, 131073, 200001):  # 2 .. 400002 values; ragged last chunks
+        _check_roundtrip(z, orc, _fp4(rng.integers(0, 256, nbytes, dtype=np.uint8)), f"fp4 {nbytes} B",
+                         chunk_bytes=65536)
+    # FP4 values come in pairs: an odd count is an argument error
+    out = torch.empty(1024, dtype=torch.uint8, device="cuda")
+    ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
+    assert z.zipnn_compress(z.FP4_E2M1, out.data_ptr(), 7, CB, None, out.data_ptr(), out.numel(), ws.data_ptr(),
+                            ws.numel(), None) == z.ERR_INVALID_ARG
+
+
+def test_fp4_plan_and_batch(z, orc):
+    from lossless_float_weight_b200 import workloads as W
+    q = W.fp4_tensor(rows=1024, cols=4096, seed=2)  # 16 chunks of 64 KiB
+    plan = z.Plan.create(q.cuda(), groups=4, seed=1, chunk_bytes=65536)
+    lens, assign, _, _ = orc.plan_build("fp4_e2m1", _host_bytes(q), z.nvalues(q), 65536, groups=4, seed=1)
+    assert plan.assignment() == assign.tolist()
+    _check_roundtrip(z, orc, q, "fp4 plan", chunk_bytes=65536, plan=plan, plan_lens=lens)
+    xs = [W.fp4_tensor(rows=r, cols=4096, seed=r, device="cuda") for r in (1, 64, 300)]
+    conts = [z.compress(x, chunk_bytes=65536) for x in xs]
+    outs = [torch.empty_like(x) for x in xs]
+    ws = z.batch_workspace(len(xs))
+    z.decompress_batch_into(conts, [c.numel() for c in conts], outs, ws, 65536)
+    torch.cuda.synchronize()
+    assert z.status(ws) == z.OK
+    for x, y in zip(xs, outs):
+        assert torch.equal(y.view(torch.uint8), x.view(torch.uint8))
 
 
 def test_histogram_entry_point(z, orc):

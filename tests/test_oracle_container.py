@@ -34,7 +34,7 @@ def test_golden_shared_code(orc):
 
 def _roundtrip(orc, dtype, x, chunk_bytes, S=1024, threads=1):
     raw = orc._bytes_view(x)
-    n = raw.size // orc.VALUE_BYTES[dtype]
+    n = orc.values_in(dtype, raw.size)
     c = orc.compress(dtype, raw, n, chunk_bytes=chunk_bytes, S=S, threads=threads)
     assert c.size <= orc.max_compressed_bytes(dtype, n, chunk_bytes)
     assert c.size % 16 == 0
