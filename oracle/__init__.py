@@ -150,7 +150,7 @@ def decompress_status(dtype, container, n, chunk_bytes=262144):
 
 
 def n_entropy(dtype):
-    return 2 if dtype == "fp8_e4m3" else 1
+    return 2 if dtype in ("fp8_e4m3", "fp4_e2m1") else 1
 
 
 def plan_build(dtype, data, n=None, chunk_bytes=262144, groups=8, seed=0):

@@ -81,3 +81,15 @@ def test_quantised_gaussian_compresses(orc):
     c = _roundtrip(orc, raw, 262144)
     # the exponent plane is skewed, so the container is smaller than the input
     assert c.size < 0.95 * raw.size
+
+
+def test_plan_with_two_entropy_streams(orc):
+    # a plan holds one code per group for the exponent and one for the mantissa
+    rng = np.random.default_rng(8)
+    raw = rng.choice(np.array([0x10, 0x21, 0x32, 0x05, 0x13, 0x20], dtype=np.uint8), size=1 << 18)
+    n = orc.values_in("fp4_e2m1", raw.size)
+    lens, assign, iters, _ = orc.plan_build("fp4_e2m1", raw, n, 16384, groups=3, seed=0)
+    assert lens.shape == (2, 3, 256) and assign.size == 16 and iters >= 1
+    assert np.all(lens[0, :, 4:] == 0) and np.all(lens[1, :, 2:] == 0)  # alphabets of 4 and 2
+    c = orc.compress("fp4_e2m1", raw, n, chunk_bytes=16384, plan_lens=lens)
+    assert np.array_equal(orc.decompress("fp4_e2m1", c, n, chunk_bytes=16384), raw)
