@@ -385,7 +385,9 @@ def run_e2e(Z, xs, csizes, dev, stream, streams, args, world):
     """Same metric through the public API with host buffers: pinned host tensors in,
     pinned host tensors out. Every step copies each tensor to the device, compresses
     it, reads its size and copies the container back, then copies each container to
-    the device, decompresses them (one batched call) and copies the values back."""
+    the device, decompresses it and copies the values back. Tensors go round-robin to the
+    streams, so host transfers in both directions overlap the kernels (one batched
+    decompress would wait for every container before any value could go back)."""
     nbytes = sum(x.numel() * 2 for x in xs)
     h_in = [x.cpu().pin_memory() for x in xs]
     h_cont = [torch.empty(c, dtype=torch.uint8).pin_memory() for c in csizes]
@@ -395,7 +397,6 @@ def run_e2e(Z, xs, csizes, dev, stream, streams, args, world):
               for x in xs]
     d_out = [torch.empty_like(x) for x in xs]
     wss = [Z.workspace(Z.BF16, max(x.numel() for x in xs), CHUNK, dev) for _ in streams]
-    bws = Z.batch_workspace(len(xs), dev)
     ns = len(streams)
 
     def step():
@@ -417,19 +418,13 @@ def run_e2e(Z, xs, csizes, dev, stream, streams, args, world):
             s = streams[i % ns]
             with torch.cuda.stream(s):
                 d_cont[i][: csizes[i]].copy_(h_cont[i], non_blocking=True)
-            if args.per_tensor_decode:
-                Z.decompress_into(d_cont[i], csizes[i], d_out[i], wss[i % ns], CHUNK, stream=s)
-                with torch.cuda.stream(s):
-                    h_out[i].copy_(d_out[i], non_blocking=True)
+            Z.decompress_into(d_cont[i], csizes[i], d_out[i], wss[i % ns], CHUNK, stream=s)
+            with torch.cuda.stream(s):
+                h_out[i].copy_(d_out[i], non_blocking=True)
         for s in streams:
             e2 = torch.cuda.Event()
             e2.record(s)
             stream.wait_event(e2)
-        if not args.per_tensor_decode:
-            Z.decompress_batch_into(d_cont, csizes, d_out, bws, CHUNK, stream=stream)
-            with torch.cuda.stream(stream):
-                for i in range(len(xs)):
-                    h_out[i].copy_(d_out[i], non_blocking=True)
 
     steps = max(1, min(args.steps, 3))
     step()
