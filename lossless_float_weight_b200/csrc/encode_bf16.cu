@@ -6,8 +6,10 @@
 // count(tile, e) * len(e). The histogram pass counts per tile and the code build turns
 // the counts into tile offsets, so every tile knows its offset before it packs a bit.
 // Blocks are persistent: each takes tiles blockIdx.x, blockIdx.x + gridDim.x, ... and
-// encodes a tile in two passes of 16384 values (256 threads of 64); the second pass
-// starts where the first one's bits end. In each pass it
+// encodes a tile in passes of kBPassValues values (kBThreads threads of 64 values);
+// each pass starts where the previous one's bits end. Small blocks (four warps, eight
+// per SM) keep the barriers of a pass short and let the blocks' load and compute phases
+// interleave. In each pass it
 //  * loads its 64 values per thread (128-bit loads) and writes the sign/fraction plane
 //    (and an exponent plane that did not compress) with 16-byte stores;
 //  * packs its exponent codes, two per step, most significant bit first, into private
@@ -15,8 +17,7 @@
 //  * moves the private words into a staging copy of the tile's bitstream at its final
 //    alignment (shared atomicOr on each thread's two edge words), then stores it with
 //    coalesced 32-bit stores, clearing the staging words as it reads them. The word
-//    shared by the two passes is carried in shared memory into the second pass's first
-//    word. A word that straddles two tiles is merged in a workspace slot: each side adds
+//    shared by two passes is carried in shared memory into the next pass's first word. A word that straddles two tiles is merged in a workspace slot: each side adds
 //    (1 << 32 | its bits) and the side that arrives second stores the complete word.
 // The sub-block index idx[j] (bit offset of symbol j*S) is written by the thread that
 // owns symbol j*S; the first tile writes a local code record, the last the padding.
@@ -26,10 +27,10 @@
 
 namespace zipnn {
 
-constexpr int kBThreads = 256;
+constexpr int kBThreads = 128;
 constexpr int kBValues = kGroupValues * kEncGroups;             // 64 values per thread
-constexpr int kBPassValues = kBThreads * kBValues;              // 16384
-constexpr int kBPasses = kBf16TileValues / kBPassValues;        // 2
+constexpr int kBPassValues = kBThreads * kBValues;              // 8192
+constexpr int kBPasses = kBf16TileValues / kBPassValues;        // 4
 constexpr int kBStageWords = kBPassValues * kLmax / 32 + 2;     // one pass's bitstream
 constexpr int kBPrivStride = kBValues * kLmax / 32 + 1;         // odd: conflict-free
 static_assert(kBPasses * kBPassValues == kBf16TileValues, "a tile is a whole number of passes");
@@ -52,7 +53,7 @@ __device__ __forceinline__ uint32_t bf16_pair_plane(uint32_t w, int s) {
   return s == 0 ? (w >> 7) & 0x00FF00FFu : (w & 0x007F007Fu) | ((w >> 8) & 0x00800080u);
 }
 
-__global__ void __launch_bounds__(kBThreads, 4) k_encode_bf16(const uint8_t* __restrict__ src, Geo g, Ws ws,
+__global__ void __launch_bounds__(kBThreads, 8) k_encode_bf16(const uint8_t* __restrict__ src, Geo g, Ws ws,
                                                                    uint8_t* __restrict__ out) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   Bf16EncodeSmem& sm = *reinterpret_cast<Bf16EncodeSmem*>(smem_raw);
@@ -72,7 +73,7 @@ __global__ void __launch_bounds__(kBThreads, 4) k_encode_bf16(const uint8_t* __r
     const uint64_t off0 = ws.eoff[2ull * c], off1 = ws.eoff[2ull * c + 1];
     uint64_t P = 0;  // the pass's bit offset in the chunk
     if (mode0 == kModeHuff) {
-      sm.enc[tid] = ws.enc[(uint64_t)c * 256 + tid];
+      for (int i = tid; i < 256; i += kBThreads) sm.enc[i] = ws.enc[(uint64_t)c * 256 + i];
       P = ws.tile_off[tile];
     }
     __syncthreads();  // the code is visible; the previous tile's stores and clears are done
@@ -210,8 +211,8 @@ __global__ void __launch_bounds__(kBThreads, 4) k_encode_bf16(const uint8_t* __r
         sm.stage[i] = 0;
         if (i == 0 && pass > 0 && (P & 31) != 0) word |= sm.carry;  // the first pass's last bits
         uint32_t* dst = bs + W0 + i;
-        // (a first pass that is not the tile's last has 16384 values, so i == 0 and the
-        // carried word are never the same word)
+        // (a first pass that is not the tile's last has kBPassValues values, so i == 0 and
+        // the carried word are never the same word)
         if (i == nwt - 1 && (end & 31) != 0 && !tile_end) sm.carry = word;  // completed by the next pass
         else if (i == 0 && pass == 0 && (P & 31) != 0) bf16_slot_merge(ws.slot + tile, word, dst);
         else if (i == nwt - 1 && (end & 31) != 0 && !last) bf16_slot_merge(ws.slot + tile + 1, word, dst);
