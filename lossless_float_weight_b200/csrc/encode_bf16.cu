@@ -131,8 +131,9 @@ __global__ void __launch_bounds__(kBThreads, 8) k_encode_bf16(const uint8_t* __r
       if (mode0 != kModeHuff) continue;  // uniform
 
       // the local code record heads the payload (4-bit lengths)
-      if (rec && ti == 0 && pass == 0 && tid < 128)
-        payload[tid] = (uint8_t)((sm.enc[2 * tid] >> 16) | ((sm.enc[2 * tid + 1] >> 16) << 4));
+      if (rec && ti == 0 && pass == 0)
+        for (int i = tid; i < 128; i += kBThreads)
+          payload[i] = (uint8_t)((sm.enc[2 * i] >> 16) | ((sm.enc[2 * i + 1] >> 16) << 4));
       // pack my codes from bit 0 of my private words
       uint32_t* pw = sm.priv + tid * kBPrivStride;
       uint32_t nw = 0, nfill = 0, mybits = 0;
