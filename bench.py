@@ -386,8 +386,9 @@ def run_e2e(Z, xs, csizes, dev, stream, streams, args, world):
     pinned host tensors out. Every step copies each tensor to the device, compresses
     it, reads its size and copies the container back, then copies each container to
     the device, decompresses it and copies the values back. Tensors go round-robin to the
-    streams, so host transfers in both directions overlap the kernels (one batched
-    decompress would wait for every container before any value could go back)."""
+    streams and the two halves are pipelined (one tensor's upload and compress beside an
+    earlier tensor's container round trip and decompress), so host transfers in both
+    directions overlap each other and the kernels."""
     nbytes = sum(x.numel() * 2 for x in xs)
     h_in = [x.cpu().pin_memory() for x in xs]
     h_cont = [torch.empty(c, dtype=torch.uint8).pin_memory() for c in csizes]
@@ -399,28 +400,38 @@ def run_e2e(Z, xs, csizes, dev, stream, streams, args, world):
     wss = [Z.workspace(Z.BF16, max(x.numel() for x in xs), CHUNK, dev) for _ in streams]
     ns = len(streams)
 
+    lag = 2 * ns  # tensors whose compress is queued before the first one's size is read
+
     def step():
         ev = torch.cuda.Event()
         ev.record(stream)
         for s in streams:
             s.wait_event(ev)
-        for i in range(len(xs)):
+
+        def first_half(i):
             s = streams[i % ns]
             with torch.cuda.stream(s):
                 d_in[i].copy_(h_in[i], non_blocking=True)
             Z.compress_into(d_in[i], d_cont[i], wss[i % ns], CHUNK, stream=s)
-        for i in range(len(xs)):
+
+        def second_half(i):
             s = streams[i % ns]
-            size = Z.compressed_size(d_cont[i], stream=s)
+            size = Z.compressed_size(d_cont[i], stream=s)  # waits for this tensor's compress only
             with torch.cuda.stream(s):
                 h_cont[i][:size].copy_(d_cont[i][:size], non_blocking=True)
-        for i in range(len(xs)):
-            s = streams[i % ns]
-            with torch.cuda.stream(s):
-                d_cont[i][: csizes[i]].copy_(h_cont[i], non_blocking=True)
-            Z.decompress_into(d_cont[i], csizes[i], d_out[i], wss[i % ns], CHUNK, stream=s)
+                d_cont[i][:size].copy_(h_cont[i][:size], non_blocking=True)
+            Z.decompress_into(d_cont[i], size, d_out[i], wss[i % ns], CHUNK, stream=s)
             with torch.cuda.stream(s):
                 h_out[i].copy_(d_out[i], non_blocking=True)
+
+        # a software pipeline: while tensor i uploads and compresses, the container of
+        # tensor i - lag goes down and back up and is decompressed, so the two directions
+        # of the host link are busy at once
+        for i in range(len(xs) + lag):
+            if i < len(xs):
+                first_half(i)
+            if i >= lag:
+                second_half(i - lag)
         for s in streams:
             e2 = torch.cuda.Event()
             e2.record(s)
