@@ -40,7 +40,7 @@ struct Bf16EncodeSmem {
   uint32_t stage[kBStageWords];                  // the tile's bitstream at its final alignment
   uint32_t enc[256];                             // the chunk's code: len << 16 | code
   uint32_t warp[kBThreads / 32];
-  uint32_t carry;  // the bits of the word shared with the next pass
+  uint32_t carry[2];  // the bits of the word shared with the next pass, by pass parity
 };
 
 __device__ __forceinline__ void bf16_slot_merge(uint64_t* slot, uint32_t part, uint32_t* dst) {
@@ -210,11 +210,13 @@ __global__ void __launch_bounds__(kBThreads, 8) k_encode_bf16(const uint8_t* __r
       for (uint32_t i = tid; i < nwt; i += kBThreads) {
         uint32_t word = sm.stage[i];
         sm.stage[i] = 0;
-        if (i == 0 && pass > 0 && (P & 31) != 0) word |= sm.carry;  // the first pass's last bits
+        // the previous pass's last bits; a pass reads one carry slot and writes the other,
+        // so the slot it reads is not written again before the barriers of the next pass
+        if (i == 0 && pass > 0 && (P & 31) != 0) word |= sm.carry[(pass - 1) & 1];
         uint32_t* dst = bs + W0 + i;
         // (a first pass that is not the tile's last has kBPassValues values, so i == 0 and
         // the carried word are never the same word)
-        if (i == nwt - 1 && (end & 31) != 0 && !tile_end) sm.carry = word;  // completed by the next pass
+        if (i == nwt - 1 && (end & 31) != 0 && !tile_end) sm.carry[pass & 1] = word;  // completed by the next pass
         else if (i == 0 && pass == 0 && (P & 31) != 0) bf16_slot_merge(ws.slot + tile, word, dst);
         else if (i == nwt - 1 && (end & 31) != 0 && !last) bf16_slot_merge(ws.slot + tile + 1, word, dst);
         else *dst = bswap32(word);
