@@ -228,6 +228,12 @@ __device__ __forceinline__ int decode_bf16_fast(const uint32_t* lut, const uint8
 // 8r + (k ^ (r / 4 mod 8)): the row-per-thread stores and the unit-per-thread loads
 // of the merge both touch 32 distinct banks, with no padding.
 constexpr uint32_t kWindowBytes = 48 * 1024;
+// A bitstream of 48 to 56 KB (exponents of more than 3 bits on average, as in K/V
+// caches) still decodes from shared memory: its last 8 KB go to the first half of the
+// decode table's 16 KB, and the second half holds a single-symbol table (u16 entries:
+// symbol << 4 | length, bit 15 invalid) instead of the two-symbol one.
+constexpr uint32_t kWideWindowBytes = 56 * 1024;
+constexpr uint32_t kWindowWords = kWindowBytes / 4, kWideWords = kWideWindowBytes / 4;
 constexpr int kRound = 32;  // exponents of a sub-block decoded per round
 constexpr int kRowWords = kRound / 4;
 constexpr uint32_t kWaitLimit = 1u << 26;
@@ -265,15 +271,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
 }
 
 // Bit reader over words in shared memory; the next word is always already loaded.
+// WIDE: words from kWindowWords on are in a second region, w2.
+template <bool WIDE = false>
 struct SmemBitReader {
   const uint32_t* w;
+  const uint32_t* w2;
   uint32_t pos, end;
   uint64_t buf;
   int nb;
   uint32_t q;
-  __device__ __forceinline__ uint32_t ld(uint32_t i) const { return i < end ? bswap32(w[i]) : 0u; }
-  __device__ __forceinline__ void init(const uint32_t* words, uint32_t nwords, uint64_t bit) {
+  __device__ __forceinline__ uint32_t ld(uint32_t i) const {
+    if (i >= end) return 0u;
+    if constexpr (WIDE) return bswap32(i < kWindowWords ? w[i] : w2[i - kWindowWords]);
+    return bswap32(w[i]);
+  }
+  __device__ __forceinline__ void init(const uint32_t* words, uint32_t nwords, uint64_t bit,
+                                       const uint32_t* words2 = nullptr) {
     w = words;
+    w2 = words2;
     end = nwords;
     const uint32_t p0 = (uint32_t)(bit >> 5);
     buf = (uint64_t)ld(p0) << 32;
@@ -300,6 +315,15 @@ struct SmemBitReader {
     acc |= e;
     return lut_symbol(e);
   }
+  // single-symbol table: symbol << 4 | length, bit 15 invalid
+  __device__ __forceinline__ uint32_t huff(const uint16_t* lut, uint32_t& acc) {
+    const uint32_t e = lut[buf >> 52];
+    const uint32_t l = e & 15u;
+    buf <<= l;
+    nb -= (int)l;
+    acc |= e;
+    return (e >> 4) & 0xFFu;
+  }
   __device__ __forceinline__ uint64_t position() const { return (uint64_t)(pos - 1) * 32 - (uint64_t)nb; }
 };
 
@@ -307,12 +331,16 @@ __device__ __forceinline__ uint32_t ex_word(uint32_t row, uint32_t k) {
   return row * kRowWords + (k ^ ((row >> 2) & (kRowWords - 1)));
 }
 
-// One chunk, all threads of the block; one sub-block per thread and batch. smp: the
-// chunk's sign/fraction payload (RAW) or nullptr (ZERO); outc: the chunk's first
-// output value. Returns nonzero if the stream is inconsistent.
-__device__ int decode_bf16_staged(StagedSmem& st, const uint32_t* lut, const uint32_t* __restrict__ idx,
-                                  uint32_t bs_words, const uint8_t* __restrict__ smp, uint32_t m, uint32_t S,
-                                  uint32_t nsub, uint8_t* __restrict__ outc) {
+// One chunk, all threads of the block; one sub-block per thread and batch. WIDE: the
+// bitstream continues in `tail` after the window and lut is the single-symbol table;
+// else lut is the two-symbol table. smp: the chunk's sign/fraction payload (RAW) or
+// nullptr (ZERO); outc: the chunk's first output value. Returns nonzero if the stream is
+// inconsistent.
+template <bool WIDE, class Lut>
+__device__ int decode_bf16_staged(StagedSmem& st, const Lut* lut, const uint32_t* tail,
+                                  const uint32_t* __restrict__ idx, uint32_t bs_words,
+                                  const uint8_t* __restrict__ smp, uint32_t m, uint32_t S, uint32_t nsub,
+                                  uint8_t* __restrict__ outc) {
   const int tid = threadIdx.x;
   int bad = 0;
   const uint64_t cap_bits = (uint64_t)bs_words * 32;
@@ -321,7 +349,7 @@ __device__ int decode_bf16_staged(StagedSmem& st, const uint32_t* lut, const uin
   for (uint32_t batch = 0; batch < nsub; batch += kDecodeThreads) {
     const uint32_t j = batch + tid;
     const uint32_t count = j < nsub ? min32(S, m - j * S) : 0;
-    SmemBitReader br;
+    SmemBitReader<WIDE> br;
     uint32_t acc = 0;
     uint64_t expect = 0;
     bool exact = false;
@@ -330,7 +358,7 @@ __device__ int decode_bf16_staged(StagedSmem& st, const uint32_t* lut, const uin
       exact = j + 1 < nsub;
       expect = exact ? __ldg(idx + j + 1) : cap_bits;
       if ((j == 0 && start != 0) || start > cap_bits || expect < start || expect > cap_bits) bad = 1;
-      br.init(st.bits, bs_words, bad ? 0 : start);
+      br.init(st.bits, bs_words, bad ? 0 : start, tail);
     }
     // my merge units: unit u = tid + 256p is part u % 4 (values 8(u % 4)..) of row u / 4
     // of the batch; ubase is its first value in round 0, urem the values its row has
@@ -372,10 +400,20 @@ __device__ int decode_bf16_staged(StagedSmem& st, const uint32_t* lut, const uin
         if (base + kRound <= count) {
 #pragma unroll
           for (int k = 0; k < kRowWords; k++) {
-            br.refill();
-            const uint32_t a = huff_pair(br, lut, acc);
-            const uint32_t b = huff_pair(br, lut, acc);
-            st.ex[ex_word(tid, k)] = __byte_perm(a, b, 0x7632);
+            if constexpr (WIDE) {
+              br.refill();
+              const uint32_t e0 = br.huff(lut, acc);
+              const uint32_t e1 = br.huff(lut, acc);
+              br.refill();
+              const uint32_t e2 = br.huff(lut, acc);
+              const uint32_t e3 = br.huff(lut, acc);
+              st.ex[ex_word(tid, k)] = e0 | (e1 << 8) | (e2 << 16) | (e3 << 24);
+            } else {
+              br.refill();
+              const uint32_t a = huff_pair(br, lut, acc);
+              const uint32_t b = huff_pair(br, lut, acc);
+              st.ex[ex_word(tid, k)] = __byte_perm(a, b, 0x7632);
+            }
           }
         } else {
           const uint32_t n = count - base;
@@ -446,7 +484,7 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
                                              uint32_t c, uint8_t* __restrict__ out, uint32_t* status) {
   constexpr int NS = n_streams(DT), NE = n_entropy(DT), VB = value_bytes(DT);
   constexpr int GV = DT == kBF16 ? 8 : DT == kFP32 ? 4 : 16;  // values per store (16 bytes; FP4 8)
-  __shared__ DecodeSmem<DT> sm;
+  __shared__ __align__(16) DecodeSmem<DT> sm;  // 16-byte aligned: a bulk copy may target its table
   extern __shared__ __align__(128) uint8_t dyn_smem[];  // StagedSmem for BF16 launches
   const int tid = threadIdx.x;
   const uint64_t clo = (uint64_t)c * g.m0;
@@ -519,21 +557,24 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
     sm.bad = bad;
     sm.staged = 0;
     if constexpr (DT == kBF16) {
-      // staged path: HUFF exponents, RAW or ZERO sign/fraction bytes, bitstream in the window
+      // staged path: HUFF exponents, RAW or ZERO sign/fraction bytes, bitstream in the
+      // window (1), or in the window and the table's first half (2, the wide window)
       if (!bad && sm.mode[0] == kModeHuff && sm.mode[1] != kModeHuff) {
         const uint64_t nsub = ceil_div(m, S);
         const uint32_t rec = sm.code[0] == kNoCode ? record_bytes(DT, 0) : 0;
         const uint64_t bs_off = sm.off[0] + rec + round16(4 * nsub);
         const uint64_t bs_bytes = sm.end[0] > bs_off ? sm.end[0] - bs_off : 0;
-        if (bs_off <= sm.end[0] && bs_bytes <= kWindowBytes && nsub <= 0xFFFFFFFFull) {
+        if (bs_off <= sm.end[0] && bs_bytes <= kWideWindowBytes && nsub <= 0xFFFFFFFFull) {
           StagedSmem& stg = *reinterpret_cast<StagedSmem*>(dyn_smem);
           mbar_init(&stg.bar, 1);
           mbar_expect_tx(&stg.bar, (uint32_t)bs_bytes);
-          for (uint64_t o = 0; o < bs_bytes; o += 16384) {
+          for (uint64_t o = 0; o < bs_bytes; o += 16384) {  // 16 KB pieces; 48 KB is a piece boundary
             const uint32_t nb = (uint32_t)min64(16384, bs_bytes - o);
-            bulk_g2s(reinterpret_cast<uint8_t*>(stg.bits) + o, in + bs_off + o, nb, &stg.bar);
+            uint8_t* dst = o < kWindowBytes ? reinterpret_cast<uint8_t*>(stg.bits) + o
+                                            : reinterpret_cast<uint8_t*>(sm.lut[0]) + (o - kWindowBytes);
+            bulk_g2s(dst, in + bs_off + o, nb, &stg.bar);
           }
-          sm.staged = 1;
+          sm.staged = bs_bytes <= kWindowBytes ? 1 : 2;
         }
       }
     }
@@ -611,6 +652,14 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
   __syncthreads();
   if (sm.bad) {
     if (tid == 0) set_status(status, kStCorrupt);
+    if constexpr (DT == kBF16) {
+      // a bitstream copy may be in flight into this block's shared memory: let it land
+      // (bounded) before the block exits
+      if (sm.staged) {
+        StagedSmem& stg = *reinterpret_cast<StagedSmem*>(dyn_smem);
+        for (uint32_t k = 0; k < kWaitLimit && !mbar_try_wait(&stg.bar, 0); k++) __nanosleep(256);
+      }
+    }
     return;
   }
 #pragma unroll
@@ -623,19 +672,23 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
     }
   }
   __syncthreads();
+  // BF16 with the wide window: the single-symbol table in the table's second half (the
+  // bulk copy may still be writing the first half)
+  const bool wide = DT == kBF16 && sm.staged == 2;
+  uint16_t* const lut16 = reinterpret_cast<uint16_t*>(sm.lut[0] + (kWideWords - kWindowWords));
 #pragma unroll
   for (int e = 0; e < NE; e++) {
     if (sm.mode[e] != kModeHuff) continue;
     for (uint32_t x = tid; x < 4096; x += kDecodeThreads) {
-      uint32_t entry = kLutInvalid | 1u;
-      if (x < sm.limit[e][kLmax]) {
-        uint32_t l = 1;
+      uint32_t sym = 0, l = 1;
+      const bool valid = x < sm.limit[e][kLmax];
+      if (valid) {
 #pragma unroll
         for (int j = 1; j < kLmax; j++) l += x >= sm.limit[e][j];
-        const uint32_t sym = sm.sorted[e][sm.offset[e][l] + (x >> (kLmax - l)) - sm.first[e][l]];
-        entry = (sym << 16) | l;
+        sym = sm.sorted[e][sm.offset[e][l] + (x >> (kLmax - l)) - sm.first[e][l]];
       }
-      sm.lut[e][x] = entry;
+      if (wide) lut16[x] = (uint16_t)(valid ? (sym << 4) | l : kLutInvalid | 1u);
+      else sm.lut[e][x] = valid ? (sym << 16) | l : kLutInvalid | 1u;
     }
   }
   __syncthreads();
@@ -644,7 +697,7 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
     // decides it when that code ends inside the 12 known bits (a prefix code's entry
     // does not depend on the bits after the code). Updating in place is safe: the
     // fields read here (first length, first symbol, invalid flag) never change.
-    if (sm.mode[0] == kModeHuff) {
+    if (sm.mode[0] == kModeHuff && !wide) {
       for (uint32_t x = tid; x < 4096; x += kDecodeThreads) {
         const uint32_t e0 = sm.lut[0][x];
         if (e0 & kLutInvalid) continue;
@@ -676,7 +729,10 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
       const uint64_t bs_off = sm.off[0] + rec + round16(4 * nsub);
       const uint32_t bs_words = (uint32_t)((sm.end[0] - bs_off) / 4);
       const uint8_t* smp = sm.mode[1] == kModeRaw ? in + sm.off[1] : nullptr;
-      const int bad = decode_bf16_staged(stg, sm.lut[0], idx, bs_words, smp, m, S, (uint32_t)nsub, out + clo * VB);
+      const int bad = wide ? decode_bf16_staged<true>(stg, lut16, sm.lut[0], idx, bs_words, smp, m, S,
+                                                      (uint32_t)nsub, out + clo * VB)
+                           : decode_bf16_staged<false>(stg, sm.lut[0], nullptr, idx, bs_words, smp, m, S,
+                                                       (uint32_t)nsub, out + clo * VB);
       if (bad) set_status(status, kStCorrupt);
       return;
     }

@@ -125,6 +125,58 @@ def test_fp8(z, orc):
     assert c.size / q.numel() < 0.9
 
 
+def _spread_bf16(n, binades, seed):
+    # exponents uniform over `binades` binades: about log2(binades) bits each, so a 256 KiB
+    # chunk's exponent bitstream is 45 KB (6), 53 KB (9), 56 KB (10) or 65 KB (16)
+    g = torch.Generator().manual_seed(seed)
+    e = torch.randint(0, binades, (n,), generator=g).float()
+    m = torch.rand(n, generator=g) + 1.0
+    sgn = torch.randint(0, 2, (n,), generator=g).float() * 2 - 1
+    return (sgn * m * torch.pow(2.0, -e - 1)).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("binades", [6, 9, 10, 16])
+def test_bf16_high_entropy_exponents(z, orc, binades):
+    # the three decode paths: the 48 KB window with the two-symbol table, the 56 KB window
+    # with the single-symbol table (9, and 10 at the limit), and the global-memory reader
+    x = _spread_bf16(131072 * 3 + 1001, binades, binades)
+    _check_roundtrip(z, orc, x, f"bf16 {binades} binades")
+    _check_roundtrip(z, orc, x, f"bf16 {binades} binades S=256", subblock=256)
+    conts = [z.compress(x.cuda()), z.compress(x.cuda(), subblock=1024)]
+    outs = [torch.empty(x.numel(), dtype=torch.bfloat16, device="cuda") for _ in conts]
+    ws = z.batch_workspace(2)
+    z.decompress_batch_into(conts, [c.numel() for c in conts], outs, ws)
+    torch.cuda.synchronize()
+    assert z.status(ws) == z.OK
+    for o in outs:
+        assert torch.equal(o.view(torch.int16).cpu(), x.view(torch.int16))
+
+
+def test_bf16_wide_window_corrupt(z, orc):
+    # chunk 0's bitstream (53 KB) is in flight into shared memory when its code record
+    # fails the Kraft check; flips in its last 8 KB (the part kept in the table region)
+    # are detected or decode, never fault
+    import struct
+    x = _spread_bf16(131072 * 2, 9, 3)
+    c = z.compress(x.cuda()).cpu().numpy()
+    off0 = struct.unpack_from("<Q", c, 64 + 8)[0]
+    end0 = struct.unpack_from("<Q", c, 64 + 16 + 8)[0]
+    assert 48 * 1024 < end0 - off0 - 128 - 4 * 256 <= 56 * 1024
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    out = torch.empty(x.numel(), dtype=torch.bfloat16, device="cuda")
+    d = c.copy(); d[off0: off0 + 128] = 0x11
+    z.decompress_into(torch.from_numpy(d).cuda(), d.size, out, ws)
+    assert z.status(ws) == z.ERR_CORRUPT
+    assert orc.decompress_status("bf16", d, x.numel()) == orc.ECORRUPT
+    rng = np.random.default_rng(9)
+    for _ in range(20):
+        d = c.copy()
+        d[int(rng.integers(end0 - 8192, end0))] ^= 1 << int(rng.integers(0, 8))
+        z.decompress_into(torch.from_numpy(d).cuda(), d.size, out, ws)
+        assert z.status(ws) in (z.OK, z.ERR_CORRUPT)
+    torch.cuda.synchronize()
+
+
 def _fp4(raw):
     return torch.from_numpy(np.ascontiguousarray(raw, dtype=np.uint8)).view(torch.float4_e2m1fn_x2)
 
