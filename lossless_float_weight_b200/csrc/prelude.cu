@@ -6,6 +6,7 @@
 //                    Huffman code, then HUFF / RAW / ZERO;
 //   k_layout       : exclusive scan of payload sizes (single-pass decoupled look-back)
 //                    into payload offsets; writes header, chunk table, shared records.
+#include "bulk.cuh"
 #include "common.cuh"
 #include "fields.cuh"
 #include "huffman.cuh"
@@ -185,6 +186,144 @@ __global__ void __launch_bounds__(kHistThreads) k_split_hist(const uint8_t* __re
   }
 }
 
+// ---------------------------------------------------------------- BF16 histogram
+// k_split_hist_bf16: the same results as k_split_hist<kBF16>, with loads that stay in
+// flight. Blocks are persistent: each takes tiles (histogram slices) blockIdx.x,
+// blockIdx.x + gridDim.x, ... Thread 0 streams the block's tiles, 16 KB pieces in
+// order, through a ring of kHbStages shared-memory buffers with bulk copies, so up to
+// kHbStages pieces are on their way while the block counts and sums columns. The code
+// builds, latency-bound, are a kernel of their own (k_build_chunks) that follows.
+// Counting is that of k_split_hist (one counter per exponent and lane, both
+// halves of a word); thread t takes the 16-byte units t, t + 256, ... of a piece, so a
+// warp's shared loads are conflict-free. Only the tensor's last piece can end in fewer
+// than 8 values (chunks are whole multiples of 16 bytes); thread 0 loads those itself.
+constexpr int kHbStages = 4;
+constexpr uint32_t kHbPieceValues = 8192;  // 16 KB
+constexpr size_t kHbRegion = 256 * 32 * 4;  // the counters
+constexpr size_t kHbSmemBytes = kHbRegion + (size_t)kHbStages * kHbPieceValues * 2 + kHbStages * 8;
+constexpr uint32_t kHbWaitLimit = 1u << 26;
+
+// Values of tile `tile` (0 past the end of a ragged last chunk) and its first value.
+__device__ __forceinline__ uint32_t hb_tile_values(const Geo& g, uint32_t tile, uint64_t& vlo) {
+  const uint32_t c = tile / g.tiles_per_chunk, ti = tile - c * g.tiles_per_chunk;
+  const uint64_t clo = (uint64_t)c * g.m0;
+  const uint32_t m = (uint32_t)min64(g.m0, g.n - clo), lo = ti * kHistSlice;
+  vlo = clo + lo;
+  return lo < m ? min32(kHistSlice, m - lo) : 0u;
+}
+
+__global__ void __launch_bounds__(kHistThreads) k_split_hist_bf16(const uint8_t* __restrict__ src, Geo g,
+                                                                  uint32_t* __restrict__ hist,
+                                                                  uint32_t* __restrict__ nonzero, Ws ws) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];  // table, stages, barriers
+  uint32_t* const sh = reinterpret_cast<uint32_t*>(smem_raw);
+  uint8_t* const stages = smem_raw + kHbRegion;
+  uint64_t* const bar = reinterpret_cast<uint64_t*>(stages + (size_t)kHbStages * kHbPieceValues * 2);
+  const int tid = threadIdx.x, lane = tid & 31;
+  const uint32_t T = g.tiles_per_chunk;
+  for (int i = tid; i < 256 * 32; i += kHistThreads) sh[i] = 0;
+  if (tid == 0)
+    for (int s = 0; s < kHbStages; s++) mbar_init(bar + s, 1);
+  __syncthreads();
+
+  // thread 0's cursor: the next piece to load
+  uint32_t p_tile = blockIdx.x, p_piece = 0;
+  auto issue = [&](int s) {
+    for (; p_tile < g.n_tiles; p_tile += gridDim.x, p_piece = 0) {
+      uint64_t vlo;
+      const uint32_t nv = hb_tile_values(g, p_tile, vlo);
+      if (p_piece * kHbPieceValues >= nv) continue;
+      const uint32_t bytes = (min32(kHbPieceValues, nv - p_piece * kHbPieceValues) & ~7u) * 2;
+      fence_proxy_async_smem();  // the stage's earlier reads come first
+      mbar_expect_tx(bar + s, bytes);
+      if (bytes)
+        bulk_g2s(stages + (size_t)s * kHbPieceValues * 2, src + (vlo + (uint64_t)p_piece * kHbPieceValues) * 2, bytes,
+                 bar + s);
+      p_piece++;
+      return;
+    }
+  };
+  if (tid == 0)
+    for (int s = 0; s < kHbStages; s++) issue(s);
+
+  uint8_t* const colb = reinterpret_cast<uint8_t*>(sh + lane);
+  uint32_t q = 0;  // pieces consumed
+  for (uint32_t tile = blockIdx.x; tile < g.n_tiles; tile += gridDim.x) {
+    uint64_t vlo;
+    const uint32_t nv = hb_tile_values(g, tile, vlo);
+    if (nv == 0) continue;  // uniform
+    const uint32_t c = tile / T, sl = tile - c * T;
+    uint32_t nz0 = 0, nz1 = 0;
+    for (uint32_t p0 = 0; p0 < nv; p0 += kHbPieceValues, q++) {
+      const int s = (int)(q % kHbStages);
+      if (!mbar_wait_bounded(bar + s, (q / kHbStages) & 1u, kHbWaitLimit) && ws.status) set_status(ws.status, kStTimeout);
+      const uint32_t pv = min32(kHbPieceValues, nv - p0), nb = pv & ~7u;
+      const uint4* st4 = reinterpret_cast<const uint4*>(stages + (size_t)s * kHbPieceValues * 2);
+#pragma unroll
+      for (int k = 0; k < (int)(kHbPieceValues / 8 / kHistThreads); k++) {
+        const uint32_t i = (uint32_t)(k * kHistThreads + tid);
+        if (i * 8 < nb) {
+          const uint4 v = st4[i];
+          const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int j = 0; j < 4; j++) {
+            // the low value's exponent is bits 14..7: its counter (row e, 32 words) is
+            // at byte offset w & 0x7F80; the high value's at (w >> 16) & 0x7F80
+            atomicAdd(reinterpret_cast<uint32_t*>(colb + (x[j] & 0x7F80u)), 1u);
+            atomicAdd(reinterpret_cast<uint32_t*>(colb + ((x[j] >> 16) & 0x7F80u)), 1u);
+            nz0 |= x[j] & 0x7F807F80u;
+            nz1 |= x[j] & 0x807F807Fu;
+          }
+        }
+      }
+      if (tid == 0 && nb < pv) {
+        const uint16_t* t = reinterpret_cast<const uint16_t*>(src) + vlo + p0 + nb;
+        for (uint32_t i = 0; i < pv - nb; i++) {
+          const uint32_t v = t[i];
+          atomicAdd(reinterpret_cast<uint32_t*>(colb + (v & 0x7F80u)), 1u);
+          nz0 |= v & 0x7F80u;
+          nz1 |= v & 0x807Fu;
+        }
+      }
+      __syncthreads();  // stage s is read, and the tile's counts are complete after the last piece
+      if (tid == 0) issue(s);
+    }
+    nz0 = __reduce_or_sync(0xFFFFFFFFu, nz0);
+    nz1 = __reduce_or_sync(0xFFFFFFFFu, nz1);
+    if (nonzero && lane == 0) {
+      if (nz0) atomicOr(&nonzero[(uint64_t)c * 2], nz0);
+      if (nz1) atomicOr(&nonzero[(uint64_t)c * 2 + 1], nz1);
+    }
+    // row b (exponent b): thread b sums it from lane b on (32 banks a warp) and clears it
+    {
+      const int b = tid;
+      uint32_t sum = 0;
+#pragma unroll 8
+      for (int l = 0; l < 32; l++) {
+        const int a = b * 32 + ((l + b) & 31);
+        sum += sh[a];
+        sh[a] = 0;
+      }
+      if (sum) atomicAdd(&hist[(uint64_t)c * 256 + b], sum);
+      if (ws.tile_hist) ws.tile_hist[((uint64_t)c * T + sl) * 256 + b] = (uint16_t)sum;
+    }
+    __syncthreads();  // every row is clear before the next tile's counts
+  }
+}
+
+// One block per chunk: the chunk's code choice (build_chunk_table) for each entropy
+// stream, once the histogram pass is complete.
+template <int DT>
+__global__ void __launch_bounds__(kHuffWarps * 32) k_build_chunks(Geo g, Ws ws, PlanDev plan) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  HuffBlockSmem& hs = *reinterpret_cast<HuffBlockSmem*>(smem_raw);
+#pragma unroll
+  for (int e = 0; e < n_entropy(DT); e++) {
+    build_chunk_table<DT>(g, ws, plan, blockIdx.x, (uint32_t)e, hs);
+    __syncthreads();
+  }
+}
+
 // Stand-alone code lengths for `count` histograms (u64 x 256 each); also used by the
 // plan for its group codes. Optionally writes canonical code values.
 __global__ void __launch_bounds__(kHuffWarps * 32) k_code_lengths(const uint64_t* __restrict__ hist, uint32_t alphabet_size,
@@ -327,6 +466,36 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout(Geo g, Ws ws, PlanDev
 
 // ---------------------------------------------------------------- launchers
 
+// BF16: a persistent grid of as many histogram blocks as fit on the device at once,
+// then (compress) one code-build block per chunk.
+static cudaError_t split_hist_bf16(const void* src, const Geo& g, uint32_t* hist, uint32_t* nonzero, const Ws* ws,
+                                   const PlanDev& plan, cudaStream_t st) {
+  static int resident[128] = {0};  // blocks per device, once the attributes are set
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  int per_device = dev >= 0 && dev < 128 ? resident[dev] : 0;
+  if (!per_device) {
+    e = cudaFuncSetAttribute(k_split_hist_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kHbSmemBytes);
+    int per_sm = 0, sms = 0;
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_split_hist_bf16, kHistThreads, kHbSmemBytes);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    per_device = (per_sm > 0 ? per_sm : 1) * (sms > 0 ? sms : 1);
+    if (dev >= 0 && dev < 128) resident[dev] = per_device;
+  }
+  Ws w{};
+  if (ws) w = *ws;
+  const uint32_t blocks = (uint32_t)min64((uint64_t)per_device, g.n_tiles);
+  k_split_hist_bf16<<<blocks, kHistThreads, kHbSmemBytes, st>>>(static_cast<const uint8_t*>(src), g, hist, nonzero,
+                                                                  w);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || !ws) return e;
+  k_build_chunks<kBF16><<<g.n_chunks, kHuffWarps * 32, sizeof(HuffBlockSmem), st>>>(g, w, plan);
+  return cudaGetLastError();
+}
+
 template <int DT>
 static cudaError_t split_hist_t(const void* src, const Geo& g, uint32_t* hist, uint32_t* nonzero, const Ws* ws,
                                 const PlanDev& plan, cudaStream_t st) {
@@ -346,7 +515,7 @@ static cudaError_t split_hist_t(const void* src, const Geo& g, uint32_t* hist, u
 cudaError_t launch_split_hist(const void* src, const Geo& g, uint32_t* hist, uint32_t* nonzero, const Ws* ws,
                               const PlanDev& plan, cudaStream_t st) {
   switch (g.dt) {
-    case kBF16: return split_hist_t<kBF16>(src, g, hist, nonzero, ws, plan, st);
+    case kBF16: return split_hist_bf16(src, g, hist, nonzero, ws, plan, st);
     case kFP32: return split_hist_t<kFP32>(src, g, hist, nonzero, ws, plan, st);
     case kFP8: return split_hist_t<kFP8>(src, g, hist, nonzero, ws, plan, st);
     default: return split_hist_t<kFP4>(src, g, hist, nonzero, ws, plan, st);
