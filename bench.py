@@ -82,7 +82,7 @@ def rank_seed(rank):
 # ncu summaries under profiles/ that give a kernel's DRAM bytes per value; each names the
 # kernel sources it was taken from, by hash, so a summary of an older kernel is not used
 PROFILE_OF = {"decode_merge": "decode_merge_embedding_bf16.txt", "encode": "encode_bf16_embedding_bf16.txt",
-              "split_hist_tables": "split_hist_tables_embedding_bf16.txt"}
+              "split_hist": "split_hist_embedding_bf16.txt", "code_build": "build_chunks_embedding_bf16.txt"}
 
 
 def profile_traffic(kernel, values_per_launch):
@@ -264,8 +264,8 @@ def run_ours(args):
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     clocks = ClockSampler(local)
-    # launches of our kernels per step: split+histogram+code build, layout scan and
-    # encode per compress call, decode per decompress call (events count them below)
+    # launches of our kernels per step: split+histogram, code build (BF16), layout scan
+    # and encode per compress call, decode per decompress call (events count them below)
     barrier(world, dev)
     torch.cuda.synchronize()
     clocks.start()
@@ -309,8 +309,8 @@ def run_ours(args):
     algo_bytes = nbytes + cbytes  # read + written, per direction
     gpu_launches = sum(v[1] for v in ktimes.values())  # the same count as the timed region
     # algorithmic bytes per step of each kernel (reads + writes the method needs)
-    kbytes = {"decode_merge": cbytes + nbytes, "encode": nbytes + cbytes, "split_hist_tables": nbytes,
-              "layout_scan": 0}
+    kbytes = {"decode_merge": cbytes + nbytes, "encode": nbytes + cbytes, "split_hist": nbytes,
+              "code_build": 0, "layout_scan": 0}
     # dominant kernel: the one with the largest share of device time
     dom = max(ktimes.items(), key=lambda kv: kv[1][0])
     dom_name, (dom_ms, dom_n) = dom

@@ -175,6 +175,10 @@ zipnn_status zipnn_compress_ex(zipnn_dtype dtype, const void* src, uint64_t n, u
     TimedLaunch t(kIdHist, st);
     e = launch_split_hist(src, g, w.hist, w.nonzero, &w, pd, st);
   }
+  if (e == cudaSuccess && g.dt == kBF16) {
+    TimedLaunch t(kIdBuild, st);
+    e = launch_build_chunks(g, w, pd, st);
+  }
   if (e == cudaSuccess) {
     TimedLaunch t(kIdLayout, st);
     e = launch_layout(g, w, pd, static_cast<uint8_t*>(out), st);

@@ -6,7 +6,7 @@
 namespace zipnn {
 
 // Kernel ids of the optional event timing (timing.cu).
-enum KernelId { kIdHist = 0, kIdTables, kIdLayout, kIdEncode, kIdDecode, kIdCodeLengths, kIdPlan, kNumKernelIds };
+enum KernelId { kIdHist = 0, kIdBuild, kIdLayout, kIdEncode, kIdDecode, kIdCodeLengths, kIdPlan, kNumKernelIds };
 
 // Brackets one launch with CUDA events on `st` while timing is enabled.
 class TimedLaunch {
@@ -22,9 +22,12 @@ class TimedLaunch {
   cudaEvent_t start_ = nullptr, stop_ = nullptr;
 };
 
-// Histograms; with ws, the last block of each chunk also builds the chunk's codes.
+// Histograms. With ws (compress), also the chunks' codes: for BF16 in a second kernel,
+// launch_build_chunks; for the other types the last block of each chunk builds them.
 cudaError_t launch_split_hist(const void* src, const Geo& g, uint32_t* hist, uint32_t* nonzero, const Ws* ws,
                               const PlanDev& plan, cudaStream_t st);
+// BF16 compress: the chunks' codes, after launch_split_hist (one block per chunk).
+cudaError_t launch_build_chunks(const Geo& g, const Ws& ws, const PlanDev& plan, cudaStream_t st);
 cudaError_t launch_code_lengths(const uint64_t* hist, uint32_t count, uint32_t alphabet_size, uint8_t* lens,
                                 uint32_t* enc, cudaStream_t st);
 cudaError_t launch_layout(const Geo& g, const Ws& ws, const PlanDev& plan, uint8_t* out, cudaStream_t st);

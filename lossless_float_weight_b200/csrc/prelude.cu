@@ -466,8 +466,7 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout(Geo g, Ws ws, PlanDev
 
 // ---------------------------------------------------------------- launchers
 
-// BF16: a persistent grid of as many histogram blocks as fit on the device at once,
-// then (compress) one code-build block per chunk.
+// BF16: a persistent grid of as many histogram blocks as fit on the device at once.
 static cudaError_t split_hist_bf16(const void* src, const Geo& g, uint32_t* hist, uint32_t* nonzero, const Ws* ws,
                                    const PlanDev& plan, cudaStream_t st) {
   static int resident[128] = {0};  // blocks per device, once the attributes are set
@@ -490,9 +489,12 @@ static cudaError_t split_hist_bf16(const void* src, const Geo& g, uint32_t* hist
   const uint32_t blocks = (uint32_t)min64((uint64_t)per_device, g.n_tiles);
   k_split_hist_bf16<<<blocks, kHistThreads, kHbSmemBytes, st>>>(static_cast<const uint8_t*>(src), g, hist, nonzero,
                                                                   w);
-  e = cudaGetLastError();
-  if (e != cudaSuccess || !ws) return e;
-  k_build_chunks<kBF16><<<g.n_chunks, kHuffWarps * 32, sizeof(HuffBlockSmem), st>>>(g, w, plan);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_build_chunks(const Geo& g, const Ws& ws, const PlanDev& plan, cudaStream_t st) {
+  if (g.dt != kBF16) return cudaErrorInvalidValue;
+  k_build_chunks<kBF16><<<g.n_chunks, kHuffWarps * 32, sizeof(HuffBlockSmem), st>>>(g, ws, plan);
   return cudaGetLastError();
 }
 

@@ -10,7 +10,7 @@
 namespace zipnn {
 namespace {
 
-const char* const kNames[kNumKernelIds] = {"split_hist_tables", "unused", "layout_scan", "encode",
+const char* const kNames[kNumKernelIds] = {"split_hist", "code_build", "layout_scan", "encode",
                                            "decode_merge", "code_lengths", "plan"};
 
 struct Pending {
