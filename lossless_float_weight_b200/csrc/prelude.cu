@@ -93,7 +93,7 @@ __device__ void build_chunk_table(const Geo& g, const Ws& ws, const PlanDev& pla
 // the 32 lanes of a warp always add into 32 different banks (lane l owns column l);
 // warps share the table through shared atomics. The columns are summed at the end.
 template <int DT>
-__global__ void __launch_bounds__(kHistThreads) k_split_hist(const uint8_t* __restrict__ src, Geo g, uint32_t slices,
+__global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* __restrict__ src, Geo g, uint32_t slices,
                                                              uint32_t* __restrict__ hist, uint32_t* __restrict__ nonzero,
                                                              Ws ws, PlanDev plan, int build) {
   constexpr int NS = n_streams(DT), NE = n_entropy(DT);
@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(kHistThreads) k_split_hist_bf16(const uint8_t*
 // One block per chunk: the chunk's code choice (build_chunk_table) for each entropy
 // stream, once the histogram pass is complete.
 template <int DT>
-__global__ void __launch_bounds__(kHuffWarps * 32) k_build_chunks(Geo g, Ws ws, PlanDev plan) {
+__global__ void __launch_bounds__(kHuffWarps * 32, 4) k_build_chunks(Geo g, Ws ws, PlanDev plan) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   HuffBlockSmem& hs = *reinterpret_cast<HuffBlockSmem*>(smem_raw);
 #pragma unroll
