@@ -29,7 +29,7 @@ import torch
 METRIC = "decompress/compress GB/s (uncompressed) at 1 B200; % of HBM roofline"
 WORKLOAD = ("BF16 7B-shaped checkpoint: 32 x [q,k,v,o 4096x4096; gate,up,down 4096x11008] + embedding "
             "32000x4096, 225 tensors, 6,607,077,376 values (13.21 GB), sigma_t log-uniform [0.005, 0.05], "
-            "256 KiB chunks; compress: one zipnn call per tensor, tensors spread round-robin over 4 streams")
+            "256 KiB chunks; compress: one zipnn call per tensor, tensors spread round-robin over {ns} streams")
 CHUNK = 262144
 SUBBLOCK = 512  # the library default (include/zipnn.h)
 FALLBACK_HBM_GBS = 6650.0
@@ -336,7 +336,7 @@ def run_ours(args):
             "dtype": "u32",
             "data": "synthetic (seeded N(0, sigma_t^2) BF16 tensors of a 7B checkpoint's shapes; no trained weights)",
             "config": {
-                "workload": WORKLOAD,
+                "workload": WORKLOAD.format(ns=args.streams),
                 "step": "compress all 225 tensors (one zipnn_compress each), then decompress all 225 ("
                         + ("one zipnn_decompress each" if args.per_tensor_decode else "one zipnn_decompress_batch")
                         + ") (value = uncompressed bytes per "
@@ -489,7 +489,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "u32", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "sample": sample},
+        "config": {"workload": WORKLOAD.format(ns=args.streams), "sample": sample},
         "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
@@ -502,7 +502,7 @@ def run_plan_transfer(args):
     layers 16-31 are compressed with it, as they are and with 5% relative noise added
     (weights after further training). Reports the size against per-chunk codes, the
     fraction of chunks that fall back to a local code, the setup time and the compress
-    throughput with and without the plan (4 streams, as the main benchmark)."""
+    throughput with and without the plan (on --streams streams, as the main benchmark)."""
     from lossless_float_weight_b200 import workloads as W
     from lossless_float_weight_b200 import zipnn as Z
     dev = torch.device("cuda", 0)
@@ -675,7 +675,7 @@ def main():
                     help="only the first T tensors of the checkpoint (small cases for profilers)")
     ap.add_argument("--only", type=int, default=None, help="only tensor IDX of the checkpoint (profiler cases)")
     ap.add_argument("--no-extras", action="store_true", help="skip the e2e and CPU-baseline legs")
-    ap.add_argument("--streams", type=int, default=4, help="CUDA streams the tensors are spread over")
+    ap.add_argument("--streams", type=int, default=8, help="CUDA streams the tensors are spread over")
     ap.add_argument("--workload", default="checkpoint_7b",
                     choices=["checkpoint_7b", "fp32", "fp32_clean", "fp8", "fp4", "kv_cache"],
                     help="another workload than the benchmark's: one tensor, compress and decompress timed apart")
