@@ -1,9 +1,13 @@
 // prelude.cu -- the compress steps before encoding:
-//   k_split_hist   : byte-plane split + order-0 histogram per chunk (warp-aggregated
-//                    shared-memory atomics) + all-zero detection per chunk stream;
-//                    the last block of each chunk then builds the chunk's codes: per
-//                    entropy stream a shared group code or a local length-limited
-//                    Huffman code, then HUFF / RAW / ZERO;
+//   k_split_hist_bf16 (BF16) / k_split_hist (FP32, FP8, FP4): byte-plane split +
+//                    order-0 histogram per chunk (per-lane shared-memory counters) +
+//                    all-zero detection per chunk stream; BF16 also keeps the counts
+//                    of each encode tile;
+//   code build     : per chunk and entropy stream a shared group code or a local
+//                    length-limited Huffman code, then HUFF / RAW / ZERO. BF16:
+//                    k_build_chunks, one block per chunk after the histogram pass
+//                    (it also turns the tile counts into tile bit offsets); the other
+//                    types: the last histogram block of each chunk;
 //   k_layout       : exclusive scan of payload sizes (single-pass decoupled look-back)
 //                    into payload offsets; writes header, chunk table, shared records.
 #include "bulk.cuh"
@@ -92,6 +96,7 @@ __device__ void build_chunk_table(const Geo& g, const Ws& ws, const PlanDev& pla
 // of each symbol. The block keeps one counter per (symbol, lane) in shared memory, so
 // the 32 lanes of a warp always add into 32 different banks (lane l owns column l);
 // warps share the table through shared atomics. The columns are summed at the end.
+// FP32, FP8 and FP4 (BF16 has k_split_hist_bf16 below).
 template <int DT>
 __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* __restrict__ src, Geo g, uint32_t slices,
                                                              uint32_t* __restrict__ hist, uint32_t* __restrict__ nonzero,
@@ -120,37 +125,17 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
     if (cnt > 0) {
       RawValues<DT, NV> raw;
       load_values<DT, NV>(src + value_offset(DT, clo + v0), cnt, raw);
-      bool done = false;
-      if constexpr (DT == kBF16) {
-        if (cnt == NV) {
-          // a whole word at a time: the exponent e of the low value is bits 14..7, so its
-          // counter (column offset e * 32 words) is at byte offset w & 0x7F80; the high
-          // value's at (w >> 16) & 0x7F80. Zero detection needs only the masked words.
-          uint8_t* colb = reinterpret_cast<uint8_t*>(col0);
 #pragma unroll
-          for (int j = 0; j < NV / 2; j++) {
-            const uint32_t w = raw.w[j];
-            atomicAdd(reinterpret_cast<uint32_t*>(colb + (w & 0x7F80u)), 1u);
-            atomicAdd(reinterpret_cast<uint32_t*>(colb + ((w >> 16) & 0x7F80u)), 1u);
-            nz[0] |= w & 0x7F807F80u;
-            nz[NS - 1] |= w & 0x807F807Fu;
-          }
-          done = true;
+      for (int i = 0; i < NV; i++) {
+        if (i < cnt) {
+          atomicAdd(col0 + symbol<DT, NV>(raw, 0, i) * 32, 1u);
+          if (NE > 1) atomicAdd(col1 + symbol<DT, NV>(raw, 1, i) * 32, 1u);
         }
       }
-      if (!done) {
 #pragma unroll
-        for (int i = 0; i < NV; i++) {
-          if (i < cnt) {
-            atomicAdd(col0 + symbol<DT, NV>(raw, 0, i) * 32, 1u);
-            if (NE > 1) atomicAdd(col1 + symbol<DT, NV>(raw, 1, i) * 32, 1u);
-          }
-        }
+      for (int i = 0; i < NV; i++)
 #pragma unroll
-        for (int i = 0; i < NV; i++)
-#pragma unroll
-          for (int s = 0; s < NS; s++) nz[s] |= symbol<DT, NV>(raw, s, i);
-      }
+        for (int s = 0; s < NS; s++) nz[s] |= symbol<DT, NV>(raw, s, i);
     }
   }
 #pragma unroll
@@ -166,8 +151,6 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
     for (int l = 0; l < 32; l++) sum += sh[b * 32 + ((l + b) & 31)];
     const int e = b < A0 ? 0 : 1, sym = b < A0 ? b : b - A0;
     if (sum) atomicAdd(&hist[((uint64_t)c * NE + e) * 256 + sym], sum);
-    // BF16 compress: the slice is one encode tile; its counts give the tile offsets
-    if (DT == kBF16 && ws.tile_hist) ws.tile_hist[((uint64_t)c * g.tiles_per_chunk + sl) * 256 + b] = (uint16_t)sum;
   }
   if (!build) return;
   // the last block to finish a chunk builds that chunk's codes (its histogram is then
@@ -187,14 +170,14 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
 }
 
 // ---------------------------------------------------------------- BF16 histogram
-// k_split_hist_bf16: the same results as k_split_hist<kBF16>, with loads that stay in
-// flight. Blocks are persistent: each takes tiles (histogram slices) blockIdx.x,
+// k_split_hist_bf16: the histogram pass of BF16, with loads that stay in flight. Blocks are persistent: each takes tiles (histogram slices) blockIdx.x,
 // blockIdx.x + gridDim.x, ... Thread 0 streams the block's tiles, 16 KB pieces in
 // order, through a ring of kHbStages shared-memory buffers with bulk copies, so up to
 // kHbStages pieces are on their way while the block counts and sums columns. The code
 // builds, latency-bound, are a kernel of their own (k_build_chunks) that follows.
-// Counting is that of k_split_hist (one counter per exponent and lane, both
-// halves of a word); thread t takes the 16-byte units t, t + 256, ... of a piece, so a
+// The counters are those of k_split_hist (one per exponent and lane), taking both
+// halves of a word at a time; each tile's column sums are also its encode-tile counts.
+// Thread t takes the 16-byte units t, t + 256, ... of a piece, so a
 // warp's shared loads are conflict-free. Only the tensor's last piece can end in fewer
 // than 8 values (chunks are whole multiples of 16 bytes); thread 0 loads those itself.
 constexpr int kHbStages = 4;
