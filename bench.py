@@ -85,10 +85,27 @@ PROFILE_OF = {"decode_merge": "decode_merge_embedding_bf16.txt", "encode": "enco
               "split_hist": "split_hist_embedding_bf16.txt", "code_build": "build_chunks_embedding_bf16.txt"}
 
 
+def code_digest(files, csrc=None):
+    """sha256 over the code of the given source files (sorted by name; in the package's csrc
+    unless `csrc` names another folder), comments removed and runs of white space made one
+    space: a change to the code changes it, a change to a comment or to the layout does not."""
+    import hashlib
+    import re
+    csrc = csrc or os.path.join(ROOT, "lossless_float_weight_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(files):
+        with open(os.path.join(csrc, f)) as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(re.sub(r"\s+", " ", text).strip().encode())
+        h.update(b"\0")
+    return h.hexdigest()
+
+
 def profile_traffic(kernel, values_per_launch):
     """DRAM bytes of one launch of `kernel`, from its committed ncu summary scaled by the values
-    the launch processes; None without a summary or when the sources changed since."""
-    import hashlib
+    the launch processes; None without a summary or when the kernel's code changed since."""
     import re
     name = PROFILE_OF.get(kernel)
     path = os.path.join(ROOT, "profiles", name) if name else None
@@ -96,14 +113,10 @@ def profile_traffic(kernel, values_per_launch):
         return None
     text = open(path).read()
     bpv = re.search(r"DRAM bytes per value\s+([0-9.]+)", text)
-    src = re.search(r"kernel sources sha256 \(([^)]*)\): ([0-9a-f]{64})", text)
+    src = re.search(r"kernel code sha256 \(([^)]*)\): ([0-9a-f]{64})", text)
     if not bpv or not src:
         return None
-    h = hashlib.sha256()
-    for f in sorted(src.group(1).split()):
-        with open(os.path.join(ROOT, "lossless_float_weight_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
-    if h.hexdigest() != src.group(2):
+    if code_digest(src.group(1).split()) != src.group(2):
         return None
     return round(float(bpv.group(1)) * values_per_launch)
 

@@ -26,7 +26,8 @@ constexpr int kGroupValues = 16;
 constexpr int kEncGroups = 4;
 constexpr int kEncodeThreads = 256;
 constexpr int kTileValues = kEncodeThreads * kGroupValues * kEncGroups;  // 16384
-// BF16 encode: 512 threads of 64 values; the tile is also one histogram block's slice
+// BF16: the encode tile (512 groups of 64 values; the encode kernel takes it in passes
+// of its own block) is also one histogram tile, whose counts give its bit offset
 constexpr int kBf16EncodeThreads = 512;
 constexpr int kBf16TileValues = kBf16EncodeThreads * kGroupValues * kEncGroups;  // 32768
 __host__ __device__ constexpr uint32_t tile_values(int dt) {

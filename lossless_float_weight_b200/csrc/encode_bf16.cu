@@ -1,7 +1,7 @@
 // encode_bf16.cu -- k_encode_bf16: the encode of BF16 tensors.
 //
 // The same output as k_encode (encode.cu), with no wait between blocks. A tile is
-// 32768 consecutive values of one chunk (one histogram block's slice); its exponent
+// 32768 consecutive values of one chunk (one histogram tile); its exponent
 // bits start, inside the chunk's bitstream, at the sum over the chunk's lower tiles of
 // count(tile, e) * len(e). The histogram pass counts per tile and the code build turns
 // the counts into tile offsets, so every tile knows its offset before it packs a bit.

@@ -7,7 +7,7 @@
 //                    length-limited Huffman code, then HUFF / RAW / ZERO. BF16:
 //                    k_build_chunks, one block per chunk after the histogram pass
 //                    (it also turns the tile counts into tile bit offsets); the other
-//                    types: the last histogram block of each chunk;
+//                    types: the histogram block that finishes a chunk last;
 //   k_layout       : exclusive scan of payload sizes (single-pass decoupled look-back)
 //                    into payload offsets; writes header, chunk table, shared records.
 #include "bulk.cuh"
@@ -19,7 +19,7 @@
 namespace zipnn {
 
 constexpr int kHistThreads = 256;
-constexpr uint32_t kHistSlice = 32768;  // values of one chunk per histogram block
+constexpr uint32_t kHistSlice = 32768;  // values of one chunk per histogram tile
 static_assert(kHistSlice == kBf16TileValues, "a BF16 histogram slice is one encode tile");
 
 // BF16 with a HUFF exponent stream: the bit offset of each encode tile in the chunk's
@@ -170,16 +170,17 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
 }
 
 // ---------------------------------------------------------------- BF16 histogram
-// k_split_hist_bf16: the histogram pass of BF16, with loads that stay in flight. Blocks are persistent: each takes tiles (histogram slices) blockIdx.x,
+// k_split_hist_bf16: the histogram pass of BF16, with loads that stay in flight.
+// Blocks are persistent: each takes tiles (32768-value slices of a chunk) blockIdx.x,
 // blockIdx.x + gridDim.x, ... Thread 0 streams the block's tiles, 16 KB pieces in
 // order, through a ring of kHbStages shared-memory buffers with bulk copies, so up to
 // kHbStages pieces are on their way while the block counts and sums columns. The code
 // builds, latency-bound, are a kernel of their own (k_build_chunks) that follows.
 // The counters are those of k_split_hist (one per exponent and lane), taking both
 // halves of a word at a time; each tile's column sums are also its encode-tile counts.
-// Thread t takes the 16-byte units t, t + 256, ... of a piece, so a
-// warp's shared loads are conflict-free. Only the tensor's last piece can end in fewer
-// than 8 values (chunks are whole multiples of 16 bytes); thread 0 loads those itself.
+// Thread t takes the 16-byte units t, t + 256, ... of a piece, so a warp's shared
+// loads are conflict-free. Only the tensor's last piece can end in fewer than 8 values
+// (chunks are whole multiples of 16 bytes); thread 0 loads those itself.
 constexpr int kHbStages = 4;
 constexpr uint32_t kHbPieceValues = 8192;  // 16 KB
 constexpr size_t kHbRegion = 256 * 32 * 4;  // the counters
