@@ -114,3 +114,15 @@ def kv_cache(shape=(32, 2, 16, 8, 4096, 128), seed=0, device="cpu"):
         x = torch.randn((kv, batch, heads, seq, dim), generator=g, device=device)
         out[layer] = (x * std[layer]).to(torch.bfloat16)
     return out.reshape(-1)
+
+
+def spread_bf16(n, binades, seed):
+    """BF16 values whose exponents are uniform over `binades` binades below 0.5 (random
+    sign, fraction uniform in [1, 2)): about log2(binades) bits of exponent entropy, more
+    than trained weights have. A 256 KiB chunk's exponent bitstream comes to about 45 KB
+    for 6 binades, 53 KB for 9, 56 KB for 10 and 65 KB for 16."""
+    g = torch.Generator().manual_seed(seed)
+    e = torch.randint(0, binades, (n,), generator=g).float()
+    m = torch.rand(n, generator=g) + 1.0
+    sgn = torch.randint(0, 2, (n,), generator=g).float() * 2 - 1
+    return (sgn * m * torch.pow(2.0, -e - 1)).to(torch.bfloat16)

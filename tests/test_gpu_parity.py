@@ -126,13 +126,8 @@ def test_fp8(z, orc):
 
 
 def _spread_bf16(n, binades, seed):
-    # exponents uniform over `binades` binades: about log2(binades) bits each, so a 256 KiB
-    # chunk's exponent bitstream is 45 KB (6), 53 KB (9), 56 KB (10) or 65 KB (16)
-    g = torch.Generator().manual_seed(seed)
-    e = torch.randint(0, binades, (n,), generator=g).float()
-    m = torch.rand(n, generator=g) + 1.0
-    sgn = torch.randint(0, 2, (n,), generator=g).float() * 2 - 1
-    return (sgn * m * torch.pow(2.0, -e - 1)).to(torch.bfloat16)
+    from lossless_float_weight_b200 import workloads as W
+    return W.spread_bf16(n, binades, seed)
 
 
 @pytest.mark.parametrize("binades", [6, 9, 10, 16])
