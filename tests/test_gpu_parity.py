@@ -99,6 +99,37 @@ def test_constant_and_zero_tensors(z, orc):
         _check_roundtrip(z, orc, x, f"constant {x.dtype}")
 
 
+def _mixed_modes_bf16():
+    # one tensor whose chunks take every pair of stream modes: zeros (ZERO, ZERO), weights
+    # (HUFF, RAW), positive powers of two (HUFF, ZERO), every bit pattern at random
+    # (RAW, RAW), and a ragged tail of weights (HUFF, RAW)
+    m0 = 131072
+    g = torch.Generator().manual_seed(11)
+    parts = [torch.zeros(m0), torch.randn(m0, generator=g) * 0.02,
+             torch.pow(2.0, -torch.randint(1, 20, (m0,), generator=g).float()), None,
+             torch.randn(1001, generator=g) * 0.02]
+    pat = torch.randint(0, 65536, (m0,), generator=g, dtype=torch.int32).to(torch.int16).view(torch.bfloat16)
+    return torch.cat([p.to(torch.bfloat16) if p is not None else pat for p in parts])
+
+
+def test_bf16_mixed_chunk_modes(z, orc):
+    import struct
+    x = _mixed_modes_bf16()
+    got = _check_roundtrip(z, orc, x, "bf16 mixed modes")
+    modes = [struct.unpack_from("<I", got, 64 + 16 * k)[0] & 0xFF for k in range(10)]
+    assert modes == [1, 1, 2, 0, 2, 1, 0, 0, 2, 0]  # ZERO 1, HUFF 2, RAW 0; (exp, sign/fraction) per chunk
+    # decoded in one batch beside a tensor of weights
+    w = (torch.randn(300001, generator=torch.Generator().manual_seed(12)) * 0.03).to(torch.bfloat16)
+    conts = [z.compress(x.cuda()), z.compress(w.cuda())]
+    outs = [torch.empty(t.numel(), dtype=torch.bfloat16, device="cuda") for t in (x, w)]
+    ws = z.batch_workspace(2)
+    z.decompress_batch_into(conts, [c.numel() for c in conts], outs, ws)
+    torch.cuda.synchronize()
+    assert z.status(ws) == z.OK
+    for o, t in zip(outs, (x, w)):
+        assert torch.equal(o.view(torch.int16).cpu(), t.view(torch.int16))
+
+
 def test_fp32_and_clean(z, orc):
     from lossless_float_weight_b200 import workloads as W
     x = W.fp32_tensor(n=(1 << 21) + 333)
