@@ -99,6 +99,20 @@ def test_constant_and_zero_tensors(z, orc):
         _check_roundtrip(z, orc, x, f"constant {x.dtype}")
 
 
+def test_bf16_largest_chunk(z, orc):
+    # chunk_bytes = 2^28, the largest the ABI takes: a chunk of 2^27 values (4096 encode
+    # tiles, 262,144 sub-blocks, a bitstream far beyond the shared-memory window) and a
+    # second chunk of 5 values
+    cb = 1 << 28
+    n = (1 << 27) + 5
+    x = (torch.randn(n, generator=torch.Generator().manual_seed(13)) * 0.02).to(torch.bfloat16)
+    _check_roundtrip(z, orc, x, "bf16 2^28-byte chunks", chunk_bytes=cb)
+    h = z.histogram(x.cuda(), chunk_bytes=cb).cpu().numpy()
+    hb = _host_bytes(x)
+    for c, (lo, hi) in enumerate(((0, 1 << 27), (1 << 27, n))):
+        assert np.array_equal(h[c, 0].astype(np.uint64), orc.histogram("bf16", hb, lo, hi, 0)), c
+
+
 def _mixed_modes_bf16():
     # one tensor whose chunks take every pair of stream modes: zeros (ZERO, ZERO), weights
     # (HUFF, RAW), positive powers of two (HUFF, ZERO), every bit pattern at random
