@@ -19,14 +19,14 @@
  *  - Grouped chunks with shared Huffman codes from a reusable setup: "NeuralZip:
  *    Reusable Setup for Fast Lossless Compression", abstract.
  *
- * Readings where the pages are silent (each one is listed in the design notes):
+ * Readings where the pages are silent:
  *  - Huffman ties: the two nodes with the smallest (weight, order) keys merge first;
  *    a leaf's order is its symbol value, the i-th merged node's order is 256 + i.
  *  - Length limit 12: halve every non-zero frequency (never below 1) and rebuild,
  *    until the longest code is at most 12 bits.
  *  - Canonical code values: the deflate rule (RFC 1951, section 3.2.2).
- *  - Container layout, sub-block index, ZERO/RAW/HUFF choice: the format written in
- *    the design notes; pinned by a hand-derived golden container, not by the pages.
+ *  - Container layout, sub-block index, ZERO/RAW/HUFF choice: the format stated under
+ *    "layout rules" below; pinned by a hand-derived golden container, not by the pages.
  *  - Grouping: Lloyd's k-means with SplitMix64 seeding (parity unpinned by the pages:
  *    pinned only by invariants and small separable cases).
  */
@@ -255,6 +255,24 @@ static uint64_t get_u64(const uint8_t* p) {
 }
 
 /* ------------------------------------------------------------------ layout rules */
+/*
+ * The container (little-endian; every section and payload starts on a 16-byte
+ * boundary; every pad byte and pad bit is zero):
+ *  - header, 64 bytes: "ZN" "N1"; version 1 (u16); dtype (u8); streams per chunk (u8);
+ *    n values (u64); chunk_bytes (u32); S (u32); chunks (u32); shared records (u32);
+ *    offset of the code section (u64); offset of the payloads (u64); total bytes
+ *    (u64); L_MAX = 12 (u8); groups (u8); zeros to byte 64;
+ *  - chunk table, 16 bytes per entry k = chunk * streams + stream: mode (u8: RAW 0,
+ *    ZERO 1, HUFF 2) and three zero bytes; code (u32: the shared record's index, or
+ *    0xFFFFFFFF for a code of the chunk's own); payload offset (u64);
+ *  - code section: the shared records, those of entropy stream 0 for every group,
+ *    then stream 1's; a record is the alphabet's code lengths, 4 bits each (symbol
+ *    2i in the low nibble of byte i), rounded up to 16 bytes;
+ *  - payloads in entry order, each offset the sum of the sizes before it: RAW, the
+ *    stream's symbols at their fixed width, MSB first; ZERO, nothing; HUFF, the
+ *    chunk's own record (when code is 0xFFFFFFFF), then the bit offset (u32) of every
+ *    S-th symbol padded to 16 bytes, then the codes MSB first padded to 16 bytes.
+ */
 
 static uint64_t ceil_div(uint64_t a, uint64_t b) { return (a + b - 1) / b; }
 

@@ -18,8 +18,8 @@
  *    grouped by exponent-distribution similarity share one Huffman code, chosen
  *    once by a reusable setup (the plan).
  * The byte layout of the container, the length limit and the grouping procedure
- * are not given by the pages; the readings this oracle implements are listed in
- * the repository's design notes.
+ * are not given by the pages; the readings this oracle implements are stated in
+ * zipnn_oracle.c (the container layout under "layout rules").
  */
 #ifndef ZIPNN_ORACLE_H
 #define ZIPNN_ORACLE_H
