@@ -117,9 +117,10 @@ def kv_cache(shape=(32, 2, 16, 8, 4096, 128), seed=0, device="cpu"):
 
 
 def spread_bf16(n, binades, seed):
-    """BF16 values whose exponents are uniform over `binades` binades below 0.5 (random
-    sign, fraction uniform in [1, 2)): about log2(binades) bits of exponent entropy, more
-    than trained weights have. A 256 KiB chunk's exponent bitstream comes to about 45 KB
+    """BF16 values whose magnitudes are m * 2^-(e + 1), m uniform in [1, 2) and e uniform
+    in {0, ..., binades - 1}, with a random sign: exponents uniform over the `binades`
+    binades below 1 (rounding to BF16 lifts the few largest to 1.0), about
+    log2(binades) bits of exponent entropy, more than trained weights have. A 256 KiB chunk's exponent bitstream comes to about 45 KB
     for 6 binades, 53 KB for 9, 56 KB for 10 and 65 KB for 16."""
     g = torch.Generator().manual_seed(seed)
     e = torch.randint(0, binades, (n,), generator=g).float()
