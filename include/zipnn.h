@@ -45,6 +45,7 @@
  *   when that payload is strictly smaller than RAW, else RAW.
  *
  * Conventions for every call:
+ *  - n (values) is at most 2^56 - 1, and a tensor has at most 2^31 - 1 chunk entries.
  *  - Device pointers (src, out, in, ws) are owned by the caller, must be 16-byte
  *    aligned, and are only read or written on `stream`, in stream order.
  *  - Compress and decompress are asynchronous; they allocate nothing. Argument errors
@@ -116,9 +117,14 @@ zipnn_status zipnn_compress_ex(zipnn_dtype dtype, const void* src, uint64_t n, u
                                void* ws, size_t ws_bytes, zipnn_stream_t stream);
 
 /* Decompress the container `in` (device, in_bytes readable bytes) into n values at
- * `out` (device). The container must have been made for the same dtype, n and
- * chunk_bytes; anything else, and any damage found, sets ZIPNN_ERR_CORRUPT in the
- * workspace (output contents are then unspecified). Every read stays inside in_bytes. */
+ * `out` (device): the inverse of zipnn_compress, giving back every value bit for bit
+ * ("ZipNN: Lossless Compression for AI Models", abstract: lossless, with decompression
+ * speed as a goal). Each chunk's streams are decoded and merged back into whole values
+ * (the inverse of the split of THEORY-599, "Per-field compressibility (Table II)").
+ * The container must have been made for the same dtype, n and chunk_bytes; anything
+ * else, and any damage found, sets ZIPNN_ERR_CORRUPT in the workspace (output contents
+ * are then unspecified). Every read stays inside in_bytes. ws: at least 256 bytes (only
+ * its status word is used). */
 zipnn_status zipnn_decompress(zipnn_dtype dtype, const void* in, size_t in_bytes, uint64_t n,
                               uint32_t chunk_bytes, void* out, void* ws, size_t ws_bytes,
                               zipnn_stream_t stream);
@@ -155,46 +161,63 @@ zipnn_status zipnn_compressed_size(const void* out, zipnn_stream_t stream, uint6
 /* Wait for `stream`, then return the device-side status of the last call on `ws`. */
 zipnn_status zipnn_get_status(const void* ws, zipnn_stream_t stream);
 
-/* Order-0 histograms (step "split + histogram" alone): hist_out (device, u32) receives
- * n_chunks x n_entropy x 256 counts for the entropy streams of every chunk. */
+/* Order-0 histograms (step "split + histogram" alone; THEORY-599 note, "Order-0 only
+ * (section III-A b)": the model of a chunk is the count of each exponent value, no
+ * context): hist_out (device, u32, 4-byte aligned) receives n_chunks x n_entropy
+ * x 256 counts for the entropy streams of every chunk, symbols past a stream's alphabet
+ * 0. Asynchronous; arguments as for zipnn_compress. */
 zipnn_status zipnn_histogram(zipnn_dtype dtype, const void* src, uint64_t n, uint32_t chunk_bytes,
                              uint32_t* hist_out, zipnn_stream_t stream);
 
-/* Code lengths (step "code build" alone): for `count` histograms of 256 u64 counts
- * (device), writes 256 length bytes each (device): minimum-variance Huffman lengths
- * with ties by (weight, order), limited to ZIPNN_LMAX by halving the counts. Symbols
- * at or above `alphabet` must have count 0. */
+/* Code lengths (step "code build" alone; THEORY-599 note, "Order-0 only (section III-A
+ * b)": a Huffman code built from the order-0 histogram): for `count` histograms of 256
+ * u64 counts (device), writes 256 length bytes each (device): minimum-variance Huffman
+ * lengths with ties by (weight, order), limited to ZIPNN_LMAX by halving the counts.
+ * Counts are full 64-bit values (compared as (count, symbol) pairs); each histogram's
+ * total must stay below 2^64. Symbols at or above `alphabet` (1..256) must have count 0.
+ * count is at most 2^31 - 1. Asynchronous. */
 zipnn_status zipnn_code_lengths(const uint64_t* hist, uint32_t count, uint32_t alphabet, uint8_t* lens_out,
                                 zipnn_stream_t stream);
 
-/* Build a plan on the tensor at `src`: k-means (Lloyd, SplitMix64(seed) seeding, at
- * most 100 passes) over the chunks' normalised exponent histograms into `groups`
- * groups (1..ZIPNN_MAX_GROUPS), then one length-limited Huffman code per group and
- * entropy stream from the group's summed histograms. Setup call: it allocates the
- * plan's device tables and synchronises `stream`. ws as for compress. */
+/* Build a plan ("NeuralZip: Reusable Setup for Fast Lossless Compression", abstract:
+ * chunks with similar exponent distributions are grouped and share a Huffman code, and
+ * this setup is prepared once, before the encodings that use it) on the tensor at `src`:
+ * k-means (Lloyd, SplitMix64(seed) seeding, at most 100 passes) over the chunks'
+ * normalised exponent histograms into `groups` groups (1..ZIPNN_MAX_GROUPS), then one
+ * length-limited Huffman code per group and entropy stream from the group's summed
+ * histograms. Setup call: it allocates the plan's device tables (the caller releases
+ * them with zipnn_plan_destroy) and synchronises `stream`. ws as for compress. */
 zipnn_status zipnn_plan_create(zipnn_dtype dtype, const void* src, uint64_t n, uint32_t chunk_bytes,
                                uint32_t groups, uint64_t seed, void* ws, size_t ws_bytes,
                                zipnn_stream_t stream, zipnn_plan_t** plan);
 
-/* Serialise a plan into host memory: "ZNP1", u8 dtype, u8 groups, 2 zero bytes, then
- * the code records as in the container. *bytes receives the size; host_buf may be NULL
- * to query it. */
+/* Serialise a plan into host memory, so that the setup can be stored and transferred
+ * to other tensors or another compatible model (NeuralZip, abstract: the setup is
+ * precomputed, transferred and reused as the weights evolve): "ZNP1", u8 dtype, u8
+ * groups, 2 zero bytes, then the code records as in the container. *bytes receives the
+ * size; host_buf may be NULL to query it; ZIPNN_ERR_OUT_TOO_SMALL if cap is short. */
 zipnn_status zipnn_plan_export(const zipnn_plan_t* plan, void* host_buf, size_t cap, size_t* bytes);
 
-/* Rebuild a plan from exported bytes (host memory); allocates its device tables. */
+/* Rebuild a plan from exported bytes (host memory; NeuralZip, abstract: a transferred
+ * setup is reused without being rebuilt); allocates its device tables. Records whose
+ * lengths exceed ZIPNN_LMAX or whose Kraft sum exceeds 1, or a damaged header, give
+ * ZIPNN_ERR_CORRUPT. */
 zipnn_status zipnn_plan_import(const void* host_buf, size_t bytes, zipnn_plan_t** plan);
 
-/* Per-chunk group chosen by the plan's k-means (host memory, n_chunks entries of the
- * tensor the plan was built on); *count receives the number of entries. */
+/* Per-chunk group chosen by the plan's k-means (NeuralZip, abstract: grouping of chunks
+ * by exponent distribution) for the tensor the plan was built on (host memory, n_chunks
+ * entries; empty for an imported plan); *count receives the number of entries. */
 zipnn_status zipnn_plan_assignment(const zipnn_plan_t* plan, uint32_t* host_buf, size_t cap, size_t* count);
 
+/* Release a plan and its device tables (NULL is ignored). */
 void zipnn_plan_destroy(zipnn_plan_t* plan);
 
 /* Compress without allocating (the pages have no counterpart of this call). For callers
- * that cannot allocate device memory: code that runs while a CUDA stream capture is
- * active (cudaMalloc is not allowed then), code whose memory is owned by a framework
- * allocator it cannot reach from C, and latency-critical paths that cannot afford the
- * device synchronisation an allocation implies. It behaves as zipnn_compress without a
+ * that cannot allocate device memory: code whose device memory is owned by a framework's
+ * caching allocator that it cannot reach from C (a cudaMalloc of its own would fight
+ * that allocator for memory it has already reserved), and latency-critical paths that
+ * cannot afford the device synchronisation a cudaMalloc/cudaFree pair implies. It
+ * behaves as zipnn_compress without a
  * plan, but its workspace is a file-scope device array of ZIPNN_NOALLOC_SCRATCH_BYTES
  * (8 MiB) that every GPU loading the library holds until the process exits; tensors
  * whose zipnn_workspace_bytes exceed it are rejected with ZIPNN_ERR_UNSUPPORTED before
@@ -206,6 +229,15 @@ void zipnn_plan_destroy(zipnn_plan_t* plan);
 #define ZIPNN_NOALLOC_SCRATCH_BYTES (8u << 20)
 zipnn_status zipnn_compress_noalloc(zipnn_dtype dtype, const void* src, uint64_t n, uint32_t chunk_bytes, void* out,
                                     size_t out_cap, zipnn_stream_t stream);
+
+/* Test aid (not a step of the codec): the number of polls after which a wait on another
+ * block of the same launch (the decoupled look-back of the layout scan and of the FP32,
+ * FP8 and FP4 encode) gives up and records ZIPNN_ERR_TIMEOUT; 0 restores the default
+ * (2^22). It applies to calls made after it, in every host thread. A wait that gives up
+ * has summed only part of its prefix, so every offset it yields is at most the true one
+ * and every write stays inside the output; the container is then invalid and the status
+ * says so. Always returns ZIPNN_OK. */
+zipnn_status zipnn_test_lookback_limit(uint32_t polls);
 
 /* Kernel timing, a measurement aid (off by default; not a step of the codec). While
  * enabled, every kernel the library launches is bracketed by two CUDA events on its

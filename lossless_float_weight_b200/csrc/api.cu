@@ -1,6 +1,7 @@
 // api.cu -- the C ABI of include/zipnn.h: argument checks, workspace carving, launches.
 // No call here computes any part of the codec on the host: histograms, codes, layout,
 // encoding, decoding and the plan's grouping all run in the kernels.
+#include <atomic>
 #include <cstdlib>
 #include <cstring>
 #include <new>
@@ -25,13 +26,19 @@ namespace {
 
 constexpr uint64_t kAlign = 256;
 constexpr uint32_t kMaxChunkBytes = 1u << 28;
+// Largest value count: a plan's group histograms sum up to n counts, and every count
+// stays far below the 64-bit range of the code builder's weights.
+constexpr uint64_t kMaxValues = 1ull << 56;
+
+// Polls after which a look-back wait gives up (zipnn_test_lookback_limit; 0 = default).
+std::atomic<uint32_t> g_spin_limit{0};
 
 inline uint64_t align_up(uint64_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 inline bool valid_dtype(int dt) { return dt == kBF16 || dt == kFP32 || dt == kFP8 || dt == kFP4; }
 
 bool make_geo(int dt, uint64_t n, uint32_t chunk_bytes, uint32_t S, uint32_t G, Geo& g) {
-  if (!valid_dtype(dt) || n == 0) return false;
+  if (!valid_dtype(dt) || n == 0 || n >= kMaxValues) return false;
   if (dt == kFP4 && n % 2) return false;  // FP4 values come in byte pairs
   if (chunk_bytes < 16 || chunk_bytes % 16 || chunk_bytes > kMaxChunkBytes) return false;
   if (S < 16 || S % 16 || S > 65536) return false;
@@ -50,6 +57,8 @@ bool make_geo(int dt, uint64_t n, uint32_t chunk_bytes, uint32_t S, uint32_t G, 
   g.n_entries = (uint32_t)(chunks * n_streams(dt));
   g.off_codes = kHeaderBytes + (uint64_t)kEntryBytes * g.n_entries;
   g.off_payload = g.off_codes + shared_bytes(dt, G);
+  const uint32_t lim = g_spin_limit.load(std::memory_order_relaxed);
+  g.spin_limit = lim ? lim : kSpinLimit;
   return true;
 }
 
@@ -128,18 +137,26 @@ PlanDev plan_dev(const zipnn_plan* p) {
   return d;
 }
 
-// The kernels are built for sm_100a only; the answer is cached per device.
-bool device_ok() {
-  static int cache[128] = {0};  // 0 unknown, 1 usable, 2 not
+}  // namespace
+
+// The kernels are built for sm_100a only; the answer is cached per device (several host
+// threads may ask at once).
+bool zipnn::device_ok() {
+  static std::atomic<int> cache[128];  // 0 unknown, 1 usable, 2 not
   int dev = 0, major = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return false;
-  if (dev >= 0 && dev < 128 && cache[dev]) return cache[dev] == 1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  if (dev >= 0 && dev < 128) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c) return c == 1;
+  }
   const bool ok = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) == cudaSuccess && major == 10;
-  if (dev >= 0 && dev < 128) cache[dev] = ok ? 1 : 2;
+  if (!ok) cudaGetLastError();
+  if (dev >= 0 && dev < 128) cache[dev].store(ok ? 1 : 2, std::memory_order_relaxed);
   return ok;
 }
-
-}  // namespace
 
 extern "C" {
 
@@ -288,7 +305,7 @@ zipnn_status zipnn_histogram(zipnn_dtype dtype, const void* src, uint64_t n, uin
 
 zipnn_status zipnn_code_lengths(const uint64_t* hist, uint32_t count, uint32_t alphabet, uint8_t* lens_out,
                                 zipnn_stream_t stream) {
-  if (!hist || !lens_out || alphabet < 1 || alphabet > 256) return ZIPNN_ERR_INVALID_ARG;
+  if (!hist || !lens_out || alphabet < 1 || alphabet > 256 || count > 0x7FFFFFFFu) return ZIPNN_ERR_INVALID_ARG;
   if (!device_ok()) return ZIPNN_ERR_UNSUPPORTED;
   return cuda_status(launch_code_lengths(hist, count, alphabet, lens_out, nullptr, reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -470,6 +487,11 @@ void zipnn_plan_destroy(zipnn_plan_t* plan) {
   if (plan->d_lens) cudaFree(plan->d_lens);
   if (plan->d_enc) cudaFree(plan->d_enc);
   delete plan;
+}
+
+zipnn_status zipnn_test_lookback_limit(uint32_t polls) {
+  g_spin_limit.store(polls, std::memory_order_relaxed);
+  return ZIPNN_OK;
 }
 
 const char* zipnn_status_string(zipnn_status status) {

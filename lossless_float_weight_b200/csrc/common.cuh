@@ -79,6 +79,7 @@ struct Geo {
   uint32_t n_tiles;           // n_chunks * tiles_per_chunk
   uint32_t n_entries;         // n_chunks * n_streams
   uint64_t off_codes, off_payload;
+  uint32_t spin_limit;        // polls after which a look-back wait gives up (kSpinLimit by default)
 };
 
 // Workspace carve-up (device pointers). The first group is cleared by every
@@ -114,8 +115,9 @@ __device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 
 // ---------------------------------------------------------------- look-back
 // Descriptor: bits 63..62 flag (0 empty, 1 aggregate, 2 inclusive prefix), 61..0 value.
 constexpr uint64_t kFlagAgg = 1ull << 62, kFlagPrefix = 2ull << 62, kValueMask = (1ull << 62) - 1;
-// Spin limit for every wait on another block; after it the wait records a timeout and
-// continues, so no kernel can hang on a descriptor that is never written.
+// Default spin limit for every wait on another block; after it the wait records a timeout
+// and continues, so no kernel can hang on a descriptor that is never written. A call can
+// lower it (Geo::spin_limit) so that a test can make a healthy wait run out.
 constexpr uint32_t kSpinLimit = 1u << 22;
 
 __device__ __forceinline__ void publish(uint64_t* d, uint64_t v) {
@@ -133,9 +135,11 @@ __device__ __forceinline__ uint64_t observe(uint64_t* d) {
 // otherwise all 32 aggregates are summed and the window moves back. Publishes the
 // inclusive prefix and returns the exclusive one (to every lane). Tiles are handed out
 // in launch order (a ticket), so every predecessor has started and the walk ends; the
-// spin limit only guards against bugs.
+// spin limit only guards against bugs. A walk that gives up returns the part of the
+// prefix it has summed, never more than the true prefix, so every offset derived from it
+// stays inside the true extent (payloads may then overlap, and the status says timeout).
 __device__ inline uint64_t warp_lookback(uint64_t* desc, uint32_t tile, uint32_t first, uint64_t aggregate,
-                                         uint32_t* status) {
+                                         uint32_t* status, uint32_t limit = kSpinLimit) {
   const int lane = threadIdx.x & 31;
   if (tile == first) {
     if (lane == 0) publish(desc + tile, kFlagPrefix | aggregate);
@@ -154,7 +158,7 @@ __device__ inline uint64_t warp_lookback(uint64_t* desc, uint32_t tile, uint32_t
     const int pl = is_prefix ? __ffs(is_prefix) - 1 : 32;  // nearest prefix
     const uint32_t need = pl == 32 ? 0xFFFFFFFFu : (uint32_t)((2ull << pl) - 1);
     if (not_ready & need) {
-      if (++spins > kSpinLimit) {
+      if (++spins > limit) {
         if (lane == 0) set_status(status, kStTimeout);
         break;
       }

@@ -15,6 +15,8 @@
 // offset idx[j], merges the streams back into BF16/FP32/FP8 words and writes them to
 // HBM with 16-byte stores: no intermediate plane is materialised. A sub-block must end
 // exactly where the next one starts.
+#include <atomic>
+
 #include "bulk.cuh"
 #include "common.cuh"
 #include "fields.cuh"
@@ -898,15 +900,15 @@ __global__ void __launch_bounds__(kDecodeThreads, DT == kBF16 ? 3 : 1)
 
 // Dynamic shared memory (the BF16 staging window) once per device and kernel.
 template <class K>
-static cudaError_t decode_attributes(K kernel, size_t dyn, int* done) {
+static cudaError_t decode_attributes(K kernel, size_t dyn, std::atomic<int>* done) {
   if (!dyn) return cudaSuccess;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < 128 && done[dev]) return cudaSuccess;
+  if (dev >= 0 && dev < 128 && done[dev].load(std::memory_order_relaxed)) return cudaSuccess;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-  if (e == cudaSuccess && dev >= 0 && dev < 128) done[dev] = 1;
+  if (e == cudaSuccess && dev >= 0 && dev < 128) done[dev].store(1, std::memory_order_relaxed);
   return e;
 }
 
@@ -914,7 +916,7 @@ template <int DT>
 static cudaError_t decode_t(const uint8_t* in, uint64_t in_bytes, const Geo& g, uint8_t* out, uint32_t* status,
                             cudaStream_t st) {
   const size_t dyn = DT == kBF16 ? sizeof(StagedSmem) : 0;
-  static int done[128] = {0};
+  static std::atomic<int> done[128];
   cudaError_t e = decode_attributes(k_decode<DT>, dyn, done);
   if (e != cudaSuccess) return e;
   k_decode<DT><<<g.n_chunks, kDecodeThreads, dyn, st>>>(in, in_bytes, g, out, status);
@@ -925,7 +927,7 @@ template <int DT>
 static cudaError_t decode_batch_t(const DecodeItem* items, uint32_t count, const Geo& g, uint32_t total_chunks,
                                   uint32_t* status, cudaStream_t st) {
   const size_t dyn = DT == kBF16 ? sizeof(StagedSmem) : 0;
-  static int done[128] = {0};
+  static std::atomic<int> done[128];
   cudaError_t e = decode_attributes(k_decode_batch<DT>, dyn, done);
   if (e != cudaSuccess) return e;
   k_decode_batch<DT><<<total_chunks, kDecodeThreads, dyn, st>>>(items, count, g, status);

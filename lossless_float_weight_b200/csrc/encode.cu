@@ -18,6 +18,8 @@
 //  * the sub-block index idx[j] (bit offset of symbol j*S) is written by the thread
 //    that owns symbol j*S; the first tile writes a local code record, the last tile the
 //    zero padding.
+#include <atomic>
+
 #include "common.cuh"
 #include "fields.cuh"
 #include "launch.h"
@@ -185,7 +187,8 @@ __global__ void __launch_bounds__(kEncodeThreads) k_encode(const uint8_t* __rest
       if (huff) {
         const uint32_t e = s < NE ? s : 0;
         const uint64_t p =
-            warp_lookback(ws.tile_desc + (uint64_t)e * g.n_tiles, tile, c * g.tiles_per_chunk, tile_bits, ws.status);
+            warp_lookback(ws.tile_desc + (uint64_t)e * g.n_tiles, tile, c * g.tiles_per_chunk, tile_bits, ws.status,
+                          g.spin_limit);
         if (tid == 0) sm.prefix = p;
       } else if (tid == 0) {
         sm.prefix = (uint64_t)tlo * (uint64_t)w;
@@ -259,15 +262,15 @@ __global__ void __launch_bounds__(kEncodeThreads) k_encode(const uint8_t* __rest
 template <int DT>
 static cudaError_t encode_t(const void* src, const Geo& g, const Ws& ws, uint8_t* out, cudaStream_t st) {
   const size_t smem = sizeof(EncodeSmem<DT>);
-  static int done[128] = {0};
+  static std::atomic<int> done[128];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 128 || !done[dev]) {
+  if (dev < 0 || dev >= 128 || !done[dev].load(std::memory_order_relaxed)) {
     e = cudaFuncSetAttribute(k_encode<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(k_encode<DT>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 128) done[dev] = 1;
+    if (dev >= 0 && dev < 128) done[dev].store(1, std::memory_order_relaxed);
   }
   k_encode<DT><<<g.n_tiles, kEncodeThreads, smem, st>>>(static_cast<const uint8_t*>(src), g, ws, out);
   return cudaGetLastError();

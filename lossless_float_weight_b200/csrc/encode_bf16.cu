@@ -21,6 +21,8 @@
 //    (1 << 32 | its bits) and the side that arrives second stores the complete word.
 // The sub-block index idx[j] (bit offset of symbol j*S) is written by the thread that
 // owns symbol j*S; the first tile writes a local code record, the last the padding.
+#include <atomic>
+
 #include "common.cuh"
 #include "fields.cuh"
 #include "launch.h"
@@ -234,11 +236,11 @@ __global__ void __launch_bounds__(kBThreads, 8) k_encode_bf16(const uint8_t* __r
 // Launch: a persistent grid of as many blocks as fit on the device at once.
 cudaError_t launch_encode_bf16(const void* src, const Geo& g, const Ws& ws, uint8_t* out, cudaStream_t st) {
   const size_t smem = sizeof(Bf16EncodeSmem);
-  static int resident[128] = {0};  // blocks per device, once the attributes are set
+  static std::atomic<int> resident[128];  // blocks per device, once the attributes are set
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  int per_device = dev >= 0 && dev < 128 ? resident[dev] : 0;
+  int per_device = dev >= 0 && dev < 128 ? resident[dev].load(std::memory_order_relaxed) : 0;
   if (!per_device) {
     e = cudaFuncSetAttribute(k_encode_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(k_encode_bf16, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
@@ -247,7 +249,7 @@ cudaError_t launch_encode_bf16(const void* src, const Geo& g, const Ws& ws, uint
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     per_device = (per_sm > 0 ? per_sm : 1) * (sms > 0 ? sms : 1);
-    if (dev >= 0 && dev < 128) resident[dev] = per_device;
+    if (dev >= 0 && dev < 128) resident[dev].store(per_device, std::memory_order_relaxed);
   }
   const uint32_t blocks = (uint32_t)min64((uint64_t)per_device, g.n_tiles);
   k_encode_bf16<<<blocks, kBThreads, smem, st>>>(static_cast<const uint8_t*>(src), g, ws, out);

@@ -7,7 +7,8 @@
 //  * ties: the two nodes with the smallest (weight, order) keys merge first, a leaf's
 //    order being its symbol and the i-th merged node's order 256 + i (minimum-variance
 //    Huffman). Leaves sorted by (weight, symbol) and merged nodes in creation order
-//    form two queues whose heads give that minimum, a leaf winning a weight tie;
+//    form two queues whose heads give that minimum, a leaf winning a weight tie.
+//    Weights are full 64-bit counts, compared as (weight, symbol) pairs;
 //  * length limit 12: the code of the weights max(1, f >> k) for the smallest k >= 0
 //    whose longest code is at most 12 bits. The eight warps of a block try eight
 //    values of k at once;
@@ -20,8 +21,10 @@ namespace zipnn {
 constexpr int kHuffWarps = 8;
 
 struct HuffScratch {
-  uint64_t sorted[256];  // leaves (weight << 8 | symbol), ascending
-  uint64_t iw[256];      // unsorted leaf keys, then merged-node weights
+  uint64_t sorted[256];  // leaf weights in ascending (weight, symbol) order
+  uint64_t iw[256];      // leaf weights in symbol order, then merged-node weights
+  uint8_t ssym[256];     // symbol of sorted leaf i
+  uint8_t isym[256];     // symbol of leaf iw[i] (read only before the merge reuses iw)
   uint16_t lpar[256];    // parent (merged-node index) of sorted leaf i
   uint16_t ipar[256];    // parent of merged node i
   uint8_t idep[256];     // depth of merged node i
@@ -46,22 +49,30 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
-// The same code as warp_huffman below for 2 <= n <= 32 present symbols whose keys
-// (weight << 8 | symbol) are in sc.iw[0..n), with every per-node quantity in registers:
-// lane p holds the p-th smallest leaf and the p-th merged node. The two-queue merge
-// runs on all lanes in step (its indices and sums are warp-uniform) and fetches queue
-// heads by shuffle; depths follow by pointer jumping towards the root.
+// The same code as warp_huffman below for 2 <= n <= 32 present symbols whose weights and
+// symbols are in sc.iw[0..n) and sc.isym[0..n), with every per-node quantity in
+// registers: lane p holds the p-th smallest leaf and the p-th merged node. The two-queue
+// merge runs on all lanes in step (its indices and sums are warp-uniform) and fetches
+// queue heads by shuffle; depths follow by pointer jumping towards the root.
 __device__ inline int warp_huffman_regs(HuffScratch& sc, int n) {
   const int lane = threadIdx.x & 31;
-  const uint64_t key = lane < n ? sc.iw[lane] : ~0ull;
-  // rank of my key among the n distinct keys, then leaves in ascending key order
+  const uint64_t w = lane < n ? sc.iw[lane] : ~0ull;
+  const uint32_t sy = lane < n ? sc.isym[lane] : 0xFFu;
+  // rank of my leaf among the n leaves in (weight, symbol) order (symbols are distinct)
   int r = 0;
 #pragma unroll
-  for (int q = 0; q < 32; q++) r += __shfl_sync(0xFFFFFFFFu, key, q) < key;
-  if (lane < n) sc.sorted[r] = key;
+  for (int q = 0; q < 32; q++) {
+    const uint64_t wq = __shfl_sync(0xFFFFFFFFu, w, q);
+    const uint32_t sq = __shfl_sync(0xFFFFFFFFu, sy, q);
+    r += q < n && (wq < w || (wq == w && sq < sy));
+  }
+  if (lane < n) {
+    sc.sorted[r] = w;
+    sc.ssym[r] = (uint8_t)sy;
+  }
   __syncwarp();
-  const uint64_t leaf_key = lane < n ? sc.sorted[lane] : ~0ull;
-  const uint64_t leaf_w = leaf_key >> 8;
+  const uint64_t leaf_w = lane < n ? sc.sorted[lane] : ~0ull;
+  const uint32_t leaf_s = sc.ssym[lane];
   uint64_t node_w = 0;
   uint32_t leaf_par = 0, node_par = 0;
   uint32_t li = 0, ii = 0;
@@ -98,7 +109,7 @@ __device__ inline int warp_huffman_regs(HuffScratch& sc, int n) {
     up = uu;
   }
   const uint32_t len = __shfl_sync(0xFFFFFFFFu, d, leaf_par & 31) + 1;
-  if (lane < n) sc.lens[leaf_key & 0xFF] = (uint8_t)len;
+  if (lane < n) sc.lens[leaf_s] = (uint8_t)len;
   __syncwarp();
   return (int)__reduce_max_sync(0xFFFFFFFFu, lane < n ? len : 0u);
 }
@@ -117,7 +128,9 @@ __device__ inline int warp_huffman(const uint64_t* f, int A, int k, HuffScratch&
     if (p) {
       uint64_t g = k < 64 ? (fs >> k) : 0;
       if (g == 0) g = 1;
-      sc.iw[n + __popc(b & lanemask_lt())] = (g << 8) | (uint64_t)s;
+      const int at = n + __popc(b & lanemask_lt());
+      sc.iw[at] = g;
+      sc.isym[at] = (uint8_t)s;
     }
     n += __popc(b);
   }
@@ -125,17 +138,22 @@ __device__ inline int warp_huffman(const uint64_t* f, int A, int k, HuffScratch&
   __syncwarp();
   if (n == 0) return 0;
   if (n == 1) {
-    if (lane == 0) sc.lens[sc.iw[0] & 0xFF] = 1;
+    if (lane == 0) sc.lens[sc.isym[0]] = 1;
     __syncwarp();
     return 1;
   }
   if (n <= 32) return warp_huffman_regs(sc, n);
   // rank sort of the distinct keys (weight, symbol)
   for (int p = lane; p < n; p += 32) {
-    const uint64_t kp = sc.iw[p];
+    const uint64_t wp = sc.iw[p];
+    const uint32_t sp = sc.isym[p];
     int r = 0;
-    for (int q = 0; q < n; q++) r += sc.iw[q] < kp;
-    sc.sorted[r] = kp;
+    for (int q = 0; q < n; q++) {
+      const uint64_t wq = sc.iw[q];
+      r += wq < wp || (wq == wp && sc.isym[q] < sp);
+    }
+    sc.sorted[r] = wp;
+    sc.ssym[r] = (uint8_t)sp;
   }
   __syncwarp();
   if (lane == 0) {
@@ -145,9 +163,9 @@ __device__ inline int warp_huffman(const uint64_t* f, int A, int k, HuffScratch&
       uint64_t sum = 0;
 #pragma unroll
       for (int pick = 0; pick < 2; pick++) {
-        const bool leaf = li < n && (ii >= t || (sc.sorted[li] >> 8) <= sc.iw[ii]);
+        const bool leaf = li < n && (ii >= t || sc.sorted[li] <= sc.iw[ii]);
         if (leaf) {
-          sum += sc.sorted[li] >> 8;
+          sum += sc.sorted[li];
           sc.lpar[li] = (uint16_t)t;
           li++;
         } else {
@@ -165,7 +183,7 @@ __device__ inline int warp_huffman(const uint64_t* f, int A, int k, HuffScratch&
   int mx = 0;
   for (int p = lane; p < n; p += 32) {
     const int d = sc.idep[sc.lpar[p]] + 1;
-    sc.lens[sc.sorted[p] & 0xFF] = (uint8_t)(d > 255 ? 255 : d);
+    sc.lens[sc.ssym[p]] = (uint8_t)(d > 255 ? 255 : d);
     mx = d > mx ? d : mx;
   }
   __syncwarp();

@@ -5,6 +5,10 @@
 
 namespace zipnn {
 
+// True when the current device is an sm_100 part that can run the kernels (cached per
+// device).
+bool device_ok();
+
 // Kernel ids of the optional event timing (timing.cu).
 enum KernelId { kIdHist = 0, kIdBuild, kIdLayout, kIdEncode, kIdDecode, kIdCodeLengths, kIdPlan, kNumKernelIds };
 

@@ -4,6 +4,7 @@
 #include <mutex>
 
 #include "zipnn.h"
+#include "launch.h"
 
 namespace {
 
@@ -22,8 +23,14 @@ extern "C" zipnn_status zipnn_compress_noalloc(zipnn_dtype dtype, const void* sr
   const size_t need = zipnn_workspace_bytes(dtype, n, chunk_bytes);
   if (need == 0) return ZIPNN_ERR_INVALID_ARG;
   if (need > ZIPNN_NOALLOC_SCRATCH_BYTES) return ZIPNN_ERR_UNSUPPORTED;  // tensor beyond the fixed scratch
+  // the same device check as zipnn_compress, before the module is touched: on a device
+  // the kernels were not built for, the symbol lookup below would fail
+  if (!zipnn::device_ok()) return ZIPNN_ERR_UNSUPPORTED;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return ZIPNN_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) {
+    cudaGetLastError();
+    return ZIPNN_ERR_CUDA;
+  }
   void* ws = nullptr;
   {
     // once per device, with that device current: the device address of the array (the
@@ -31,7 +38,10 @@ extern "C" zipnn_status zipnn_compress_noalloc(zipnn_dtype dtype, const void* sr
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
     if (!g_noalloc_addr[dev]) {
       void* p = nullptr;
-      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return ZIPNN_ERR_CUDA;
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+        cudaGetLastError();  // leave no sticky error behind for the caller's own checks
+        return ZIPNN_ERR_CUDA;
+      }
       g_noalloc_addr[dev] = p;
     }
     ws = g_noalloc_addr[dev];

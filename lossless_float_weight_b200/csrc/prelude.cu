@@ -10,6 +10,8 @@
 //                    types: the histogram block that finishes a chunk last;
 //   k_layout       : exclusive scan of payload sizes (single-pass decoupled look-back)
 //                    into payload offsets; writes header, chunk table, shared records.
+#include <atomic>
+
 #include "bulk.cuh"
 #include "common.cuh"
 #include "fields.cuh"
@@ -391,7 +393,7 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout(Geo g, Ws ws, PlanDev
   uint64_t total;
   uint64_t before = block_scan_u64(mine, s_warp, total);
   if (tid < 32) {
-    const uint64_t p = warp_lookback(ws.scan_desc, tile, 0, total, ws.status);
+    const uint64_t p = warp_lookback(ws.scan_desc, tile, 0, total, ws.status, g.spin_limit);
     if (tid == 0) s_prefix = p;
   }
   __syncthreads();
@@ -450,14 +452,29 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout(Geo g, Ws ws, PlanDev
 
 // ---------------------------------------------------------------- launchers
 
-// BF16: a persistent grid of as many histogram blocks as fit on the device at once.
-static cudaError_t split_hist_bf16(const void* src, const Geo& g, uint32_t* hist, uint32_t* nonzero, const Ws* ws,
-                                   const PlanDev& plan, cudaStream_t st) {
-  static int resident[128] = {0};  // blocks per device, once the attributes are set
+// Opt a kernel into more than 48 KB of dynamic shared memory, once per device. Slots:
+// 3 k_code_lengths, 4 k_build_chunks, 4 + DT k_split_hist<DT>.
+template <typename K>
+static cudaError_t allow_smem(K kernel, size_t bytes, int slot) {
+  static std::atomic<int> done[8][128];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  int per_device = dev >= 0 && dev < 128 ? resident[dev] : 0;
+  if (dev >= 0 && dev < 128 && done[slot][dev].load(std::memory_order_relaxed)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < 128) done[slot][dev].store(1, std::memory_order_relaxed);
+  return e;
+}
+
+
+// BF16: a persistent grid of as many histogram blocks as fit on the device at once.
+static cudaError_t split_hist_bf16(const void* src, const Geo& g, uint32_t* hist, uint32_t* nonzero, const Ws* ws,
+                                   const PlanDev& plan, cudaStream_t st) {
+  static std::atomic<int> resident[128];  // blocks per device, once the attributes are set
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  int per_device = dev >= 0 && dev < 128 ? resident[dev].load(std::memory_order_relaxed) : 0;
   if (!per_device) {
     e = cudaFuncSetAttribute(k_split_hist_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kHbSmemBytes);
     int per_sm = 0, sms = 0;
@@ -466,7 +483,7 @@ static cudaError_t split_hist_bf16(const void* src, const Geo& g, uint32_t* hist
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     per_device = (per_sm > 0 ? per_sm : 1) * (sms > 0 ? sms : 1);
-    if (dev >= 0 && dev < 128) resident[dev] = per_device;
+    if (dev >= 0 && dev < 128) resident[dev].store(per_device, std::memory_order_relaxed);
   }
   Ws w{};
   if (ws) w = *ws;
@@ -478,6 +495,8 @@ static cudaError_t split_hist_bf16(const void* src, const Geo& g, uint32_t* hist
 
 cudaError_t launch_build_chunks(const Geo& g, const Ws& ws, const PlanDev& plan, cudaStream_t st) {
   if (g.dt != kBF16) return cudaErrorInvalidValue;
+  const cudaError_t e = allow_smem(k_build_chunks<kBF16>, sizeof(HuffBlockSmem), 4);
+  if (e != cudaSuccess) return e;
   k_build_chunks<kBF16><<<g.n_chunks, kHuffWarps * 32, sizeof(HuffBlockSmem), st>>>(g, ws, plan);
   return cudaGetLastError();
 }
@@ -491,6 +510,8 @@ static cudaError_t split_hist_t(const void* src, const Geo& g, uint32_t* hist, u
   constexpr int NE = n_entropy(DT);
   constexpr size_t cols = (size_t)(alphabet(DT, 0) + (NE > 1 ? alphabet(DT, 1) : 0)) * 32 * 4;
   const size_t smem = ws ? (sizeof(HuffBlockSmem) > cols ? sizeof(HuffBlockSmem) : cols) : cols;
+  const cudaError_t e = allow_smem(k_split_hist<DT>, sizeof(HuffBlockSmem) > cols ? sizeof(HuffBlockSmem) : cols, 4 + DT);
+  if (e != cudaSuccess) return e;
   Ws w{};
   if (ws) w = *ws;
   k_split_hist<DT><<<(uint32_t)blocks, kHistThreads, smem, st>>>(static_cast<const uint8_t*>(src), g, slices, hist,
@@ -506,19 +527,6 @@ cudaError_t launch_split_hist(const void* src, const Geo& g, uint32_t* hist, uin
     case kFP8: return split_hist_t<kFP8>(src, g, hist, nonzero, ws, plan, st);
     default: return split_hist_t<kFP4>(src, g, hist, nonzero, ws, plan, st);
   }
-}
-
-// Opt a kernel into more than 48 KB of dynamic shared memory, once per device.
-template <typename K>
-static cudaError_t allow_smem(K kernel, size_t bytes, int slot) {
-  static int done[8][128] = {{0}};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < 128 && done[slot][dev]) return cudaSuccess;
-  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-  if (e == cudaSuccess && dev >= 0 && dev < 128) done[slot][dev] = 1;
-  return e;
 }
 
 cudaError_t launch_code_lengths(const uint64_t* hist, uint32_t count, uint32_t alphabet_size, uint8_t* lens,

@@ -56,6 +56,7 @@ zipnn_timing_collect = _sig("zipnn_timing_collect", _i, _vp, _vp, _u32)
 zipnn_kernel_count = _sig("zipnn_kernel_count", _u32)
 zipnn_kernel_name = _sig("zipnn_kernel_name", ctypes.c_char_p, _u32)
 zipnn_compress_noalloc = _sig("zipnn_compress_noalloc", _i, _i, _vp, _u64, _u32, _vp, _sz, _vp)
+zipnn_test_lookback_limit = _sig("zipnn_test_lookback_limit", _i, _u32)
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -74,7 +75,7 @@ C_ABI_NAMES = [
     "zipnn_plan_create", "zipnn_plan_export", "zipnn_plan_import", "zipnn_plan_assignment", "zipnn_plan_destroy",
     "zipnn_status_string", "zipnn_timing_enable", "zipnn_timing_collect", "zipnn_kernel_count",
     "zipnn_kernel_name", "zipnn_compress_noalloc", "zipnn_decompress_batch_workspace_bytes",
-    "zipnn_decompress_batch",
+    "zipnn_decompress_batch", "zipnn_test_lookback_limit",
 ]
 
 

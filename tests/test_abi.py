@@ -79,3 +79,32 @@ def test_batch_argument_errors_without_a_device(lib):
     assert Z.zipnn_decompress_batch(Z.BF16, 1000, 2, good, fake, ws_bytes, None) == Z.ERR_INVALID_ARG
     # a workspace one byte short
     assert Z.zipnn_decompress_batch(Z.BF16, 262144, 2, good, fake, ws_bytes - 1, None) == Z.ERR_OUT_TOO_SMALL
+
+
+def test_code_lengths_and_size_limits_without_a_device(lib):
+    from lossless_float_weight_b200 import zipnn as Z
+    fake = 1 << 20  # never dereferenced: each case is rejected before a launch
+    for alphabet in (0, 257, 1000):
+        assert Z.zipnn_code_lengths(fake, 1, alphabet, fake, None) == Z.ERR_INVALID_ARG
+    assert Z.zipnn_code_lengths(fake, 1 << 31, 256, fake, None) == Z.ERR_INVALID_ARG
+    # value counts at or above 2^56 are outside the library's range
+    assert Z.zipnn_max_compressed_bytes(Z.BF16, 1 << 56, 262144) == 0
+    assert Z.zipnn_workspace_bytes(Z.FP8_E4M3, (1 << 56) + 16, 262144) == 0
+    assert Z.zipnn_compress(Z.BF16, fake, 1 << 56, 262144, None, fake, 1 << 62, fake, 1 << 40, None) \
+        == Z.ERR_INVALID_ARG
+
+
+def test_lookback_limit_is_a_host_setting(lib):
+    from lossless_float_weight_b200 import zipnn as Z
+    assert Z.zipnn_test_lookback_limit(1) == Z.OK
+    assert Z.zipnn_test_lookback_limit(0) == Z.OK  # back to the default
+
+
+def test_no_device_is_reported_as_unsupported(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    from lossless_float_weight_b200 import zipnn as Z
+    fake = 1 << 20
+    assert Z.zipnn_code_lengths(fake, 1, 256, fake, None) == Z.ERR_UNSUPPORTED
+    assert Z.zipnn_compress_noalloc(Z.BF16, fake, 1000, 262144, fake, 1 << 20, None) == Z.ERR_UNSUPPORTED
