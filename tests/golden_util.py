@@ -33,12 +33,79 @@ def three_chunk_input():
     return x
 
 
+def fp8_two_chunk_input():
+    """The 293 FP8 E4M3 values of fp8_two_chunks.json: built from their numeric meaning
+    (-1)^sign * (1 + M/8) * 2^(E - 7), cast to float8_e4m3fn, and checked against the
+    bit layout the fixture states (sign bit 7, exponent bits 6..3, mantissa bits 2..0)."""
+    E = [7, 7, 6, 9]
+    M = [0] * 12 + [1, 1, 2, 3]
+    vals, bits = [], []
+    for i in range(256):
+        s, e, m = int(i % 8 == 0), E[i % 4], M[i % 16]
+        vals.append((-1.0) ** s * (1 + m / 8) * 2.0 ** (e - 7))
+        bits.append(s << 7 | e << 3 | m)
+    for j in range(37):
+        vals.append(1 + (j % 8) / 8)
+        bits.append(7 << 3 | (j % 8))
+    x = torch.tensor(vals, dtype=torch.float64).to(torch.float8_e4m3fn)
+    assert x.view(torch.uint8).tolist() == bits
+    assert torch.equal(x.to(torch.float64), torch.tensor(vals, dtype=torch.float64))  # exact in E4M3
+    return x
+
+
+def fp32_clean_two_chunk_input():
+    """The 261 FP32 values of fp32_clean_two_chunks.json, from their numeric meaning, with
+    the stated fields checked: chunk 0 has zero fraction bits 15..0, chunk 1 fraction j+1."""
+    E = [127, 127, 126, 128]
+    vals, bits = [], []
+    for i in range(256):
+        b = 255 - i
+        vals.append((-1.0) ** (b >> 7) * (1 + (b & 127) / 128) * 2.0 ** (E[i % 4] - 127))
+        bits.append((b >> 7) << 31 | E[i % 4] << 23 | (b & 127) << 16)
+    for j in range(5):
+        vals.append(-2.0 * (1 + (j + 1) * 2.0 ** -23))
+        bits.append(1 << 31 | 128 << 23 | (j + 1))
+    x = torch.tensor(vals, dtype=torch.float64).to(torch.float32)
+    assert torch.equal(x.to(torch.float64), torch.tensor(vals, dtype=torch.float64))  # exact in FP32
+    assert [v & 0xFFFFFFFF for v in x.view(torch.int32).tolist()] == bits
+    return x
+
+
+def _e2m1(nibble):
+    """The number an E2M1 nibble stands for: sign bit 3, exponent bits 2..1, mantissa bit 0;
+    exponent 0 is subnormal (mantissa * 0.5), else (1 + mantissa/2) * 2^(exponent - 1)."""
+    s, e, m = nibble >> 3, (nibble >> 1) & 3, nibble & 1
+    mag = m * 0.5 if e == 0 else (1 + m / 2) * 2.0 ** (e - 1)
+    return -mag if s else mag
+
+
+def fp4_two_chunk_input():
+    """The 522 FP4 values of fp4_two_chunks.json as torch.float4_e2m1fn_x2 (value 2i in the
+    low nibble of byte i). The nibbles are built from the rule's fields, and their numbers
+    are checked against the E2M1 table of the workloads (0, 0.5, 1, 1.5, 2, 3, 4, 6)."""
+    from lossless_float_weight_b200.workloads import FP4_GRID
+    X = [1, 1, 1, 1, 1, 1, 0, 2]
+    nib = []
+    for v in range(512):
+        nib.append(int(v % 4 == 3) << 3 | X[v % 8] << 1 | int(v % 8 == 1))
+    for j in range(10):
+        nib.append((3 - j % 4) << 1 | 1)
+    assert [_e2m1(k) for k in range(8)] == list(FP4_GRID)
+    assert nib[:8] == [0x2, 0x3, 0x2, 0xA, 0x2, 0x2, 0x0, 0xC]
+    data = bytes(nib[2 * i] | nib[2 * i + 1] << 4 for i in range(len(nib) // 2))
+    assert data[:4] == bytes.fromhex("32a222c0") and data[256:] == bytes.fromhex("5713571357")
+    return torch.frombuffer(bytearray(data), dtype=torch.uint8).view(torch.float4_e2m1fn_x2)
+
+
 def plan_lens(fx):
+    """A fixture's hand-written plan as (entropy streams, groups, 256) length bytes."""
     G = fx["plan"]["n_groups"]
-    lens = np.zeros((1, G, 256), dtype=np.uint8)
-    for g, d in fx["plan"]["lens"].items():
-        for sym, ln in d.items():
-            lens[0, int(g), int(sym)] = ln
+    by_stream = fx["plan"].get("lens_by_stream") or [fx["plan"]["lens"]]
+    lens = np.zeros((len(by_stream), G, 256), dtype=np.uint8)
+    for e, groups in enumerate(by_stream):
+        for g, d in groups.items():
+            for sym, ln in d.items():
+                lens[e, int(g), int(sym)] = ln
     return lens
 
 
@@ -52,6 +119,9 @@ def _part_bytes(p):
     if "hex_range" in p:
         lo, hi = p["hex_range"]
         out += bytes(range(lo, hi + 1))
+    if "hex_range_down" in p:
+        hi, lo = p["hex_range_down"]
+        out += bytes(range(hi, lo - 1, -1))
     if "u32" in p:
         raw = b"".join(struct.pack("<I", v) for v in p["u32"])
         out += raw + b"\0" * ((-len(raw)) % 16)

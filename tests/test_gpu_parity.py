@@ -65,6 +65,38 @@ def test_golden_containers(z, orc):
     assert torch.equal(y.cpu(), x.cpu())
 
 
+# every hand-derived golden container: (fixture, input builder, shared-code plan?)
+GOLDEN_ALL = [
+    ("bf16_three_chunks.json", GU.three_chunk_input, False),
+    ("bf16_shared_code.json", GU.three_chunk_input, True),
+    ("fp8_two_chunks.json", GU.fp8_two_chunk_input, False),
+    ("fp8_shared_code.json", GU.fp8_two_chunk_input, True),
+    ("fp32_clean_two_chunks.json", GU.fp32_clean_two_chunk_input, False),
+    ("fp4_two_chunks.json", GU.fp4_two_chunk_input, False),
+]
+
+
+@pytest.mark.parametrize("name,make,with_plan", GOLDEN_ALL)
+def test_golden_containers_every_dtype(z, name, make, with_plan):
+    """The library writes each hand-derived container byte for byte and decodes it back.
+    A fixture's hand-written plan enters through zipnn_plan_import: its exported form is
+    "ZNP1", dtype, groups, two zero bytes, then the container's shared records."""
+    fx = GU.load(name)
+    src = GU.load(fx["input"]["same_as"]) if "same_as" in fx["input"] else fx
+    exp = GU.expected_bytes(fx)
+    h = fx["header"]
+    plan = None
+    if with_plan:
+        blob = b"ZNP1" + bytes([h["dtype"], h["n_groups"], 0, 0]) + exp[h["off_codes"]: h["off_payload"]].tobytes()
+        plan = z.Plan.from_bytes(blob)
+    x = make().cuda()
+    got = z.compress(x, chunk_bytes=src["input"]["chunk_bytes"], subblock=src["input"]["S"], plan=plan)
+    got = got.cpu().numpy()
+    assert got.size == exp.size and np.array_equal(got, exp), np.nonzero(got[: exp.size] != exp[: got.size])[0][:8]
+    y = z.decompress(torch.from_numpy(exp.copy()).cuda(), x.dtype, x.numel(), chunk_bytes=src["input"]["chunk_bytes"])
+    assert torch.equal(y.cpu().view(torch.uint8), x.cpu().view(torch.uint8))
+
+
 @pytest.mark.parametrize("n", [1, 7, 8, 15, 16, 17, 1023, 4095, 4096, 4097, 131071, 131072, 131073, 400000])
 def test_bf16_ragged_sizes(z, orc, n):
     x = (torch.randn(n, generator=torch.Generator().manual_seed(n)) * 0.02).to(torch.bfloat16)

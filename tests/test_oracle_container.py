@@ -135,3 +135,31 @@ def test_corruption_is_reported(orc):
         d = c.copy()
         d[off0 + 128 + 512 + int(rng.integers(0, 20000))] ^= 1 << int(rng.integers(0, 8))
         assert orc.decompress_status("bf16", d, 300000) in (orc.OK, orc.ECORRUPT)
+
+
+# Hand-derived containers of the other dtypes: FP8 (a HUFF exponent and a HUFF mantissa,
+# 3-bit and 1-bit RAW packing, a 4-bit RAW exponent, a ragged chunk), the same FP8 input
+# with a two-group plan (shared records of both entropy streams), a clean FP32 tensor
+# (ZERO low fraction planes) and FP4 (2-bit and 1-bit packing).
+GOLDEN_OTHER = [
+    ("fp8_two_chunks.json", "fp8_e4m3", GU.fp8_two_chunk_input, False),
+    ("fp8_shared_code.json", "fp8_e4m3", GU.fp8_two_chunk_input, True),
+    ("fp32_clean_two_chunks.json", "fp32", GU.fp32_clean_two_chunk_input, False),
+    ("fp4_two_chunks.json", "fp4_e2m1", GU.fp4_two_chunk_input, False),
+]
+
+
+@pytest.mark.parametrize("name,dtype,make,with_plan", GOLDEN_OTHER)
+def test_golden_other_dtypes(orc, name, dtype, make, with_plan):
+    fx = GU.load(name)
+    src = GU.load(fx["input"]["same_as"]) if "same_as" in fx["input"] else fx
+    x = make()
+    n = src["input"]["n"]
+    got = orc.compress(dtype, x, n, chunk_bytes=src["input"]["chunk_bytes"], S=src["input"]["S"],
+                       plan_lens=GU.plan_lens(fx) if with_plan else None)
+    exp = GU.expected_bytes(fx)
+    assert got.size == exp.size, (got.size, exp.size)
+    bad = np.nonzero(got != exp)[0]
+    assert bad.size == 0, f"first differing bytes at {bad[:8]}"
+    y = orc.decompress(dtype, got, n, chunk_bytes=src["input"]["chunk_bytes"])
+    assert np.array_equal(y, orc._bytes_view(x))
