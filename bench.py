@@ -1,11 +1,13 @@
 """Benchmark: ZipNN-style compress + decompress of a 7B-shaped BF16 checkpoint on B200.
 
 One step = zipnn_compress of each of the 225 tensors of the checkpoint (6,607,077,376
-BF16 values, 13.21 GB), issued round-robin on 4 CUDA streams (one workspace each), then
-zipnn_decompress of each.
+BF16 values, 13.21 GB), issued round-robin on 8 CUDA streams (one workspace each), then
+one zipnn_decompress_batch over all 225 containers.
 The metric is GB/s of uncompressed bytes; `value` is the round-trip rate (uncompressed
 bytes / (compress time + decompress time)) summed over all ranks, and the JSON line
-also carries each direction and its fraction of the measured HBM copy bandwidth.
+also carries each direction and its fraction of the HBM roofline (algorithmic bytes
+read + written / time), against the measured copy bandwidth and against the nominal
+8 TB/s.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 Under torchrun (N > 1) every rank compresses its own checkpoint (weak scaling, no
@@ -24,6 +26,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
+import numpy as np
 import torch
 
 METRIC = "decompress/compress GB/s (uncompressed) at 1 B200; % of HBM roofline"
@@ -33,6 +36,7 @@ WORKLOAD = ("BF16 7B-shaped checkpoint: 32 x [q,k,v,o 4096x4096; gate,up,down 40
 CHUNK = 262144
 SUBBLOCK = 512  # the library default (include/zipnn.h)
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0  # the B200 figure the metric names ("about 8 TB/s")
 
 
 # ------------------------------------------------------------------ distributed helpers
@@ -193,31 +197,107 @@ def make_workload(device, rank, tensors=None, only=None):
     return [W.checkpoint_7b_tensor(t + rank_seed(rank), shapes[t][1], sig[t], device).reshape(-1) for t in pick]
 
 
-def cpu_baseline(xs, budget_s=15.0):
-    """The oracle as it stands, on this host's cores, over a bounded sample of the
-    workload's tensors (chunk-parallel threads); same round-trip metric."""
-    import oracle
-    threads = os.cpu_count() or 1
-    done_bytes, t_c, t_d, used = 0, 0.0, 0.0, 0
-    for x in xs:
-        h = x.cpu().view(torch.uint8).numpy()
+def _oracle_leg(oracle, dtype, pieces, threads, budget_s, plan_lens=None):
+    """Time the oracle's compress and decompress over host pieces (uint8 numpy arrays, each
+    a whole number of chunks of its tensor) until budget_s seconds of work are done."""
+    done, t_c, t_d, used = 0, 0.0, 0.0, 0
+    for h in pieces:
+        n = oracle.values_in(dtype, h.size)
         t0 = time.perf_counter()
-        c = oracle.compress("bf16", h, x.numel(), CHUNK, SUBBLOCK, threads=threads)
+        c = oracle.compress(dtype, h, n, CHUNK, SUBBLOCK, plan_lens=plan_lens, threads=threads)
         t1 = time.perf_counter()
-        y = oracle.decompress("bf16", c, x.numel(), CHUNK, threads=threads)
+        y = oracle.decompress(dtype, c, n, CHUNK, threads=threads)
         t2 = time.perf_counter()
-        assert (y == h).all()
+        assert np.array_equal(y, h)
         t_c += t1 - t0
         t_d += t2 - t1
-        done_bytes += h.size
+        done += h.size
         used += 1
         if t_c + t_d > budget_s:
             break
+    return done, t_c, t_d, used
+
+
+def _slices(x, piece_bytes):
+    """Host pieces of a device tensor, each piece_bytes (whole chunks) or the rest."""
+    flat = x.reshape(-1).view(torch.uint8)
+    for lo in range(0, flat.numel(), piece_bytes):
+        yield flat[lo: lo + piece_bytes].cpu().numpy()
+
+
+def cpu_baseline(xs, dev, budget_all=5.0, budget_one=6.0):
+    """The oracle as it stands on this host's cores (a reported baseline, not the target),
+    on bounded samples of every workload: (i) one thread on the 2 MiB BF16 tensor, FP32,
+    FP8 and the first two layers of the checkpoint; (ii) all threads (chunk-parallel) on
+    all five workloads. Each leg stops after its time budget; `sample` says how much of
+    the workload it covered. `value` is the checkpoint leg on all threads."""
+    import oracle
+    from lossless_float_weight_b200 import workloads as W
+    threads = os.cpu_count() or 1
+    legs = []
+
+    def leg(config, dtype, pieces, nthreads, budget, total_bytes, plan_lens=None, note=""):
+        done, t_c, t_d, used = _oracle_leg(oracle, dtype, pieces, nthreads, budget, plan_lens)
+        legs.append({"config": config, "threads": nthreads, "bytes": done,
+                     "sample": f"{done / 1e9:.3f} of {total_bytes / 1e9:.3f} GB{note}",
+                     "compress_GBps": round(done / t_c / 1e9, 4), "decompress_GBps": round(done / t_d / 1e9, 4),
+                     "roundtrip_GBps": round(done / (t_c + t_d) / 1e9, 4)})
+        return legs[-1]
+
+    small = W.bf16_small().view(torch.uint8).numpy()
+    ckpt = lambda: (x.view(torch.uint8).cpu().numpy() for x in xs)  # noqa: E731
+    two_layers = lambda: (x.view(torch.uint8).cpu().numpy() for x in xs[:14])  # noqa: E731
+    ckpt_bytes = sum(x.numel() * 2 for x in xs)
+    piece = 64 << 20
+    fp32 = W.fp32_tensor(n=268435456, device=dev)
+    fp8 = W.fp8_tensor(rows=262144, cols=4096, device=dev)
+    # (i) one thread
+    leg("1: BF16 1,048,576 values", "bf16", [small], 1, budget_one, small.size)
+    leg("2: BF16 7B checkpoint, first 2 layers (subset)", "bf16", two_layers(), 1, budget_one,
+        sum(x.numel() * 2 for x in xs[:14]), note=" (layers 0-1 only)")
+    leg("3: FP32 268,435,456 values", "fp32", _slices(fp32, piece), 1, budget_one, fp32.numel() * 4)
+    leg("4: FP8 E4M3 262,144 x 4096", "fp8_e4m3", _slices(fp8, piece), 1, budget_one, fp8.numel())
+    # (ii) every thread
+    leg("1: BF16 1,048,576 values", "bf16", [small], threads, budget_all, small.size)
+    main = leg("2: BF16 7B checkpoint", "bf16", ckpt(), threads, 3 * budget_all, ckpt_bytes)
+    leg("3: FP32 268,435,456 values", "fp32", _slices(fp32, 4 * piece), threads, budget_all, fp32.numel() * 4)
+    clean = fp32.to(torch.bfloat16).to(torch.float32)
+    del fp32
+    leg("3: FP32 clean (rounded through BF16)", "fp32", _slices(clean, 4 * piece), threads, budget_all,
+        clean.numel() * 4)
+    del clean
+    leg("4: FP8 E4M3 262,144 x 4096", "fp8_e4m3", _slices(fp8, 4 * piece), threads, budget_all, fp8.numel())
+    del fp8
+    kv = W.kv_cache(device=dev)
+    kv_sample = kv[: (1 << 30) // 2].view(torch.uint8).cpu().numpy()  # the first 1 GiB: 4096 chunks
+    kv_total = kv.numel() * 2
+    del kv
+    lens, _, _, _ = oracle.plan_build("bf16", kv_sample, groups=8, seed=0)
+    leg("5: BF16 K/V cache, 8-group plan (built by the oracle on the sample, not timed)", "bf16",
+        (kv_sample[lo: lo + 4 * piece] for lo in range(0, kv_sample.size, 4 * piece)), threads, budget_all,
+        kv_total, plan_lens=lens)
     return {
-        "value": done_bytes / (t_c + t_d) / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
-        "compress_GBps": done_bytes / t_c / 1e9, "decompress_GBps": done_bytes / t_d / 1e9,
-        "sample": f"first {used} of 225 tensors ({done_bytes / 1e9:.3f} GB), compress+decompress, "
-                  f"{threads} threads (chunk-parallel)",
+        "value": main["roundtrip_GBps"], "unit": "GB/s", "cores": threads, "kind": "oracle",
+        "compress_GBps": main["compress_GBps"], "decompress_GBps": main["decompress_GBps"],
+        "sample": f"checkpoint leg: {main['sample']} (first tensors in order), compress+decompress, "
+                  f"{threads} threads (chunk-parallel); every leg below is a bounded sample",
+        "legs": legs,
+    }
+
+
+def bench_config(args, world, nbytes):
+    """The `config` of the JSON line: the workload and how a step runs (both arms)."""
+    return {
+        "workload": WORKLOAD.format(ns=args.streams),
+        "step": "compress all 225 tensors (one zipnn_compress each), then decompress all 225 ("
+                + ("one zipnn_decompress each" if args.per_tensor_decode else "one zipnn_decompress_batch")
+                + ") (value = uncompressed bytes per step / step time, x ranks)",
+        "global_batch": world * nbytes,
+        "parallelism": f"weak scaling, {world} independent checkpoint(s), no collective on the data path",
+        "l2": "inputs larger than L2 (13.2 GB per rank; no flush needed)",
+        "subblock": SUBBLOCK,
+        "streams": args.streams,
+        "chunk_bytes": CHUNK,
     }
 
 
@@ -334,7 +414,7 @@ def run_ours(args):
     e2e = run_e2e(Z, xs, csizes, dev, stream, streams, args, world) if not args.no_extras else None
 
     if rank == 0:
-        cpu = cpu_baseline(xs) if world == 1 and not args.no_extras else None
+        cpu = cpu_baseline(xs, dev) if world == 1 and not args.no_extras else None
         line = {
             "metric": METRIC,
             "value": round(world * nbytes / (ms_step / 1e3) / 1e9, 2),
@@ -348,23 +428,13 @@ def run_ours(args):
             "vs_baseline": None,
             "dtype": "u32",
             "data": "synthetic (seeded N(0, sigma_t^2) BF16 tensors of a 7B checkpoint's shapes; no trained weights)",
-            "config": {
-                "workload": WORKLOAD.format(ns=args.streams),
-                "step": "compress all 225 tensors (one zipnn_compress each), then decompress all 225 ("
-                        + ("one zipnn_decompress each" if args.per_tensor_decode else "one zipnn_decompress_batch")
-                        + ") (value = uncompressed bytes per "
-                        "step / step time, x ranks)",
-                "global_batch": world * nbytes,
-                "parallelism": f"weak scaling, {world} independent checkpoint(s), no collective on the data path",
-                "l2": "inputs larger than L2 (13.2 GB per rank; no flush needed)",
-                "subblock": SUBBLOCK,
-                "streams": args.streams,
-                "chunk_bytes": CHUNK,
-            },
+            "config": bench_config(args, world, nbytes),
             "compress": {"GBps": round(world * nbytes / (comp_ms / 1e3) / 1e9, 2), "ms": round(comp_ms, 4),
-                         "hbm_frac": round(algo_bytes / (comp_ms / 1e3) / 1e9 / peak, 4)},
+                         "hbm_frac": round(algo_bytes / (comp_ms / 1e3) / 1e9 / peak, 4),
+                         "hbm_frac_nominal_8TBps": round(algo_bytes / (comp_ms / 1e3) / 1e9 / NOMINAL_HBM_GBS, 4)},
             "decompress": {"GBps": round(world * nbytes / (dec_ms / 1e3) / 1e9, 2), "ms": round(dec_ms, 4),
-                           "hbm_frac": round(algo_bytes / (dec_ms / 1e3) / 1e9 / peak, 4)},
+                           "hbm_frac": round(algo_bytes / (dec_ms / 1e3) / 1e9 / peak, 4),
+                           "hbm_frac_nominal_8TBps": round(algo_bytes / (dec_ms / 1e3) / 1e9 / NOMINAL_HBM_GBS, 4)},
             "compression_ratio": round(cbytes / nbytes, 5),
             "roofline": {
                 "kernel": dom_name,
@@ -374,6 +444,7 @@ def run_ours(args):
                 "peak_source": peak_src,
                 "unit": "GB/s",
                 "frac": round(achieved / peak, 4),
+                "frac_nominal_8TBps": round(achieved / NOMINAL_HBM_GBS, 4),
                 "traffic": profile_traffic(dom_name, nbytes / 2 / len(xs)),
                 "traffic_note": "DRAM bytes per launch: the kernel's ncu bytes per value on the embedding tensor "
                                 "(profiles/) times the average values per launch; null if the kernel changed since",
@@ -450,7 +521,7 @@ def run_e2e(Z, xs, csizes, dev, stream, streams, args, world):
             e2.record(s)
             stream.wait_event(e2)
 
-    steps = max(1, min(args.steps, 3))
+    steps = max(1, args.steps)
     step()
     torch.cuda.synchronize()
     barrier(world, dev)
@@ -471,6 +542,9 @@ def run_e2e(Z, xs, csizes, dev, stream, streams, args, world):
 # ------------------------------------------------------------------ reference arm (the oracle)
 
 def run_reference(args):
+    """The oracle (the plain C definition of the method) on the host cores, on this arm's
+    config and metric; each step is a bounded sample of the workload: the seven tensors of
+    layer 0 of the checkpoint (386 MB), compressed and decompressed chunk-parallel."""
     rank, world, local = dist_env()
     if rank != 0:
         return
@@ -479,30 +553,32 @@ def run_reference(args):
     shapes = W.checkpoint_7b_shapes()
     sig = W.checkpoint_7b_sigmas(len(shapes))
     threads = os.cpu_count() or 1
-    # bounded sample: the first tensor of the checkpoint (4096 x 4096), generated on the CPU
-    x = W.checkpoint_7b_tensor(0, shapes[0][1], sig[0], "cpu").reshape(-1)
-    h = x.view(torch.uint8).numpy()
-    nb = h.size
+    layer = [W.checkpoint_7b_tensor(t, shapes[t][1], sig[t], "cpu").reshape(-1) for t in range(7)]
+    hs = [x.view(torch.uint8).numpy() for x in layer]
+    nb = sum(h.size for h in hs)
+    total = sum(math.prod(sh) * 2 for _, sh in shapes)
 
     def step():
-        c = oracle.compress("bf16", h, x.numel(), CHUNK, SUBBLOCK, threads=threads)
-        y = oracle.decompress("bf16", c, x.numel(), CHUNK, threads=threads)
-        return c, y
+        for x, h in zip(layer, hs):
+            c = oracle.compress("bf16", h, x.numel(), CHUNK, SUBBLOCK, threads=threads)
+            y = oracle.decompress("bf16", c, x.numel(), CHUNK, threads=threads)
+        return y, h
 
     for _ in range(args.warmup):
         step()
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        c, y = step()
+        y, h = step()
     dt = (time.perf_counter() - t0) / args.steps
-    assert (y == h).all()
+    assert np.array_equal(y, h)
     v = nb / dt / 1e9
-    sample = f"tensor 0 of 225 (4096x4096, {nb / 1e6:.1f} MB), compress+decompress per step, {threads} threads"
+    sample = (f"layer 0 of the checkpoint (7 tensors, {nb / 1e6:.1f} MB of {total / 1e9:.2f} GB, generated on the "
+              f"host) per step, compress+decompress, {threads} threads (chunk-parallel)")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "u32", "data": "synthetic",
-        "config": {"workload": WORKLOAD.format(ns=args.streams), "sample": sample},
+        "config": bench_config(args, world, total),
         "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
