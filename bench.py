@@ -10,8 +10,13 @@ read + written / time), against the measured copy bandwidth and against the nomi
 8 TB/s.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-Under torchrun (N > 1) every rank compresses its own checkpoint (weak scaling, no
-collective on the data path); time is the max over ranks.
+Under torchrun (N > 1) the checkpoint is N times as wide (every tensor has N times the
+rows) and rank r holds chunks [r * C_t, (r + 1) * C_t) of each tensor t, C_t being the
+chunks of the one-GPU tensor: weak scaling, every rank compresses the same amount. Each
+step ends the compress half with the one exchange the path has: the payload sizes of the
+rank's 225 shards (zipnn_shard_sizes), one all-gather of them (225 u64 per rank), and
+the relocation of the rank's chunk tables into the whole containers (zipnn_shard_tables).
+At N = 1 the same calls run without the all-gather. Time is the max over ranks.
 """
 import argparse
 import json
@@ -190,6 +195,8 @@ class ClockSampler:
 # ------------------------------------------------------------------ our arm
 
 def make_workload(device, rank, tensors=None, only=None):
+    """Rank r's slice of every tensor of the (N-times-wider) checkpoint: the one-GPU
+    tensor's shape, its values drawn from the tensor's seed shifted by rank_seed(r)."""
     from lossless_float_weight_b200 import workloads as W
     shapes = W.checkpoint_7b_shapes()
     sig = W.checkpoint_7b_sigmas(len(shapes))
@@ -293,7 +300,12 @@ def bench_config(args, world, nbytes):
                 + ("one zipnn_decompress each" if args.per_tensor_decode else "one zipnn_decompress_batch")
                 + ") (value = uncompressed bytes per step / step time, x ranks)",
         "global_batch": world * nbytes,
-        "parallelism": f"weak scaling, {world} independent checkpoint(s), no collective on the data path",
+        "parallelism": (f"weak scaling over {world} rank(s): each rank holds a contiguous chunk range of every tensor of "
+                        f"a checkpoint {world}x as wide; per step one all-gather of the 225 shard payload sizes "
+                        "(u64, the only exchange) and the relocation of the rank's chunk tables into the whole "
+                        "containers" if world > 1 else
+                        "one GPU; the shard-size and chunk-table steps run as they do on N GPUs, without the "
+                        "all-gather"),
         "l2": "inputs larger than L2 (13.2 GB per rank; no flush needed)",
         "subblock": SUBBLOCK,
         "streams": args.streams,
@@ -332,8 +344,25 @@ def run_ours(args):
             e2.record(s)
             stream.wait_event(e2)
 
+    # the shards of one container: rank r holds chunks [r * C_t, (r + 1) * C_t) of tensor t
+    from lossless_float_weight_b200 import shard as SH
+    n_slice = [x.numel() for x in xs]
+    n_totals = [world * n for n in n_slice]
+    chunk_los = [rank * -(-n // (CHUNK // 2)) for n in n_slice]
+    sizes_buf = torch.empty(len(xs), dtype=torch.int64, device=dev)
+    sh_ws = torch.empty(Z.zipnn_shard_workspace_bytes(len(xs)), dtype=torch.uint8, device=dev)
+    tables = [torch.empty(SH.table_bytes(Z.BF16, n), dtype=torch.uint8, device=dev) for n in n_slice]
+    headers = [torch.empty(64, dtype=torch.uint8, device=dev) if lo == 0 else None for lo in chunk_los]
+
+    def exchange_and_relocate(st):
+        SH.shard_sizes(outs, n_totals, chunk_los, stream=st, out=sizes_buf, ws=sh_ws)
+        all_sizes = SH.exchange_sizes(sizes_buf)  # NCCL all-gather of 225 u64 per rank (N > 1)
+        SH.shard_tables(Z.BF16, outs, n_totals, chunk_los, all_sizes, rank, world, CHUNK, stream=st,
+                        tables=tables, headers=headers, ws=sh_ws)
+
     def compress_all():
         fan_out(lambda i, s, w: Z.compress_into(xs[i], outs[i], w, CHUNK, stream=s))
+        exchange_and_relocate(stream)
 
     bws = Z.batch_workspace(len(xs), dev)
 
@@ -351,6 +380,10 @@ def run_ours(args):
     ok = all(torch.equal(d.view(torch.int16), x.view(torch.int16)) for d, x in zip(decs, xs))
     if not ok:
         raise RuntimeError("round trip mismatch")
+    if Z.status(sh_ws) != Z.OK:
+        raise RuntimeError("shard tables reported a mismatch")
+    if world == 1 and not all(torch.equal(t, o[64: 64 + t.numel()]) for t, o in zip(tables, outs)):
+        raise RuntimeError("one shard: the relocated tables must equal the containers' own")
     cbytes = sum(csizes)
 
     # timed region: K steps, events on the launching stream, kernel events on
@@ -389,6 +422,7 @@ def run_ours(args):
     for k in range(args.steps):
         for i in range(len(xs)):
             Z.compress_into(xs[i], outs[i], wss[0], CHUNK, stream=stream)
+        exchange_and_relocate(stream)
         if args.per_tensor_decode:
             for i in range(len(xs)):
                 Z.decompress_into(outs[i], outs[i].numel(), decs[i], wss[0], CHUNK, stream=stream)
@@ -403,7 +437,7 @@ def run_ours(args):
     gpu_launches = sum(v[1] for v in ktimes.values())  # the same count as the timed region
     # algorithmic bytes per step of each kernel (reads + writes the method needs)
     kbytes = {"decode_merge": cbytes + nbytes, "encode": nbytes + cbytes, "split_hist": nbytes,
-              "code_build": 0, "layout_scan": 0}
+              "code_build": 0, "layout_scan": 0, "shard_tables": 0}
     # dominant kernel: the one with the largest share of device time
     dom = max(ktimes.items(), key=lambda kv: kv[1][0])
     dom_name, (dom_ms, dom_n) = dom

@@ -212,6 +212,52 @@ zipnn_status zipnn_plan_assignment(const zipnn_plan_t* plan, uint32_t* host_buf,
 /* Release a plan and its device tables (NULL is ignored). */
 void zipnn_plan_destroy(zipnn_plan_t* plan);
 
+/* ---- One container from shards compressed on several GPUs ---------------------------
+ * "ZipNN: Lossless Compression for AI Models" (abstract): a model's chunks are coded
+ * independently, so a tensor splits across GPUs into contiguous ranges of whole chunks
+ * (only the last range may end in a partial chunk). Each GPU compresses its range with
+ * zipnn_compress as a tensor of its own (a shard container; the same dtype, chunk_bytes,
+ * sub-block length and plan on every GPU). The container of the whole tensor is
+ *   [header][chunk table][shared records][payloads of shard 0][payloads of shard 1]...
+ * where shard r's relocated entries (zipnn_shard_tables) go to byte
+ * 64 + 16 * n_streams * chunk_lo_r, the shared records are bytes off_codes..off_payload of
+ * any shard's container (put at the whole container's off_codes), and shard r's payload
+ * section (bytes off_payload..total_bytes of its container) starts at the whole
+ * container's off_payload plus the payload bytes of the shards before it. The result
+ * equals, byte for byte, the container that one call on the whole tensor writes. The only
+ * exchange between GPUs is one u64 per shard and rank: an all-gather of the output of
+ * zipnn_shard_sizes. The caller moves the bytes (a file write at each offset, or a copy). */
+typedef struct zipnn_shard_item {
+  const void* shard;    /* device, 16-byte aligned: the shard container */
+  uint64_t shard_bytes; /* readable bytes at shard */
+  uint64_t n_total;     /* values of the whole tensor */
+  uint64_t chunk_lo;    /* index in the whole tensor of the shard's first chunk */
+  void* table_out;      /* device, 16-byte aligned: 16 * n_streams * (shard's chunks) bytes */
+  void* header_out;     /* device, 16-byte aligned, 64 bytes, or NULL: the whole header */
+} zipnn_shard_item;
+
+/* Workspace bytes (device, 16-byte aligned) for zipnn_shard_sizes / zipnn_shard_tables of
+ * `count` items: a status word and a copy of the item table. */
+size_t zipnn_shard_workspace_bytes(uint32_t count);
+
+/* sizes_out[i] (device u64) = payload bytes (total_bytes - off_payload) of items[i].shard.
+ * `items` is a host array read before the call returns. Asynchronous; a shard that is
+ * not a container gets 0 and sets ZIPNN_ERR_CORRUPT in the workspace status. */
+zipnn_status zipnn_shard_sizes(uint32_t count, const zipnn_shard_item* items, uint64_t* sizes_out, void* ws,
+                               size_t ws_bytes, zipnn_stream_t stream);
+
+/* For each item i of this rank: writes its chunk-table entries, payload offsets moved to
+ * the whole container (the shard's payload base is the sum of all_sizes[r * count + i]
+ * over ranks r < rank), to table_out, and when header_out is not NULL the whole container's
+ * header (total_bytes = its off_payload plus the sum over all ranks). all_sizes: device,
+ * world * count u64, rank-major (the all-gather of every rank's zipnn_shard_sizes). A shard
+ * that is not the values [chunk_lo * m0, ...) of a tensor of n_total values with this dtype
+ * and chunk_bytes, or whose size differs from all_sizes, sets ZIPNN_ERR_CORRUPT (nothing is
+ * written for it). Asynchronous. */
+zipnn_status zipnn_shard_tables(zipnn_dtype dtype, uint32_t chunk_bytes, uint32_t count, const zipnn_shard_item* items,
+                                const uint64_t* all_sizes, uint32_t rank, uint32_t world, void* ws, size_t ws_bytes,
+                                zipnn_stream_t stream);
+
 /* Compress without allocating (the pages have no counterpart of this call). For callers
  * that cannot allocate device memory: code whose device memory is owned by a framework's
  * caching allocator that it cannot reach from C (a cudaMalloc of its own would fight

@@ -166,6 +166,16 @@ __device__ __forceinline__ void next_symbols(StreamState& st, uint32_t (&o)[GV],
 }
 
 
+// Two BF16 words (the merge) from two sign/fraction bytes, bytes 2*sf_hi and 2*sf_hi + 1
+// of sf, and two exponents, bytes 2*ex_hi and 2*ex_hi + 1 of ex. Each sign/fraction byte
+// is copied into both bytes of its 16-bit half; the mask keeps its fraction bits 6..0
+// and, from the copy one byte up, its sign at bit 15; the exponent, moved to bits 7..14
+// by a multiply by 128, adds in without carries (those bits are clear in the masked word).
+__device__ __forceinline__ uint32_t bf16_merge_pair(uint32_t sf, int sf_hi, uint32_t ex, int ex_hi) {
+  const uint32_t y = __byte_perm(sf, 0, sf_hi ? 0x3322 : 0x1100) & 0x807F807Fu;
+  return __byte_perm(ex, 0, ex_hi ? 0x4342 : 0x4140) * 128u + y;
+}
+
 // BF16 with a HUFF exponent stream and a RAW (or ZERO) sign/fraction stream: the case
 // of every chunk of a trained or Gaussian checkpoint. 16 values per step; the
 // sign/fraction bytes of the next step are requested one step ahead.
@@ -202,10 +212,7 @@ __device__ __forceinline__ int decode_bf16_fast(const uint32_t* lut, const uint8
     }
     uint32_t o[8];
 #pragma unroll
-    for (int q = 0; q < 8; q++) {
-      const uint32_t t = SM_ZERO ? 0u : __byte_perm(x[q >> 1], 0, (q & 1) ? 0x4342 : 0x4140);
-      o[q] = (t & 0x007F007Fu) | ((t & 0x00800080u) << 8) | (__byte_perm(pr[q], 0, 0x4342) << 7);
-    }
+    for (int q = 0; q < 8; q++) o[q] = bf16_merge_pair(SM_ZERO ? 0u : x[q >> 1], q & 1, pr[q], 1);
     uint4* d = reinterpret_cast<uint4*>(dst + (uint64_t)gi * 32);
     d[0] = make_uint4(o[0], o[1], o[2], o[3]);
     d[1] = make_uint4(o[4], o[5], o[6], o[7]);
@@ -258,8 +265,11 @@ struct SmemBitReader {
   uint64_t buf;
   int nb;
   uint32_t q;
+  // Word i of the bitstream. Past the end a reader sees the word at `end` (stale data or
+  // the next buffer, always inside the block's shared memory): a valid sub-block never
+  // consumes those bits, and one that does ends past its bound and is reported.
   __device__ __forceinline__ uint32_t ld(uint32_t i) const {
-    if (i >= end) return 0u;
+    i = min(i, end);
     if constexpr (WIDE) return bswap32(i < kWindowWords ? w[i] : w2[i - kWindowWords]);
     return bswap32(w[i]);
   }
@@ -318,7 +328,7 @@ template <bool WIDE, class Lut>
 __device__ int decode_bf16_staged(StagedSmem& st, const Lut* lut, const uint32_t* tail,
                                   const uint32_t* __restrict__ idx, uint32_t bs_words,
                                   const uint8_t* __restrict__ smp, uint32_t m, uint32_t S, uint32_t nsub,
-                                  uint8_t* __restrict__ outc) {
+                                  uint8_t* __restrict__ outc, uint32_t pre_start, uint32_t pre_next) {
   const int tid = threadIdx.x;
   int bad = 0;
   const uint64_t cap_bits = (uint64_t)bs_words * 32;
@@ -332,9 +342,10 @@ __device__ int decode_bf16_staged(StagedSmem& st, const Lut* lut, const uint32_t
     uint64_t expect = 0;
     bool exact = false;
     if (count) {
-      const uint64_t start = __ldg(idx + j);
+      // the first batch's bounds were loaded by the caller while it built the tables
+      const uint64_t start = batch == 0 ? pre_start : __ldg(idx + j);
       exact = j + 1 < nsub;
-      expect = exact ? __ldg(idx + j + 1) : cap_bits;
+      expect = exact ? (batch == 0 ? pre_next : __ldg(idx + j + 1)) : cap_bits;
       if ((j == 0 && start != 0) || start > cap_bits || expect < start || expect > cap_bits) bad = 1;
       br.init(st.bits, bs_words, bad ? 0 : start, tail);
     }
@@ -412,11 +423,7 @@ __device__ int decode_bf16_staged(StagedSmem& st, const Lut* lut, const uint32_t
         const uint32_t xs[2] = {smv[p].x, smv[p].y};
         uint32_t o[4];
 #pragma unroll
-        for (int q = 0; q < 4; q++) {
-          const uint32_t t = __byte_perm(xs[q >> 1], 0, (q & 1) ? 0x4342 : 0x4140);
-          const uint32_t ee = __byte_perm(es[q >> 1], 0, (q & 1) ? 0x4342 : 0x4140);
-          o[q] = (t & 0x007F007Fu) | ((t & 0x00800080u) << 8) | (ee << 7);
-        }
+        for (int q = 0; q < 4; q++) o[q] = bf16_merge_pair(xs[q >> 1], q & 1, es[q >> 1], q & 1);
         uint8_t* d = outc + (uint64_t)uval[p] * 2;
         if (ucnt[p] == 8) {
           *reinterpret_cast<uint4*>(d) = make_uint4(o[0], o[1], o[2], o[3]);
@@ -439,9 +446,12 @@ __device__ int decode_bf16_staged(StagedSmem& st, const Lut* lut, const uint32_t
 template <int DT>
 struct DecodeSmem {
   uint32_t lut[n_entropy(DT)][4096];
-  uint8_t lens[n_entropy(DT)][256];
-  uint32_t enc[n_entropy(DT)][256];
-  uint8_t sorted[n_entropy(DT)][256];
+  uint8_t sorted[n_entropy(DT)][256];     // symbols in canonical order: by length, then symbol
+  uint8_t slen[n_entropy(DT)][256];       // length of sorted[k]
+  uint16_t base[n_entropy(DT)][8][16];    // canonical index of warp w's first symbol of length l
+  uint8_t cnt[n_entropy(DT)][8][16];      // symbols of length l among the 32 of warp w
+  uint32_t kraft[n_entropy(DT)][8];       // per warp: sum of 2^(12 - len)
+  uint32_t flags[n_entropy(DT)][8];       // per warp: 1 a length above 12, 2 a symbol present
   uint32_t limit[n_entropy(DT)][kLmax + 1];
   uint32_t first[n_entropy(DT)][kLmax + 1];
   uint32_t offset[n_entropy(DT)][kLmax + 1];
@@ -454,6 +464,42 @@ struct DecodeSmem {
 
 // three BF16 decode blocks share an SM: 228 KB of shared memory, 1 KB reserved per block
 static_assert(sizeof(StagedSmem) + sizeof(DecodeSmem<kBF16>) + 1024 <= 233472 / 3, "BF16 decode: 3 blocks per SM");
+
+// Fill the decode table of one HUFF stream from its canonical tables, 16 consecutive
+// entries per thread. Canonical codes left-aligned to 12 bits tile [0, limit[12]) in
+// canonical order: code k covers 2^(12 - len_k) entries and the next code starts where
+// it ends. A thread finds the code of its first entry from the length limits, then
+// walks on. Entries from limit[12] on match no code (only when the Kraft sum is below 1).
+// WIDE: u16 entries symbol << 4 | length (the single-symbol table); else u32 entries
+// symbol << 16 | length.
+template <bool WIDE>
+__device__ __forceinline__ void fill_lut(void* lut, const uint8_t* sorted, const uint8_t* slen,
+                                         const uint32_t* limit, const uint32_t* first, const uint32_t* offset) {
+  const uint32_t x0 = threadIdx.x * 16u, lim = limit[kLmax];
+  uint32_t l = 1;
+  while (l < (uint32_t)kLmax && x0 >= limit[l]) l++;
+  uint32_t k = 0, end = 0, e = 0;
+  if (x0 < lim) {
+    const uint32_t c = x0 >> (kLmax - l);
+    k = offset[l] + c - first[l];
+    end = (c + 1) << (kLmax - l);
+    e = WIDE ? ((uint32_t)sorted[k] << 4) | l : ((uint32_t)sorted[k] << 16) | l;
+  }
+#pragma unroll
+  for (uint32_t i = 0; i < 16; i++) {
+    const uint32_t x = x0 + i;
+    if (x < lim && x == end) {
+      k++;
+      const uint32_t lk = slen[k];
+      end += 1u << (kLmax - lk);
+      e = WIDE ? ((uint32_t)sorted[k] << 4) | lk : ((uint32_t)sorted[k] << 16) | lk;
+    }
+    if constexpr (WIDE) static_cast<uint16_t*>(lut)[x] = (uint16_t)(x < lim ? e : (kLutInvalid | 1u));
+    else static_cast<uint32_t*>(lut)[x] = x < lim ? e : (kLutInvalid | 1u);
+  }
+}
+
+static_assert(kDecodeThreads * 16 == 4096, "fill_lut: 16 table entries per thread");
 
 // Chunk c of the container `in` (in_bytes readable) of a tensor with geometry g, into
 // `out` (the tensor's first value). All threads of the block.
@@ -470,21 +516,33 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
 
   if (tid == 0) {
     int bad = 0;
-    const uint32_t* h = reinterpret_cast<const uint32_t*>(in);
     uint64_t total = 0, off_codes = 0, off_payload = 0;
     uint32_t S = 0, G = 0;
-    if (in_bytes < kHeaderBytes) {
+    const uint64_t entries = (uint64_t)g.n_chunks * NS;
+    const uint64_t k0 = (uint64_t)c * NS;
+    if (in_bytes < kHeaderBytes + kEntryBytes * (k0 + NS)) {
       bad = 1;
     } else {
-      uint32_t hv[16];
-      for (int i = 0; i < 16; i++) hv[i] = h[i];
+      // the header and this chunk's entries (and the next one's offset) in one round trip;
+      // every address is inside in_bytes
+      uint4 hq[4], ent[NS + 1];
+#pragma unroll
+      for (int i = 0; i < 4; i++) hq[i] = reinterpret_cast<const uint4*>(in)[i];
+#pragma unroll
+      for (int s = 0; s <= NS; s++) {
+        const uint64_t k = k0 + s;
+        ent[s] = (s < NS || (k < entries && kHeaderBytes + kEntryBytes * (k + 1) <= in_bytes))
+                     ? *reinterpret_cast<const uint4*>(in + kHeaderBytes + kEntryBytes * k)
+                     : make_uint4(0, 0, 0, 0);
+      }
+      const uint32_t hv[16] = {hq[0].x, hq[0].y, hq[0].z, hq[0].w, hq[1].x, hq[1].y, hq[1].z, hq[1].w,
+                               hq[2].x, hq[2].y, hq[2].z, hq[2].w, hq[3].x, hq[3].y, hq[3].z, hq[3].w};
       const uint64_t n = hv[2] | ((uint64_t)hv[3] << 32);
       S = hv[5];
       G = (hv[14] >> 8) & 0xFF;
       off_codes = hv[8] | ((uint64_t)hv[9] << 32);
       off_payload = hv[10] | ((uint64_t)hv[11] << 32);
       total = hv[12] | ((uint64_t)hv[13] << 32);
-      const uint64_t entries = (uint64_t)g.n_chunks * NS;
       if (hv[0] != 0x314E4E5Au || hv[1] != (1u | ((uint32_t)DT << 16) | ((uint32_t)NS << 24))) bad = 1;
       if (n != g.n || hv[4] != g.chunk_bytes || hv[6] != g.n_chunks) bad = 1;
       if (S == 0 || (S & 15) || S > 65536) bad = 1;
@@ -493,38 +551,31 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
       if (off_codes != kHeaderBytes + entries * kEntryBytes) bad = 1;
       if (!bad && off_payload != off_codes + shared_bytes(DT, G)) bad = 1;
       if (total > in_bytes || total < off_payload || (total & 15)) bad = 1;
-    }
-    if (!bad) {
-      const uint64_t entries = (uint64_t)g.n_chunks * NS;
-      for (int s = 0; s < NS && !bad; s++) {
-        const uint64_t k = (uint64_t)c * NS + s;
-        const uint4 ent = *reinterpret_cast<const uint4*>(in + kHeaderBytes + kEntryBytes * k);
-        const uint64_t off = ent.z | ((uint64_t)ent.w << 32);
-        uint64_t end = total;
-        if (k + 1 < entries) {
-          const uint4 nx = *reinterpret_cast<const uint4*>(in + kHeaderBytes + kEntryBytes * (k + 1));
-          end = nx.z | ((uint64_t)nx.w << 32);
-        }
-        const uint32_t mode = ent.x & 0xFF;
-        if ((ent.x >> 8) != 0 || mode > kModeHuff) bad = 1;
+#pragma unroll
+      for (int s = 0; s < NS; s++) {
+        const uint64_t k = k0 + s;
+        const uint64_t off = ent[s].z | ((uint64_t)ent[s].w << 32);
+        const uint64_t end = k + 1 < entries ? (ent[s + 1].z | ((uint64_t)ent[s + 1].w << 32)) : total;
+        const uint32_t mode = ent[s].x & 0xFF;
+        if ((ent[s].x >> 8) != 0 || mode > kModeHuff) bad = 1;
         if ((off & 15) || (end & 15) || off > end || end > total || off < off_payload) bad = 1;
         if (k == 0 && off != off_payload) bad = 1;
         const uint64_t extent = end - off;
         const int w = raw_width(DT, s);
         if (mode == kModeRaw) {
-          if (ent.y != kNoCode || extent * 8 < (uint64_t)m * w) bad = 1;
+          if (ent[s].y != kNoCode || extent * 8 < (uint64_t)m * w) bad = 1;
         } else if (mode == kModeZero) {
-          if (ent.y != kNoCode) bad = 1;
-        } else if (mode == kModeHuff) {
+          if (ent[s].y != kNoCode) bad = 1;
+        } else if (mode == kModeHuff && S != 0) {
           const uint64_t nsub = ceil_div(m, S);
           uint64_t need = round16(4 * nsub);
           if (!is_entropy(DT, s)) bad = 1;
-          else if (ent.y == kNoCode) need += record_bytes(DT, s);
-          else if (G == 0 || ent.y >= G * NE || ent.y / G != (uint32_t)s) bad = 1;
+          else if (ent[s].y == kNoCode) need += record_bytes(DT, s);
+          else if (G == 0 || ent[s].y >= G * NE || ent[s].y / G != (uint32_t)s) bad = 1;
           if (extent < need) bad = 1;
         }
         sm.mode[s] = mode;
-        sm.code[s] = ent.y;
+        sm.code[s] = ent[s].y;
         sm.off[s] = off;
         sm.end[s] = end;
       }
@@ -563,68 +614,101 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
     return;
   }
   const uint32_t S = sm.S;
+  const uint64_t nsub = ceil_div(m, S);
+  const int warp = tid >> 5, lane = tid & 31;
 
-  // code lengths of the HUFF streams
+  // BF16 staged path: this thread's first sub-block bounds, requested now so that the
+  // loads return while the tables are built
+  uint32_t idx_start = 0, idx_next = 0;
+  if constexpr (DT == kBF16) {
+    if (sm.staged && (uint64_t)tid < nsub) {
+      const uint32_t rec = sm.code[0] == kNoCode ? record_bytes(DT, 0) : 0;
+      const uint32_t* idx = reinterpret_cast<const uint32_t*>(in + sm.off[0] + rec);
+      idx_start = __ldg(idx + tid);
+      if ((uint64_t)tid + 1 < nsub) idx_next = __ldg(idx + tid + 1);
+    }
+  }
+
+  // Canonical tables of each HUFF stream, from its 4-bit code lengths. Thread t takes
+  // symbol t: each warp counts its 32 symbols of every length (ballots) and each symbol's
+  // rank among the warp's symbols of its length (match), with the Kraft sum, a length
+  // above 12, and whether any symbol is present.
+  uint32_t my_len[NE], my_rank[NE];
 #pragma unroll
   for (int e = 0; e < NE; e++) {
-    if (sm.mode[e] != kModeHuff) continue;
-    const uint8_t* rp = sm.code[e] == kNoCode
-                            ? in + sm.off[e]
-                            : in + sm.off_codes + shared_record_pos(DT, sm.G, sm.code[e]);
-    const int A = alphabet(DT, e);
-    for (int s = tid; s < 256; s += kDecodeThreads) {
-      uint32_t l = 0;
-      if (s < A) {
-        const uint32_t b = rp[s >> 1];
-        l = (s & 1) ? (b >> 4) : (b & 15u);
-      }
-      sm.lens[e][s] = (uint8_t)l;
+    my_len[e] = 0;
+    my_rank[e] = 0;
+    if (sm.mode[e] != kModeHuff) continue;  // uniform
+    const uint8_t* rp = sm.code[e] == kNoCode ? in + sm.off[e]
+                                              : in + sm.off_codes + shared_record_pos(DT, sm.G, sm.code[e]);
+    uint32_t l = 0;
+    if (tid < alphabet(DT, e)) {
+      const uint32_t b = rp[tid >> 1];
+      l = (tid & 1) ? (b >> 4) : (b & 15u);
+    }
+    const uint32_t same = __match_any_sync(0xFFFFFFFFu, l);
+    my_len[e] = l;
+    my_rank[e] = __popc(same & lanemask_lt());
+    uint32_t c = 0;
+#pragma unroll
+    for (int q = 1; q <= kLmax; q++) {
+      const uint32_t b = __popc(__ballot_sync(0xFFFFFFFFu, l == (uint32_t)q));
+      if (lane == q) c = b;
+    }
+    if (lane < 16) sm.cnt[e][warp][lane] = (uint8_t)c;
+    const uint32_t kw = __reduce_add_sync(0xFFFFFFFFu, (l && l <= (uint32_t)kLmax) ? 1u << (kLmax - l) : 0u);
+    const uint32_t fl = (__any_sync(0xFFFFFFFFu, l > (uint32_t)kLmax) ? 1u : 0u) | (__any_sync(0xFFFFFFFFu, l != 0) ? 2u : 0u);
+    if (lane == 0) {
+      sm.kraft[e][warp] = kw;
+      sm.flags[e][warp] = fl;
     }
   }
   __syncthreads();
-  // check each code (lengths <= 12, at least one symbol, Kraft sum <= 1), build the
-  // canonical values and the decode tables
-  const int warp = tid >> 5, lane = tid & 31;
+  // warp e: lengths' counts, first codes (RFC 1951, 3.2.2: first[l] = (first[l-1] +
+  // count[l-1]) << 1, i.e. the sum over q < l of count[q] << (l - q)), canonical index
+  // offsets, left-aligned limits, and every warp's base index for each length; lane l
+  // takes length l. A length above 12, no symbol, or a Kraft sum above 1 is corrupt.
   if (warp < NE && sm.mode[warp] == kModeHuff) {
     const int e = warp;
-    uint32_t kraft = 0, present = 0, toolong = 0;
-    for (int s = lane; s < 256; s += 32) {
-      const uint32_t l = sm.lens[e][s];
-      if (l > kLmax) toolong = 1;
-      else if (l) {
-        present++;
-        kraft += 1u << (kLmax - l);
+    uint32_t kraft = 0, fl = 0;
+#pragma unroll
+    for (int w = 0; w < 8; w++) {
+      kraft += sm.kraft[e][w];
+      fl |= sm.flags[e][w];
+    }
+    const bool in_range = lane >= 1 && lane <= kLmax;
+    uint32_t count = 0;
+    if (in_range)
+#pragma unroll
+      for (int w = 0; w < 8; w++) count += sm.cnt[e][w][lane];
+    uint32_t incl = count;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const uint32_t offs = incl - count;
+    uint32_t fst = 0;
+#pragma unroll
+    for (int q = 1; q < kLmax; q++) {
+      const uint32_t cq = __shfl_sync(0xFFFFFFFFu, count, q);
+      if (q < lane) fst += cq << (lane - q);
+    }
+    if (lane <= kLmax) {
+      sm.first[e][lane] = fst;
+      sm.offset[e][lane] = offs;
+      sm.limit[e][lane] = in_range ? (fst + count) << (kLmax - lane) : 0u;
+    }
+    if (in_range) {
+      uint32_t run = offs;
+#pragma unroll
+      for (int w = 0; w < 8; w++) {
+        sm.base[e][w][lane] = (uint16_t)run;
+        run += sm.cnt[e][w][lane];
       }
     }
-    for (int o = 16; o; o >>= 1) {
-      kraft += __shfl_xor_sync(0xFFFFFFFFu, kraft, o);
-      present += __shfl_xor_sync(0xFFFFFFFFu, present, o);
-      toolong |= __shfl_xor_sync(0xFFFFFFFFu, toolong, o);
-    }
-    if (toolong || !present || kraft > (1u << kLmax)) {
+    if ((fl & 1u) || !(fl & 2u) || kraft > (1u << kLmax)) {
       if (lane == 0) sm.bad = 1;
-    } else {
-      warp_canonical(sm.lens[e], sm.enc[e]);
-      // number of codes of each length, by ballots over the 256 symbols
-      uint32_t L[8];
-#pragma unroll
-      for (int i = 0; i < 8; i++) L[i] = sm.lens[e][i * 32 + lane];
-      uint32_t code = 0, offs = 0, prev = 0;
-      if (lane == 0) sm.limit[e][0] = 0;
-#pragma unroll
-      for (int l = 1; l <= kLmax; l++) {
-        uint32_t cnt = 0;
-#pragma unroll
-        for (int i = 0; i < 8; i++) cnt += __popc(__ballot_sync(0xFFFFFFFFu, L[i] == (uint32_t)l));
-        code = (code + prev) << 1;
-        if (lane == 0) {
-          sm.first[e][l] = code;
-          sm.offset[e][l] = offs;
-          sm.limit[e][l] = (code + cnt) << (kLmax - l);
-        }
-        offs += cnt;
-        prev = cnt;
-      }
     }
   }
   __syncthreads();
@@ -640,14 +724,13 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
     }
     return;
   }
+  // symbols in canonical order
 #pragma unroll
   for (int e = 0; e < NE; e++) {
-    if (sm.mode[e] != kModeHuff) continue;
-    for (int s = tid; s < 256; s += kDecodeThreads) {
-      const uint32_t v = sm.enc[e][s];
-      const uint32_t l = v >> 16;
-      if (l) sm.sorted[e][sm.offset[e][l] + (v & 0xFFFFu) - sm.first[e][l]] = (uint8_t)s;
-    }
+    if (sm.mode[e] != kModeHuff || !my_len[e]) continue;
+    const uint32_t k = sm.base[e][warp][my_len[e]] + my_rank[e];
+    sm.sorted[e][k] = (uint8_t)tid;
+    sm.slen[e][k] = (uint8_t)my_len[e];
   }
   __syncthreads();
   // BF16 with the wide window: the single-symbol table in the table's second half (the
@@ -657,17 +740,8 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
 #pragma unroll
   for (int e = 0; e < NE; e++) {
     if (sm.mode[e] != kModeHuff) continue;
-    for (uint32_t x = tid; x < 4096; x += kDecodeThreads) {
-      uint32_t sym = 0, l = 1;
-      const bool valid = x < sm.limit[e][kLmax];
-      if (valid) {
-#pragma unroll
-        for (int j = 1; j < kLmax; j++) l += x >= sm.limit[e][j];
-        sym = sm.sorted[e][sm.offset[e][l] + (x >> (kLmax - l)) - sm.first[e][l]];
-      }
-      if (wide) lut16[x] = (uint16_t)(valid ? (sym << 4) | l : kLutInvalid | 1u);
-      else sm.lut[e][x] = valid ? (sym << 16) | l : kLutInvalid | 1u;
-    }
+    if (wide) fill_lut<true>(lut16, sm.sorted[e], sm.slen[e], sm.limit[e], sm.first[e], sm.offset[e]);
+    else fill_lut<false>(sm.lut[e], sm.sorted[e], sm.slen[e], sm.limit[e], sm.first[e], sm.offset[e]);
   }
   __syncthreads();
   if constexpr (DT == kBF16) {
@@ -689,7 +763,6 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
     }
   }
 
-  const uint64_t nsub = ceil_div(m, S);
   if constexpr (DT == kBF16) {
     if (sm.staged) {
       StagedSmem& stg = *reinterpret_cast<StagedSmem*>(dyn_smem);
@@ -708,9 +781,9 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
       const uint32_t bs_words = (uint32_t)((sm.end[0] - bs_off) / 4);
       const uint8_t* smp = sm.mode[1] == kModeRaw ? in + sm.off[1] : nullptr;
       const int bad = wide ? decode_bf16_staged<true>(stg, lut16, sm.lut[0], idx, bs_words, smp, m, S,
-                                                      (uint32_t)nsub, out + clo * VB)
+                                                      (uint32_t)nsub, out + clo * VB, idx_start, idx_next)
                            : decode_bf16_staged<false>(stg, sm.lut[0], nullptr, idx, bs_words, smp, m, S,
-                                                       (uint32_t)nsub, out + clo * VB);
+                                                       (uint32_t)nsub, out + clo * VB, idx_start, idx_next);
       if (bad) set_status(status, kStCorrupt);
       return;
     }

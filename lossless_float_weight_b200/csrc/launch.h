@@ -10,7 +10,7 @@ namespace zipnn {
 bool device_ok();
 
 // Kernel ids of the optional event timing (timing.cu).
-enum KernelId { kIdHist = 0, kIdBuild, kIdLayout, kIdEncode, kIdDecode, kIdCodeLengths, kIdPlan, kNumKernelIds };
+enum KernelId { kIdHist = 0, kIdBuild, kIdLayout, kIdEncode, kIdDecode, kIdCodeLengths, kIdPlan, kIdShard, kNumKernelIds };
 
 // Brackets one launch with CUDA events on `st` while timing is enabled.
 class TimedLaunch {

@@ -11,7 +11,7 @@ namespace zipnn {
 namespace {
 
 const char* const kNames[kNumKernelIds] = {"split_hist", "code_build", "layout_scan", "encode",
-                                           "decode_merge", "code_lengths", "plan"};
+                                           "decode_merge", "code_lengths", "plan", "shard_tables"};
 
 struct Pending {
   int id;

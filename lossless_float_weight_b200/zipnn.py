@@ -69,13 +69,25 @@ zipnn_decompress_batch_workspace_bytes = _sig("zipnn_decompress_batch_workspace_
 zipnn_decompress_batch = _sig("zipnn_decompress_batch", _i, _i, _u32, _u32, ctypes.POINTER(DecompressItem), _vp,
                               _sz, _vp)
 
+class ShardItem(ctypes.Structure):
+    """zipnn_shard_item: one shard container and where its relocated pieces go."""
+    _fields_ = [("shard", _vp), ("shard_bytes", _u64), ("n_total", _u64), ("chunk_lo", _u64),
+                ("table_out", _vp), ("header_out", _vp)]
+
+
+zipnn_shard_workspace_bytes = _sig("zipnn_shard_workspace_bytes", _sz, _u32)
+zipnn_shard_sizes = _sig("zipnn_shard_sizes", _i, _u32, ctypes.POINTER(ShardItem), _vp, _vp, _sz, _vp)
+zipnn_shard_tables = _sig("zipnn_shard_tables", _i, _i, _u32, _u32, ctypes.POINTER(ShardItem), _vp, _u32, _u32, _vp,
+                          _sz, _vp)
+
 C_ABI_NAMES = [
     "zipnn_max_compressed_bytes", "zipnn_workspace_bytes", "zipnn_compress", "zipnn_compress_ex",
     "zipnn_decompress", "zipnn_compressed_size", "zipnn_get_status", "zipnn_histogram", "zipnn_code_lengths",
     "zipnn_plan_create", "zipnn_plan_export", "zipnn_plan_import", "zipnn_plan_assignment", "zipnn_plan_destroy",
     "zipnn_status_string", "zipnn_timing_enable", "zipnn_timing_collect", "zipnn_kernel_count",
     "zipnn_kernel_name", "zipnn_compress_noalloc", "zipnn_decompress_batch_workspace_bytes",
-    "zipnn_decompress_batch", "zipnn_test_lookback_limit",
+    "zipnn_decompress_batch", "zipnn_test_lookback_limit", "zipnn_shard_workspace_bytes", "zipnn_shard_sizes",
+    "zipnn_shard_tables",
 ]
 
 
