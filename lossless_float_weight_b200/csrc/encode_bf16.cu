@@ -36,12 +36,13 @@ constexpr int kBPasses = kBf16TileValues / kBPassValues;        // 4
 constexpr int kBStageWords = kBPassValues * kLmax / 32 + 2;     // one pass's bitstream
 constexpr int kBPrivStride = kBValues * kLmax / 32 + 1;         // odd: conflict-free
 static_assert(kBPasses * kBPassValues == kBf16TileValues, "a tile is a whole number of passes");
+static_assert(kBThreads == 128, "the pass scan adds four warp totals");
 
 struct Bf16EncodeSmem {
   uint32_t priv[kBThreads * kBPrivStride];  // each thread's codes, packed from bit 0
   uint32_t stage[kBStageWords];                  // the tile's bitstream at its final alignment
   uint32_t enc[256];                             // the chunk's code: len << 16 | code
-  uint32_t warp[kBThreads / 32];
+  alignas(16) uint32_t warp[2][kBThreads / 32];  // warp bit totals, by pass parity
   uint32_t carry[2];  // the bits of the word shared with the next pass, by pass parity
 };
 
@@ -182,8 +183,25 @@ __global__ void __launch_bounds__(kBThreads, 8) k_encode_bf16(const uint8_t* __r
         }
       }
       if (nfill) pw[nw++] = (uint32_t)(acc << (32 - nfill));
-      uint32_t pass_bits;
-      const uint32_t myoff = block_exclusive_scan<kBThreads>(mybits, sm.warp, pass_bits);
+      // my bit offset in the pass: a warp scan, then the four warp totals, which every
+      // thread adds itself after one barrier. The totals alternate between two slots by
+      // pass parity: a slot is written again two passes later, after the barrier of the
+      // pass between, when every thread has read it.
+      uint32_t pass_bits, myoff;
+      {
+        const int lane = tid & 31, warp = tid >> 5;
+        uint32_t x = mybits;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+          if (lane >= o) x += y;
+        }
+        if (lane == 31) sm.warp[pass & 1][warp] = x;
+        __syncthreads();
+        const uint4 t = *reinterpret_cast<const uint4*>(sm.warp[pass & 1]);
+        pass_bits = t.x + t.y + t.z + t.w;
+        myoff = x - mybits + (warp > 0 ? t.x : 0u) + (warp > 1 ? t.y : 0u) + (warp > 2 ? t.z : 0u);
+      }
       if (cnt > 0) {
         uint32_t rr = v0 % g.S;
 #pragma unroll

@@ -43,6 +43,8 @@
 #define MODE_RAW 0
 #define MODE_ZERO 1
 #define MODE_HUFF 2
+#define MODE_ZRUN 3
+#define ZRUN_BLOCK 32 /* symbols of one zero-run block */
 #define NO_CODE 0xFFFFFFFFu
 
 /* ------------------------------------------------------------------ field map */
@@ -271,7 +273,16 @@ static uint64_t get_u64(const uint8_t* p) {
  *  - payloads in entry order, each offset the sum of the sizes before it: RAW, the
  *    stream's symbols at their fixed width, MSB first; ZERO, nothing; HUFF, the
  *    chunk's own record (when code is 0xFFFFFFFF), then the bit offset (u32) of every
- *    S-th symbol padded to 16 bytes, then the codes MSB first padded to 16 bytes.
+ *    S-th symbol padded to 16 bytes, then the codes MSB first padded to 16 bytes;
+ *    ZRUN (mode 3, zero runs of a byte plane), the chunk's symbols taken in blocks of 32
+ *    (the last block may be shorter): one bit per block, MSB first, 1 when the block
+ *    holds a non-zero symbol, padded to 16 bytes, then the symbols of the marked blocks
+ *    in order, padded to 16 bytes.
+ *  - choice for a stream: ZERO when every symbol is 0. An entropy stream is HUFF when
+ *    that payload is strictly smaller than RAW, else RAW. A byte plane (8-bit symbols
+ *    that are not entropy-coded: BF16's sign/fraction byte, FP32's three fraction
+ *    planes) is ZRUN when that payload is strictly smaller than RAW, else RAW. The 1-bit
+ *    sign streams of FP8 and FP4 are RAW.
  */
 
 static uint64_t ceil_div(uint64_t a, uint64_t b) { return (a + b - 1) / b; }
@@ -410,6 +421,41 @@ static int encode_entry(const job_t* jb, uint64_t lo, uint64_t m, int s, entry_t
       for (uint64_t i = 0; i < m; i++) {
         if (i % jb->S == 0) put_u32(p + 4 * (i / jb->S), (uint32_t)t);
         put_bits(bs, &t, code[sym[i]], len[sym[i]]);
+      }
+      free(sym);
+      return ORC_OK;
+    }
+  }
+  if (!is_entropy(dt, s) && w == 8) {
+    /* zero runs of a byte plane: mark every block of 32 symbols that holds a non-zero
+     * one; keep only the marked blocks' symbols */
+    uint64_t blocks = ceil_div(m, ZRUN_BLOCK), kept = 0;
+    for (uint64_t b = 0; b < blocks; b++) {
+      uint64_t lo = b * ZRUN_BLOCK, hi = lo + ZRUN_BLOCK < m ? lo + ZRUN_BLOCK : m;
+      int marked = 0;
+      for (uint64_t i = lo; i < hi; i++)
+        if (sym[i]) marked = 1;
+      if (marked) kept += hi - lo;
+    }
+    uint64_t map_bytes = round16(ceil_div(blocks, 8));
+    uint64_t p_zrun = map_bytes + round16(ceil_div(kept * (uint64_t)w, 8));
+    if (p_zrun < p_raw) {
+      en->mode = MODE_ZRUN;
+      en->size = p_zrun;
+      en->bytes = (uint8_t*)calloc(p_zrun, 1);
+      if (!en->bytes) {
+        free(sym);
+        return ORC_EINVAL;
+      }
+      uint64_t tm = 0, td = 0;
+      for (uint64_t b = 0; b < blocks; b++) {
+        uint64_t lo = b * ZRUN_BLOCK, hi = lo + ZRUN_BLOCK < m ? lo + ZRUN_BLOCK : m;
+        int marked = 0;
+        for (uint64_t i = lo; i < hi; i++)
+          if (sym[i]) marked = 1;
+        put_bits(en->bytes, &tm, (uint32_t)marked, 1);
+        if (marked)
+          for (uint64_t i = lo; i < hi; i++) put_bits(en->bytes + map_bytes, &td, sym[i], w);
       }
       free(sym);
       return ORC_OK;
@@ -616,6 +662,27 @@ static int decode_entry(const djob_t* jb, uint64_t c, int s, uint64_t m, uint8_t
       uint32_t v = 0;
       for (int b = 0; b < w; b++) v = (v << 1) | (uint32_t)get_bit(jb->in + off, cap_bits, &t);
       sym[i] = (uint8_t)v;
+    }
+    return ORC_OK;
+  }
+  if (mode == MODE_ZRUN) {
+    if (code_ix != NO_CODE || is_entropy(dt, s) || w != 8) return ORC_ECORRUPT;
+    uint64_t blocks = ceil_div(m, ZRUN_BLOCK), map_bytes = round16(ceil_div(blocks, 8));
+    if (end - off < map_bytes) return ORC_ECORRUPT;
+    const uint8_t* map = jb->in + off;
+    const uint8_t* data = map + map_bytes;
+    uint64_t data_bits = (end - off - map_bytes) * 8, td = 0, tm = 0;
+    for (uint64_t b = 0; b < blocks; b++) {
+      uint64_t lo = b * ZRUN_BLOCK, hi = lo + ZRUN_BLOCK < m ? lo + ZRUN_BLOCK : m;
+      int marked = get_bit(map, map_bytes * 8, &tm);
+      for (uint64_t i = lo; i < hi; i++) {
+        uint32_t v = 0;
+        if (marked) {
+          if (td + (uint64_t)w > data_bits) return ORC_ECORRUPT;
+          for (int k = 0; k < w; k++) v = (v << 1) | (uint32_t)get_bit(data, data_bits, &td);
+        }
+        sym[i] = (uint8_t)v;
+      }
     }
     return ORC_OK;
   }

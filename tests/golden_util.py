@@ -33,6 +33,22 @@ def three_chunk_input():
     return x
 
 
+def zero_runs_input():
+    """The 296 BF16 values of bf16_zero_runs.json, from their numeric meaning."""
+    vals = []
+    for i in range(256):
+        if 32 <= i < 96:
+            vals.append(0.0)
+        else:
+            e = 127 if i % 2 == 0 else 126
+            vals.append((-1.0) ** (i >> 7) * (1 + (i & 127) / 128) * 2.0 ** (e - 127))
+    for j in range(40):
+        vals.append(0.0 if j < 32 else 1 + (j - 32) / 128)
+    x = torch.tensor(vals, dtype=torch.float64).to(torch.bfloat16)
+    assert torch.equal(x.to(torch.float64), torch.tensor(vals, dtype=torch.float64))  # exact in BF16
+    return x
+
+
 def fp8_two_chunk_input():
     """The 293 FP8 E4M3 values of fp8_two_chunks.json: built from their numeric meaning
     (-1)^sign * (1 + M/8) * 2^(E - 7), cast to float8_e4m3fn, and checked against the

@@ -73,6 +73,7 @@ GOLDEN_ALL = [
     ("fp8_shared_code.json", GU.fp8_two_chunk_input, True),
     ("fp32_clean_two_chunks.json", GU.fp32_clean_two_chunk_input, False),
     ("fp4_two_chunks.json", GU.fp4_two_chunk_input, False),
+    ("bf16_zero_runs.json", GU.zero_runs_input, False),
 ]
 
 

@@ -146,6 +146,7 @@ GOLDEN_OTHER = [
     ("fp8_shared_code.json", "fp8_e4m3", GU.fp8_two_chunk_input, True),
     ("fp32_clean_two_chunks.json", "fp32", GU.fp32_clean_two_chunk_input, False),
     ("fp4_two_chunks.json", "fp4_e2m1", GU.fp4_two_chunk_input, False),
+    ("bf16_zero_runs.json", "bf16", GU.zero_runs_input, False),
 ]
 
 
@@ -163,3 +164,65 @@ def test_golden_other_dtypes(orc, name, dtype, make, with_plan):
     assert bad.size == 0, f"first differing bytes at {bad[:8]}"
     y = orc.decompress(dtype, got, n, chunk_bytes=src["input"]["chunk_bytes"])
     assert np.array_equal(y, orc._bytes_view(x))
+
+
+def _entry_modes(c):
+    import container_util as CU
+    h, mode, code, off, ends = CU.payload_spans(c)
+    return h, mode, off, ends
+
+
+def test_zero_runs_round_trip_and_choice(orc):
+    """Byte planes with zeroed blocks take ZRUN exactly when it is strictly smaller than
+    RAW; the exponent (an entropy stream) never does; every case round-trips."""
+    g = torch.Generator().manual_seed(12)
+    # BF16 rows of 256 values; some rows zeroed (pruned), so whole 32-value blocks are zero
+    x = (torch.randn(64, 256, generator=g) * 0.02).to(torch.bfloat16)
+    x[torch.arange(64) % 3 == 0] = 0
+    c = _roundtrip(orc, "bf16", x.reshape(-1), 4096, S=64)
+    h, mode, off, ends = _entry_modes(c)
+    assert set(mode[1::2].tolist()) == {3}         # every sign/fraction plane: ZRUN
+    assert 3 not in mode[0::2].tolist()            # exponent: HUFF or RAW
+    # the ZRUN payload: bitmap of 2048/32 = 64 blocks (16 bytes) + kept bytes
+    for k in range(1, len(mode), 2):
+        assert ends[k] - off[k] < 2048              # smaller than RAW
+    # FP32 where every other 32-value block is clean: the two low planes keep half their
+    # blocks (whole clean chunks would be ZERO instead)
+    y = (torch.randn(1 << 16, generator=g) * 0.02).float()
+    clean = (torch.arange(1 << 16) // 32) % 2 == 0
+    y[clean] = y[clean].bfloat16().float()
+    c = _roundtrip(orc, "fp32", y, 1 << 16)
+    h, mode, off, ends = _entry_modes(c)
+    assert mode.reshape(-1, 4)[:, 2:].tolist() == [[3, 3]] * 4
+    # a plane with no zero block stays RAW; all zero stays ZERO
+    z = (torch.randn(4096, generator=g) * 0.02).to(torch.bfloat16)
+    c = _roundtrip(orc, "bf16", z, 8192)
+    assert _entry_modes(c)[1][1] == 0
+    c = _roundtrip(orc, "bf16", torch.zeros(4096, dtype=torch.bfloat16), 8192)
+    assert _entry_modes(c)[1].tolist() == [1, 1]
+
+
+def test_zero_runs_break_even(orc):
+    """ZRUN costs a 16-byte bitmap (padded) for a 4096-byte plane of 128 blocks; one zero
+    block saves 32 bytes but the kept bytes pad to 16 again: 16 + 4064 = 4080 < 4096, so
+    one zero block already makes ZRUN; the RAW tie (never here) would keep RAW."""
+    g = torch.Generator().manual_seed(13)
+    x = (torch.randn(4096, generator=g) * 0.02).to(torch.bfloat16)
+    x[:32] = 0
+    c = _roundtrip(orc, "bf16", x, 8192)
+    h, mode, off, ends = _entry_modes(c)
+    assert mode[1] == 3 and ends[1] - off[1] == 16 + 4064
+
+
+def test_zero_runs_corruption(orc):
+    import container_util as CU
+    g = torch.Generator().manual_seed(14)
+    x = (torch.randn(4096, generator=g) * 0.02).to(torch.bfloat16)
+    x[:1024] = 0
+    c = orc.compress("bf16", x, 4096, chunk_bytes=8192, S=64)
+    h, mode, off, ends = _entry_modes(c)
+    assert mode[1] == 3
+    d = c.copy(); d[64] = 3                           # ZRUN on the exponent (entropy) stream
+    assert orc.decompress_status("bf16", d, 4096, chunk_bytes=8192) == orc.ECORRUPT
+    d = c.copy(); d[off[1]: off[1] + 16] = 0xFF        # every block marked: data too short
+    assert orc.decompress_status("bf16", d, 4096, chunk_bytes=8192) == orc.ECORRUPT
