@@ -59,23 +59,27 @@ bool make_geo(int dt, uint64_t n, uint32_t chunk_bytes, uint32_t S, uint32_t G, 
   g.off_payload = g.off_codes + shared_bytes(dt, G);
   const uint32_t lim = g_spin_limit.load(std::memory_order_relaxed);
   g.spin_limit = lim ? lim : kSpinLimit;
+  g.zwords = (uint32_t)ceil_div(ceil_div(g.m0, kZBlock), 32);
   return true;
 }
 
 struct WsPlan {
-  uint64_t status, hist, nonzero, scan_desc, tile_desc, slot, zero_end;
+  uint64_t status, hist, nonzero, zmap, scan_desc, tile_desc, slot, zero_end;
   uint64_t esize, emode, ecode, eoff, enc, tile_hist, tile_off;
   uint64_t km_mu, km_perm, km_assign, km_changed, km_gsum, total;
   bool tile_counts;  // per-tile exponent histograms (BF16)
+  int dt;
 };
 
 WsPlan ws_plan(const Geo& g) {
   const uint64_t C = g.n_chunks, NE = (uint64_t)n_entropy(g.dt), K = g.n_entries;
   WsPlan p;
+  p.dt = g.dt;
   uint64_t o = 0;
   p.status = o;     o = align_up(o + 16 + C * 4);  // status, tickets, per-chunk counters
   p.hist = o;       o = align_up(o + C * NE * 256 * 4);
   p.nonzero = o;    o = align_up(o + K * 4);
+  p.zmap = o;       o = align_up(o + C * (uint64_t)n_byte_planes(g.dt) * g.zwords * 4);
   p.scan_desc = o;  o = align_up(o + (uint64_t)layout_tiles(g.n_entries) * 8);
   p.tile_desc = o;  o = align_up(o + NE * g.n_tiles * 8);
   p.slot = o;       o = align_up(o + NE * g.n_tiles * 8);
@@ -103,6 +107,7 @@ Ws carve(const WsPlan& p, void* base) {
   w.status = reinterpret_cast<uint32_t*>(b + p.status);
   w.hist = reinterpret_cast<uint32_t*>(b + p.hist);
   w.nonzero = reinterpret_cast<uint32_t*>(b + p.nonzero);
+  w.zmap = n_byte_planes(p.dt) ? reinterpret_cast<uint32_t*>(b + p.zmap) : nullptr;
   w.scan_desc = reinterpret_cast<uint64_t*>(b + p.scan_desc);
   w.tile_desc = reinterpret_cast<uint64_t*>(b + p.tile_desc);
   w.slot = reinterpret_cast<uint64_t*>(b + p.slot);

@@ -13,7 +13,10 @@ namespace zipnn {
 
 constexpr int kLmax = 12;
 constexpr uint32_t kNoCode = 0xFFFFFFFFu;
-constexpr uint32_t kModeRaw = 0, kModeZero = 1, kModeHuff = 2;
+constexpr uint32_t kModeRaw = 0, kModeZero = 1, kModeHuff = 2, kModeZrun = 3;
+// Zero runs: a byte plane is taken in blocks of 32 symbols; ZRUN keeps a bitmap of the
+// blocks that hold a non-zero byte and the bytes of those blocks only.
+constexpr uint32_t kZBlock = 32;
 constexpr int kBF16 = 0, kFP32 = 1, kFP8 = 2, kFP4 = 3;
 constexpr int kHeaderBytes = 64, kEntryBytes = 16;
 constexpr uint32_t kMaxGroups = 64;
@@ -54,6 +57,13 @@ __host__ __device__ constexpr uint32_t min32(uint32_t a, uint32_t b) { return a 
 __host__ __device__ constexpr uint64_t round16(uint64_t x) { return (x + 15) & ~uint64_t(15); }
 __host__ __device__ constexpr uint64_t ceil_div(uint64_t a, uint64_t b) { return (a + b - 1) / b; }
 __host__ __device__ constexpr uint32_t record_bytes(int dt, int s) { return (uint32_t)round16(alphabet(dt, s) / 2); }
+// Byte planes (8-bit streams that are not entropy-coded) may take zero runs: BF16's
+// sign/fraction byte (stream 1) and FP32's three fraction planes (streams 1..3).
+__host__ __device__ constexpr bool is_byte_plane(int dt, int s) { return !is_entropy(dt, s) && raw_width(dt, s) == 8; }
+__host__ __device__ constexpr int n_byte_planes(int dt) { return dt == kBF16 ? 1 : dt == kFP32 ? 3 : 0; }
+// ZRUN payload of m symbols with `kept` symbols in marked blocks: the bitmap, then the bytes.
+__host__ __device__ constexpr uint64_t zrun_map_bytes(uint64_t m) { return round16(ceil_div(ceil_div(m, kZBlock), 8)); }
+__host__ __device__ constexpr uint64_t zrun_payload(uint64_t m, uint64_t kept) { return zrun_map_bytes(m) + round16(kept); }
 __host__ __device__ constexpr uint64_t raw_payload(uint64_t m, int w) { return round16(ceil_div(m * (uint64_t)w, 8)); }
 
 // Bytes of all shared code records for g groups, and the position of record r.
@@ -80,6 +90,7 @@ struct Geo {
   uint32_t n_entries;         // n_chunks * n_streams
   uint64_t off_codes, off_payload;
   uint32_t spin_limit;        // polls after which a look-back wait gives up (kSpinLimit by default)
+  uint32_t zwords;            // words of one chunk's zero-run block bitmap: ceil(ceil(m0 / 32) / 32)
 };
 
 // Workspace carve-up (device pointers). The first group is cleared by every
@@ -89,6 +100,8 @@ struct Ws {
                         // finished histogram blocks
   uint32_t* hist;       // [n_chunks][n_entropy][256]
   uint32_t* nonzero;    // [n_entries]: OR of the stream's symbols
+  uint32_t* zmap;       // [n_chunks][n_byte_planes][zwords]: bit i of word w set when block
+                        // 32w + i of the plane holds a non-zero byte
   uint64_t* scan_desc;  // [layout tiles] look-back descriptors
   uint64_t* tile_desc;  // [n_tiles][n_entropy] look-back descriptors
   uint64_t* slot;       // [n_tiles][n_entropy] shared boundary words

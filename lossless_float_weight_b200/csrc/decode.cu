@@ -106,15 +106,30 @@ __device__ __forceinline__ uint32_t huff_pair(Reader& br, const uint32_t* lut, u
   return (e & 0x00FF0000u) | ((e2 & 0x00FF0000u) << 8);
 }
 
-enum Kind : int { kKZero = 0, kKBytes = 1, kKBits = 2, kKHuff = 3 };
+enum Kind : int { kKZero = 0, kKBytes = 1, kKBits = 2, kKHuff = 3, kKZrun = 4 };
 
 struct StreamState {
   int kind, width;
-  const uint8_t* bytes;  // kKBytes: this sub-block's first byte
+  const uint8_t* bytes;  // kKBytes: this sub-block's first byte; kKZrun: the kept bytes
   BitReader br;
   const uint32_t* lut;
   uint32_t acc;
+  // kKZrun: the block bitmap (MSB first), the kept bytes available, the sub-block's first
+  // value in the chunk, and the marked blocks before the current one
+  const uint8_t* zmap;
+  uint64_t zlimit;
+  uint32_t zbase, zrank, zmarked, zbad;
 };
+
+// Marked blocks before block b0 of a zero-run bitmap (MSB first within each byte).
+__device__ __forceinline__ uint32_t zrun_rank(const uint8_t* map, uint32_t b0) {
+  uint32_t r = 0;
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(map);
+  for (uint32_t i = 0; i < (b0 >> 5); i++) r += __popc(__ldg(w + i));
+  for (uint32_t i = (b0 >> 5) * 4; i < (b0 >> 3); i++) r += __popc((uint32_t)map[i]);
+  if (b0 & 7u) r += __popc((uint32_t)map[b0 >> 3] >> (8 - (b0 & 7u)));
+  return r;
+}
 
 // Decode GV consecutive symbols of one stream (GV a multiple of 2; n <= GV valid).
 template <int GV, bool FULL>
@@ -159,6 +174,37 @@ __device__ __forceinline__ void next_symbols(StreamState& st, uint32_t (&o)[GV],
         for (int i = 0; i < GV; i++) o[i] = i < n ? (uint32_t)st.bytes[v + i] : 0u;
       }
       break;
+    case kKZrun: {
+      // zero runs: a group of GV values (GV divides 32) lies in one block; a block's
+      // bytes are kept when its bitmap bit is set, at 32 x (marked blocks before it)
+      const uint32_t vv = st.zbase + v;
+      if (v == 0 || (vv & 31u) == 0) {
+        if (v != 0) st.zrank += st.zmarked;
+        st.zmarked = ((uint32_t)st.zmap[vv >> 8] >> (7 - ((vv >> 5) & 7u))) & 1u;
+      }
+      const uint64_t at = (uint64_t)st.zrank * kZBlock + (vv & 31u);
+      if (st.zmarked && at + GV <= st.zlimit) {
+        const uint8_t* src = st.bytes + at;
+        if (FULL) {
+          if constexpr (GV == 8) {
+            const uint2 q = __ldg(reinterpret_cast<const uint2*>(src));
+#pragma unroll
+            for (int i = 0; i < 8; i++) o[i] = ((i < 4 ? q.x : q.y) >> (8 * (i & 3))) & 0xFFu;
+          } else {
+#pragma unroll
+            for (int i = 0; i < GV; i++) o[i] = src[i];
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < GV; i++) o[i] = i < n ? (uint32_t)src[i] : 0u;
+        }
+      } else {
+        if (st.zmarked) st.zbad = 1;  // kept bytes past the payload: corrupt
+#pragma unroll
+        for (int i = 0; i < GV; i++) o[i] = 0;
+      }
+      break;
+    }
     default:
 #pragma unroll
       for (int i = 0; i < GV; i++) o[i] = 0;
@@ -324,11 +370,15 @@ __device__ __forceinline__ uint32_t ex_word(uint32_t row, uint32_t k) {
 // else lut is the two-symbol table. smp: the chunk's sign/fraction payload (RAW) or
 // nullptr (ZERO); outc: the chunk's first output value. Returns nonzero if the stream is
 // inconsistent.
-template <bool WIDE, class Lut>
+// ZRUN: the sign/fraction plane has zero runs; smp is its kept bytes, zmap / zpre the
+// chunk's block bitmap words (bit i of word w: block 32w + i) and the marked blocks before
+// each word, in shared memory.
+template <bool WIDE, bool ZRUN, class Lut>
 __device__ int decode_bf16_staged(StagedSmem& st, const Lut* lut, const uint32_t* tail,
                                   const uint32_t* __restrict__ idx, uint32_t bs_words,
                                   const uint8_t* __restrict__ smp, uint32_t m, uint32_t S, uint32_t nsub,
-                                  uint8_t* __restrict__ outc, uint32_t pre_start, uint32_t pre_next) {
+                                  uint8_t* __restrict__ outc, uint32_t pre_start, uint32_t pre_next,
+                                  const uint32_t* zmap, const uint32_t* zpre) {
   const int tid = threadIdx.x;
   int bad = 0;
   const uint64_t cap_bits = (uint64_t)bs_words * 32;
@@ -372,11 +422,19 @@ __device__ int decode_bf16_staged(StagedSmem& st, const Lut* lut, const uint32_t
         uval[p] = ubase[p] + off;
         ucnt[p] = n;
         smv[p] = make_uint2(0, 0);
-        if (smp && n == 8) smv[p] = __ldg(reinterpret_cast<const uint2*>(smp + uval[p]));
-        else if (smp && n) {
+        const uint8_t* src = nullptr;
+        if constexpr (ZRUN) {
+          const uint32_t b = uval[p] >> 5, word = zmap[b >> 5], bit = b & 31u;
+          if (n && ((word >> bit) & 1u))
+            src = smp + (uint64_t)(zpre[b >> 5] + __popc(word & ((1u << bit) - 1u))) * kZBlock + (uval[p] & 31u);
+        } else if (smp) {
+          src = smp + uval[p];
+        }
+        if (src && n == 8) smv[p] = __ldg(reinterpret_cast<const uint2*>(src));
+        else if (src && n) {
           uint32_t lo = 0, hi = 0;
           for (uint32_t i = 0; i < n; i++) {
-            const uint32_t b = smp[uval[p] + i];
+            const uint32_t b = src[i];
             if (i < 4) lo |= b << (8 * i);
             else hi |= b << (8 * (i - 4));
           }
@@ -455,6 +513,10 @@ struct DecodeSmem {
   uint32_t limit[n_entropy(DT)][kLmax + 1];
   uint32_t first[n_entropy(DT)][kLmax + 1];
   uint32_t offset[n_entropy(DT)][kLmax + 1];
+  // BF16 staged path with a ZRUN sign/fraction plane: the chunk's block bitmap (up to
+  // kZStagedWords words, bit i of word w = block 32w + i), the marked blocks before each
+  // word, and each warp's marked blocks while the prefix is built
+  uint32_t zmap[DT == kBF16 ? 128 : 1], zpre[DT == kBF16 ? 128 : 1], ztot[4];
   uint32_t mode[n_streams(DT)], code[n_streams(DT)];
   uint64_t off[n_streams(DT)], end[n_streams(DT)];
   uint64_t off_codes;
@@ -501,13 +563,182 @@ __device__ __forceinline__ void fill_lut(void* lut, const uint8_t* sorted, const
 
 static_assert(kDecodeThreads * 16 == 4096, "fill_lut: 16 table entries per thread");
 
+
+constexpr uint32_t kZStagedWords = 128;  // zero-run bitmap words the staged path holds: 4096 blocks
+static_assert(kDecodeThreads >= kZStagedWords, "one thread per bitmap word");
+
+// Every chunk the staged BF16 path does not take (FP32, FP8, FP4; BF16 with a RAW
+// exponent stream, a bitstream over 56 KB, or a ZRUN plane of more than 4096 blocks): one
+// sub-block per thread per pass, every stream read through its own reader. All threads.
+template <int DT>
+__device__ __noinline__ void decode_generic(const uint8_t* __restrict__ in, const DecodeSmem<DT>& sm, uint32_t m,
+                                            uint32_t S, uint64_t nsub, uint64_t clo, uint8_t* __restrict__ out,
+                                            uint32_t* status) {
+  constexpr int NS = n_streams(DT), NE = n_entropy(DT), VB = value_bytes(DT);
+  constexpr int GV = DT == kBF16 ? 8 : DT == kFP32 ? 4 : 16;  // values per store (16 bytes; FP4 8)
+  const int tid = threadIdx.x;
+  for (uint64_t j = tid; j < nsub; j += kDecodeThreads) {
+    const uint32_t sb_lo = (uint32_t)(j * S);
+    const uint32_t count = min32(S, m - sb_lo);
+    if constexpr (DT == kBF16) {
+      if (sm.mode[0] == kModeHuff && (sm.mode[1] == kModeRaw || sm.mode[1] == kModeZero)) {
+        const uint32_t rec = sm.code[0] == kNoCode ? record_bytes(DT, 0) : 0;
+        const uint32_t* idx = reinterpret_cast<const uint32_t*>(in + sm.off[0] + rec);
+        const uint64_t bs_off = sm.off[0] + rec + round16(4 * nsub);
+        const uint64_t cap_bits = (sm.end[0] - bs_off) * 8;
+        const uint64_t start = __ldg(idx + j);
+        const bool exact = j + 1 < nsub;
+        const uint64_t expect = exact ? __ldg(idx + j + 1) : cap_bits;
+        int bad = (j == 0 && start != 0) || start > cap_bits || expect < start || expect > cap_bits;
+        const uint32_t* bs = reinterpret_cast<const uint32_t*>(in + bs_off);
+        uint8_t* dst = out + (clo + sb_lo) * VB;
+        if (sm.mode[1] == kModeZero)
+          bad |= decode_bf16_fast<true>(sm.lut[0], nullptr, bs, (uint32_t)(cap_bits / 32), bad ? 0 : start,
+                                                   expect, exact, count, dst);
+        else
+          bad |= decode_bf16_fast<false>(sm.lut[0], in + sm.off[1] + sb_lo, bs, (uint32_t)(cap_bits / 32),
+                                                    bad ? 0 : start, expect, exact, count, dst);
+        if (bad) set_status(status, kStCorrupt);
+        continue;
+      }
+    }
+    StreamState st[NS];
+    uint64_t expect_end[NS];
+    bool check_exact[NS];
+    int bad = 0;
+#pragma unroll
+    for (int s = 0; s < NS; s++) {
+      const uint32_t mode = sm.mode[s];
+      const int w = raw_width(DT, s);
+      st[s].acc = 0;
+      st[s].width = w;
+      st[s].lut = nullptr;
+      st[s].bytes = nullptr;
+      st[s].zbad = 0;
+      check_exact[s] = false;
+      expect_end[s] = 0;
+      if (mode == kModeZero) {
+        st[s].kind = kKZero;
+      } else if (mode == kModeZrun) {
+        // zero runs (a byte plane): the bitmap, then the kept bytes; the marked blocks
+        // before my first block give my first rank
+        const uint64_t map_bytes = zrun_map_bytes(m);
+        st[s].kind = kKZrun;
+        st[s].zmap = in + sm.off[s];
+        st[s].bytes = in + sm.off[s] + map_bytes;
+        st[s].zlimit = sm.end[s] - sm.off[s] - map_bytes;
+        st[s].zbase = sb_lo;
+        st[s].zrank = zrun_rank(st[s].zmap, sb_lo / kZBlock);
+        st[s].zmarked = 0;
+      } else if (mode == kModeRaw) {
+        if (w == 8) {
+          st[s].kind = kKBytes;
+          st[s].bytes = in + sm.off[s] + sb_lo;
+        } else {
+          st[s].kind = kKBits;
+          st[s].br.init(reinterpret_cast<const uint32_t*>(in + sm.off[s]), (uint32_t)((sm.end[s] - sm.off[s]) / 4),
+                        (uint64_t)sb_lo * w);
+        }
+      } else {
+        const int e = s < NE ? s : 0;
+        const uint32_t rec = sm.code[s] == kNoCode ? record_bytes(DT, s) : 0;
+        const uint32_t* idx = reinterpret_cast<const uint32_t*>(in + sm.off[s] + rec);
+        const uint64_t bs_off = sm.off[s] + rec + round16(4 * nsub);
+        const uint64_t cap_bits = (sm.end[s] - bs_off) * 8;
+        const uint64_t start = __ldg(idx + j);
+        if (j == 0 && start != 0) bad = 1;
+        if (start > cap_bits) bad = 1;
+        if (j + 1 < nsub) {
+          expect_end[s] = __ldg(idx + j + 1);
+          check_exact[s] = true;
+          if (expect_end[s] < start || expect_end[s] > cap_bits) bad = 1;
+        } else {
+          expect_end[s] = cap_bits;
+        }
+        st[s].kind = kKHuff;
+        st[s].lut = sm.lut[e];
+        st[s].br.init(reinterpret_cast<const uint32_t*>(in + bs_off), (uint32_t)(cap_bits / 32), bad ? 0 : start);
+      }
+    }
+    uint8_t* dst = out + value_offset(DT, clo + sb_lo);
+    const uint32_t full = count / GV;
+    for (uint32_t gi = 0; gi < full; gi++) {
+      uint32_t sy[NS][GV];
+#pragma unroll
+      for (int s = 0; s < NS; s++) next_symbols<GV, true>(st[s], sy[s], GV, gi * GV);
+      if constexpr (DT == kFP4) {  // two values a byte, the first in the low nibble
+        uint32_t wv[2];
+#pragma unroll
+        for (int q = 0; q < 2; q++) {
+          uint32_t x = 0;
+#pragma unroll
+          for (int b = 0; b < 8; b++) x |= merge_value<DT>(sy[0][8 * q + b], sy[1][8 * q + b], sy[2][8 * q + b], 0) << (4 * b);
+          wv[q] = x;
+        }
+        *reinterpret_cast<uint2*>(dst + (uint64_t)gi * 8) = make_uint2(wv[0], wv[1]);
+      } else {
+        uint32_t wv[4];
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+          if constexpr (DT == kBF16) {
+            wv[q] = merge_value<DT>(sy[0][2 * q], sy[1][2 * q], 0, 0) |
+                    (merge_value<DT>(sy[0][2 * q + 1], sy[1][2 * q + 1], 0, 0) << 16);
+          } else if constexpr (DT == kFP32) {
+            wv[q] = merge_value<DT>(sy[0][q], sy[1][q], sy[2][q], sy[3][q]);
+          } else {
+            uint32_t x = 0;
+#pragma unroll
+            for (int b = 0; b < 4; b++) x |= merge_value<DT>(sy[0][4 * q + b], sy[1][4 * q + b], sy[2][4 * q + b], 0) << (8 * b);
+            wv[q] = x;
+          }
+        }
+        *reinterpret_cast<uint4*>(dst + (uint64_t)gi * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+      }
+    }
+    const uint32_t rem = count - full * GV;
+    if (rem) {
+      uint32_t sy[NS][GV];
+#pragma unroll
+      for (int s = 0; s < NS; s++) next_symbols<GV, false>(st[s], sy[s], (int)rem, full * GV);
+      if constexpr (DT == kFP4) {  // rem is even: values come in byte pairs
+#pragma unroll
+        for (uint32_t i = 0; i < (uint32_t)GV; i += 2) {
+          if (i >= rem) break;
+          const uint32_t lo = merge_value<DT>(sy[0][i], sy[1][i], sy[2][i], 0);
+          const uint32_t hi = merge_value<DT>(sy[0][i + 1], sy[1][i + 1], sy[2][i + 1], 0);
+          dst[(full * GV + i) / 2] = (uint8_t)(lo | (hi << 4));
+        }
+      } else {
+#pragma unroll
+        for (uint32_t i = 0; i < (uint32_t)GV; i++) {
+          if (i >= rem) break;
+          const uint32_t v = merge_value<DT>(sy[0][i], sy[1][i], NS > 2 ? sy[NS > 2 ? 2 : 0][i] : 0,
+                                             NS > 3 ? sy[NS > 3 ? 3 : 0][i] : 0);
+          uint8_t* p = dst + (uint64_t)(full * GV + i) * VB;
+          if constexpr (VB == 2) *reinterpret_cast<uint16_t*>(p) = (uint16_t)v;
+          else if constexpr (VB == 4) *reinterpret_cast<uint32_t*>(p) = v;
+          else *p = (uint8_t)v;
+        }
+      }
+    }
+#pragma unroll
+    for (int s = 0; s < NS; s++) {
+      if (st[s].kind == kKZrun && st[s].zbad) bad = 1;
+      if (st[s].kind != kKHuff) continue;
+      const uint64_t pos = st[s].br.position();
+      if (st[s].acc & kLutInvalid) bad = 1;
+      if (check_exact[s] ? pos != expect_end[s] : pos > expect_end[s]) bad = 1;
+    }
+    if (bad) set_status(status, kStCorrupt);
+  }
+}
+
 // Chunk c of the container `in` (in_bytes readable) of a tensor with geometry g, into
 // `out` (the tensor's first value). All threads of the block.
 template <int DT>
 __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uint64_t in_bytes, const Geo& g,
                                              uint32_t c, uint8_t* __restrict__ out, uint32_t* status) {
   constexpr int NS = n_streams(DT), NE = n_entropy(DT), VB = value_bytes(DT);
-  constexpr int GV = DT == kBF16 ? 8 : DT == kFP32 ? 4 : 16;  // values per store (16 bytes; FP4 8)
   __shared__ __align__(16) DecodeSmem<DT> sm;  // 16-byte aligned: a bulk copy may target its table
   extern __shared__ __align__(128) uint8_t dyn_smem[];  // StagedSmem for BF16 launches
   const int tid = threadIdx.x;
@@ -557,7 +788,7 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
         const uint64_t off = ent[s].z | ((uint64_t)ent[s].w << 32);
         const uint64_t end = k + 1 < entries ? (ent[s + 1].z | ((uint64_t)ent[s + 1].w << 32)) : total;
         const uint32_t mode = ent[s].x & 0xFF;
-        if ((ent[s].x >> 8) != 0 || mode > kModeHuff) bad = 1;
+        if ((ent[s].x >> 8) != 0 || mode > kModeZrun) bad = 1;
         if ((off & 15) || (end & 15) || off > end || end > total || off < off_payload) bad = 1;
         if (k == 0 && off != off_payload) bad = 1;
         const uint64_t extent = end - off;
@@ -566,6 +797,8 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
           if (ent[s].y != kNoCode || extent * 8 < (uint64_t)m * w) bad = 1;
         } else if (mode == kModeZero) {
           if (ent[s].y != kNoCode) bad = 1;
+        } else if (mode == kModeZrun) {
+          if (!is_byte_plane(DT, s) || ent[s].y != kNoCode || extent < zrun_map_bytes(m)) bad = 1;
         } else if (mode == kModeHuff && S != 0) {
           const uint64_t nsub = ceil_div(m, S);
           uint64_t need = round16(4 * nsub);
@@ -588,7 +821,8 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
     if constexpr (DT == kBF16) {
       // staged path: HUFF exponents, RAW or ZERO sign/fraction bytes, bitstream in the
       // window (1), or in the window and the table's first half (2, the wide window)
-      if (!bad && sm.mode[0] == kModeHuff && sm.mode[1] != kModeHuff) {
+      if (!bad && sm.mode[0] == kModeHuff && sm.mode[1] != kModeHuff &&
+          (sm.mode[1] != kModeZrun || ceil_div(ceil_div(m, kZBlock), 32) <= kZStagedWords)) {
         const uint64_t nsub = ceil_div(m, S);
         const uint32_t rec = sm.code[0] == kNoCode ? record_bytes(DT, 0) : 0;
         const uint64_t bs_off = sm.off[0] + rec + round16(4 * nsub);
@@ -629,6 +863,26 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
     }
   }
 
+  // BF16 staged path, ZRUN sign/fraction plane: thread w < 128 takes bitmap word w (the
+  // payload's bytes are MSB first: reversing the bits of each byte gives bit i = block
+  // 32w + i) and its in-warp prefix of marked blocks; the warps' totals join below.
+  const bool zstaged = DT == kBF16 && sm.staged && sm.mode[1] == kModeZrun;
+  if (zstaged && tid < (int)kZStagedWords) {
+    const uint32_t used = (uint32_t)ceil_div(ceil_div(m, kZBlock), 32);
+    const uint32_t raw = tid < (int)used ? __ldg(reinterpret_cast<const uint32_t*>(in + sm.off[1]) + tid) : 0u;
+    const uint32_t word = __byte_perm(__brev(raw), 0, 0x0123);
+    const uint32_t pc = __popc(word);
+    uint32_t incl = pc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    sm.zmap[tid] = word;
+    sm.zpre[tid] = incl - pc;
+    if (lane == 31) sm.ztot[warp] = incl;
+  }
+
   // Canonical tables of each HUFF stream, from its 4-bit code lengths. Thread t takes
   // symbol t: each warp counts its 32 symbols of every length (ballots) and each symbol's
   // rank among the warp's symbols of its length (match), with the Kraft sum, a length
@@ -664,6 +918,20 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
     }
   }
   __syncthreads();
+  if (zstaged && tid < (int)kZStagedWords) {
+    uint32_t before = 0;
+    for (int w = 0; w < (tid >> 5); w++) before += sm.ztot[w];
+    sm.zpre[tid] += before;
+    if (tid == 0) {
+      // the kept bytes must lie inside the payload: 32 per marked block, less what a marked
+      // short last block lacks, padded to 16
+      const uint32_t total = sm.ztot[0] + sm.ztot[1] + sm.ztot[2] + sm.ztot[3];
+      const uint64_t last = (m - 1) / kZBlock;
+      uint64_t kept = (uint64_t)total * kZBlock;
+      if ((m % kZBlock) && ((sm.zmap[last >> 5] >> (last & 31)) & 1u)) kept -= kZBlock - m % kZBlock;
+      if (sm.end[1] - sm.off[1] < zrun_payload(m, kept)) sm.bad = 1;
+    }
+  }
   // warp e: lengths' counts, first codes (RFC 1951, 3.2.2: first[l] = (first[l-1] +
   // count[l-1]) << 1, i.e. the sum over q < l of count[q] << (l - q)), canonical index
   // offsets, left-aligned limits, and every warp's base index for each length; lane l
@@ -779,157 +1047,29 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
       const uint32_t* idx = reinterpret_cast<const uint32_t*>(in + sm.off[0] + rec);
       const uint64_t bs_off = sm.off[0] + rec + round16(4 * nsub);
       const uint32_t bs_words = (uint32_t)((sm.end[0] - bs_off) / 4);
-      const uint8_t* smp = sm.mode[1] == kModeRaw ? in + sm.off[1] : nullptr;
-      const int bad = wide ? decode_bf16_staged<true>(stg, lut16, sm.lut[0], idx, bs_words, smp, m, S,
-                                                      (uint32_t)nsub, out + clo * VB, idx_start, idx_next)
-                           : decode_bf16_staged<false>(stg, sm.lut[0], nullptr, idx, bs_words, smp, m, S,
-                                                       (uint32_t)nsub, out + clo * VB, idx_start, idx_next);
+      const uint8_t* smp = sm.mode[1] == kModeRaw    ? in + sm.off[1]
+                           : sm.mode[1] == kModeZrun ? in + sm.off[1] + zrun_map_bytes(m)
+                                                     : nullptr;
+      int bad;
+      if (sm.mode[1] == kModeZrun)
+        bad = wide ? decode_bf16_staged<true, true>(stg, lut16, sm.lut[0], idx, bs_words, smp, m, S, (uint32_t)nsub,
+                                                    out + clo * VB, idx_start, idx_next, sm.zmap, sm.zpre)
+                   : decode_bf16_staged<false, true>(stg, sm.lut[0], nullptr, idx, bs_words, smp, m, S,
+                                                     (uint32_t)nsub, out + clo * VB, idx_start, idx_next, sm.zmap,
+                                                     sm.zpre);
+      else
+        bad = wide ? decode_bf16_staged<true, false>(stg, lut16, sm.lut[0], idx, bs_words, smp, m, S, (uint32_t)nsub,
+                                                     out + clo * VB, idx_start, idx_next, nullptr, nullptr)
+                   : decode_bf16_staged<false, false>(stg, sm.lut[0], nullptr, idx, bs_words, smp, m, S,
+                                                      (uint32_t)nsub, out + clo * VB, idx_start, idx_next, nullptr,
+                                                      nullptr);
       if (bad) set_status(status, kStCorrupt);
       return;
     }
   }
-  // decode: one sub-block per thread per pass
-  for (uint64_t j = tid; j < nsub; j += kDecodeThreads) {
-    const uint32_t sb_lo = (uint32_t)(j * S);
-    const uint32_t count = min32(S, m - sb_lo);
-    if constexpr (DT == kBF16) {
-      if (sm.mode[0] == kModeHuff && sm.mode[1] != kModeHuff) {
-        const uint32_t rec = sm.code[0] == kNoCode ? record_bytes(DT, 0) : 0;
-        const uint32_t* idx = reinterpret_cast<const uint32_t*>(in + sm.off[0] + rec);
-        const uint64_t bs_off = sm.off[0] + rec + round16(4 * nsub);
-        const uint64_t cap_bits = (sm.end[0] - bs_off) * 8;
-        const uint64_t start = __ldg(idx + j);
-        const bool exact = j + 1 < nsub;
-        const uint64_t expect = exact ? __ldg(idx + j + 1) : cap_bits;
-        int bad = (j == 0 && start != 0) || start > cap_bits || expect < start || expect > cap_bits;
-        const uint32_t* bs = reinterpret_cast<const uint32_t*>(in + bs_off);
-        uint8_t* dst = out + (clo + sb_lo) * VB;
-        if (sm.mode[1] == kModeZero)
-          bad |= decode_bf16_fast<true>(sm.lut[0], nullptr, bs, (uint32_t)(cap_bits / 32), bad ? 0 : start,
-                                                   expect, exact, count, dst);
-        else
-          bad |= decode_bf16_fast<false>(sm.lut[0], in + sm.off[1] + sb_lo, bs, (uint32_t)(cap_bits / 32),
-                                                    bad ? 0 : start, expect, exact, count, dst);
-        if (bad) set_status(status, kStCorrupt);
-        continue;
-      }
-    }
-    StreamState st[NS];
-    uint64_t expect_end[NS];
-    bool check_exact[NS];
-    int bad = 0;
-#pragma unroll
-    for (int s = 0; s < NS; s++) {
-      const uint32_t mode = sm.mode[s];
-      const int w = raw_width(DT, s);
-      st[s].acc = 0;
-      st[s].width = w;
-      st[s].lut = nullptr;
-      st[s].bytes = nullptr;
-      check_exact[s] = false;
-      expect_end[s] = 0;
-      if (mode == kModeZero) {
-        st[s].kind = kKZero;
-      } else if (mode == kModeRaw) {
-        if (w == 8) {
-          st[s].kind = kKBytes;
-          st[s].bytes = in + sm.off[s] + sb_lo;
-        } else {
-          st[s].kind = kKBits;
-          st[s].br.init(reinterpret_cast<const uint32_t*>(in + sm.off[s]), (uint32_t)((sm.end[s] - sm.off[s]) / 4),
-                        (uint64_t)sb_lo * w);
-        }
-      } else {
-        const int e = s < NE ? s : 0;
-        const uint32_t rec = sm.code[s] == kNoCode ? record_bytes(DT, s) : 0;
-        const uint32_t* idx = reinterpret_cast<const uint32_t*>(in + sm.off[s] + rec);
-        const uint64_t bs_off = sm.off[s] + rec + round16(4 * nsub);
-        const uint64_t cap_bits = (sm.end[s] - bs_off) * 8;
-        const uint64_t start = __ldg(idx + j);
-        if (j == 0 && start != 0) bad = 1;
-        if (start > cap_bits) bad = 1;
-        if (j + 1 < nsub) {
-          expect_end[s] = __ldg(idx + j + 1);
-          check_exact[s] = true;
-          if (expect_end[s] < start || expect_end[s] > cap_bits) bad = 1;
-        } else {
-          expect_end[s] = cap_bits;
-        }
-        st[s].kind = kKHuff;
-        st[s].lut = sm.lut[e];
-        st[s].br.init(reinterpret_cast<const uint32_t*>(in + bs_off), (uint32_t)(cap_bits / 32), bad ? 0 : start);
-      }
-    }
-    uint8_t* dst = out + value_offset(DT, clo + sb_lo);
-    const uint32_t full = count / GV;
-    for (uint32_t gi = 0; gi < full; gi++) {
-      uint32_t sy[NS][GV];
-#pragma unroll
-      for (int s = 0; s < NS; s++) next_symbols<GV, true>(st[s], sy[s], GV, gi * GV);
-      if constexpr (DT == kFP4) {  // two values a byte, the first in the low nibble
-        uint32_t wv[2];
-#pragma unroll
-        for (int q = 0; q < 2; q++) {
-          uint32_t x = 0;
-#pragma unroll
-          for (int b = 0; b < 8; b++) x |= merge_value<DT>(sy[0][8 * q + b], sy[1][8 * q + b], sy[2][8 * q + b], 0) << (4 * b);
-          wv[q] = x;
-        }
-        *reinterpret_cast<uint2*>(dst + (uint64_t)gi * 8) = make_uint2(wv[0], wv[1]);
-      } else {
-        uint32_t wv[4];
-#pragma unroll
-        for (int q = 0; q < 4; q++) {
-          if constexpr (DT == kBF16) {
-            wv[q] = merge_value<DT>(sy[0][2 * q], sy[1][2 * q], 0, 0) |
-                    (merge_value<DT>(sy[0][2 * q + 1], sy[1][2 * q + 1], 0, 0) << 16);
-          } else if constexpr (DT == kFP32) {
-            wv[q] = merge_value<DT>(sy[0][q], sy[1][q], sy[2][q], sy[3][q]);
-          } else {
-            uint32_t x = 0;
-#pragma unroll
-            for (int b = 0; b < 4; b++) x |= merge_value<DT>(sy[0][4 * q + b], sy[1][4 * q + b], sy[2][4 * q + b], 0) << (8 * b);
-            wv[q] = x;
-          }
-        }
-        *reinterpret_cast<uint4*>(dst + (uint64_t)gi * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-      }
-    }
-    const uint32_t rem = count - full * GV;
-    if (rem) {
-      uint32_t sy[NS][GV];
-#pragma unroll
-      for (int s = 0; s < NS; s++) next_symbols<GV, false>(st[s], sy[s], (int)rem, full * GV);
-      if constexpr (DT == kFP4) {  // rem is even: values come in byte pairs
-#pragma unroll
-        for (uint32_t i = 0; i < (uint32_t)GV; i += 2) {
-          if (i >= rem) break;
-          const uint32_t lo = merge_value<DT>(sy[0][i], sy[1][i], sy[2][i], 0);
-          const uint32_t hi = merge_value<DT>(sy[0][i + 1], sy[1][i + 1], sy[2][i + 1], 0);
-          dst[(full * GV + i) / 2] = (uint8_t)(lo | (hi << 4));
-        }
-      } else {
-#pragma unroll
-        for (uint32_t i = 0; i < (uint32_t)GV; i++) {
-          if (i >= rem) break;
-          const uint32_t v = merge_value<DT>(sy[0][i], sy[1][i], NS > 2 ? sy[NS > 2 ? 2 : 0][i] : 0,
-                                             NS > 3 ? sy[NS > 3 ? 3 : 0][i] : 0);
-          uint8_t* p = dst + (uint64_t)(full * GV + i) * VB;
-          if constexpr (VB == 2) *reinterpret_cast<uint16_t*>(p) = (uint16_t)v;
-          else if constexpr (VB == 4) *reinterpret_cast<uint32_t*>(p) = v;
-          else *p = (uint8_t)v;
-        }
-      }
-    }
-#pragma unroll
-    for (int s = 0; s < NS; s++) {
-      if (st[s].kind != kKHuff) continue;
-      const uint64_t pos = st[s].br.position();
-      if (st[s].acc & kLutInvalid) bad = 1;
-      if (check_exact[s] ? pos != expect_end[s] : pos > expect_end[s]) bad = 1;
-    }
-    if (bad) set_status(status, kStCorrupt);
-  }
+  // the other cases: one sub-block per thread per pass, in a function of its own so that
+  // its register needs do not weigh on the staged path above
+  decode_generic<DT>(in, sm, m, S, nsub, clo, out, status);
 }
 
 template <int DT>

@@ -43,6 +43,8 @@ struct EncodeSmem {
   uint32_t stage[kStageWords];                  // the tile's bitstream, at its final bit alignment
   uint32_t enc[n_entropy(DT)][256];
   uint32_t warp[kEncodeThreads / 32];
+  uint32_t zmap[32];  // ZRUN byte plane: the tile's block-bitmap words (16 of them)
+  uint32_t zpre[32];  // marked blocks of the chunk before each of those words
   uint64_t prefix;
   uint64_t off[n_streams(DT)];
   uint32_t mode[n_streams(DT)], code[n_streams(DT)];
@@ -123,6 +125,70 @@ __global__ void __launch_bounds__(kEncodeThreads) k_encode(const uint8_t* __rest
           }
           *reinterpret_cast<uint4*>(out + sm.off[s] + v0 + 16 * q) = make_uint4(x[0], x[1], x[2], x[3]);
         }
+      }
+      continue;
+    }
+    if (mode == kModeZrun) {
+      if constexpr (n_byte_planes(DT) > 0) {
+        // zero runs of a byte plane: the tile's 512 blocks are bitmap words 16 ti ..
+        // 16 ti + 15; warp 0 loads them with each word's rank base (the chunk's marked
+        // blocks before it) and writes them into the payload's bitmap (MSB first), the
+        // last tile also the bitmap's zero padding
+        constexpr uint32_t kTileWords = kTileValues / kZBlock / 32;
+        const uint64_t map_bytes = zrun_map_bytes(m);
+        if (tid < 32) {
+          const uint32_t* map = ws.zmap + ((uint64_t)c * n_byte_planes(DT) + (s - 1)) * g.zwords;
+          const uint32_t w0 = ti * kTileWords, used = (uint32_t)ceil_div(ceil_div(m, kZBlock), 32);
+          uint32_t base = 0;
+          for (uint32_t w = tid; w < w0; w += 32) base += __popc(__ldcg(map + w));
+          base = __reduce_add_sync(0xFFFFFFFFu, base);
+          const uint32_t word = (tid < (int)kTileWords && w0 + tid < used) ? __ldcg(map + w0 + tid) : 0u;
+          const uint32_t pc = __popc(word);
+          uint32_t incl = pc;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (tid >= o) incl += y;
+          }
+          sm.zmap[tid] = word;
+          sm.zpre[tid] = base + incl - pc;
+          uint32_t* mp = reinterpret_cast<uint32_t*>(out + sm.off[s]);
+          if (tid < (int)kTileWords && w0 + tid < used) mp[w0 + tid] = __byte_perm(__brev(word), 0, 0x0123);
+          if (last)
+            for (uint32_t w = used + tid; w < map_bytes / 4; w += 32) mp[w] = 0;
+        }
+        __syncthreads();
+        // my values are blocks v0 / 32 and v0 / 32 + 1: a marked block's bytes go to 32 x
+        // (its rank) after the bitmap, in 16-byte groups (zero past cnt, so the chunk's
+        // short last block ends with its padding); an unmarked block is not stored
+        if (cnt > 0) {
+          uint8_t* half[2];
+#pragma unroll
+          for (int h = 0; h < 2; h++) {
+            const uint32_t lb = (v0 - tlo) / kZBlock + (uint32_t)h;
+            const uint32_t word = sm.zmap[lb >> 5], bit = lb & 31u;
+            half[h] = ((word >> bit) & 1u) ? out + sm.off[s] + map_bytes +
+                                                 (uint64_t)(sm.zpre[lb >> 5] + __popc(word & ((1u << bit) - 1u))) * kZBlock
+                                           : nullptr;
+          }
+#pragma unroll
+          for (int q = 0; q < kEncValues / 16; q++) {
+            if (16 * q < cnt && half[q >> 1]) {
+              uint32_t x[4];
+#pragma unroll
+              for (int j = 0; j < 4; j++) {
+                x[j] = 0;
+#pragma unroll
+                for (int b = 0; b < 4; b++) {
+                  const int i = 16 * q + 4 * j + b;
+                  if (i < cnt) x[j] |= symbol<DT, kEncValues>(raw, s, i) << (8 * b);
+                }
+              }
+              *reinterpret_cast<uint4*>(half[q >> 1] + 16 * (q & 1)) = make_uint4(x[0], x[1], x[2], x[3]);
+            }
+          }
+        }
+        __syncthreads();  // the next stream's tables may reuse zmap / zpre
       }
       continue;
     }

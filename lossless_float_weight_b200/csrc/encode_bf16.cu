@@ -43,6 +43,8 @@ struct Bf16EncodeSmem {
   uint32_t stage[kBStageWords];                  // the tile's bitstream at its final alignment
   uint32_t enc[256];                             // the chunk's code: len << 16 | code
   alignas(16) uint32_t warp[2][kBThreads / 32];  // warp bit totals, by pass parity
+  uint32_t zmap[32];  // ZRUN sign/fraction plane: the tile's 32 block-bitmap words
+  uint32_t zpre[32];  // marked blocks of the chunk before each of those words
   uint32_t carry[2];  // the bits of the word shared with the next pass, by pass parity
 };
 
@@ -79,6 +81,31 @@ __global__ void __launch_bounds__(kBThreads, 8) k_encode_bf16(const uint8_t* __r
       for (int i = tid; i < 256; i += kBThreads) sm.enc[i] = ws.enc[(uint64_t)c * 256 + i];
       P = ws.tile_off[tile];
     }
+    if (mode1 == kModeZrun && tid < 32) {
+      // zero runs: the tile's 1024 blocks are bitmap words 32 ti .. 32 ti + 31; each word's
+      // rank base is the chunk's marked blocks before it. The tile also writes its words of
+      // the payload's bitmap (MSB first: bits reversed within each byte), and the last tile
+      // the bitmap's zero padding.
+      const uint32_t* map = ws.zmap + (uint64_t)c * g.zwords;
+      const uint32_t w0 = ti * 32u, used = (uint32_t)ceil_div(ceil_div(m, kZBlock), 32);
+      uint32_t base = 0;
+      for (uint32_t w = tid; w < w0; w += 32) base += __popc(__ldcg(map + w));
+      base = __reduce_add_sync(0xFFFFFFFFu, base);
+      const uint32_t word = w0 + tid < used ? __ldcg(map + w0 + tid) : 0u;
+      const uint32_t pc = __popc(word);
+      uint32_t incl = pc;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (tid >= o) incl += y;
+      }
+      sm.zmap[tid] = word;
+      sm.zpre[tid] = base + incl - pc;
+      uint32_t* mp = reinterpret_cast<uint32_t*>(out + off1);
+      if (w0 + tid < used) mp[w0 + tid] = __byte_perm(__brev(word), 0, 0x0123);
+      if (tlo + (uint32_t)kBf16TileValues >= m)
+        for (uint32_t w = used + tid; w < zrun_map_bytes(m) / 4; w += 32) mp[w] = 0;
+    }
     __syncthreads();  // the code is visible; the previous tile's stores and clears are done
     const uint64_t nsub = ceil_div(m, g.S);
     const uint32_t rec = code0 == kNoCode ? record_bytes(kBF16, 0) : 0;
@@ -99,9 +126,28 @@ __global__ void __launch_bounds__(kBThreads, 8) k_encode_bf16(const uint8_t* __r
 
 #pragma unroll
       for (int s = 0; s < 2; s++) {
-        if ((s == 0 ? mode0 : mode1) != kModeRaw || cnt == 0) continue;
-        // RAW byte plane (the sign/fraction bytes; an exponent stream that did not compress)
-        uint8_t* dst = out + (s == 0 ? off0 : off1) + v0;
+        const uint32_t mode = s == 0 ? mode0 : mode1;
+        if ((mode != kModeRaw && !(s == 1 && mode == kModeZrun)) || cnt == 0) continue;
+        // a byte plane: RAW (the sign/fraction bytes; an exponent stream that did not
+        // compress) at the values' own offset; ZRUN (sign/fraction bytes with zero runs):
+        // my values are blocks v0 / 32 and v0 / 32 + 1, and a marked block's 32 bytes go to
+        // 32 x (its rank among the chunk's marked blocks) after the bitmap; an unmarked
+        // block is not stored
+        uint8_t* half[2];
+        if (mode == kModeRaw) {
+          half[0] = out + (s == 0 ? off0 : off1) + v0;
+          half[1] = half[0] + 32;
+        } else {
+          uint8_t* data = out + off1 + zrun_map_bytes(m);
+#pragma unroll
+          for (int h = 0; h < 2; h++) {
+            const uint32_t lb = (v0 - tlo) / kZBlock + (uint32_t)h;  // block within the tile
+            const uint32_t word = sm.zmap[lb >> 5], bit = lb & 31u;
+            half[h] = ((word >> bit) & 1u)
+                          ? data + (uint64_t)(sm.zpre[lb >> 5] + __popc(word & ((1u << bit) - 1u))) * kZBlock
+                          : nullptr;
+          }
+        }
         if (cnt == kBValues) {
 #pragma unroll
           for (int q = 0; q < kBValues / 16; q++) {
@@ -110,12 +156,14 @@ __global__ void __launch_bounds__(kBThreads, 8) k_encode_bf16(const uint8_t* __r
             for (int k = 0; k < 4; k++)
               x[k] = __byte_perm(bf16_pair_plane(raw.w[8 * q + 2 * k], s),
                                  bf16_pair_plane(raw.w[8 * q + 2 * k + 1], s), 0x6420);
-            *reinterpret_cast<uint4*>(dst + 16 * q) = make_uint4(x[0], x[1], x[2], x[3]);
+            if (half[q >> 1]) *reinterpret_cast<uint4*>(half[q >> 1] + 16 * (q & 1)) = make_uint4(x[0], x[1], x[2], x[3]);
           }
         } else {
+          // the chunk's last values: 16-byte groups, zero past cnt (a ZRUN block's data
+          // then ends with the zero padding to its 16-byte boundary)
 #pragma unroll
           for (int q = 0; q < kBValues / 16; q++) {
-            if (16 * q < cnt) {
+            if (16 * q < cnt && half[q >> 1]) {
               uint32_t x[4];
 #pragma unroll
               for (int j = 0; j < 4; j++) {
@@ -126,7 +174,7 @@ __global__ void __launch_bounds__(kBThreads, 8) k_encode_bf16(const uint8_t* __r
                   if (i < cnt) x[j] |= symbol<kBF16, kBValues>(raw, s, i) << (8 * b);
                 }
               }
-              *reinterpret_cast<uint4*>(dst + 16 * q) = make_uint4(x[0], x[1], x[2], x[3]);
+              *reinterpret_cast<uint4*>(half[q >> 1] + 16 * (q & 1)) = make_uint4(x[0], x[1], x[2], x[3]);
             }
           }
         }

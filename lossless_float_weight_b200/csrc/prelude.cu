@@ -62,6 +62,37 @@ __device__ void tile_offsets(const Geo& g, const Ws& ws, uint32_t c, const uint3
   }
 }
 
+// Byte plane s of chunk c (all threads of the block): ZERO when every byte is 0; else
+// ZRUN when its payload (the block bitmap, then the bytes of the blocks that hold a
+// non-zero byte) is strictly smaller than RAW; else RAW. kept = 32 x marked blocks, less
+// what the chunk's short last block lacks when it is marked.
+template <int DT>
+__device__ void decide_byte_plane(const Geo& g, const Ws& ws, uint32_t c, int s, uint32_t* red) {
+  constexpr int NS = n_streams(DT);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t k = c * NS + s;
+  const uint64_t m = min64(g.m0, g.n - (uint64_t)c * g.m0);
+  const uint32_t* map = ws.zmap + ((uint64_t)c * n_byte_planes(DT) + (s - 1)) * g.zwords;
+  uint32_t cnt = 0;
+  for (uint32_t w = tid; w < g.zwords; w += blockDim.x) cnt += __popc(__ldcg(map + w));
+  cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
+  if (lane == 0) red[warp] = cnt;
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t marked = 0;
+    for (uint32_t i = 0; i < blockDim.x / 32; i++) marked += red[i];
+    const uint64_t last = (m - 1) / kZBlock;
+    uint64_t kept = (uint64_t)marked * kZBlock;
+    if ((m % kZBlock) && ((__ldcg(map + last / 32) >> (last % 32)) & 1u)) kept -= kZBlock - m % kZBlock;
+    const uint64_t raw = raw_payload(m, 8), zrun = zrun_payload(m, kept);
+    const bool zero = __ldcg(ws.nonzero + k) == 0;
+    ws.emode[k] = zero ? kModeZero : zrun < raw ? kModeZrun : kModeRaw;
+    ws.ecode[k] = kNoCode;
+    ws.esize[k] = zero ? 0 : zrun < raw ? zrun : raw;
+  }
+  __syncthreads();
+}
+
 // Per (chunk, entropy stream), one block of kHuffWarps warps: ZERO when every symbol is
 // 0, else the code choice of decide_code.
 template <int DT>
@@ -134,10 +165,38 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
           if (NE > 1) atomicAdd(col1 + symbol<DT, NV>(raw, 1, i) * 32, 1u);
         }
       }
+      if constexpr (DT == kFP32) {
+        // every stream is a bit field of the value, so the OR of the words holds the OR of
+        // each stream's symbols: of my 64 values for the all-zero flags, and of each half
+        // (zero-run blocks v0 / 32 and v0 / 32 + 1, an even pair) for the fraction planes
+        static_assert(NV == 2 * kZBlock, "a thread's values are two zero-run blocks");
+        RawValues<DT, NV> o;
+        uint32_t a = 0, b = 0;
 #pragma unroll
-      for (int i = 0; i < NV; i++)
+        for (int i = 0; i < NV / 2; i++) {
+          a |= raw.w[i];
+          b |= raw.w[NV / 2 + i];
+        }
+        o.w[0] = a;
+        o.w[1] = b;
+        o.w[2] = a | b;
 #pragma unroll
-        for (int s = 0; s < NS; s++) nz[s] |= symbol<DT, NV>(raw, s, i);
+        for (int s = 0; s < NS; s++) nz[s] |= symbol<DT, NV>(o, s, 2);
+        if (ws.zmap) {
+          const uint32_t blk = v0 / kZBlock;
+#pragma unroll
+          for (int s = 1; s < NS; s++) {
+            const uint32_t bits = (symbol<DT, NV>(o, s, 0) ? 1u : 0u) | (symbol<DT, NV>(o, s, 1) ? 2u : 0u);
+            if (bits)
+              atomicOr(ws.zmap + ((uint64_t)c * n_byte_planes(DT) + (s - 1)) * g.zwords + blk / 32, bits << (blk % 32));
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < NV; i++)
+#pragma unroll
+          for (int s = 0; s < NS; s++) nz[s] |= symbol<DT, NV>(raw, s, i);
+      }
     }
   }
 #pragma unroll
@@ -169,6 +228,9 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
     build_chunk_table<DT>(g, ws, plan, c, (uint32_t)e, hs);
     __syncthreads();
   }
+#pragma unroll
+  for (int s = 0; s < NS; s++)
+    if (is_byte_plane(DT, s)) decide_byte_plane<DT>(g, ws, c, s, hs.red32);
 }
 
 // ---------------------------------------------------------------- BF16 histogram
@@ -233,6 +295,7 @@ __global__ void __launch_bounds__(kHistThreads) k_split_hist_bf16(const uint8_t*
     for (int s = 0; s < kHbStages; s++) issue(s);
 
   uint8_t* const colb = reinterpret_cast<uint8_t*>(sh + lane);
+  const int warp = tid >> 5;
   uint32_t q = 0;  // pieces consumed
   for (uint32_t tile = blockIdx.x; tile < g.n_tiles; tile += gridDim.x) {
     uint64_t vlo;
@@ -248,6 +311,7 @@ __global__ void __launch_bounds__(kHistThreads) k_split_hist_bf16(const uint8_t*
 #pragma unroll
       for (int k = 0; k < (int)(kHbPieceValues / 8 / kHistThreads); k++) {
         const uint32_t i = (uint32_t)(k * kHistThreads + tid);
+        uint32_t sfnz = 0;  // sign/fraction bits of my 8 values
         if (i * 8 < nb) {
           const uint4 v = st4[i];
           const uint32_t x[4] = {v.x, v.y, v.z, v.w};
@@ -258,17 +322,36 @@ __global__ void __launch_bounds__(kHistThreads) k_split_hist_bf16(const uint8_t*
             atomicAdd(reinterpret_cast<uint32_t*>(colb + (x[j] & 0x7F80u)), 1u);
             atomicAdd(reinterpret_cast<uint32_t*>(colb + ((x[j] >> 16) & 0x7F80u)), 1u);
             nz0 |= x[j] & 0x7F807F80u;
-            nz1 |= x[j] & 0x807F807Fu;
+            sfnz |= x[j] & 0x807F807Fu;
+          }
+          nz1 |= sfnz;
+        }
+        if (ws.zmap) {
+          // zero-run blocks: the warp's 32 units of 8 values are 8 blocks of 32 values
+          // (four units each), blocks 8w + 64k on from the piece's first block
+          const uint32_t b = __ballot_sync(0xFFFFFFFFu, sfnz != 0);
+          if (lane == 0 && b) {
+            uint32_t m8 = 0;
+#pragma unroll
+            for (int j = 0; j < 8; j++) m8 |= ((b >> (4 * j)) & 0xFu) ? 1u << j : 0u;
+            const uint32_t blk = (sl * kHistSlice + p0) / kZBlock + (uint32_t)(64 * k + 8 * warp);
+            atomicOr(ws.zmap + (uint64_t)c * g.zwords + blk / 32, m8 << (blk % 32));
           }
         }
       }
       if (tid == 0 && nb < pv) {
         const uint16_t* t = reinterpret_cast<const uint16_t*>(src) + vlo + p0 + nb;
+        uint32_t sfnz = 0;
         for (uint32_t i = 0; i < pv - nb; i++) {
           const uint32_t v = t[i];
           atomicAdd(reinterpret_cast<uint32_t*>(colb + (v & 0x7F80u)), 1u);
           nz0 |= v & 0x7F80u;
-          nz1 |= v & 0x807Fu;
+          sfnz |= v & 0x807Fu;
+        }
+        nz1 |= sfnz;
+        if (ws.zmap && sfnz) {  // the tail (under 8 values) lies in one block
+          const uint32_t blk = (sl * kHistSlice + p0 + nb) / kZBlock;
+          atomicOr(ws.zmap + (uint64_t)c * g.zwords + blk / 32, 1u << (blk % 32));
         }
       }
       __syncthreads();  // stage s is read, and the tile's counts are complete after the last piece
@@ -308,6 +391,9 @@ __global__ void __launch_bounds__(kHuffWarps * 32, 4) k_build_chunks(Geo g, Ws w
     build_chunk_table<DT>(g, ws, plan, blockIdx.x, (uint32_t)e, hs);
     __syncthreads();
   }
+#pragma unroll
+  for (int s = 0; s < n_streams(DT); s++)
+    if (is_byte_plane(DT, s)) decide_byte_plane<DT>(g, ws, blockIdx.x, s, hs.red32);
 }
 
 // Stand-alone code lengths for `count` histograms (u64 x 256 each); also used by the
@@ -372,7 +458,7 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout(Geo g, Ws ws, PlanDev
     code[i] = kNoCode;
     if (k < g.n_entries) {
       const uint32_t s = k % NS;
-      if (is_entropy(DT, (int)s)) {
+      if (is_entropy(DT, (int)s) || is_byte_plane(DT, (int)s)) {
         mode[i] = ws.emode[k];
         code[i] = ws.ecode[k];
         size[i] = ws.esize[k];

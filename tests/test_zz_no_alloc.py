@@ -1,7 +1,9 @@
 """zipnn_compress_noalloc: the compress entry point for callers that cannot allocate
-device memory (for example code running under CUDA stream capture, where cudaMalloc is
-not allowed). It must produce exactly the container zipnn_compress produces, call after
-call, although its fixed scratch array keeps whatever the previous call left there.
+device memory (code whose device memory belongs to a framework's caching allocator it
+cannot reach from C, or a latency-critical path that cannot afford the synchronisation
+of a cudaMalloc/cudaFree pair). It must produce exactly the container zipnn_compress
+produces, call after call, although its fixed scratch array keeps whatever the previous
+call left there.
 Collected last on purpose: a failure here leaves every other test already run."""
 import ctypes
 
