@@ -451,3 +451,52 @@ def test_argument_errors(z):
     with pytest.raises(z.ZipnnError) as ei:
         z.compress_into(x, out, ws, subblock=24)
     assert ei.value.status == z.ERR_INVALID_ARG
+
+
+def _pruned_bf16(rows, cols, seed, every=3):
+    g = torch.Generator().manual_seed(seed)
+    x = (torch.randn(rows, cols, generator=g) * 0.02).to(torch.bfloat16)
+    x[torch.arange(rows) % every == 0] = 0  # pruned rows: runs of zero sign/fraction bytes
+    return x.reshape(-1)
+
+
+@pytest.mark.parametrize("chunk_bytes,subblock", [(262144, 512), (4096, 64), (1 << 20, 512), (65536, 16)])
+def test_zero_runs_bf16(z, orc, chunk_bytes, subblock):
+    """Pruned rows make ZRUN sign/fraction planes; 1 MiB chunks (16384 blocks) take the
+    generic decode instead of the staged one. Ragged sizes end in a short block."""
+    import container_util as CU
+    for n_extra in (0, 77):
+        x = torch.cat([_pruned_bf16(600, 1000, chunk_bytes), (torch.randn(n_extra) * 0.02).to(torch.bfloat16)])
+        got = _check_roundtrip(z, orc, x, "bf16 pruned", chunk_bytes=chunk_bytes, subblock=subblock)
+        h, mode, code, off, ends = CU.payload_spans(got)
+        assert 3 in mode[1::2].tolist()
+
+
+def test_zero_runs_fp32(z, orc):
+    g = torch.Generator().manual_seed(21)
+    y = (torch.randn(1 << 20, generator=g) * 0.02).float()
+    clean = (torch.arange(1 << 20) // 96) % 3 == 0  # runs of clean values, not aligned to blocks
+    y[clean] = y[clean].bfloat16().float()
+    y[5000:9000] = 0
+    got = _check_roundtrip(z, orc, y, "fp32 partly clean")
+    import container_util as CU
+    h, mode, code, off, ends = CU.payload_spans(got)
+    assert 3 in mode.reshape(-1, 4)[:, 2].tolist() and 3 in mode.reshape(-1, 4)[:, 3].tolist()
+
+
+def test_zero_runs_corrupt(z, orc):
+    """A ZRUN bitmap that marks every block asks for more kept bytes than the payload holds:
+    CORRUPT on the staged and on the generic path, never a fault."""
+    import container_util as CU
+    for cb in (262144, 1 << 20):
+        x = _pruned_bf16(300, 1000, 5, every=2)
+        c = z.compress(x.cuda(), chunk_bytes=cb).cpu().numpy()
+        h, mode, code, off, ends = CU.payload_spans(c)
+        k = [i for i in range(1, len(mode), 2) if mode[i] == 3][0]
+        d = c.copy()
+        d[off[k]: off[k] + 16] = 0xFF
+        ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+        out = torch.empty(x.numel(), dtype=torch.bfloat16, device="cuda")
+        z.decompress_into(torch.from_numpy(d).cuda(), d.size, out, ws, chunk_bytes=cb)
+        assert z.status(ws) == z.ERR_CORRUPT
+        assert orc.decompress_status("bf16", d, x.numel(), chunk_bytes=cb) == orc.ECORRUPT
