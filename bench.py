@@ -772,6 +772,14 @@ def run_single(args):
     c_ms = timed(lambda: Z.compress_into(x, out, ws, CHUNK, plan=plan, stream=stream))
     cbytes = Z.compressed_size(out)
     d_ms = timed(lambda: Z.decompress_into(out, cbytes, y, ws, CHUNK, stream=stream))
+    # per-kernel device time of one compress and one decompress (events around each launch)
+    Z.zipnn_timing_enable(1)
+    Z.kernel_times()
+    Z.compress_into(x, out, ws, CHUNK, plan=plan, stream=stream)
+    Z.decompress_into(out, cbytes, y, ws, CHUNK, stream=stream)
+    torch.cuda.synchronize()
+    ktimes = {k: round(v[0], 4) for k, v in Z.kernel_times().items() if v[1]}
+    Z.zipnn_timing_enable(0)
     ok = torch.equal(y.view(torch.uint8), x.view(torch.uint8)) and Z.status(ws) == Z.OK
     peak, peak_src = measured_peaks()
     algo = nbytes + cbytes
@@ -784,6 +792,7 @@ def run_single(args):
         "compression_ratio": round(cbytes / nbytes, 5), "bytes": nbytes, "values": n,
         "peak": peak, "peak_source": peak_src, "steps": args.steps, "warmup": args.warmup,
         "plan_setup_ms": None if setup_ms is None else round(setup_ms, 2), "roundtrip_ok": bool(ok),
+        "kernel_ms": ktimes,
     }
     print(json.dumps(line), flush=True)
 
