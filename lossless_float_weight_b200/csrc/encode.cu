@@ -193,6 +193,37 @@ __global__ void __launch_bounds__(kEncodeThreads) k_encode(const uint8_t* __rest
       continue;
     }
     if (s >= NB) continue;  // unreachable: only streams < NB can be bit-packed
+    if (mode == kModeRaw) {
+      // a RAW stream of w < 8 bits a symbol: value v starts at bit v * w of the payload,
+      // and my 64 values fill 2w whole words from word v0 * w / 32, so I pack them in
+      // registers and store the words myself (no scan, no staging, no shared edge words).
+      // The last value's word ends in zero bits; the chunk's last tile zeroes the words
+      // after it up to the payload's 16-byte padding.
+      static_assert(kEncValues * 1 % 32 == 0, "64 values of any width are whole words");
+      uint32_t* words = reinterpret_cast<uint32_t*>(out + sm.off[s]);
+      const uint32_t wbase = (uint32_t)((uint64_t)v0 * w / 32);
+      if (cnt > 0) {
+        uint64_t acc = 0;
+        uint32_t nfill = 0, nw = 0;
+#pragma unroll
+        for (int i = 0; i < kEncValues; i++) {
+          if (i < cnt) {
+            acc = (acc << w) | symbol<DT, kEncValues>(raw, s, i);
+            nfill += (uint32_t)w;
+            if (nfill >= 32) {
+              nfill -= 32;
+              words[wbase + nw++] = bswap32((uint32_t)(acc >> nfill));
+            }
+          }
+        }
+        if (nfill) words[wbase + nw] = bswap32((uint32_t)(acc << (32 - nfill)));
+      }
+      if (last) {
+        const uint64_t used = ceil_div((uint64_t)m * w, 32), padded = raw_payload(m, w) / 4;
+        for (uint64_t i = used + tid; i < padded; i += kEncodeThreads) words[i] = 0;
+      }
+      continue;
+    }
     const bool huff = mode == kModeHuff;
     const uint32_t* enc = sm.enc[s < NE ? s : 0];
     // pack my codes, most significant bit first, into my private words from bit 0

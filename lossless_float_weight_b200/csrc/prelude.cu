@@ -136,11 +136,14 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
                                                              Ws ws, PlanDev plan, int build) {
   constexpr int NS = n_streams(DT), NE = n_entropy(DT);
   constexpr int A0 = alphabet(DT, 0), A1 = NE > 1 ? alphabet(DT, 1) : 0;
+  // counters: one per (bin, lane); FP8 and FP4 count the joint (exponent, mantissa) bin,
+  // exponent * A1 + mantissa, so one shared atomic counts both entropy streams
+  constexpr int AJ = NE > 1 ? A0 * A1 : A0;
   extern __shared__ __align__(16) uint8_t smem_raw[];  // histogram columns, then the code builder
   uint32_t* sh = reinterpret_cast<uint32_t*>(smem_raw);
   __shared__ int s_last;
   const int tid = threadIdx.x, lane = tid & 31;
-  for (int i = tid; i < (A0 + A1) * 32; i += kHistThreads) sh[i] = 0;
+  for (int i = tid; i < AJ * 32; i += kHistThreads) sh[i] = 0;
   __syncthreads();
   const uint32_t c = blockIdx.x / slices, sl = blockIdx.x % slices;
   const uint64_t clo = (uint64_t)c * g.m0;
@@ -150,7 +153,6 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
 #pragma unroll
   for (int s = 0; s < NS; s++) nz[s] = 0;
   uint32_t* col0 = sh + lane;
-  uint32_t* col1 = sh + A0 * 32 + lane;
   constexpr int NV = 64;  // consecutive values per thread per pass, loaded up front
   for (uint32_t t0 = lo; t0 < hi; t0 += kHistThreads * NV) {
     const uint32_t v0 = t0 + tid * NV;
@@ -161,8 +163,9 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
 #pragma unroll
       for (int i = 0; i < NV; i++) {
         if (i < cnt) {
-          atomicAdd(col0 + symbol<DT, NV>(raw, 0, i) * 32, 1u);
-          if (NE > 1) atomicAdd(col1 + symbol<DT, NV>(raw, 1, i) * 32, 1u);
+          const uint32_t bin = NE > 1 ? symbol<DT, NV>(raw, 0, i) * A1 + symbol<DT, NV>(raw, 1, i)
+                                      : symbol<DT, NV>(raw, 0, i);
+          atomicAdd(col0 + bin * 32, 1u);
         }
       }
       if constexpr (DT == kFP32) {
@@ -206,12 +209,32 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
   }
   __syncthreads();
   // column sums: thread b reads its row starting at lane b, so a warp hits 32 banks
-  for (int b = tid; b < A0 + A1; b += kHistThreads) {
-    uint32_t sum = 0;
+  if constexpr (NE == 1) {
+    for (int b = tid; b < A0; b += kHistThreads) {
+      uint32_t sum = 0;
 #pragma unroll 8
-    for (int l = 0; l < 32; l++) sum += sh[b * 32 + ((l + b) & 31)];
-    const int e = b < A0 ? 0 : 1, sym = b < A0 ? b : b - A0;
-    if (sum) atomicAdd(&hist[((uint64_t)c * NE + e) * 256 + sym], sum);
+      for (int l = 0; l < 32; l++) sum += sh[b * 32 + ((l + b) & 31)];
+      if (sum) atomicAdd(&hist[(uint64_t)c * 256 + b], sum);
+    }
+  } else {
+    // joint bins, then each stream's counts as sums over the other stream's symbols
+    uint32_t* joint = sh + AJ * 32;
+    for (int b = tid; b < AJ; b += kHistThreads) {
+      uint32_t sum = 0;
+#pragma unroll 8
+      for (int l = 0; l < 32; l++) sum += sh[b * 32 + ((l + b) & 31)];
+      joint[b] = sum;
+    }
+    __syncthreads();
+    for (int t = tid; t < A0 + A1; t += kHistThreads) {
+      uint32_t sum = 0;
+      if (t < A0) {
+        for (int j = 0; j < A1; j++) sum += joint[t * A1 + j];
+      } else {
+        for (int e = 0; e < A0; e++) sum += joint[e * A1 + (t - A0)];
+      }
+      if (sum) atomicAdd(&hist[((uint64_t)c * NE + (t < A0 ? 0 : 1)) * 256 + (t < A0 ? t : t - A0)], sum);
+    }
   }
   if (!build) return;
   // the last block to finish a chunk builds that chunk's codes (its histogram is then
@@ -594,7 +617,8 @@ static cudaError_t split_hist_t(const void* src, const Geo& g, uint32_t* hist, u
   const uint64_t blocks = (uint64_t)g.n_chunks * slices;
   if (blocks > 0x7FFFFFFFull) return cudaErrorInvalidConfiguration;
   constexpr int NE = n_entropy(DT);
-  constexpr size_t cols = (size_t)(alphabet(DT, 0) + (NE > 1 ? alphabet(DT, 1) : 0)) * 32 * 4;
+  constexpr size_t AJ = NE > 1 ? (size_t)alphabet(DT, 0) * alphabet(DT, 1) : (size_t)alphabet(DT, 0);
+  constexpr size_t cols = (AJ * 32 + (NE > 1 ? AJ : 0)) * 4;  // counters (+ the joint sums)
   const size_t smem = ws ? (sizeof(HuffBlockSmem) > cols ? sizeof(HuffBlockSmem) : cols) : cols;
   const cudaError_t e = allow_smem(k_split_hist<DT>, sizeof(HuffBlockSmem) > cols ? sizeof(HuffBlockSmem) : cols, 4 + DT);
   if (e != cudaSuccess) return e;
