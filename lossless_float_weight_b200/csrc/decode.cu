@@ -131,86 +131,97 @@ __device__ __forceinline__ uint32_t zrun_rank(const uint8_t* map, uint32_t b0) {
   return r;
 }
 
-// Decode GV consecutive symbols of one stream (GV a multiple of 2; n <= GV valid).
-template <int GV, bool FULL>
-__device__ __forceinline__ void next_symbols(StreamState& st, uint32_t (&o)[GV], int n, uint32_t v) {
+// The symbols of one stream for GV consecutive values (GV a multiple of 2; n <= GV
+// valid), packed into one register: symbol i at bits SB * i (SB = 4 for FP8 and FP4,
+// whose symbols have at most 4 bits; 8 otherwise). v: the group's first value in the
+// sub-block.
+template <int GV, int SB, bool FULL>
+__device__ __forceinline__ uint64_t next_packed(StreamState& st, int n, uint32_t v) {
+  static_assert(GV * SB <= 64, "a group's symbols fit one register");
+  uint64_t o = 0;
   switch (st.kind) {
     case kKHuff:
 #pragma unroll
       for (int i = 0; i < GV; i += 2) {
         st.br.refill();
-        if (FULL || i < n) o[i] = st.br.huff(st.lut, st.acc);
-        else o[i] = 0;
-        if (FULL || i + 1 < n) o[i + 1] = st.br.huff(st.lut, st.acc);
-        else o[i + 1] = 0;
+        uint32_t a, b;
+        if (FULL) {  // two symbols a lookup when the 12-bit window holds both codes
+          const uint32_t p = huff_pair(st.br, st.lut, st.acc);
+          a = (p >> 16) & 0xFFu;
+          b = p >> 24;
+        } else {
+          a = i < n ? st.br.huff(st.lut, st.acc) : 0u;
+          b = i + 1 < n ? st.br.huff(st.lut, st.acc) : 0u;
+        }
+        o |= (uint64_t)(a | (b << SB)) << (SB * i);
       }
       break;
     case kKBits:
 #pragma unroll
       for (int i = 0; i < GV; i += 2) {
         st.br.refill();
-        o[i] = (FULL || i < n) ? st.br.fixed(st.width) : 0u;
-        o[i + 1] = (FULL || i + 1 < n) ? st.br.fixed(st.width) : 0u;
+        const uint32_t a = (FULL || i < n) ? st.br.fixed(st.width) : 0u;
+        const uint32_t b = (FULL || i + 1 < n) ? st.br.fixed(st.width) : 0u;
+        o |= (uint64_t)(a | (b << SB)) << (SB * i);
       }
       break;
     case kKBytes:
-      if (FULL) {
-        if constexpr (GV == 16) {
-          const uint4 q = __ldg(reinterpret_cast<const uint4*>(st.bytes + v));
-          const uint32_t x[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-          for (int i = 0; i < 16; i++) o[i] = (x[i >> 2] >> (8 * (i & 3))) & 0xFFu;
-        } else if constexpr (GV == 8) {
-          const uint2 q = __ldg(reinterpret_cast<const uint2*>(st.bytes + v));
-#pragma unroll
-          for (int i = 0; i < 8; i++) o[i] = ((i < 4 ? q.x : q.y) >> (8 * (i & 3))) & 0xFFu;
-        } else {
-          const uint32_t q = __ldg(reinterpret_cast<const uint32_t*>(st.bytes + v));
-#pragma unroll
-          for (int i = 0; i < GV; i++) o[i] = (q >> (8 * i)) & 0xFFu;
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < GV; i++) o[i] = i < n ? (uint32_t)st.bytes[v + i] : 0u;
-      }
-      break;
-    case kKZrun: {
-      // zero runs: a group of GV values (GV divides 32) lies in one block; a block's
-      // bytes are kept when its bitmap bit is set, at 32 x (marked blocks before it)
-      const uint32_t vv = st.zbase + v;
-      if (v == 0 || (vv & 31u) == 0) {
-        if (v != 0) st.zrank += st.zmarked;
-        st.zmarked = ((uint32_t)st.zmap[vv >> 8] >> (7 - ((vv >> 5) & 7u))) & 1u;
-      }
-      const uint64_t at = (uint64_t)st.zrank * kZBlock + (vv & 31u);
-      if (st.zmarked && at + GV <= st.zlimit) {
-        const uint8_t* src = st.bytes + at;
+      if constexpr (SB == 8) {
         if (FULL) {
           if constexpr (GV == 8) {
-            const uint2 q = __ldg(reinterpret_cast<const uint2*>(src));
-#pragma unroll
-            for (int i = 0; i < 8; i++) o[i] = ((i < 4 ? q.x : q.y) >> (8 * (i & 3))) & 0xFFu;
+            const uint2 q = __ldg(reinterpret_cast<const uint2*>(st.bytes + v));
+            o = q.x | ((uint64_t)q.y << 32);
           } else {
-#pragma unroll
-            for (int i = 0; i < GV; i++) o[i] = src[i];
+            o = __ldg(reinterpret_cast<const uint32_t*>(st.bytes + v));
           }
         } else {
 #pragma unroll
-          for (int i = 0; i < GV; i++) o[i] = i < n ? (uint32_t)src[i] : 0u;
+          for (int i = 0; i < GV; i++)
+            if (i < n) o |= (uint64_t)st.bytes[v + i] << (8 * i);
         }
-      } else {
-        if (st.zmarked) st.zbad = 1;  // kept bytes past the payload: corrupt
-#pragma unroll
-        for (int i = 0; i < GV; i++) o[i] = 0;
       }
       break;
-    }
-    default:
+    case kKZrun:
+      if constexpr (SB == 8) {
+        // zero runs: a group (GV divides 32) lies in one block; a block's bytes are kept
+        // when its bitmap bit is set, at 32 x (marked blocks before it)
+        const uint32_t vv = st.zbase + v;
+        if (v == 0 || (vv & 31u) == 0) {
+          if (v != 0) st.zrank += st.zmarked;
+          st.zmarked = ((uint32_t)st.zmap[vv >> 8] >> (7 - ((vv >> 5) & 7u))) & 1u;
+        }
+        const uint64_t at = (uint64_t)st.zrank * kZBlock + (vv & 31u);
+        if (st.zmarked && at + GV <= st.zlimit) {
+          const uint8_t* src = st.bytes + at;
+          if (FULL) {
+            if constexpr (GV == 8) {
+              const uint2 q = __ldg(reinterpret_cast<const uint2*>(src));
+              o = q.x | ((uint64_t)q.y << 32);
+            } else {
+              o = __ldg(reinterpret_cast<const uint32_t*>(src));
+            }
+          } else {
 #pragma unroll
-      for (int i = 0; i < GV; i++) o[i] = 0;
+            for (int i = 0; i < GV; i++)
+              if (i < n) o |= (uint64_t)src[i] << (8 * i);
+          }
+        } else if (st.zmarked) {
+          st.zbad = 1;  // kept bytes past the payload: corrupt
+        }
+      }
+      break;
+    default:
+      break;
   }
+  return o;
 }
 
+// FP8: eight 4-bit symbols (nibble i of x) as eight bytes, in two words.
+__device__ __forceinline__ void nibbles_to_bytes(uint32_t x, uint32_t& w0, uint32_t& w1) {
+  const uint32_t lo = x & 0x0F0F0F0Fu, hi = (x >> 4) & 0x0F0F0F0Fu;  // nibbles 0,2,4,6 / 1,3,5,7
+  w0 = __byte_perm(lo, hi, 0x5140);
+  w1 = __byte_perm(lo, hi, 0x7362);
+}
 
 // Two BF16 words (the merge) from two sign/fraction bytes, bytes 2*sf_hi and 2*sf_hi + 1
 // of sf, and two exponents, bytes 2*ex_hi and 2*ex_hi + 1 of ex. Each sign/fraction byte
@@ -661,59 +672,70 @@ __device__ __noinline__ void decode_generic(const uint8_t* __restrict__ in, cons
       }
     }
     uint8_t* dst = out + value_offset(DT, clo + sb_lo);
+    constexpr int SB = DT == kFP8 || DT == kFP4 ? 4 : 8;
     const uint32_t full = count / GV;
     for (uint32_t gi = 0; gi < full; gi++) {
-      uint32_t sy[NS][GV];
+      uint64_t P[NS];
 #pragma unroll
-      for (int s = 0; s < NS; s++) next_symbols<GV, true>(st[s], sy[s], GV, gi * GV);
-      if constexpr (DT == kFP4) {  // two values a byte, the first in the low nibble
-        uint32_t wv[2];
+      for (int s = 0; s < NS; s++) P[s] = next_packed<GV, SB, true>(st[s], GV, gi * GV);
+      if constexpr (DT == kFP4) {
+        // nibble i is value i (value 2i is the low nibble of byte i): sign << 3 |
+        // exponent << 1 | mantissa, lane by lane
+        const uint64_t v = (P[2] << 3) | (P[0] << 1) | P[1];
+        *reinterpret_cast<uint2*>(dst + (uint64_t)gi * 8) = make_uint2((uint32_t)v, (uint32_t)(v >> 32));
+      } else if constexpr (DT == kFP8) {
+        // byte i: sign << 7 | exponent << 3 | mantissa
+        uint32_t wv[4];
 #pragma unroll
-        for (int q = 0; q < 2; q++) {
-          uint32_t x = 0;
-#pragma unroll
-          for (int b = 0; b < 8; b++) x |= merge_value<DT>(sy[0][8 * q + b], sy[1][8 * q + b], sy[2][8 * q + b], 0) << (4 * b);
-          wv[q] = x;
+        for (int h = 0; h < 2; h++) {
+          uint32_t e0, e1, m0, m1, s0, s1;
+          nibbles_to_bytes((uint32_t)(P[0] >> (32 * h)), e0, e1);
+          nibbles_to_bytes((uint32_t)(P[1] >> (32 * h)), m0, m1);
+          nibbles_to_bytes((uint32_t)(P[2] >> (32 * h)), s0, s1);
+          wv[2 * h] = (s0 << 7) | (e0 << 3) | m0;
+          wv[2 * h + 1] = (s1 << 7) | (e1 << 3) | m1;
         }
-        *reinterpret_cast<uint2*>(dst + (uint64_t)gi * 8) = make_uint2(wv[0], wv[1]);
+        *reinterpret_cast<uint4*>(dst + (uint64_t)gi * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+      } else if constexpr (DT == kBF16) {
+        uint32_t wv[4];
+#pragma unroll
+        for (int q = 0; q < 4; q++)
+          wv[q] = bf16_merge_pair((uint32_t)(P[1] >> (32 * (q >> 1))), q & 1, (uint32_t)(P[0] >> (32 * (q >> 1))), q & 1);
+        *reinterpret_cast<uint4*>(dst + (uint64_t)gi * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
       } else {
         uint32_t wv[4];
 #pragma unroll
-        for (int q = 0; q < 4; q++) {
-          if constexpr (DT == kBF16) {
-            wv[q] = merge_value<DT>(sy[0][2 * q], sy[1][2 * q], 0, 0) |
-                    (merge_value<DT>(sy[0][2 * q + 1], sy[1][2 * q + 1], 0, 0) << 16);
-          } else if constexpr (DT == kFP32) {
-            wv[q] = merge_value<DT>(sy[0][q], sy[1][q], sy[2][q], sy[3][q]);
-          } else {
-            uint32_t x = 0;
-#pragma unroll
-            for (int b = 0; b < 4; b++) x |= merge_value<DT>(sy[0][4 * q + b], sy[1][4 * q + b], sy[2][4 * q + b], 0) << (8 * b);
-            wv[q] = x;
-          }
-        }
+        for (int q = 0; q < 4; q++)
+          wv[q] = merge_value<DT>((uint32_t)(P[0] >> (8 * q)) & 0xFFu, (uint32_t)(P[1] >> (8 * q)) & 0xFFu,
+                                  (uint32_t)(P[NS > 2 ? 2 : 0] >> (8 * q)) & 0xFFu,
+                                  (uint32_t)(P[NS > 3 ? 3 : 0] >> (8 * q)) & 0xFFu);
         *reinterpret_cast<uint4*>(dst + (uint64_t)gi * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
       }
     }
     const uint32_t rem = count - full * GV;
     if (rem) {
-      uint32_t sy[NS][GV];
+      uint64_t P[NS];
 #pragma unroll
-      for (int s = 0; s < NS; s++) next_symbols<GV, false>(st[s], sy[s], (int)rem, full * GV);
+      for (int s = 0; s < NS; s++) P[s] = next_packed<GV, SB, false>(st[s], (int)rem, full * GV);
+      constexpr uint32_t mask = (1u << SB) - 1u;
       if constexpr (DT == kFP4) {  // rem is even: values come in byte pairs
 #pragma unroll
         for (uint32_t i = 0; i < (uint32_t)GV; i += 2) {
           if (i >= rem) break;
-          const uint32_t lo = merge_value<DT>(sy[0][i], sy[1][i], sy[2][i], 0);
-          const uint32_t hi = merge_value<DT>(sy[0][i + 1], sy[1][i + 1], sy[2][i + 1], 0);
+          const uint32_t lo = merge_value<DT>((uint32_t)(P[0] >> (SB * i)) & mask, (uint32_t)(P[1] >> (SB * i)) & mask,
+                                              (uint32_t)(P[2] >> (SB * i)) & mask, 0);
+          const uint32_t hi = merge_value<DT>((uint32_t)(P[0] >> (SB * (i + 1))) & mask,
+                                              (uint32_t)(P[1] >> (SB * (i + 1))) & mask,
+                                              (uint32_t)(P[2] >> (SB * (i + 1))) & mask, 0);
           dst[(full * GV + i) / 2] = (uint8_t)(lo | (hi << 4));
         }
       } else {
 #pragma unroll
         for (uint32_t i = 0; i < (uint32_t)GV; i++) {
           if (i >= rem) break;
-          const uint32_t v = merge_value<DT>(sy[0][i], sy[1][i], NS > 2 ? sy[NS > 2 ? 2 : 0][i] : 0,
-                                             NS > 3 ? sy[NS > 3 ? 3 : 0][i] : 0);
+          const uint32_t v = merge_value<DT>((uint32_t)(P[0] >> (SB * i)) & mask, (uint32_t)(P[1] >> (SB * i)) & mask,
+                                             NS > 2 ? (uint32_t)(P[NS > 2 ? 2 : 0] >> (SB * i)) & mask : 0u,
+                                             NS > 3 ? (uint32_t)(P[NS > 3 ? 3 : 0] >> (SB * i)) & mask : 0u);
           uint8_t* p = dst + (uint64_t)(full * GV + i) * VB;
           if constexpr (VB == 2) *reinterpret_cast<uint16_t*>(p) = (uint16_t)v;
           else if constexpr (VB == 4) *reinterpret_cast<uint32_t*>(p) = v;
@@ -1012,23 +1034,28 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
     else fill_lut<false>(sm.lut[e], sm.sorted[e], sm.slen[e], sm.limit[e], sm.first[e], sm.offset[e]);
   }
   __syncthreads();
-  if constexpr (DT == kBF16) {
-    // second code of each window: the entry of the window shifted by the first length
-    // decides it when that code ends inside the 12 known bits (a prefix code's entry
-    // does not depend on the bits after the code). Updating in place is safe: the
-    // fields read here (first length, first symbol, invalid flag) never change.
-    if (sm.mode[0] == kModeHuff && !wide) {
+  // second code of each window: the entry of the window shifted by the first length
+  // decides it when that code ends inside the 12 known bits (a prefix code's entry does
+  // not depend on the bits after the code). Updating in place is safe: the fields read
+  // here (first length, first symbol, invalid flag) never change. Every two-symbol table
+  // (not the wide window's single-symbol one).
+  if (!wide) {
+    bool any = false;
+#pragma unroll
+    for (int e = 0; e < NE; e++) {
+      if (sm.mode[e] != kModeHuff) continue;
+      any = true;
       for (uint32_t x = tid; x < 4096; x += kDecodeThreads) {
-        const uint32_t e0 = sm.lut[0][x];
+        const uint32_t e0 = sm.lut[e][x];
         if (e0 & kLutInvalid) continue;
         const uint32_t l0 = e0 & 15u;
-        const uint32_t e1 = sm.lut[0][(x << l0) & 4095u];
+        const uint32_t e1 = sm.lut[e][(x << l0) & 4095u];
         const uint32_t l1 = e1 & 15u;
         if (!(e1 & kLutInvalid) && l0 + l1 <= (uint32_t)kLmax)
-          sm.lut[0][x] = e0 | ((l0 + l1) << 4) | ((e1 & 0x00FF0000u) << 8);
+          sm.lut[e][x] = e0 | ((l0 + l1) << 4) | ((e1 & 0x00FF0000u) << 8);
       }
-      __syncthreads();
     }
+    if (any) __syncthreads();
   }
 
   if constexpr (DT == kBF16) {
