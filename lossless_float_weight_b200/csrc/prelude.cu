@@ -195,10 +195,18 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
           }
         }
       } else {
+        // FP8 and FP4: the same bit-field argument; the OR of the words folded onto its
+        // first value (byte 0 for FP8, nibble 0 for FP4) holds the OR of every value's bits
+        uint32_t x = 0;
 #pragma unroll
-        for (int i = 0; i < NV; i++)
+        for (int i = 0; i < RawValues<DT, NV>::kWords; i++) x |= raw.w[i];
+        x |= x >> 16;
+        x |= x >> 8;
+        if constexpr (DT == kFP4) x |= x >> 4;
+        RawValues<DT, NV> o;
+        o.w[0] = x;
 #pragma unroll
-          for (int s = 0; s < NS; s++) nz[s] |= symbol<DT, NV>(raw, s, i);
+        for (int s = 0; s < NS; s++) nz[s] |= symbol<DT, NV>(o, s, 0);
       }
     }
   }
