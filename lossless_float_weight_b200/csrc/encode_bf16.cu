@@ -58,6 +58,16 @@ __device__ __forceinline__ uint32_t bf16_pair_plane(uint32_t w, int s) {
   return s == 0 ? (w >> 7) & 0x00FF00FFu : (w & 0x007F007Fu) | ((w >> 8) & 0x00800080u);
 }
 
+// The plane bytes of the four BF16 values in words a and b, in value order. Sign/fraction
+// (s == 1): the values' low bytes (fraction bits 6..0 under exponent bit 0) and high bytes
+// (the sign over exponent bits 7..1), gathered by two byte permutes, then the sign bits
+// taken from the high bytes and the rest from the low bytes (one bit select).
+__device__ __forceinline__ uint32_t bf16_quad_plane(uint32_t a, uint32_t b, int s) {
+  if (s == 0) return __byte_perm(bf16_pair_plane(a, 0), bf16_pair_plane(b, 0), 0x6420);
+  const uint32_t lo = __byte_perm(a, b, 0x6420), hi = __byte_perm(a, b, 0x7531);
+  return (lo & 0x7F7F7F7Fu) | (hi & 0x80808080u);
+}
+
 __global__ void __launch_bounds__(kBThreads, 8) k_encode_bf16(const uint8_t* __restrict__ src, Geo g, Ws ws,
                                                                    uint8_t* __restrict__ out) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -153,9 +163,7 @@ __global__ void __launch_bounds__(kBThreads, 8) k_encode_bf16(const uint8_t* __r
           for (int q = 0; q < kBValues / 16; q++) {
             uint32_t x[4];
 #pragma unroll
-            for (int k = 0; k < 4; k++)
-              x[k] = __byte_perm(bf16_pair_plane(raw.w[8 * q + 2 * k], s),
-                                 bf16_pair_plane(raw.w[8 * q + 2 * k + 1], s), 0x6420);
+            for (int k = 0; k < 4; k++) x[k] = bf16_quad_plane(raw.w[8 * q + 2 * k], raw.w[8 * q + 2 * k + 1], s);
             if (half[q >> 1]) *reinterpret_cast<uint4*>(half[q >> 1] + 16 * (q & 1)) = make_uint4(x[0], x[1], x[2], x[3]);
           }
         } else {
