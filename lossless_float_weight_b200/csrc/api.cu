@@ -64,7 +64,7 @@ bool make_geo(int dt, uint64_t n, uint32_t chunk_bytes, uint32_t S, uint32_t G, 
 }
 
 struct WsPlan {
-  uint64_t status, hist, nonzero, zmap, scan_desc, tile_desc, slot, zero_end;
+  uint64_t status, hist, nonzero, zmap, zcount, scan_desc, tile_desc, slot, zero_end;
   uint64_t esize, emode, ecode, eoff, enc, tile_hist, tile_off;
   uint64_t km_mu, km_perm, km_assign, km_changed, km_gsum, total;
   bool tile_counts;  // per-tile exponent histograms (BF16)
@@ -80,6 +80,7 @@ WsPlan ws_plan(const Geo& g) {
   p.hist = o;       o = align_up(o + C * NE * 256 * 4);
   p.nonzero = o;    o = align_up(o + K * 4);
   p.zmap = o;       o = align_up(o + C * (uint64_t)n_byte_planes(g.dt) * g.zwords * 4);
+  p.zcount = o;     o = align_up(o + C * (uint64_t)n_byte_planes(g.dt) * 4);
   p.scan_desc = o;  o = align_up(o + (uint64_t)layout_tiles(g.n_entries) * 8);
   p.tile_desc = o;  o = align_up(o + NE * g.n_tiles * 8);
   p.slot = o;       o = align_up(o + NE * g.n_tiles * 8);
@@ -108,6 +109,7 @@ Ws carve(const WsPlan& p, void* base) {
   w.hist = reinterpret_cast<uint32_t*>(b + p.hist);
   w.nonzero = reinterpret_cast<uint32_t*>(b + p.nonzero);
   w.zmap = n_byte_planes(p.dt) ? reinterpret_cast<uint32_t*>(b + p.zmap) : nullptr;
+  w.zcount = n_byte_planes(p.dt) ? reinterpret_cast<uint32_t*>(b + p.zcount) : nullptr;
   w.scan_desc = reinterpret_cast<uint64_t*>(b + p.scan_desc);
   w.tile_desc = reinterpret_cast<uint64_t*>(b + p.tile_desc);
   w.slot = reinterpret_cast<uint64_t*>(b + p.slot);

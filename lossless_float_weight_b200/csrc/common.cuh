@@ -102,6 +102,7 @@ struct Ws {
   uint32_t* nonzero;    // [n_entries]: OR of the stream's symbols
   uint32_t* zmap;       // [n_chunks][n_byte_planes][zwords]: bit i of word w set when block
                         // 32w + i of the plane holds a non-zero byte
+  uint32_t* zcount;     // [n_chunks][n_byte_planes]: blocks set in zmap
   uint64_t* scan_desc;  // [layout tiles] look-back descriptors
   uint64_t* tile_desc;  // [n_tiles][n_entropy] look-back descriptors
   uint64_t* slot;       // [n_tiles][n_entropy] shared boundary words

@@ -62,35 +62,26 @@ __device__ void tile_offsets(const Geo& g, const Ws& ws, uint32_t c, const uint3
   }
 }
 
-// Byte plane s of chunk c (all threads of the block): ZERO when every byte is 0; else
-// ZRUN when its payload (the block bitmap, then the bytes of the blocks that hold a
-// non-zero byte) is strictly smaller than RAW; else RAW. kept = 32 x marked blocks, less
-// what the chunk's short last block lacks when it is marked.
+// Byte plane s of chunk c (thread 0): ZERO when every byte is 0; else ZRUN when its
+// payload (the block bitmap, then the bytes of the blocks that hold a non-zero byte) is
+// strictly smaller than RAW; else RAW. kept = 32 x marked blocks (counted by the
+// histogram pass), less what the chunk's short last block lacks when it is marked.
 template <int DT>
-__device__ void decide_byte_plane(const Geo& g, const Ws& ws, uint32_t c, int s, uint32_t* red) {
+__device__ void decide_byte_plane(const Geo& g, const Ws& ws, uint32_t c, int s) {
   constexpr int NS = n_streams(DT);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (threadIdx.x != 0) return;
   const uint32_t k = c * NS + s;
   const uint64_t m = min64(g.m0, g.n - (uint64_t)c * g.m0);
-  const uint32_t* map = ws.zmap + ((uint64_t)c * n_byte_planes(DT) + (s - 1)) * g.zwords;
-  uint32_t cnt = 0;
-  for (uint32_t w = tid; w < g.zwords; w += blockDim.x) cnt += __popc(__ldcg(map + w));
-  cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
-  if (lane == 0) red[warp] = cnt;
-  __syncthreads();
-  if (tid == 0) {
-    uint32_t marked = 0;
-    for (uint32_t i = 0; i < blockDim.x / 32; i++) marked += red[i];
-    const uint64_t last = (m - 1) / kZBlock;
-    uint64_t kept = (uint64_t)marked * kZBlock;
-    if ((m % kZBlock) && ((__ldcg(map + last / 32) >> (last % 32)) & 1u)) kept -= kZBlock - m % kZBlock;
-    const uint64_t raw = raw_payload(m, 8), zrun = zrun_payload(m, kept);
-    const bool zero = __ldcg(ws.nonzero + k) == 0;
-    ws.emode[k] = zero ? kModeZero : zrun < raw ? kModeZrun : kModeRaw;
-    ws.ecode[k] = kNoCode;
-    ws.esize[k] = zero ? 0 : zrun < raw ? zrun : raw;
-  }
-  __syncthreads();
+  const uint64_t plane = (uint64_t)c * n_byte_planes(DT) + (s - 1);
+  const uint32_t* map = ws.zmap + plane * g.zwords;
+  const uint64_t last = (m - 1) / kZBlock;
+  uint64_t kept = (uint64_t)__ldcg(ws.zcount + plane) * kZBlock;
+  if ((m % kZBlock) && ((__ldcg(map + last / 32) >> (last % 32)) & 1u)) kept -= kZBlock - m % kZBlock;
+  const uint64_t raw = raw_payload(m, 8), zrun = zrun_payload(m, kept);
+  const bool zero = __ldcg(ws.nonzero + k) == 0;
+  ws.emode[k] = zero ? kModeZero : zrun < raw ? kModeZrun : kModeRaw;
+  ws.ecode[k] = kNoCode;
+  ws.esize[k] = zero ? 0 : zrun < raw ? zrun : raw;
 }
 
 // Per (chunk, entropy stream), one block of kHuffWarps warps: ZERO when every symbol is
@@ -190,8 +181,8 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
 #pragma unroll
           for (int s = 1; s < NS; s++) {
             const uint32_t bits = (symbol<DT, NV>(o, s, 0) ? 1u : 0u) | (symbol<DT, NV>(o, s, 1) ? 2u : 0u);
-            if (bits)
-              atomicOr(ws.zmap + ((uint64_t)c * n_byte_planes(DT) + (s - 1)) * g.zwords + blk / 32, bits << (blk % 32));
+            const uint64_t plane = (uint64_t)c * n_byte_planes(DT) + (s - 1);
+            if (bits) atomicOr(ws.zmap + plane * g.zwords + blk / 32, bits << (blk % 32));
           }
         }
       } else {
@@ -215,6 +206,7 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
     const uint32_t v = __reduce_or_sync(0xFFFFFFFFu, nz[s]);
     if (nonzero && lane == 0 && v) atomicOr(&nonzero[(uint64_t)c * NS + s], v);
   }
+
   __syncthreads();
   // column sums: thread b reads its row starting at lane b, so a warp hits 32 banks
   if constexpr (NE == 1) {
@@ -260,8 +252,23 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
     __syncthreads();
   }
 #pragma unroll
-  for (int s = 0; s < NS; s++)
-    if (is_byte_plane(DT, s)) decide_byte_plane<DT>(g, ws, c, s, hs.red32);
+  for (int s = 0; s < NS; s++) {
+    if (!is_byte_plane(DT, s)) continue;
+    // the plane's marked blocks: every block's bit is final (this is the chunk's last block)
+    const uint64_t plane = (uint64_t)c * n_byte_planes(DT) + (s - 1);
+    uint32_t cnt = 0;
+    for (uint32_t w = tid; w < g.zwords; w += kHistThreads) cnt += __popc(__ldcg(ws.zmap + plane * g.zwords + w));
+    cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
+    if (lane == 0) hs.red32[tid >> 5] = cnt;
+    __syncthreads();
+    if (tid == 0) {
+      uint32_t t = 0;
+      for (int i = 0; i < kHistThreads / 32; i++) t += hs.red32[i];
+      ws.zcount[plane] = t;
+      decide_byte_plane<DT>(g, ws, c, s);
+    }
+    __syncthreads();
+  }
 }
 
 // ---------------------------------------------------------------- BF16 histogram
@@ -279,7 +286,8 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
 constexpr int kHbStages = 4;
 constexpr uint32_t kHbPieceValues = 8192;  // 16 KB
 constexpr size_t kHbRegion = 256 * 32 * 4;  // the counters
-constexpr size_t kHbSmemBytes = kHbRegion + (size_t)kHbStages * kHbPieceValues * 2 + kHbStages * 8;
+constexpr size_t kHbZbits = 32 * 4;         // the tile's zero-run bitmap: 1024 blocks
+constexpr size_t kHbSmemBytes = kHbRegion + (size_t)kHbStages * kHbPieceValues * 2 + kHbStages * 8 + kHbZbits;
 constexpr uint32_t kHbWaitLimit = 1u << 26;
 
 // Values of tile `tile` (0 past the end of a ragged last chunk) and its first value.
@@ -298,9 +306,11 @@ __global__ void __launch_bounds__(kHistThreads) k_split_hist_bf16(const uint8_t*
   uint32_t* const sh = reinterpret_cast<uint32_t*>(smem_raw);
   uint8_t* const stages = smem_raw + kHbRegion;
   uint64_t* const bar = reinterpret_cast<uint64_t*>(stages + (size_t)kHbStages * kHbPieceValues * 2);
+  uint32_t* const zbits = reinterpret_cast<uint32_t*>(bar + kHbStages);
   const int tid = threadIdx.x, lane = tid & 31;
   const uint32_t T = g.tiles_per_chunk;
   for (int i = tid; i < 256 * 32; i += kHistThreads) sh[i] = 0;
+  if (tid < 32) zbits[tid] = 0;
   if (tid == 0)
     for (int s = 0; s < kHbStages; s++) mbar_init(bar + s, 1);
   __syncthreads();
@@ -339,6 +349,7 @@ __global__ void __launch_bounds__(kHistThreads) k_split_hist_bf16(const uint8_t*
       if (!mbar_wait_bounded(bar + s, (q / kHbStages) & 1u, kHbWaitLimit) && ws.status) set_status(ws.status, kStTimeout);
       const uint32_t pv = min32(kHbPieceValues, nv - p0), nb = pv & ~7u;
       const uint4* st4 = reinterpret_cast<const uint4*>(stages + (size_t)s * kHbPieceValues * 2);
+      uint32_t my4 = 0;  // bit k: my unit of iteration k holds a non-zero sign/fraction byte
 #pragma unroll
       for (int k = 0; k < (int)(kHbPieceValues / 8 / kHistThreads); k++) {
         const uint32_t i = (uint32_t)(k * kHistThreads + tid);
@@ -357,17 +368,23 @@ __global__ void __launch_bounds__(kHistThreads) k_split_hist_bf16(const uint8_t*
           }
           nz1 |= sfnz;
         }
-        if (ws.zmap) {
-          // zero-run blocks: the warp's 32 units of 8 values are 8 blocks of 32 values
-          // (four units each), blocks 8w + 64k on from the piece's first block
-          const uint32_t b = __ballot_sync(0xFFFFFFFFu, sfnz != 0);
-          if (lane == 0 && b) {
-            uint32_t m8 = 0;
+        my4 |= (sfnz != 0 ? 1u : 0u) << k;
+      }
+      if (ws.zmap) {
+        // zero-run blocks: in iteration k the warp's 32 units of 8 values are the tile's 8
+        // blocks 8w + 64k + piece offset; four units make a block. Ballot, then fold each
+        // nibble of the ballot onto one bit and gather the 8 bits (no branch per lane).
 #pragma unroll
-            for (int j = 0; j < 8; j++) m8 |= ((b >> (4 * j)) & 0xFu) ? 1u << j : 0u;
-            const uint32_t blk = (sl * kHistSlice + p0) / kZBlock + (uint32_t)(64 * k + 8 * warp);
-            atomicOr(ws.zmap + (uint64_t)c * g.zwords + blk / 32, m8 << (blk % 32));
-          }
+        for (int k = 0; k < (int)(kHbPieceValues / 8 / kHistThreads); k++) {
+          uint32_t b = __ballot_sync(0xFFFFFFFFu, (my4 >> k) & 1u);
+          b |= b >> 1;
+          b |= b >> 2;
+          b &= 0x11111111u;  // bit 4j: block j of the eight
+          b = (b | (b >> 3)) & 0x03030303u;
+          b = (b | (b >> 6)) & 0x000F000Fu;
+          b = (b | (b >> 12)) & 0xFFu;
+          const uint32_t blk = p0 / kZBlock + (uint32_t)(64 * k + 8 * warp);  // within the tile
+          if (lane == k && b) atomicOr(zbits + blk / 32, b << (blk % 32));
         }
       }
       if (tid == 0 && nb < pv) {
@@ -381,8 +398,8 @@ __global__ void __launch_bounds__(kHistThreads) k_split_hist_bf16(const uint8_t*
         }
         nz1 |= sfnz;
         if (ws.zmap && sfnz) {  // the tail (under 8 values) lies in one block
-          const uint32_t blk = (sl * kHistSlice + p0 + nb) / kZBlock;
-          atomicOr(ws.zmap + (uint64_t)c * g.zwords + blk / 32, 1u << (blk % 32));
+          const uint32_t blk = (p0 + nb) / kZBlock;
+          atomicOr(zbits + blk / 32, 1u << (blk % 32));
         }
       }
       __syncthreads();  // stage s is read, and the tile's counts are complete after the last piece
@@ -407,7 +424,16 @@ __global__ void __launch_bounds__(kHistThreads) k_split_hist_bf16(const uint8_t*
       if (sum) atomicAdd(&hist[(uint64_t)c * 256 + b], sum);
       if (ws.tile_hist) ws.tile_hist[((uint64_t)c * T + sl) * 256 + b] = (uint16_t)sum;
     }
-    __syncthreads();  // every row is clear before the next tile's counts
+    if (ws.zmap && tid < 32) {
+      // the tile's 32 bitmap words (complete since the last piece's barrier) go out as
+      // plain stores, their marked blocks into the chunk's count; then cleared
+      const uint32_t word = zbits[tid], wi = sl * 32u + (uint32_t)tid;
+      if (wi < g.zwords) ws.zmap[(uint64_t)c * g.zwords + wi] = word;
+      const uint32_t marked = __reduce_add_sync(0xFFFFFFFFu, __popc(word));
+      if (tid == 0 && marked) atomicAdd(ws.zcount + c, marked);
+      zbits[tid] = 0;
+    }
+    __syncthreads();  // every row and bitmap word is clear before the next tile's counts
   }
 }
 
@@ -424,7 +450,7 @@ __global__ void __launch_bounds__(kHuffWarps * 32, 4) k_build_chunks(Geo g, Ws w
   }
 #pragma unroll
   for (int s = 0; s < n_streams(DT); s++)
-    if (is_byte_plane(DT, s)) decide_byte_plane<DT>(g, ws, blockIdx.x, s, hs.red32);
+    if (is_byte_plane(DT, s)) decide_byte_plane<DT>(g, ws, blockIdx.x, s);
 }
 
 // Stand-alone code lengths for `count` histograms (u64 x 256 each); also used by the

@@ -60,7 +60,7 @@ CASES = [
     ("bf16", 2048 * 3, 8, 4096),        # more ranks than chunks
     ("fp32", 65536 * 3 + 17, 2, 262144),
     ("fp8_e4m3", 1 << 20, 3, 65536),
-    ("fp4_e2m1", (1 << 20) + 2, 2, 65536),
+    ("fp4_e2m1", (1 << 20) + 4, 2, 65536),
     ("bf16", 300001, 1, 262144),
 ]
 
