@@ -384,7 +384,10 @@ __device__ __forceinline__ uint32_t ex_word(uint32_t row, uint32_t k) {
 // ZRUN: the sign/fraction plane has zero runs; smp is its kept bytes, zmap / zpre the
 // chunk's block bitmap words (bit i of word w: block 32w + i) and the marked blocks before
 // each word, in shared memory.
-template <bool WIDE, bool ZRUN, class Lut>
+// ALLFULL: every sub-block of the chunk holds S values, S is a multiple of the round and
+// the sub-blocks fill whole batches, so every round decodes 32 exponents a thread and every
+// merge unit holds 8 values (the case of every chunk of a weight checkpoint).
+template <bool WIDE, bool ZRUN, bool ALLFULL, class Lut>
 __device__ int decode_bf16_staged(StagedSmem& st, const Lut* lut, const uint32_t* tail,
                                   const uint32_t* __restrict__ idx, uint32_t bs_words,
                                   const uint8_t* __restrict__ smp, uint32_t m, uint32_t S, uint32_t nsub,
@@ -397,7 +400,7 @@ __device__ int decode_bf16_staged(StagedSmem& st, const Lut* lut, const uint32_t
   uint8_t* exb = reinterpret_cast<uint8_t*>(st.ex);
   for (uint32_t batch = 0; batch < nsub; batch += kDecodeThreads) {
     const uint32_t j = batch + tid;
-    const uint32_t count = j < nsub ? min32(S, m - j * S) : 0;
+    const uint32_t count = ALLFULL ? S : j < nsub ? min32(S, m - j * S) : 0;
     SmemBitReader<WIDE> br;
     uint32_t acc = 0;
     uint64_t expect = 0;
@@ -429,7 +432,7 @@ __device__ int decode_bf16_staged(StagedSmem& st, const Lut* lut, const uint32_t
 #pragma unroll
       for (int p = 0; p < 4; p++) {
         const uint32_t off = r * kRound;
-        const uint32_t n = off < urem[p] ? min32(8, urem[p] - off) : 0;
+        const uint32_t n = ALLFULL ? 8u : off < urem[p] ? min32(8, urem[p] - off) : 0;
         uval[p] = ubase[p] + off;
         ucnt[p] = n;
         smv[p] = make_uint2(0, 0);
@@ -454,8 +457,8 @@ __device__ int decode_bf16_staged(StagedSmem& st, const Lut* lut, const uint32_t
       }
       // decode up to 32 exponents of my sub-block, two per lookup
       const uint32_t base = r * kRound;
-      if (base < count) {
-        if (base + kRound <= count) {
+      if (ALLFULL || base < count) {
+        if (ALLFULL || base + kRound <= count) {
 #pragma unroll
           for (int k = 0; k < kRowWords; k++) {
             if constexpr (WIDE) {
@@ -486,7 +489,7 @@ __device__ int decode_bf16_staged(StagedSmem& st, const Lut* lut, const uint32_t
 #pragma unroll
       for (int p = 0; p < 4; p++) {
         const uint32_t u = tid + p * kDecodeThreads;
-        if (!ucnt[p]) continue;
+        if (!ALLFULL && !ucnt[p]) continue;
         const uint32_t row = u >> 2, part = u & 3;
         const uint32_t es[2] = {st.ex[ex_word(row, 2 * part)], st.ex[ex_word(row, 2 * part + 1)]};
         const uint32_t xs[2] = {smv[p].x, smv[p].y};
@@ -494,7 +497,7 @@ __device__ int decode_bf16_staged(StagedSmem& st, const Lut* lut, const uint32_t
 #pragma unroll
         for (int q = 0; q < 4; q++) o[q] = bf16_merge_pair(xs[q >> 1], q & 1, es[q >> 1], q & 1);
         uint8_t* d = outc + (uint64_t)uval[p] * 2;
-        if (ucnt[p] == 8) {
+        if (ALLFULL || ucnt[p] == 8) {
           *reinterpret_cast<uint4*>(d) = make_uint4(o[0], o[1], o[2], o[3]);
         } else {
 #pragma unroll
@@ -1077,19 +1080,23 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
       const uint8_t* smp = sm.mode[1] == kModeRaw    ? in + sm.off[1]
                            : sm.mode[1] == kModeZrun ? in + sm.off[1] + zrun_map_bytes(m)
                                                      : nullptr;
+      const bool allfull = (uint64_t)m == nsub * S && S % kRound == 0 && nsub % kDecodeThreads == 0;
       int bad;
-      if (sm.mode[1] == kModeZrun)
-        bad = wide ? decode_bf16_staged<true, true>(stg, lut16, sm.lut[0], idx, bs_words, smp, m, S, (uint32_t)nsub,
-                                                    out + clo * VB, idx_start, idx_next, sm.zmap, sm.zpre)
-                   : decode_bf16_staged<false, true>(stg, sm.lut[0], nullptr, idx, bs_words, smp, m, S,
-                                                     (uint32_t)nsub, out + clo * VB, idx_start, idx_next, sm.zmap,
-                                                     sm.zpre);
-      else
-        bad = wide ? decode_bf16_staged<true, false>(stg, lut16, sm.lut[0], idx, bs_words, smp, m, S, (uint32_t)nsub,
-                                                     out + clo * VB, idx_start, idx_next, nullptr, nullptr)
-                   : decode_bf16_staged<false, false>(stg, sm.lut[0], nullptr, idx, bs_words, smp, m, S,
-                                                      (uint32_t)nsub, out + clo * VB, idx_start, idx_next, nullptr,
-                                                      nullptr);
+#define ZIPNN_STAGED(W, Z, F, L, T, ZM, ZP) \
+  decode_bf16_staged<W, Z, F>(stg, L, T, idx, bs_words, smp, m, S, (uint32_t)nsub, out + clo * VB, idx_start, \
+                              idx_next, ZM, ZP)
+      if (sm.mode[1] == kModeZrun) {
+        if (wide) bad = allfull ? ZIPNN_STAGED(true, true, true, lut16, sm.lut[0], sm.zmap, sm.zpre)
+                                : ZIPNN_STAGED(true, true, false, lut16, sm.lut[0], sm.zmap, sm.zpre);
+        else bad = allfull ? ZIPNN_STAGED(false, true, true, sm.lut[0], nullptr, sm.zmap, sm.zpre)
+                           : ZIPNN_STAGED(false, true, false, sm.lut[0], nullptr, sm.zmap, sm.zpre);
+      } else {
+        if (wide) bad = allfull ? ZIPNN_STAGED(true, false, true, lut16, sm.lut[0], nullptr, nullptr)
+                                : ZIPNN_STAGED(true, false, false, lut16, sm.lut[0], nullptr, nullptr);
+        else bad = allfull ? ZIPNN_STAGED(false, false, true, sm.lut[0], nullptr, nullptr, nullptr)
+                           : ZIPNN_STAGED(false, false, false, sm.lut[0], nullptr, nullptr, nullptr);
+      }
+#undef ZIPNN_STAGED
       if (bad) set_status(status, kStCorrupt);
       return;
     }
