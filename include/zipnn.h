@@ -6,8 +6,9 @@
  *  - "ZipNN: Lossless Compression for AI Models" (abstract) and the THEORY-599 note
  *    on it, "Per-field compressibility (Table II)": every value is split into its
  *    exponent field and its sign/fraction bytes; the exponent field is entropy-coded,
- *    the sign/fraction bytes are stored as they are ("raw"), or omitted when a chunk of
- *    them is all zero (the "clean" models of the same table).
+ *    the sign/fraction bytes are stored as they are ("raw"), omitted when a chunk of them
+ *    is all zero (the "clean" models of the same table), or stored without their runs of
+ *    zero bytes (ZRUN).
  *  - THEORY-599, "Order-0 only (section III-A b)": one order-0 symbol histogram and one
  *    Huffman code per chunk; no context model.
  *  - "Lossless Compression of Neural Network Components: Weights, Checkpoints, and K/V
@@ -23,7 +24,7 @@
  *     u64 n | u32 chunk_bytes | u32 S | u32 n_chunks | u32 n_shared | u64 off_codes |
  *     u64 off_payload | u64 total_bytes | u8 L_MAX=12 | u8 n_groups | 6 zero bytes
  *   chunk table at 64: one 16-byte entry per (chunk c, stream s), index k = c*n_streams+s:
- *     u8 mode (0 RAW, 1 ZERO, 2 HUFF) | 3 zero bytes | u32 code | u64 payload offset.
+ *     u8 mode (0 RAW, 1 ZERO, 2 HUFF, 3 ZRUN) | 3 zero bytes | u32 code | u64 payload offset.
  *     code is the shared record index for a HUFF entry coded with a plan's code, and
  *     0xFFFFFFFF otherwise.
  *   shared code records at off_codes (n_shared = n_groups * entropy streams), record
@@ -34,6 +35,9 @@
  *     ZERO: nothing (every symbol of that chunk and stream is 0).
  *     HUFF: [local code record if code == 0xFFFFFFFF] [u32 idx[ceil(m/S)], padded]
  *           [bitstream, padded]; idx[j] is the bit offset of symbol j*S.
+ *     ZRUN: zero runs of a byte plane: the chunk's symbols in blocks of 32 (the last may
+ *           be shorter); [one bit per block, most significant first, 1 when the block
+ *           holds a non-zero byte, padded] [the bytes of the marked blocks, padded].
  *   Streams: BF16 [exponent, sign+fraction byte]; FP32 [exponent, sign + fraction
  *   bits 22..16, fraction bits 15..8, fraction bits 7..0]; FP8 E4M3 [exponent (4 bits),
  *   mantissa (3 bits), sign (1 bit)]; FP4 E2M1 [exponent (2 bits), mantissa (1 bit),
@@ -42,7 +46,9 @@
  *   (sign bit 3, exponent bits 2..1, mantissa bit 0); n counts values and is even.
  *   Codes are canonical (RFC 1951 rule), at most 12 bits long.
  *   A stream is ZERO when all its symbols in the chunk are 0; an entropy stream is HUFF
- *   when that payload is strictly smaller than RAW, else RAW.
+ *   when that payload is strictly smaller than RAW, else RAW; a byte plane (BF16's
+ *   sign+fraction byte, FP32's three fraction planes) is ZRUN when that payload is
+ *   strictly smaller than RAW, else RAW; the 1-bit sign streams of FP8 and FP4 are RAW.
  *
  * Conventions for every call:
  *  - n (values) is at most 2^56 - 1, and a tensor has at most 2^31 - 1 chunk entries.
