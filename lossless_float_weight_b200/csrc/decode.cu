@@ -346,11 +346,13 @@ struct SmemBitReader {
     refill();
   }
   __device__ __forceinline__ void refill() {
-    if (nb <= 32) {
-      buf |= (uint64_t)q << (32 - nb);
-      nb += 32;
-      q = ld(pos++);
-    }
+    const bool r = nb <= 32;
+    const uint64_t add = (uint64_t)q << ((32 - nb) & 63);
+    const uint32_t nq = ld(pos);
+    buf |= r ? add : 0ull;
+    q = r ? nq : q;
+    pos += r ? 1u : 0u;
+    nb += r ? 32 : 0;
   }
   __device__ __forceinline__ uint32_t huff(const uint32_t* lut, uint32_t& acc) {
     const uint32_t e = lut[buf >> 52];
@@ -541,41 +543,45 @@ struct DecodeSmem {
 // three BF16 decode blocks share an SM: 228 KB of shared memory, 1 KB reserved per block
 static_assert(sizeof(StagedSmem) + sizeof(DecodeSmem<kBF16>) + 1024 <= 233472 / 3, "BF16 decode: 3 blocks per SM");
 
-// Fill the decode table of one HUFF stream from its canonical tables, 16 consecutive
-// entries per thread. Canonical codes left-aligned to 12 bits tile [0, limit[12]) in
-// canonical order: code k covers 2^(12 - len_k) entries and the next code starts where
-// it ends. A thread finds the code of its first entry from the length limits, then
-// walks on. Entries from limit[12] on match no code (only when the Kraft sum is below 1).
+// Fill the decode table of one HUFF stream from its canonical tables. Canonical codes
+// left-aligned to 12 bits tile [0, limit[12]) in canonical order: code k covers
+// 2^(12 - len_k) entries and the next code starts where it ends. Warp w fills entries
+// [512w, 512w + 512), lane l the entries 512w + l + 32j (so each store of a warp covers 32
+// consecutive entries, one per bank): the lane finds the code of its first entry from the
+// length limits, then walks forward over the codes that end before its next entry.
+// Entries from limit[12] on match no code (only when the Kraft sum is below 1).
 // WIDE: u16 entries symbol << 4 | length (the single-symbol table); else u32 entries
 // symbol << 16 | length.
 template <bool WIDE>
 __device__ __forceinline__ void fill_lut(void* lut, const uint8_t* sorted, const uint8_t* slen,
                                          const uint32_t* limit, const uint32_t* first, const uint32_t* offset) {
-  const uint32_t x0 = threadIdx.x * 16u, lim = limit[kLmax];
+  const uint32_t x0 = (threadIdx.x >> 5) * 512u + (threadIdx.x & 31u), lim = limit[kLmax];
   uint32_t l = 1;
   while (l < (uint32_t)kLmax && x0 >= limit[l]) l++;
-  uint32_t k = 0, end = 0, e = 0;
+  uint32_t k = 0, end = 0;
   if (x0 < lim) {
     const uint32_t c = x0 >> (kLmax - l);
     k = offset[l] + c - first[l];
     end = (c + 1) << (kLmax - l);
-    e = WIDE ? ((uint32_t)sorted[k] << 4) | l : ((uint32_t)sorted[k] << 16) | l;
   }
-#pragma unroll
-  for (uint32_t i = 0; i < 16; i++) {
-    const uint32_t x = x0 + i;
-    if (x < lim && x == end) {
-      k++;
-      const uint32_t lk = slen[k];
-      end += 1u << (kLmax - lk);
-      e = WIDE ? ((uint32_t)sorted[k] << 4) | lk : ((uint32_t)sorted[k] << 16) | lk;
+#pragma unroll 4
+  for (uint32_t j = 0; j < 16; j++) {
+    const uint32_t x = x0 + 32u * j;
+    uint32_t e = kLutInvalid | 1u;
+    if (x < lim) {
+      while (x >= end) {  // codes that end before x (each ends inside [0, lim))
+        k++;
+        l = slen[k];
+        end += 1u << (kLmax - l);
+      }
+      e = WIDE ? ((uint32_t)sorted[k] << 4) | l : ((uint32_t)sorted[k] << 16) | l;
     }
-    if constexpr (WIDE) static_cast<uint16_t*>(lut)[x] = (uint16_t)(x < lim ? e : (kLutInvalid | 1u));
-    else static_cast<uint32_t*>(lut)[x] = x < lim ? e : (kLutInvalid | 1u);
+    if constexpr (WIDE) static_cast<uint16_t*>(lut)[x] = (uint16_t)e;
+    else static_cast<uint32_t*>(lut)[x] = e;
   }
 }
 
-static_assert(kDecodeThreads * 16 == 4096, "fill_lut: 16 table entries per thread");
+static_assert(kDecodeThreads * 16 == 4096, "fill_lut: 8 warps of 512 table entries");
 
 
 constexpr uint32_t kZStagedWords = 128;  // zero-run bitmap words the staged path holds: 4096 blocks
@@ -585,9 +591,9 @@ static_assert(kDecodeThreads >= kZStagedWords, "one thread per bitmap word");
 // exponent stream, a bitstream over 56 KB, or a ZRUN plane of more than 4096 blocks): one
 // sub-block per thread per pass, every stream read through its own reader. All threads.
 template <int DT>
-__device__ __noinline__ void decode_generic(const uint8_t* __restrict__ in, const DecodeSmem<DT>& sm, uint32_t m,
-                                            uint32_t S, uint64_t nsub, uint64_t clo, uint8_t* __restrict__ out,
-                                            uint32_t* status) {
+__device__ __forceinline__ void decode_generic(const uint8_t* __restrict__ in, const DecodeSmem<DT>& sm, uint32_t m,
+                                               uint32_t S, uint64_t nsub, uint64_t clo, uint8_t* __restrict__ out,
+                                               uint32_t* status) {
   constexpr int NS = n_streams(DT), NE = n_entropy(DT), VB = value_bytes(DT);
   constexpr int GV = DT == kBF16 ? 8 : DT == kFP32 ? 4 : 16;  // values per store (16 bytes; FP4 8)
   const int tid = threadIdx.x;
@@ -756,6 +762,13 @@ __device__ __noinline__ void decode_generic(const uint8_t* __restrict__ in, cons
     }
     if (bad) set_status(status, kStCorrupt);
   }
+}
+
+template <int DT>
+__device__ __noinline__ void decode_generic_apart(const uint8_t* __restrict__ in, const DecodeSmem<DT>& sm, uint32_t m,
+                                                  uint32_t S, uint64_t nsub, uint64_t clo, uint8_t* __restrict__ out,
+                                                  uint32_t* status) {
+  decode_generic<DT>(in, sm, m, S, nsub, clo, out, status);
 }
 
 // Chunk c of the container `in` (in_bytes readable) of a tensor with geometry g, into
@@ -1101,13 +1114,20 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
       return;
     }
   }
-  // the other cases: one sub-block per thread per pass, in a function of its own so that
-  // its register needs do not weigh on the staged path above
-  decode_generic<DT>(in, sm, m, S, nsub, clo, out, status);
+  // the other cases: one sub-block per thread per pass. For BF16 (a rare fallback) in a
+  // function of its own, so that its register needs do not weigh on the staged path
+  // above; the other types have no staged path and keep it inline (their table reads stay
+  // shared-memory loads)
+  if constexpr (DT == kBF16) decode_generic_apart<DT>(in, sm, m, S, nsub, clo, out, status);
+  else decode_generic<DT>(in, sm, m, S, nsub, clo, out, status);
 }
 
+// Blocks per SM the decode kernels are built for: three (24 warps) where the registers
+// allow it without spilling; FP32's four readers need two.
+constexpr int decode_blocks_per_sm(int dt) { return dt == kFP32 ? 2 : 3; }
+
 template <int DT>
-__global__ void __launch_bounds__(kDecodeThreads, DT == kBF16 ? 3 : 1)
+__global__ void __launch_bounds__(kDecodeThreads, decode_blocks_per_sm(DT))
     k_decode(const uint8_t* __restrict__ in, uint64_t in_bytes, Geo g, uint8_t* __restrict__ out, uint32_t* status) {
   decode_chunk<DT>(in, in_bytes, g, blockIdx.x, out, status);
 }
@@ -1131,7 +1151,7 @@ __device__ __forceinline__ uint32_t find_item(const DecodeItem* __restrict__ ite
 
 // Many tensors in one launch: block b decodes global chunk b.
 template <int DT>
-__global__ void __launch_bounds__(kDecodeThreads, DT == kBF16 ? 3 : 1)
+__global__ void __launch_bounds__(kDecodeThreads, decode_blocks_per_sm(DT))
     k_decode_batch(const DecodeItem* __restrict__ items, uint32_t count, Geo g, uint32_t* status) {
   __shared__ uint32_t s_item;
   if (threadIdx.x < 32) {

@@ -269,21 +269,27 @@ __global__ void __launch_bounds__(kBThreads, 8) k_encode_bf16(const uint8_t* __r
       }
       if (mybits) {
         const uint32_t q0 = (uint32_t)(P & 31) + myoff;
-        const uint32_t sh = q0 & 31, d0 = q0 >> 5, dlast = (q0 + mybits - 1) >> 5;
-        uint32_t prev = 0;
-        for (uint32_t k = 0; k <= dlast - d0; k++) {
-          const uint32_t cur = k < nw ? pw[k] : 0u;
-          const uint32_t o = (sh ? prev << (32 - sh) : 0u) | (cur >> sh);
-          if (k == 0 || k == dlast - d0) atomicOr(sm.stage + d0 + k, o);
-          else sm.stage[d0 + k] = o;
-          prev = cur;
+        const uint32_t sh = q0 & 31, d0 = q0 >> 5, nk = ((q0 + mybits - 1) >> 5) - d0 + 1;
+        uint32_t cur = pw[0];
+        atomicOr(sm.stage + d0, __funnelshift_r(cur, 0u, sh));
+        for (uint32_t k = 1; k + 1 < nk; k++) {
+          const uint32_t prev = cur;
+          cur = pw[k];
+          sm.stage[d0 + k] = __funnelshift_r(cur, prev, sh);
         }
+        if (nk > 1) atomicOr(sm.stage + d0 + nk - 1, __funnelshift_r(nk - 1 < nw ? pw[nk - 1] : 0u, cur, sh));
       }
       __syncthreads();
       const uint64_t end = P + pass_bits;
       const uint32_t nwt = (uint32_t)(((P & 31) + pass_bits + 31) >> 5);
       const uint64_t W0 = P >> 5;
-      for (uint32_t i = tid; i < nwt; i += kBThreads) {
+      for (uint32_t i = 1 + tid; i + 1 < nwt; i += kBThreads) {  // middle words: plain
+        const uint32_t word = sm.stage[i];
+        sm.stage[i] = 0;
+        bs[W0 + i] = bswap32(word);
+      }
+      if (tid < 2 && nwt > 0 && (tid == 0 || nwt > 1)) {  // edge words: thread 0 the first, 1 the last
+        const uint32_t i = tid == 0 ? 0u : nwt - 1;
         uint32_t word = sm.stage[i];
         sm.stage[i] = 0;
         // the previous pass's last bits; a pass reads one carry slot and writes the other,

@@ -133,8 +133,13 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
   extern __shared__ __align__(16) uint8_t smem_raw[];  // histogram columns, then the code builder
   uint32_t* sh = reinterpret_cast<uint32_t*>(smem_raw);
   __shared__ int s_last;
+  // FP32: the slice's zero-run block bits of the three fraction planes (a slice of 32768
+  // values is 1024 blocks, 32 words a plane, words no other slice holds)
+  constexpr int NBP = n_byte_planes(DT) > 0 ? n_byte_planes(DT) : 1;
+  __shared__ uint32_t s_zbits[NBP][32];
   const int tid = threadIdx.x, lane = tid & 31;
   for (int i = tid; i < AJ * 32; i += kHistThreads) sh[i] = 0;
+  if (tid < NBP * 32) s_zbits[tid / 32][tid % 32] = 0;
   __syncthreads();
   const uint32_t c = blockIdx.x / slices, sl = blockIdx.x % slices;
   const uint64_t clo = (uint64_t)c * g.m0;
@@ -144,7 +149,9 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
 #pragma unroll
   for (int s = 0; s < NS; s++) nz[s] = 0;
   uint32_t* col0 = sh + lane;
-  constexpr int NV = 64;  // consecutive values per thread per pass, loaded up front
+  // consecutive values per thread per pass, loaded up front (FP32: 32, one zero-run block,
+  // so that the values fit the registers)
+  constexpr int NV = DT == kFP32 ? 32 : 64;
   for (uint32_t t0 = lo; t0 < hi; t0 += kHistThreads * NV) {
     const uint32_t v0 = t0 + tid * NV;
     const int cnt = v0 < hi ? (int)min32(NV, hi - v0) : 0;
@@ -160,30 +167,22 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
         }
       }
       if constexpr (DT == kFP32) {
-        // every stream is a bit field of the value, so the OR of the words holds the OR of
-        // each stream's symbols: of my 64 values for the all-zero flags, and of each half
-        // (zero-run blocks v0 / 32 and v0 / 32 + 1, an even pair) for the fraction planes
-        static_assert(NV == 2 * kZBlock, "a thread's values are two zero-run blocks");
+        // every stream is a bit field of the value, so the OR of my words holds the OR of
+        // each stream's symbols: for the all-zero flags, and for my values' zero-run block
+        // (v0 / 32) of each fraction plane
+        static_assert(NV == kZBlock, "a thread's values are one zero-run block");
         RawValues<DT, NV> o;
-        uint32_t a = 0, b = 0;
+        uint32_t a = 0;
 #pragma unroll
-        for (int i = 0; i < NV / 2; i++) {
-          a |= raw.w[i];
-          b |= raw.w[NV / 2 + i];
-        }
+        for (int i = 0; i < NV; i++) a |= raw.w[i];
         o.w[0] = a;
-        o.w[1] = b;
-        o.w[2] = a | b;
 #pragma unroll
-        for (int s = 0; s < NS; s++) nz[s] |= symbol<DT, NV>(o, s, 2);
+        for (int s = 0; s < NS; s++) nz[s] |= symbol<DT, NV>(o, s, 0);
         if (ws.zmap) {
-          const uint32_t blk = v0 / kZBlock;
+          const uint32_t blk = (v0 - lo) / kZBlock;  // within the slice
 #pragma unroll
-          for (int s = 1; s < NS; s++) {
-            const uint32_t bits = (symbol<DT, NV>(o, s, 0) ? 1u : 0u) | (symbol<DT, NV>(o, s, 1) ? 2u : 0u);
-            const uint64_t plane = (uint64_t)c * n_byte_planes(DT) + (s - 1);
-            if (bits) atomicOr(ws.zmap + plane * g.zwords + blk / 32, bits << (blk % 32));
-          }
+          for (int s = 1; s < NS; s++)
+            if (symbol<DT, NV>(o, s, 0)) atomicOr(&s_zbits[s - 1][blk / 32], 1u << (blk % 32));
         }
       } else {
         // FP8 and FP4: the same bit-field argument; the OR of the words folded onto its
@@ -208,6 +207,12 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
   }
 
   __syncthreads();
+  if constexpr (n_byte_planes(DT) > 0) {
+    if (ws.zmap && tid < NBP * 32) {  // the slice's bitmap words, plain stores
+      const uint32_t wi = sl * 32u + (uint32_t)(tid % 32);
+      if (wi < g.zwords) ws.zmap[((uint64_t)c * NBP + tid / 32) * g.zwords + wi] = s_zbits[tid / 32][tid % 32];
+    }
+  }
   // column sums: thread b reads its row starting at lane b, so a warp hits 32 banks
   if constexpr (NE == 1) {
     for (int b = tid; b < A0; b += kHistThreads) {
