@@ -340,15 +340,21 @@ __global__ void __launch_bounds__(kHistThreads) k_split_hist_bf16(const uint8_t*
   if (tid == 0)
     for (int s = 0; s < kHbStages; s++) issue(s);
 
-  uint8_t* const colb = reinterpret_cast<uint8_t*>(sh + lane);
+  // counter of exponent e for this lane: byte (e << 7) | (lane << 2) of the table, one
+  // LOP3 from the value's word (the exponent field is bits 14..7 of the low value)
+  uint8_t* const tab = reinterpret_cast<uint8_t*>(sh);
+  const uint32_t l4 = (uint32_t)lane << 2;
+  uint8_t* const zbytes = reinterpret_cast<uint8_t*>(zbits);
   const int warp = tid >> 5;
+  constexpr int kUnits = (int)(kHbPieceValues / 8 / kHistThreads);  // 16-byte units a thread takes per piece
   uint32_t q = 0;  // pieces consumed
   for (uint32_t tile = blockIdx.x; tile < g.n_tiles; tile += gridDim.x) {
     uint64_t vlo;
     const uint32_t nv = hb_tile_values(g, tile, vlo);
     if (nv == 0) continue;  // uniform
     const uint32_t c = tile / T, sl = tile - c * T;
-    uint32_t nz0 = 0, nz1 = 0;
+    uint32_t nzall = 0;   // OR of every word I counted
+    uint32_t tail_nz = 0; // thread 0: OR of the sign/fraction bits of the tile's last < 8 values
     for (uint32_t p0 = 0; p0 < nv; p0 += kHbPieceValues, q++) {
       const int s = (int)(q % kHbStages);
       if (!mbar_wait_bounded(bar + s, (q / kHbStages) & 1u, kHbWaitLimit) && ws.status) set_status(ws.status, kStTimeout);
@@ -356,87 +362,94 @@ __global__ void __launch_bounds__(kHistThreads) k_split_hist_bf16(const uint8_t*
       const uint4* st4 = reinterpret_cast<const uint4*>(stages + (size_t)s * kHbPieceValues * 2);
       uint32_t my4 = 0;  // bit k: my unit of iteration k holds a non-zero sign/fraction byte
 #pragma unroll
-      for (int k = 0; k < (int)(kHbPieceValues / 8 / kHistThreads); k++) {
+      for (int k = 0; k < kUnits; k++) {
         const uint32_t i = (uint32_t)(k * kHistThreads + tid);
-        uint32_t sfnz = 0;  // sign/fraction bits of my 8 values
         if (i * 8 < nb) {
           const uint4 v = st4[i];
           const uint32_t x[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
           for (int j = 0; j < 4; j++) {
-            // the low value's exponent is bits 14..7: its counter (row e, 32 words) is
-            // at byte offset w & 0x7F80; the high value's at (w >> 16) & 0x7F80
-            atomicAdd(reinterpret_cast<uint32_t*>(colb + (x[j] & 0x7F80u)), 1u);
-            atomicAdd(reinterpret_cast<uint32_t*>(colb + ((x[j] >> 16) & 0x7F80u)), 1u);
-            nz0 |= x[j] & 0x7F807F80u;
-            sfnz |= x[j] & 0x807F807Fu;
+            atomicAdd(reinterpret_cast<uint32_t*>(tab + ((x[j] & 0x7F80u) | l4)), 1u);
+            atomicAdd(reinterpret_cast<uint32_t*>(tab + (((x[j] >> 16) & 0x7F80u) | l4)), 1u);
           }
-          nz1 |= sfnz;
+          const uint32_t o = v.x | v.y | v.z | v.w;
+          nzall |= o;
+          my4 |= ((o & 0x807F807Fu) != 0 ? 1u : 0u) << k;
         }
-        my4 |= (sfnz != 0 ? 1u : 0u) << k;
       }
-      if (ws.zmap) {
-        // zero-run blocks: in iteration k the warp's 32 units of 8 values are the tile's 8
-        // blocks 8w + 64k + piece offset; four units make a block. Ballot, then fold each
-        // nibble of the ballot onto one bit and gather the 8 bits (no branch per lane).
+      // zero-run blocks (32 values: four units, four lanes): only a warp that saw a unit
+      // with no non-zero sign/fraction byte records anything. In iteration k the warp's
+      // 32 units are the tile's 8 blocks 8w + 64k + piece offset: a ballot of the zero
+      // units, each nibble folded onto one bit (its four lanes all zero), the 8 bits
+      // gathered into the byte of those blocks (a byte no other warp or iteration writes).
+      if (ws.zmap && !__all_sync(0xFFFFFFFFu, my4 == (1u << kUnits) - 1u)) {
 #pragma unroll
-        for (int k = 0; k < (int)(kHbPieceValues / 8 / kHistThreads); k++) {
-          uint32_t b = __ballot_sync(0xFFFFFFFFu, (my4 >> k) & 1u);
-          b |= b >> 1;
-          b |= b >> 2;
-          b &= 0x11111111u;  // bit 4j: block j of the eight
+        for (int k = 0; k < kUnits; k++) {
+          uint32_t b = __ballot_sync(0xFFFFFFFFu, ((my4 >> k) & 1u) == 0);
+          b &= b >> 1;
+          b &= b >> 2;
+          b &= 0x11111111u;  // bit 4j: block j of the eight is all zero
           b = (b | (b >> 3)) & 0x03030303u;
           b = (b | (b >> 6)) & 0x000F000Fu;
           b = (b | (b >> 12)) & 0xFFu;
-          const uint32_t blk = p0 / kZBlock + (uint32_t)(64 * k + 8 * warp);  // within the tile
-          if (lane == k && b) atomicOr(zbits + blk / 32, b << (blk % 32));
+          if (lane == k) zbytes[p0 / (kZBlock * 8) + (uint32_t)(8 * k + warp)] = (uint8_t)b;
         }
       }
       if (tid == 0 && nb < pv) {
         const uint16_t* t = reinterpret_cast<const uint16_t*>(src) + vlo + p0 + nb;
-        uint32_t sfnz = 0;
         for (uint32_t i = 0; i < pv - nb; i++) {
           const uint32_t v = t[i];
-          atomicAdd(reinterpret_cast<uint32_t*>(colb + (v & 0x7F80u)), 1u);
-          nz0 |= v & 0x7F80u;
-          sfnz |= v & 0x807Fu;
-        }
-        nz1 |= sfnz;
-        if (ws.zmap && sfnz) {  // the tail (under 8 values) lies in one block
-          const uint32_t blk = (p0 + nb) / kZBlock;
-          atomicOr(zbits + blk / 32, 1u << (blk % 32));
+          atomicAdd(reinterpret_cast<uint32_t*>(tab + ((v & 0x7F80u) | l4)), 1u);
+          nzall |= v;
+          tail_nz |= v & 0x807Fu;
         }
       }
       __syncthreads();  // stage s is read, and the tile's counts are complete after the last piece
       if (tid == 0) issue(s);
     }
-    nz0 = __reduce_or_sync(0xFFFFFFFFu, nz0);
-    nz1 = __reduce_or_sync(0xFFFFFFFFu, nz1);
+    const uint32_t nz0 = __reduce_or_sync(0xFFFFFFFFu, nzall & 0x7F807F80u);
+    const uint32_t nz1 = __reduce_or_sync(0xFFFFFFFFu, nzall & 0x807F807Fu);
     if (nonzero && lane == 0) {
       if (nz0) atomicOr(&nonzero[(uint64_t)c * 2], nz0);
       if (nz1) atomicOr(&nonzero[(uint64_t)c * 2 + 1], nz1);
     }
-    // row b (exponent b): thread b sums it from lane b on (32 banks a warp) and clears it
+    // row b (exponent b): thread b sums it (eight 16-byte loads, rotated so that the
+    // eight lanes of a quarter warp take eight different bank groups) and clears it
     {
       const int b = tid;
+      uint4* row = reinterpret_cast<uint4*>(sh + b * 32);
       uint32_t sum = 0;
-#pragma unroll 8
-      for (int l = 0; l < 32; l++) {
-        const int a = b * 32 + ((l + b) & 31);
-        sum += sh[a];
-        sh[a] = 0;
+#pragma unroll
+      for (int j = 0; j < 8; j++) {
+        const int gi = (j + b) & 7;
+        const uint4 v = row[gi];
+        sum += v.x + v.y + v.z + v.w;
+        row[gi] = make_uint4(0u, 0u, 0u, 0u);
       }
       if (sum) atomicAdd(&hist[(uint64_t)c * 256 + b], sum);
       if (ws.tile_hist) ws.tile_hist[((uint64_t)c * T + sl) * 256 + b] = (uint16_t)sum;
     }
-    if (ws.zmap && tid < 32) {
-      // the tile's 32 bitmap words (complete since the last piece's barrier) go out as
-      // plain stores, their marked blocks into the chunk's count; then cleared
-      const uint32_t word = zbits[tid], wi = sl * 32u + (uint32_t)tid;
-      if (wi < g.zwords) ws.zmap[(uint64_t)c * g.zwords + wi] = word;
-      const uint32_t marked = __reduce_add_sync(0xFFFFFFFFu, __popc(word));
-      if (tid == 0 && marked) atomicAdd(ws.zcount + c, marked);
-      zbits[tid] = 0;
+    if (ws.zmap) {
+      // the tile's last values (under 8, the tensor's end): a non-zero sign/fraction
+      // byte there marks their block, whatever its earlier units held
+      if (nv & 7u) {
+        if (tid == 0 && tail_nz) {
+          const uint32_t blk = (nv - 1) / kZBlock;
+          zbytes[blk / 8] &= (uint8_t)~(1u << (blk % 8));
+        }
+        __syncthreads();
+      }
+      if (tid < 32) {
+        // the tile's 32 bitmap words go out as plain stores: a block is marked when it
+        // lies in the tile and is not all zero; the marked count goes into the chunk's
+        const uint32_t nvb = ceil_div(nv, kZBlock), lo = (uint32_t)tid * 32u;
+        const uint32_t valid = lo >= nvb ? 0u : nvb - lo >= 32u ? 0xFFFFFFFFu : (1u << (nvb - lo)) - 1u;
+        const uint32_t word = ~zbits[tid] & valid, wi = sl * 32u + (uint32_t)tid;
+        if (wi < g.zwords) ws.zmap[(uint64_t)c * g.zwords + wi] = word;
+        const uint32_t marked = __reduce_add_sync(0xFFFFFFFFu, __popc(word));
+        if (tid == 0 && marked) atomicAdd(ws.zcount + c, marked);
+        zbits[tid] = 0;
+      }
     }
     __syncthreads();  // every row and bitmap word is clear before the next tile's counts
   }

@@ -500,3 +500,30 @@ def test_zero_runs_corrupt(z, orc):
         z.decompress_into(torch.from_numpy(d).cuda(), d.size, out, ws, chunk_bytes=cb)
         assert z.status(ws) == z.ERR_CORRUPT
         assert orc.decompress_status("bf16", d, x.numel(), chunk_bytes=cb) == orc.ECORRUPT
+
+
+@pytest.mark.parametrize("name", ["bf16", "fp32", "fp8_e4m3"])
+def test_input_16_byte_aligned_only(z, orc, name):
+    """A tensor that starts 16 bytes past a 32-byte boundary (the encode then reads it with
+    128-bit loads instead of 256-bit ones): the same container as the oracle's."""
+    from lossless_float_weight_b200 import workloads as W
+    g = torch.Generator().manual_seed(16)
+    n = 131072 * 3 + 4096
+    if name == "bf16":
+        x = (torch.randn(n + 8, generator=g) * 0.02).to(torch.bfloat16)
+        shift = 8
+    elif name == "fp32":
+        x = (torch.randn(n + 4, generator=g) * 0.02).float()
+        shift = 4
+    else:
+        x = W.fp8_tensor(rows=(n + 4096) // 4096, cols=4096, seed=16).reshape(-1)
+        shift = 16
+    base = x.cuda()
+    assert base.data_ptr() % 32 == 0
+    xd = base[shift:shift + n]
+    assert xd.data_ptr() % 32 == 16
+    cont = z.compress(xd).cpu().numpy()
+    ref = orc.compress(name, _host_bytes(x[shift:shift + n]), n, chunk_bytes=CB, S=S_DEFAULT, threads=8)
+    assert np.array_equal(cont, ref)
+    y = z.decompress(torch.from_numpy(ref).cuda(), x.dtype, n)
+    assert torch.equal(y.view(torch.uint8).cpu(), torch.from_numpy(_host_bytes(x[shift:shift + n]).copy()))
