@@ -730,14 +730,18 @@ def run_single(args):
     stream = torch.cuda.current_stream(dev)
     w = args.workload
     if w in ("fp32", "fp32_clean"):
-        x = W.fp32_tensor(n=268435456, device=dev, clean=(w == "fp32_clean"))
-        desc = "FP32 268,435,456 values N(0, 0.02^2)" + (", rounded through BF16" if w == "fp32_clean" else "")
+        rows = args.rows or 65536
+        x = W.fp32_tensor(n=rows * 4096, device=dev, clean=(w == "fp32_clean"))
+        desc = f"FP32 {rows * 4096:,} values N(0, 0.02^2)" + (", rounded through BF16" if w == "fp32_clean" else "")
     elif w == "fp8":
-        x = W.fp8_tensor(rows=262144, cols=4096, device=dev)
-        desc = "FP8 E4M3 262,144 x 4096, N(0, 1) x per-row scale log-uniform [0.25, 4]"
+        rows = args.rows or 262144
+        x = W.fp8_tensor(rows=rows, cols=4096, device=dev)
+        desc = f"FP8 E4M3 {rows:,} x 4096, N(0, 1) x per-row scale log-uniform [0.25, 4]"
     elif w == "fp4":
-        x = W.fp4_tensor(rows=262144, cols=4096, device=dev)
-        desc = "FP4 E2M1 262,144 x 4096 (1,073,741,824 values), N(0, 1) x per-row scale log-uniform [0.25, 4]"
+        rows = args.rows or 262144
+        x = W.fp4_tensor(rows=rows, cols=4096, device=dev)
+        desc = (f"FP4 E2M1 {rows:,} x 4096 ({rows * 4096:,} values), N(0, 1) x per-row scale "
+                "log-uniform [0.25, 4]")
     else:
         x = W.kv_cache(device=dev)
         desc = "BF16 K/V cache [32, 2, 16, 8, 4096, 128], per-channel std log-normal, 8-group plan"
@@ -811,6 +815,9 @@ def main():
     ap.add_argument("--workload", default="checkpoint_7b",
                     choices=["checkpoint_7b", "fp32", "fp32_clean", "fp8", "fp4", "kv_cache"],
                     help="another workload than the benchmark's: one tensor, compress and decompress timed apart")
+    ap.add_argument("--rows", type=int, default=None,
+                    help="rows of 4096 values for --workload fp32/fp32_clean/fp8/fp4 (profiler cases; "
+                         "default 65536 FP32, 262144 FP8/FP4)")
     ap.add_argument("--plan-transfer", action="store_true",
                     help="instead of the benchmark: build a shared-code plan on layers 0-15 and reuse it on 16-31")
     ap.add_argument("--groups", type=int, default=8, help="plan groups for --plan-transfer")

@@ -126,6 +126,13 @@ __device__ __forceinline__ void set_status(uint32_t* st, uint32_t code) { atomic
 
 __device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
 
+// 32 bytes to global memory in one 256-bit store (sm_100: st.global.v8; p 32-byte aligned).
+__device__ __forceinline__ void st_v8(void* p, const uint32_t* r) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+               :: "l"(p), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
 // 32 bytes from global memory in one 256-bit load (sm_100: ld.global.v8; p 32-byte
 // aligned), through the read-only path. A warp whose lanes read consecutive 128-byte
 // runs asks L1 for one sector a lane per load instead of half a sector.

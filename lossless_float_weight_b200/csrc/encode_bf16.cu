@@ -11,8 +11,8 @@
 // per SM) keep the barriers of a pass short and let the blocks' load and compute phases
 // interleave. In each pass it
 //  * loads its 64 values per thread (256-bit loads; 128-bit ones when the tensor is only
-//    16-byte aligned) and writes the sign/fraction plane
-//    (and an exponent plane that did not compress) with 16-byte stores;
+//    16-byte aligned) and writes the sign/fraction plane (and an exponent plane that
+//    did not compress) with 32-byte stores (two 16-byte ones where only 16-byte aligned);
 //  * packs its exponent codes, two per step, most significant bit first, into private
 //    shared words from bit 0; a block scan gives each thread its bit offset in the tile;
 //  * moves the private words into a staging copy of the tile's bitstream at its final
@@ -168,11 +168,17 @@ __global__ void __launch_bounds__(kBThreads, 8) k_encode_bf16(const uint8_t* __r
         }
         if (cnt == kBValues) {
 #pragma unroll
-          for (int q = 0; q < kBValues / 16; q++) {
-            uint32_t x[4];
+          for (int h = 0; h < 2; h++) {
+            uint32_t x[8];
 #pragma unroll
-            for (int k = 0; k < 4; k++) x[k] = bf16_quad_plane(raw.w[8 * q + 2 * k], raw.w[8 * q + 2 * k + 1], s);
-            if (half[q >> 1]) *reinterpret_cast<uint4*>(half[q >> 1] + 16 * (q & 1)) = make_uint4(x[0], x[1], x[2], x[3]);
+            for (int k = 0; k < 8; k++) x[k] = bf16_quad_plane(raw.w[16 * h + 2 * k], raw.w[16 * h + 2 * k + 1], s);
+            if (!half[h]) continue;
+            if ((reinterpret_cast<uintptr_t>(half[h]) & 31) == 0) {
+              st_v8(half[h], x);
+            } else {
+              *reinterpret_cast<uint4*>(half[h]) = make_uint4(x[0], x[1], x[2], x[3]);
+              *reinterpret_cast<uint4*>(half[h] + 16) = make_uint4(x[4], x[5], x[6], x[7]);
+            }
           }
         } else {
           // the chunk's last values: 16-byte groups, zero past cnt (a ZRUN block's data
