@@ -77,32 +77,32 @@ struct BitReader {
     acc |= e;
     return lut_symbol(e);
   }
+  __device__ __forceinline__ uint32_t peek12() const { return (uint32_t)(buf >> 52); }
+  __device__ __forceinline__ void skip(uint32_t l) {
+    buf <<= l;
+    nb -= (int)l;
+  }
   // absolute index of the next unread bit
   __device__ __forceinline__ uint64_t position() const { return (uint64_t)(pos - 2) * 32 - (uint64_t)nb; }
 };
 
 // Two symbols from either bit reader, returned in bits 16..31 (the first in 16..23).
-// Needs at least 12 valid bits on entry and leaves at least 0; when the window holds
-// only one whole code the reader refills once between the two lookups.
+// Needs a full 12-bit window on entry; when the window holds only one whole code the
+// reader refills once between the two lookups.
 template <class Reader>
 __device__ __forceinline__ uint32_t huff_pair(Reader& br, const uint32_t* lut, uint32_t& acc) {
-  const uint32_t e = lut[br.buf >> 52];
+  const uint32_t e = lut[br.peek12()];
   acc |= e;
   const uint32_t lp = (e >> 4) & 15u;
   if (lp) {
-    br.buf <<= lp;
-    br.nb -= (int)lp;
+    br.skip(lp);
     return e;
   }
-  const uint32_t l0 = e & 15u;
-  br.buf <<= l0;
-  br.nb -= (int)l0;
+  br.skip(e & 15u);
   br.refill();
-  const uint32_t e2 = lut[br.buf >> 52];
+  const uint32_t e2 = lut[br.peek12()];
   acc |= e2;
-  const uint32_t l1 = e2 & 15u;
-  br.buf <<= l1;
-  br.nb -= (int)l1;
+  br.skip(e2 & 15u);
   return (e & 0x00FF0000u) | ((e2 & 0x00FF0000u) << 8);
 }
 
@@ -312,16 +312,16 @@ struct StagedSmem {
 };
 
 
-// Bit reader over words in shared memory; the next word is always already loaded.
-// WIDE: words from kWindowWords on are in a second region, w2.
+// Bit reader over words in shared memory, by position: c holds words p and p + 1 (p in
+// the high half), bp of its bits are consumed, q is word p + 2. A refill advances one word
+// when bp reaches 32 (the next word is requested one refill ahead), so a 12-bit window at
+// bp <= 52 lies inside c. WIDE: words from kWindowWords on are in a second region, w2.
 template <bool WIDE = false>
 struct SmemBitReader {
   const uint32_t* w;
   const uint32_t* w2;
-  uint32_t pos, end;
-  uint64_t buf;
-  int nb;
-  uint32_t q;
+  uint32_t p, end, bp, q;
+  uint64_t c;
   // Word i of the bitstream. Past the end a reader sees the word at `end` (stale data or
   // the next buffer, always inside the block's shared memory): a valid sub-block never
   // consumes those bits, and one that does ends past its bound and is reported.
@@ -335,43 +335,35 @@ struct SmemBitReader {
     w = words;
     w2 = words2;
     end = nwords;
-    const uint32_t p0 = (uint32_t)(bit >> 5);
-    buf = (uint64_t)ld(p0) << 32;
-    q = ld(p0 + 1);
-    pos = p0 + 2;
-    nb = 32;
-    const int skip = (int)(bit & 31);
-    buf <<= skip;
-    nb -= skip;
-    refill();
+    p = (uint32_t)(bit >> 5);
+    c = ((uint64_t)ld(p) << 32) | ld(p + 1);
+    q = ld(p + 2);
+    bp = (uint32_t)(bit & 31);
   }
   __device__ __forceinline__ void refill() {
-    const bool r = nb <= 32;
-    const uint64_t add = (uint64_t)q << ((32 - nb) & 63);
-    const uint32_t nq = ld(pos);
-    buf |= r ? add : 0ull;
-    q = r ? nq : q;
-    pos += r ? 1u : 0u;
-    nb += r ? 32 : 0;
+    const bool t = bp >= 32;
+    const uint32_t nq = ld(p + 3);
+    c = t ? (c << 32) | q : c;
+    q = t ? nq : q;
+    p += t ? 1u : 0u;
+    bp -= t ? 32u : 0u;
   }
+  __device__ __forceinline__ uint32_t peek12() const { return (uint32_t)((c << bp) >> 52); }
+  __device__ __forceinline__ void skip(uint32_t l) { bp += l; }
   __device__ __forceinline__ uint32_t huff(const uint32_t* lut, uint32_t& acc) {
-    const uint32_t e = lut[buf >> 52];
-    const uint32_t l = e & 15u;
-    buf <<= l;
-    nb -= (int)l;
+    const uint32_t e = lut[peek12()];
+    bp += e & 15u;
     acc |= e;
     return lut_symbol(e);
   }
   // single-symbol table: symbol << 4 | length, bit 15 invalid
   __device__ __forceinline__ uint32_t huff(const uint16_t* lut, uint32_t& acc) {
-    const uint32_t e = lut[buf >> 52];
-    const uint32_t l = e & 15u;
-    buf <<= l;
-    nb -= (int)l;
+    const uint32_t e = lut[peek12()];
+    bp += e & 15u;
     acc |= e;
     return (e >> 4) & 0xFFu;
   }
-  __device__ __forceinline__ uint64_t position() const { return (uint64_t)(pos - 1) * 32 - (uint64_t)nb; }
+  __device__ __forceinline__ uint64_t position() const { return (uint64_t)p * 32 + bp; }
 };
 
 __device__ __forceinline__ uint32_t ex_word(uint32_t row, uint32_t k) {
