@@ -67,7 +67,7 @@ struct WsPlan {
   uint64_t status, hist, nonzero, zmap, zcount, scan_desc, tile_desc, slot, zero_end;
   uint64_t esize, emode, ecode, eoff, enc, tile_hist, tile_off;
   uint64_t km_mu, km_perm, km_assign, km_changed, km_gsum, total;
-  bool tile_counts;  // per-tile exponent histograms (BF16)
+  bool tile_counts;  // per-tile histograms and bit offsets (BF16, FP8, FP4)
   int dt;
 };
 
@@ -90,9 +90,9 @@ WsPlan ws_plan(const Geo& g) {
   p.ecode = o;      o = align_up(o + K * 4);
   p.eoff = o;       o = align_up(o + K * 8);
   p.enc = o;        o = align_up(o + C * NE * 256 * 4);
-  p.tile_counts = g.dt == kBF16;
-  p.tile_hist = o;  o = align_up(o + (p.tile_counts ? (uint64_t)g.n_tiles * 256 * 2 : 0));
-  p.tile_off = o;   o = align_up(o + (p.tile_counts ? (uint64_t)g.n_tiles * 4 : 0));
+  p.tile_counts = g.dt != kFP32;
+  p.tile_hist = o;  o = align_up(o + (p.tile_counts ? (uint64_t)g.n_tiles * tile_bins(g.dt) * 2 : 0));
+  p.tile_off = o;   o = align_up(o + (p.tile_counts ? NE * g.n_tiles * 4 : 0));
   p.km_mu = o;      o = align_up(o + (uint64_t)kMaxGroups * 256 * 8);
   p.km_perm = o;    o = align_up(o + C * 4);
   p.km_assign = o;  o = align_up(o + C * 4);
@@ -210,7 +210,8 @@ zipnn_status zipnn_compress_ex(zipnn_dtype dtype, const void* src, uint64_t n, u
   if (e == cudaSuccess) {
     TimedLaunch t(kIdEncode, st);
     e = g.dt == kBF16 ? launch_encode_bf16(src, g, w, static_cast<uint8_t*>(out), st)
-                      : launch_encode(src, g, w, static_cast<uint8_t*>(out), st);
+        : g.dt == kFP32 ? launch_encode(src, g, w, static_cast<uint8_t*>(out), st)
+                        : launch_encode_sub(src, g, w, static_cast<uint8_t*>(out), st);
   }
   return cuda_status(e);
 }

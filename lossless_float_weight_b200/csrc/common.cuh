@@ -29,13 +29,16 @@ constexpr int kGroupValues = 16;
 constexpr int kEncGroups = 4;
 constexpr int kEncodeThreads = 256;
 constexpr int kTileValues = kEncodeThreads * kGroupValues * kEncGroups;  // 16384
-// BF16: the encode tile (512 groups of 64 values; the encode kernel takes it in passes
-// of its own block) is also one histogram tile, whose counts give its bit offset
+// BF16, FP8 and FP4: the encode tile (32768 values; the encode kernels take it in passes
+// of their own blocks) is also one histogram tile, whose counts give its bit offsets
 constexpr int kBf16EncodeThreads = 512;
 constexpr int kBf16TileValues = kBf16EncodeThreads * kGroupValues * kEncGroups;  // 32768
 __host__ __device__ constexpr uint32_t tile_values(int dt) {
-  return dt == kBF16 ? (uint32_t)kBf16TileValues : (uint32_t)kTileValues;
+  return dt == kFP32 ? (uint32_t)kTileValues : (uint32_t)kBf16TileValues;
 }
+// Counters a tile keeps for its bit offsets: BF16 the 256 exponents; FP8 and FP4 the joint
+// (exponent, mantissa) bins, exponent * mantissa alphabet + mantissa (FP8 16 x 8, FP4 4 x 2).
+__host__ __device__ constexpr uint32_t tile_bins(int dt) { return dt == kBF16 ? 256u : dt == kFP8 ? 128u : dt == kFP4 ? 8u : 0u; }
 
 __host__ __device__ constexpr int n_streams(int dt) { return dt == kBF16 ? 2 : dt == kFP32 ? 4 : 3; }
 // FP8 and FP4 entropy-code exponent and mantissa independently
@@ -111,8 +114,9 @@ struct Ws {
   uint32_t* ecode;      // [n_entries]
   uint64_t* eoff;       // [n_entries] payload offsets
   uint32_t* enc;        // [n_chunks][n_entropy][256]: len << 16 | code
-  uint16_t* tile_hist;  // [n_tiles][256] (BF16 compress): exponent counts of each encode tile
-  uint32_t* tile_off;   // [n_tiles] (BF16 compress): bit offset of each tile in its chunk's bitstream
+  uint16_t* tile_hist;  // [n_tiles][tile_bins] (BF16, FP8, FP4 compress): counts of each encode tile
+  uint32_t* tile_off;   // [n_entropy][n_tiles] (BF16, FP8, FP4 compress): bit offset of each tile
+                        // in its chunk's bitstream of that entropy stream
 };
 
 // Device-side tables of a plan.

@@ -1,20 +1,21 @@
-// encode.cu -- k_encode: writes every payload byte of the container.
+// encode.cu -- k_encode: writes every payload byte of an FP32 container (BF16 has
+// k_encode_bf16, FP8 and FP4 k_encode_sub; the kernel is written for any type, and the
+// sub-byte RAW branch below serves only those).
 //
 // One block per tile of 16384 values of one chunk; each of the 256 threads owns 64
 // consecutive values, all loaded up front (128-bit loads) so that a block keeps
-// 32 KB (BF16) of input in flight.
-//  * RAW byte planes (8-bit streams: BF16/FP32 sign+fraction bytes, an exponent that
-//    did not compress) go out as 16-byte stores.
-//  * bit streams (HUFF streams; FP8's 4-, 3- and 1-bit RAW streams): each thread sums
-//    the code lengths of its symbols; a block-wide warp-shuffle scan gives its bit
-//    offset inside the tile; the tile's offset inside the chunk comes from the previous
-//    tiles of the same chunk by single-pass decoupled look-back (one warp inspects 32
-//    predecessors at a time; fixed offsets for RAW streams). Codes are emitted most
-//    significant bit first into a shared staging buffer, whole words with plain stores
-//    and the two edge words of each thread with shared atomicOr; the block then stores
-//    the staged words. A word that straddles two tiles is merged in a workspace slot:
-//    each side adds (1 << 32 | its bits) and the side that arrives second stores the
-//    complete word, so no output pre-clearing and no wait between blocks is needed.
+// 64 KB of input in flight.
+//  * byte planes (the three fraction planes; an exponent that did not compress) go out
+//    as 16-byte stores, RAW at the values' own offset, ZRUN only for marked blocks.
+//  * HUFF: each thread sums the code lengths of its symbols; a block-wide warp-shuffle
+//    scan gives its bit offset inside the tile; the tile's offset inside the chunk comes
+//    from the previous tiles of the same chunk by single-pass decoupled look-back (one
+//    warp inspects 32 predecessors at a time). Codes are emitted most significant bit
+//    first into a shared staging buffer, whole words with plain stores and the two edge
+//    words of each thread with shared atomicOr; the block then stores the staged words.
+//    A word that straddles two tiles is merged in a workspace slot: each side adds
+//    (1 << 32 | its bits) and the side that arrives second stores the complete word, so
+//    no output pre-clearing and no wait between blocks is needed.
 //  * the sub-block index idx[j] (bit offset of symbol j*S) is written by the thread
 //    that owns symbol j*S; the first tile writes a local code record, the last tile the
 //    zero padding.
@@ -373,14 +374,10 @@ static cudaError_t encode_t(const void* src, const Geo& g, const Ws& ws, uint8_t
   return cudaGetLastError();
 }
 
-// FP32, FP8 and FP4 (BF16 has k_encode_bf16).
+// FP32 (BF16 has k_encode_bf16, FP8 and FP4 k_encode_sub).
 cudaError_t launch_encode(const void* src, const Geo& g, const Ws& ws, uint8_t* out, cudaStream_t st) {
-  switch (g.dt) {
-    case kFP32: return encode_t<kFP32>(src, g, ws, out, st);
-    case kFP8: return encode_t<kFP8>(src, g, ws, out, st);
-    case kFP4: return encode_t<kFP4>(src, g, ws, out, st);
-    default: return cudaErrorInvalidValue;
-  }
+  if (g.dt != kFP32) return cudaErrorInvalidValue;
+  return encode_t<kFP32>(src, g, ws, out, st);
 }
 
 }  // namespace zipnn

@@ -10,7 +10,7 @@
 // each pass starts where the previous one's bits end. Small blocks (four warps, eight
 // per SM) keep the barriers of a pass short and let the blocks' load and compute phases
 // interleave. In each pass it
-//  * loads its 64 values per thread (256-bit loads; 128-bit ones when the tensor is only
+//  * loads its 64 values per thread (256-bit loads; 128-bit ones where they start only
 //    16-byte aligned) and writes the sign/fraction plane (and an exponent plane that
 //    did not compress) with 32-byte stores (two 16-byte ones where only 16-byte aligned);
 //  * packs its exponent codes, two per step, most significant bit first, into private
@@ -76,8 +76,6 @@ __global__ void __launch_bounds__(kBThreads, 8) k_encode_bf16(const uint8_t* __r
   const int tid = threadIdx.x;
   const uint32_t T = g.tiles_per_chunk;
   for (int i = tid; i < kBStageWords; i += kBThreads) sm.stage[i] = 0;
-  // a tensor that starts 32-byte aligned is read with 256-bit loads (128 bytes a thread)
-  const bool src32 = (reinterpret_cast<uintptr_t>(src) & 31) == 0;
 
   for (uint32_t tile = blockIdx.x; tile < g.n_tiles; tile += gridDim.x) {
     const uint32_t c = tile / T, ti = tile - c * T;
@@ -135,11 +133,12 @@ __global__ void __launch_bounds__(kBThreads, 8) k_encode_bf16(const uint8_t* __r
       const uint32_t v0 = plo + tid * kBValues;
       const int cnt = v0 < m ? (int)min32(kBValues, m - v0) : 0;
       RawValues<kBF16, kBValues> raw;
-      if (cnt == kBValues && src32) {
+      const uint8_t* vp = src + (clo + v0) * 2;
+      if (cnt == kBValues && (reinterpret_cast<uintptr_t>(vp) & 31) == 0) {
 #pragma unroll
-        for (int j = 0; j < kBValues / 16; j++) ld_nc_v8(src + (clo + v0) * 2 + 32 * j, raw.w + 8 * j);
+        for (int j = 0; j < kBValues / 16; j++) ld_nc_v8(vp + 32 * j, raw.w + 8 * j);
       } else if (cnt > 0) {
-        load_values<kBF16, kBValues>(src + (clo + v0) * 2, cnt, raw);
+        load_values<kBF16, kBValues>(vp, cnt, raw);
       }
 
 #pragma unroll

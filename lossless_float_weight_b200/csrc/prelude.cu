@@ -116,6 +116,40 @@ __device__ void build_chunk_table(const Geo& g, const Ws& ws, const PlanDev& pla
   }
 }
 
+// FP8 and FP4, each entropy stream with a HUFF code: the bit offset of every encode tile
+// of chunk c in the stream's bitstream, the running sum over the lower tiles of
+// sum over the joint bins (e, m) of count(tile, e, m) * len(the stream's symbol of the
+// bin). The tiles' joint counts are complete: this is the chunk's last histogram block.
+template <int DT>
+__device__ void joint_tile_offsets(const Geo& g, const Ws& ws, uint32_t c, HuffBlockSmem& hs) {
+  constexpr int NS = n_streams(DT), A0 = alphabet(DT, 0), A1 = alphabet(DT, 1), AJ = A0 * A1;
+  static_assert(AJ == (int)tile_bins(DT), "one counter a joint bin");
+  const int tid = threadIdx.x;
+  const uint32_t T = g.tiles_per_chunk;
+#pragma unroll
+  for (int e = 0; e < 2; e++) {
+    if (ws.emode[(uint64_t)c * NS + e] != kModeHuff) continue;  // uniform
+    constexpr int AMAX = A0 > A1 ? A0 : A1;
+    uint32_t L[AMAX];
+#pragma unroll
+    for (int a = 0; a < AMAX; a++) L[a] = a < (e == 0 ? A0 : A1) ? ws.enc[((uint64_t)c * 2 + e) * 256 + a] >> 16 : 0u;
+    uint32_t carry = 0;
+    for (uint32_t base = 0; base < T; base += kHistThreads) {
+      const uint32_t t = base + tid;
+      uint32_t bits = 0;
+      if (t < T) {
+        const uint16_t* h = ws.tile_hist + ((uint64_t)c * T + t) * AJ;
+#pragma unroll
+        for (int b = 0; b < AJ; b++) bits += (uint32_t)__ldcg(h + b) * L[e == 0 ? b / A1 : b % A1];
+      }
+      uint32_t total;
+      const uint32_t before = block_exclusive_scan<kHistThreads>(bits, hs.red32, total);
+      if (t < T) ws.tile_off[(uint64_t)e * g.n_tiles + (uint64_t)c * T + t] = carry + before;
+      carry += total;
+    }
+  }
+}
+
 // THEORY-599 note, "Order-0 only (section III-A b)": the model of a chunk is the count
 // of each symbol. The block keeps one counter per (symbol, lane) in shared memory, so
 // the 32 lanes of a warp always add into 32 different banks (lane l owns column l);
@@ -229,6 +263,8 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
 #pragma unroll 8
       for (int l = 0; l < 32; l++) sum += sh[b * 32 + ((l + b) & 31)];
       joint[b] = sum;
+      // the slice is encode tile sl of the chunk: its joint counts give its bit offsets
+      if (ws.tile_hist) ws.tile_hist[((uint64_t)c * g.tiles_per_chunk + sl) * AJ + b] = (uint16_t)sum;
     }
     __syncthreads();
     for (int t = tid; t < A0 + A1; t += kHistThreads) {
@@ -255,6 +291,9 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
   for (int e = 0; e < NE; e++) {
     build_chunk_table<DT>(g, ws, plan, c, (uint32_t)e, hs);
     __syncthreads();
+  }
+  if constexpr (NE > 1) {
+    if (ws.tile_off) joint_tile_offsets<DT>(g, ws, c, hs);
   }
 #pragma unroll
   for (int s = 0; s < NS; s++) {
