@@ -284,6 +284,171 @@ __device__ __forceinline__ int decode_bf16_fast(const uint32_t* lut, const uint8
   return (acc & kLutInvalid) || (exact ? pos != expect : pos > expect);
 }
 
+// FP8 and FP4 with a HUFF exponent stream and RAW (or ZERO: MZ, SZ) mantissa and sign
+// streams, the case of every chunk whose mantissas are near uniform: one sub-block, 32
+// values a step. The exponents come two a lookup; the step's RAW words (FP8: three
+// mantissa words and one sign word, FP4: one of each; value v's bits at v * width, so a
+// step of 32 values starts on a word) are loaded one step ahead, and their fields are
+// spread into the output bytes or nibbles with shifts, masks and multiplies. mwp / swp:
+// the sub-block's first mantissa / sign word (S is a multiple of 32), or nullptr (ZERO).
+// Returns nonzero if the stream is inconsistent.
+template <int DT, bool MZ, bool SZ>
+__device__ __forceinline__ int decode_sub_fast(const uint32_t* lut, const uint32_t* bs, uint32_t bs_words,
+                                               uint64_t start, uint64_t expect, bool exact, const uint32_t* mwp,
+                                               const uint32_t* swp, uint32_t count, uint8_t* __restrict__ dst) {
+  constexpr int WM = raw_width(DT, 1);  // mantissa bits: FP8 3, FP4 1
+  BitReader br;
+  br.init(bs, bs_words, start);
+  uint32_t acc = 0;
+  const uint32_t full = count / 32;
+  uint32_t mc[WM], mn[WM], sc = 0, sn = 0;  // this step's and the next step's RAW words (MSB first)
+#pragma unroll
+  for (int i = 0; i < WM; i++) mc[i] = mn[i] = 0;
+  if (full > 0) {
+#pragma unroll
+    for (int i = 0; i < WM; i++) mc[i] = MZ ? 0u : bswap32(__ldg(mwp + i));
+    sc = SZ ? 0u : bswap32(__ldg(swp));
+  }
+  if (full > 1) {
+#pragma unroll
+    for (int i = 0; i < WM; i++) mn[i] = MZ ? 0u : bswap32(__ldg(mwp + WM + i));
+    sn = SZ ? 0u : bswap32(__ldg(swp + 1));
+  }
+  for (uint32_t gi = 0; gi < full; gi++) {
+    uint32_t pr[16];  // exponent pairs in bits 16..31
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+      br.refill();
+      pr[i] = huff_pair(br, lut, acc);
+      pr[i + 1] = huff_pair(br, lut, acc);
+    }
+    uint32_t M[WM], Sg = sc;
+#pragma unroll
+    for (int i = 0; i < WM; i++) {
+      M[i] = mc[i];
+      mc[i] = mn[i];
+    }
+    sc = sn;
+    if (gi + 2 < full) {
+#pragma unroll
+      for (int i = 0; i < WM; i++) mn[i] = MZ ? 0u : bswap32(__ldg(mwp + (gi + 2) * WM + i));
+      sn = SZ ? 0u : bswap32(__ldg(swp + gi + 2));
+    }
+    if constexpr (DT == kFP8) {
+      // byte of value 4k + i: sign << 7 | exponent << 3 | mantissa
+      uint32_t o[8];
+#pragma unroll
+      for (int k = 0; k < 8; k++) {
+        const uint32_t ew = __byte_perm(pr[2 * k], pr[2 * k + 1], 0x7632);
+        const int a = 12 * k / 32, b = 12 * k % 32;  // the four mantissas: bits [12k, 12k + 12)
+        const uint32_t y = __funnelshift_l(a + 1 < WM ? M[a + 1 < WM ? a + 1 : 0] : 0u, M[a], b) >> 20;
+        const uint32_t mw = (y >> 9) | ((y << 2) & 0x700u) | ((y << 13) & 0x70000u) | ((y << 24) & 0x7000000u);
+        const uint32_t sw = (((Sg >> (28 - 4 * k)) & 0xFu) * 0x80402010u) & 0x80808080u;
+        o[k] = (ew << 3) | mw | sw;
+      }
+      uint4* d = reinterpret_cast<uint4*>(dst + (uint64_t)gi * 32);
+      d[0] = make_uint4(o[0], o[1], o[2], o[3]);
+      d[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    } else {
+      // nibble of value 8k + i (value 2j the low nibble of byte j): sign << 3 |
+      // exponent << 1 | mantissa; a byte of bits (value 8k first) spreads to bit 0 of the
+      // eight nibbles after its bits are reversed
+      auto spread = [](uint32_t byte) {
+        uint32_t t = __brev(byte) >> 24;
+        t = (t | (t << 12)) & 0x000F000Fu;
+        t = (t | (t << 6)) & 0x03030303u;
+        return (t | (t << 3)) & 0x11111111u;
+      };
+      uint32_t o[4];
+#pragma unroll
+      for (int k = 0; k < 4; k++) {
+        const uint32_t e0 = __byte_perm(pr[4 * k], pr[4 * k + 1], 0x7632);
+        const uint32_t e1 = __byte_perm(pr[4 * k + 2], pr[4 * k + 3], 0x7632);
+        const uint32_t en = __byte_perm(e0 | (e0 >> 4), e1 | (e1 >> 4), 0x6420);
+        const uint32_t mb = (M[0] >> (24 - 8 * k)) & 0xFFu, sb = (Sg >> (24 - 8 * k)) & 0xFFu;
+        o[k] = (en << 1) | spread(mb) | (spread(sb) << 3);
+      }
+      *reinterpret_cast<uint4*>(dst + (uint64_t)gi * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+  // the sub-block's last values (fewer than 32; FP4 an even number)
+  auto bits_at = [](const uint32_t* p, uint32_t bit, int width) {
+    const uint32_t i = bit >> 5, o = bit & 31;
+    uint32_t x = bswap32(__ldg(p + i)) << o;
+    if (o + width > 32) x |= bswap32(__ldg(p + i + 1)) >> (32 - o);
+    return x >> (32 - width);
+  };
+  for (uint32_t v = full * 32; v < count; v++) {
+    br.refill();
+    const uint32_t e = br.huff(lut, acc);
+    const uint32_t mv = MZ ? 0u : bits_at(mwp, v * WM, WM), sv = SZ ? 0u : bits_at(swp, v, 1);
+    if constexpr (DT == kFP8) {
+      dst[v] = (uint8_t)((sv << 7) | (e << 3) | mv);
+    } else {
+      const uint32_t nib = (sv << 3) | (e << 1) | mv;
+      if (v & 1) dst[v >> 1] = (uint8_t)(dst[v >> 1] | (nib << 4));
+      else dst[v >> 1] = (uint8_t)nib;
+    }
+  }
+  const uint64_t pos = br.position();
+  return (acc & kLutInvalid) || (exact ? pos != expect : pos > expect);
+}
+
+// FP32 with a HUFF exponent stream and RAW (or ZERO: nullptr) byte planes p1 (sign and
+// fraction bits 22..16), p2 (bits 15..8), p3 (bits 7..0): one sub-block, 16 values a
+// step. The exponents come two a lookup. A value's upper half is a BF16 word (p1 byte, exponent), merged two at a
+// time; its lower half is the p3 byte under the p2 byte; byte permutes join them. The
+// step's plane bytes are requested before its exponents are decoded.
+__device__ __forceinline__ int decode_fp32_fast(const uint32_t* lut, const uint32_t* bs, uint32_t bs_words,
+                                                uint64_t start, uint64_t expect, bool exact, const uint8_t* p1,
+                                                const uint8_t* p2, const uint8_t* p3, uint32_t count,
+                                                uint8_t* __restrict__ dst) {
+  BitReader br;
+  br.init(bs, bs_words, start);
+  uint32_t acc = 0;
+  const uint32_t full = count / 16;
+  const uint8_t* pl[3] = {p1, p2, p3};
+  for (uint32_t gi = 0; gi < full; gi++) {
+    // the step's plane bytes, requested before its exponents are decoded
+    uint4 pv[3];
+#pragma unroll
+    for (int k = 0; k < 3; k++)
+      pv[k] = pl[k] ? __ldg(reinterpret_cast<const uint4*>(pl[k]) + gi) : make_uint4(0, 0, 0, 0);
+    uint32_t pr[8];  // exponent pairs in bits 16..31
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      br.refill();
+      pr[i] = huff_pair(br, lut, acc);
+      pr[i + 1] = huff_pair(br, lut, acc);
+    }
+    const uint32_t x[3][4] = {{pv[0].x, pv[0].y, pv[0].z, pv[0].w},
+                              {pv[1].x, pv[1].y, pv[1].z, pv[1].w},
+                              {pv[2].x, pv[2].y, pv[2].z, pv[2].w}};
+    uint32_t o[16];
+#pragma unroll
+    for (int q = 0; q < 4; q++) {
+      const uint32_t ew = __byte_perm(pr[2 * q], pr[2 * q + 1], 0x7632);  // exponents of values 4q..4q+3
+      const uint32_t h01 = bf16_merge_pair(x[0][q], 0, ew, 0), h23 = bf16_merge_pair(x[0][q], 1, ew, 1);
+      const uint32_t l01 = __byte_perm(x[2][q], x[1][q], 0x5140), l23 = __byte_perm(x[2][q], x[1][q], 0x7362);
+      o[4 * q] = __byte_perm(l01, h01, 0x5410);
+      o[4 * q + 1] = __byte_perm(l01, h01, 0x7632);
+      o[4 * q + 2] = __byte_perm(l23, h23, 0x5410);
+      o[4 * q + 3] = __byte_perm(l23, h23, 0x7632);
+    }
+    uint4* d = reinterpret_cast<uint4*>(dst + (uint64_t)gi * 64);
+#pragma unroll
+    for (int q = 0; q < 4; q++) d[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+  }
+  for (uint32_t v = full * 16; v < count; v++) {
+    br.refill();
+    const uint32_t e = br.huff(lut, acc);
+    reinterpret_cast<uint32_t*>(dst)[v] =
+        merge_value<kFP32>(e, p1 ? p1[v] : 0u, p2 ? p2[v] : 0u, p3 ? p3[v] : 0u);
+  }
+  const uint64_t pos = br.position();
+  return (acc & kLutInvalid) || (exact ? pos != expect : pos > expect);
+}
+
 // ---------------------------------------------------------------- staged BF16 path
 // For a BF16 chunk whose exponent stream is HUFF and whose bitstream fits a 48 KB
 // window, the whole bitstream is brought into shared memory by one TMA bulk copy
@@ -578,6 +743,77 @@ static_assert(kDecodeThreads * 16 == 4096, "fill_lut: 8 warps of 512 table entri
 
 constexpr uint32_t kZStagedWords = 128;  // zero-run bitmap words the staged path holds: 4096 blocks
 static_assert(kDecodeThreads >= kZStagedWords, "one thread per bitmap word");
+
+// FP8 and FP4 chunks with a HUFF exponent stream and RAW or ZERO mantissa and sign
+// streams (sub_fast_ok): one sub-block per thread per pass through decode_sub_fast.
+template <int DT>
+__device__ __forceinline__ bool sub_fast_ok(const DecodeSmem<DT>& sm, uint32_t S) {
+  return sm.mode[0] == kModeHuff && (sm.mode[1] == kModeRaw || sm.mode[1] == kModeZero) &&
+         (sm.mode[2] == kModeRaw || sm.mode[2] == kModeZero) && S % 32 == 0;
+}
+
+template <int DT>
+__device__ __forceinline__ void decode_sub_chunk(const uint8_t* __restrict__ in, const DecodeSmem<DT>& sm, uint32_t m,
+                                                 uint32_t S, uint64_t nsub, uint64_t clo, uint8_t* __restrict__ out,
+                                                 uint32_t* status) {
+  const bool mraw = sm.mode[1] == kModeRaw, sraw = sm.mode[2] == kModeRaw;
+  for (uint64_t j = threadIdx.x; j < nsub; j += kDecodeThreads) {
+    const uint32_t sb_lo = (uint32_t)(j * S);
+    const uint32_t count = min32(S, m - sb_lo);
+    const uint32_t rec = sm.code[0] == kNoCode ? record_bytes(DT, 0) : 0;
+    const uint32_t* idx = reinterpret_cast<const uint32_t*>(in + sm.off[0] + rec);
+    const uint64_t bs_off = sm.off[0] + rec + round16(4 * nsub);
+    const uint64_t cap_bits = (sm.end[0] - bs_off) * 8;
+    const uint64_t start = __ldg(idx + j);
+    const bool exact = j + 1 < nsub;
+    const uint64_t expect = exact ? __ldg(idx + j + 1) : cap_bits;
+    int bad = (j == 0 && start != 0) || start > cap_bits || expect < start || expect > cap_bits;
+    const uint32_t* bs = reinterpret_cast<const uint32_t*>(in + bs_off);
+    const uint32_t* mwp = reinterpret_cast<const uint32_t*>(in + sm.off[1]) + (uint64_t)sb_lo * raw_width(DT, 1) / 32;
+    const uint32_t* swp = reinterpret_cast<const uint32_t*>(in + sm.off[2]) + sb_lo / 32;
+    uint8_t* dst = out + value_offset(DT, clo + sb_lo);
+    const uint32_t bw = (uint32_t)(cap_bits / 32);
+    const uint64_t st0 = bad ? 0 : start;
+    if (mraw && sraw) bad |= decode_sub_fast<DT, false, false>(sm.lut[0], bs, bw, st0, expect, exact, mwp, swp, count, dst);
+    else if (mraw) bad |= decode_sub_fast<DT, false, true>(sm.lut[0], bs, bw, st0, expect, exact, mwp, nullptr, count, dst);
+    else if (sraw) bad |= decode_sub_fast<DT, true, false>(sm.lut[0], bs, bw, st0, expect, exact, nullptr, swp, count, dst);
+    else bad |= decode_sub_fast<DT, true, true>(sm.lut[0], bs, bw, st0, expect, exact, nullptr, nullptr, count, dst);
+    if (bad) set_status(status, kStCorrupt);
+  }
+}
+
+// FP32 chunks with a HUFF exponent stream and RAW or ZERO byte planes (fp32_fast_ok):
+// one sub-block per thread per pass through decode_fp32_fast.
+__device__ __forceinline__ bool fp32_fast_ok(const DecodeSmem<kFP32>& sm) {
+  if (sm.mode[0] != kModeHuff) return false;
+  for (int s = 1; s < 4; s++)
+    if (sm.mode[s] != kModeRaw && sm.mode[s] != kModeZero) return false;
+  return true;
+}
+
+__device__ __forceinline__ void decode_fp32_chunk(const uint8_t* __restrict__ in, const DecodeSmem<kFP32>& sm,
+                                                  uint32_t m, uint32_t S, uint64_t nsub, uint64_t clo,
+                                                  uint8_t* __restrict__ out, uint32_t* status) {
+  for (uint64_t j = threadIdx.x; j < nsub; j += kDecodeThreads) {
+    const uint32_t sb_lo = (uint32_t)(j * S);
+    const uint32_t count = min32(S, m - sb_lo);
+    const uint32_t rec = sm.code[0] == kNoCode ? record_bytes(kFP32, 0) : 0;
+    const uint32_t* idx = reinterpret_cast<const uint32_t*>(in + sm.off[0] + rec);
+    const uint64_t bs_off = sm.off[0] + rec + round16(4 * nsub);
+    const uint64_t cap_bits = (sm.end[0] - bs_off) * 8;
+    const uint64_t start = __ldg(idx + j);
+    const bool exact = j + 1 < nsub;
+    const uint64_t expect = exact ? __ldg(idx + j + 1) : cap_bits;
+    int bad = (j == 0 && start != 0) || start > cap_bits || expect < start || expect > cap_bits;
+    const uint8_t* pl[3];
+#pragma unroll
+    for (int k = 0; k < 3; k++) pl[k] = sm.mode[k + 1] == kModeRaw ? in + sm.off[k + 1] + sb_lo : nullptr;
+    bad |= decode_fp32_fast(sm.lut[0], reinterpret_cast<const uint32_t*>(in + bs_off), (uint32_t)(cap_bits / 32),
+                            bad ? 0 : start, expect, exact, pl[0], pl[1], pl[2], count,
+                            out + value_offset(kFP32, clo + sb_lo));
+    if (bad) set_status(status, kStCorrupt);
+  }
+}
 
 // Every chunk the staged BF16 path does not take (FP32, FP8, FP4; BF16 with a RAW
 // exponent stream, a bitstream over 56 KB, or a ZRUN plane of more than 4096 blocks): one
@@ -1106,17 +1342,23 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
       return;
     }
   }
-  // the other cases: one sub-block per thread per pass. For BF16 (a rare fallback) in a
-  // function of its own, so that its register needs do not weigh on the staged path
-  // above; the other types have no staged path and keep it inline (their table reads stay
-  // shared-memory loads)
-  if constexpr (DT == kBF16) decode_generic_apart<DT>(in, sm, m, S, nsub, clo, out, status);
-  else decode_generic<DT>(in, sm, m, S, nsub, clo, out, status);
+  // FP8, FP4 and FP32 chunks of the common stream modes take their fast paths; the other
+  // cases (a rare fallback) go one sub-block per thread per pass through every stream's
+  // own reader, in a function of its own so that its register needs do not weigh on the
+  // main paths
+  if constexpr (DT == kFP8 || DT == kFP4) {
+    if (sub_fast_ok(sm, S)) decode_sub_chunk<DT>(in, sm, m, S, nsub, clo, out, status);
+    else decode_generic_apart<DT>(in, sm, m, S, nsub, clo, out, status);
+  } else if constexpr (DT == kFP32) {
+    if (fp32_fast_ok(sm)) decode_fp32_chunk(in, sm, m, S, nsub, clo, out, status);
+    else decode_generic_apart<DT>(in, sm, m, S, nsub, clo, out, status);
+  } else {
+    decode_generic_apart<DT>(in, sm, m, S, nsub, clo, out, status);
+  }
 }
 
-// Blocks per SM the decode kernels are built for: three (24 warps) where the registers
-// allow it without spilling; FP32's four readers need two.
-constexpr int decode_blocks_per_sm(int dt) { return dt == kFP32 ? 2 : 3; }
+// Blocks per SM the decode kernels are built for: three (24 warps).
+constexpr int decode_blocks_per_sm(int) { return 3; }
 
 template <int DT>
 __global__ void __launch_bounds__(kDecodeThreads, decode_blocks_per_sm(DT))

@@ -164,6 +164,9 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
   // counters: one per (bin, lane); FP8 and FP4 count the joint (exponent, mantissa) bin,
   // exponent * A1 + mantissa, so one shared atomic counts both entropy streams
   constexpr int AJ = NE > 1 ? A0 * A1 : A0;
+  // FP8: the joint bin is the byte's low 7 bits. FP4 counts byte pairs of values (the two
+  // joint bins of a byte, 64 counters), whose sums give the joint bins.
+  constexpr int AC = DT == kFP4 ? AJ * AJ : AJ;
   extern __shared__ __align__(16) uint8_t smem_raw[];  // histogram columns, then the code builder
   uint32_t* sh = reinterpret_cast<uint32_t*>(smem_raw);
   __shared__ int s_last;
@@ -172,7 +175,7 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
   constexpr int NBP = n_byte_planes(DT) > 0 ? n_byte_planes(DT) : 1;
   __shared__ uint32_t s_zbits[NBP][32];
   const int tid = threadIdx.x, lane = tid & 31;
-  for (int i = tid; i < AJ * 32; i += kHistThreads) sh[i] = 0;
+  for (int i = tid; i < AC * 32; i += kHistThreads) sh[i] = 0;
   if (tid < NBP * 32) s_zbits[tid / 32][tid % 32] = 0;
   __syncthreads();
   const uint32_t c = blockIdx.x / slices, sl = blockIdx.x % slices;
@@ -191,14 +194,41 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
     const int cnt = v0 < hi ? (int)min32(NV, hi - v0) : 0;
     if (cnt > 0) {
       RawValues<DT, NV> raw;
-      load_values<DT, NV>(src + value_offset(DT, clo + v0), cnt, raw);
+      const uint8_t* vp = src + value_offset(DT, clo + v0);
+      constexpr int W = RawValues<DT, NV>::kWords;
+      if (W % 8 == 0 && cnt == NV && (reinterpret_cast<uintptr_t>(vp) & 31) == 0) {
 #pragma unroll
-      for (int i = 0; i < NV; i++) {
-        if (i < cnt) {
-          const uint32_t bin = NE > 1 ? symbol<DT, NV>(raw, 0, i) * A1 + symbol<DT, NV>(raw, 1, i)
-                                      : symbol<DT, NV>(raw, 0, i);
-          atomicAdd(col0 + bin * 32, 1u);
+        for (int j = 0; j < W / 8; j++) ld_nc_v8(vp + 32 * j, raw.w + 8 * j);
+      } else {
+        load_values<DT, NV>(vp, cnt, raw);
+      }
+      if constexpr (DT == kFP8 || DT == kFP4) {
+        // counter (bin, lane) at byte bin << 7 | lane << 2: FP8 bin = byte & 0x7F (exponent
+        // bits 6..3, mantissa 2..0); FP4 bin = (low nibble & 7) | (high nibble & 7) << 3
+        uint8_t* const tab = reinterpret_cast<uint8_t*>(sh);
+        const uint32_t l4 = (uint32_t)lane << 2;
+        const int nbytes = DT == kFP8 ? cnt : cnt / 2;  // FP4: cnt is even
+#pragma unroll
+        for (int j = 0; j < RawValues<DT, NV>::kWords; j++) {
+          const uint32_t x = raw.w[j];
+#pragma unroll
+          for (int k = 0; k < 4; k++) {
+            if (4 * j + k < nbytes) {
+              uint32_t off;
+              if constexpr (DT == kFP8) {
+                off = k == 0 ? (x << 7) & 0x3F80u : (x >> (8 * k - 7)) & 0x3F80u;
+              } else {
+                const uint32_t b = x >> (8 * k);
+                off = ((b << 7) & 0x380u) | ((b << 6) & 0x1C00u);
+              }
+              atomicAdd(reinterpret_cast<uint32_t*>(tab + (off | l4)), 1u);
+            }
+          }
         }
+      } else {
+#pragma unroll
+        for (int i = 0; i < NV; i++)
+          if (i < cnt) atomicAdd(col0 + symbol<DT, NV>(raw, 0, i) * 32, 1u);
       }
       if constexpr (DT == kFP32) {
         // every stream is a bit field of the value, so the OR of my words holds the OR of
@@ -257,16 +287,28 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
     }
   } else {
     // joint bins, then each stream's counts as sums over the other stream's symbols
-    uint32_t* joint = sh + AJ * 32;
-    for (int b = tid; b < AJ; b += kHistThreads) {
+    uint32_t* csum = sh + AC * 32;
+    uint32_t* joint = csum + (AC > AJ ? AC : 0);
+    for (int b = tid; b < AC; b += kHistThreads) {
       uint32_t sum = 0;
 #pragma unroll 8
       for (int l = 0; l < 32; l++) sum += sh[b * 32 + ((l + b) & 31)];
-      joint[b] = sum;
-      // the slice is encode tile sl of the chunk: its joint counts give its bit offsets
-      if (ws.tile_hist) ws.tile_hist[((uint64_t)c * g.tiles_per_chunk + sl) * AJ + b] = (uint16_t)sum;
+      csum[b] = sum;
+    }
+    if constexpr (AC > AJ) {
+      // FP4: bin x counts the pairs with x first plus the pairs with x second
+      __syncthreads();
+      for (int x = tid; x < AJ; x += kHistThreads) {
+        uint32_t sum = 0;
+        for (int y = 0; y < AJ; y++) sum += csum[x | (y << 3)] + csum[y | (x << 3)];
+        joint[x] = sum;
+      }
     }
     __syncthreads();
+    // the slice is encode tile sl of the chunk: its joint counts give its bit offsets
+    if (ws.tile_hist)
+      for (int b = tid; b < AJ; b += kHistThreads)
+        ws.tile_hist[((uint64_t)c * g.tiles_per_chunk + sl) * AJ + b] = (uint16_t)joint[b];
     for (int t = tid; t < A0 + A1; t += kHistThreads) {
       uint32_t sum = 0;
       if (t < A0) {
@@ -709,7 +751,8 @@ static cudaError_t split_hist_t(const void* src, const Geo& g, uint32_t* hist, u
   if (blocks > 0x7FFFFFFFull) return cudaErrorInvalidConfiguration;
   constexpr int NE = n_entropy(DT);
   constexpr size_t AJ = NE > 1 ? (size_t)alphabet(DT, 0) * alphabet(DT, 1) : (size_t)alphabet(DT, 0);
-  constexpr size_t cols = (AJ * 32 + (NE > 1 ? AJ : 0)) * 4;  // counters (+ the joint sums)
+  constexpr size_t AC = DT == kFP4 ? AJ * AJ : AJ;          // FP4 counts byte pairs
+  constexpr size_t cols = (AC * 32 + (NE > 1 ? AC + AJ : 0)) * 4;  // counters (+ their sums, the joint bins)
   const size_t smem = ws ? (sizeof(HuffBlockSmem) > cols ? sizeof(HuffBlockSmem) : cols) : cols;
   const cudaError_t e = allow_smem(k_split_hist<DT>, sizeof(HuffBlockSmem) > cols ? sizeof(HuffBlockSmem) : cols, 4 + DT);
   if (e != cudaSuccess) return e;

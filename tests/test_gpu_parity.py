@@ -527,3 +527,28 @@ def test_input_16_byte_aligned_only(z, orc, name):
     assert np.array_equal(cont, ref)
     y = z.decompress(torch.from_numpy(ref).cuda(), x.dtype, n)
     assert torch.equal(y.view(torch.uint8).cpu(), torch.from_numpy(_host_bytes(x[shift:shift + n]).copy()))
+
+
+@pytest.mark.parametrize("dtype", ["fp8_e4m3", "fp4_e2m1"])
+def test_sub_byte_stream_modes(z, orc, dtype):
+    """FP8 and FP4 chunks whose mantissa or sign stream is ZERO (non-negative values;
+    values with a zero mantissa), whose counts end inside a 32-value step, and whose
+    sub-block size is not a multiple of 32 (the decode's other path): every container the
+    oracle's, every decode exact."""
+    from lossless_float_weight_b200 import workloads as W
+    if dtype == "fp8_e4m3":
+        q = W.fp8_tensor(rows=80, cols=4096, seed=5).reshape(-1)
+        b = q.view(torch.uint8)
+        cases = {"no sign": (b & 0x7F), "no mantissa": (b & 0xF8), "neither": (b & 0x78), "as is": b}
+        mk = lambda t: t.contiguous().view(torch.float8_e4m3fn)
+    else:
+        q = W.fp4_tensor(rows=80, cols=2048, seed=5).reshape(-1)
+        b = q.view(torch.uint8)
+        cases = {"no sign": (b & 0x77), "no mantissa": (b & 0xEE), "neither": (b & 0x66), "as is": b}
+        mk = lambda t: t.contiguous().view(torch.float4_e2m1fn_x2)
+    for name, t in cases.items():
+        x = mk(t)
+        _check_roundtrip(z, orc, x, f"{dtype} {name}", chunk_bytes=65536)
+        cut = mk(t[: t.numel() - 2 * 37])  # counts that end inside a step
+        _check_roundtrip(z, orc, cut, f"{dtype} {name} ragged", chunk_bytes=65536, subblock=512)
+        _check_roundtrip(z, orc, cut, f"{dtype} {name} S=48", chunk_bytes=65536, subblock=48)
