@@ -283,8 +283,8 @@ zipnn_status zipnn_compress_noalloc(zipnn_dtype dtype, const void* src, uint64_t
                                     size_t out_cap, zipnn_stream_t stream);
 
 /* Test aid (not a step of the codec): the number of polls after which a wait on another
- * block of the same launch (the decoupled look-back of the layout scan and of the FP32,
- * FP8 and FP4 encode) gives up and records ZIPNN_ERR_TIMEOUT; 0 restores the default
+ * block of the same launch (the decoupled look-back of the layout scan) gives up and
+ * records ZIPNN_ERR_TIMEOUT; 0 restores the default
  * (2^22). It applies to calls made after it, in every host thread. A wait that gives up
  * has summed only part of its prefix, so every offset it yields is at most the true one
  * and every write stays inside the output; the container is then invalid and the status

@@ -7,7 +7,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libzipnn_b200.so")
-SOURCES = ["api.cu", "prelude.cu", "encode.cu", "decode.cu", "plan.cu", "timing.cu", "noalloc.cu", "encode_bf16.cu",
+SOURCES = ["api.cu", "prelude.cu", "decode.cu", "plan.cu", "timing.cu", "noalloc.cu", "encode_bf16.cu", "encode_fp32.cu",
            "encode_sub.cu", "shard.cu"]
 HEADERS = ["bulk.cuh", "common.cuh", "fields.cuh", "huffman.cuh", "launch.h"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -64,10 +64,10 @@ bool make_geo(int dt, uint64_t n, uint32_t chunk_bytes, uint32_t S, uint32_t G, 
 }
 
 struct WsPlan {
-  uint64_t status, hist, nonzero, zmap, zcount, scan_desc, tile_desc, slot, zero_end;
+  uint64_t status, hist, nonzero, zmap, zcount, scan_desc, slot, zero_end;
   uint64_t esize, emode, ecode, eoff, enc, tile_hist, tile_off;
   uint64_t km_mu, km_perm, km_assign, km_changed, km_gsum, total;
-  bool tile_counts;  // per-tile histograms and bit offsets (BF16, FP8, FP4)
+  bool tile_counts;  // per-tile histograms and bit offsets (every compress)
   int dt;
 };
 
@@ -82,7 +82,6 @@ WsPlan ws_plan(const Geo& g) {
   p.zmap = o;       o = align_up(o + C * (uint64_t)n_byte_planes(g.dt) * g.zwords * 4);
   p.zcount = o;     o = align_up(o + C * (uint64_t)n_byte_planes(g.dt) * 4);
   p.scan_desc = o;  o = align_up(o + (uint64_t)layout_tiles(g.n_entries) * 8);
-  p.tile_desc = o;  o = align_up(o + NE * g.n_tiles * 8);
   p.slot = o;       o = align_up(o + NE * g.n_tiles * 8);
   p.zero_end = o;
   p.esize = o;      o = align_up(o + K * 8);
@@ -90,7 +89,7 @@ WsPlan ws_plan(const Geo& g) {
   p.ecode = o;      o = align_up(o + K * 4);
   p.eoff = o;       o = align_up(o + K * 8);
   p.enc = o;        o = align_up(o + C * NE * 256 * 4);
-  p.tile_counts = g.dt != kFP32;
+  p.tile_counts = true;
   p.tile_hist = o;  o = align_up(o + (p.tile_counts ? (uint64_t)g.n_tiles * tile_bins(g.dt) * 2 : 0));
   p.tile_off = o;   o = align_up(o + (p.tile_counts ? NE * g.n_tiles * 4 : 0));
   p.km_mu = o;      o = align_up(o + (uint64_t)kMaxGroups * 256 * 8);
@@ -111,7 +110,6 @@ Ws carve(const WsPlan& p, void* base) {
   w.zmap = n_byte_planes(p.dt) ? reinterpret_cast<uint32_t*>(b + p.zmap) : nullptr;
   w.zcount = n_byte_planes(p.dt) ? reinterpret_cast<uint32_t*>(b + p.zcount) : nullptr;
   w.scan_desc = reinterpret_cast<uint64_t*>(b + p.scan_desc);
-  w.tile_desc = reinterpret_cast<uint64_t*>(b + p.tile_desc);
   w.slot = reinterpret_cast<uint64_t*>(b + p.slot);
   w.esize = reinterpret_cast<uint64_t*>(b + p.esize);
   w.emode = reinterpret_cast<uint32_t*>(b + p.emode);
@@ -210,7 +208,7 @@ zipnn_status zipnn_compress_ex(zipnn_dtype dtype, const void* src, uint64_t n, u
   if (e == cudaSuccess) {
     TimedLaunch t(kIdEncode, st);
     e = g.dt == kBF16 ? launch_encode_bf16(src, g, w, static_cast<uint8_t*>(out), st)
-        : g.dt == kFP32 ? launch_encode(src, g, w, static_cast<uint8_t*>(out), st)
+        : g.dt == kFP32 ? launch_encode_fp32(src, g, w, static_cast<uint8_t*>(out), st)
                         : launch_encode_sub(src, g, w, static_cast<uint8_t*>(out), st);
   }
   return cuda_status(e);

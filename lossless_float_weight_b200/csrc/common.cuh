@@ -24,21 +24,17 @@ constexpr uint32_t kMaxGroups = 64;
 // Device status codes (the public zipnn_status values).
 constexpr uint32_t kStCorrupt = 3, kStTimeout = 7;
 
-// Values per 128-bit group of one thread, groups per encode thread, values per tile.
+// Values per 128-bit group of one thread and groups per encode thread (BF16: 64 values).
 constexpr int kGroupValues = 16;
 constexpr int kEncGroups = 4;
-constexpr int kEncodeThreads = 256;
-constexpr int kTileValues = kEncodeThreads * kGroupValues * kEncGroups;  // 16384
-// BF16, FP8 and FP4: the encode tile (32768 values; the encode kernels take it in passes
-// of their own blocks) is also one histogram tile, whose counts give its bit offsets
-constexpr int kBf16EncodeThreads = 512;
-constexpr int kBf16TileValues = kBf16EncodeThreads * kGroupValues * kEncGroups;  // 32768
-__host__ __device__ constexpr uint32_t tile_values(int dt) {
-  return dt == kFP32 ? (uint32_t)kTileValues : (uint32_t)kBf16TileValues;
-}
-// Counters a tile keeps for its bit offsets: BF16 the 256 exponents; FP8 and FP4 the joint
-// (exponent, mantissa) bins, exponent * mantissa alphabet + mantissa (FP8 16 x 8, FP4 4 x 2).
-__host__ __device__ constexpr uint32_t tile_bins(int dt) { return dt == kBF16 ? 256u : dt == kFP8 ? 128u : dt == kFP4 ? 8u : 0u; }
+// The encode tile (32768 values; the encode kernels take it in passes of their own
+// blocks) is also one histogram tile, whose counts give its bit offsets.
+constexpr int kBf16TileValues = 32768;
+__host__ __device__ constexpr uint32_t tile_values(int) { return (uint32_t)kBf16TileValues; }
+// Counters a tile keeps for its bit offsets: BF16 and FP32 the 256 exponents; FP8 and FP4
+// the joint (exponent, mantissa) bins, exponent * mantissa alphabet + mantissa (FP8
+// 16 x 8, FP4 4 x 2).
+__host__ __device__ constexpr uint32_t tile_bins(int dt) { return dt == kFP8 ? 128u : dt == kFP4 ? 8u : 256u; }
 
 __host__ __device__ constexpr int n_streams(int dt) { return dt == kBF16 ? 2 : dt == kFP32 ? 4 : 3; }
 // FP8 and FP4 entropy-code exponent and mantissa independently
@@ -107,16 +103,15 @@ struct Ws {
                         // 32w + i of the plane holds a non-zero byte
   uint32_t* zcount;     // [n_chunks][n_byte_planes]: blocks set in zmap
   uint64_t* scan_desc;  // [layout tiles] look-back descriptors
-  uint64_t* tile_desc;  // [n_tiles][n_entropy] look-back descriptors
   uint64_t* slot;       // [n_tiles][n_entropy] shared boundary words
   uint64_t* esize;      // [n_entries] payload bytes
   uint32_t* emode;      // [n_entries]
   uint32_t* ecode;      // [n_entries]
   uint64_t* eoff;       // [n_entries] payload offsets
   uint32_t* enc;        // [n_chunks][n_entropy][256]: len << 16 | code
-  uint16_t* tile_hist;  // [n_tiles][tile_bins] (BF16, FP8, FP4 compress): counts of each encode tile
-  uint32_t* tile_off;   // [n_entropy][n_tiles] (BF16, FP8, FP4 compress): bit offset of each tile
-                        // in its chunk's bitstream of that entropy stream
+  uint16_t* tile_hist;  // [n_tiles][tile_bins] (compress): counts of each encode tile
+  uint32_t* tile_off;   // [n_entropy][n_tiles] (compress): bit offset of each tile in its
+                        // chunk's bitstream of that entropy stream
 };
 
 // Device-side tables of a plan.

@@ -1,6 +1,6 @@
 // encode_bf16.cu -- k_encode_bf16: the encode of BF16 tensors.
 //
-// The same output as k_encode (encode.cu), with no wait between blocks. A tile is
+// The container bytes the oracle writes for a BF16 tensor, with no wait between blocks. A tile is
 // 32768 consecutive values of one chunk (one histogram tile); its exponent
 // bits start, inside the chunk's bitstream, at the sum over the chunk's lower tiles of
 // count(tile, e) * len(e). The histogram pass counts per tile and the code build turns
@@ -323,6 +323,7 @@ __global__ void __launch_bounds__(kBThreads, 8) k_encode_bf16(const uint8_t* __r
         for (uint64_t i = nsub + tid; i < idx_bytes / 4; i += kBThreads) idx[i] = 0;
       }
     }
+    __syncthreads();  // the tile's bitmap words are read before the next tile's setup
   }
 }
 

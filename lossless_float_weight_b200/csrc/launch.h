@@ -36,9 +36,10 @@ cudaError_t launch_code_lengths(const uint64_t* hist, uint32_t count, uint32_t a
                                 uint32_t* enc, cudaStream_t st);
 cudaError_t launch_layout(const Geo& g, const Ws& ws, const PlanDev& plan, uint8_t* out, cudaStream_t st);
 uint32_t layout_tiles(uint32_t n_entries);
-cudaError_t launch_encode(const void* src, const Geo& g, const Ws& ws, uint8_t* out, cudaStream_t st);
 // BF16 encode: persistent blocks, tile bit offsets from the per-tile histograms.
 cudaError_t launch_encode_bf16(const void* src, const Geo& g, const Ws& ws, uint8_t* out, cudaStream_t st);
+// FP32 encode: the same scheme with three byte planes.
+cudaError_t launch_encode_fp32(const void* src, const Geo& g, const Ws& ws, uint8_t* out, cudaStream_t st);
 // FP8 and FP4 encode: the same scheme, with grouped code tables and bit-parallel packing.
 cudaError_t launch_encode_sub(const void* src, const Geo& g, const Ws& ws, uint8_t* out, cudaStream_t st);
 cudaError_t launch_decode(const uint8_t* in, uint64_t in_bytes, const Geo& g, uint8_t* out, uint32_t* status,

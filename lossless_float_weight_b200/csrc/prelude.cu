@@ -24,7 +24,7 @@ constexpr int kHistThreads = 256;
 constexpr uint32_t kHistSlice = 32768;  // values of one chunk per histogram tile
 static_assert(kHistSlice == kBf16TileValues, "a BF16 histogram slice is one encode tile");
 
-// BF16 with a HUFF exponent stream: the bit offset of each encode tile in the chunk's
+// BF16 and FP32 with a HUFF exponent stream: the bit offset of each encode tile in the chunk's
 // bitstream, the running sum over the lower tiles of count(tile, e) * len(e), from the
 // per-tile counts of the histogram pass. Warp w totals tiles w, w + 8, ...; a block
 // scan turns the totals into offsets. The code builder's scratch is free by now.
@@ -108,7 +108,7 @@ __device__ void build_chunk_table(const Geo& g, const Ws& ws, const PlanDev& pla
   __syncthreads();
   uint32_t* enc = ws.enc + ((uint64_t)c * NE + e) * 256;
   decide_code(sm, A, w, record_bytes(DT, e), m, g.S, plan, e, enc, ws.emode + k, ws.ecode + k, ws.esize + k);
-  if constexpr (DT == kBF16) {
+  if constexpr (DT == kBF16 || DT == kFP32) {
     if (ws.tile_off) {
       __syncthreads();
       if (ws.emode[k] == kModeHuff) tile_offsets(g, ws, c, enc, sm);
@@ -284,6 +284,8 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
 #pragma unroll 8
       for (int l = 0; l < 32; l++) sum += sh[b * 32 + ((l + b) & 31)];
       if (sum) atomicAdd(&hist[(uint64_t)c * 256 + b], sum);
+      // the slice is encode tile sl of the chunk: its counts give its bit offset
+      if (ws.tile_hist) ws.tile_hist[((uint64_t)c * g.tiles_per_chunk + sl) * 256 + b] = (uint16_t)sum;
     }
   } else {
     // joint bins, then each stream's counts as sums over the other stream's symbols

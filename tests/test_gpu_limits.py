@@ -46,14 +46,13 @@ def _many_tiles(dtype):
     return x.to(dtype)
 
 
-@pytest.mark.parametrize("dtype,chunk_bytes", [(torch.bfloat16, 4096), (torch.float32, 262144)])
+@pytest.mark.parametrize("dtype,chunk_bytes", [(torch.bfloat16, 4096), (torch.float32, 4096)])
 def test_lookback_wait_runs_out(z, orc, dtype, chunk_bytes):
     """With a look-back limit of one poll, a wait whose predecessor has not published yet
     gives up: the call ends, the status is OK or TIMEOUT (never a fault), every write stays
     inside the output (a guard band after it stays untouched), and the process goes on.
-    BF16 with 4 KiB chunks has 3000 chunk-table entries, three layout tiles that wait on
-    each other; FP32 with 256 KiB chunks has 47 chunks of 4 encode tiles, each tile
-    waiting on the one before."""
+    With 4 KiB chunks, BF16 has 3000 chunk-table entries (three layout tiles that wait on
+    each other) and FP32 12000 (twelve)."""
     name = {torch.bfloat16: "bf16", torch.float32: "fp32"}[dtype]
     x = _many_tiles(dtype).cuda()
     n = x.numel()
