@@ -30,22 +30,25 @@ constexpr uint32_t kLutInvalid = 0x8000u;
 
 __device__ __forceinline__ uint32_t lut_symbol(uint32_t e) { return (e >> 16) & 0xFFu; }
 
-// Big-endian-within-word bit reader over 32-bit words [0, end); words past `end`
-// read as zero. buf holds nb valid bits, most significant first; the next two words
+__device__ const uint32_t kZeroWord[1] = {0};  // the word an empty stream reads
+
+// Big-endian-within-word bit reader over 32-bit words [0, nwords); a read past the last
+// word sees the last word (a valid stream never consumes those bits; one that does ends
+// past its bound and is reported). buf holds nb valid bits, most significant first; the next two words
 // are already loaded (q0, q1), so a refill never waits on memory that was requested
 // less than two refills ago.
 struct BitReader {
   const uint32_t* w;
-  uint32_t pos, end;  // pos: next word to request
+  uint32_t pos, last;  // pos: next word to request; last: the last word a read may touch
   uint64_t buf;
   int nb;
-  uint32_t q0, q1;
-  __device__ __forceinline__ uint32_t load(uint32_t i) const { return i < end ? bswap32(__ldg(w + i)) : 0u; }
+  uint32_t q0, q1;     // the next two words as stored (byte-swapped when they enter buf)
+  __device__ __forceinline__ uint32_t load(uint32_t i) const { return __ldg(w + min(i, last)); }
   __device__ __forceinline__ void init(const uint32_t* words, uint32_t nwords, uint64_t bit) {
-    w = words;
-    end = nwords;
+    w = nwords ? words : kZeroWord;
+    last = nwords ? nwords - 1 : 0;
     const uint32_t p0 = (uint32_t)(bit >> 5);
-    buf = (uint64_t)load(p0) << 32;
+    buf = (uint64_t)bswap32(load(p0)) << 32;
     q0 = load(p0 + 1);
     q1 = load(p0 + 2);
     pos = p0 + 3;
@@ -57,7 +60,7 @@ struct BitReader {
   }
   __device__ __forceinline__ void refill() {
     if (nb <= 32) {
-      buf |= (uint64_t)q0 << (32 - nb);
+      buf |= (uint64_t)bswap32(q0) << (32 - nb);
       nb += 32;
       q0 = q1;
       q1 = load(pos++);
@@ -288,7 +291,8 @@ __device__ __forceinline__ int decode_bf16_fast(const uint32_t* lut, const uint8
 // streams, the case of every chunk whose mantissas are near uniform: one sub-block, 32
 // values a step. The exponents come two a lookup; the step's RAW words (FP8: three
 // mantissa words and one sign word, FP4: one of each; value v's bits at v * width, so a
-// step of 32 values starts on a word) are loaded one step ahead, and their fields are
+// step of 32 values starts on a word) are requested two steps ahead and kept as loaded
+// (byte-swapped only when used, so no instruction waits on them early); their fields are
 // spread into the output bytes or nibbles with shifts, masks and multiplies. mwp / swp:
 // the sub-block's first mantissa / sign word (S is a multiple of 32), or nullptr (ZERO).
 // Returns nonzero if the stream is inconsistent.
@@ -306,13 +310,13 @@ __device__ __forceinline__ int decode_sub_fast(const uint32_t* lut, const uint32
   for (int i = 0; i < WM; i++) mc[i] = mn[i] = 0;
   if (full > 0) {
 #pragma unroll
-    for (int i = 0; i < WM; i++) mc[i] = MZ ? 0u : bswap32(__ldg(mwp + i));
-    sc = SZ ? 0u : bswap32(__ldg(swp));
+    for (int i = 0; i < WM; i++) mc[i] = MZ ? 0u : __ldg(mwp + i);
+    sc = SZ ? 0u : __ldg(swp);
   }
   if (full > 1) {
 #pragma unroll
-    for (int i = 0; i < WM; i++) mn[i] = MZ ? 0u : bswap32(__ldg(mwp + WM + i));
-    sn = SZ ? 0u : bswap32(__ldg(swp + 1));
+    for (int i = 0; i < WM; i++) mn[i] = MZ ? 0u : __ldg(mwp + WM + i);
+    sn = SZ ? 0u : __ldg(swp + 1);
   }
   for (uint32_t gi = 0; gi < full; gi++) {
     uint32_t pr[16];  // exponent pairs in bits 16..31
@@ -322,17 +326,17 @@ __device__ __forceinline__ int decode_sub_fast(const uint32_t* lut, const uint32
       pr[i] = huff_pair(br, lut, acc);
       pr[i + 1] = huff_pair(br, lut, acc);
     }
-    uint32_t M[WM], Sg = sc;
+    uint32_t M[WM], Sg = bswap32(sc);
 #pragma unroll
     for (int i = 0; i < WM; i++) {
-      M[i] = mc[i];
+      M[i] = bswap32(mc[i]);
       mc[i] = mn[i];
     }
     sc = sn;
     if (gi + 2 < full) {
 #pragma unroll
-      for (int i = 0; i < WM; i++) mn[i] = MZ ? 0u : bswap32(__ldg(mwp + (gi + 2) * WM + i));
-      sn = SZ ? 0u : bswap32(__ldg(swp + gi + 2));
+      for (int i = 0; i < WM; i++) mn[i] = MZ ? 0u : __ldg(mwp + (gi + 2) * WM + i);
+      sn = SZ ? 0u : __ldg(swp + gi + 2);
     }
     if constexpr (DT == kFP8) {
       // byte of value 4k + i: sign << 7 | exponent << 3 | mantissa
