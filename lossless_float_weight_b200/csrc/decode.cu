@@ -291,8 +291,9 @@ __device__ __forceinline__ int decode_bf16_fast(const uint32_t* lut, const uint8
 // streams, the case of every chunk whose mantissas are near uniform: one sub-block, 32
 // values a step. The exponents come two a lookup; the step's RAW words (FP8: three
 // mantissa words and one sign word, FP4: one of each; value v's bits at v * width, so a
-// step of 32 values starts on a word) are requested two steps ahead and kept as loaded
-// (byte-swapped only when used, so no instruction waits on them early); their fields are
+// step of 32 values starts on a word) are requested two steps ahead into one of two
+// register sets and kept as loaded (byte-swapped only when used, so no instruction waits
+// on them early); their fields are
 // spread into the output bytes or nibbles with shifts, masks and multiplies. mwp / swp:
 // the sub-block's first mantissa / sign word (S is a multiple of 32), or nullptr (ZERO).
 // Returns nonzero if the stream is inconsistent.
@@ -305,20 +306,17 @@ __device__ __forceinline__ int decode_sub_fast(const uint32_t* lut, const uint32
   br.init(bs, bs_words, start);
   uint32_t acc = 0;
   const uint32_t full = count / 32;
-  uint32_t mc[WM], mn[WM], sc = 0, sn = 0;  // this step's and the next step's RAW words (MSB first)
+  // the RAW words of two steps in flight, as loaded: set 0 for even steps, set 1 for odd;
+  // a set is refilled for the step two ahead right after its words are used
+  uint32_t mw[2][WM], sw[2];
+  auto fetch = [&](int k, uint32_t g) {
 #pragma unroll
-  for (int i = 0; i < WM; i++) mc[i] = mn[i] = 0;
-  if (full > 0) {
-#pragma unroll
-    for (int i = 0; i < WM; i++) mc[i] = MZ ? 0u : __ldg(mwp + i);
-    sc = SZ ? 0u : __ldg(swp);
-  }
-  if (full > 1) {
-#pragma unroll
-    for (int i = 0; i < WM; i++) mn[i] = MZ ? 0u : __ldg(mwp + WM + i);
-    sn = SZ ? 0u : __ldg(swp + 1);
-  }
-  for (uint32_t gi = 0; gi < full; gi++) {
+    for (int i = 0; i < WM; i++) mw[k][i] = MZ || g >= full ? 0u : __ldg(mwp + g * WM + i);
+    sw[k] = SZ || g >= full ? 0u : __ldg(swp + g);
+  };
+  fetch(0, 0);
+  fetch(1, 1);
+  auto step = [&](uint32_t gi, int k) {
     uint32_t pr[16];  // exponent pairs in bits 16..31
 #pragma unroll
     for (int i = 0; i < 16; i += 2) {
@@ -326,36 +324,29 @@ __device__ __forceinline__ int decode_sub_fast(const uint32_t* lut, const uint32
       pr[i] = huff_pair(br, lut, acc);
       pr[i + 1] = huff_pair(br, lut, acc);
     }
-    uint32_t M[WM], Sg = bswap32(sc);
+    uint32_t M[WM];
 #pragma unroll
-    for (int i = 0; i < WM; i++) {
-      M[i] = bswap32(mc[i]);
-      mc[i] = mn[i];
-    }
-    sc = sn;
-    if (gi + 2 < full) {
-#pragma unroll
-      for (int i = 0; i < WM; i++) mn[i] = MZ ? 0u : __ldg(mwp + (gi + 2) * WM + i);
-      sn = SZ ? 0u : __ldg(swp + gi + 2);
-    }
+    for (int i = 0; i < WM; i++) M[i] = bswap32(mw[k][i]);
+    const uint32_t Sg = bswap32(sw[k]);
+    fetch(k, gi + 2);
     if constexpr (DT == kFP8) {
       // byte of value 4k + i: sign << 7 | exponent << 3 | mantissa
       uint32_t o[8];
 #pragma unroll
-      for (int k = 0; k < 8; k++) {
-        const uint32_t ew = __byte_perm(pr[2 * k], pr[2 * k + 1], 0x7632);
-        const int a = 12 * k / 32, b = 12 * k % 32;  // the four mantissas: bits [12k, 12k + 12)
+      for (int q = 0; q < 8; q++) {
+        const uint32_t ew = __byte_perm(pr[2 * q], pr[2 * q + 1], 0x7632);
+        const int a = 12 * q / 32, b = 12 * q % 32;  // the four mantissas: bits [12q, 12q + 12)
         const uint32_t y = __funnelshift_l(a + 1 < WM ? M[a + 1 < WM ? a + 1 : 0] : 0u, M[a], b) >> 20;
-        const uint32_t mw = (y >> 9) | ((y << 2) & 0x700u) | ((y << 13) & 0x70000u) | ((y << 24) & 0x7000000u);
-        const uint32_t sw = (((Sg >> (28 - 4 * k)) & 0xFu) * 0x80402010u) & 0x80808080u;
-        o[k] = (ew << 3) | mw | sw;
+        const uint32_t mv = (y >> 9) | ((y << 2) & 0x700u) | ((y << 13) & 0x70000u) | ((y << 24) & 0x7000000u);
+        const uint32_t sv = (((Sg >> (28 - 4 * q)) & 0xFu) * 0x80402010u) & 0x80808080u;
+        o[q] = (ew << 3) | mv | sv;
       }
       uint4* d = reinterpret_cast<uint4*>(dst + (uint64_t)gi * 32);
       d[0] = make_uint4(o[0], o[1], o[2], o[3]);
       d[1] = make_uint4(o[4], o[5], o[6], o[7]);
     } else {
-      // nibble of value 8k + i (value 2j the low nibble of byte j): sign << 3 |
-      // exponent << 1 | mantissa; a byte of bits (value 8k first) spreads to bit 0 of the
+      // nibble of value 8q + i (value 2j the low nibble of byte j): sign << 3 |
+      // exponent << 1 | mantissa; a byte of bits (value 8q first) spreads to bit 0 of the
       // eight nibbles after its bits are reversed
       auto spread = [](uint32_t byte) {
         uint32_t t = __brev(byte) >> 24;
@@ -365,15 +356,19 @@ __device__ __forceinline__ int decode_sub_fast(const uint32_t* lut, const uint32
       };
       uint32_t o[4];
 #pragma unroll
-      for (int k = 0; k < 4; k++) {
-        const uint32_t e0 = __byte_perm(pr[4 * k], pr[4 * k + 1], 0x7632);
-        const uint32_t e1 = __byte_perm(pr[4 * k + 2], pr[4 * k + 3], 0x7632);
+      for (int q = 0; q < 4; q++) {
+        const uint32_t e0 = __byte_perm(pr[4 * q], pr[4 * q + 1], 0x7632);
+        const uint32_t e1 = __byte_perm(pr[4 * q + 2], pr[4 * q + 3], 0x7632);
         const uint32_t en = __byte_perm(e0 | (e0 >> 4), e1 | (e1 >> 4), 0x6420);
-        const uint32_t mb = (M[0] >> (24 - 8 * k)) & 0xFFu, sb = (Sg >> (24 - 8 * k)) & 0xFFu;
-        o[k] = (en << 1) | spread(mb) | (spread(sb) << 3);
+        const uint32_t mb = (M[0] >> (24 - 8 * q)) & 0xFFu, sb = (Sg >> (24 - 8 * q)) & 0xFFu;
+        o[q] = (en << 1) | spread(mb) | (spread(sb) << 3);
       }
       *reinterpret_cast<uint4*>(dst + (uint64_t)gi * 16) = make_uint4(o[0], o[1], o[2], o[3]);
     }
+  };
+  for (uint32_t gi = 0; gi < full; gi += 2) {
+    step(gi, 0);
+    if (gi + 1 < full) step(gi + 1, 1);
   }
   // the sub-block's last values (fewer than 32; FP4 an even number)
   auto bits_at = [](const uint32_t* p, uint32_t bit, int width) {

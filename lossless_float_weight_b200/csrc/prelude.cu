@@ -186,10 +186,10 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* _
 #pragma unroll
   for (int s = 0; s < NS; s++) nz[s] = 0;
   uint32_t* col0 = sh + lane;
-  // consecutive values per thread per pass, loaded up front: FP8 and FP4 the thread's
-  // whole share of the slice (128 bytes, four 256-bit loads in flight at once); FP32 32,
-  // one zero-run block, so that the values fit the registers
-  constexpr int NV = DT == kFP32 ? 32 : (int)(kHistSlice / kHistThreads);
+  // consecutive values per thread per pass, loaded up front (64 bytes: FP8 64 values,
+  // FP4 128, both in two 256-bit loads); FP32 32, one zero-run block, so that the values
+  // fit the registers
+  constexpr int NV = DT == kFP32 ? 32 : DT == kFP8 ? 64 : 128;
   for (uint32_t t0 = lo; t0 < hi; t0 += kHistThreads * NV) {
     const uint32_t v0 = t0 + tid * NV;
     const int cnt = v0 < hi ? (int)min32(NV, hi - v0) : 0;
