@@ -27,6 +27,7 @@ namespace zipnn {
 
 constexpr int kDecodeThreads = 256;
 constexpr uint32_t kLutInvalid = 0x8000u;
+constexpr uint32_t kQuadInvalid = 0x4000u;  // FP4 four-symbol entries: not four valid codes
 
 __device__ __forceinline__ uint32_t lut_symbol(uint32_t e) { return (e >> 16) & 0xFFu; }
 
@@ -294,17 +295,18 @@ __device__ __forceinline__ int decode_bf16_fast(const uint32_t* lut, const uint8
 // step of 32 values starts on a word) are requested two steps ahead into one of two
 // register sets and kept as loaded (byte-swapped only when used, so no instruction waits
 // on them early); their fields are
-// spread into the output bytes or nibbles with shifts, masks and multiplies. mwp / swp:
+// spread into the output bytes or nibbles with shifts, masks and multiplies. QUAD (FP4
+// exponents of at most 3 bits): four exponents a lookup. mwp / swp:
 // the sub-block's first mantissa / sign word (S is a multiple of 32), or nullptr (ZERO).
 // Returns nonzero if the stream is inconsistent.
-template <int DT, bool MZ, bool SZ>
+template <int DT, bool MZ, bool SZ, bool QUAD = false>
 __device__ __forceinline__ int decode_sub_fast(const uint32_t* lut, const uint32_t* bs, uint32_t bs_words,
                                                uint64_t start, uint64_t expect, bool exact, const uint32_t* mwp,
                                                const uint32_t* swp, uint32_t count, uint8_t* __restrict__ dst) {
   constexpr int WM = raw_width(DT, 1);  // mantissa bits: FP8 3, FP4 1
   BitReader br;
   br.init(bs, bs_words, start);
-  uint32_t acc = 0;
+  uint32_t acc = 0, qacc = 0;  // OR of the entries: single / pair lookups, four-symbol lookups
   const uint32_t full = count / 32;
   // the RAW words of two steps in flight, as loaded: set 0 for even steps, set 1 for odd;
   // a set is refilled for the step two ahead right after its words are used
@@ -317,12 +319,26 @@ __device__ __forceinline__ int decode_sub_fast(const uint32_t* lut, const uint32
   fetch(0, 0);
   fetch(1, 1);
   auto step = [&](uint32_t gi, int k) {
-    uint32_t pr[16];  // exponent pairs in bits 16..31
+    uint32_t pr[16];  // exponent pairs in bits 16..31 (QUAD: four exponents in bits 0..7 of pr[0..7])
+    if constexpr (QUAD) {
 #pragma unroll
-    for (int i = 0; i < 16; i += 2) {
-      br.refill();
-      pr[i] = huff_pair(br, lut, acc);
-      pr[i + 1] = huff_pair(br, lut, acc);
+      for (int i = 0; i < 8; i += 2) {
+        br.refill();
+#pragma unroll
+        for (int j = 0; j < 2; j++) {
+          const uint32_t e = lut[br.peek12()];
+          qacc |= e;
+          br.skip((e >> 4) & 15u);
+          pr[i + j] = e >> 24;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; i += 2) {
+        br.refill();
+        pr[i] = huff_pair(br, lut, acc);
+        pr[i + 1] = huff_pair(br, lut, acc);
+      }
     }
     uint32_t M[WM];
 #pragma unroll
@@ -357,9 +373,18 @@ __device__ __forceinline__ int decode_sub_fast(const uint32_t* lut, const uint32
       uint32_t o[4];
 #pragma unroll
       for (int q = 0; q < 4; q++) {
-        const uint32_t e0 = __byte_perm(pr[4 * q], pr[4 * q + 1], 0x7632);
-        const uint32_t e1 = __byte_perm(pr[4 * q + 2], pr[4 * q + 3], 0x7632);
-        const uint32_t en = __byte_perm(e0 | (e0 >> 4), e1 | (e1 >> 4), 0x6420);
+        uint32_t en;
+        if constexpr (QUAD) {
+          // eight 2-bit exponents (value 8q first, lowest) spread to nibbles
+          uint32_t t = pr[2 * q] | (pr[2 * q + 1] << 8);
+          t = (t | (t << 8)) & 0x00FF00FFu;
+          t = (t | (t << 4)) & 0x0F0F0F0Fu;
+          en = (t | (t << 2)) & 0x33333333u;
+        } else {
+          const uint32_t e0 = __byte_perm(pr[4 * q], pr[4 * q + 1], 0x7632);
+          const uint32_t e1 = __byte_perm(pr[4 * q + 2], pr[4 * q + 3], 0x7632);
+          en = __byte_perm(e0 | (e0 >> 4), e1 | (e1 >> 4), 0x6420);
+        }
         const uint32_t mb = (M[0] >> (24 - 8 * q)) & 0xFFu, sb = (Sg >> (24 - 8 * q)) & 0xFFu;
         o[q] = (en << 1) | spread(mb) | (spread(sb) << 3);
       }
@@ -390,7 +415,7 @@ __device__ __forceinline__ int decode_sub_fast(const uint32_t* lut, const uint32
     }
   }
   const uint64_t pos = br.position();
-  return (acc & kLutInvalid) || (exact ? pos != expect : pos > expect);
+  return (acc & kLutInvalid) || (qacc & (kLutInvalid | kQuadInvalid)) || (exact ? pos != expect : pos > expect);
 }
 
 // FP32 with a HUFF exponent stream and RAW (or ZERO: nullptr) byte planes p1 (sign and
@@ -694,6 +719,7 @@ struct DecodeSmem {
   uint64_t off_codes;
   uint32_t S, G;
   int bad, staged;
+  int quad;  // FP4 exponent stream with codes of at most 3 bits: table entries hold 4 symbols
 };
 
 // three BF16 decode blocks share an SM: 228 KB of shared memory, 1 KB reserved per block
@@ -773,10 +799,18 @@ __device__ __forceinline__ void decode_sub_chunk(const uint8_t* __restrict__ in,
     uint8_t* dst = out + value_offset(DT, clo + sb_lo);
     const uint32_t bw = (uint32_t)(cap_bits / 32);
     const uint64_t st0 = bad ? 0 : start;
-    if (mraw && sraw) bad |= decode_sub_fast<DT, false, false>(sm.lut[0], bs, bw, st0, expect, exact, mwp, swp, count, dst);
-    else if (mraw) bad |= decode_sub_fast<DT, false, true>(sm.lut[0], bs, bw, st0, expect, exact, mwp, nullptr, count, dst);
-    else if (sraw) bad |= decode_sub_fast<DT, true, false>(sm.lut[0], bs, bw, st0, expect, exact, nullptr, swp, count, dst);
-    else bad |= decode_sub_fast<DT, true, true>(sm.lut[0], bs, bw, st0, expect, exact, nullptr, nullptr, count, dst);
+    if (DT == kFP4 && sm.quad) {
+      constexpr bool Q = DT == kFP4;
+      if (mraw && sraw) bad |= decode_sub_fast<DT, false, false, Q>(sm.lut[0], bs, bw, st0, expect, exact, mwp, swp, count, dst);
+      else if (mraw) bad |= decode_sub_fast<DT, false, true, Q>(sm.lut[0], bs, bw, st0, expect, exact, mwp, nullptr, count, dst);
+      else if (sraw) bad |= decode_sub_fast<DT, true, false, Q>(sm.lut[0], bs, bw, st0, expect, exact, nullptr, swp, count, dst);
+      else bad |= decode_sub_fast<DT, true, true, Q>(sm.lut[0], bs, bw, st0, expect, exact, nullptr, nullptr, count, dst);
+    } else {
+      if (mraw && sraw) bad |= decode_sub_fast<DT, false, false>(sm.lut[0], bs, bw, st0, expect, exact, mwp, swp, count, dst);
+      else if (mraw) bad |= decode_sub_fast<DT, false, true>(sm.lut[0], bs, bw, st0, expect, exact, mwp, nullptr, count, dst);
+      else if (sraw) bad |= decode_sub_fast<DT, true, false>(sm.lut[0], bs, bw, st0, expect, exact, nullptr, swp, count, dst);
+      else bad |= decode_sub_fast<DT, true, true>(sm.lut[0], bs, bw, st0, expect, exact, nullptr, nullptr, count, dst);
+    }
     if (bad) set_status(status, kStCorrupt);
   }
 }
@@ -1284,10 +1318,33 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
   // (not the wide window's single-symbol one).
   if (!wide) {
     bool any = false;
+    // FP4 exponents whose codes have at most 3 bits (every Huffman code of 4 symbols): any
+    // 12-bit window holds 4 whole codes, so entry x also gets their total length (bits
+    // 4..7) and the 4 symbols (2 bits each, the first lowest, bits 24..31), read from the
+    // entries of the window shifted past each code; a window that is not 4 valid codes
+    // gets kQuadInvalid (bit 14, which no other entry's computation reads)
+    const bool quad = DT == kFP4 && sm.mode[0] == kModeHuff && sm.limit[0][3] == sm.limit[0][kLmax] &&
+                      sub_fast_ok(sm, sm.S);  // only the fast path reads four-symbol entries
+    if (tid == 0) sm.quad = quad;
 #pragma unroll
     for (int e = 0; e < NE; e++) {
       if (sm.mode[e] != kModeHuff) continue;
       any = true;
+      if (e == 0 && quad) {
+        for (uint32_t x = tid; x < 4096; x += kDecodeThreads) {
+          uint32_t total = 0, syms = 0, inval = 0;
+#pragma unroll
+          for (int k = 0; k < 4; k++) {
+            const uint32_t ek = sm.lut[0][(x << total) & 4095u];
+            inval |= ek & kLutInvalid;
+            syms |= ((ek >> 16) & 3u) << (2 * k);
+            total += ek & 15u;
+          }
+          const uint32_t e0 = sm.lut[0][x];
+          sm.lut[0][x] = (e0 & 0x00FF800Fu) | (total << 4) | (syms << 24) | (inval || total > (uint32_t)kLmax ? kQuadInvalid : 0u);
+        }
+        continue;
+      }
       for (uint32_t x = tid; x < 4096; x += kDecodeThreads) {
         const uint32_t e0 = sm.lut[e][x];
         if (e0 & kLutInvalid) continue;

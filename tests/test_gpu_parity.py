@@ -552,3 +552,28 @@ def test_sub_byte_stream_modes(z, orc, dtype):
         cut = mk(t[: t.numel() - 2 * 37])  # counts that end inside a step
         _check_roundtrip(z, orc, cut, f"{dtype} {name} ragged", chunk_bytes=65536, subblock=512)
         _check_roundtrip(z, orc, cut, f"{dtype} {name} S=48", chunk_bytes=65536, subblock=48)
+
+
+def test_fp4_plan_with_long_exponent_codes(z, orc):
+    """An FP4 plan whose exponent code has a 12-bit length (a valid prefix code, though no
+    Huffman code of four symbols has one): a 12-bit window then need not hold four whole
+    codes, so the decode takes its two-symbol table. The plan is written by hand as the
+    export format ("ZNP1", dtype, groups, two zero bytes, then the records: 4-bit lengths,
+    two symbols a byte, 16 bytes a record)."""
+    import struct
+    lens_e, lens_m = [1, 2, 3, 12], [1, 1]
+    rec_e = bytes([lens_e[0] | lens_e[1] << 4, lens_e[2] | lens_e[3] << 4]) + bytes(14)
+    rec_m = bytes([lens_m[0] | lens_m[1] << 4]) + bytes(15)
+    blob = b"ZNP1" + struct.pack("<BBH", z.FP4_E2M1, 1, 0) + rec_e + rec_m
+    plan = z.Plan.from_bytes(blob)
+    plan_lens = np.zeros((2, 1, 256), dtype=np.uint8)
+    plan_lens[0, 0, :4] = lens_e
+    plan_lens[1, 0, :2] = lens_m
+    # exponents mostly 0 and 1, one in a thousand 3: the plan's code beats RAW
+    rng = np.random.default_rng(44)
+    n = 700000
+    e = rng.choice(4, size=n, p=[0.6, 0.3, 0.099, 0.001]).astype(np.uint8)
+    nib = (e << 1) | rng.integers(0, 2, n, dtype=np.uint8) | (rng.integers(0, 2, n, dtype=np.uint8) << 3)
+    q = _fp4((nib[0::2] | (nib[1::2] << 4)).astype(np.uint8))
+    c = _check_roundtrip(z, orc, q, "fp4 long exponent code", chunk_bytes=65536, plan=plan, plan_lens=plan_lens)
+    assert c.size < 0.95 * (n // 2)  # the exponent stream is coded
