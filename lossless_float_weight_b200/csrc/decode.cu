@@ -318,7 +318,7 @@ __device__ __forceinline__ int decode_sub_fast(const uint32_t* lut, const uint32
   };
   fetch(0, 0);
   fetch(1, 1);
-  auto step = [&](uint32_t gi, int k) {
+  auto step = [&](uint32_t gi, int k, uint32_t* out16) {
     uint32_t pr[16];  // exponent pairs in bits 16..31 (QUAD: four exponents in bits 0..7 of pr[0..7])
     if constexpr (QUAD) {
 #pragma unroll
@@ -357,9 +357,14 @@ __device__ __forceinline__ int decode_sub_fast(const uint32_t* lut, const uint32
         const uint32_t sv = (((Sg >> (28 - 4 * q)) & 0xFu) * 0x80402010u) & 0x80808080u;
         o[q] = (ew << 3) | mv | sv;
       }
-      uint4* d = reinterpret_cast<uint4*>(dst + (uint64_t)gi * 32);
-      d[0] = make_uint4(o[0], o[1], o[2], o[3]);
-      d[1] = make_uint4(o[4], o[5], o[6], o[7]);
+      uint8_t* dp = dst + (uint64_t)gi * 32;
+      if ((reinterpret_cast<uintptr_t>(dp) & 31) == 0) {
+        st_v8(dp, o);
+      } else {
+        uint4* d = reinterpret_cast<uint4*>(dp);
+        d[0] = make_uint4(o[0], o[1], o[2], o[3]);
+        d[1] = make_uint4(o[4], o[5], o[6], o[7]);
+      }
     } else {
       // nibble of value 8q + i (value 2j the low nibble of byte j): sign << 3 |
       // exponent << 1 | mantissa; a byte of bits (value 8q first) spreads to bit 0 of the
@@ -388,12 +393,31 @@ __device__ __forceinline__ int decode_sub_fast(const uint32_t* lut, const uint32
         const uint32_t mb = (M[0] >> (24 - 8 * q)) & 0xFFu, sb = (Sg >> (24 - 8 * q)) & 0xFFu;
         o[q] = (en << 1) | spread(mb) | (spread(sb) << 3);
       }
-      *reinterpret_cast<uint4*>(dst + (uint64_t)gi * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+#pragma unroll
+      for (int q = 0; q < 4; q++) out16[q] = o[q];
     }
   };
   for (uint32_t gi = 0; gi < full; gi += 2) {
-    step(gi, 0);
-    if (gi + 1 < full) step(gi + 1, 1);
+    if constexpr (DT == kFP8) {
+      step(gi, 0, nullptr);
+      if (gi + 1 < full) step(gi + 1, 1, nullptr);
+    } else {
+      // FP4: the two steps' 16 bytes each go out as one 32-byte store where aligned
+      uint32_t o8[8];
+      step(gi, 0, o8);
+      uint8_t* dp = dst + (uint64_t)gi * 16;
+      if (gi + 1 < full) {
+        step(gi + 1, 1, o8 + 4);
+        if ((reinterpret_cast<uintptr_t>(dp) & 31) == 0) {
+          st_v8(dp, o8);
+        } else {
+          *reinterpret_cast<uint4*>(dp) = make_uint4(o8[0], o8[1], o8[2], o8[3]);
+          *reinterpret_cast<uint4*>(dp + 16) = make_uint4(o8[4], o8[5], o8[6], o8[7]);
+        }
+      } else {
+        *reinterpret_cast<uint4*>(dp) = make_uint4(o8[0], o8[1], o8[2], o8[3]);
+      }
+    }
   }
   // the sub-block's last values (fewer than 32; FP4 an even number)
   auto bits_at = [](const uint32_t* p, uint32_t bit, int width) {
@@ -459,9 +483,15 @@ __device__ __forceinline__ int decode_fp32_fast(const uint32_t* lut, const uint3
       o[4 * q + 2] = __byte_perm(l23, h23, 0x5410);
       o[4 * q + 3] = __byte_perm(l23, h23, 0x7632);
     }
-    uint4* d = reinterpret_cast<uint4*>(dst + (uint64_t)gi * 64);
+    uint8_t* dp = dst + (uint64_t)gi * 64;
+    if ((reinterpret_cast<uintptr_t>(dp) & 31) == 0) {
+      st_v8(dp, o);
+      st_v8(dp + 32, o + 8);
+    } else {
+      uint4* d = reinterpret_cast<uint4*>(dp);
 #pragma unroll
-    for (int q = 0; q < 4; q++) d[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+      for (int q = 0; q < 4; q++) d[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+    }
   }
   for (uint32_t v = full * 16; v < count; v++) {
     br.refill();
