@@ -539,8 +539,128 @@ __global__ void __launch_bounds__(kHistThreads) k_split_hist_bf16(const uint8_t*
   }
 }
 
-// One block per chunk: the chunk's code choice (build_chunk_table) for each entropy
-// stream, once the histogram pass is complete.
+// FP8 and FP4 compress: the histogram pass alone, in persistent blocks (each takes tiles
+// blockIdx.x, blockIdx.x + gridDim.x, ...; a tile is one 32768-value slice of a chunk): the
+// tile's joint counts (its encode-tile counts), the chunks' histograms and all-zero flags.
+// The counters and their addressing are k_split_hist's; a tile's column sums also clear
+// them for the next tile. The code builds follow in k_build_chunks, so no block waits on
+// another and none stalls its stream of tiles on a build.
+template <int DT>
+__global__ void __launch_bounds__(kHistThreads, 3) k_split_hist_tiles(const uint8_t* __restrict__ src, Geo g,
+                                                                     uint32_t* __restrict__ hist,
+                                                                     uint32_t* __restrict__ nonzero, Ws ws) {
+  static_assert(DT == kFP8 || DT == kFP4, "sub-byte types");
+  constexpr int NS = n_streams(DT), A0 = alphabet(DT, 0), A1 = alphabet(DT, 1), AJ = A0 * A1;
+  constexpr int AC = DT == kFP4 ? AJ * AJ : AJ;
+  constexpr int NV = DT == kFP8 ? 64 : 128;  // 64 bytes a thread per pass
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  uint32_t* sh = reinterpret_cast<uint32_t*>(smem_raw);
+  uint32_t* csum = sh + AC * 32;
+  uint32_t* joint = csum + (AC > AJ ? AC : 0);
+  uint8_t* const tab = reinterpret_cast<uint8_t*>(sh);
+  const int tid = threadIdx.x, lane = tid & 31;
+  const uint32_t l4 = (uint32_t)lane << 2;
+  for (int i = tid; i < AC * 32; i += kHistThreads) sh[i] = 0;
+  __syncthreads();
+  const uint32_t T = g.tiles_per_chunk;
+  for (uint32_t tile = blockIdx.x; tile < g.n_tiles; tile += gridDim.x) {
+    const uint32_t c = tile / T, sl = tile - c * T;
+    const uint64_t clo = (uint64_t)c * g.m0;
+    const uint32_t m = (uint32_t)min64(g.m0, g.n - clo);
+    const uint32_t lo = sl * kHistSlice, hi = min(lo + kHistSlice, m);
+    if (lo >= m) continue;  // past the end of a ragged last chunk (uniform)
+    uint32_t nzw = 0;  // OR of my words
+    for (uint32_t t0 = lo; t0 < hi; t0 += kHistThreads * NV) {
+      const uint32_t v0 = t0 + tid * NV;
+      const int cnt = v0 < hi ? (int)min32(NV, hi - v0) : 0;
+      if (cnt == 0) continue;
+      RawValues<DT, NV> raw;
+      const uint8_t* vp = src + value_offset(DT, clo + v0);
+      constexpr int W = RawValues<DT, NV>::kWords;
+      if (cnt == NV && (reinterpret_cast<uintptr_t>(vp) & 31) == 0) {
+#pragma unroll
+        for (int j = 0; j < W / 8; j++) ld_nc_v8(vp + 32 * j, raw.w + 8 * j);
+      } else {
+        load_values<DT, NV>(vp, cnt, raw);
+      }
+      // counter (bin, lane) at byte bin << 7 | lane << 2: FP8 bin = byte & 0x7F; FP4 bin =
+      // (low nibble & 7) | (high nibble & 7) << 3
+      const int nbytes = DT == kFP8 ? cnt : cnt / 2;  // FP4: cnt is even
+#pragma unroll
+      for (int j = 0; j < W; j++) {
+        const uint32_t x = raw.w[j];
+        nzw |= x;
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+          if (4 * j + k < nbytes) {
+            uint32_t off;
+            if constexpr (DT == kFP8) {
+              off = k == 0 ? (x << 7) & 0x3F80u : (x >> (8 * k - 7)) & 0x3F80u;
+            } else {
+              const uint32_t b = x >> (8 * k);
+              off = ((b << 7) & 0x380u) | ((b << 6) & 0x1C00u);
+            }
+            atomicAdd(reinterpret_cast<uint32_t*>(tab + (off | l4)), 1u);
+          }
+        }
+      }
+    }
+    // all-zero flags: the OR of the words folded onto the first value's bits holds every
+    // value's (values past the end load as zero)
+    {
+      uint32_t x = __reduce_or_sync(0xFFFFFFFFu, nzw);
+      x |= x >> 16;
+      x |= x >> 8;
+      if constexpr (DT == kFP4) x |= x >> 4;
+      RawValues<DT, NV> o;
+      o.w[0] = x;
+      if (nonzero && lane == 0) {
+#pragma unroll
+        for (int s = 0; s < NS; s++) {
+          const uint32_t v = symbol<DT, NV>(o, s, 0);
+          if (v) atomicOr(&nonzero[(uint64_t)c * NS + s], v);
+        }
+      }
+    }
+    __syncthreads();  // the tile's counts are complete
+    for (int b = tid; b < AC; b += kHistThreads) {
+      uint32_t sum = 0;
+#pragma unroll 8
+      for (int l = 0; l < 32; l++) {
+        const int a = b * 32 + ((l + b) & 31);
+        sum += sh[a];
+        sh[a] = 0;
+      }
+      csum[b] = sum;
+    }
+    __syncthreads();
+    if constexpr (AC > AJ) {
+      // FP4: bin x counts the pairs with x first plus the pairs with x second
+      for (int x = tid; x < AJ; x += kHistThreads) {
+        uint32_t sum = 0;
+        for (int y = 0; y < AJ; y++) sum += csum[x | (y << 3)] + csum[y | (x << 3)];
+        joint[x] = sum;
+      }
+      __syncthreads();
+    }
+    if (ws.tile_hist)
+      for (int b = tid; b < AJ; b += kHistThreads) ws.tile_hist[(uint64_t)tile * AJ + b] = (uint16_t)joint[b];
+    for (int t = tid; t < A0 + A1; t += kHistThreads) {
+      uint32_t sum = 0;
+      if (t < A0) {
+        for (int j = 0; j < A1; j++) sum += joint[t * A1 + j];
+      } else {
+        for (int e = 0; e < A0; e++) sum += joint[e * A1 + (t - A0)];
+      }
+      if (sum) atomicAdd(&hist[((uint64_t)c * 2 + (t < A0 ? 0 : 1)) * 256 + (t < A0 ? t : t - A0)], sum);
+    }
+    __syncthreads();  // the sums are read before the next tile's fold writes them
+  }
+}
+
+// One block per chunk (BF16, FP8, FP4 compress): the chunk's code choice
+// (build_chunk_table) for each entropy stream and the tiles' bit offsets, once the
+// histogram pass is complete.
 template <int DT>
 __global__ void __launch_bounds__(kHuffWarps * 32, 4) k_build_chunks(Geo g, Ws ws, PlanDev plan) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -549,6 +669,9 @@ __global__ void __launch_bounds__(kHuffWarps * 32, 4) k_build_chunks(Geo g, Ws w
   for (int e = 0; e < n_entropy(DT); e++) {
     build_chunk_table<DT>(g, ws, plan, blockIdx.x, (uint32_t)e, hs);
     __syncthreads();
+  }
+  if constexpr (n_entropy(DT) > 1) {
+    if (ws.tile_off) joint_tile_offsets<DT>(g, ws, blockIdx.x, hs);
   }
 #pragma unroll
   for (int s = 0; s < n_streams(DT); s++)
@@ -698,10 +821,10 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout(Geo g, Ws ws, PlanDev
 // ---------------------------------------------------------------- launchers
 
 // Opt a kernel into more than 48 KB of dynamic shared memory, once per device. Slots:
-// 3 k_code_lengths, 4 k_build_chunks, 4 + DT k_split_hist<DT>.
+// 3 k_code_lengths, 4 + DT k_split_hist<DT>, 8 + DT k_build_chunks<DT>.
 template <typename K>
 static cudaError_t allow_smem(K kernel, size_t bytes, int slot) {
-  static std::atomic<int> done[8][128];
+  static std::atomic<int> done[12][128];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -738,11 +861,44 @@ static cudaError_t split_hist_bf16(const void* src, const Geo& g, uint32_t* hist
   return cudaGetLastError();
 }
 
-cudaError_t launch_build_chunks(const Geo& g, const Ws& ws, const PlanDev& plan, cudaStream_t st) {
-  if (g.dt != kBF16) return cudaErrorInvalidValue;
-  const cudaError_t e = allow_smem(k_build_chunks<kBF16>, sizeof(HuffBlockSmem), 4);
+template <int DT>
+static cudaError_t build_chunks_t(const Geo& g, const Ws& ws, const PlanDev& plan, cudaStream_t st) {
+  const cudaError_t e = allow_smem(k_build_chunks<DT>, sizeof(HuffBlockSmem), 8 + DT);
   if (e != cudaSuccess) return e;
-  k_build_chunks<kBF16><<<g.n_chunks, kHuffWarps * 32, sizeof(HuffBlockSmem), st>>>(g, ws, plan);
+  k_build_chunks<DT><<<g.n_chunks, kHuffWarps * 32, sizeof(HuffBlockSmem), st>>>(g, ws, plan);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_build_chunks(const Geo& g, const Ws& ws, const PlanDev& plan, cudaStream_t st) {
+  switch (g.dt) {
+    case kBF16: return build_chunks_t<kBF16>(g, ws, plan, st);
+    case kFP8: return build_chunks_t<kFP8>(g, ws, plan, st);
+    case kFP4: return build_chunks_t<kFP4>(g, ws, plan, st);
+    default: return cudaErrorInvalidValue;  // FP32: the histogram's last block per chunk builds
+  }
+}
+
+// FP8 / FP4 compress: a persistent grid of as many histogram blocks as fit on the device.
+template <int DT>
+static cudaError_t split_hist_tiles_t(const void* src, const Geo& g, uint32_t* hist, uint32_t* nonzero, const Ws& ws,
+                                      cudaStream_t st) {
+  constexpr size_t AJ = (size_t)alphabet(DT, 0) * alphabet(DT, 1), AC = DT == kFP4 ? AJ * AJ : AJ;
+  constexpr size_t smem = (AC * 32 + AC + AJ) * 4;
+  static std::atomic<int> resident[128];  // blocks per device, once known
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  int per_device = dev >= 0 && dev < 128 ? resident[dev].load(std::memory_order_relaxed) : 0;
+  if (!per_device) {
+    int per_sm = 0, sms = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_split_hist_tiles<DT>, kHistThreads, smem);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    per_device = (per_sm > 0 ? per_sm : 1) * (sms > 0 ? sms : 1);
+    if (dev >= 0 && dev < 128) resident[dev].store(per_device, std::memory_order_relaxed);
+  }
+  const uint32_t blocks = (uint32_t)min64((uint64_t)per_device, g.n_tiles);
+  k_split_hist_tiles<DT><<<blocks, kHistThreads, smem, st>>>(static_cast<const uint8_t*>(src), g, hist, nonzero, ws);
   return cudaGetLastError();
 }
 
@@ -771,8 +927,10 @@ cudaError_t launch_split_hist(const void* src, const Geo& g, uint32_t* hist, uin
   switch (g.dt) {
     case kBF16: return split_hist_bf16(src, g, hist, nonzero, ws, plan, st);
     case kFP32: return split_hist_t<kFP32>(src, g, hist, nonzero, ws, plan, st);
-    case kFP8: return split_hist_t<kFP8>(src, g, hist, nonzero, ws, plan, st);
-    default: return split_hist_t<kFP4>(src, g, hist, nonzero, ws, plan, st);
+    case kFP8: return ws ? split_hist_tiles_t<kFP8>(src, g, hist, nonzero, *ws, st)
+                         : split_hist_t<kFP8>(src, g, hist, nonzero, ws, plan, st);
+    default: return ws ? split_hist_tiles_t<kFP4>(src, g, hist, nonzero, *ws, st)
+                       : split_hist_t<kFP4>(src, g, hist, nonzero, ws, plan, st);
   }
 }
 
