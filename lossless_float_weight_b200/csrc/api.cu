@@ -197,7 +197,7 @@ zipnn_status zipnn_compress_ex(zipnn_dtype dtype, const void* src, uint64_t n, u
     TimedLaunch t(kIdHist, st);
     e = launch_split_hist(src, g, w.hist, w.nonzero, &w, pd, st);
   }
-  if (e == cudaSuccess && g.dt != kFP32) {
+  if (e == cudaSuccess) {
     TimedLaunch t(kIdBuild, st);
     e = launch_build_chunks(g, w, pd, st);
   }

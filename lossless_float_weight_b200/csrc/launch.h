@@ -26,11 +26,11 @@ class TimedLaunch {
   cudaEvent_t start_ = nullptr, stop_ = nullptr;
 };
 
-// Histograms. With ws (compress), also the chunks' codes: for BF16, FP8 and FP4 in a
-// second kernel, launch_build_chunks; for FP32 the last block of each chunk builds them.
+// Histograms. With ws (compress), also every tile's counts (and FP32's zero-run bitmaps);
+// the chunks' codes follow in launch_build_chunks.
 cudaError_t launch_split_hist(const void* src, const Geo& g, uint32_t* hist, uint32_t* nonzero, const Ws* ws,
                               const PlanDev& plan, cudaStream_t st);
-// BF16, FP8, FP4 compress: the chunks' codes, after launch_split_hist (one block per chunk).
+// Compress: the chunks' codes and tile offsets, after launch_split_hist (one block per chunk).
 cudaError_t launch_build_chunks(const Geo& g, const Ws& ws, const PlanDev& plan, cudaStream_t st);
 cudaError_t launch_code_lengths(const uint64_t* hist, uint32_t count, uint32_t alphabet_size, uint8_t* lens,
                                 uint32_t* enc, cudaStream_t st);

@@ -539,28 +539,34 @@ __global__ void __launch_bounds__(kHistThreads) k_split_hist_bf16(const uint8_t*
   }
 }
 
-// FP8 and FP4 compress: the histogram pass alone, in persistent blocks (each takes tiles
-// blockIdx.x, blockIdx.x + gridDim.x, ...; a tile is one 32768-value slice of a chunk): the
-// tile's joint counts (its encode-tile counts), the chunks' histograms and all-zero flags.
-// The counters and their addressing are k_split_hist's; a tile's column sums also clear
-// them for the next tile. The code builds follow in k_build_chunks, so no block waits on
-// another and none stalls its stream of tiles on a build.
+// FP32, FP8 and FP4 compress: the histogram pass alone, in persistent blocks (each takes
+// tiles blockIdx.x, blockIdx.x + gridDim.x, ...; a tile is one 32768-value slice of a
+// chunk): the tile's counts (its encode-tile counts: FP32 the exponents, FP8/FP4 the joint
+// bins), the chunks' histograms and all-zero flags, and for FP32 the zero-run block bits
+// of the three fraction planes with each tile's marked count. The counters and their
+// addressing are k_split_hist's; a tile's column sums also clear them for the next tile.
+// The code builds follow in k_build_chunks, so no block waits on another and none stalls
+// its stream of tiles on a build.
 template <int DT>
 __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist_tiles(const uint8_t* __restrict__ src, Geo g,
                                                                      uint32_t* __restrict__ hist,
                                                                      uint32_t* __restrict__ nonzero, Ws ws) {
-  static_assert(DT == kFP8 || DT == kFP4, "sub-byte types");
-  constexpr int NS = n_streams(DT), A0 = alphabet(DT, 0), A1 = alphabet(DT, 1), AJ = A0 * A1;
+  constexpr bool F32 = DT == kFP32;
+  constexpr int NS = n_streams(DT), NE = n_entropy(DT);
+  constexpr int A0 = alphabet(DT, 0), A1 = NE > 1 ? alphabet(DT, 1) : 1, AJ = A0 * A1;
   constexpr int AC = DT == kFP4 ? AJ * AJ : AJ;
-  constexpr int NV = DT == kFP8 ? 64 : 128;  // 64 bytes a thread per pass
+  // values a thread per pass: FP32 32 (one zero-run block), FP8 64, FP4 128 (64 bytes)
+  constexpr int NV = F32 ? 32 : DT == kFP8 ? 64 : 128;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint32_t* sh = reinterpret_cast<uint32_t*>(smem_raw);
   uint32_t* csum = sh + AC * 32;
   uint32_t* joint = csum + (AC > AJ ? AC : 0);
   uint8_t* const tab = reinterpret_cast<uint8_t*>(sh);
+  __shared__ uint32_t s_zbits[3][32];  // FP32: the tile's zero-run block bits of each fraction plane
   const int tid = threadIdx.x, lane = tid & 31;
   const uint32_t l4 = (uint32_t)lane << 2;
   for (int i = tid; i < AC * 32; i += kHistThreads) sh[i] = 0;
+  if (tid < 96) s_zbits[tid / 32][tid % 32] = 0;
   __syncthreads();
   const uint32_t T = g.tiles_per_chunk;
   for (uint32_t tile = blockIdx.x; tile < g.n_tiles; tile += gridDim.x) {
@@ -581,37 +587,57 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist_tiles(const uint
 #pragma unroll
         for (int j = 0; j < W / 8; j++) ld_nc_v8(vp + 32 * j, raw.w + 8 * j);
       } else {
-        load_values<DT, NV>(vp, cnt, raw);
+        load_values<DT, NV>(vp, cnt, raw);  // zero past cnt
       }
-      // counter (bin, lane) at byte bin << 7 | lane << 2: FP8 bin = byte & 0x7F; FP4 bin =
-      // (low nibble & 7) | (high nibble & 7) << 3
-      const int nbytes = DT == kFP8 ? cnt : cnt / 2;  // FP4: cnt is even
+      if constexpr (F32) {
+        // counter (exponent, lane) at byte exponent << 7 | lane << 2: bits 30..23 of the
+        // value moved to 14..7; my 32 values are one zero-run block of every fraction plane
+        uint32_t a = 0;
 #pragma unroll
-      for (int j = 0; j < W; j++) {
-        const uint32_t x = raw.w[j];
-        nzw |= x;
+        for (int j = 0; j < NV; j++) {
+          if (j < cnt) atomicAdd(reinterpret_cast<uint32_t*>(tab + (((raw.w[j] >> 16) & 0x7F80u) | l4)), 1u);
+          a |= raw.w[j];
+        }
+        nzw |= a;
+        const uint32_t blk = (v0 - lo) / kZBlock;  // within the tile
+        RawValues<DT, NV> o;
+        o.w[0] = a;
 #pragma unroll
-        for (int k = 0; k < 4; k++) {
-          if (4 * j + k < nbytes) {
-            uint32_t off;
-            if constexpr (DT == kFP8) {
-              off = k == 0 ? (x << 7) & 0x3F80u : (x >> (8 * k - 7)) & 0x3F80u;
-            } else {
-              const uint32_t b = x >> (8 * k);
-              off = ((b << 7) & 0x380u) | ((b << 6) & 0x1C00u);
+        for (int s = 1; s < 4; s++)
+          if (symbol<DT, NV>(o, s, 0)) atomicOr(&s_zbits[s - 1][blk / 32], 1u << (blk % 32));
+      } else {
+        // counter (bin, lane) at byte bin << 7 | lane << 2: FP8 bin = byte & 0x7F; FP4 bin =
+        // (low nibble & 7) | (high nibble & 7) << 3
+        const int nbytes = DT == kFP8 ? cnt : cnt / 2;  // FP4: cnt is even
+#pragma unroll
+        for (int j = 0; j < W; j++) {
+          const uint32_t x = raw.w[j];
+          nzw |= x;
+#pragma unroll
+          for (int k = 0; k < 4; k++) {
+            if (4 * j + k < nbytes) {
+              uint32_t off;
+              if constexpr (DT == kFP8) {
+                off = k == 0 ? (x << 7) & 0x3F80u : (x >> (8 * k - 7)) & 0x3F80u;
+              } else {
+                const uint32_t b = x >> (8 * k);
+                off = ((b << 7) & 0x380u) | ((b << 6) & 0x1C00u);
+              }
+              atomicAdd(reinterpret_cast<uint32_t*>(tab + (off | l4)), 1u);
             }
-            atomicAdd(reinterpret_cast<uint32_t*>(tab + (off | l4)), 1u);
           }
         }
       }
     }
-    // all-zero flags: the OR of the words folded onto the first value's bits holds every
-    // value's (values past the end load as zero)
+    // all-zero flags: every stream is a bit field, so the OR of the words (FP8/FP4 folded
+    // onto the first value's bits) holds the OR of each stream's symbols
     {
       uint32_t x = __reduce_or_sync(0xFFFFFFFFu, nzw);
-      x |= x >> 16;
-      x |= x >> 8;
-      if constexpr (DT == kFP4) x |= x >> 4;
+      if constexpr (!F32) {
+        x |= x >> 16;
+        x |= x >> 8;
+        if constexpr (DT == kFP4) x |= x >> 4;
+      }
       RawValues<DT, NV> o;
       o.w[0] = x;
       if (nonzero && lane == 0) {
@@ -622,7 +648,7 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist_tiles(const uint
         }
       }
     }
-    __syncthreads();  // the tile's counts are complete
+    __syncthreads();  // the tile's counts and bitmaps are complete
     for (int b = tid; b < AC; b += kHistThreads) {
       uint32_t sum = 0;
 #pragma unroll 8
@@ -632,6 +658,18 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist_tiles(const uint
         sh[a] = 0;
       }
       csum[b] = sum;
+    }
+    if constexpr (F32) {
+      if (ws.zmap && tid < 96) {
+        // the tile's bitmap words of each plane (plain stores; no other tile holds them),
+        // their marked blocks into the chunk's count; then cleared
+        const int p = tid / 32, wl = tid % 32;
+        const uint32_t word = s_zbits[p][wl], wi = sl * 32u + (uint32_t)wl;
+        if (wi < g.zwords) ws.zmap[((uint64_t)c * 3 + p) * g.zwords + wi] = word;
+        const uint32_t marked = __reduce_add_sync(0xFFFFFFFFu, __popc(word));
+        if (wl == 0 && marked) atomicAdd(ws.zcount + (uint64_t)c * 3 + p, marked);
+        s_zbits[p][wl] = 0;
+      }
     }
     __syncthreads();
     if constexpr (AC > AJ) {
@@ -645,20 +683,25 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist_tiles(const uint
     }
     if (ws.tile_hist)
       for (int b = tid; b < AJ; b += kHistThreads) ws.tile_hist[(uint64_t)tile * AJ + b] = (uint16_t)joint[b];
-    for (int t = tid; t < A0 + A1; t += kHistThreads) {
-      uint32_t sum = 0;
-      if (t < A0) {
-        for (int j = 0; j < A1; j++) sum += joint[t * A1 + j];
-      } else {
-        for (int e = 0; e < A0; e++) sum += joint[e * A1 + (t - A0)];
+    if constexpr (F32) {
+      for (int b = tid; b < A0; b += kHistThreads)
+        if (joint[b]) atomicAdd(&hist[(uint64_t)c * 256 + b], joint[b]);
+    } else {
+      for (int t = tid; t < A0 + A1; t += kHistThreads) {
+        uint32_t sum = 0;
+        if (t < A0) {
+          for (int j = 0; j < A1; j++) sum += joint[t * A1 + j];
+        } else {
+          for (int e = 0; e < A0; e++) sum += joint[e * A1 + (t - A0)];
+        }
+        if (sum) atomicAdd(&hist[((uint64_t)c * 2 + (t < A0 ? 0 : 1)) * 256 + (t < A0 ? t : t - A0)], sum);
       }
-      if (sum) atomicAdd(&hist[((uint64_t)c * 2 + (t < A0 ? 0 : 1)) * 256 + (t < A0 ? t : t - A0)], sum);
     }
     __syncthreads();  // the sums are read before the next tile's fold writes them
   }
 }
 
-// One block per chunk (BF16, FP8, FP4 compress): the chunk's code choice
+// One block per chunk (compress): the chunk's code choice
 // (build_chunk_table) for each entropy stream and the tiles' bit offsets, once the
 // histogram pass is complete.
 template <int DT>
@@ -872,17 +915,18 @@ static cudaError_t build_chunks_t(const Geo& g, const Ws& ws, const PlanDev& pla
 cudaError_t launch_build_chunks(const Geo& g, const Ws& ws, const PlanDev& plan, cudaStream_t st) {
   switch (g.dt) {
     case kBF16: return build_chunks_t<kBF16>(g, ws, plan, st);
+    case kFP32: return build_chunks_t<kFP32>(g, ws, plan, st);
     case kFP8: return build_chunks_t<kFP8>(g, ws, plan, st);
-    case kFP4: return build_chunks_t<kFP4>(g, ws, plan, st);
-    default: return cudaErrorInvalidValue;  // FP32: the histogram's last block per chunk builds
+    default: return build_chunks_t<kFP4>(g, ws, plan, st);
   }
 }
 
-// FP8 / FP4 compress: a persistent grid of as many histogram blocks as fit on the device.
+// FP32 / FP8 / FP4 compress: a persistent grid of as many histogram blocks as fit on the device.
 template <int DT>
 static cudaError_t split_hist_tiles_t(const void* src, const Geo& g, uint32_t* hist, uint32_t* nonzero, const Ws& ws,
                                       cudaStream_t st) {
-  constexpr size_t AJ = (size_t)alphabet(DT, 0) * alphabet(DT, 1), AC = DT == kFP4 ? AJ * AJ : AJ;
+  constexpr size_t AJ = (size_t)alphabet(DT, 0) * (n_entropy(DT) > 1 ? alphabet(DT, 1) : 1);
+  constexpr size_t AC = DT == kFP4 ? AJ * AJ : AJ;
   constexpr size_t smem = (AC * 32 + AC + AJ) * 4;
   static std::atomic<int> resident[128];  // blocks per device, once known
   int dev = 0;
@@ -898,6 +942,7 @@ static cudaError_t split_hist_tiles_t(const void* src, const Geo& g, uint32_t* h
     if (dev >= 0 && dev < 128) resident[dev].store(per_device, std::memory_order_relaxed);
   }
   const uint32_t blocks = (uint32_t)min64((uint64_t)per_device, g.n_tiles);
+  static_assert(smem <= 48 * 1024, "the default dynamic shared memory suffices");
   k_split_hist_tiles<DT><<<blocks, kHistThreads, smem, st>>>(static_cast<const uint8_t*>(src), g, hist, nonzero, ws);
   return cudaGetLastError();
 }
@@ -926,7 +971,8 @@ cudaError_t launch_split_hist(const void* src, const Geo& g, uint32_t* hist, uin
                               const PlanDev& plan, cudaStream_t st) {
   switch (g.dt) {
     case kBF16: return split_hist_bf16(src, g, hist, nonzero, ws, plan, st);
-    case kFP32: return split_hist_t<kFP32>(src, g, hist, nonzero, ws, plan, st);
+    case kFP32: return ws ? split_hist_tiles_t<kFP32>(src, g, hist, nonzero, *ws, st)
+                          : split_hist_t<kFP32>(src, g, hist, nonzero, ws, plan, st);
     case kFP8: return ws ? split_hist_tiles_t<kFP8>(src, g, hist, nonzero, *ws, st)
                          : split_hist_t<kFP8>(src, g, hist, nonzero, ws, plan, st);
     default: return ws ? split_hist_tiles_t<kFP4>(src, g, hist, nonzero, *ws, st)
