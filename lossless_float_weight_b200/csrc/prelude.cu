@@ -1,13 +1,13 @@
 // prelude.cu -- the compress steps before encoding:
-//   k_split_hist_bf16 (BF16) / k_split_hist (FP32, FP8, FP4): byte-plane split +
+//   k_split_hist_bf16 (BF16) / k_split_hist_tiles (FP32, FP8, FP4): byte-plane split +
 //                    order-0 histogram per chunk (per-lane shared-memory counters) +
-//                    all-zero detection per chunk stream; BF16 also keeps the counts
-//                    of each encode tile;
-//   code build     : per chunk and entropy stream a shared group code or a local
-//                    length-limited Huffman code, then HUFF / RAW / ZERO. BF16:
-//                    k_build_chunks, one block per chunk after the histogram pass
-//                    (it also turns the tile counts into tile bit offsets); the other
-//                    types: the histogram block that finishes a chunk last;
+//                    all-zero detection per chunk stream, in persistent blocks; in a
+//                    compress also the counts of each encode tile (and the zero-run
+//                    block bitmaps of the byte planes);
+//   k_build_chunks : one block per chunk after the histogram pass: per entropy stream a
+//                    shared group code or a local length-limited Huffman code, then
+//                    HUFF / RAW / ZERO (ZRUN for byte planes), and the tiles' bit offsets
+//                    from their counts;
 //   k_layout       : exclusive scan of payload sizes (single-pass decoupled look-back)
 //                    into payload offsets; writes header, chunk table, shared records.
 #include <atomic>
@@ -22,7 +22,7 @@ namespace zipnn {
 
 constexpr int kHistThreads = 256;
 constexpr uint32_t kHistSlice = 32768;  // values of one chunk per histogram tile
-static_assert(kHistSlice == kBf16TileValues, "a BF16 histogram slice is one encode tile");
+static_assert(kHistSlice == kBf16TileValues, "a histogram slice is one encode tile");
 
 // BF16 and FP32 with a HUFF exponent stream: the bit offset of each encode tile in the chunk's
 // bitstream, the running sum over the lower tiles of count(tile, e) * len(e), from the
@@ -147,216 +147,6 @@ __device__ void joint_tile_offsets(const Geo& g, const Ws& ws, uint32_t c, HuffB
       if (t < T) ws.tile_off[(uint64_t)e * g.n_tiles + (uint64_t)c * T + t] = carry + before;
       carry += total;
     }
-  }
-}
-
-// THEORY-599 note, "Order-0 only (section III-A b)": the model of a chunk is the count
-// of each symbol. The block keeps one counter per (symbol, lane) in shared memory, so
-// the 32 lanes of a warp always add into 32 different banks (lane l owns column l);
-// warps share the table through shared atomics. The columns are summed at the end.
-// FP32, FP8 and FP4 (BF16 has k_split_hist_bf16 below).
-template <int DT>
-__global__ void __launch_bounds__(kHistThreads, 3) k_split_hist(const uint8_t* __restrict__ src, Geo g, uint32_t slices,
-                                                             uint32_t* __restrict__ hist, uint32_t* __restrict__ nonzero,
-                                                             Ws ws, PlanDev plan, int build) {
-  constexpr int NS = n_streams(DT), NE = n_entropy(DT);
-  constexpr int A0 = alphabet(DT, 0), A1 = NE > 1 ? alphabet(DT, 1) : 0;
-  // counters: one per (bin, lane); FP8 and FP4 count the joint (exponent, mantissa) bin,
-  // exponent * A1 + mantissa, so one shared atomic counts both entropy streams
-  constexpr int AJ = NE > 1 ? A0 * A1 : A0;
-  // FP8: the joint bin is the byte's low 7 bits. FP4 counts byte pairs of values (the two
-  // joint bins of a byte, 64 counters), whose sums give the joint bins.
-  constexpr int AC = DT == kFP4 ? AJ * AJ : AJ;
-  extern __shared__ __align__(16) uint8_t smem_raw[];  // histogram columns, then the code builder
-  uint32_t* sh = reinterpret_cast<uint32_t*>(smem_raw);
-  __shared__ int s_last;
-  // FP32: the slice's zero-run block bits of the three fraction planes (a slice of 32768
-  // values is 1024 blocks, 32 words a plane, words no other slice holds)
-  constexpr int NBP = n_byte_planes(DT) > 0 ? n_byte_planes(DT) : 1;
-  __shared__ uint32_t s_zbits[NBP][32];
-  const int tid = threadIdx.x, lane = tid & 31;
-  for (int i = tid; i < AC * 32; i += kHistThreads) sh[i] = 0;
-  if (tid < NBP * 32) s_zbits[tid / 32][tid % 32] = 0;
-  __syncthreads();
-  const uint32_t c = blockIdx.x / slices, sl = blockIdx.x % slices;
-  const uint64_t clo = (uint64_t)c * g.m0;
-  const uint32_t m = (uint32_t)min64(g.m0, g.n - clo);
-  const uint32_t lo = sl * kHistSlice, hi = min(lo + kHistSlice, m);
-  uint32_t nz[NS];
-#pragma unroll
-  for (int s = 0; s < NS; s++) nz[s] = 0;
-  uint32_t* col0 = sh + lane;
-  // consecutive values per thread per pass, loaded up front (64 bytes: FP8 64 values,
-  // FP4 128, both in two 256-bit loads); FP32 32, one zero-run block, so that the values
-  // fit the registers
-  constexpr int NV = DT == kFP32 ? 32 : DT == kFP8 ? 64 : 128;
-  for (uint32_t t0 = lo; t0 < hi; t0 += kHistThreads * NV) {
-    const uint32_t v0 = t0 + tid * NV;
-    const int cnt = v0 < hi ? (int)min32(NV, hi - v0) : 0;
-    if (cnt > 0) {
-      RawValues<DT, NV> raw;
-      const uint8_t* vp = src + value_offset(DT, clo + v0);
-      constexpr int W = RawValues<DT, NV>::kWords;
-      if (W % 8 == 0 && cnt == NV && (reinterpret_cast<uintptr_t>(vp) & 31) == 0) {
-#pragma unroll
-        for (int j = 0; j < W / 8; j++) ld_nc_v8(vp + 32 * j, raw.w + 8 * j);
-      } else {
-        load_values<DT, NV>(vp, cnt, raw);
-      }
-      if constexpr (DT == kFP8 || DT == kFP4) {
-        // counter (bin, lane) at byte bin << 7 | lane << 2: FP8 bin = byte & 0x7F (exponent
-        // bits 6..3, mantissa 2..0); FP4 bin = (low nibble & 7) | (high nibble & 7) << 3
-        uint8_t* const tab = reinterpret_cast<uint8_t*>(sh);
-        const uint32_t l4 = (uint32_t)lane << 2;
-        const int nbytes = DT == kFP8 ? cnt : cnt / 2;  // FP4: cnt is even
-#pragma unroll
-        for (int j = 0; j < RawValues<DT, NV>::kWords; j++) {
-          const uint32_t x = raw.w[j];
-#pragma unroll
-          for (int k = 0; k < 4; k++) {
-            if (4 * j + k < nbytes) {
-              uint32_t off;
-              if constexpr (DT == kFP8) {
-                off = k == 0 ? (x << 7) & 0x3F80u : (x >> (8 * k - 7)) & 0x3F80u;
-              } else {
-                const uint32_t b = x >> (8 * k);
-                off = ((b << 7) & 0x380u) | ((b << 6) & 0x1C00u);
-              }
-              atomicAdd(reinterpret_cast<uint32_t*>(tab + (off | l4)), 1u);
-            }
-          }
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < NV; i++)
-          if (i < cnt) atomicAdd(col0 + symbol<DT, NV>(raw, 0, i) * 32, 1u);
-      }
-      if constexpr (DT == kFP32) {
-        // every stream is a bit field of the value, so the OR of my words holds the OR of
-        // each stream's symbols: for the all-zero flags, and for my values' zero-run block
-        // (v0 / 32) of each fraction plane
-        static_assert(NV == kZBlock, "a thread's values are one zero-run block");
-        RawValues<DT, NV> o;
-        uint32_t a = 0;
-#pragma unroll
-        for (int i = 0; i < NV; i++) a |= raw.w[i];
-        o.w[0] = a;
-#pragma unroll
-        for (int s = 0; s < NS; s++) nz[s] |= symbol<DT, NV>(o, s, 0);
-        if (ws.zmap) {
-          const uint32_t blk = (v0 - lo) / kZBlock;  // within the slice
-#pragma unroll
-          for (int s = 1; s < NS; s++)
-            if (symbol<DT, NV>(o, s, 0)) atomicOr(&s_zbits[s - 1][blk / 32], 1u << (blk % 32));
-        }
-      } else {
-        // FP8 and FP4: the same bit-field argument; the OR of the words folded onto its
-        // first value (byte 0 for FP8, nibble 0 for FP4) holds the OR of every value's bits
-        uint32_t x = 0;
-#pragma unroll
-        for (int i = 0; i < RawValues<DT, NV>::kWords; i++) x |= raw.w[i];
-        x |= x >> 16;
-        x |= x >> 8;
-        if constexpr (DT == kFP4) x |= x >> 4;
-        RawValues<DT, NV> o;
-        o.w[0] = x;
-#pragma unroll
-        for (int s = 0; s < NS; s++) nz[s] |= symbol<DT, NV>(o, s, 0);
-      }
-    }
-  }
-#pragma unroll
-  for (int s = 0; s < NS; s++) {
-    const uint32_t v = __reduce_or_sync(0xFFFFFFFFu, nz[s]);
-    if (nonzero && lane == 0 && v) atomicOr(&nonzero[(uint64_t)c * NS + s], v);
-  }
-
-  __syncthreads();
-  if constexpr (n_byte_planes(DT) > 0) {
-    if (ws.zmap && tid < NBP * 32) {  // the slice's bitmap words, plain stores
-      const uint32_t wi = sl * 32u + (uint32_t)(tid % 32);
-      if (wi < g.zwords) ws.zmap[((uint64_t)c * NBP + tid / 32) * g.zwords + wi] = s_zbits[tid / 32][tid % 32];
-    }
-  }
-  // column sums: thread b reads its row starting at lane b, so a warp hits 32 banks
-  if constexpr (NE == 1) {
-    for (int b = tid; b < A0; b += kHistThreads) {
-      uint32_t sum = 0;
-#pragma unroll 8
-      for (int l = 0; l < 32; l++) sum += sh[b * 32 + ((l + b) & 31)];
-      if (sum) atomicAdd(&hist[(uint64_t)c * 256 + b], sum);
-      // the slice is encode tile sl of the chunk: its counts give its bit offset
-      if (ws.tile_hist) ws.tile_hist[((uint64_t)c * g.tiles_per_chunk + sl) * 256 + b] = (uint16_t)sum;
-    }
-  } else {
-    // joint bins, then each stream's counts as sums over the other stream's symbols
-    uint32_t* csum = sh + AC * 32;
-    uint32_t* joint = csum + (AC > AJ ? AC : 0);
-    for (int b = tid; b < AC; b += kHistThreads) {
-      uint32_t sum = 0;
-#pragma unroll 8
-      for (int l = 0; l < 32; l++) sum += sh[b * 32 + ((l + b) & 31)];
-      csum[b] = sum;
-    }
-    if constexpr (AC > AJ) {
-      // FP4: bin x counts the pairs with x first plus the pairs with x second
-      __syncthreads();
-      for (int x = tid; x < AJ; x += kHistThreads) {
-        uint32_t sum = 0;
-        for (int y = 0; y < AJ; y++) sum += csum[x | (y << 3)] + csum[y | (x << 3)];
-        joint[x] = sum;
-      }
-    }
-    __syncthreads();
-    // the slice is encode tile sl of the chunk: its joint counts give its bit offsets
-    if (ws.tile_hist)
-      for (int b = tid; b < AJ; b += kHistThreads)
-        ws.tile_hist[((uint64_t)c * g.tiles_per_chunk + sl) * AJ + b] = (uint16_t)joint[b];
-    for (int t = tid; t < A0 + A1; t += kHistThreads) {
-      uint32_t sum = 0;
-      if (t < A0) {
-        for (int j = 0; j < A1; j++) sum += joint[t * A1 + j];
-      } else {
-        for (int e = 0; e < A0; e++) sum += joint[e * A1 + (t - A0)];
-      }
-      if (sum) atomicAdd(&hist[((uint64_t)c * NE + (t < A0 ? 0 : 1)) * 256 + (t < A0 ? t : t - A0)], sum);
-    }
-  }
-  if (!build) return;
-  // the last block to finish a chunk builds that chunk's codes (its histogram is then
-  // complete), so the serial part of the code build overlaps other blocks' loads
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = atomicAdd(ws.status + 4 + c, 1u) == slices - 1;
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  HuffBlockSmem& hs = *reinterpret_cast<HuffBlockSmem*>(smem_raw);
-#pragma unroll
-  for (int e = 0; e < NE; e++) {
-    build_chunk_table<DT>(g, ws, plan, c, (uint32_t)e, hs);
-    __syncthreads();
-  }
-  if constexpr (NE > 1) {
-    if (ws.tile_off) joint_tile_offsets<DT>(g, ws, c, hs);
-  }
-#pragma unroll
-  for (int s = 0; s < NS; s++) {
-    if (!is_byte_plane(DT, s)) continue;
-    // the plane's marked blocks: every block's bit is final (this is the chunk's last block)
-    const uint64_t plane = (uint64_t)c * n_byte_planes(DT) + (s - 1);
-    uint32_t cnt = 0;
-    for (uint32_t w = tid; w < g.zwords; w += kHistThreads) cnt += __popc(__ldcg(ws.zmap + plane * g.zwords + w));
-    cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
-    if (lane == 0) hs.red32[tid >> 5] = cnt;
-    __syncthreads();
-    if (tid == 0) {
-      uint32_t t = 0;
-      for (int i = 0; i < kHistThreads / 32; i++) t += hs.red32[i];
-      ws.zcount[plane] = t;
-      decide_byte_plane<DT>(g, ws, c, s);
-    }
-    __syncthreads();
   }
 }
 
@@ -539,14 +329,19 @@ __global__ void __launch_bounds__(kHistThreads) k_split_hist_bf16(const uint8_t*
   }
 }
 
-// FP32, FP8 and FP4 compress: the histogram pass alone, in persistent blocks (each takes
-// tiles blockIdx.x, blockIdx.x + gridDim.x, ...; a tile is one 32768-value slice of a
-// chunk): the tile's counts (its encode-tile counts: FP32 the exponents, FP8/FP4 the joint
-// bins), the chunks' histograms and all-zero flags, and for FP32 the zero-run block bits
-// of the three fraction planes with each tile's marked count. The counters and their
-// addressing are k_split_hist's; a tile's column sums also clear them for the next tile.
-// The code builds follow in k_build_chunks, so no block waits on another and none stalls
-// its stream of tiles on a build.
+// FP32, FP8 and FP4 (BF16 has k_split_hist_bf16 below). THEORY-599 note, "Order-0 only
+// (section III-A b)": the model of a chunk is the count of each symbol. The block keeps one
+// counter per (symbol, lane) in shared memory, so the 32 lanes of a warp always add into
+// 32 different banks (lane l owns column l); warps share the table through shared
+// atomics, and a tile's column sums also clear it for the next tile. FP8 and FP4 count the
+// joint (exponent, mantissa) bin, exponent * mantissa alphabet + mantissa, so one atomic
+// counts both entropy streams (FP4 one atomic per byte, for its pair of joint bins).
+// Blocks are persistent (each takes tiles blockIdx.x, blockIdx.x + gridDim.x, ...; a tile
+// is one 32768-value slice of a chunk) and write the chunks' histograms and all-zero
+// flags; in a compress (ws set) also each tile's counts (its encode-tile counts: FP32 the
+// exponents, FP8/FP4 the joint bins) and FP32's zero-run block bits of the three fraction
+// planes with each tile's marked count. The code builds follow in k_build_chunks, so no
+// block waits on another and none stalls its stream of tiles on a build.
 template <int DT>
 __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist_tiles(const uint8_t* __restrict__ src, Geo g,
                                                                      uint32_t* __restrict__ hist,
@@ -864,7 +659,7 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout(Geo g, Ws ws, PlanDev
 // ---------------------------------------------------------------- launchers
 
 // Opt a kernel into more than 48 KB of dynamic shared memory, once per device. Slots:
-// 3 k_code_lengths, 4 + DT k_split_hist<DT>, 8 + DT k_build_chunks<DT>.
+// 3 k_code_lengths, 8 + DT k_build_chunks<DT>.
 template <typename K>
 static cudaError_t allow_smem(K kernel, size_t bytes, int slot) {
   static std::atomic<int> done[12][128];
@@ -921,7 +716,7 @@ cudaError_t launch_build_chunks(const Geo& g, const Ws& ws, const PlanDev& plan,
   }
 }
 
-// FP32 / FP8 / FP4 compress: a persistent grid of as many histogram blocks as fit on the device.
+// FP32 / FP8 / FP4: a persistent grid of as many histogram blocks as fit on the device.
 template <int DT>
 static cudaError_t split_hist_tiles_t(const void* src, const Geo& g, uint32_t* hist, uint32_t* nonzero, const Ws& ws,
                                       cudaStream_t st) {
@@ -947,36 +742,13 @@ static cudaError_t split_hist_tiles_t(const void* src, const Geo& g, uint32_t* h
   return cudaGetLastError();
 }
 
-template <int DT>
-static cudaError_t split_hist_t(const void* src, const Geo& g, uint32_t* hist, uint32_t* nonzero, const Ws* ws,
-                                const PlanDev& plan, cudaStream_t st) {
-  const uint32_t slices = (uint32_t)ceil_div(g.m0, kHistSlice);
-  const uint64_t blocks = (uint64_t)g.n_chunks * slices;
-  if (blocks > 0x7FFFFFFFull) return cudaErrorInvalidConfiguration;
-  constexpr int NE = n_entropy(DT);
-  constexpr size_t AJ = NE > 1 ? (size_t)alphabet(DT, 0) * alphabet(DT, 1) : (size_t)alphabet(DT, 0);
-  constexpr size_t AC = DT == kFP4 ? AJ * AJ : AJ;          // FP4 counts byte pairs
-  constexpr size_t cols = (AC * 32 + (NE > 1 ? AC + AJ : 0)) * 4;  // counters (+ their sums, the joint bins)
-  const size_t smem = ws ? (sizeof(HuffBlockSmem) > cols ? sizeof(HuffBlockSmem) : cols) : cols;
-  const cudaError_t e = allow_smem(k_split_hist<DT>, sizeof(HuffBlockSmem) > cols ? sizeof(HuffBlockSmem) : cols, 4 + DT);
-  if (e != cudaSuccess) return e;
-  Ws w{};
-  if (ws) w = *ws;
-  k_split_hist<DT><<<(uint32_t)blocks, kHistThreads, smem, st>>>(static_cast<const uint8_t*>(src), g, slices, hist,
-                                                                 nonzero, w, plan, ws ? 1 : 0);
-  return cudaGetLastError();
-}
-
 cudaError_t launch_split_hist(const void* src, const Geo& g, uint32_t* hist, uint32_t* nonzero, const Ws* ws,
                               const PlanDev& plan, cudaStream_t st) {
   switch (g.dt) {
     case kBF16: return split_hist_bf16(src, g, hist, nonzero, ws, plan, st);
-    case kFP32: return ws ? split_hist_tiles_t<kFP32>(src, g, hist, nonzero, *ws, st)
-                          : split_hist_t<kFP32>(src, g, hist, nonzero, ws, plan, st);
-    case kFP8: return ws ? split_hist_tiles_t<kFP8>(src, g, hist, nonzero, *ws, st)
-                         : split_hist_t<kFP8>(src, g, hist, nonzero, ws, plan, st);
-    default: return ws ? split_hist_tiles_t<kFP4>(src, g, hist, nonzero, *ws, st)
-                       : split_hist_t<kFP4>(src, g, hist, nonzero, ws, plan, st);
+    case kFP32: return split_hist_tiles_t<kFP32>(src, g, hist, nonzero, ws ? *ws : Ws{}, st);
+    case kFP8: return split_hist_tiles_t<kFP8>(src, g, hist, nonzero, ws ? *ws : Ws{}, st);
+    default: return split_hist_tiles_t<kFP4>(src, g, hist, nonzero, ws ? *ws : Ws{}, st);
   }
 }
 
