@@ -11,8 +11,10 @@ the movement of model weights).
 
 `exchange_containers` is the collective part alone (torch.distributed, NCCL between GPUs
 or gloo on CPU); `all_gather_compressed` adds the compress and the batched decompress,
-which run in the CUDA library. No peer memory is read by a kernel here: the containers
-arrive through the all-gather into local memory first.
+which run in the CUDA library. With peer_read the all-gather of containers is replaced by
+`share_containers` (CUDA IPC views of the peers' containers) and the decode reads the
+peers' memory itself: the transfer and the decode are one kernel. Its loads are plain,
+never multicast, bulk copies and loads.
 """
 import torch
 
@@ -42,23 +44,76 @@ def exchange_containers(container, group=None):
     return buf, sizes, slot
 
 
-def all_gather_compressed(x_local, group=None, chunk_bytes=Z.DEFAULT_CHUNK_BYTES, stream=None):
+def share_containers(container, group=None):
+    """Every rank's container, readable in place: this rank's own tensor and, for each peer,
+    a view of the peer's device memory opened through CUDA IPC (the handles travel in one
+    all-gather of small host objects). A kernel that reads a peer's view reads the peer's
+    memory directly: over NVLink between GPUs, with nothing copied first. Peer access is
+    enabled from this device to each peer's. Returns (views, sizes). Every rank keeps its
+    container alive, and unchanged, until all ranks are done reading (a barrier)."""
+    import torch.distributed as dist
+    from torch.multiprocessing.reductions import reduce_tensor, rebuild_cuda_tensor
+    world, rank = dist.get_world_size(group), dist.get_rank(group)
+    _, args = reduce_tensor(container)
+    objs = [None] * world
+    dist.all_gather_object(objs, (container.numel(), container.device.index, args), group=group)
+    here = container.device.index
+    views = []
+    for r, (n, dev, a) in enumerate(objs):
+        if r == rank:
+            views.append(container)
+            continue
+        if dev != here and torch.cuda.can_device_access_peer(here, dev):
+            _enable_peer_access(here, dev)
+        views.append(rebuild_cuda_tensor(*a))
+    return views, [n for n, _, _ in objs]
+
+
+def _enable_peer_access(here, peer):
+    from cuda.bindings import runtime as rt
+    with torch.cuda.device(here):
+        err, = rt.cudaDeviceEnablePeerAccess(peer, 0)
+    if err not in (rt.cudaError_t.cudaSuccess, rt.cudaError_t.cudaErrorPeerAccessAlreadyEnabled):
+        raise RuntimeError(f"cudaDeviceEnablePeerAccess({peer}) from device {here}: {err}")
+    rt.cudaGetLastError()  # an already-enabled peer leaves its code behind
+
+
+def all_gather_compressed(x_local, group=None, chunk_bytes=Z.DEFAULT_CHUNK_BYTES, stream=None, peer_read=False):
     """The gathered tensor (rank r's shard at [r * n, (r + 1) * n) of the flattened result,
     n = x_local's values), with the shards moved compressed. Every rank of the group calls
-    it with a shard of the same dtype and size. Returns (gathered, bytes moved per rank
-    into the all-gather of containers)."""
+    it with a shard of the same dtype and size.
+
+    peer_read=False: the containers travel in one all-gather (exchange_containers), then
+    one batched decode. peer_read=True (the decode fused with the transfer): the ranks
+    share their containers in place (share_containers) and one batched decode reads the
+    peers' containers where they are, so each peer's bitstream crosses the link once,
+    straight into the shared memory of the block that decodes it, and its sign/fraction
+    bytes straight into registers; the decoded values land in local memory. Barriers on
+    both sides keep every container complete while it is read and alive until every rank
+    is done.
+
+    Returns (gathered, bytes each rank contributed to an all-gather of containers: the
+    padded slot, or 0 with peer_read)."""
     import torch.distributed as dist
     world = dist.get_world_size(group) if dist.is_available() and dist.is_initialized() else 1
     xf = x_local.reshape(-1)
     if (xf.numel() * xf.element_size()) % 16:
         raise ValueError("all_gather_compressed: a shard must be a multiple of 16 bytes (each lands 16-byte aligned)")
-    cont = Z.compress(xf, chunk_bytes=chunk_bytes, stream=stream)
-    buf, sizes, slot = exchange_containers(cont, group)
-    out = torch.empty(world * xf.numel(), dtype=xf.dtype, device=xf.device)
+    cont = Z.compress(xf, chunk_bytes=chunk_bytes, stream=stream)  # synchronises: the container is complete
     n = xf.numel()
-    items = [buf[r * slot: r * slot + sizes[r]] for r in range(world)]
+    out = torch.empty(world * n, dtype=xf.dtype, device=xf.device)
     outs = [out[r * n: (r + 1) * n] for r in range(world)]
     ws = Z.batch_workspace(world, xf.device)
+    if peer_read and world > 1:
+        views, sizes = share_containers(cont, group)
+        dist.barrier(group=group)  # every rank's container is complete before anyone reads it
+        Z.decompress_batch_into(views, sizes, outs, ws, chunk_bytes, stream=stream)
+        Z.check(Z.status(ws, stream), "all_gather_compressed: decompress")  # synchronises
+        del views
+        dist.barrier(group=group)  # every rank is done reading before any container is freed
+        return out, 0
+    buf, sizes, slot = exchange_containers(cont, group)
+    items = [buf[r * slot: r * slot + sizes[r]] for r in range(world)]
     Z.decompress_batch_into(items, sizes, outs, ws, chunk_bytes, stream=stream)
     Z.check(Z.status(ws, stream), "all_gather_compressed: decompress")
     return out, slot
