@@ -52,6 +52,19 @@ def lib():
         L.orc_plan_build.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_uint64, ctypes.c_uint32,
                                      ctypes.c_uint32, ctypes.c_uint64, ctypes.c_void_p, ctypes.c_void_p,
                                      ctypes.POINTER(ctypes.c_int), ctypes.c_void_p]
+        L.orc_compress_packed.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_uint64, ctypes.c_uint32,
+                                          ctypes.c_uint32, ctypes.c_void_p, ctypes.c_uint32, ctypes.c_void_p,
+                                          ctypes.c_void_p, ctypes.c_uint32, ctypes.c_void_p, ctypes.c_uint64, u64p,
+                                          ctypes.c_int]
+        L.orc_max_compressed_bytes_packed.argtypes = [ctypes.c_int, ctypes.c_uint64, ctypes.c_uint32,
+                                                      ctypes.c_uint32, ctypes.c_uint32]
+        L.orc_max_compressed_bytes_packed.restype = ctypes.c_uint64
+        L.orc_pack_histogram.argtypes = [ctypes.c_void_p, ctypes.c_uint64, ctypes.c_uint64, ctypes.c_void_p,
+                                         ctypes.c_uint32, u64p, u64p]
+        L.orc_pack_histogram.restype = None
+        L.orc_plan_pack.argtypes = [ctypes.c_void_p, ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32,
+                                    ctypes.c_void_p, ctypes.c_uint32, ctypes.c_void_p, ctypes.c_void_p,
+                                    ctypes.POINTER(ctypes.c_uint32)]
         L.orc_splitmix64.argtypes = [u64p]
         L.orc_splitmix64.restype = ctypes.c_uint64
         _lib = L
@@ -107,12 +120,13 @@ def histogram(dtype, data, lo, hi, stream):
     return h
 
 
-def max_compressed_bytes(dtype, n, chunk_bytes, n_groups=0):
-    return int(lib().orc_max_compressed_bytes(DTYPES[dtype], n, chunk_bytes, n_groups))
+def max_compressed_bytes(dtype, n, chunk_bytes, n_groups=0, K=0):
+    return int(lib().orc_max_compressed_bytes_packed(DTYPES[dtype], n, chunk_bytes, n_groups, K))
 
 
-def compress(dtype, data, n=None, chunk_bytes=262144, S=512, plan_lens=None, threads=1):
-    """Return the container (numpy uint8) for the n values held in data."""
+def compress(dtype, data, n=None, chunk_bytes=262144, S=512, plan_lens=None, threads=1, pack=None):
+    """Return the container (numpy uint8) for the n values held in data. pack: the plan's
+    packed exponents (exps, pack_lens[groups, 256]) as plan_pack returns them, or None."""
     b = _bytes_view(data)
     if n is None:
         n = values_in(dtype, b.size)
@@ -123,14 +137,47 @@ def compress(dtype, data, n=None, chunk_bytes=262144, S=512, plan_lens=None, thr
         pl = np.ascontiguousarray(plan_lens, dtype=np.uint8)
         G = pl.shape[1]
         plan_ptr = pl.ctypes.data
-    cap = max_compressed_bytes(dtype, n, chunk_bytes, G)
+    K, exps_ptr, plens_ptr = 0, None, None
+    if pack is not None and len(pack[0]):
+        ex = np.zeros(16, dtype=np.uint8)
+        ex[: len(pack[0])] = np.asarray(pack[0], dtype=np.uint8)
+        pk = np.ascontiguousarray(pack[1], dtype=np.uint8)
+        K, exps_ptr, plens_ptr = len(pack[0]), ex.ctypes.data, pk.ctypes.data
+    cap = max_compressed_bytes(dtype, n, chunk_bytes, G, K)
     out = np.zeros(cap, dtype=np.uint8)
     size = ctypes.c_uint64(0)
-    st = lib().orc_compress(DTYPES[dtype], b.ctypes.data, n, chunk_bytes, S, plan_ptr, G,
-                            out.ctypes.data, cap, ctypes.byref(size), threads)
+    st = lib().orc_compress_packed(DTYPES[dtype], b.ctypes.data, n, chunk_bytes, S, plan_ptr, G, plens_ptr,
+                                   exps_ptr, K, out.ctypes.data, cap, ctypes.byref(size), threads)
     if st != OK:
         raise OracleError(st)
     return out[: size.value].copy()
+
+
+def pack_histogram(data, lo, m, exps):
+    """Pair-symbol counts (256) and escaped exponents of BF16 values [lo, lo + m)."""
+    b = _bytes_view(data)
+    ex = np.zeros(16, dtype=np.uint8)
+    ex[: len(exps)] = np.asarray(exps, dtype=np.uint8)
+    h = np.zeros(256, dtype=np.uint64)
+    esc = np.zeros(1, dtype=np.uint64)
+    lib().orc_pack_histogram(b.ctypes.data, lo, m, ex.ctypes.data, len(exps), _u64(h), _u64(esc))
+    return h, int(esc[0])
+
+
+def plan_pack(data, assign, groups, max_pack=15, n=None, chunk_bytes=262144):
+    """Packed exponents of a BF16 plan: (exps (K bytes), pack_lens[groups, 256])."""
+    b = _bytes_view(data)
+    if n is None:
+        n = values_in("bf16", b.size)
+    a = np.ascontiguousarray(assign, dtype=np.uint32)
+    ex = np.zeros(16, dtype=np.uint8)
+    lens = np.zeros((groups, 256), dtype=np.uint8)
+    K = ctypes.c_uint32(0)
+    st = lib().orc_plan_pack(b.ctypes.data, n, chunk_bytes, groups, a.ctypes.data, max_pack, ex.ctypes.data,
+                             lens.ctypes.data, ctypes.byref(K))
+    if st != OK:
+        raise OracleError(st)
+    return ex[: K.value].copy(), lens
 
 
 def decompress(dtype, container, n, chunk_bytes=262144, threads=1):

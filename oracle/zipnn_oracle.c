@@ -29,6 +29,13 @@
  *    "layout rules" below; pinned by a hand-derived golden container, not by the pages.
  *  - Grouping: Lloyd's k-means with SplitMix64 seeding (parity unpinned by the pages:
  *    pinned only by invariants and small separable cases).
+ *  - Packed exponent tuples (NeuralZip, abstract: recurring exponent tuples represented
+ *    by packed exponents, chosen by the setup; the pages give no format). Reading, BF16
+ *    only: the setup lists the K <= 15 most frequent exponents of its tensor; a pair of
+ *    exponents at values (2j, 2j+1) becomes one 8-bit symbol, the two list indices as
+ *    nibbles (first value high), 15 for an exponent not in the list, whose 8 bits then
+ *    follow the pair's code. Each group gets a second code over these pair symbols, and
+ *    a chunk takes whichever shared code, plain or packed, codes it in the fewest bits.
  */
 #include "zipnn_oracle.h"
 
@@ -44,6 +51,10 @@
 #define MODE_ZERO 1
 #define MODE_HUFF 2
 #define MODE_ZRUN 3
+#define MODE_PACK 4
+#define PACK_MAX 15   /* packed exponents a plan may list; nibble 15 is the escape */
+#define PACK_ESC 15
+#define PACK_LIST_BYTES 16
 #define ZRUN_BLOCK 32 /* symbols of one zero-run block */
 #define NO_CODE 0xFFFFFFFFu
 
@@ -278,6 +289,12 @@ static uint64_t get_u64(const uint8_t* p) {
  *    (the last block may be shorter): one bit per block, MSB first, 1 when the block
  *    holds a non-zero symbol, padded to 16 bytes, then the symbols of the marked blocks
  *    in order, padded to 16 bytes.
+ *  - packed exponents (BF16 with a plan that lists K > 0 exponents): header byte 58 is
+ *    K; the code section holds, after the plain records, one packed record per group
+ *    (a code over the 256 pair symbols), then the K listed exponents padded to 16 bytes;
+ *    a PACK entry (mode 4, code = groups + g) holds the bit offset (u32) of every S-th
+ *    value's pair padded to 16 bytes, then for every pair its code followed by the raw
+ *    8 bits of each escaped exponent (first, then second), MSB first, padded to 16 bytes.
  *  - choice for a stream: ZERO when every symbol is 0. An entropy stream is HUFF when
  *    that payload is strictly smaller than RAW, else RAW. A byte plane (8-bit symbols
  *    that are not entropy-coded: BF16's sign/fraction byte, FP32's three fraction
@@ -297,11 +314,23 @@ static uint64_t table_end(int dtype, uint64_t n_chunks) {
   return HEADER_BYTES + (uint64_t)ENTRY_BYTES * n_chunks * (uint64_t)orc_n_streams(dtype);
 }
 
-/* bytes of all shared code records for n_groups groups */
+/* bytes of all plain shared code records for n_groups groups */
 static uint64_t shared_bytes(int dtype, uint32_t n_groups) {
   uint64_t b = 0;
   for (int s = 0; s < orc_n_entropy(dtype); s++) b += (uint64_t)n_groups * record_bytes(dtype, s);
   return b;
+}
+
+/* the code section with K packed exponents: plain records, packed records, the list */
+static uint64_t code_section_bytes(int dtype, uint32_t n_groups, uint32_t K) {
+  uint64_t b = shared_bytes(dtype, n_groups);
+  if (K) b += (uint64_t)n_groups * record_bytes(dtype, 0) + PACK_LIST_BYTES;
+  return b;
+}
+
+/* byte position of group g's packed record inside the code section */
+static uint64_t packed_record_pos(int dtype, uint32_t n_groups, uint32_t g) {
+  return shared_bytes(dtype, n_groups) + (uint64_t)g * record_bytes(dtype, 0);
 }
 
 /* byte position of shared record r = e * n_groups + g inside the code section */
@@ -314,16 +343,45 @@ static uint64_t shared_record_pos(int dtype, uint32_t n_groups, uint32_t r) {
 
 static uint64_t raw_payload_bytes(uint64_t m, int width) { return round16(ceil_div(m * (uint64_t)width, 8)); }
 
-uint64_t orc_max_compressed_bytes(int dtype, uint64_t n, uint32_t chunk_bytes, uint32_t n_groups) {
+/* header, table, code section and every payload stored RAW: a HUFF, PACK or ZRUN
+ * payload is only chosen when it is smaller */
+uint64_t orc_max_compressed_bytes_packed(int dtype, uint64_t n, uint32_t chunk_bytes, uint32_t n_groups, uint32_t K) {
   uint64_t m0 = chunk_values(dtype, chunk_bytes);
   if (m0 == 0 || n == 0) return 0;
   uint64_t chunks = ceil_div(n, m0);
-  uint64_t total = table_end(dtype, chunks) + shared_bytes(dtype, n_groups);
+  uint64_t total = table_end(dtype, chunks) + code_section_bytes(dtype, n_groups, K);
   for (uint64_t c = 0; c < chunks; c++) {
     uint64_t m = (c + 1) * m0 <= n ? m0 : n - c * m0;
     for (int s = 0; s < orc_n_streams(dtype); s++) total += raw_payload_bytes(m, raw_width(dtype, s));
   }
   return total;
+}
+
+uint64_t orc_max_compressed_bytes(int dtype, uint64_t n, uint32_t chunk_bytes, uint32_t n_groups) {
+  return orc_max_compressed_bytes_packed(dtype, n, chunk_bytes, n_groups, 0);
+}
+
+/* Nibble of exponent x in a pair symbol: its index in the plan's list, else the escape. */
+static uint32_t pack_nibble(uint8_t x, const uint8_t* exps, uint32_t K) {
+  for (uint32_t i = 0; i < K; i++)
+    if (exps[i] == x) return i;
+  return PACK_ESC;
+}
+
+/* Pair symbols of the BF16 values [lo, lo + m) (m even): the exponents of values
+ * lo + 2j and lo + 2j + 1 give symbol nibble(first) << 4 | nibble(second). hist (256)
+ * receives the symbol counts and *escapes the number of escaped exponents. */
+void orc_pack_histogram(const void* src, uint64_t lo, uint64_t m, const uint8_t* exps, uint32_t K, uint64_t* hist,
+                        uint64_t* escapes) {
+  const uint8_t* in = (const uint8_t*)src;
+  for (int k = 0; k < 256; k++) hist[k] = 0;
+  *escapes = 0;
+  for (uint64_t j = 0; j + 1 < m; j += 2) {
+    uint32_t a = pack_nibble(orc_field(ORC_BF16, in, lo + j, 0), exps, K);
+    uint32_t b = pack_nibble(orc_field(ORC_BF16, in, lo + j + 1, 0), exps, K);
+    hist[(a << 4) | b]++;
+    *escapes += (a == PACK_ESC) + (b == PACK_ESC);
+  }
 }
 
 /* ------------------------------------------------------------------ compress */
@@ -342,6 +400,9 @@ typedef struct {
   uint32_t S;
   const uint8_t* plan_lens;
   uint32_t n_groups;
+  const uint8_t* pack_lens; /* n_groups x 256 packed-code lengths, when K > 0 */
+  const uint8_t* pack_exps; /* the K listed exponents */
+  uint32_t K;
   entry_t* entries;
   int thread, threads;
   int status;
@@ -394,36 +455,88 @@ static int encode_entry(const job_t* jb, uint64_t lo, uint64_t m, int s, entry_t
         }
       }
     }
-    if (use_group >= 0) memcpy(len, jb->plan_lens + ((uint64_t)e * jb->n_groups + (uint32_t)use_group) * 256, 256);
-    else orc_limited_lengths(hist, a, LMAX, len);
-    uint64_t bits = 0;
-    for (int k = 0; k < a; k++) bits += hist[k] * len[k];
-    uint64_t nsub = ceil_div(m, jb->S);
-    uint64_t rec = use_group >= 0 ? 0 : record_bytes(dt, s);
-    uint64_t p_huff = rec + round16(4 * nsub) + round16(ceil_div(bits, 8));
-    if (p_huff < p_raw) {
-      en->mode = MODE_HUFF;
-      en->code = use_group >= 0 ? (uint32_t)e * jb->n_groups + (uint32_t)use_group : NO_CODE;
-      en->size = p_huff;
-      en->bytes = (uint8_t*)calloc(p_huff, 1);
-      if (!en->bytes) {
+    /* packed exponents (BF16 exponent stream, even chunk and sub-block lengths): each
+     * group's packed code competes with the plain codes; strictly fewer bits win */
+    int use_pack = -1;
+    if (jb->plan_lens && jb->K && dt == ORC_BF16 && s == 0 && m % 2 == 0 && jb->S % 2 == 0) {
+      uint64_t hp[256], esc = 0;
+      orc_pack_histogram(jb->src, lo, m, jb->pack_exps, jb->K, hp, &esc);
+      for (uint32_t g = 0; g < jb->n_groups; g++) {
+        const uint8_t* lp = jb->pack_lens + (uint64_t)g * 256;
+        int ok = 1;
+        uint64_t bits = 8 * esc;
+        for (int k = 0; k < 256; k++) {
+          if (hp[k] == 0) continue;
+          if (lp[k] == 0) ok = 0;
+          bits += hp[k] * lp[k];
+        }
+        if (ok && ((use_group < 0 && use_pack < 0) || bits < best_bits)) {
+          use_pack = (int)g;
+          best_bits = bits;
+        }
+      }
+      if (use_pack >= 0) use_group = -1;
+    }
+    if (use_pack >= 0) {
+      const uint8_t* lp = jb->pack_lens + (uint64_t)use_pack * 256;
+      uint64_t nsub = ceil_div(m, jb->S);
+      uint64_t p_pack = round16(4 * nsub) + round16(ceil_div(best_bits, 8));
+      if (p_pack < p_raw) {
+        en->mode = MODE_PACK;
+        en->code = jb->n_groups * (uint32_t)orc_n_entropy(dt) + (uint32_t)use_pack;
+        en->size = p_pack;
+        en->bytes = (uint8_t*)calloc(p_pack, 1);
+        if (!en->bytes) {
+          free(sym);
+          return ORC_EINVAL;
+        }
+        orc_canonical_codes(lp, 256, code);
+        uint8_t* bs = en->bytes + round16(4 * nsub);
+        uint64_t t = 0;
+        for (uint64_t i = 0; i < m; i += 2) {
+          if (i % jb->S == 0) put_u32(en->bytes + 4 * (i / jb->S), (uint32_t)t);
+          uint32_t a = pack_nibble(sym[i], jb->pack_exps, jb->K), b = pack_nibble(sym[i + 1], jb->pack_exps, jb->K);
+          uint32_t ps = (a << 4) | b;
+          put_bits(bs, &t, code[ps], lp[ps]);
+          if (a == PACK_ESC) put_bits(bs, &t, sym[i], 8);
+          if (b == PACK_ESC) put_bits(bs, &t, sym[i + 1], 8);
+        }
         free(sym);
-        return ORC_EINVAL;
+        return ORC_OK;
       }
-      uint8_t* p = en->bytes;
-      if (rec) {
-        for (int k = 0; k < a / 2; k++) p[k] = (uint8_t)(len[2 * k] | (len[2 * k + 1] << 4));
-        p += rec;
+    }
+    if (use_pack < 0) {
+      if (use_group >= 0) memcpy(len, jb->plan_lens + ((uint64_t)e * jb->n_groups + (uint32_t)use_group) * 256, 256);
+      else orc_limited_lengths(hist, a, LMAX, len);
+      uint64_t bits = 0;
+      for (int k = 0; k < a; k++) bits += hist[k] * len[k];
+      uint64_t nsub = ceil_div(m, jb->S);
+      uint64_t rec = use_group >= 0 ? 0 : record_bytes(dt, s);
+      uint64_t p_huff = rec + round16(4 * nsub) + round16(ceil_div(bits, 8));
+      if (p_huff < p_raw) {
+        en->mode = MODE_HUFF;
+        en->code = use_group >= 0 ? (uint32_t)e * jb->n_groups + (uint32_t)use_group : NO_CODE;
+        en->size = p_huff;
+        en->bytes = (uint8_t*)calloc(p_huff, 1);
+        if (!en->bytes) {
+          free(sym);
+          return ORC_EINVAL;
+        }
+        uint8_t* p = en->bytes;
+        if (rec) {
+          for (int k = 0; k < a / 2; k++) p[k] = (uint8_t)(len[2 * k] | (len[2 * k + 1] << 4));
+          p += rec;
+        }
+        orc_canonical_codes(len, a, code);
+        uint8_t* bs = p + round16(4 * nsub);
+        uint64_t t = 0;
+        for (uint64_t i = 0; i < m; i++) {
+          if (i % jb->S == 0) put_u32(p + 4 * (i / jb->S), (uint32_t)t);
+          put_bits(bs, &t, code[sym[i]], len[sym[i]]);
+        }
+        free(sym);
+        return ORC_OK;
       }
-      orc_canonical_codes(len, a, code);
-      uint8_t* bs = p + round16(4 * nsub);
-      uint64_t t = 0;
-      for (uint64_t i = 0; i < m; i++) {
-        if (i % jb->S == 0) put_u32(p + 4 * (i / jb->S), (uint32_t)t);
-        put_bits(bs, &t, code[sym[i]], len[sym[i]]);
-      }
-      free(sym);
-      return ORC_OK;
     }
   }
   if (!is_entropy(dt, s) && w == 8) {
@@ -518,14 +631,23 @@ static int run_jobs(job_t* base, int threads, void* (*fn)(void*)) {
 int orc_compress(int dtype, const void* src, uint64_t n, uint32_t chunk_bytes, uint32_t S,
                  const uint8_t* plan_lens, uint32_t n_groups, void* out, uint64_t cap,
                  uint64_t* out_bytes, int threads) {
+  return orc_compress_packed(dtype, src, n, chunk_bytes, S, plan_lens, n_groups, NULL, NULL, 0, out, cap, out_bytes,
+                             threads);
+}
+
+int orc_compress_packed(int dtype, const void* src, uint64_t n, uint32_t chunk_bytes, uint32_t S,
+                        const uint8_t* plan_lens, uint32_t n_groups, const uint8_t* pack_lens,
+                        const uint8_t* pack_exps, uint32_t K, void* out, uint64_t cap, uint64_t* out_bytes,
+                        int threads) {
   if (dtype < 0 || dtype > 3 || !src || !out || bad_count(dtype, n) || S == 0) return ORC_EINVAL;
   if (chunk_bytes == 0 || chunk_bytes % (uint32_t)value_bytes(dtype) != 0) return ORC_EINVAL;
   if (plan_lens && (n_groups == 0 || n_groups > MAX_GROUPS)) return ORC_EINVAL;
   if (!plan_lens) n_groups = 0;
+  if (K > PACK_MAX || (K && (dtype != ORC_BF16 || !plan_lens || !pack_lens || !pack_exps))) return ORC_EINVAL;
   int ns = orc_n_streams(dtype);
   uint64_t m0 = chunk_values(dtype, chunk_bytes);
   uint64_t chunks = ceil_div(n, m0);
-  if (cap < orc_max_compressed_bytes(dtype, n, chunk_bytes, n_groups)) return ORC_ESMALL;
+  if (cap < orc_max_compressed_bytes_packed(dtype, n, chunk_bytes, n_groups, K)) return ORC_ESMALL;
   entry_t* entries = (entry_t*)calloc(chunks * (uint64_t)ns, sizeof(entry_t));
   if (!entries) return ORC_EINVAL;
   job_t jb;
@@ -538,12 +660,15 @@ int orc_compress(int dtype, const void* src, uint64_t n, uint32_t chunk_bytes, u
   jb.S = S;
   jb.plan_lens = plan_lens;
   jb.n_groups = n_groups;
+  jb.pack_lens = pack_lens;
+  jb.pack_exps = pack_exps;
+  jb.K = K;
   jb.entries = entries;
   int st = run_jobs(&jb, threads, compress_worker);
   if (st == ORC_OK) {
     uint8_t* o = (uint8_t*)out;
     uint64_t off_codes = table_end(dtype, chunks);
-    uint64_t off_payload = off_codes + shared_bytes(dtype, n_groups);
+    uint64_t off_payload = off_codes + code_section_bytes(dtype, n_groups, K);
     memset(o, 0, off_payload);
     /* header */
     o[0] = 'Z';
@@ -558,11 +683,12 @@ int orc_compress(int dtype, const void* src, uint64_t n, uint32_t chunk_bytes, u
     put_u32(o + 16, chunk_bytes);
     put_u32(o + 20, S);
     put_u32(o + 24, (uint32_t)chunks);
-    put_u32(o + 28, n_groups * (uint32_t)orc_n_entropy(dtype));
+    put_u32(o + 28, n_groups * (uint32_t)orc_n_entropy(dtype) + (K ? n_groups : 0));
     put_u64(o + 32, off_codes);
     put_u64(o + 40, off_payload);
     o[56] = LMAX;
     o[57] = (uint8_t)n_groups;
+    o[58] = (uint8_t)K;
     /* shared code records */
     for (int e = 0; e < orc_n_entropy(dtype) && n_groups; e++) {
       int a = orc_alphabet(dtype, e);
@@ -571,6 +697,15 @@ int orc_compress(int dtype, const void* src, uint64_t n, uint32_t chunk_bytes, u
         uint8_t* rp = o + off_codes + shared_record_pos(dtype, n_groups, (uint32_t)e * n_groups + g);
         for (int k = 0; k < a / 2; k++) rp[k] = (uint8_t)(lg[2 * k] | (lg[2 * k + 1] << 4));
       }
+    }
+    /* packed records and the list of packed exponents */
+    if (K) {
+      for (uint32_t g = 0; g < n_groups; g++) {
+        const uint8_t* lp = pack_lens + (uint64_t)g * 256;
+        uint8_t* rp = o + off_codes + packed_record_pos(dtype, n_groups, g);
+        for (int k = 0; k < 128; k++) rp[k] = (uint8_t)(lp[2 * k] | (lp[2 * k + 1] << 4));
+      }
+      memcpy(o + off_codes + code_section_bytes(dtype, n_groups, K) - PACK_LIST_BYTES, pack_exps, K);
     }
     /* chunk table and payloads, in entry order: offsets are the running sum */
     uint64_t pos = off_payload;
@@ -596,7 +731,8 @@ typedef struct {
   int dtype;
   const uint8_t* in;
   uint64_t in_bytes, n, m0, chunks, total, off_codes;
-  uint32_t S, n_groups;
+  uint32_t S, n_groups, K;
+  const uint8_t* pack_exps; /* the K listed exponents, in the container */
   uint8_t* out;
   int thread, threads;
   int status;
@@ -686,6 +822,58 @@ static int decode_entry(const djob_t* jb, uint64_t c, int s, uint64_t m, uint8_t
     }
     return ORC_OK;
   }
+  if (mode == MODE_PACK) {
+    /* pairs of exponents as packed symbols, escaped exponents inline */
+    uint8_t plen[256];
+    if (dt != ORC_BF16 || s != 0 || !jb->K || m % 2 || jb->S % 2) return ORC_ECORRUPT;
+    uint32_t NE = (uint32_t)orc_n_entropy(dt);
+    if (code_ix < jb->n_groups * NE || code_ix >= jb->n_groups * NE + jb->n_groups) return ORC_ECORRUPT;
+    uint32_t g = code_ix - jb->n_groups * NE;
+    if (read_record(jb->in + jb->off_codes + packed_record_pos(dt, jb->n_groups, g), 256, plen) != ORC_OK)
+      return ORC_ECORRUPT;
+    uint64_t nsub = ceil_div(m, jb->S), avail = end - off;
+    const uint8_t* p = jb->in + off;
+    if (avail < round16(4 * nsub)) return ORC_ECORRUPT;
+    const uint8_t* bs = p + round16(4 * nsub);
+    uint64_t cap_bits = (avail - round16(4 * nsub)) * 8;
+    uint32_t count[LMAX + 1] = {0};
+    uint8_t sorted[256];
+    int ns_sorted = 0;
+    for (int l = 1; l <= LMAX; l++)
+      for (int k2 = 0; k2 < 256; k2++)
+        if (plen[k2] == l) {
+          sorted[ns_sorted++] = (uint8_t)k2;
+          count[l]++;
+        }
+    if (get_u32(p) != 0) return ORC_ECORRUPT;
+    for (uint64_t j = 0; j < nsub; j++) {
+      uint64_t t = get_u32(p + 4 * j);
+      if (t > cap_bits) return ORC_ECORRUPT;
+      uint64_t lo = j * jb->S, hi = lo + jb->S < m ? lo + jb->S : m;
+      for (uint64_t i = lo; i < hi; i += 2) {
+        int v = decode_symbol(bs, cap_bits, &t, count, sorted);
+        if (v < 0) return ORC_ECORRUPT;
+        uint32_t nib[2] = {(uint32_t)v >> 4, (uint32_t)v & 15u};
+        for (int h = 0; h < 2; h++) {
+          if (nib[h] == PACK_ESC) {
+            uint32_t x = 0;
+            for (int b = 0; b < 8; b++) {
+              int bit = get_bit(bs, cap_bits, &t);
+              if (bit < 0) return ORC_ECORRUPT;
+              x = (x << 1) | (uint32_t)bit;
+            }
+            sym[i + h] = (uint8_t)x;
+          } else if (nib[h] < jb->K) {
+            sym[i + h] = jb->pack_exps[nib[h]];
+          } else {
+            return ORC_ECORRUPT;
+          }
+        }
+      }
+      if (j + 1 < nsub && t != get_u32(p + 4 * (j + 1))) return ORC_ECORRUPT;
+    }
+    return ORC_OK;
+  }
   if (mode != MODE_HUFF || !is_entropy(dt, s)) return ORC_ECORRUPT;
   uint8_t len[256];
   const uint8_t* p = jb->in + off;
@@ -767,13 +955,18 @@ int orc_decompress(int dtype, const void* in, uint64_t in_bytes, uint64_t n, uin
   uint64_t m0 = chunk_values(dtype, chunk_bytes);
   uint64_t chunks = ceil_div(n, m0);
   if (h[6] != dtype || h[7] != ns || get_u64(h + 8) != n || get_u32(h + 16) != chunk_bytes) return ORC_ECORRUPT;
-  uint32_t S = get_u32(h + 20), n_groups = h[57];
+  uint32_t S = get_u32(h + 20), n_groups = h[57], K = h[58];
   if (S == 0 || get_u32(h + 24) != chunks || h[56] != LMAX || n_groups > MAX_GROUPS) return ORC_ECORRUPT;
-  if (get_u32(h + 28) != n_groups * (uint32_t)orc_n_entropy(dtype)) return ORC_ECORRUPT;
-  if (h[58] || h[59] || get_u32(h + 60)) return ORC_ECORRUPT;
+  if (K > PACK_MAX || (K && (dtype != ORC_BF16 || n_groups == 0))) return ORC_ECORRUPT;
+  if (get_u32(h + 28) != n_groups * (uint32_t)orc_n_entropy(dtype) + (K ? n_groups : 0)) return ORC_ECORRUPT;
+  if (h[59] || get_u32(h + 60)) return ORC_ECORRUPT;
   uint64_t off_codes = get_u64(h + 32), off_payload = get_u64(h + 40), total = get_u64(h + 48);
-  if (off_codes != table_end(dtype, chunks) || off_payload != off_codes + shared_bytes(dtype, n_groups))
+  if (off_codes != table_end(dtype, chunks) || off_payload != off_codes + code_section_bytes(dtype, n_groups, K))
     return ORC_ECORRUPT;
+  if (total > in_bytes || total < off_payload) return ORC_ECORRUPT;
+  /* the list of packed exponents: K entries, then zeros */
+  for (uint32_t i = K; K && i < PACK_LIST_BYTES; i++)
+    if (h[off_payload - PACK_LIST_BYTES + i]) return ORC_ECORRUPT;
   if (total > in_bytes || total < off_payload) return ORC_ECORRUPT;
   if (get_u64(h + HEADER_BYTES + 8) != off_payload) return ORC_ECORRUPT;
   djob_t jb;
@@ -788,6 +981,8 @@ int orc_decompress(int dtype, const void* in, uint64_t in_bytes, uint64_t n, uin
   jb.off_codes = off_codes;
   jb.S = S;
   jb.n_groups = n_groups;
+  jb.K = K;
+  jb.pack_exps = K ? h + off_payload - PACK_LIST_BYTES : NULL;
   jb.out = (uint8_t*)out;
   if (threads < 1) threads = 1;
   if (threads > 256) threads = 256;
@@ -942,5 +1137,54 @@ int orc_plan_build(int dtype, const void* src, uint64_t n, uint32_t chunk_bytes,
   free(mu);
   free(assign);
   free(perm);
+  return ORC_OK;
+}
+
+/* Packed exponents of a plan (BF16; reading stated at the top of this file):
+ *  1. count every exponent of the setup tensor;
+ *  2. list the K = min(max_pack, exponents present) most frequent ones, a larger count
+ *     first, equal counts by the smaller exponent;
+ *  3. for each group, the length-limited Huffman code of the summed pair-symbol
+ *     histograms of its member chunks that hold an even number of values (a group
+ *     without such pairs gets no packed code).
+ * exps_out: 16 bytes (the list, then zeros); lens_out: n_groups x 256; *K_out. */
+int orc_plan_pack(const void* src, uint64_t n, uint32_t chunk_bytes, uint32_t n_groups, const uint32_t* assign,
+                  uint32_t max_pack, uint8_t* exps_out, uint8_t* lens_out, uint32_t* K_out) {
+  if (!src || n == 0 || !assign || n_groups == 0 || n_groups > MAX_GROUPS || max_pack > PACK_MAX) return ORC_EINVAL;
+  if (chunk_bytes == 0 || chunk_bytes % 2 != 0) return ORC_EINVAL;
+  const uint8_t* in = (const uint8_t*)src;
+  uint64_t total[256];
+  for (int k = 0; k < 256; k++) total[k] = 0;
+  for (uint64_t i = 0; i < n; i++) total[orc_field(ORC_BF16, in, i, 0)]++;
+  uint8_t taken[256];
+  memset(taken, 0, sizeof(taken));
+  memset(exps_out, 0, PACK_LIST_BYTES);
+  uint32_t K = 0;
+  while (K < max_pack) {
+    int best = -1;
+    for (int k = 0; k < 256; k++)
+      if (!taken[k] && total[k] > 0 && (best < 0 || total[k] > total[best])) best = k;
+    if (best < 0) break;
+    taken[best] = 1;
+    exps_out[K++] = (uint8_t)best;
+  }
+  *K_out = K;
+  memset(lens_out, 0, (size_t)n_groups * 256);
+  if (!K) return ORC_OK;
+  uint64_t m0 = chunk_bytes / 2, C = ceil_div(n, m0);
+  for (uint32_t g = 0; g < n_groups; g++) {
+    uint64_t sum[256], hp[256], esc;
+    int any = 0;
+    for (int k = 0; k < 256; k++) sum[k] = 0;
+    for (uint64_t c = 0; c < C; c++) {
+      uint64_t lo = c * m0, m = lo + m0 <= n ? m0 : n - lo;
+      if (assign[c] != g || m % 2) continue;
+      orc_pack_histogram(in, lo, m, exps_out, K, hp, &esc);
+      for (int k = 0; k < 256; k++) sum[k] += hp[k];
+    }
+    for (int k = 0; k < 256; k++)
+      if (sum[k]) any = 1;
+    if (any) orc_limited_lengths(sum, 256, LMAX, lens_out + (uint64_t)g * 256);
+  }
   return ORC_OK;
 }

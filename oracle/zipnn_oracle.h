@@ -71,6 +71,24 @@ int orc_compress(int dtype, const void* src, uint64_t n, uint32_t chunk_bytes, u
                  const uint8_t* plan_lens, uint32_t n_groups, void* out, uint64_t cap,
                  uint64_t* out_bytes, int threads);
 
+/* As orc_compress, with a plan's packed exponents (BF16): pack_lens (n_groups x 256
+ * packed-code lengths) and pack_exps (K listed exponents); K = 0 is orc_compress. */
+int orc_compress_packed(int dtype, const void* src, uint64_t n, uint32_t chunk_bytes, uint32_t S,
+                        const uint8_t* plan_lens, uint32_t n_groups, const uint8_t* pack_lens,
+                        const uint8_t* pack_exps, uint32_t K, void* out, uint64_t cap, uint64_t* out_bytes,
+                        int threads);
+uint64_t orc_max_compressed_bytes_packed(int dtype, uint64_t n, uint32_t chunk_bytes, uint32_t n_groups, uint32_t K);
+
+/* Pair-symbol histogram of the BF16 values [lo, lo + m) (m even) for K listed exponents,
+ * and the number of escaped exponents. */
+void orc_pack_histogram(const void* src, uint64_t lo, uint64_t m, const uint8_t* exps, uint32_t K, uint64_t* hist,
+                        uint64_t* escapes);
+
+/* Packed exponents of a plan (BF16): the list (16 bytes) and each group's packed code
+ * from the chunks' assignment. */
+int orc_plan_pack(const void* src, uint64_t n, uint32_t chunk_bytes, uint32_t n_groups, const uint32_t* assign,
+                  uint32_t max_pack, uint8_t* exps_out, uint8_t* lens_out, uint32_t* K_out);
+
 /* Decompress a container into n values. */
 int orc_decompress(int dtype, const void* in, uint64_t in_bytes, uint64_t n, uint32_t chunk_bytes,
                    void* out, int threads);

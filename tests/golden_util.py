@@ -87,6 +87,18 @@ def fp32_clean_two_chunk_input():
     return x
 
 
+def packed_pairs_input():
+    """The 64 BF16 values of bf16_packed_pairs.json: 2^(E - 127) for the stated exponents
+    (sign and fraction 0), with the exponent field (bits 14..7) checked."""
+    E = [127, 127, 126, 127, 127, 127, 127, 126] * 8
+    E[63] = 128
+    vals = [2.0 ** (e - 127) for e in E]
+    x = torch.tensor(vals, dtype=torch.float64).to(torch.bfloat16)
+    assert torch.equal(x.to(torch.float64), torch.tensor(vals, dtype=torch.float64))  # exact in BF16
+    assert [(v >> 7) & 0xFF for v in x.view(torch.int16).tolist()] == E
+    return x
+
+
 def _e2m1(nibble):
     """The number an E2M1 nibble stands for: sign bit 3, exponent bits 2..1, mantissa bit 0;
     exponent 0 is subnormal (mantissa * 0.5), else (1 + mantissa/2) * 2^(exponent - 1)."""
@@ -150,7 +162,8 @@ def expected_bytes(fx):
     buf = bytearray(h["total_bytes"])
     struct.pack_into("<4sHBBQIIIIQQQBBHI", buf, 0, h["magic"].encode(), h["version"], h["dtype"],
                      h["n_streams"], h["n"], h["chunk_bytes"], h["S"], h["n_chunks"], h["n_shared"],
-                     h["off_codes"], h["off_payload"], h["total_bytes"], h["lmax"], h["n_groups"], 0, 0)
+                     h["off_codes"], h["off_payload"], h["total_bytes"], h["lmax"], h["n_groups"],
+                     h.get("n_packed", 0), 0)
     for k, e in enumerate(fx["entries"]):
         struct.pack_into("<BBHIQ", buf, 64 + 16 * k, e["mode"], 0, 0, e["code"], e["offset"])
     for r in fx.get("records", []):
