@@ -745,6 +745,8 @@ def run_single(args):
     else:
         x = W.kv_cache(device=dev)
         desc = "BF16 K/V cache [32, 2, 16, 8, 4096, 128], per-channel std log-normal, 8-group plan"
+        if args.max_pack:
+            desc += f", up to {args.max_pack} packed exponents"
     x = x.reshape(-1)
     n = Z.nvalues(x)
     nbytes = x.numel() * x.element_size()
@@ -756,7 +758,7 @@ def run_single(args):
     if w == "kv_cache":
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        plan = Z.Plan.create(x, groups=8, seed=0, ws=ws)
+        plan = Z.Plan.create(x, groups=8, seed=0, ws=ws, max_pack=args.max_pack)
         e1.record(stream)
         torch.cuda.synchronize()
         setup_ms = e0.elapsed_time(e1)
@@ -796,6 +798,7 @@ def run_single(args):
         "compression_ratio": round(cbytes / nbytes, 5), "bytes": nbytes, "values": n,
         "peak": peak, "peak_source": peak_src, "steps": args.steps, "warmup": args.warmup,
         "plan_setup_ms": None if setup_ms is None else round(setup_ms, 2), "roundtrip_ok": bool(ok),
+        "max_pack": args.max_pack if w == "kv_cache" else None,
         "kernel_ms": ktimes,
     }
     print(json.dumps(line), flush=True)
@@ -818,6 +821,8 @@ def main():
     ap.add_argument("--rows", type=int, default=None,
                     help="rows of 4096 values for --workload fp32/fp32_clean/fp8/fp4 (profiler cases; "
                          "default 65536 FP32, 262144 FP8/FP4)")
+    ap.add_argument("--max-pack", type=int, default=0,
+                    help="--workload kv_cache: the plan also lists up to this many packed exponents (BF16, <= 15)")
     ap.add_argument("--plan-transfer", action="store_true",
                     help="instead of the benchmark: build a shared-code plan on layers 0-15 and reuse it on 16-31")
     ap.add_argument("--groups", type=int, default=8, help="plan groups for --plan-transfer")

@@ -16,20 +16,25 @@
  *    are entropy-coded independently.
  *  - "NeuralZip: Reusable Setup for Fast Lossless Compression" (abstract): chunks are
  *    grouped by the similarity of their exponent distributions, each group shares one
- *    Huffman code, and this setup (a "plan") is built once and reused.
+ *    Huffman code, and this setup (a "plan") is built once and reused. The same setup may
+ *    also choose packed exponents for recurring exponent tuples (BF16; see PACK below).
  *
  * Container format (all integers little-endian; every section and payload starts on a
  * 16-byte boundary; every pad byte and pad bit is zero):
  *   header, 64 bytes: 'Z','N','N','1' | u16 version=1 | u8 dtype | u8 n_streams |
  *     u64 n | u32 chunk_bytes | u32 S | u32 n_chunks | u32 n_shared | u64 off_codes |
- *     u64 off_payload | u64 total_bytes | u8 L_MAX=12 | u8 n_groups | 6 zero bytes
+ *     u64 off_payload | u64 total_bytes | u8 L_MAX=12 | u8 n_groups | u8 n_packed |
+ *     5 zero bytes
  *   chunk table at 64: one 16-byte entry per (chunk c, stream s), index k = c*n_streams+s:
- *     u8 mode (0 RAW, 1 ZERO, 2 HUFF, 3 ZRUN) | 3 zero bytes | u32 code | u64 payload offset.
- *     code is the shared record index for a HUFF entry coded with a plan's code, and
- *     0xFFFFFFFF otherwise.
- *   shared code records at off_codes (n_shared = n_groups * entropy streams), record
- *     r = e*n_groups + g: code lengths, 4 bits each (byte i = len[2i] | len[2i+1] << 4),
- *     padded to 16 bytes (128 bytes for a 256-symbol alphabet, 16 for FP8's).
+ *     u8 mode (0 RAW, 1 ZERO, 2 HUFF, 3 ZRUN, 4 PACK) | 3 zero bytes | u32 code |
+ *     u64 payload offset. code is the shared record index for a HUFF or PACK entry coded
+ *     with a plan's code, and 0xFFFFFFFF otherwise.
+ *   shared code records at off_codes (n_shared = n_groups * entropy streams, plus n_groups
+ *     with packed exponents), record r = e*n_groups + g: code lengths, 4 bits each (byte
+ *     i = len[2i] | len[2i+1] << 4), padded to 16 bytes (128 bytes for a 256-symbol
+ *     alphabet, 16 for FP8's). With n_packed = K > 0 (BF16 only): record n_groups + g is
+ *     group g's packed code over the 256 pair symbols, and the K packed exponents follow
+ *     the records, padded with zeros to 16 bytes.
  *   payloads at off_payload in increasing k, each at the running offset:
  *     RAW : the chunk's symbols at a fixed width, most significant bit first, padded.
  *     ZERO: nothing (every symbol of that chunk and stream is 0).
@@ -38,6 +43,14 @@
  *     ZRUN: zero runs of a byte plane: the chunk's symbols in blocks of 32 (the last may
  *           be shorter); [one bit per block, most significant first, 1 when the block
  *           holds a non-zero byte, padded] [the bytes of the marked blocks, padded].
+ *     PACK: packed exponent tuples (NeuralZip, abstract: recurring exponent tuples
+ *           represented by packed exponents), a BF16 exponent stream of a chunk with an
+ *           even value count: the exponents of values 2j and 2j+1 form the pair symbol
+ *           i(first) << 4 | i(second), i(x) = x's index among the K packed exponents, or
+ *           15 when x is not among them. [u32 idx[ceil(m/S)], padded] [bitstream, padded]:
+ *           every pair's code, followed by the 8 bits of its first exponent when that
+ *           one's index is 15, then of its second when that one's is; idx[j] is the bit
+ *           offset of the pair of value j*S.
  *   Streams: BF16 [exponent, sign+fraction byte]; FP32 [exponent, sign + fraction
  *   bits 22..16, fraction bits 15..8, fraction bits 7..0]; FP8 E4M3 [exponent (4 bits),
  *   mantissa (3 bits), sign (1 bit)]; FP4 E2M1 [exponent (2 bits), mantissa (1 bit),
@@ -46,7 +59,8 @@
  *   (sign bit 3, exponent bits 2..1, mantissa bit 0); n counts values and is even.
  *   Codes are canonical (RFC 1951 rule), at most 12 bits long.
  *   A stream is ZERO when all its symbols in the chunk are 0; an entropy stream is HUFF
- *   when that payload is strictly smaller than RAW, else RAW; a byte plane (BF16's
+ *   (PACK when the plan's packed code of a group codes it in strictly fewer bits than any
+ *   plain shared code) when that payload is strictly smaller than RAW, else RAW; a byte plane (BF16's
  *   sign+fraction byte, FP32's three fraction planes) is ZRUN when that payload is
  *   strictly smaller than RAW, else RAW; the 1-bit sign streams of FP8 and FP4 are RAW.
  *
@@ -93,9 +107,11 @@ typedef struct zipnn_plan zipnn_plan_t; /* opaque; owns device code tables */
 #define ZIPNN_DEFAULT_SUBBLOCK 512u       /* symbols per sub-block index entry */
 #define ZIPNN_MAX_GROUPS 64u
 #define ZIPNN_LMAX 12u
+#define ZIPNN_MAX_PACKED 15u
 
 /* Upper bound of the container size for n values: header, chunk table, room for
- * ZIPNN_MAX_GROUPS shared records, and every payload stored RAW (a HUFF payload is
+ * ZIPNN_MAX_GROUPS shared records (and, for BF16, their packed records and a list of
+ * ZIPNN_MAX_PACKED exponents), and every payload stored RAW (a HUFF payload is
  * only chosen when it is smaller). Returns 0 for invalid arguments.
  * chunk_bytes: a multiple of 16 in [16, 2^28]. */
 size_t zipnn_max_compressed_bytes(zipnn_dtype dtype, uint64_t n, uint32_t chunk_bytes);
@@ -197,17 +213,34 @@ zipnn_status zipnn_plan_create(zipnn_dtype dtype, const void* src, uint64_t n, u
                                uint32_t groups, uint64_t seed, void* ws, size_t ws_bytes,
                                zipnn_stream_t stream, zipnn_plan_t** plan);
 
+/* As zipnn_plan_create, and for BF16 with max_pack in 1..ZIPNN_MAX_PACKED also packed
+ * exponents ("NeuralZip: Reusable Setup for Fast Lossless Compression", abstract: the
+ * setup selectively represents recurring exponent tuples with packed exponents): the
+ * plan lists the K = min(max_pack, exponents present) most frequent exponents of the
+ * tensor (a larger count first, equal counts by the smaller exponent), and each group
+ * gets a second, packed code: the length-limited Huffman code of its member chunks'
+ * summed pair-symbol counts (chunks with an odd value count excluded; a group without
+ * pairs gets none). A chunk coded with such a plan takes the shared code, plain or
+ * packed, with the fewest bits (PACK in the container format). max_pack 0 is
+ * zipnn_plan_create; max_pack > 0 for another dtype, or above ZIPNN_MAX_PACKED, is
+ * ZIPNN_ERR_INVALID_ARG. */
+zipnn_status zipnn_plan_create_packed(zipnn_dtype dtype, const void* src, uint64_t n, uint32_t chunk_bytes,
+                                      uint32_t groups, uint64_t seed, uint32_t max_pack, void* ws, size_t ws_bytes,
+                                      zipnn_stream_t stream, zipnn_plan_t** plan);
+
 /* Serialise a plan into host memory, so that the setup can be stored and transferred
  * to other tensors or another compatible model (NeuralZip, abstract: the setup is
  * precomputed, transferred and reused as the weights evolve): "ZNP1", u8 dtype, u8
- * groups, 2 zero bytes, then the code records as in the container. *bytes receives the
+ * groups, u8 K (packed exponents, 0 for none), 1 zero byte, then the code section as in
+ * the container (plain records; with K > 0 the packed records and the list). *bytes receives the
  * size; host_buf may be NULL to query it; ZIPNN_ERR_OUT_TOO_SMALL if cap is short. */
 zipnn_status zipnn_plan_export(const zipnn_plan_t* plan, void* host_buf, size_t cap, size_t* bytes);
 
 /* Rebuild a plan from exported bytes (host memory; NeuralZip, abstract: a transferred
  * setup is reused without being rebuilt); allocates its device tables. Records whose
- * lengths exceed ZIPNN_LMAX or whose Kraft sum exceeds 1, or a damaged header, give
- * ZIPNN_ERR_CORRUPT. */
+ * lengths exceed ZIPNN_LMAX or whose Kraft sum exceeds 1, K above ZIPNN_MAX_PACKED (or
+ * above 0 for a dtype other than BF16), a non-zero byte past the list, or a damaged
+ * header, give ZIPNN_ERR_CORRUPT. */
 zipnn_status zipnn_plan_import(const void* host_buf, size_t bytes, zipnn_plan_t** plan);
 
 /* Per-chunk group chosen by the plan's k-means (NeuralZip, abstract: grouping of chunks

@@ -8,7 +8,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libzipnn_b200.so")
 SOURCES = ["api.cu", "prelude.cu", "decode.cu", "plan.cu", "timing.cu", "noalloc.cu", "encode_bf16.cu", "encode_fp32.cu",
-           "encode_sub.cu", "shard.cu"]
+           "encode_sub.cu", "shard.cu", "pack.cu"]
 HEADERS = ["bulk.cuh", "common.cuh", "fields.cuh", "huffman.cuh", "launch.h"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

@@ -20,6 +20,11 @@ struct zipnn_plan {
   uint32_t* d_enc;   // [n_entropy][groups][256]
   std::vector<uint8_t> h_lens;
   std::vector<uint32_t> assign;
+  // packed exponents (BF16): K listed, and one device block holding the list (16 bytes),
+  // K as a u32, the packed lengths [groups][256] and their codes [groups][256]
+  uint32_t pack_k = 0;
+  uint8_t* d_pack = nullptr;
+  std::vector<uint8_t> h_pack_exps, h_pack_lens;
 };
 
 namespace {
@@ -37,7 +42,7 @@ inline uint64_t align_up(uint64_t x) { return (x + kAlign - 1) & ~(kAlign - 1); 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 inline bool valid_dtype(int dt) { return dt == kBF16 || dt == kFP32 || dt == kFP8 || dt == kFP4; }
 
-bool make_geo(int dt, uint64_t n, uint32_t chunk_bytes, uint32_t S, uint32_t G, Geo& g) {
+bool make_geo(int dt, uint64_t n, uint32_t chunk_bytes, uint32_t S, uint32_t G, Geo& g, uint32_t K = 0) {
   if (!valid_dtype(dt) || n == 0 || n >= kMaxValues) return false;
   if (dt == kFP4 && n % 2) return false;  // FP4 values come in byte pairs
   if (chunk_bytes < 16 || chunk_bytes % 16 || chunk_bytes > kMaxChunkBytes) return false;
@@ -52,11 +57,12 @@ bool make_geo(int dt, uint64_t n, uint32_t chunk_bytes, uint32_t S, uint32_t G, 
   g.n_chunks = (uint32_t)chunks;
   g.S = S;
   g.n_groups = G;
+  g.n_packed = K;
   g.tiles_per_chunk = (uint32_t)tpc;
   g.n_tiles = (uint32_t)(chunks * tpc);
   g.n_entries = (uint32_t)(chunks * n_streams(dt));
   g.off_codes = kHeaderBytes + (uint64_t)kEntryBytes * g.n_entries;
-  g.off_payload = g.off_codes + shared_bytes(dt, G);
+  g.off_payload = g.off_codes + code_section_bytes(dt, G, K);
   const uint32_t lim = g_spin_limit.load(std::memory_order_relaxed);
   g.spin_limit = lim ? lim : kSpinLimit;
   g.zwords = (uint32_t)ceil_div(ceil_div(g.m0, kZBlock), 32);
@@ -65,7 +71,7 @@ bool make_geo(int dt, uint64_t n, uint32_t chunk_bytes, uint32_t S, uint32_t G, 
 
 struct WsPlan {
   uint64_t status, hist, nonzero, zmap, zcount, scan_desc, slot, zero_end;
-  uint64_t esize, emode, ecode, eoff, enc, tile_hist, tile_off;
+  uint64_t esize, emode, ecode, eoff, enc, tile_hist, tile_off, pack_hist, pack_esc;
   uint64_t km_mu, km_perm, km_assign, km_changed, km_gsum, total;
   bool tile_counts;  // per-tile histograms and bit offsets (every compress)
   int dt;
@@ -92,6 +98,8 @@ WsPlan ws_plan(const Geo& g) {
   p.tile_counts = true;
   p.tile_hist = o;  o = align_up(o + (p.tile_counts ? (uint64_t)g.n_tiles * tile_bins(g.dt) * 2 : 0));
   p.tile_off = o;   o = align_up(o + (p.tile_counts ? NE * g.n_tiles * 4 : 0));
+  p.pack_hist = o;  o = align_up(o + (g.dt == kBF16 ? C * 256 * 4 : 0));
+  p.pack_esc = o;   o = align_up(o + (g.dt == kBF16 ? C * 4 : 0));
   p.km_mu = o;      o = align_up(o + (uint64_t)kMaxGroups * 256 * 8);
   p.km_perm = o;    o = align_up(o + C * 4);
   p.km_assign = o;  o = align_up(o + C * 4);
@@ -118,11 +126,13 @@ Ws carve(const WsPlan& p, void* base) {
   w.enc = reinterpret_cast<uint32_t*>(b + p.enc);
   w.tile_hist = p.tile_counts ? reinterpret_cast<uint16_t*>(b + p.tile_hist) : nullptr;
   w.tile_off = p.tile_counts ? reinterpret_cast<uint32_t*>(b + p.tile_off) : nullptr;
+  w.pack_hist = p.dt == kBF16 ? reinterpret_cast<uint32_t*>(b + p.pack_hist) : nullptr;
+  w.pack_esc = p.dt == kBF16 ? reinterpret_cast<uint32_t*>(b + p.pack_esc) : nullptr;
   return w;
 }
 
 uint64_t max_bytes(const Geo& g) {
-  uint64_t total = g.off_codes + shared_bytes(g.dt, kMaxGroups);
+  uint64_t total = g.off_codes + code_section_bytes(g.dt, kMaxGroups, g.dt == kBF16 ? kPackMax : 0);
   const uint64_t full = g.n / g.m0, tail = g.n % g.m0;
   for (int s = 0; s < n_streams(g.dt); s++) {
     const int w = raw_width(g.dt, s);
@@ -139,6 +149,10 @@ PlanDev plan_dev(const zipnn_plan* p) {
   d.lens = p ? p->d_lens : nullptr;
   d.enc = p ? p->d_enc : nullptr;
   d.groups = p ? p->groups : 0;
+  d.pack_k = p ? p->pack_k : 0;
+  d.pack_exps = p && p->d_pack ? p->d_pack : nullptr;
+  d.pack_lens = p && p->d_pack ? p->d_pack + 32 : nullptr;
+  d.pack_enc = p && p->d_pack ? reinterpret_cast<const uint32_t*>(p->d_pack + 32 + (size_t)p->groups * 256) : nullptr;
   return d;
 }
 
@@ -184,7 +198,8 @@ zipnn_status zipnn_compress_ex(zipnn_dtype dtype, const void* src, uint64_t n, u
   if (!src || !out || !ws || !aligned16(src) || !aligned16(out) || !aligned16(ws)) return ZIPNN_ERR_INVALID_ARG;
   if (plan && plan->dt != (int)dtype) return ZIPNN_ERR_PLAN_MISMATCH;
   Geo g;
-  if (!make_geo(dtype, n, chunk_bytes, subblock, plan ? plan->groups : 0, g)) return ZIPNN_ERR_INVALID_ARG;
+  if (!make_geo(dtype, n, chunk_bytes, subblock, plan ? plan->groups : 0, g, plan ? plan->pack_k : 0))
+    return ZIPNN_ERR_INVALID_ARG;
   if (out_cap < max_bytes(g)) return ZIPNN_ERR_OUT_TOO_SMALL;
   const WsPlan wp = ws_plan(g);
   if (ws_bytes < wp.total) return ZIPNN_ERR_OUT_TOO_SMALL;
@@ -196,6 +211,10 @@ zipnn_status zipnn_compress_ex(zipnn_dtype dtype, const void* src, uint64_t n, u
   if (e == cudaSuccess) {
     TimedLaunch t(kIdHist, st);
     e = launch_split_hist(src, g, w.hist, w.nonzero, &w, pd, st);
+  }
+  if (e == cudaSuccess && pd.pack_k) {
+    TimedLaunch t(kIdPackHist, st);
+    e = launch_pack_hist(src, g, w, pd, st);
   }
   if (e == cudaSuccess) {
     TimedLaunch t(kIdBuild, st);
@@ -210,6 +229,10 @@ zipnn_status zipnn_compress_ex(zipnn_dtype dtype, const void* src, uint64_t n, u
     e = g.dt == kBF16 ? launch_encode_bf16(src, g, w, static_cast<uint8_t*>(out), st)
         : g.dt == kFP32 ? launch_encode_fp32(src, g, w, static_cast<uint8_t*>(out), st)
                         : launch_encode_sub(src, g, w, static_cast<uint8_t*>(out), st);
+  }
+  if (e == cudaSuccess && pd.pack_k) {
+    TimedLaunch t(kIdPackEncode, st);
+    e = launch_encode_pack(src, g, w, pd, static_cast<uint8_t*>(out), st);
   }
   return cuda_status(e);
 }
@@ -336,9 +359,28 @@ static zipnn_status plan_alloc(int dt, uint32_t groups, zipnn_plan** out) {
   return ZIPNN_OK;
 }
 
+static zipnn_status pack_alloc(zipnn_plan* p) {
+  const size_t bytes = 32 + (size_t)p->groups * 256 * 5;
+  if (cudaMalloc(&p->d_pack, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    p->d_pack = nullptr;
+    return ZIPNN_ERR_CUDA;
+  }
+  p->h_pack_exps.assign(kPackListBytes, 0);
+  p->h_pack_lens.assign((size_t)p->groups * 256, 0);
+  return ZIPNN_OK;
+}
+
 zipnn_status zipnn_plan_create(zipnn_dtype dtype, const void* src, uint64_t n, uint32_t chunk_bytes, uint32_t groups,
                                uint64_t seed, void* ws, size_t ws_bytes, zipnn_stream_t stream, zipnn_plan_t** plan) {
+  return zipnn_plan_create_packed(dtype, src, n, chunk_bytes, groups, seed, 0, ws, ws_bytes, stream, plan);
+}
+
+zipnn_status zipnn_plan_create_packed(zipnn_dtype dtype, const void* src, uint64_t n, uint32_t chunk_bytes,
+                                      uint32_t groups, uint64_t seed, uint32_t max_pack, void* ws, size_t ws_bytes,
+                                      zipnn_stream_t stream, zipnn_plan_t** plan) {
   if (!src || !ws || !plan || !aligned16(src) || !aligned16(ws)) return ZIPNN_ERR_INVALID_ARG;
+  if (max_pack > kPackMax || (max_pack && dtype != ZIPNN_BF16)) return ZIPNN_ERR_INVALID_ARG;
   if (groups < 1 || groups > kMaxGroups) return ZIPNN_ERR_INVALID_ARG;
   Geo g;
   if (!make_geo(dtype, n, chunk_bytes, ZIPNN_DEFAULT_SUBBLOCK, 0, g)) return ZIPNN_ERR_INVALID_ARG;
@@ -388,6 +430,31 @@ zipnn_status zipnn_plan_create(zipnn_dtype dtype, const void* src, uint64_t n, u
   for (int ei = 0; ei < NE && e == cudaSuccess; ei++)
     e = launch_code_lengths(k.gsum + (size_t)ei * groups * 256, groups, (uint32_t)alphabet(dtype, ei),
                             p->d_lens + (size_t)ei * groups * 256, p->d_enc + (size_t)ei * groups * 256, st);
+  if (e == cudaSuccess && max_pack) {
+    // packed exponents: the list from the exponent counts, the chunks' pair counts, and
+    // each group's packed code from its members' summed pair counts
+    if (pack_alloc(p) != ZIPNN_OK) e = cudaErrorMemoryAllocation;
+    uint32_t K = 0;
+    if (e == cudaSuccess)
+      e = launch_pack_select(w.hist, g.n_chunks, (uint32_t)NE, max_pack, p->d_pack,
+                             reinterpret_cast<uint32_t*>(p->d_pack + 16), st);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&K, p->d_pack + 16, 4, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e == cudaSuccess && K) {
+      p->pack_k = K;
+      const PlanDev pd = plan_dev(p);
+      e = launch_pack_hist(src, g, w, pd, st);
+      if (e == cudaSuccess) e = cudaMemsetAsync(k.gsum, 0, (size_t)groups * 256 * 8, st);
+      if (e == cudaSuccess) e = launch_pack_group_sums(w.pack_hist, k.assign, g.n_chunks, k.gsum, st);
+      if (e == cudaSuccess)
+        e = launch_code_lengths(k.gsum, groups, 256, p->d_pack + 32,
+                                reinterpret_cast<uint32_t*>(p->d_pack + 32 + (size_t)groups * 256), st);
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync(p->h_pack_exps.data(), p->d_pack, kPackListBytes, cudaMemcpyDeviceToHost, st);
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync(p->h_pack_lens.data(), p->d_pack + 32, p->h_pack_lens.size(), cudaMemcpyDeviceToHost, st);
+    }
+  }
   if (e == cudaSuccess) {
     p->assign.resize(g.n_chunks);
     e = cudaMemcpyAsync(p->h_lens.data(), p->d_lens, p->h_lens.size(), cudaMemcpyDeviceToHost, st);
@@ -406,7 +473,8 @@ zipnn_status zipnn_plan_create(zipnn_dtype dtype, const void* src, uint64_t n, u
 zipnn_status zipnn_plan_export(const zipnn_plan_t* plan, void* host_buf, size_t cap, size_t* bytes) {
   if (!plan || !bytes) return ZIPNN_ERR_INVALID_ARG;
   const int dt = plan->dt, NE = n_entropy(dt);
-  const size_t need = 8 + shared_bytes(dt, plan->groups);
+  const uint32_t G = plan->groups, K = plan->pack_k;
+  const size_t need = 8 + code_section_bytes(dt, G, K);
   *bytes = need;
   if (!host_buf) return ZIPNN_OK;
   if (cap < need) return ZIPNN_ERR_OUT_TOO_SMALL;
@@ -417,59 +485,89 @@ zipnn_status zipnn_plan_export(const zipnn_plan_t* plan, void* host_buf, size_t 
   o[2] = 'P';
   o[3] = '1';
   o[4] = (uint8_t)dt;
-  o[5] = (uint8_t)plan->groups;
+  o[5] = (uint8_t)G;
+  o[6] = (uint8_t)K;
   for (int e = 0; e < NE; e++) {
     const int A = alphabet(dt, e);
-    for (uint32_t gi = 0; gi < plan->groups; gi++) {
-      const uint8_t* l = plan->h_lens.data() + ((size_t)e * plan->groups + gi) * 256;
-      uint8_t* r = o + 8 + shared_record_pos(dt, plan->groups, (uint32_t)e * plan->groups + gi);
+    for (uint32_t gi = 0; gi < G; gi++) {
+      const uint8_t* l = plan->h_lens.data() + ((size_t)e * G + gi) * 256;
+      uint8_t* r = o + 8 + shared_record_pos(dt, G, (uint32_t)e * G + gi);
       for (int i = 0; i < A / 2; i++) r[i] = (uint8_t)(l[2 * i] | (l[2 * i + 1] << 4));
     }
   }
+  if (K) {
+    for (uint32_t gi = 0; gi < G; gi++) {
+      const uint8_t* l = plan->h_pack_lens.data() + (size_t)gi * 256;
+      uint8_t* r = o + 8 + packed_record_pos(dt, G, gi);
+      for (int i = 0; i < 128; i++) r[i] = (uint8_t)(l[2 * i] | (l[2 * i + 1] << 4));
+    }
+    std::memcpy(o + need - kPackListBytes, plan->h_pack_exps.data(), K);
+  }
   return ZIPNN_OK;
+}
+
+// 4-bit lengths of a record into l[0..A): every length at most 12, the Kraft sum at most 1,
+// and the record's bytes past the alphabet zero.
+static bool read_lengths(const uint8_t* r, int A, uint32_t rb, uint8_t* l) {
+  uint64_t kraft = 0;
+  for (int i = 0; i < A; i++) {
+    l[i] = (i & 1) ? (r[i >> 1] >> 4) : (r[i >> 1] & 15);
+    if (l[i] > kLmax) return false;
+    if (l[i]) kraft += 1ull << (kLmax - l[i]);
+  }
+  for (uint32_t i = (uint32_t)A / 2; i < rb; i++)
+    if (r[i]) return false;
+  return kraft <= (1ull << kLmax);
 }
 
 zipnn_status zipnn_plan_import(const void* host_buf, size_t bytes, zipnn_plan_t** plan) {
   if (!host_buf || !plan || bytes < 8) return ZIPNN_ERR_INVALID_ARG;
   const uint8_t* in = static_cast<const uint8_t*>(host_buf);
-  if (in[0] != 'Z' || in[1] != 'N' || in[2] != 'P' || in[3] != '1' || in[6] || in[7]) return ZIPNN_ERR_CORRUPT;
+  if (in[0] != 'Z' || in[1] != 'N' || in[2] != 'P' || in[3] != '1' || in[7]) return ZIPNN_ERR_CORRUPT;
   const int dt = in[4];
-  const uint32_t groups = in[5];
+  const uint32_t groups = in[5], K = in[6];
   if (!valid_dtype(dt) || groups < 1 || groups > kMaxGroups) return ZIPNN_ERR_CORRUPT;
-  if (bytes < 8 + shared_bytes(dt, groups)) return ZIPNN_ERR_CORRUPT;
+  if (K > kPackMax || (K && dt != kBF16)) return ZIPNN_ERR_CORRUPT;
+  const size_t need = 8 + code_section_bytes(dt, groups, K);
+  if (bytes < need) return ZIPNN_ERR_CORRUPT;
+  for (size_t i = need - kPackListBytes + K; K && i < need; i++)
+    if (in[i]) return ZIPNN_ERR_CORRUPT;
   if (!device_ok()) return ZIPNN_ERR_UNSUPPORTED;
   zipnn_plan* p = nullptr;
   zipnn_status zs = plan_alloc(dt, groups, &p);
   if (zs != ZIPNN_OK) return zs;
   const int NE = n_entropy(dt);
-  for (int e = 0; e < NE; e++) {
-    const int A = alphabet(dt, e);
-    const uint32_t rb = record_bytes(dt, e);
-    for (uint32_t gi = 0; gi < groups; gi++) {
-      const uint8_t* r = in + 8 + shared_record_pos(dt, groups, (uint32_t)e * groups + gi);
-      uint8_t* l = p->h_lens.data() + ((size_t)e * groups + gi) * 256;
-      uint64_t kraft = 0;
-      for (int i = 0; i < A; i++) {
-        l[i] = (i & 1) ? (r[i >> 1] >> 4) : (r[i >> 1] & 15);
-        if (l[i] > kLmax) {
-          zipnn_plan_destroy(p);
-          return ZIPNN_ERR_CORRUPT;
-        }
-        if (l[i]) kraft += 1ull << (kLmax - l[i]);
-      }
-      for (uint32_t i = (uint32_t)A / 2; i < rb; i++)
-        if (r[i]) {
-          zipnn_plan_destroy(p);
-          return ZIPNN_ERR_CORRUPT;
-        }
-      if (kraft > (1ull << kLmax)) {
-        zipnn_plan_destroy(p);
-        return ZIPNN_ERR_CORRUPT;
-      }
+  bool ok = true;
+  for (int e = 0; e < NE && ok; e++)
+    for (uint32_t gi = 0; gi < groups && ok; gi++)
+      ok = read_lengths(in + 8 + shared_record_pos(dt, groups, (uint32_t)e * groups + gi), alphabet(dt, e),
+                        record_bytes(dt, e), p->h_lens.data() + ((size_t)e * groups + gi) * 256);
+  if (ok && K) {
+    if (pack_alloc(p) != ZIPNN_OK) {
+      zipnn_plan_destroy(p);
+      return ZIPNN_ERR_CUDA;
     }
+    p->pack_k = K;
+    std::memcpy(p->h_pack_exps.data(), in + need - kPackListBytes, kPackListBytes);
+    for (uint32_t gi = 0; gi < groups && ok; gi++)
+      ok = read_lengths(in + 8 + packed_record_pos(dt, groups, gi), 256, 128, p->h_pack_lens.data() + (size_t)gi * 256);
+  }
+  if (!ok) {
+    zipnn_plan_destroy(p);
+    return ZIPNN_ERR_CORRUPT;
   }
   cudaError_t e = cudaMemcpy(p->d_lens, p->h_lens.data(), p->h_lens.size(), cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = launch_canonical(p->d_lens, (uint32_t)NE * groups, p->d_enc, 0);
+  if (e == cudaSuccess && K) {
+    uint8_t head[32] = {0};
+    std::memcpy(head, p->h_pack_exps.data(), kPackListBytes);
+    std::memcpy(head + 16, &K, 4);
+    e = cudaMemcpy(p->d_pack, head, 32, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess)
+      e = cudaMemcpy(p->d_pack + 32, p->h_pack_lens.data(), p->h_pack_lens.size(), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess)
+      e = launch_canonical(p->d_pack + 32, groups, reinterpret_cast<uint32_t*>(p->d_pack + 32 + (size_t)groups * 256), 0);
+  }
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
     zipnn_plan_destroy(p);
@@ -492,6 +590,7 @@ void zipnn_plan_destroy(zipnn_plan_t* plan) {
   if (!plan) return;
   if (plan->d_lens) cudaFree(plan->d_lens);
   if (plan->d_enc) cudaFree(plan->d_enc);
+  if (plan->d_pack) cudaFree(plan->d_pack);
   delete plan;
 }
 

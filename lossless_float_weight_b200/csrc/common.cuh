@@ -13,7 +13,12 @@ namespace zipnn {
 
 constexpr int kLmax = 12;
 constexpr uint32_t kNoCode = 0xFFFFFFFFu;
-constexpr uint32_t kModeRaw = 0, kModeZero = 1, kModeHuff = 2, kModeZrun = 3;
+constexpr uint32_t kModeRaw = 0, kModeZero = 1, kModeHuff = 2, kModeZrun = 3, kModePack = 4;
+// Packed exponents (BF16 with a plan that lists them): a pair of exponents is one 8-bit
+// symbol, each exponent's index in the plan's list as a nibble, kPackEsc for one that is
+// not listed (its 8 bits follow the pair's code). The list holds at most kPackMax entries
+// and takes kPackListBytes at the end of the code section.
+constexpr uint32_t kPackMax = 15, kPackEsc = 15, kPackListBytes = 16;
 // Zero runs: a byte plane is taken in blocks of 32 symbols; ZRUN keeps a bitmap of the
 // blocks that hold a non-zero byte and the bytes of those blocks only.
 constexpr uint32_t kZBlock = 32;
@@ -78,12 +83,22 @@ __host__ __device__ inline uint64_t shared_record_pos(int dt, uint32_t g, uint32
   return pos + (uint64_t)k * record_bytes(dt, (int)e);
 }
 
+// The code section with K packed exponents: the plain records, then (K > 0) one packed
+// record per group and the list.
+__host__ __device__ inline uint64_t code_section_bytes(int dt, uint32_t g, uint32_t K) {
+  return shared_bytes(dt, g) + (K ? (uint64_t)g * record_bytes(dt, 0) + kPackListBytes : 0);
+}
+__host__ __device__ inline uint64_t packed_record_pos(int dt, uint32_t g, uint32_t gi) {
+  return shared_bytes(dt, g) + (uint64_t)gi * record_bytes(dt, 0);
+}
+
 // Geometry of one call.
 struct Geo {
   int dt;
   uint64_t n;
   uint32_t chunk_bytes, m0, n_chunks, S;
   uint32_t n_groups;          // 0 without a plan
+  uint32_t n_packed;          // packed exponents the plan lists (BF16), 0 for none
   uint32_t tiles_per_chunk;   // encode tiles (tile_values(dt) values) per chunk
   uint32_t n_tiles;           // n_chunks * tiles_per_chunk
   uint32_t n_entries;         // n_chunks * n_streams
@@ -112,6 +127,8 @@ struct Ws {
   uint16_t* tile_hist;  // [n_tiles][tile_bins] (compress): counts of each encode tile
   uint32_t* tile_off;   // [n_entropy][n_tiles] (compress): bit offset of each tile in its
                         // chunk's bitstream of that entropy stream
+  uint32_t* pack_hist;  // [n_chunks][256] (BF16 with packed exponents): pair-symbol counts
+  uint32_t* pack_esc;   // [n_chunks]: escaped exponents
 };
 
 // Device-side tables of a plan.
@@ -119,6 +136,10 @@ struct PlanDev {
   const uint8_t* lens;  // [n_entropy][groups][256]
   const uint32_t* enc;  // [n_entropy][groups][256]: len << 16 | code
   uint32_t groups;
+  uint32_t pack_k;           // packed exponents listed (BF16), 0 for none
+  const uint8_t* pack_exps;  // [16]: the list, then zeros
+  const uint8_t* pack_lens;  // [groups][256]: packed code lengths
+  const uint32_t* pack_enc;  // [groups][256]: len << 16 | code
 };
 
 __device__ __forceinline__ void set_status(uint32_t* st, uint32_t code) { atomicCAS(st, 0u, code); }

@@ -33,6 +33,9 @@ __device__ __forceinline__ uint32_t lut_symbol(uint32_t e) { return (e >> 16) & 
 
 __device__ const uint32_t kZeroWord[1] = {0};  // the word an empty stream reads
 
+// Streams decoded through a code table: HUFF, and PACK (packed exponent pairs).
+__device__ __forceinline__ bool coded(uint32_t mode) { return mode == kModeHuff || mode == kModePack; }
+
 // Big-endian-within-word bit reader over 32-bit words [0, nwords); a read past the last
 // word sees the last word (a valid stream never consumes those bits; one that does ends
 // past its bound and is reported). buf holds nb valid bits, most significant first; the next two words
@@ -110,10 +113,11 @@ __device__ __forceinline__ uint32_t huff_pair(Reader& br, const uint32_t* lut, u
   return (e & 0x00FF0000u) | ((e2 & 0x00FF0000u) << 8);
 }
 
-enum Kind : int { kKZero = 0, kKBytes = 1, kKBits = 2, kKHuff = 3, kKZrun = 4 };
+enum Kind : int { kKZero = 0, kKBytes = 1, kKBits = 2, kKHuff = 3, kKZrun = 4, kKPack = 5 };
 
 struct StreamState {
-  int kind, width;
+  int kind, width;       // kKPack: width is the number of packed exponents K
+  const uint8_t* pexp;   // kKPack: the packed exponents
   const uint8_t* bytes;  // kKBytes: this sub-block's first byte; kKZrun: the kept bytes
   BitReader br;
   const uint32_t* lut;
@@ -158,6 +162,24 @@ __device__ __forceinline__ uint64_t next_packed(StreamState& st, int n, uint32_t
           b = i + 1 < n ? st.br.huff(st.lut, st.acc) : 0u;
         }
         o |= (uint64_t)(a | (b << SB)) << (SB * i);
+      }
+      break;
+    case kKPack:
+      if constexpr (SB == 8) {
+        // packed exponent pairs: one code a pair (a refill leaves at least 32 bits: a
+        // code and two escaped exponents take at most 28)
+#pragma unroll
+        for (int i = 0; i < GV; i += 2) {
+          if (!FULL && i >= n) break;
+          st.br.refill();
+          const uint32_t p = st.br.huff(st.lut, st.acc);
+          const uint32_t hi = p >> 4, lo = p & 15u;
+          const uint32_t a = hi == kPackEsc ? st.br.fixed(8) : st.pexp[hi];
+          const uint32_t b = lo == kPackEsc ? st.br.fixed(8) : st.pexp[lo];
+          if ((hi != kPackEsc && hi >= (uint32_t)st.width) || (lo != kPackEsc && lo >= (uint32_t)st.width))
+            st.acc |= kLutInvalid;  // an index past the list: corrupt
+          o |= (uint64_t)(a | (b << 8)) << (8 * i);
+        }
       }
       break;
     case kKBits:
@@ -747,7 +769,8 @@ struct DecodeSmem {
   uint32_t mode[n_streams(DT)], code[n_streams(DT)];
   uint64_t off[n_streams(DT)], end[n_streams(DT)];
   uint64_t off_codes;
-  uint32_t S, G;
+  uint32_t S, G, K;                 // K: packed exponents (BF16), 0 for none
+  uint8_t pack_exps[kPackListBytes];
   int bad, staged;
   int quad;  // FP4 exponent stream with codes of at most 3 bits: table entries hold 4 symbols
 };
@@ -966,7 +989,9 @@ __device__ __forceinline__ void decode_generic(const uint8_t* __restrict__ in, c
         } else {
           expect_end[s] = cap_bits;
         }
-        st[s].kind = kKHuff;
+        st[s].kind = mode == kModePack ? kKPack : kKHuff;
+        st[s].width = (int)sm.K;
+        st[s].pexp = sm.pack_exps;
         st[s].lut = sm.lut[e];
         st[s].br.init(reinterpret_cast<const uint32_t*>(in + bs_off), (uint32_t)(cap_bits / 32), bad ? 0 : start);
       }
@@ -1046,7 +1071,7 @@ __device__ __forceinline__ void decode_generic(const uint8_t* __restrict__ in, c
 #pragma unroll
     for (int s = 0; s < NS; s++) {
       if (st[s].kind == kKZrun && st[s].zbad) bad = 1;
-      if (st[s].kind != kKHuff) continue;
+      if (st[s].kind != kKHuff && st[s].kind != kKPack) continue;
       const uint64_t pos = st[s].br.position();
       if (st[s].acc & kLutInvalid) bad = 1;
       if (check_exact[s] ? pos != expect_end[s] : pos > expect_end[s]) bad = 1;
@@ -1077,7 +1102,7 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
   if (tid == 0) {
     int bad = 0;
     uint64_t total = 0, off_codes = 0, off_payload = 0;
-    uint32_t S = 0, G = 0;
+    uint32_t S = 0, G = 0, K = 0;
     const uint64_t entries = (uint64_t)g.n_chunks * NS;
     const uint64_t k0 = (uint64_t)c * NS;
     if (in_bytes < kHeaderBytes + kEntryBytes * (k0 + NS)) {
@@ -1106,18 +1131,31 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
       if (hv[0] != 0x314E4E5Au || hv[1] != (1u | ((uint32_t)DT << 16) | ((uint32_t)NS << 24))) bad = 1;
       if (n != g.n || hv[4] != g.chunk_bytes || hv[6] != g.n_chunks) bad = 1;
       if (S == 0 || (S & 15) || S > 65536) bad = 1;
-      if ((hv[14] & 0xFF) != (uint32_t)kLmax || (hv[14] >> 16) != 0 || hv[15] != 0) bad = 1;
-      if (G > kMaxGroups || hv[7] != G * NE) bad = 1;
+      K = (hv[14] >> 16) & 0xFF;
+      if ((hv[14] & 0xFF) != (uint32_t)kLmax || (hv[14] >> 24) != 0 || hv[15] != 0) bad = 1;
+      if (K > kPackMax || (K && (DT != kBF16 || G == 0))) bad = 1;
+      if (G > kMaxGroups || hv[7] != G * NE + (K ? G : 0u)) bad = 1;
       if (off_codes != kHeaderBytes + entries * kEntryBytes) bad = 1;
-      if (!bad && off_payload != off_codes + shared_bytes(DT, G)) bad = 1;
+      if (!bad && off_payload != off_codes + code_section_bytes(DT, G, K)) bad = 1;
       if (total > in_bytes || total < off_payload || (total & 15)) bad = 1;
+      if (!bad && K) {
+        // the list of packed exponents: K entries, then zeros
+        const uint4 q = *reinterpret_cast<const uint4*>(in + off_payload - kPackListBytes);
+        const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int i = 0; i < 16; i++) {
+          const uint32_t b = (qw[i >> 2] >> (8 * (i & 3))) & 0xFFu;
+          sm.pack_exps[i] = (uint8_t)b;
+          if (i >= (int)K && b) bad = 1;
+        }
+      }
 #pragma unroll
       for (int s = 0; s < NS; s++) {
         const uint64_t k = k0 + s;
         const uint64_t off = ent[s].z | ((uint64_t)ent[s].w << 32);
         const uint64_t end = k + 1 < entries ? (ent[s + 1].z | ((uint64_t)ent[s + 1].w << 32)) : total;
         const uint32_t mode = ent[s].x & 0xFF;
-        if ((ent[s].x >> 8) != 0 || mode > kModeZrun) bad = 1;
+        if ((ent[s].x >> 8) != 0 || mode > kModePack) bad = 1;
         if ((off & 15) || (end & 15) || off > end || end > total || off < off_payload) bad = 1;
         if (k == 0 && off != off_payload) bad = 1;
         const uint64_t extent = end - off;
@@ -1135,6 +1173,11 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
           else if (ent[s].y == kNoCode) need += record_bytes(DT, s);
           else if (G == 0 || ent[s].y >= G * NE || ent[s].y / G != (uint32_t)s) bad = 1;
           if (extent < need) bad = 1;
+        } else if (mode == kModePack && S != 0) {
+          // packed exponent pairs: a BF16 exponent stream of whole pairs, a packed record
+          if (DT != kBF16 || s != 0 || K == 0 || (m & 1u)) bad = 1;
+          else if (ent[s].y < G * NE || ent[s].y >= G * NE + G) bad = 1;
+          if (extent < round16(4 * ceil_div(m, S))) bad = 1;
         }
         sm.mode[s] = mode;
         sm.code[s] = ent[s].y;
@@ -1145,6 +1188,7 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
     sm.off_codes = off_codes;
     sm.S = S;
     sm.G = G;
+    sm.K = K;
     sm.bad = bad;
     sm.staged = 0;
     if constexpr (DT == kBF16) {
@@ -1221,9 +1265,11 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
   for (int e = 0; e < NE; e++) {
     my_len[e] = 0;
     my_rank[e] = 0;
-    if (sm.mode[e] != kModeHuff) continue;  // uniform
+    if (!coded(sm.mode[e])) continue;  // uniform
     const uint8_t* rp = sm.code[e] == kNoCode ? in + sm.off[e]
-                                              : in + sm.off_codes + shared_record_pos(DT, sm.G, sm.code[e]);
+                        : sm.mode[e] == kModePack
+                            ? in + sm.off_codes + packed_record_pos(DT, sm.G, sm.code[e] - sm.G * NE)
+                            : in + sm.off_codes + shared_record_pos(DT, sm.G, sm.code[e]);
     uint32_t l = 0;
     if (tid < alphabet(DT, e)) {
       const uint32_t b = rp[tid >> 1];
@@ -1265,7 +1311,7 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
   // count[l-1]) << 1, i.e. the sum over q < l of count[q] << (l - q)), canonical index
   // offsets, left-aligned limits, and every warp's base index for each length; lane l
   // takes length l. A length above 12, no symbol, or a Kraft sum above 1 is corrupt.
-  if (warp < NE && sm.mode[warp] == kModeHuff) {
+  if (warp < NE && coded(sm.mode[warp])) {
     const int e = warp;
     uint32_t kraft = 0, fl = 0;
 #pragma unroll
@@ -1324,7 +1370,7 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
   // symbols in canonical order
 #pragma unroll
   for (int e = 0; e < NE; e++) {
-    if (sm.mode[e] != kModeHuff || !my_len[e]) continue;
+    if (!coded(sm.mode[e]) || !my_len[e]) continue;
     const uint32_t k = sm.base[e][warp][my_len[e]] + my_rank[e];
     sm.sorted[e][k] = (uint8_t)tid;
     sm.slen[e][k] = (uint8_t)my_len[e];
@@ -1336,7 +1382,7 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
   uint16_t* const lut16 = reinterpret_cast<uint16_t*>(sm.lut[0] + (kWideWords - kWindowWords));
 #pragma unroll
   for (int e = 0; e < NE; e++) {
-    if (sm.mode[e] != kModeHuff) continue;
+    if (!coded(sm.mode[e])) continue;
     if (wide) fill_lut<true>(lut16, sm.sorted[e], sm.slen[e], sm.limit[e], sm.first[e], sm.offset[e]);
     else fill_lut<false>(sm.lut[e], sm.sorted[e], sm.slen[e], sm.limit[e], sm.first[e], sm.offset[e]);
   }
@@ -1358,7 +1404,7 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
     if (tid == 0) sm.quad = quad;
 #pragma unroll
     for (int e = 0; e < NE; e++) {
-      if (sm.mode[e] != kModeHuff) continue;
+      if (!coded(sm.mode[e])) continue;
       any = true;
       if (e == 0 && quad) {
         for (uint32_t x = tid; x < 4096; x += kDecodeThreads) {

@@ -35,8 +35,8 @@ struct HuffBlockSmem {
   uint64_t f[256];
   HuffScratch w[kHuffWarps];
   int maxlen[kHuffWarps];
-  uint64_t cost[kMaxGroups];
-  uint32_t elig[kMaxGroups];
+  uint64_t cost[2 * kMaxGroups];  // plain group codes, then packed ones
+  uint32_t elig[2 * kMaxGroups];
   uint64_t red[kHuffWarps];
   uint32_t red32[kHuffWarps];
   int pick;
@@ -252,23 +252,31 @@ __device__ inline void warp_canonical(const uint8_t* lens, uint32_t* enc) {
 // which has at least one non-zero symbol; all threads of the block (kHuffWarps warps).
 // With a plan ("NeuralZip: Reusable Setup for Fast Lossless Compression", abstract): a
 // group is eligible when its code has a length for every symbol the chunk uses; the
-// eligible group with the fewest coded bits wins (ties to the smaller group). Without
-// an eligible group, or without a plan, the chunk gets its own limited Huffman code.
-// The payload is HUFF when strictly smaller than RAW. Thread 0 writes *mode, *code and
-// *size; enc_out receives len << 16 | code for every symbol when the result is HUFF.
+// eligible group with the fewest coded bits wins (ties to the smaller group). With the
+// plan's packed exponents (pack_hist: the chunk's 256 pair-symbol counts, pack_esc its
+// escaped exponents; NULL when the chunk cannot take them) each group's packed code is a
+// candidate too, at the pairs' code bits plus 8 a escape, and wins only with strictly
+// fewer bits. Without an eligible candidate, or without a plan, the chunk gets its own
+// limited Huffman code. The payload is HUFF (PACK) when strictly smaller than RAW. Thread
+// 0 writes *mode, *code and *size; enc_out receives len << 16 | code for every symbol of
+// the chosen code when the result is HUFF or PACK.
 __device__ inline void decide_code(HuffBlockSmem& sm, int A, int w, uint32_t rec, uint64_t m, uint32_t S,
                                    const PlanDev& plan, uint32_t e, uint32_t* enc_out, uint32_t* mode,
-                                   uint32_t* code, uint64_t* size) {
+                                   uint32_t* code, uint64_t* size, const uint32_t* pack_hist = nullptr,
+                                   uint32_t pack_esc = 0) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  int group = -1;
+  int group = -1;  // 0..G-1 plain group codes, G..2G-1 packed ones
   uint64_t bits = 0;
-  if (plan.groups) {
-    for (uint32_t gi = warp; gi < plan.groups; gi += kHuffWarps) {
-      const uint8_t* lg = plan.lens + ((uint64_t)e * plan.groups + gi) * 256;
+  const uint32_t G = plan.groups, cand = pack_hist ? 2 * G : G;
+  if (G) {
+    for (uint32_t gi = warp; gi < cand; gi += kHuffWarps) {
+      const bool packed = gi >= G;
+      const uint8_t* lg = packed ? plan.pack_lens + (uint64_t)(gi - G) * 256
+                                 : plan.lens + ((uint64_t)e * G + gi) * 256;
       uint64_t cost = 0;
       bool ok = true;
-      for (int s = lane; s < A; s += 32) {
-        const uint64_t f = sm.f[s];
+      for (int s = lane; s < (packed ? 256 : A); s += 32) {
+        const uint64_t f = packed ? (uint64_t)__ldcg(pack_hist + s) : sm.f[s];
         if (f) {
           ok = ok && lg[s] != 0;
           cost += f * lg[s];
@@ -277,14 +285,14 @@ __device__ inline void decide_code(HuffBlockSmem& sm, int A, int w, uint32_t rec
       for (int o = 16; o; o >>= 1) cost += __shfl_xor_sync(0xFFFFFFFFu, cost, o);
       const bool all = __all_sync(0xFFFFFFFFu, ok);
       if (lane == 0) {
-        sm.cost[gi] = cost;
+        sm.cost[gi] = cost + (packed ? 8ull * pack_esc : 0ull);
         sm.elig[gi] = all;
       }
     }
     __syncthreads();
     if (tid == 0) {
       int best = -1;
-      for (uint32_t gi = 0; gi < plan.groups; gi++)
+      for (uint32_t gi = 0; gi < cand; gi++)
         if (sm.elig[gi] && (best < 0 || sm.cost[gi] < sm.cost[best])) best = (int)gi;
       sm.pick = best;
     }
@@ -303,18 +311,23 @@ __device__ inline void decide_code(HuffBlockSmem& sm, int A, int w, uint32_t rec
     bits = 0;
     for (int i = 0; i < kHuffWarps; i++) bits += sm.red[i];
   }
+  const bool packed = group >= (int)G;
   const uint64_t nsub = ceil_div(m, S);
   const uint64_t p_huff = (group < 0 ? rec : 0) + round16(4 * nsub) + round16(ceil_div(bits, 8));
   const uint64_t p_raw = raw_payload(m, w);
   if (p_huff < p_raw) {
-    if (group >= 0) {
-      enc_out[tid] = plan.enc[((uint64_t)e * plan.groups + group) * 256 + tid];
+    if (packed) {
+      enc_out[tid] = plan.pack_enc[(uint64_t)(group - (int)G) * 256 + tid];
+    } else if (group >= 0) {
+      enc_out[tid] = plan.enc[((uint64_t)e * G + group) * 256 + tid];
     } else if (warp == 0) {
       warp_canonical(lens, enc_out);
     }
     if (tid == 0) {
-      *mode = kModeHuff;
-      *code = group >= 0 ? e * plan.groups + (uint32_t)group : kNoCode;
+      *mode = packed ? kModePack : kModeHuff;
+      // packed codes exist for BF16 only (one entropy stream): group g's packed record
+      // follows the G plain ones, record G + g, which is the candidate index
+      *code = packed ? (uint32_t)group : group >= 0 ? e * G + (uint32_t)group : kNoCode;
       *size = p_huff;
     }
   } else if (tid == 0) {

@@ -10,7 +10,7 @@ namespace zipnn {
 bool device_ok();
 
 // Kernel ids of the optional event timing (timing.cu).
-enum KernelId { kIdHist = 0, kIdBuild, kIdLayout, kIdEncode, kIdDecode, kIdCodeLengths, kIdPlan, kIdShard, kNumKernelIds };
+enum KernelId { kIdHist = 0, kIdBuild, kIdLayout, kIdEncode, kIdDecode, kIdCodeLengths, kIdPlan, kIdShard, kIdPackHist, kIdPackEncode, kNumKernelIds };
 
 // Brackets one launch with CUDA events on `st` while timing is enabled.
 class TimedLaunch {
@@ -42,6 +42,15 @@ cudaError_t launch_encode_bf16(const void* src, const Geo& g, const Ws& ws, uint
 cudaError_t launch_encode_fp32(const void* src, const Geo& g, const Ws& ws, uint8_t* out, cudaStream_t st);
 // FP8 and FP4 encode: the same scheme, with grouped code tables and bit-parallel packing.
 cudaError_t launch_encode_sub(const void* src, const Geo& g, const Ws& ws, uint8_t* out, cudaStream_t st);
+// Packed exponents (pack.cu): the plan's list, the chunks' pair counts, the groups' sums,
+// and the PACK payloads.
+cudaError_t launch_pack_select(const uint32_t* hist, uint32_t C, uint32_t NE, uint32_t max_pack, uint8_t* exps,
+                               uint32_t* k_out, cudaStream_t st);
+cudaError_t launch_pack_hist(const void* src, const Geo& g, const Ws& ws, const PlanDev& plan, cudaStream_t st);
+cudaError_t launch_pack_group_sums(const uint32_t* pack_hist, const uint32_t* assign, uint32_t C, uint64_t* gsum,
+                                   cudaStream_t st);
+cudaError_t launch_encode_pack(const void* src, const Geo& g, const Ws& ws, const PlanDev& plan, uint8_t* out,
+                               cudaStream_t st);
 cudaError_t launch_decode(const uint8_t* in, uint64_t in_bytes, const Geo& g, uint8_t* out, uint32_t* status,
                           cudaStream_t st);
 // One tensor of a batched decode (device table); chunk0 = its first chunk in the batch.

@@ -107,7 +107,10 @@ __device__ void build_chunk_table(const Geo& g, const Ws& ws, const PlanDev& pla
   sm.f[tid] = tid < A ? __ldcg(h + tid) : 0;
   __syncthreads();
   uint32_t* enc = ws.enc + ((uint64_t)c * NE + e) * 256;
-  decide_code(sm, A, w, record_bytes(DT, e), m, g.S, plan, e, enc, ws.emode + k, ws.ecode + k, ws.esize + k);
+  // packed exponents: BF16 exponent stream of a chunk of whole pairs
+  const bool pack = DT == kBF16 && e == 0 && plan.pack_k && ws.pack_hist && m % 2 == 0;
+  decide_code(sm, A, w, record_bytes(DT, e), m, g.S, plan, e, enc, ws.emode + k, ws.ecode + k, ws.esize + k,
+              pack ? ws.pack_hist + (uint64_t)c * 256 : nullptr, pack ? __ldcg(ws.pack_esc + c) : 0u);
   if constexpr (DT == kBF16 || DT == kFP32) {
     if (ws.tile_off) {
       __syncthreads();
@@ -628,7 +631,7 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout(Geo g, Ws ws, PlanDev
     hdr[4] = g.chunk_bytes;
     hdr[5] = g.S;
     hdr[6] = g.n_chunks;
-    hdr[7] = g.n_groups * NE;
+    hdr[7] = g.n_groups * NE + (g.n_packed ? g.n_groups : 0u);
     hdr[8] = (uint32_t)g.off_codes;
     hdr[9] = (uint32_t)(g.off_codes >> 32);
     hdr[10] = (uint32_t)g.off_payload;
@@ -636,7 +639,7 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout(Geo g, Ws ws, PlanDev
     const uint64_t tb = g.off_payload + s_prefix + total;
     hdr[12] = (uint32_t)tb;
     hdr[13] = (uint32_t)(tb >> 32);
-    hdr[14] = (uint32_t)kLmax | (g.n_groups << 8);
+    hdr[14] = (uint32_t)kLmax | (g.n_groups << 8) | (g.n_packed << 16);
     hdr[15] = 0;
     for (int i = 0; i < 4; i++)
       reinterpret_cast<uint4*>(out)[i] = make_uint4(hdr[4 * i], hdr[4 * i + 1], hdr[4 * i + 2], hdr[4 * i + 3]);
@@ -652,6 +655,15 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout(Geo g, Ws ws, PlanDev
         for (uint32_t b = tid; b < rb; b += kLayoutThreads)
           rp[b] = (int)(2 * b) < A ? (uint8_t)(lg[2 * b] | (lg[2 * b + 1] << 4)) : 0;
       }
+    }
+    // packed records and the list of packed exponents
+    if (g.n_packed) {
+      for (uint32_t gi = 0; gi < plan.groups; gi++) {
+        const uint8_t* lp = plan.pack_lens + (uint64_t)gi * 256;
+        uint8_t* rp = out + g.off_codes + packed_record_pos(DT, plan.groups, gi);
+        for (uint32_t b = tid; b < 128; b += kLayoutThreads) rp[b] = (uint8_t)(lp[2 * b] | (lp[2 * b + 1] << 4));
+      }
+      if (tid < (int)kPackListBytes) out[g.off_payload - kPackListBytes + tid] = plan.pack_exps[tid];
     }
   }
 }

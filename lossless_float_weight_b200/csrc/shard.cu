@@ -71,14 +71,15 @@ __global__ void __launch_bounds__(kShardThreads) k_shard_tables(const ShardItem*
     const uint32_t* hv = reinterpret_cast<const uint32_t*>(it.shard);
     const uint64_t n = ld_u64(it.shard + 8), off_codes = ld_u64(it.shard + 32);
     const uint64_t off_payload = ld_u64(it.shard + 40), total = ld_u64(it.shard + 48);
-    const uint32_t n_chunks = hv[6], G = (hv[14] >> 8) & 0xFF;
+    const uint32_t n_chunks = hv[6], G = (hv[14] >> 8) & 0xFF, K = (hv[14] >> 16) & 0xFF;
     const uint64_t C = ceil_div(it.n_total, m0);
     const uint64_t v_lo = it.chunk_lo * (uint64_t)m0;
     if (hv[0] != 0x314E4E5Au || hv[1] != (1u | ((uint32_t)DT << 16) | ((uint32_t)NS << 24))) bad = 1;
     if (hv[4] != chunk_bytes || v_lo >= it.n_total) bad = 1;
     if (!bad && (n != min64(it.n_total - v_lo, (uint64_t)n_chunks * m0) || n_chunks != ceil_div(n, m0))) bad = 1;
-    if (G > kMaxGroups || off_codes != kHeaderBytes + (uint64_t)kEntryBytes * n_chunks * NS) bad = 1;
-    if (off_payload != off_codes + shared_bytes(DT, G) || total < off_payload || total > it.shard_bytes) bad = 1;
+    if (G > kMaxGroups || K > kPackMax || off_codes != kHeaderBytes + (uint64_t)kEntryBytes * n_chunks * NS) bad = 1;
+    if (off_payload != off_codes + code_section_bytes(DT, G, K) || total < off_payload || total > it.shard_bytes)
+      bad = 1;
     // this shard's place among the shards of the item, and the whole payload size
     uint64_t base = 0, sum = 0;
     for (uint32_t r = 0; r < world; r++) {
@@ -88,7 +89,7 @@ __global__ void __launch_bounds__(kShardThreads) k_shard_tables(const ShardItem*
     }
     if (all_sizes[(uint64_t)rank * count + blockIdx.x] != total - off_payload) bad = 1;
     const uint64_t off_codes_g = kHeaderBytes + (uint64_t)kEntryBytes * C * NS;
-    const uint64_t off_payload_g = off_codes_g + shared_bytes(DT, G);
+    const uint64_t off_payload_g = off_codes_g + code_section_bytes(DT, G, K);
     s_delta = off_payload_g + base - off_payload;
     s_entries = n_chunks * NS;
     s_bad = bad;

@@ -11,7 +11,8 @@ namespace zipnn {
 namespace {
 
 const char* const kNames[kNumKernelIds] = {"split_hist", "code_build", "layout_scan", "encode",
-                                           "decode_merge", "code_lengths", "plan", "shard_tables"};
+                                           "decode_merge", "code_lengths", "plan", "shard_tables",
+                                           "pack_hist", "pack_encode"};
 
 struct Pending {
   int id;

@@ -46,6 +46,8 @@ zipnn_histogram = _sig("zipnn_histogram", _i, _i, _vp, _u64, _u32, _vp, _vp)
 zipnn_code_lengths = _sig("zipnn_code_lengths", _i, _vp, _u32, _u32, _vp, _vp)
 zipnn_plan_create = _sig("zipnn_plan_create", _i, _i, _vp, _u64, _u32, _u32, _u64, _vp, _sz, _vp,
                          ctypes.POINTER(_vp))
+zipnn_plan_create_packed = _sig("zipnn_plan_create_packed", _i, _i, _vp, _u64, _u32, _u32, _u64, _u32, _vp, _sz,
+                                _vp, ctypes.POINTER(_vp))
 zipnn_plan_export = _sig("zipnn_plan_export", _i, _vp, _vp, _sz, ctypes.POINTER(_sz))
 zipnn_plan_import = _sig("zipnn_plan_import", _i, _vp, _sz, ctypes.POINTER(_vp))
 zipnn_plan_assignment = _sig("zipnn_plan_assignment", _i, _vp, _vp, _sz, ctypes.POINTER(_sz))
@@ -83,7 +85,7 @@ zipnn_shard_tables = _sig("zipnn_shard_tables", _i, _i, _u32, _u32, ctypes.POINT
 C_ABI_NAMES = [
     "zipnn_max_compressed_bytes", "zipnn_workspace_bytes", "zipnn_compress", "zipnn_compress_ex",
     "zipnn_decompress", "zipnn_compressed_size", "zipnn_get_status", "zipnn_histogram", "zipnn_code_lengths",
-    "zipnn_plan_create", "zipnn_plan_export", "zipnn_plan_import", "zipnn_plan_assignment", "zipnn_plan_destroy",
+    "zipnn_plan_create", "zipnn_plan_create_packed", "zipnn_plan_export", "zipnn_plan_import", "zipnn_plan_assignment", "zipnn_plan_destroy",
     "zipnn_status_string", "zipnn_timing_enable", "zipnn_timing_collect", "zipnn_kernel_count",
     "zipnn_kernel_name", "zipnn_compress_noalloc", "zipnn_decompress_batch_workspace_bytes",
     "zipnn_decompress_batch", "zipnn_test_lookback_limit", "zipnn_shard_workspace_bytes", "zipnn_shard_sizes",
@@ -147,14 +149,17 @@ class Plan:
         self.dtype = dtype
 
     @classmethod
-    def create(cls, x, groups=8, seed=0, chunk_bytes=DEFAULT_CHUNK_BYTES, ws=None, stream=None):
+    def create(cls, x, groups=8, seed=0, chunk_bytes=DEFAULT_CHUNK_BYTES, ws=None, stream=None, max_pack=0):
+        """max_pack > 0 (BF16, at most 15): the plan also lists up to that many packed
+        exponents and gives every group a packed code over exponent pairs."""
         dt = dtype_code(x.dtype)
         xf = x.reshape(-1)
         if ws is None:
             ws = workspace(dt, nvalues(xf), chunk_bytes, xf.device)
         h = _vp()
-        check(zipnn_plan_create(dt, xf.data_ptr(), nvalues(xf), chunk_bytes, groups, seed, ws.data_ptr(),
-                                ws.numel(), _stream(stream), ctypes.byref(h)), "zipnn_plan_create")
+        check(zipnn_plan_create_packed(dt, xf.data_ptr(), nvalues(xf), chunk_bytes, groups, seed, max_pack,
+                                       ws.data_ptr(), ws.numel(), _stream(stream), ctypes.byref(h)),
+              "zipnn_plan_create_packed")
         return cls(h.value, dt)
 
     def export(self):
