@@ -262,10 +262,29 @@ __device__ __forceinline__ uint32_t bf16_merge_pair(uint32_t sf, int sf_hi, uint
 // BF16 with a HUFF exponent stream and a RAW (or ZERO) sign/fraction stream: the case
 // of every chunk of a trained or Gaussian checkpoint. 16 values per step; the
 // sign/fraction bytes of the next step are requested one step ahead.
-template <bool SM_ZERO>
+// A packed exponent pair (PACK streams) from either bit reader and either table: one code,
+// the pair symbol's two nibbles index the packed exponents (pexp, 16 entries); a nibble of
+// kPackEsc takes the next 8 bits as the exponent (first, then second). Returns the pair in
+// bits 16..31 (the first in 16..23), as huff_pair does. Needs 28 bits in the reader; an
+// index past the list (valid: bit i set for the K listed indices and for kPackEsc) marks
+// the stream corrupt.
+template <class Reader, class Lut>
+__device__ __forceinline__ uint32_t pack_pair(Reader& br, const Lut* lut, const uint8_t* pexp, uint32_t valid,
+                                              uint32_t& acc) {
+  const uint32_t p = br.huff(lut, acc);
+  const uint32_t hi = p >> 4, lo = p & 15u;
+  uint32_t a = pexp[hi], b = pexp[lo];
+  if (hi == kPackEsc) a = br.fixed(8);
+  if (lo == kPackEsc) b = br.fixed(8);
+  if (!((valid >> hi) & (valid >> lo) & 1u)) acc |= kLutInvalid;
+  return (a << 16) | (b << 24);
+}
+
+template <bool SM_ZERO, bool PACK = false>
 __device__ __forceinline__ int decode_bf16_fast(const uint32_t* lut, const uint8_t* smp, const uint32_t* bs,
                                                 uint32_t bs_words, uint64_t start, uint64_t expect, bool exact,
-                                                uint32_t count, uint8_t* __restrict__ dst) {
+                                                uint32_t count, uint8_t* __restrict__ dst,
+                                                const uint8_t* pexp = nullptr, uint32_t valid = 0) {
   BitReader br;
   br.init(bs, bs_words, start);
   uint32_t acc = 0;
@@ -280,11 +299,19 @@ __device__ __forceinline__ int decode_bf16_fast(const uint32_t* lut, const uint8
   }
   for (uint32_t gi = 0; gi < full; gi++) {
     uint32_t pr[8];  // exponent pairs in bits 16..31
+    if (PACK) {
 #pragma unroll
-    for (int i = 0; i < 8; i += 2) {
-      br.refill();
-      pr[i] = huff_pair(br, lut, acc);
-      pr[i + 1] = huff_pair(br, lut, acc);
+      for (int i = 0; i < 8; i++) {
+        br.refill();
+        pr[i] = pack_pair(br, lut, pexp, valid, acc);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; i += 2) {
+        br.refill();
+        pr[i] = huff_pair(br, lut, acc);
+        pr[i + 1] = huff_pair(br, lut, acc);
+      }
     }
     const uint32_t x[4] = {cur.x, cur.y, cur.z, cur.w};
     if (!SM_ZERO) {
@@ -300,11 +327,21 @@ __device__ __forceinline__ int decode_bf16_fast(const uint32_t* lut, const uint8
     d[0] = make_uint4(o[0], o[1], o[2], o[3]);
     d[1] = make_uint4(o[4], o[5], o[6], o[7]);
   }
-  for (uint32_t v = full * 16; v < count; v++) {
-    br.refill();
-    const uint32_t e = br.huff(lut, acc);
-    const uint32_t b = SM_ZERO ? 0u : smp[v];
-    reinterpret_cast<uint16_t*>(dst)[v] = (uint16_t)merge_value<kBF16>(e, b, 0, 0);
+  if (PACK) {  // count is even
+    for (uint32_t v = full * 16; v < count; v += 2) {
+      br.refill();
+      const uint32_t pr = pack_pair(br, lut, pexp, valid, acc);
+      const uint32_t b0 = SM_ZERO ? 0u : smp[v], b1 = SM_ZERO ? 0u : smp[v + 1];
+      reinterpret_cast<uint16_t*>(dst)[v] = (uint16_t)merge_value<kBF16>((pr >> 16) & 0xFFu, b0, 0, 0);
+      reinterpret_cast<uint16_t*>(dst)[v + 1] = (uint16_t)merge_value<kBF16>(pr >> 24, b1, 0, 0);
+    }
+  } else {
+    for (uint32_t v = full * 16; v < count; v++) {
+      br.refill();
+      const uint32_t e = br.huff(lut, acc);
+      const uint32_t b = SM_ZERO ? 0u : smp[v];
+      reinterpret_cast<uint16_t*>(dst)[v] = (uint16_t)merge_value<kBF16>(e, b, 0, 0);
+    }
   }
   const uint64_t pos = br.position();
   return (acc & kLutInvalid) || (exact ? pos != expect : pos > expect);
@@ -526,7 +563,7 @@ __device__ __forceinline__ int decode_fp32_fast(const uint32_t* lut, const uint3
 }
 
 // ---------------------------------------------------------------- staged BF16 path
-// For a BF16 chunk whose exponent stream is HUFF and whose bitstream fits a 48 KB
+// For a BF16 chunk whose exponent stream is HUFF (or PACK) and whose bitstream fits a 48 KB
 // window, the whole bitstream is brought into shared memory by one TMA bulk copy
 // (cp.async.bulk, completion on an mbarrier) while the block builds its lookup table.
 // Then, in rounds, every thread decodes the next 32 exponents of its sub-block into
@@ -591,6 +628,11 @@ struct SmemBitReader {
   }
   __device__ __forceinline__ uint32_t peek12() const { return (uint32_t)((c << bp) >> 52); }
   __device__ __forceinline__ void skip(uint32_t l) { bp += l; }
+  __device__ __forceinline__ uint32_t fixed(int width) {
+    const uint32_t v = (uint32_t)((c << bp) >> (64 - width));
+    bp += (uint32_t)width;
+    return v;
+  }
   __device__ __forceinline__ uint32_t huff(const uint32_t* lut, uint32_t& acc) {
     const uint32_t e = lut[peek12()];
     bp += e & 15u;
@@ -622,12 +664,15 @@ __device__ __forceinline__ uint32_t ex_word(uint32_t row, uint32_t k) {
 // ALLFULL: every sub-block of the chunk holds S values, S is a multiple of the round and
 // the sub-blocks fill whole batches, so every round decodes 32 exponents a thread and every
 // merge unit holds 8 values (the case of every chunk of a weight checkpoint).
-template <bool WIDE, bool ZRUN, bool ALLFULL, class Lut>
+// PACK: the exponent stream is packed pairs (pexp, valid as for pack_pair); S and every
+// count are even.
+template <bool WIDE, bool ZRUN, bool ALLFULL, bool PACK, class Lut>
 __device__ int decode_bf16_staged(StagedSmem& st, const Lut* lut, const uint32_t* tail,
                                   const uint32_t* __restrict__ idx, uint32_t bs_words,
                                   const uint8_t* __restrict__ smp, uint32_t m, uint32_t S, uint32_t nsub,
                                   uint8_t* __restrict__ outc, uint32_t pre_start, uint32_t pre_next,
-                                  const uint32_t* zmap, const uint32_t* zpre) {
+                                  const uint32_t* zmap, const uint32_t* zpre, const uint8_t* pexp,
+                                  uint32_t valid) {
   const int tid = threadIdx.x;
   int bad = 0;
   const uint64_t cap_bits = (uint64_t)bs_words * 32;
@@ -696,7 +741,13 @@ __device__ int decode_bf16_staged(StagedSmem& st, const Lut* lut, const uint32_t
         if (ALLFULL || base + kRound <= count) {
 #pragma unroll
           for (int k = 0; k < kRowWords; k++) {
-            if constexpr (WIDE) {
+            if constexpr (PACK) {
+              br.refill();
+              const uint32_t a = pack_pair(br, lut, pexp, valid, acc);
+              br.refill();
+              const uint32_t b = pack_pair(br, lut, pexp, valid, acc);
+              st.ex[ex_word(tid, k)] = __byte_perm(a, b, 0x7632);
+            } else if constexpr (WIDE) {
               br.refill();
               const uint32_t e0 = br.huff(lut, acc);
               const uint32_t e1 = br.huff(lut, acc);
@@ -713,9 +764,18 @@ __device__ int decode_bf16_staged(StagedSmem& st, const Lut* lut, const uint32_t
           }
         } else {
           const uint32_t n = count - base;
-          for (uint32_t k = 0; k < n; k++) {
-            br.refill();
-            exb[ex_word(tid, k >> 2) * 4 + (k & 3)] = (uint8_t)br.huff(lut, acc);
+          if constexpr (PACK) {
+            for (uint32_t k = 0; k < n; k += 2) {
+              br.refill();
+              const uint32_t pr = pack_pair(br, lut, pexp, valid, acc);
+              exb[ex_word(tid, k >> 2) * 4 + (k & 3)] = (uint8_t)(pr >> 16);
+              exb[ex_word(tid, k >> 2) * 4 + (k & 3) + 1] = (uint8_t)(pr >> 24);
+            }
+          } else {
+            for (uint32_t k = 0; k < n; k++) {
+              br.refill();
+              exb[ex_word(tid, k >> 2) * 4 + (k & 3)] = (uint8_t)br.huff(lut, acc);
+            }
           }
         }
       }
@@ -901,9 +961,11 @@ __device__ __forceinline__ void decode_fp32_chunk(const uint8_t* __restrict__ in
   }
 }
 
-// Every chunk the staged BF16 path does not take (FP32, FP8, FP4; BF16 with a RAW
+// Every chunk the staged BF16 path does not take (FP32, FP8, FP4; BF16 with a RAW or PACK
 // exponent stream, a bitstream over 56 KB, or a ZRUN plane of more than 4096 blocks): one
-// sub-block per thread per pass, every stream read through its own reader. All threads.
+// sub-block per thread per pass, every stream read through its own reader (BF16 with a
+// coded exponent stream and a RAW or ZERO sign/fraction plane: the register decoder,
+// which takes PACK pairs too). All threads.
 template <int DT>
 __device__ __forceinline__ void decode_generic(const uint8_t* __restrict__ in, const DecodeSmem<DT>& sm, uint32_t m,
                                                uint32_t S, uint64_t nsub, uint64_t clo, uint8_t* __restrict__ out,
@@ -915,7 +977,7 @@ __device__ __forceinline__ void decode_generic(const uint8_t* __restrict__ in, c
     const uint32_t sb_lo = (uint32_t)(j * S);
     const uint32_t count = min32(S, m - sb_lo);
     if constexpr (DT == kBF16) {
-      if (sm.mode[0] == kModeHuff && (sm.mode[1] == kModeRaw || sm.mode[1] == kModeZero)) {
+      if (coded(sm.mode[0]) && (sm.mode[1] == kModeRaw || sm.mode[1] == kModeZero)) {
         const uint32_t rec = sm.code[0] == kNoCode ? record_bytes(DT, 0) : 0;
         const uint32_t* idx = reinterpret_cast<const uint32_t*>(in + sm.off[0] + rec);
         const uint64_t bs_off = sm.off[0] + rec + round16(4 * nsub);
@@ -926,12 +988,20 @@ __device__ __forceinline__ void decode_generic(const uint8_t* __restrict__ in, c
         int bad = (j == 0 && start != 0) || start > cap_bits || expect < start || expect > cap_bits;
         const uint32_t* bs = reinterpret_cast<const uint32_t*>(in + bs_off);
         uint8_t* dst = out + (clo + sb_lo) * VB;
-        if (sm.mode[1] == kModeZero)
-          bad |= decode_bf16_fast<true>(sm.lut[0], nullptr, bs, (uint32_t)(cap_bits / 32), bad ? 0 : start,
-                                                   expect, exact, count, dst);
-        else
-          bad |= decode_bf16_fast<false>(sm.lut[0], in + sm.off[1] + sb_lo, bs, (uint32_t)(cap_bits / 32),
-                                                    bad ? 0 : start, expect, exact, count, dst);
+        const uint8_t* smp = sm.mode[1] == kModeZero ? nullptr : in + sm.off[1] + sb_lo;
+        const uint32_t bw = (uint32_t)(cap_bits / 32);
+        const uint64_t from = bad ? 0 : start;
+        if (sm.mode[0] == kModePack) {
+          const uint32_t valid = ((1u << sm.K) - 1u) | (1u << kPackEsc);
+          if (!smp) bad |= decode_bf16_fast<true, true>(sm.lut[0], smp, bs, bw, from, expect, exact, count, dst,
+                                                        sm.pack_exps, valid);
+          else bad |= decode_bf16_fast<false, true>(sm.lut[0], smp, bs, bw, from, expect, exact, count, dst,
+                                                    sm.pack_exps, valid);
+        } else if (!smp) {
+          bad |= decode_bf16_fast<true>(sm.lut[0], smp, bs, bw, from, expect, exact, count, dst);
+        } else {
+          bad |= decode_bf16_fast<false>(sm.lut[0], smp, bs, bw, from, expect, exact, count, dst);
+        }
         if (bad) set_status(status, kStCorrupt);
         continue;
       }
@@ -1194,7 +1264,7 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
     if constexpr (DT == kBF16) {
       // staged path: HUFF exponents, RAW or ZERO sign/fraction bytes, bitstream in the
       // window (1), or in the window and the table's first half (2, the wide window)
-      if (!bad && sm.mode[0] == kModeHuff && sm.mode[1] != kModeHuff &&
+      if (!bad && coded(sm.mode[0]) && sm.mode[1] != kModeHuff &&
           (sm.mode[1] != kModeZrun || ceil_div(ceil_div(m, kZBlock), 32) <= kZStagedWords)) {
         const uint64_t nsub = ceil_div(m, S);
         const uint32_t rec = sm.code[0] == kNoCode ? record_bytes(DT, 0) : 0;
@@ -1455,19 +1525,32 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
                                                      : nullptr;
       const bool allfull = (uint64_t)m == nsub * S && S % kRound == 0 && nsub % kDecodeThreads == 0;
       int bad;
-#define ZIPNN_STAGED(W, Z, F, L, T, ZM, ZP) \
-  decode_bf16_staged<W, Z, F>(stg, L, T, idx, bs_words, smp, m, S, (uint32_t)nsub, out + clo * VB, idx_start, \
-                              idx_next, ZM, ZP)
-      if (sm.mode[1] == kModeZrun) {
-        if (wide) bad = allfull ? ZIPNN_STAGED(true, true, true, lut16, sm.lut[0], sm.zmap, sm.zpre)
-                                : ZIPNN_STAGED(true, true, false, lut16, sm.lut[0], sm.zmap, sm.zpre);
-        else bad = allfull ? ZIPNN_STAGED(false, true, true, sm.lut[0], nullptr, sm.zmap, sm.zpre)
-                           : ZIPNN_STAGED(false, true, false, sm.lut[0], nullptr, sm.zmap, sm.zpre);
+#define ZIPNN_STAGED(W, Z, F, P, L, T, ZM, ZP)                                                                \
+  decode_bf16_staged<W, Z, F, P>(stg, L, T, idx, bs_words, smp, m, S, (uint32_t)nsub, out + clo * VB, idx_start, \
+                                 idx_next, ZM, ZP, sm.pack_exps, valid)
+      const uint32_t valid = ((1u << sm.K) - 1u) | (1u << kPackEsc);
+      if (sm.mode[0] == kModePack) {
+        if (sm.mode[1] == kModeZrun) {
+          if (wide) bad = allfull ? ZIPNN_STAGED(true, true, true, true, lut16, sm.lut[0], sm.zmap, sm.zpre)
+                                  : ZIPNN_STAGED(true, true, false, true, lut16, sm.lut[0], sm.zmap, sm.zpre);
+          else bad = allfull ? ZIPNN_STAGED(false, true, true, true, sm.lut[0], nullptr, sm.zmap, sm.zpre)
+                             : ZIPNN_STAGED(false, true, false, true, sm.lut[0], nullptr, sm.zmap, sm.zpre);
+        } else {
+          if (wide) bad = allfull ? ZIPNN_STAGED(true, false, true, true, lut16, sm.lut[0], nullptr, nullptr)
+                                  : ZIPNN_STAGED(true, false, false, true, lut16, sm.lut[0], nullptr, nullptr);
+          else bad = allfull ? ZIPNN_STAGED(false, false, true, true, sm.lut[0], nullptr, nullptr, nullptr)
+                             : ZIPNN_STAGED(false, false, false, true, sm.lut[0], nullptr, nullptr, nullptr);
+        }
+      } else if (sm.mode[1] == kModeZrun) {
+        if (wide) bad = allfull ? ZIPNN_STAGED(true, true, true, false, lut16, sm.lut[0], sm.zmap, sm.zpre)
+                                : ZIPNN_STAGED(true, true, false, false, lut16, sm.lut[0], sm.zmap, sm.zpre);
+        else bad = allfull ? ZIPNN_STAGED(false, true, true, false, sm.lut[0], nullptr, sm.zmap, sm.zpre)
+                           : ZIPNN_STAGED(false, true, false, false, sm.lut[0], nullptr, sm.zmap, sm.zpre);
       } else {
-        if (wide) bad = allfull ? ZIPNN_STAGED(true, false, true, lut16, sm.lut[0], nullptr, nullptr)
-                                : ZIPNN_STAGED(true, false, false, lut16, sm.lut[0], nullptr, nullptr);
-        else bad = allfull ? ZIPNN_STAGED(false, false, true, sm.lut[0], nullptr, nullptr, nullptr)
-                           : ZIPNN_STAGED(false, false, false, sm.lut[0], nullptr, nullptr, nullptr);
+        if (wide) bad = allfull ? ZIPNN_STAGED(true, false, true, false, lut16, sm.lut[0], nullptr, nullptr)
+                                : ZIPNN_STAGED(true, false, false, false, lut16, sm.lut[0], nullptr, nullptr);
+        else bad = allfull ? ZIPNN_STAGED(false, false, true, false, sm.lut[0], nullptr, nullptr, nullptr)
+                           : ZIPNN_STAGED(false, false, false, false, sm.lut[0], nullptr, nullptr, nullptr);
       }
 #undef ZIPNN_STAGED
       if (bad) set_status(status, kStCorrupt);

@@ -160,16 +160,21 @@ struct PackWriter {
 };
 
 // One block per chunk whose exponent stream is PACK (others return at once). The payload
-// [index of ceil(m / S) u32, padded][bitstream, padded] is zeroed; then, a round of
-// kPackThreads sub-blocks at a time, each thread sizes its sub-block (the pairs' code
-// lengths plus 8 bits an escape), a block scan gives the sub-blocks' bit offsets (the
-// index), and each thread writes its sub-block's codes at its offset.
+// [index of ceil(m / S) u32, padded][bitstream, padded] is zeroed first. Then, a round at
+// a time, each warp takes one sub-block, lane l the pairs [p0 + l q, p0 + (l + 1) q) (q =
+// ceil(pairs / 32); at most 8 are held in registers): the lanes size their runs (code
+// lengths plus 8 bits an escape), a warp scan places the runs, the warps' totals (one
+// barrier a round, double-buffered) place the sub-blocks after the rounds before, and each
+// lane writes its codes. The input is read once when S <= 512.
+constexpr int kPackRegPairs = 8;
+
 __global__ void __launch_bounds__(kPackThreads) k_encode_pack(const uint8_t* __restrict__ src, Geo g, Ws ws,
                                                               PlanDev plan, uint8_t* __restrict__ out) {
+  constexpr int NW = kPackThreads / 32;
   __shared__ uint32_t enc[256];
   __shared__ uint8_t nib[256];
-  __shared__ uint32_t s_warp[kPackThreads / 32];
-  const int tid = threadIdx.x;
+  __shared__ uint32_t s_tot[2][NW];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t c = blockIdx.x;
   if (ws.emode[2ull * c] != kModePack) return;  // uniform
   const uint64_t clo = (uint64_t)c * g.m0;
@@ -178,41 +183,79 @@ __global__ void __launch_bounds__(kPackThreads) k_encode_pack(const uint8_t* __r
   const uint64_t nsub = ceil_div(m, S);
   uint8_t* payload = out + ws.eoff[2ull * c];
   const uint64_t size = ws.esize[2ull * c];
-  uint32_t* pw = reinterpret_cast<uint32_t*>(payload);
-  for (uint64_t i = tid; i < size / 4; i += kPackThreads) pw[i] = 0;
+  uint4* pz = reinterpret_cast<uint4*>(payload);
+  for (uint64_t i = tid; i < size / 16; i += kPackThreads) pz[i] = make_uint4(0, 0, 0, 0);
   enc[tid] = ws.enc[(uint64_t)c * 256 + tid];
   fill_nibbles(nib, plan.pack_exps, plan.pack_k);
   __syncthreads();
-  uint32_t* idx = pw;
+  uint32_t* idx = reinterpret_cast<uint32_t*>(payload);
   uint32_t* bs = reinterpret_cast<uint32_t*>(payload + round16(4 * nsub));
   const uint32_t* wp = reinterpret_cast<const uint32_t*>(src + clo * 2);
+  auto pair_bits = [&](uint32_t w) {
+    const uint32_t s = pair_symbol(w, nib);
+    return (enc[s] >> 16) + 8u * (((s >> 4) == kPackEsc) + ((s & 15u) == kPackEsc));
+  };
   uint32_t carry = 0;
-  for (uint64_t base = 0; base < nsub; base += kPackThreads) {
-    const uint64_t j = base + tid;
-    const uint32_t lo = (uint32_t)min64(j * S, m), hi = (uint32_t)min64(j * S + S, m);
-    uint32_t bits = 0;
-    for (uint32_t p = lo / 2; p < hi / 2; p++) {
-      const uint32_t s = pair_symbol(__ldg(wp + p), nib);
-      bits += (enc[s] >> 16) + 8u * (((s >> 4) == kPackEsc) + ((s & 15u) == kPackEsc));
-    }
-    uint32_t total;
-    const uint32_t before = block_exclusive_scan<kPackThreads>(bits, s_warp, total);
-    const uint32_t start = carry + before;
+  int buf = 0;
+  for (uint64_t base = 0; base < nsub; base += NW, buf ^= 1) {
+    const uint64_t j = base + warp;
+    uint32_t a = 0, b = 0, q = 0;
     if (j < nsub) {
-      idx[j] = start;
+      const uint32_t p0 = (uint32_t)(j * S / 2), p1 = (uint32_t)min64(j * S + S, m) / 2;
+      q = (p1 - p0 + 31) / 32;
+      a = min32(p0 + lane * q, p1);
+      b = min32(a + q, p1);
+    }
+    // a full run of 8: p0 (S / 2 j, S a multiple of 16) and 8 lane are multiples of 8 pairs,
+    // so the run starts 32 bytes into the chunk's 16-byte aligned values
+    const bool in_regs = q == (uint32_t)kPackRegPairs && b - a == (uint32_t)kPackRegPairs;
+    uint32_t w[kPackRegPairs];
+    uint32_t bits = 0;
+    if (in_regs) {
+      const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(wp + a));
+      const uint4 v1 = __ldg(reinterpret_cast<const uint4*>(wp + a) + 1);
+      w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+      w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+#pragma unroll
+      for (int i = 0; i < kPackRegPairs; i++) bits += pair_bits(w[i]);
+    } else {
+      for (uint32_t p = a; p < b; p++) bits += pair_bits(__ldg(wp + p));
+    }
+    uint32_t incl = bits;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_tot[buf][warp] = incl;
+    __syncthreads();
+    uint32_t before = 0, round_total = 0;
+#pragma unroll
+    for (int k = 0; k < NW; k++) {
+      const uint32_t t = s_tot[buf][k];
+      if (k < warp) before += t;
+      round_total += t;
+    }
+    const uint32_t sub_start = carry + before;
+    if (j < nsub && lane == 0) idx[j] = sub_start;
+    if (a < b) {
       PackWriter wr;
-      wr.init(bs, start);
-      for (uint32_t p = lo / 2; p < hi / 2; p++) {
-        const uint32_t w = __ldg(wp + p);
-        const uint32_t s = pair_symbol(w, nib);
+      wr.init(bs, (uint64_t)sub_start + incl - bits);
+      auto put_pair = [&](uint32_t x) {
+        const uint32_t s = pair_symbol(x, nib);
         wr.put(enc[s] & 0xFFFFu, (int)(enc[s] >> 16));
-        if ((s >> 4) == kPackEsc) wr.put((w >> 7) & 0xFFu, 8);
-        if ((s & 15u) == kPackEsc) wr.put((w >> 23) & 0xFFu, 8);
+        if ((s >> 4) == kPackEsc) wr.put((x >> 7) & 0xFFu, 8);
+        if ((s & 15u) == kPackEsc) wr.put((x >> 23) & 0xFFu, 8);
+      };
+      if (in_regs) {
+#pragma unroll
+        for (int i = 0; i < kPackRegPairs; i++) put_pair(w[i]);
+      } else {
+        for (uint32_t p = a; p < b; p++) put_pair(__ldg(wp + p));
       }
       wr.finish();
     }
-    carry += total;
-    __syncthreads();  // s_warp is reused by the next round's scan
+    carry += round_total;
   }
 }
 
