@@ -743,8 +743,9 @@ def run_single(args):
         desc = (f"FP4 E2M1 {rows:,} x 4096 ({rows * 4096:,} values), N(0, 1) x per-row scale "
                 "log-uniform [0.25, 4]")
     else:
-        x = W.kv_cache(device=dev)
-        desc = "BF16 K/V cache [32, 2, 16, 8, 4096, 128], per-channel std log-normal, 8-group plan"
+        layers = args.rows or 32
+        x = W.kv_cache(shape=(layers, 2, 16, 8, 4096, 128), device=dev)
+        desc = f"BF16 K/V cache [{layers}, 2, 16, 8, 4096, 128], per-channel std log-normal, 8-group plan"
         if args.max_pack:
             desc += f", up to {args.max_pack} packed exponents"
     x = x.reshape(-1)
@@ -819,8 +820,8 @@ def main():
                     choices=["checkpoint_7b", "fp32", "fp32_clean", "fp8", "fp4", "kv_cache"],
                     help="another workload than the benchmark's: one tensor, compress and decompress timed apart")
     ap.add_argument("--rows", type=int, default=None,
-                    help="rows of 4096 values for --workload fp32/fp32_clean/fp8/fp4 (profiler cases; "
-                         "default 65536 FP32, 262144 FP8/FP4)")
+                    help="rows of 4096 values for --workload fp32/fp32_clean/fp8/fp4, layers for kv_cache "
+                         "(profiler cases; default 65536 FP32, 262144 FP8/FP4, 32 layers)")
     ap.add_argument("--max-pack", type=int, default=0,
                     help="--workload kv_cache: the plan also lists up to this many packed exponents (BF16, <= 15)")
     ap.add_argument("--plan-transfer", action="store_true",

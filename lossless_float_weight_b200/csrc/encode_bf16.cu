@@ -22,6 +22,8 @@
 //    (1 << 32 | its bits) and the side that arrives second stores the complete word.
 // The sub-block index idx[j] (bit offset of symbol j*S) is written by the thread that
 // owns symbol j*S; the first tile writes a local code record, the last the padding.
+// A PACK exponent stream (packed exponent pairs) is written by k_encode_pack, which also
+// writes a RAW sign/fraction plane: such chunks are skipped here unless the plane is ZRUN.
 #include <atomic>
 
 #include "common.cuh"
@@ -85,6 +87,7 @@ __global__ void __launch_bounds__(kBThreads, 8) k_encode_bf16(const uint8_t* __r
     if (tlo >= m) continue;  // past the end of a ragged last chunk (uniform)
     // the chunk's decisions and code
     const uint32_t mode0 = ws.emode[2ull * c], mode1 = ws.emode[2ull * c + 1];
+    if (mode0 == kModePack && mode1 != kModeZrun) continue;  // k_encode_pack writes both streams (uniform)
     const uint32_t code0 = ws.ecode[2ull * c];
     const uint64_t off0 = ws.eoff[2ull * c], off1 = ws.eoff[2ull * c + 1];
     uint64_t P = 0;  // the pass's bit offset in the chunk

@@ -10,7 +10,8 @@
 //   k_pack_select     : (setup) the list, from the exponent counts of every chunk;
 //   k_pack_hist       : per chunk, the pair-symbol counts and the escaped exponents;
 //   k_pack_group_sums : (setup) each group's summed pair counts (chunks of whole pairs);
-//   k_encode_pack     : per PACK chunk, the sub-block index and the bitstream.
+//   k_encode_pack     : per PACK chunk, the sub-block index and the bitstream (and a RAW
+//                       sign/fraction plane).
 #include "common.cuh"
 #include "launch.h"
 
@@ -57,6 +58,13 @@ __device__ __forceinline__ void fill_nibbles(uint8_t* nib, const uint8_t* exps, 
       if (exps[i] == x) v = (uint32_t)i;
     nib[x] = (uint8_t)v;
   }
+}
+
+// The sign/fraction bytes of the two BF16 values of a word (bit 15 over bits 6..0), in
+// bytes 0 and 1.
+__device__ __forceinline__ uint32_t sf_pair(uint32_t w) {
+  const uint32_t t = (w & 0x007F007Fu) | ((w >> 8) & 0x00800080u);
+  return (t & 0xFFu) | ((t >> 8) & 0xFF00u);
 }
 
 // The pair symbol of one 32-bit word of BF16 input (value 2j in the low half).
@@ -124,49 +132,19 @@ __global__ void k_pack_group_sums(const uint32_t* __restrict__ pack_hist, const 
                    (unsigned long long)v);
 }
 
-// Bit writer over 32-bit words of a bitstream that is stored most significant bit first
-// (byte 0 holds bits 0..7): bits before `start` in its first word, and after its end in
-// its last word, belong to the neighbouring sub-blocks, so those two words are merged
-// with atomicOr into the zeroed payload; every other word is this writer's alone.
-struct PackWriter {
-  uint32_t* words;
-  uint64_t buf;   // pending bits, left-aligned
-  int nb;         // pending bits in buf, counting the leading bits of a shared first word
-  uint32_t wi;    // index of the word buf's top bits go to
-  bool shared;    // the word at wi is shared with the previous sub-block
-  __device__ __forceinline__ void init(uint32_t* w, uint64_t start) {
-    words = w;
-    buf = 0;
-    nb = (int)(start & 31);
-    wi = (uint32_t)(start >> 5);
-    shared = nb != 0;
-  }
-  __device__ __forceinline__ void put(uint32_t v, int len) {
-    buf |= (uint64_t)v << (64 - nb - len);
-    nb += len;
-    if (nb >= 32) {
-      const uint32_t w = bswap32((uint32_t)(buf >> 32));
-      if (shared) atomicOr(words + wi, w);
-      else words[wi] = w;
-      shared = false;
-      buf <<= 32;
-      nb -= 32;
-      wi++;
-    }
-  }
-  __device__ __forceinline__ void finish() {
-    if (nb > 0) atomicOr(words + wi, bswap32((uint32_t)(buf >> 32)));
-  }
-};
-
-// One block per chunk whose exponent stream is PACK (others return at once). The payload
+// One block per chunk whose exponent stream is PACK (others return at once); it also
+// writes the chunk's sign/fraction plane when that is RAW. The payload
 // [index of ceil(m / S) u32, padded][bitstream, padded] is zeroed first. Then, a round at
 // a time, each warp takes one sub-block, lane l the pairs [p0 + l q, p0 + (l + 1) q) (q =
-// ceil(pairs / 32); at most 8 are held in registers): the lanes size their runs (code
-// lengths plus 8 bits an escape), a warp scan places the runs, the warps' totals (one
-// barrier a round, double-buffered) place the sub-blocks after the rounds before, and each
-// lane writes its codes. The input is read once when S <= 512.
+// ceil(pairs / 32); at most kPackRegPairs held in registers): each lane forms its pairs'
+// bits (the code, then each escaped exponent's 8 bits: at most 28 a pair) and their
+// total, a warp scan places the lanes' runs and the warps' totals (one barrier a round,
+// double-buffered) place the sub-blocks after the rounds before; each lane then appends
+// its bits to a 64-bit accumulator, flushing whole words into its own shared words, and
+// moves those words to its bit offset with funnel shifts: plain stores for the middle
+// words, atomicOr for the two it may share with its neighbours.
 constexpr int kPackRegPairs = 8;
+constexpr int kPackPrivWords = kPackRegPairs * 28 / 32 + 1;  // 8 pairs of at most 28 bits
 
 __global__ void __launch_bounds__(kPackThreads) k_encode_pack(const uint8_t* __restrict__ src, Geo g, Ws ws,
                                                               PlanDev plan, uint8_t* __restrict__ out) {
@@ -174,6 +152,7 @@ __global__ void __launch_bounds__(kPackThreads) k_encode_pack(const uint8_t* __r
   __shared__ uint32_t enc[256];
   __shared__ uint8_t nib[256];
   __shared__ uint32_t s_tot[2][NW];
+  __shared__ uint32_t priv[kPackPrivWords + 1][kPackThreads];  // lane-major: conflict-free
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t c = blockIdx.x;
   if (ws.emode[2ull * c] != kModePack) return;  // uniform
@@ -185,15 +164,31 @@ __global__ void __launch_bounds__(kPackThreads) k_encode_pack(const uint8_t* __r
   const uint64_t size = ws.esize[2ull * c];
   uint4* pz = reinterpret_cast<uint4*>(payload);
   for (uint64_t i = tid; i < size / 16; i += kPackThreads) pz[i] = make_uint4(0, 0, 0, 0);
+  // a RAW sign/fraction plane is written here too, from the same loads (k_encode_bf16
+  // skips these chunks); its padding to 16 bytes is zero
+  uint8_t* plane = ws.emode[2ull * c + 1] == kModeRaw ? out + ws.eoff[2ull * c + 1] : nullptr;
+  if (plane && tid < (int)(round16(m) - m)) plane[m + tid] = 0;
   enc[tid] = ws.enc[(uint64_t)c * 256 + tid];
   fill_nibbles(nib, plan.pack_exps, plan.pack_k);
   __syncthreads();
   uint32_t* idx = reinterpret_cast<uint32_t*>(payload);
   uint32_t* bs = reinterpret_cast<uint32_t*>(payload + round16(4 * nsub));
   const uint32_t* wp = reinterpret_cast<const uint32_t*>(src + clo * 2);
-  auto pair_bits = [&](uint32_t w) {
-    const uint32_t s = pair_symbol(w, nib);
-    return (enc[s] >> 16) + 8u * (((s >> 4) == kPackEsc) + ((s & 15u) == kPackEsc));
+  // a pair's bits: the code, then each escaped exponent (value << 8 | length)
+  auto pair_code = [&](uint32_t w, uint32_t& len) {
+    const uint32_t a = nib[(w >> 7) & 0xFFu], b = nib[(w >> 23) & 0xFFu];
+    const uint32_t e = enc[(a << 4) | b];
+    uint32_t v = e & 0xFFFFu, l = e >> 16;
+    if (a == kPackEsc) {
+      v = (v << 8) | ((w >> 7) & 0xFFu);
+      l += 8;
+    }
+    if (b == kPackEsc) {
+      v = (v << 8) | ((w >> 23) & 0xFFu);
+      l += 8;
+    }
+    len = l;
+    return v;
   };
   uint32_t carry = 0;
   int buf = 0;
@@ -209,17 +204,35 @@ __global__ void __launch_bounds__(kPackThreads) k_encode_pack(const uint8_t* __r
     // a full run of 8: p0 (S / 2 j, S a multiple of 16) and 8 lane are multiples of 8 pairs,
     // so the run starts 32 bytes into the chunk's 16-byte aligned values
     const bool in_regs = q == (uint32_t)kPackRegPairs && b - a == (uint32_t)kPackRegPairs;
-    uint32_t w[kPackRegPairs];
+    uint32_t v[kPackRegPairs], l[kPackRegPairs];
     uint32_t bits = 0;
     if (in_regs) {
       const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(wp + a));
       const uint4 v1 = __ldg(reinterpret_cast<const uint4*>(wp + a) + 1);
-      w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
-      w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+      const uint32_t w[kPackRegPairs] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
-      for (int i = 0; i < kPackRegPairs; i++) bits += pair_bits(w[i]);
+      for (int i = 0; i < kPackRegPairs; i++) {
+        v[i] = pair_code(w[i], l[i]);
+        bits += l[i];
+      }
+      if (plane) {  // 16 values: 16 bytes at value 2a (a multiple of 16)
+        uint32_t o[4];
+#pragma unroll
+        for (int k = 0; k < 4; k++) o[k] = sf_pair(w[2 * k]) | (sf_pair(w[2 * k + 1]) << 16);
+        *reinterpret_cast<uint4*>(plane + 2 * (uint64_t)a) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
     } else {
-      for (uint32_t p = a; p < b; p++) bits += pair_bits(__ldg(wp + p));
+      for (uint32_t p = a; p < b; p++) {
+        uint32_t len;
+        const uint32_t w = __ldg(wp + p);
+        pair_code(w, len);
+        bits += len;
+        if (plane) {
+          const uint32_t sf = sf_pair(w);
+          plane[2 * (uint64_t)p] = (uint8_t)sf;
+          plane[2 * (uint64_t)p + 1] = (uint8_t)(sf >> 8);
+        }
+      }
     }
     uint32_t incl = bits;
 #pragma unroll
@@ -238,22 +251,47 @@ __global__ void __launch_bounds__(kPackThreads) k_encode_pack(const uint8_t* __r
     }
     const uint32_t sub_start = carry + before;
     if (j < nsub && lane == 0) idx[j] = sub_start;
-    if (a < b) {
-      PackWriter wr;
-      wr.init(bs, (uint64_t)sub_start + incl - bits);
-      auto put_pair = [&](uint32_t x) {
-        const uint32_t s = pair_symbol(x, nib);
-        wr.put(enc[s] & 0xFFFFu, (int)(enc[s] >> 16));
-        if ((s >> 4) == kPackEsc) wr.put((x >> 7) & 0xFFu, 8);
-        if ((s & 15u) == kPackEsc) wr.put((x >> 23) & 0xFFu, 8);
-      };
+    if (bits) {
+      const uint32_t start = sub_start + incl - bits;
       if (in_regs) {
+        // append the codes, whole words into my shared words (pending bits < 32 + 28)
+        uint64_t acc = 0;
+        uint32_t nfill = 0, nw = 0;
 #pragma unroll
-        for (int i = 0; i < kPackRegPairs; i++) put_pair(w[i]);
+        for (int i = 0; i < kPackRegPairs; i++) {
+          acc = (acc << l[i]) | v[i];
+          nfill += l[i];
+          if (nfill >= 32) {
+            nfill -= 32;
+            priv[nw++][tid] = (uint32_t)(acc >> nfill);
+          }
+        }
+        if (nfill) priv[nw++][tid] = (uint32_t)(acc << (32 - nfill));
+        // word k of my run goes to bitstream word d0 + k, shifted right by sh
+        const uint32_t sh = start & 31u, d0 = start >> 5, nk = ((start + bits - 1) >> 5) - d0 + 1;
+        uint32_t cur = priv[0][tid];
+        atomicOr(bs + d0, bswap32(__funnelshift_r(cur, 0u, sh)));
+        for (uint32_t k = 1; k + 1 < nk; k++) {
+          const uint32_t prev = cur;
+          cur = priv[k][tid];
+          bs[d0 + k] = bswap32(__funnelshift_r(cur, prev, sh));
+        }
+        if (nk > 1) atomicOr(bs + d0 + nk - 1, bswap32(__funnelshift_r(nk - 1 < nw ? priv[nk - 1][tid] : 0u, cur, sh)));
       } else {
-        for (uint32_t p = a; p < b; p++) put_pair(__ldg(wp + p));
+        // a long or short run (S other than 512, a chunk's last sub-block): bit by bit
+        // merges of each pair's bits into the zeroed words
+        uint32_t t = start;
+        for (uint32_t p = a; p < b; p++) {
+          uint32_t len;
+          const uint32_t x = pair_code(__ldg(wp + p), len);
+          // at most 28 bits: they span at most two words
+          const uint32_t sh = t & 31u;
+          const uint64_t placed = ((uint64_t)x << (64 - len)) >> sh;
+          atomicOr(bs + (t >> 5), bswap32((uint32_t)(placed >> 32)));
+          if (sh + len > 32) atomicOr(bs + (t >> 5) + 1, bswap32((uint32_t)placed));
+          t += len;
+        }
       }
-      wr.finish();
     }
     carry += round_total;
   }
