@@ -110,3 +110,38 @@ def test_no_device_is_reported_as_unsupported(lib):
     fake = 1 << 20
     assert Z.zipnn_code_lengths(fake, 1, 256, fake, None) == Z.ERR_UNSUPPORTED
     assert Z.zipnn_compress_noalloc(Z.BF16, fake, 1000, 262144, fake, 1 << 20, None) == Z.ERR_UNSUPPORTED
+
+
+def test_packed_plan_arguments_without_a_device(lib):
+    """Packed exponents: a list longer than 15, or packing for a dtype other than BF16, is
+    refused before anything touches the device; an exported plan whose list is longer than
+    15, names packed exponents for FP8, or has a byte past its list, does not import."""
+    import ctypes
+    from lossless_float_weight_b200 import zipnn as Z
+    fake = 1 << 20
+    h = ctypes.c_void_p()
+    assert Z.zipnn_plan_create_packed(Z.BF16, fake, 4096, 262144, 2, 0, 16, fake, 1 << 20, None,
+                                      ctypes.byref(h)) == Z.ERR_INVALID_ARG
+    assert Z.zipnn_plan_create_packed(Z.FP8_E4M3, fake, 4096, 262144, 2, 0, 3, fake, 1 << 20, None,
+                                      ctypes.byref(h)) == Z.ERR_INVALID_ARG
+    G = 1
+
+    def plan_bytes(dt, K, pad_byte=0):
+        # "ZNP1", dtype, groups, K, 0; one plain record (a 2-symbol code); K > 0: a packed
+        # record and the list
+        rec = bytearray(128 if dt == Z.BF16 else 16 * 2)
+        rec[0] = 0x11
+        body = bytes(rec)
+        if K:
+            prec = bytearray(128)
+            prec[0] = 0x11
+            lst = bytearray(16)
+            lst[:min(K, 16)] = bytes(range(100, 100 + min(K, 16)))
+            if pad_byte:
+                lst[15] = pad_byte
+            body += bytes(prec) + bytes(lst)
+        return b"ZNP1" + bytes([dt, G, K, 0]) + body
+
+    for data in (plan_bytes(Z.BF16, 16), plan_bytes(Z.FP8_E4M3, 2), plan_bytes(Z.BF16, 3, pad_byte=7)):
+        buf = (ctypes.c_uint8 * len(data)).from_buffer_copy(data)
+        assert Z.zipnn_plan_import(buf, len(data), ctypes.byref(h)) == Z.ERR_CORRUPT
