@@ -114,6 +114,20 @@ def test_packed_plan_parity_shapes(z, orc, case):
         _check(z, orc, x, groups=2, cb=65536, max_pack=3, name=case)
 
 
+def test_packed_with_zero_runs(z, orc):
+    """Pruned weights (60% of the 32-value blocks all zero): PACK exponent streams next to
+    ZRUN sign/fraction planes, which the BF16 encode writes while the packed encode writes
+    the exponents."""
+    g = torch.Generator().manual_seed(11)
+    v = (torch.randn(262144 * 2 + 8192, generator=g) * 0.02)
+    blocks = v.view(-1, 32)
+    blocks[torch.rand(blocks.shape[0], generator=g) < 0.6] = 0
+    x = v.to(torch.bfloat16)
+    got, _ = _check(z, orc, x, groups=2, cb=262144, name="pruned")
+    modes = got[64: 64 + 16 * 2 * 5: 16]
+    assert 4 in modes[0::2].tolist() and 3 in modes[1::2].tolist()
+
+
 def test_packed_plan_reuse_and_batch(z, orc):
     """A packed plan built on one tensor codes another as the oracle does; the batched
     decode takes PACK containers with others."""

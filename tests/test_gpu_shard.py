@@ -99,6 +99,17 @@ def test_shards_with_a_plan(z, orc):
     assert np.array_equal(whole, one)
 
 
+def test_shards_with_a_packed_plan(z):
+    """A plan with packed exponents: the shards carry its packed records and list too, and
+    the assembled container equals the single call's."""
+    from lossless_float_weight_b200 import workloads as W
+    x = W.kv_cache(shape=(2, 2, 2, 2, 4096, 128), device="cuda")
+    plan = z.Plan.create(x, groups=4, seed=0, max_pack=15)
+    whole = _assemble(z, x, 3, 262144, plan=plan).cpu().numpy()
+    one = z.compress(x, plan=plan).cpu().numpy()
+    assert one[58] == 15 and np.array_equal(whole, one)
+
+
 def test_shard_tables_batch_and_mismatch(z):
     """Several tensors in one call (as a multi-tensor checkpoint uses it), and a shard
     whose size or range does not match: CORRUPT, nothing written for it."""
