@@ -84,7 +84,8 @@ def test_packed_plan_parity_kv(z, orc):
     assert (modes == 4).sum() > 64
 
 
-@pytest.mark.parametrize("case", ["tail", "odd", "big_chunks", "short_subblocks", "few_exponents", "max_pack_3"])
+@pytest.mark.parametrize("case", ["tail", "odd", "big_chunks", "short_subblocks", "few_exponents", "max_pack_3",
+                                  "partial_runs"])
 def test_packed_plan_parity_shapes(z, orc, case):
     """Escapes, an odd value count (the last chunk cannot pack), chunks of 1024 sub-blocks
     (four rounds of the encoder's scan), sub-blocks of 16 values, fewer distinct exponents
@@ -109,9 +110,13 @@ def test_packed_plan_parity_shapes(z, orc, case):
         E = torch.randint(124, 130, (300000,), generator=g)
         x = torch.pow(2.0, (E - 127).to(torch.float64)).to(torch.bfloat16)
         _check(z, orc, x, groups=2, cb=65536, name=case)
-    else:
+    elif case == "max_pack_3":
         x = (torch.randn(400000, generator=g) * 0.02).to(torch.bfloat16)
         _check(z, orc, x, groups=2, cb=65536, max_pack=3, name=case)
+    else:  # a last chunk of 1000 values: its second sub-block's 244 pairs leave one lane 4
+        x = (torch.randn(65536 * 2 + 1000, generator=g) * 0.02).to(torch.bfloat16)
+        got, _ = _check(z, orc, x, groups=2, cb=131072, name=case)
+        assert got[64 + 32 * 2] == 4  # the last chunk's exponent stream is PACK
 
 
 def test_packed_with_zero_runs(z, orc):
