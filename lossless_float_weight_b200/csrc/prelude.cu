@@ -391,10 +391,18 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist_tiles(const uint
         // counter (exponent, lane) at byte exponent << 7 | lane << 2: bits 30..23 of the
         // value moved to 14..7; my 32 values are one zero-run block of every fraction plane
         uint32_t a = 0;
+        if (cnt == NV) {  // a whole pass: no test per value
 #pragma unroll
-        for (int j = 0; j < NV; j++) {
-          if (j < cnt) atomicAdd(reinterpret_cast<uint32_t*>(tab + (((raw.w[j] >> 16) & 0x7F80u) | l4)), 1u);
-          a |= raw.w[j];
+          for (int j = 0; j < NV; j++) {
+            atomicAdd(reinterpret_cast<uint32_t*>(tab + (((raw.w[j] >> 16) & 0x7F80u) | l4)), 1u);
+            a |= raw.w[j];
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < NV; j++) {
+            if (j < cnt) atomicAdd(reinterpret_cast<uint32_t*>(tab + (((raw.w[j] >> 16) & 0x7F80u) | l4)), 1u);
+            a |= raw.w[j];
+          }
         }
         nzw |= a;
         const uint32_t blk = (v0 - lo) / kZBlock;  // within the tile
@@ -407,13 +415,10 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist_tiles(const uint
         // counter (bin, lane) at byte bin << 7 | lane << 2: FP8 bin = byte & 0x7F; FP4 bin =
         // (low nibble & 7) | (high nibble & 7) << 3
         const int nbytes = DT == kFP8 ? cnt : cnt / 2;  // FP4: cnt is even
-#pragma unroll
-        for (int j = 0; j < W; j++) {
-          const uint32_t x = raw.w[j];
-          nzw |= x;
+        auto count_word = [&](uint32_t x, int k0, bool all) {
 #pragma unroll
           for (int k = 0; k < 4; k++) {
-            if (4 * j + k < nbytes) {
+            if (all || k0 + k < nbytes) {
               uint32_t off;
               if constexpr (DT == kFP8) {
                 off = k == 0 ? (x << 7) & 0x3F80u : (x >> (8 * k - 7)) & 0x3F80u;
@@ -423,6 +428,19 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist_tiles(const uint
               }
               atomicAdd(reinterpret_cast<uint32_t*>(tab + (off | l4)), 1u);
             }
+          }
+        };
+        if (cnt == NV) {  // a whole pass: no test per byte
+#pragma unroll
+          for (int j = 0; j < W; j++) {
+            nzw |= raw.w[j];
+            count_word(raw.w[j], 4 * j, true);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < W; j++) {
+            nzw |= raw.w[j];
+            count_word(raw.w[j], 4 * j, false);
           }
         }
       }
