@@ -233,8 +233,8 @@ __global__ void __launch_bounds__(kSThreads, 8) k_encode_sub(const uint8_t* __re
           uint32_t mw[nwm];
           raw_words<DT, s>(raw.w, mw);
 #pragma unroll
-          for (int k = 0; k < nwm; k++)
-            if (wbase + k < used) words[wbase + k] = mw[k];
+          for (int k = 0; k < nwm; k++)  // a whole pass's words all lie inside the stream
+            if (cnt == kSValues || wbase + k < used) words[wbase + k] = mw[k];
         }
         if (last) {
           const uint64_t padded = raw_payload(m, w) / 4;
