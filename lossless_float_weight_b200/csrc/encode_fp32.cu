@@ -186,23 +186,28 @@ __global__ void __launch_bounds__(kFThreads, 8) k_encode_fp32(const uint8_t* __r
       uint32_t qoff[kFValues / 16];
       uint64_t acc = 0;
       const uint8_t* encb = reinterpret_cast<const uint8_t*>(sm.enc);
+      auto pack_codes = [&](bool all) {  // all: a whole pass, no test per value
 #pragma unroll
-      for (int j = 0; j < kFValues / 2; j++) {
-        if ((j & 7) == 0) qoff[j >> 3] = nw * 32 + nfill;
-        if (2 * j < cnt) {
-          const uint32_t e0 = *reinterpret_cast<const uint32_t*>(encb + ((raw.w[2 * j] >> 21) & 0x3FCu));
-          const uint32_t e1 = 2 * j + 1 < cnt ? *reinterpret_cast<const uint32_t*>(encb + ((raw.w[2 * j + 1] >> 21) & 0x3FCu))
-                                              : 0u;
-          const uint32_t l1 = e1 >> 16;
-          const uint32_t l = (e0 >> 16) + l1;
-          acc = (acc << l) | (((e0 & 0xFFFFu) << l1) | (e1 & 0xFFFFu));
-          nfill += l;
-          if (nfill >= 32) {
-            nfill -= 32;
-            pw[nw++] = (uint32_t)(acc >> nfill);
+        for (int j = 0; j < kFValues / 2; j++) {
+          if ((j & 7) == 0) qoff[j >> 3] = nw * 32 + nfill;
+          if (all || 2 * j < cnt) {
+            const uint32_t e0 = *reinterpret_cast<const uint32_t*>(encb + ((raw.w[2 * j] >> 21) & 0x3FCu));
+            const uint32_t e1 = all || 2 * j + 1 < cnt
+                                    ? *reinterpret_cast<const uint32_t*>(encb + ((raw.w[2 * j + 1] >> 21) & 0x3FCu))
+                                    : 0u;
+            const uint32_t l1 = e1 >> 16;
+            const uint32_t l = (e0 >> 16) + l1;
+            acc = (acc << l) | (((e0 & 0xFFFFu) << l1) | (e1 & 0xFFFFu));
+            nfill += l;
+            if (nfill >= 32) {
+              nfill -= 32;
+              pw[nw++] = (uint32_t)(acc >> nfill);
+            }
           }
         }
-      }
+      };
+      if (cnt == kFValues) pack_codes(true);
+      else pack_codes(false);
       const uint32_t mybits = nw * 32 + nfill;
       if (nfill) pw[nw++] = (uint32_t)(acc << (32 - nfill));
       // my bit offset in the pass: a warp scan, then the four warp totals after one barrier
