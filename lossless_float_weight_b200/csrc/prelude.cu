@@ -465,15 +465,23 @@ __global__ void __launch_bounds__(kHistThreads, 3) k_split_hist_tiles(const uint
       }
     }
     __syncthreads();  // the tile's counts and bitmaps are complete
-    for (int b = tid; b < AC; b += kHistThreads) {
+    {
+      // column sums: TPB threads a bin (FP4 4, FP8 2, FP32 1: every thread one share of
+      // 32 / TPB lanes), joined by shuffles between neighbouring lanes; the rotation by the
+      // bin keeps a warp's loads on 32 different banks
+      constexpr int TPB = kHistThreads / AC >= 1 ? kHistThreads / AC : 1;
+      static_assert(AC * TPB == kHistThreads, "one share a thread");
+      const int b = tid / TPB, part = tid % TPB;
       uint32_t sum = 0;
 #pragma unroll 8
-      for (int l = 0; l < 32; l++) {
-        const int a = b * 32 + ((l + b) & 31);
+      for (int i = 0; i < 32 / TPB; i++) {
+        const int a = b * 32 + ((part * (32 / TPB) + i + b) & 31);
         sum += sh[a];
         sh[a] = 0;
       }
-      csum[b] = sum;
+#pragma unroll
+      for (int o = 1; o < TPB; o <<= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+      if (part == 0) csum[b] = sum;
     }
     if constexpr (F32) {
       if (ws.zmap && tid < 96) {
