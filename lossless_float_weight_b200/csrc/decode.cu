@@ -567,8 +567,9 @@ __device__ __forceinline__ int decode_fp32_fast(const uint32_t* lut, const uint3
 // window, the whole bitstream is brought into shared memory by one TMA bulk copy
 // (cp.async.bulk, completion on an mbarrier) while the block builds its lookup table.
 // Then, in rounds, every thread decodes the next 32 exponents of its sub-block into
-// its row of a shared buffer, and the block merges the rows with the sign/fraction
-// bytes: those are loaded as whole 32-byte sectors one round ahead of use, and the
+// its row of a shared buffer, and each warp merges its own 32 rows with the sign/fraction
+// bytes (so a round needs only warp barriers, and the warps of a block run at their own
+// pace): those are loaded as whole 32-byte sectors one round ahead of use, and the
 // merged words leave as whole 64-byte row segments. Word k of row r sits at
 // 8r + (k ^ (r / 4 mod 8)): the row-per-thread stores and the unit-per-thread loads
 // of the merge both touch 32 distinct banks, with no padding.
@@ -693,14 +694,15 @@ __device__ int decode_bf16_staged(StagedSmem& st, const Lut* lut, const uint32_t
       if ((j == 0 && start != 0) || start > cap_bits || expect < start || expect > cap_bits) bad = 1;
       br.init(st.bits, bs_words, bad ? 0 : start, tail);
     }
-    // my merge units: unit u = tid + 256p is part u % 4 (values 8(u % 4)..) of row u / 4
-    // of the batch; ubase is its first value in round 0, urem the values its row has
-    // from there on
+    // my merge units: unit p is part tid % 4 (values 8(tid % 4)..) of row 32w + 8p +
+    // lane / 4 of the batch, a row of my own warp (w), so a warp merges only the rows its
+    // lanes decoded and its rounds need no block barrier; ubase is the unit's first value
+    // in round 0, urem the values its row has from there on
     uint32_t ubase[4], urem[4];
 #pragma unroll
     for (int p = 0; p < 4; p++) {
-      const uint32_t u = tid + p * kDecodeThreads;
-      const uint32_t row = batch + (u >> 2), part = u & 3;
+      const uint32_t rw = ((uint32_t)tid & ~31u) + 8u * p + (((uint32_t)tid & 31u) >> 2);
+      const uint32_t row = batch + rw, part = (uint32_t)tid & 3u;
       const uint32_t rc = row < nsub ? min32(S, m - row * S) : 0;
       ubase[p] = row * S + part * 8;
       urem[p] = rc > part * 8 ? rc - part * 8 : 0;
@@ -779,13 +781,12 @@ __device__ int decode_bf16_staged(StagedSmem& st, const Lut* lut, const uint32_t
           }
         }
       }
-      __syncthreads();
+      __syncwarp();
       // merge and store
 #pragma unroll
       for (int p = 0; p < 4; p++) {
-        const uint32_t u = tid + p * kDecodeThreads;
         if (!ALLFULL && !ucnt[p]) continue;
-        const uint32_t row = u >> 2, part = u & 3;
+        const uint32_t row = ((uint32_t)tid & ~31u) + 8u * p + (((uint32_t)tid & 31u) >> 2), part = (uint32_t)tid & 3u;
         const uint32_t es[2] = {st.ex[ex_word(row, 2 * part)], st.ex[ex_word(row, 2 * part + 1)]};
         const uint32_t xs[2] = {smv[p].x, smv[p].y};
         uint32_t o[4];
@@ -800,7 +801,7 @@ __device__ int decode_bf16_staged(StagedSmem& st, const Lut* lut, const uint32_t
             if (i < ucnt[p]) reinterpret_cast<uint16_t*>(d)[i] = (uint16_t)(o[i >> 1] >> (16 * (i & 1)));
         }
       }
-      __syncthreads();
+      __syncwarp();
     }
     if (count) {
       const uint64_t pos = br.position();
