@@ -619,13 +619,22 @@ struct SmemBitReader {
     q = ld(p + 2);
     bp = (uint32_t)(bit & 31);
   }
+  // The 48 KB window loads its next word only when the reader advances (fewer shared
+  // loads, so fewer bank conflicts on the table's lookups); the wide window selects.
   __device__ __forceinline__ void refill() {
-    const bool t = bp >= 32;
-    const uint32_t nq = ld(p + 3);
-    c = t ? (c << 32) | q : c;
-    q = t ? nq : q;
-    p += t ? 1u : 0u;
-    bp -= t ? 32u : 0u;
+    if constexpr (WIDE) {
+      const bool t = bp >= 32;
+      const uint32_t nq = ld(p + 3);
+      c = t ? (c << 32) | q : c;
+      q = t ? nq : q;
+      p += t ? 1u : 0u;
+      bp -= t ? 32u : 0u;
+    } else if (bp >= 32) {
+      c = (c << 32) | q;
+      q = ld(p + 3);
+      p++;
+      bp -= 32;
+    }
   }
   __device__ __forceinline__ uint32_t peek12() const { return (uint32_t)((c << bp) >> 52); }
   __device__ __forceinline__ void skip(uint32_t l) { bp += l; }
