@@ -28,6 +28,8 @@ namespace zipnn {
 constexpr int kDecodeThreads = 256;
 constexpr uint32_t kLutInvalid = 0x8000u;
 constexpr uint32_t kQuadInvalid = 0x4000u;  // FP4 four-symbol entries: not four valid codes
+// The wide window's table (11-bit windows): a window that starts a 12-bit code
+constexpr uint32_t kLong11 = 0x4000u;
 
 __device__ __forceinline__ uint32_t lut_symbol(uint32_t e) { return (e >> 16) & 0xFFu; }
 
@@ -576,8 +578,8 @@ __device__ __forceinline__ int decode_fp32_fast(const uint32_t* lut, const uint3
 constexpr uint32_t kWindowBytes = 48 * 1024;
 // A bitstream of 48 to 56 KB (exponents of more than 3 bits on average, as in K/V
 // caches) still decodes from shared memory: its last 8 KB go to the first half of the
-// decode table's 16 KB, and the second half holds a single-symbol table (u16 entries:
-// symbol << 4 | length, bit 15 invalid) instead of the two-symbol one.
+// decode table's 16 KB, and the second half holds a two-symbol table of 11-bit windows
+// (2048 u32 entries) instead of the 12-bit one.
 constexpr uint32_t kWideWindowBytes = 56 * 1024;
 constexpr uint32_t kWindowWords = kWindowBytes / 4, kWideWords = kWideWindowBytes / 4;
 constexpr int kRound = 32;  // exponents of a sub-block decoded per round
@@ -649,13 +651,7 @@ struct SmemBitReader {
     acc |= e;
     return lut_symbol(e);
   }
-  // single-symbol table: symbol << 4 | length, bit 15 invalid
-  __device__ __forceinline__ uint32_t huff(const uint16_t* lut, uint32_t& acc) {
-    const uint32_t e = lut[peek12()];
-    bp += e & 15u;
-    acc |= e;
-    return (e >> 4) & 0xFFu;
-  }
+  __device__ __forceinline__ uint32_t peek11() const { return (uint32_t)((c << bp) >> 53); }
   __device__ __forceinline__ uint64_t position() const { return (uint64_t)p * 32 + bp; }
 };
 
@@ -663,9 +659,71 @@ __device__ __forceinline__ uint32_t ex_word(uint32_t row, uint32_t k) {
   return row * kRowWords + (k ^ ((row >> 2) & (kRowWords - 1)));
 }
 
+// The wide window's table is indexed by 11 bits (2048 u32 entries in 8 KB, the room the
+// window leaves): an entry holds the first code's symbol and length and, when the second
+// code also ends inside the 11 bits, its symbol and the pair's length (the two-symbol
+// layout of the 12-bit table); a window that starts a 12-bit code is kLong11, and that code
+// is decoded from the canonical tables (its first value, index offset and limit).
+struct Long12 {
+  const uint8_t* sorted;
+  uint32_t first, offset, limit;
+};
+
+__device__ __forceinline__ uint32_t huff12_long(SmemBitReader<true>& br, const Long12& lg, uint32_t& acc) {
+  const uint32_t w12 = br.peek12();
+  if (w12 >= lg.limit || w12 < lg.first) acc |= kLutInvalid;  // no 12-bit code here: corrupt
+  br.skip(12);
+  return lg.sorted[(lg.offset + w12 - lg.first) & 255u];
+}
+
+// One symbol from the 11-bit table.
+__device__ __forceinline__ uint32_t huff11(SmemBitReader<true>& br, const uint32_t* lut, const Long12& lg,
+                                           uint32_t& acc) {
+  const uint32_t e = lut[br.peek11()];
+  if (e & kLong11) return huff12_long(br, lg, acc);
+  acc |= e;
+  br.skip(e & 15u);
+  return lut_symbol(e);
+}
+
+// Two symbols from the 11-bit table, in bits 16..31 as huff_pair returns them (refilling
+// once between two lookups when the window holds one code).
+__device__ __forceinline__ uint32_t huff_pair11(SmemBitReader<true>& br, const uint32_t* lut, const Long12& lg,
+                                                uint32_t& acc) {
+  const uint32_t e = lut[br.peek11()];
+  uint32_t s0;
+  if (e & kLong11) {
+    s0 = huff12_long(br, lg, acc);
+  } else {
+    acc |= e;
+    const uint32_t lp = (e >> 4) & 15u;
+    if (lp) {
+      br.skip(lp);
+      return e;
+    }
+    br.skip(e & 15u);
+    s0 = lut_symbol(e);
+  }
+  br.refill();
+  const uint32_t s1 = huff11(br, lut, lg, acc);
+  return (s0 << 16) | (s1 << 24);
+}
+
+// A packed exponent pair from the 11-bit table (as pack_pair).
+__device__ __forceinline__ uint32_t pack_pair11(SmemBitReader<true>& br, const uint32_t* lut, const Long12& lg,
+                                                const uint8_t* pexp, uint32_t valid, uint32_t& acc) {
+  const uint32_t p = huff11(br, lut, lg, acc);
+  const uint32_t hi = p >> 4, lo = p & 15u;
+  uint32_t a = pexp[hi], b = pexp[lo];
+  if (hi == kPackEsc) a = br.fixed(8);
+  if (lo == kPackEsc) b = br.fixed(8);
+  if (!((valid >> hi) & (valid >> lo) & 1u)) acc |= kLutInvalid;
+  return (a << 16) | (b << 24);
+}
+
 // One chunk, all threads of the block; one sub-block per thread and batch. WIDE: the
-// bitstream continues in `tail` after the window and lut is the single-symbol table;
-// else lut is the two-symbol table. smp: the chunk's sign/fraction payload (RAW) or
+// bitstream continues in `tail` after the window and lut is the 11-bit two-symbol table;
+// else lut is the 12-bit two-symbol table. smp: the chunk's sign/fraction payload (RAW) or
 // nullptr (ZERO); outc: the chunk's first output value. Returns nonzero if the stream is
 // inconsistent.
 // ZRUN: the sign/fraction plane has zero runs; smp is its kept bytes, zmap / zpre the
@@ -676,13 +734,14 @@ __device__ __forceinline__ uint32_t ex_word(uint32_t row, uint32_t k) {
 // merge unit holds 8 values (the case of every chunk of a weight checkpoint).
 // PACK: the exponent stream is packed pairs (pexp, valid as for pack_pair); S and every
 // count are even.
-template <bool WIDE, bool ZRUN, bool ALLFULL, bool PACK, class Lut>
-__device__ int decode_bf16_staged(StagedSmem& st, const Lut* lut, const uint32_t* tail,
+// WIDE: lut is the 11-bit table of the wide window (lg: its 12-bit codes).
+template <bool WIDE, bool ZRUN, bool ALLFULL, bool PACK>
+__device__ int decode_bf16_staged(StagedSmem& st, const uint32_t* lut, const uint32_t* tail,
                                   const uint32_t* __restrict__ idx, uint32_t bs_words,
                                   const uint8_t* __restrict__ smp, uint32_t m, uint32_t S, uint32_t nsub,
                                   uint8_t* __restrict__ outc, uint32_t pre_start, uint32_t pre_next,
                                   const uint32_t* zmap, const uint32_t* zpre, const uint8_t* pexp,
-                                  uint32_t valid) {
+                                  uint32_t valid, Long12 lg) {
   const int tid = threadIdx.x;
   int bad = 0;
   const uint64_t cap_bits = (uint64_t)bs_words * 32;
@@ -752,7 +811,13 @@ __device__ int decode_bf16_staged(StagedSmem& st, const Lut* lut, const uint32_t
         if (ALLFULL || base + kRound <= count) {
 #pragma unroll
           for (int k = 0; k < kRowWords; k++) {
-            if constexpr (PACK) {
+            if constexpr (PACK && WIDE) {
+              br.refill();
+              const uint32_t a = pack_pair11(br, lut, lg, pexp, valid, acc);
+              br.refill();
+              const uint32_t b = pack_pair11(br, lut, lg, pexp, valid, acc);
+              st.ex[ex_word(tid, k)] = __byte_perm(a, b, 0x7632);
+            } else if constexpr (PACK) {
               br.refill();
               const uint32_t a = pack_pair(br, lut, pexp, valid, acc);
               br.refill();
@@ -760,12 +825,9 @@ __device__ int decode_bf16_staged(StagedSmem& st, const Lut* lut, const uint32_t
               st.ex[ex_word(tid, k)] = __byte_perm(a, b, 0x7632);
             } else if constexpr (WIDE) {
               br.refill();
-              const uint32_t e0 = br.huff(lut, acc);
-              const uint32_t e1 = br.huff(lut, acc);
-              br.refill();
-              const uint32_t e2 = br.huff(lut, acc);
-              const uint32_t e3 = br.huff(lut, acc);
-              st.ex[ex_word(tid, k)] = e0 | (e1 << 8) | (e2 << 16) | (e3 << 24);
+              const uint32_t a = huff_pair11(br, lut, lg, acc);
+              const uint32_t b = huff_pair11(br, lut, lg, acc);
+              st.ex[ex_word(tid, k)] = __byte_perm(a, b, 0x7632);
             } else {
               br.refill();
               const uint32_t a = huff_pair(br, lut, acc);
@@ -778,14 +840,19 @@ __device__ int decode_bf16_staged(StagedSmem& st, const Lut* lut, const uint32_t
           if constexpr (PACK) {
             for (uint32_t k = 0; k < n; k += 2) {
               br.refill();
-              const uint32_t pr = pack_pair(br, lut, pexp, valid, acc);
+              uint32_t pr;
+              if constexpr (WIDE) pr = pack_pair11(br, lut, lg, pexp, valid, acc);
+              else pr = pack_pair(br, lut, pexp, valid, acc);
               exb[ex_word(tid, k >> 2) * 4 + (k & 3)] = (uint8_t)(pr >> 16);
               exb[ex_word(tid, k >> 2) * 4 + (k & 3) + 1] = (uint8_t)(pr >> 24);
             }
           } else {
             for (uint32_t k = 0; k < n; k++) {
               br.refill();
-              exb[ex_word(tid, k >> 2) * 4 + (k & 3)] = (uint8_t)br.huff(lut, acc);
+              uint32_t sym;
+              if constexpr (WIDE) sym = huff11(br, lut, lg, acc);
+              else sym = br.huff(lut, acc);
+              exb[ex_word(tid, k >> 2) * 4 + (k & 3)] = (uint8_t)sym;
             }
           }
         }
@@ -854,11 +921,9 @@ static_assert(sizeof(StagedSmem) + sizeof(DecodeSmem<kBF16>) + 1024 <= 233472 / 
 // [512w, 512w + 512), lane l the entries 512w + l + 32j (so each store of a warp covers 32
 // consecutive entries, one per bank): the lane finds the code of its first entry from the
 // length limits, then walks forward over the codes that end before its next entry.
-// Entries from limit[12] on match no code (only when the Kraft sum is below 1).
-// WIDE: u16 entries symbol << 4 | length (the single-symbol table); else u32 entries
-// symbol << 16 | length.
-template <bool WIDE>
-__device__ __forceinline__ void fill_lut(void* lut, const uint8_t* sorted, const uint8_t* slen,
+// Entries from limit[12] on match no code (only when the Kraft sum is below 1). Entries
+// are symbol << 16 | length.
+__device__ __forceinline__ void fill_lut(uint32_t* lut, const uint8_t* sorted, const uint8_t* slen,
                                          const uint32_t* limit, const uint32_t* first, const uint32_t* offset) {
   const uint32_t x0 = (threadIdx.x >> 5) * 512u + (threadIdx.x & 31u), lim = limit[kLmax];
   uint32_t l = 1;
@@ -879,14 +944,31 @@ __device__ __forceinline__ void fill_lut(void* lut, const uint8_t* sorted, const
         l = slen[k];
         end += 1u << (kLmax - l);
       }
-      e = WIDE ? ((uint32_t)sorted[k] << 4) | l : ((uint32_t)sorted[k] << 16) | l;
+      e = ((uint32_t)sorted[k] << 16) | l;
     }
-    if constexpr (WIDE) static_cast<uint16_t*>(lut)[x] = (uint16_t)e;
-    else static_cast<uint32_t*>(lut)[x] = e;
+    lut[x] = e;
   }
 }
 
 static_assert(kDecodeThreads * 16 == 4096, "fill_lut: 8 warps of 512 table entries");
+
+// The wide window's 11-bit table (first codes only; the second codes follow): window x
+// is the 12-bit window x << 1; a code of at most 11 bits there gives its symbol and length,
+// a 12-bit code gives kLong11, and no code (a Kraft sum below 1) gives kLutInvalid.
+__device__ __forceinline__ void fill_lut11(uint32_t* lut, const uint8_t* sorted, const uint32_t* limit,
+                                           const uint32_t* first, const uint32_t* offset) {
+  for (uint32_t x = threadIdx.x; x < 2048; x += kDecodeThreads) {
+    const uint32_t w = x << 1;
+    uint32_t e = kLutInvalid | 1u;
+    if (w < limit[kLmax]) {
+      uint32_t l = 1;
+      while (l < (uint32_t)kLmax && w >= limit[l]) l++;
+      if (l == (uint32_t)kLmax) e = kLong11 | (uint32_t)kLmax;
+      else e = ((uint32_t)sorted[(offset[l] + (w >> (kLmax - l)) - first[l]) & 255u] << 16) | l;
+    }
+    lut[x] = e;
+  }
+}
 
 
 constexpr uint32_t kZStagedWords = 128;  // zero-run bitmap words the staged path holds: 4096 blocks
@@ -1456,22 +1538,37 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
     sm.slen[e][k] = (uint8_t)my_len[e];
   }
   __syncthreads();
-  // BF16 with the wide window: the single-symbol table in the table's second half (the
-  // bulk copy may still be writing the first half)
+  // BF16 with the wide window: the 11-bit table in the table's second half (the bulk copy
+  // may still be writing the first half)
   const bool wide = DT == kBF16 && sm.staged == 2;
-  uint16_t* const lut16 = reinterpret_cast<uint16_t*>(sm.lut[0] + (kWideWords - kWindowWords));
+  uint32_t* const lut11 = sm.lut[0] + (kWideWords - kWindowWords);
 #pragma unroll
   for (int e = 0; e < NE; e++) {
     if (!coded(sm.mode[e])) continue;
-    if (wide) fill_lut<true>(lut16, sm.sorted[e], sm.slen[e], sm.limit[e], sm.first[e], sm.offset[e]);
-    else fill_lut<false>(sm.lut[e], sm.sorted[e], sm.slen[e], sm.limit[e], sm.first[e], sm.offset[e]);
+    if (wide) fill_lut11(lut11, sm.sorted[e], sm.limit[e], sm.first[e], sm.offset[e]);
+    else fill_lut(sm.lut[e], sm.sorted[e], sm.slen[e], sm.limit[e], sm.first[e], sm.offset[e]);
   }
   __syncthreads();
+  if (wide) {
+    // the 11-bit table's second codes, as for the 12-bit table below (in place: the first
+    // code's fields of an entry never change)
+    for (uint32_t x = tid; x < 2048; x += kDecodeThreads) {
+      const uint32_t e0 = lut11[x];
+      if (e0 & (kLutInvalid | kLong11)) continue;
+      const uint32_t l0 = e0 & 15u;
+      if (l0 >= 11) continue;
+      const uint32_t e1 = lut11[(x << l0) & 2047u];
+      const uint32_t l1 = e1 & 15u;
+      if (!(e1 & (kLutInvalid | kLong11)) && l0 + l1 <= 11)
+        lut11[x] = e0 | ((l0 + l1) << 4) | ((e1 & 0x00FF0000u) << 8);
+    }
+    __syncthreads();
+  }
   // second code of each window: the entry of the window shifted by the first length
   // decides it when that code ends inside the 12 known bits (a prefix code's entry does
   // not depend on the bits after the code). Updating in place is safe: the fields read
-  // here (first length, first symbol, invalid flag) never change. Every two-symbol table
-  // (not the wide window's single-symbol one).
+  // here (first length, first symbol, invalid flag) never change. Every 12-bit table (the
+  // wide window's 11-bit table had its own pass above).
   if (!wide) {
     bool any = false;
     // FP4 exponents whose codes have at most 3 bits (every Huffman code of 4 symbols): any
@@ -1537,28 +1634,29 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
       int bad;
 #define ZIPNN_STAGED(W, Z, F, P, L, T, ZM, ZP)                                                                \
   decode_bf16_staged<W, Z, F, P>(stg, L, T, idx, bs_words, smp, m, S, (uint32_t)nsub, out + clo * VB, idx_start, \
-                                 idx_next, ZM, ZP, sm.pack_exps, valid)
+                                 idx_next, ZM, ZP, sm.pack_exps, valid, lg)
+      const Long12 lg{sm.sorted[0], sm.first[0][kLmax], sm.offset[0][kLmax], sm.limit[0][kLmax]};
       const uint32_t valid = ((1u << sm.K) - 1u) | (1u << kPackEsc);
       if (sm.mode[0] == kModePack) {
         if (sm.mode[1] == kModeZrun) {
-          if (wide) bad = allfull ? ZIPNN_STAGED(true, true, true, true, lut16, sm.lut[0], sm.zmap, sm.zpre)
-                                  : ZIPNN_STAGED(true, true, false, true, lut16, sm.lut[0], sm.zmap, sm.zpre);
+          if (wide) bad = allfull ? ZIPNN_STAGED(true, true, true, true, lut11, sm.lut[0], sm.zmap, sm.zpre)
+                                  : ZIPNN_STAGED(true, true, false, true, lut11, sm.lut[0], sm.zmap, sm.zpre);
           else bad = allfull ? ZIPNN_STAGED(false, true, true, true, sm.lut[0], nullptr, sm.zmap, sm.zpre)
                              : ZIPNN_STAGED(false, true, false, true, sm.lut[0], nullptr, sm.zmap, sm.zpre);
         } else {
-          if (wide) bad = allfull ? ZIPNN_STAGED(true, false, true, true, lut16, sm.lut[0], nullptr, nullptr)
-                                  : ZIPNN_STAGED(true, false, false, true, lut16, sm.lut[0], nullptr, nullptr);
+          if (wide) bad = allfull ? ZIPNN_STAGED(true, false, true, true, lut11, sm.lut[0], nullptr, nullptr)
+                                  : ZIPNN_STAGED(true, false, false, true, lut11, sm.lut[0], nullptr, nullptr);
           else bad = allfull ? ZIPNN_STAGED(false, false, true, true, sm.lut[0], nullptr, nullptr, nullptr)
                              : ZIPNN_STAGED(false, false, false, true, sm.lut[0], nullptr, nullptr, nullptr);
         }
       } else if (sm.mode[1] == kModeZrun) {
-        if (wide) bad = allfull ? ZIPNN_STAGED(true, true, true, false, lut16, sm.lut[0], sm.zmap, sm.zpre)
-                                : ZIPNN_STAGED(true, true, false, false, lut16, sm.lut[0], sm.zmap, sm.zpre);
+        if (wide) bad = allfull ? ZIPNN_STAGED(true, true, true, false, lut11, sm.lut[0], sm.zmap, sm.zpre)
+                                : ZIPNN_STAGED(true, true, false, false, lut11, sm.lut[0], sm.zmap, sm.zpre);
         else bad = allfull ? ZIPNN_STAGED(false, true, true, false, sm.lut[0], nullptr, sm.zmap, sm.zpre)
                            : ZIPNN_STAGED(false, true, false, false, sm.lut[0], nullptr, sm.zmap, sm.zpre);
       } else {
-        if (wide) bad = allfull ? ZIPNN_STAGED(true, false, true, false, lut16, sm.lut[0], nullptr, nullptr)
-                                : ZIPNN_STAGED(true, false, false, false, lut16, sm.lut[0], nullptr, nullptr);
+        if (wide) bad = allfull ? ZIPNN_STAGED(true, false, true, false, lut11, sm.lut[0], nullptr, nullptr)
+                                : ZIPNN_STAGED(true, false, false, false, lut11, sm.lut[0], nullptr, nullptr);
         else bad = allfull ? ZIPNN_STAGED(false, false, true, false, sm.lut[0], nullptr, nullptr, nullptr)
                            : ZIPNN_STAGED(false, false, false, false, sm.lut[0], nullptr, nullptr, nullptr);
       }
