@@ -30,6 +30,9 @@ constexpr uint32_t kLutInvalid = 0x8000u;
 constexpr uint32_t kQuadInvalid = 0x4000u;  // FP4 four-symbol entries: not four valid codes
 // The wide window's table (11-bit windows): a window that starts a 12-bit code
 constexpr uint32_t kLong11 = 0x4000u;
+// A PACK stream's table entries hold the pair's exponents (bits 16..23 the first, 24..31
+// the second) and these flags for an escaped one (whose 8 bits follow the code)
+constexpr uint32_t kPackEscHi = 0x10u, kPackEscLo = 0x20u;
 
 __device__ __forceinline__ uint32_t lut_symbol(uint32_t e) { return (e >> 16) & 0xFFu; }
 
@@ -174,12 +177,11 @@ __device__ __forceinline__ uint64_t next_packed(StreamState& st, int n, uint32_t
         for (int i = 0; i < GV; i += 2) {
           if (!FULL && i >= n) break;
           st.br.refill();
-          const uint32_t p = st.br.huff(st.lut, st.acc);
-          const uint32_t hi = p >> 4, lo = p & 15u;
-          const uint32_t a = hi == kPackEsc ? st.br.fixed(8) : st.pexp[hi];
-          const uint32_t b = lo == kPackEsc ? st.br.fixed(8) : st.pexp[lo];
-          if ((hi != kPackEsc && hi >= (uint32_t)st.width) || (lo != kPackEsc && lo >= (uint32_t)st.width))
-            st.acc |= kLutInvalid;  // an index past the list: corrupt
+          const uint32_t e = st.lut[st.br.peek12()];  // a pair entry with its exponents
+          st.acc |= e;
+          st.br.skip(e & 15u);
+          const uint32_t a = (e & kPackEscHi) ? st.br.fixed(8) : (e >> 16) & 0xFFu;
+          const uint32_t b = (e & kPackEscLo) ? st.br.fixed(8) : e >> 24;
           o |= (uint64_t)(a | (b << 8)) << (8 * i);
         }
       }
@@ -264,21 +266,19 @@ __device__ __forceinline__ uint32_t bf16_merge_pair(uint32_t sf, int sf_hi, uint
 // BF16 with a HUFF exponent stream and a RAW (or ZERO) sign/fraction stream: the case
 // of every chunk of a trained or Gaussian checkpoint. 16 values per step; the
 // sign/fraction bytes of the next step are requested one step ahead.
-// A packed exponent pair (PACK streams) from either bit reader and either table: one code,
-// the pair symbol's two nibbles index the packed exponents (pexp, 16 entries); a nibble of
-// kPackEsc takes the next 8 bits as the exponent (first, then second). Returns the pair in
-// bits 16..31 (the first in 16..23), as huff_pair does. Needs 28 bits in the reader; an
-// index past the list (valid: bit i set for the K listed indices and for kPackEsc) marks
-// the stream corrupt.
-template <class Reader, class Lut>
-__device__ __forceinline__ uint32_t pack_pair(Reader& br, const Lut* lut, const uint8_t* pexp, uint32_t valid,
-                                              uint32_t& acc) {
-  const uint32_t p = br.huff(lut, acc);
-  const uint32_t hi = p >> 4, lo = p & 15u;
-  uint32_t a = pexp[hi], b = pexp[lo];
-  if (hi == kPackEsc) a = br.fixed(8);
-  if (lo == kPackEsc) b = br.fixed(8);
-  if (!((valid >> hi) & (valid >> lo) & 1u)) acc |= kLutInvalid;
+// A packed exponent pair (PACK streams) from either bit reader: one code, whose table
+// entry already holds the pair's two exponents (set when the table is built: the pair
+// symbol's nibbles index the packed exponents) and flags for the escaped ones, whose
+// 8 bits follow the code (first, then second). Returns the pair in bits 16..31 (the
+// first in 16..23), as huff_pair does. Needs 28 bits in the reader.
+template <class Reader>
+__device__ __forceinline__ uint32_t pack_pair(Reader& br, const uint32_t* lut, uint32_t& acc) {
+  const uint32_t e = lut[br.peek12()];
+  acc |= e;
+  br.skip(e & 15u);
+  uint32_t a = (e >> 16) & 0xFFu, b = e >> 24;
+  if (e & kPackEscHi) a = br.fixed(8);
+  if (e & kPackEscLo) b = br.fixed(8);
   return (a << 16) | (b << 24);
 }
 
@@ -305,7 +305,7 @@ __device__ __forceinline__ int decode_bf16_fast(const uint32_t* lut, const uint8
 #pragma unroll
       for (int i = 0; i < 8; i++) {
         br.refill();
-        pr[i] = pack_pair(br, lut, pexp, valid, acc);
+        pr[i] = pack_pair(br, lut, acc);
       }
     } else {
 #pragma unroll
@@ -332,7 +332,7 @@ __device__ __forceinline__ int decode_bf16_fast(const uint32_t* lut, const uint8
   if (PACK) {  // count is even
     for (uint32_t v = full * 16; v < count; v += 2) {
       br.refill();
-      const uint32_t pr = pack_pair(br, lut, pexp, valid, acc);
+      const uint32_t pr = pack_pair(br, lut, acc);
       const uint32_t b0 = SM_ZERO ? 0u : smp[v], b1 = SM_ZERO ? 0u : smp[v + 1];
       reinterpret_cast<uint16_t*>(dst)[v] = (uint16_t)merge_value<kBF16>((pr >> 16) & 0xFFu, b0, 0, 0);
       reinterpret_cast<uint16_t*>(dst)[v + 1] = (uint16_t)merge_value<kBF16>(pr >> 24, b1, 0, 0);
@@ -712,12 +712,21 @@ __device__ __forceinline__ uint32_t huff_pair11(SmemBitReader<true>& br, const u
 // A packed exponent pair from the 11-bit table (as pack_pair).
 __device__ __forceinline__ uint32_t pack_pair11(SmemBitReader<true>& br, const uint32_t* lut, const Long12& lg,
                                                 const uint8_t* pexp, uint32_t valid, uint32_t& acc) {
-  const uint32_t p = huff11(br, lut, lg, acc);
-  const uint32_t hi = p >> 4, lo = p & 15u;
-  uint32_t a = pexp[hi], b = pexp[lo];
-  if (hi == kPackEsc) a = br.fixed(8);
-  if (lo == kPackEsc) b = br.fixed(8);
-  if (!((valid >> hi) & (valid >> lo) & 1u)) acc |= kLutInvalid;
+  const uint32_t e = lut[br.peek11()];
+  if (e & kLong11) {  // a 12-bit pair code: its symbol's nibbles index the list here
+    const uint32_t p = huff12_long(br, lg, acc);
+    const uint32_t hi = p >> 4, lo = p & 15u;
+    uint32_t a = pexp[hi], b = pexp[lo];
+    if (hi == kPackEsc) a = br.fixed(8);
+    if (lo == kPackEsc) b = br.fixed(8);
+    if (!((valid >> hi) & (valid >> lo) & 1u)) acc |= kLutInvalid;
+    return (a << 16) | (b << 24);
+  }
+  acc |= e;
+  br.skip(e & 15u);
+  uint32_t a = (e >> 16) & 0xFFu, b = e >> 24;
+  if (e & kPackEscHi) a = br.fixed(8);
+  if (e & kPackEscLo) b = br.fixed(8);
   return (a << 16) | (b << 24);
 }
 
@@ -819,9 +828,9 @@ __device__ int decode_bf16_staged(StagedSmem& st, const uint32_t* lut, const uin
               st.ex[ex_word(tid, k)] = __byte_perm(a, b, 0x7632);
             } else if constexpr (PACK) {
               br.refill();
-              const uint32_t a = pack_pair(br, lut, pexp, valid, acc);
+              const uint32_t a = pack_pair(br, lut, acc);
               br.refill();
-              const uint32_t b = pack_pair(br, lut, pexp, valid, acc);
+              const uint32_t b = pack_pair(br, lut, acc);
               st.ex[ex_word(tid, k)] = __byte_perm(a, b, 0x7632);
             } else if constexpr (WIDE) {
               br.refill();
@@ -842,7 +851,7 @@ __device__ int decode_bf16_staged(StagedSmem& st, const uint32_t* lut, const uin
               br.refill();
               uint32_t pr;
               if constexpr (WIDE) pr = pack_pair11(br, lut, lg, pexp, valid, acc);
-              else pr = pack_pair(br, lut, pexp, valid, acc);
+              else pr = pack_pair(br, lut, acc);
               exb[ex_word(tid, k >> 2) * 4 + (k & 3)] = (uint8_t)(pr >> 16);
               exb[ex_word(tid, k >> 2) * 4 + (k & 3) + 1] = (uint8_t)(pr >> 24);
             }
@@ -1549,7 +1558,24 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
     else fill_lut(sm.lut[e], sm.sorted[e], sm.slen[e], sm.limit[e], sm.first[e], sm.offset[e]);
   }
   __syncthreads();
-  if (wide) {
+  const bool pack = DT == kBF16 && sm.mode[0] == kModePack;
+  if (pack) {
+    // a PACK stream: each entry's pair symbol becomes its two exponents (the list's entries
+    // for its nibbles) and escape flags; a nibble past the list makes the entry invalid
+    uint32_t* const t = wide ? lut11 : sm.lut[0];
+    const uint32_t ne = wide ? 2048u : 4096u;
+    for (uint32_t x = tid; x < ne; x += kDecodeThreads) {
+      const uint32_t e = t[x];
+      if (e & (kLutInvalid | kLong11)) continue;
+      const uint32_t sym = lut_symbol(e), hi = sym >> 4, lo = sym & 15u;
+      const bool bad = (hi != kPackEsc && hi >= sm.K) || (lo != kPackEsc && lo >= sm.K);
+      const uint32_t a = hi == kPackEsc ? 0u : sm.pack_exps[hi], b = lo == kPackEsc ? 0u : sm.pack_exps[lo];
+      t[x] = (e & 15u) | (hi == kPackEsc ? kPackEscHi : 0u) | (lo == kPackEsc ? kPackEscLo : 0u) |
+             (bad ? kLutInvalid : 0u) | (a << 16) | (b << 24);
+    }
+    __syncthreads();
+  }
+  if (wide && !pack) {
     // the 11-bit table's second codes, as for the 12-bit table below (in place: the first
     // code's fields of an entry never change)
     for (uint32_t x = tid; x < 2048; x += kDecodeThreads) {
@@ -1581,7 +1607,7 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* __restrict__ in, uin
     if (tid == 0) sm.quad = quad;
 #pragma unroll
     for (int e = 0; e < NE; e++) {
-      if (!coded(sm.mode[e])) continue;
+      if (sm.mode[e] != kModeHuff) continue;  // PACK entries hold exponents, not second codes
       any = true;
       if (e == 0 && quad) {
         for (uint32_t x = tid; x < 4096; x += kDecodeThreads) {
