@@ -133,6 +133,19 @@ def test_packed_with_zero_runs(z, orc):
     assert 4 in modes[0::2].tolist() and 3 in modes[1::2].tolist()
 
 
+def test_packed_with_zero_runs_unstaged(z, orc):
+    """The same pruned weights in 1 MiB chunks: bitstreams too long for the shared-memory
+    window, so PACK exponents beside ZRUN planes go through the per-stream readers."""
+    g = torch.Generator().manual_seed(12)
+    v = (torch.randn(524288 * 2 + 4096, generator=g) * 0.02)
+    blocks = v.view(-1, 32)
+    blocks[torch.rand(blocks.shape[0], generator=g) < 0.5] = 0
+    x = v.to(torch.bfloat16)
+    got, _ = _check(z, orc, x, groups=2, cb=1 << 20, name="pruned, 1 MiB chunks")
+    modes = got[64: 64 + 16 * 2 * 3: 16]
+    assert 4 in modes[0::2].tolist() and 3 in modes[1::2].tolist()
+
+
 def test_packed_plan_reuse_and_batch(z, orc):
     """A packed plan built on one tensor codes another as the oracle does; the batched
     decode takes PACK containers with others."""
