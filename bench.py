@@ -165,7 +165,17 @@ class ClockSampler:
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
-    def stop(self):
+    def wait_first(self, timeout_s=3.0):
+        """Wait (bounded) until nvidia-smi has printed its first sample, so that a short
+        timed region that starts now is sampled."""
+        t0 = time.time()
+        while self.proc is not None and not self.lines and time.time() - t0 < timeout_s:
+            time.sleep(0.01)
+
+    def mark(self):
+        return len(self.lines)
+
+    def stop(self, lo=None, hi=None):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -175,7 +185,10 @@ class ClockSampler:
             self.proc.kill()
         mhz, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        # the samples taken while the timed region ran (lo..hi), plus the one just after it;
+        # all of them when the region was too short to catch any
+        window = self.lines[lo:hi + 1] if lo is not None and hi is not None and hi + 1 > lo else []
+        for ln in window or self.lines:
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
@@ -395,6 +408,8 @@ def run_ours(args):
     barrier(world, dev)
     torch.cuda.synchronize()
     clocks.start()
+    clocks.wait_first()
+    clk_lo = clocks.mark()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
@@ -406,8 +421,9 @@ def run_ours(args):
         ev[k][2].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
+    clk_hi = clocks.mark()
     barrier(world, dev)
-    clk = clocks.stop()
+    clk = clocks.stop(clk_lo, clk_hi)
     total_ms = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
     comp_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps, world, dev)
     dec_ms = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps, world, dev)
